@@ -1,0 +1,375 @@
+"""Pins for the CPU oracle, checked against things other than the oracle itself:
+closed forms, exact rational arithmetic, torch's bf16 conversions (library
+routines), a hand-written fixture, brute-force loops and invariants.
+
+CPU only (no GPU marker)."""
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from activation_sparse_gated_gemm_b200 import synth
+from oracle import twell_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def torch_bf16_bits(values_f32: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 (round to nearest even) by torch, as raw bits."""
+    t = torch.from_numpy(np.ascontiguousarray(values_f32, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_of_exact(values) -> np.ndarray:
+    """bf16 bits of values that are exactly representable in bf16."""
+    v = np.asarray(values, dtype=np.float32)
+    b = torch_bf16_bits(v)
+    assert np.array_equal(O.bf16_bits_to_f64(b), v.astype(np.float64))
+    return b
+
+
+# ---------------------------------------------------------------------------
+# bf16 conversions
+
+
+def test_bf16_decode_matches_torch():
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 1 << 16, size=20000, dtype=np.uint32).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]  # finite only
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.bf16_bits_to_f64(bits), ref)
+
+
+def test_bf16_round_matches_torch_on_fp32_inputs():
+    rng = np.random.default_rng(2)
+    raw = rng.integers(0, 1 << 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    raw = raw[(raw & 0x7F800000) != 0x7F800000]  # finite
+    raw = raw[(raw & 0x7F800000) < 0x7F000000]  # keep clear of overflow to inf
+    ties = (rng.integers(0, 1 << 16, size=5000, dtype=np.uint32) << 16) | 0x8000
+    ties = ties[(ties & 0x7F800000) < 0x7F000000].astype(np.uint32)
+    vals = np.concatenate([raw, ties]).view(np.float32)
+    assert np.array_equal(O.f64_to_bf16_bits(vals.astype(np.float64)), torch_bf16_bits(vals))
+
+
+def _all_finite_bf16():
+    bits = np.arange(0, 0x7F80, dtype=np.uint16)  # +0 .. largest finite
+    return bits, O.bf16_bits_to_f64(bits)
+
+
+def test_bf16_round_bruteforce_nearest_even():
+    """Direct fp64 -> bf16 rounding equals the nearest entry of the full table
+    of bf16 values, ties to the even bit pattern (no double rounding)."""
+    tb, tv = _all_finite_bf16()
+    rng = np.random.default_rng(3)
+    x = np.concatenate([
+        rng.standard_normal(4000) * 10.0 ** rng.integers(-30, 30, size=4000),
+        np.ldexp(rng.random(500), -rng.integers(120, 134, size=500)),  # bf16 subnormals
+        [1 + 2.0**-8, 1 + 3 * 2.0**-8, 1 + 2.0**-8 + 2.0**-30, 0.0, -0.0, 2.0**-133, 3 * 2.0**-134],
+    ])
+    got = O.f64_to_bf16_bits(x)
+    for xi, gi in zip(x, got):
+        a = abs(xi)
+        k = int(np.searchsorted(tv, a))
+        cands = [c for c in (k - 1, k) if 0 <= c < len(tv)]
+        best = min(cands, key=lambda c: (abs(tv[c] - a), int(tb[c]) & 1))
+        want = int(tb[best]) | (0x8000 if math.copysign(1.0, xi) < 0 else 0)
+        assert int(gi) == want, (xi, hex(int(gi)), hex(want))
+    # the case where rounding through fp32 first would differ
+    assert int(O.f64_to_bf16_bits(np.array([1 + 2.0**-8 + 2.0**-30]))[0]) == 0x3F81
+
+
+# ---------------------------------------------------------------------------
+# TwELL pack against a hand-derived fixture
+
+
+def load_golden_pack(path):
+    z = None
+    counts, slots, ovf = {}, {}, {}
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        tok = line.split()
+        if tok[0] == "shape":
+            T, f, tile, W = map(int, tok[1:])
+            z = np.full((T, f), -1.0)
+        elif tok[0] == "z":
+            z[int(tok[1]), int(tok[2])] = float(tok[3])
+        elif tok[0] == "counts":
+            counts[(int(tok[1]), int(tok[2]))] = int(tok[3])
+        elif tok[0] == "slot":
+            slots[(int(tok[1]), int(tok[2]), int(tok[3]))] = (int(tok[4]), int(tok[5], 16))
+        elif tok[0] == "ovf":
+            ovf[int(tok[1])] = int(tok[2])
+    return z, tile, W, counts, slots, ovf
+
+
+def test_pack_matches_hand_fixture():
+    z, tile, W, counts, slots, ovf = load_golden_pack(os.path.join(GOLDEN, "twell_pack_small.txt"))
+    tw = O.twell_pack(z, tile, W)
+    for (t, c), n in counts.items():
+        assert tw["counts"][t, c] == n
+    for (t, c, s), (j, v) in slots.items():
+        assert tw["idx"][t, c, s] == j and tw["vals"][t, c, s] == v
+    # every slot past the stored ones is padding
+    T, nT, _ = tw["idx"].shape
+    for t in range(T):
+        for c in range(nT):
+            for s in range(min(counts[(t, c)], W), W):
+                assert tw["idx"][t, c, s] == -1 and tw["vals"][t, c, s] == 0
+    assert [int(v) for v in tw["row_ovf"]] == [ovf[t] for t in range(T)]
+    assert O.route_rows(tw["counts"], W).tolist() == [t for t in range(T) if ovf[t]]
+
+
+# ---------------------------------------------------------------------------
+# TwELL pack by brute force
+
+
+def pack_by_loops(z, tile, W):
+    T, f = z.shape
+    nT = f // tile
+    counts = np.zeros((T, nT), dtype=np.int64)
+    idx = np.full((T, nT, W), -1, dtype=np.int64)
+    vals = np.zeros((T, nT, W), dtype=np.int64)
+    for t in range(T):
+        for c in range(nT):
+            n = 0
+            for k in range(tile):
+                j = c * tile + k
+                if z[t, j] > 0:
+                    if n < W:
+                        idx[t, c, n] = j
+                        vals[t, c, n] = int(torch_bf16_bits(np.array([z[t, j]], np.float32))[0])
+                    n += 1
+            counts[t, c] = n
+    return counts, idx, vals
+
+
+@pytest.mark.parametrize("W", [1, 2, 16, 128])
+@pytest.mark.parametrize("seed", range(4))
+def test_pack_bruteforce(W, seed):
+    rng = np.random.default_rng(100 + seed)
+    T, f, tile = int(rng.integers(1, 9)), 256, 128
+    density = rng.choice([0.02, 0.1, 0.5, 0.95])
+    z = rng.standard_normal((T, f)).astype(np.float32)
+    z = np.where(rng.random((T, f)) < density, np.abs(z), -np.abs(z))
+    z[rng.random((T, f)) < 0.05] = 0.0  # exact zeros are inactive
+    z = z.astype(np.float64)  # fp32-exact values, so torch's rounding applies
+    tw = O.twell_pack(z, tile, W)
+    counts, idx, vals = pack_by_loops(z, tile, W)
+    assert np.array_equal(tw["counts"], counts)
+    assert np.array_equal(tw["idx"], idx)
+    assert np.array_equal(tw["vals"].astype(np.int64), vals)
+    assert np.array_equal(tw["row_ovf"], (counts > W).any(axis=1).astype(np.uint8))
+
+
+def test_pack_unpack_roundtrip_full_width():
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((16, 512)).astype(np.float32).astype(np.float64)
+    tw = O.twell_pack(z, 128, 128)
+    g = O.twell_unpack(tw["counts"], tw["idx"], tw["vals"], 512)
+    want = torch_bf16_bits(np.maximum(z, 0).astype(np.float32))
+    assert np.array_equal(g, want)
+    assert tw["row_ovf"].sum() == 0
+
+
+MID = synth.LayerConfig("mid", T=512, d=256, f=1024, tile=128, W=16, density=0.05,
+                        sigma=0.5, dead_frac=0.03)
+HEAVY = synth.LayerConfig("heavy", T=1024, d=256, f=2304, tile=128, W=24, density=0.012,
+                          sigma=0.5, heavy_frac=0.08, heavy_lo=0.25, heavy_hi=0.40)
+
+
+@pytest.mark.parametrize("cfg", [synth.CONFIGS["tiny"], MID], ids=lambda c: c.name)
+def test_pack_invariants_on_synthetic_layers(cfg):
+    L = synth.make_layer(cfg, seed=0)
+    z = O.gate_preactivation(L["x"], L["WgT"])
+    tw = O.twell_pack(z, cfg.tile, cfg.W)
+    assert tw["counts"].astype(np.int64).sum() == int((z > 0).sum())
+    n = np.minimum(tw["counts"], cfg.W)
+    for t in range(cfg.T):
+        for c in range(cfg.nT):
+            js = tw["idx"][t, c, : n[t, c]].astype(np.int64)
+            assert np.all(np.diff(js) > 0)
+            assert np.all((js >= c * cfg.tile) & (js < (c + 1) * cfg.tile))
+            assert np.all(z[t, js] > 0)
+            assert np.array_equal(tw["vals"][t, c, : n[t, c]], O.f64_to_bf16_bits(z[t, js]))
+    assert np.array_equal(tw["row_ovf"], (tw["counts"] > cfg.W).any(axis=1).astype(np.uint8))
+
+
+def test_route_is_the_overflow_predicate():
+    rng = np.random.default_rng(7)
+    counts = rng.integers(0, 40, size=(300, 9)).astype(np.int16)
+    for W in (8, 16, 24, 32, 39):
+        want = [t for t in range(counts.shape[0]) if any(int(c) > W for c in counts[t])]
+        assert O.route_rows(counts, W).tolist() == want
+
+
+# ---------------------------------------------------------------------------
+# The dense layer: closed forms and exact arithmetic
+
+
+def test_dense_permutation_closed_form():
+    """With permutation matrices the layer is an index shuffle:
+    z_j = x[pa(j)], u_j = x[pb(j)], y[pc(j)] = ReLU(z_j) * u_j. A transposed
+    operand would apply the inverse permutation and fail."""
+    rng = np.random.default_rng(8)
+    n, T = 32, 5
+    pa, pb, pc = rng.permutation(n), rng.permutation(n), rng.permutation(n)
+    assert not np.array_equal(pa, np.argsort(pa))
+    eye = np.eye(n)
+    WgT, WuT, Wd = eye[pa], eye[pb], eye[pc]  # WgT[j, pa(j)] = 1, Wd[j, pc(j)] = 1
+    xv = (rng.integers(-40, 40, size=(T, n)) / 8.0)
+    x = bits_of_exact(xv)
+    y = O.gated_ffn(x, bits_of_exact(WgT), bits_of_exact(WuT), bits_of_exact(Wd))
+    want = np.zeros((T, n))
+    for j in range(n):
+        want[:, pc[j]] = np.maximum(xv[:, pa[j]], 0) * xv[:, pb[j]]
+    assert np.array_equal(y, want)
+
+
+def test_dense_exact_rational_bruteforce():
+    rng = np.random.default_rng(9)
+    T, d, f = 3, 6, 10
+    x = torch_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    WgT = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    WuT = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    Wd = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    F = lambda b: [[Fraction(float(v)) for v in row] for row in O.bf16_bits_to_f64(b)]
+    xf, gf, uf, df = F(x), F(WgT), F(WuT), F(Wd)
+    y = O.gated_ffn(x, WgT, WuT, Wd)
+    for t in range(T):
+        for k in range(d):
+            acc = Fraction(0)
+            for j in range(f):
+                zj = sum(xf[t][i] * gf[j][i] for i in range(d))
+                uj = sum(xf[t][i] * uf[j][i] for i in range(d))
+                acc += max(zj, Fraction(0)) * uj * df[j][k]
+            assert abs(y[t, k] - float(acc)) <= 1e-12 * max(1.0, abs(float(acc)))
+
+
+def test_dense_special_cases():
+    L = synth.make_layer(synth.CONFIGS["tiny"], seed=3)
+    x, WgT, WuT, Wd = L["x"], L["WgT"], L["WuT"], L["Wd"]
+    y = O.gated_ffn(x, WgT, WuT, Wd)
+    # scaling x by 2 scales both z and u: y quadruples (exact powers of two)
+    x2 = bits_of_exact(2 * O.bf16_bits_to_f64(x))
+    assert np.array_equal(O.gated_ffn(x2, WgT, WuT, Wd), 4 * y)
+    # scaling Wd by 2 doubles y
+    assert np.array_equal(O.gated_ffn(x, WgT, WuT, bits_of_exact(2 * O.bf16_bits_to_f64(Wd))), 2 * y)
+    # an all-negative gate gives y == 0 and an empty pack
+    neg = O.bf16_bits_to_f64(WgT).copy()
+    neg[:, -1] = -64.0
+    negb = bits_of_exact(neg)
+    assert not np.any(O.gated_ffn(x, negb, WuT, Wd))
+    tw = O.twell_pack(O.gate_preactivation(x, negb), 128, 16)
+    assert tw["counts"].sum() == 0 and tw["row_ovf"].sum() == 0
+    # one active column j*: y = relu(z_j*) * u_j* * Wd[j*, :]
+    one = neg.copy()
+    js = 77
+    one[js, -1] = 64.0
+    oneb = bits_of_exact(one)
+    xf = O.bf16_bits_to_f64(x)
+    zj = xf @ O.bf16_bits_to_f64(oneb)[js]
+    uj = xf @ O.bf16_bits_to_f64(WuT)[js]
+    want = (zj * uj)[:, None] * O.bf16_bits_to_f64(Wd)[js][None, :]
+    assert np.all(zj > 0)
+    np.testing.assert_allclose(O.gated_ffn(x, oneb, WuT, Wd), want, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# sparse == dense
+
+
+def test_sparse_equals_dense_when_gate_is_bf16_exact():
+    """Small-integer inputs keep z exactly representable in bf16, so the
+    stored values are exact and the sparse sum equals the dense layer."""
+    rng = np.random.default_rng(11)
+    T, d, f = 24, 8, 256
+    x = bits_of_exact(rng.integers(-3, 4, size=(T, d)).astype(np.float64))
+    WgT = bits_of_exact(rng.integers(-3, 4, size=(f, d)).astype(np.float64))
+    WuT = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    Wd = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    z = O.gate_preactivation(x, WgT)
+    tw = O.twell_pack(z, 128, 128)
+    assert np.array_equal(O.bf16_bits_to_f64(O.f64_to_bf16_bits(z)), z)
+    ys = O.sparse_ffn_from_twell(tw, x, WuT, Wd)
+    yd = O.gated_ffn(x, WgT, WuT, Wd)
+    np.testing.assert_allclose(ys, yd, rtol=1e-12, atol=1e-12 * np.abs(yd).max())
+
+
+def test_sparse_within_bf16_bound_of_dense():
+    """With the stored bf16 gate, each term h_j Wd[j,k] moves by at most
+    2^-8 relative (one nearest rounding to 8 significant bits), which bounds
+    |y_sparse - y_dense|."""
+    cfg = synth.CONFIGS["tiny"]
+    L = synth.make_layer(cfg, seed=0)
+    z = O.gate_preactivation(L["x"], L["WgT"])
+    tw = O.twell_pack(z, cfg.tile, cfg.W)
+    keep = np.nonzero(tw["row_ovf"] == 0)[0]
+    ys = O.sparse_ffn_from_twell(tw, L["x"], L["WuT"], L["Wd"], rows=keep)
+    yd = O.gated_ffn(L["x"][keep], L["WgT"], L["WuT"], L["Wd"])
+    xf = O.bf16_bits_to_f64(L["x"][keep])
+    g = np.maximum(z[keep], 0)
+    u = xf @ O.bf16_bits_to_f64(L["WuT"]).T
+    bound = (np.abs(g * u) @ np.abs(O.bf16_bits_to_f64(L["Wd"]))) * 2.0**-8 + 1e-12
+    assert np.all(np.abs(ys - yd) <= bound)
+    assert np.abs(ys - yd).max() > 0  # the rounding is visible
+
+
+def test_hybrid_routes_heavy_tokens_and_combines_branches():
+    L = synth.make_layer(HEAVY, seed=0)
+    out = O.hybrid_ffn(L["x"], L["WgT"], L["WuT"], L["Wd"], HEAVY.tile, HEAVY.W)
+    ovf = out["ovf_rows"]
+    assert np.all(np.diff(ovf) > 0)
+    heavy = np.nonzero(L["p_t"] >= HEAVY.heavy_lo)[0]
+    assert set(heavy.tolist()) <= set(ovf.tolist())  # Binomial tail: a miss is ~1e-12
+    assert len(ovf) < len(heavy) + 0.05 * HEAVY.T
+    yd = O.gated_ffn(L["x"], L["WgT"], L["WuT"], L["Wd"])
+    assert np.array_equal(out["y"][ovf], yd[ovf])
+    rms = np.sqrt(np.mean(yd**2))
+    assert np.abs(out["y"] - yd).max() <= 1e-2 * rms
+
+
+# ---------------------------------------------------------------------------
+# The generator keeps the gate exact in fp32 under any summation order
+
+
+@pytest.mark.parametrize("cfg", [synth.CONFIGS["tiny"], MID, HEAVY], ids=lambda c: c.name)
+def test_generator_gate_is_order_free_in_fp32(cfg):
+    L = synth.make_layer(cfg, seed=0)
+    xf = O.bf16_bits_to_f64(L["x"])
+    wf = O.bf16_bits_to_f64(L["WgT"])
+    d = cfg.d
+    e = int(math.floor(math.log2(math.sqrt(d)))) + 5
+    assert np.array_equal(np.rint(xf[:, : d - 2] * 8), xf[:, : d - 2] * 8)
+    assert np.array_equal(np.rint(wf[:, : d - 2] * 2.0**e), wf[:, : d - 2] * 2.0**e)
+    assert np.array_equal(np.rint(xf[:, d - 2:] * 32), xf[:, d - 2:] * 32)
+    assert np.array_equal(np.rint(wf[:, d - 2:] * 32), wf[:, d - 2:] * 32)
+    assert e + 3 <= 13
+    # Cauchy-Schwarz bound on every partial sum of |x_k w_k|
+    bound = (np.linalg.norm(xf[:, : d - 2], axis=1).max() * np.linalg.norm(wf[:, : d - 2], axis=1).max()
+             + np.abs(xf[:, d - 2]).max() + np.abs(wf[:, d - 1]).max())
+    assert bound < 2.0**11
+    z64 = O.gate_preactivation(L["x"], L["WgT"])
+    z32 = (torch.from_numpy(xf.astype(np.float32)) @ torch.from_numpy(wf.astype(np.float32)).T).numpy()
+    assert np.array_equal(z32.astype(np.float64), z64)
+
+
+def test_generator_density_and_determinism():
+    cfg = synth.CONFIGS["tiny"]
+    a = synth.make_layer(cfg, seed=0)
+    b = synth.make_layer(cfg, seed=0)
+    c = synth.make_layer(cfg, seed=1)
+    for k in ("x", "WgT", "WuT", "Wd"):
+        assert np.array_equal(a[k], b[k])
+        assert not np.array_equal(a[k], c[k])
+    z = O.gate_preactivation(a["x"], a["WgT"])
+    assert abs((z > 0).mean() - 0.05) < 0.006
+    L = synth.make_layer(MID, seed=0)
+    z = O.gate_preactivation(L["x"], L["WgT"])
+    assert not np.any(z[:, L["dead"]] > 0)
+    assert abs((z > 0).mean() - MID.density) < 0.01
