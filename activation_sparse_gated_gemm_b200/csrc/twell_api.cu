@@ -1,0 +1,418 @@
+// C ABI of the TwELL sparse gated FFN (declared in include/twell.h): argument
+// checks, TMA tensor maps and kernel launches. Host code only; the kernels
+// live in umma_gemm.cuh and sparse_ffn.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "twell.h"
+#include "sparse_ffn.cuh"
+#include "umma_gemm.cuh"
+
+namespace {
+
+using namespace twell;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ device
+
+struct DeviceInfo {
+  std::atomic<int> state{0};  // 0 unknown, 1 ok, 2 unsupported
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+twell_status current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TWELL_ERR_CUDA;
+  DeviceInfo& info = g_dev[dev];
+  int st = info.state.load(std::memory_order_acquire);
+  if (st == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return TWELL_ERR_CUDA;
+    info.num_sms = sms;
+    st = (major == 10 && minor == 0) ? 1 : 2;
+    info.state.store(st, std::memory_order_release);
+  }
+  if (st != 1) return TWELL_ERR_DEVICE;
+  *dev_out = dev;
+  *sms_out = info.num_sms;
+  return TWELL_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [outer][inner] with 128-byte swizzled boxes of
+// box_inner x box_outer elements.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ checks
+
+twell_status check_shape(int T, int d, int f) {
+  if (T < 0) return TWELL_ERR_SHAPE;
+  if (d < 64 || d > 4096 || d % 64 != 0) return TWELL_ERR_SHAPE;
+  if (f < 128 || f > 32767 || f % 128 != 0) return TWELL_ERR_SHAPE;
+  return TWELL_OK;
+}
+
+twell_status check_tw(const twell_t* tw, int T, int f) {
+  if (tw == nullptr) return TWELL_ERR_NULL;
+  if (tw->T != T || tw->f != f || tw->tile != 128) return TWELL_ERR_SHAPE;
+  if (tw->W < 8 || tw->W > 128 || tw->W % 8 != 0) return TWELL_ERR_SHAPE;
+  if (T > 0) {
+    if (!tw->counts || !tw->idx || !tw->vals || !tw->row_ovf) return TWELL_ERR_NULL;
+    if (!aligned16(tw->counts) || !aligned16(tw->idx) || !aligned16(tw->vals) || !aligned16(tw->row_ovf))
+      return TWELL_ERR_ALIGN;
+  }
+  return TWELL_OK;
+}
+
+twell_status check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p == nullptr) return TWELL_ERR_NULL;
+  for (const void* p : ps)
+    if (!aligned16(p)) return TWELL_ERR_ALIGN;
+  return TWELL_OK;
+}
+
+#define TW_TRY(expr)                    \
+  do {                                  \
+    twell_status _s = (expr);           \
+    if (_s != TWELL_OK) return _s;      \
+  } while (0)
+
+twell_status cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return TWELL_OK;
+  (void)cudaGetLastError();
+  return TWELL_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ launches
+
+template <int MODE>
+twell_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
+                         int grid, cudaStream_t s) {
+  auto kern = umma_gemm_kernel<MODE>;
+  TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes)));
+  kern<<<grid, kGemmThreads, kGemmSmemBytes, s>>>(a, b0, b1, p);
+  return cuda_ok(cudaGetLastError());
+}
+
+int gemm_grid(int M, int N, int tile_n, int sms) {
+  const long long tiles = static_cast<long long>((M + kBM - 1) / kBM) * ((N + tile_n - 1) / tile_n);
+  return static_cast<int>(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);
+}
+
+twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
+                            int32_t* dev_status, cudaStream_t s, int sms) {
+  TW_TRY(cuda_ok(cudaMemsetAsync(tw->row_ovf, 0, static_cast<size_t>(T), s)));
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mb, WgT, d, f, kBK, kBN)) return TWELL_ERR_CUDA;
+  GemmParams p{};
+  p.M = T;
+  p.N = f;
+  p.K = d;
+  p.counts = tw->counts;
+  p.idx = tw->idx;
+  p.vals = tw->vals;
+  p.row_ovf = tw->row_ovf;
+  p.nT = f / 128;
+  p.W = tw->W;
+  p.dev_status = dev_status;
+  return launch_gemm<kModeTwell>(ma, mb, mb, p, gemm_grid(T, f, kBN, sms), s);
+}
+
+template <int NCH>
+twell_status launch_sparse_n(const SparseParams& p, cudaStream_t s) {
+  const int blocks = (p.T + kSparseWarps - 1) / kSparseWarps;
+  sparse_ffn_warp_kernel<NCH><<<blocks, kSparseWarps * 32, 0, s>>>(p);
+  return cuda_ok(cudaGetLastError());
+}
+
+twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
+                         const twell_t* tw, int skip, uint16_t* y, int32_t* dev_status, cudaStream_t s) {
+  SparseParams p{};
+  p.x = x;
+  p.WuT = WuT;
+  p.Wd = Wd;
+  p.counts = tw->counts;
+  p.idx = tw->idx;
+  p.vals = tw->vals;
+  p.row_ovf = tw->row_ovf;
+  p.y = y;
+  p.T = T;
+  p.d = d;
+  p.f = f;
+  p.nT = f / 128;
+  p.W = tw->W;
+  p.skip_ovf = skip ? 1 : 0;
+  p.dev_status = dev_status;
+  switch ((d + 255) / 256) {
+    case 1: return launch_sparse_n<1>(p, s);
+    case 2: return launch_sparse_n<2>(p, s);
+    case 3: return launch_sparse_n<3>(p, s);
+    case 4: return launch_sparse_n<4>(p, s);
+    case 5: return launch_sparse_n<5>(p, s);
+    case 6: return launch_sparse_n<6>(p, s);
+    case 7: return launch_sparse_n<7>(p, s);
+    case 8: return launch_sparse_n<8>(p, s);
+    case 9: return launch_sparse_n<9>(p, s);
+    case 10: return launch_sparse_n<10>(p, s);
+    case 11: return launch_sparse_n<11>(p, s);
+    case 12: return launch_sparse_n<12>(p, s);
+    case 13: return launch_sparse_n<13>(p, s);
+    case 14: return launch_sparse_n<14>(p, s);
+    case 15: return launch_sparse_n<15>(p, s);
+    case 16: return launch_sparse_n<16>(p, s);
+    default: return TWELL_ERR_SHAPE;
+  }
+}
+
+// Dense gated FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu)
+// into h_buf [M][f], then out[row_map[i]] = h[i] Wd (row_map null: identity).
+twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const uint16_t* WgT, const uint16_t* WuT,
+                        const uint16_t* Wd, int d, int f, uint16_t* h_buf, const int* row_map, uint16_t* y,
+                        int y_rows, int32_t* dev_status, cudaStream_t s, int sms) {
+  CUtensorMap ma, mg, mu, mh, md;
+  if (!make_map(&ma, a_rows, d, M, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, 128) ||
+      !make_map(&mu, WuT, d, f, kBK, 128) || !make_map(&mh, h_buf, f, M, kBK, kBM) ||
+      !make_map(&md, Wd, d, f, 64, kBK))
+    return TWELL_ERR_CUDA;
+  GemmParams p1{};
+  p1.M = M;
+  p1.M_dev = M_dev;
+  p1.N = f;
+  p1.K = d;
+  p1.out = h_buf;
+  p1.ldo = f;
+  p1.dev_status = dev_status;
+  const int g1 = M_dev ? sms : gemm_grid(M, f, 128, sms);
+  TW_TRY(launch_gemm<kModeGateUp>(ma, mg, mu, p1, g1, s));
+  GemmParams p2{};
+  p2.M = M;
+  p2.M_dev = M_dev;
+  p2.N = d;
+  p2.K = f;
+  p2.out = y;
+  p2.ldo = d;
+  p2.row_map = row_map;
+  p2.out_rows = y_rows;
+  p2.dev_status = dev_status;
+  const int g2 = M_dev ? sms : gemm_grid(M, d, kBN, sms);
+  return launch_gemm<kModeDown>(mh, md, md, p2, g2, s);
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Dense branch: gather x[rows[i]] into xo, dense gated FFN into ho, scatter to y.
+twell_status dense_rows_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
+                             int T, int d, int f, const int32_t* rows, const int32_t* n_rows, uint16_t* y,
+                             uint16_t* xo, uint16_t* ho, int32_t* dev_status, cudaStream_t s, int sms) {
+  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, rows, n_rows, T, xo, dev_status);
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  return dense_impl(xo, T, n_rows, WgT, WuT, Wd, d, f, ho, rows, y, T, dev_status, s, sms);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+twell_status twell_gate_pack(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
+                             int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return gate_pack_impl(x, WgT, T, d, f, tw, dev_status, static_cast<cudaStream_t>(stream), sms);
+}
+
+twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
+                              const twell_t* tw, int skip_overflow_rows, uint16_t* y, int32_t* dev_status,
+                              void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WuT, Wd, y, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return sparse_impl(x, WuT, Wd, T, d, f, tw, skip_overflow_rows, y, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
+                               int T, int d, int f, const twell_t* tw, uint16_t* y, int32_t* dev_status,
+                               void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, y, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
+  return sparse_impl(x, WuT, Wd, T, d, f, tw, 0, y, dev_status, s);
+}
+
+twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream) {
+  if (tw == nullptr) return TWELL_ERR_NULL;
+  TW_TRY(check_tw(tw, tw->T, tw->f));
+  TW_TRY(check_ptrs({ovf_rows, n_ovf}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  route_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(tw->row_ovf, tw->T, ovf_rows, n_ovf);
+  return cuda_ok(cudaGetLastError());
+}
+
+size_t twell_hybrid_workspace_bytes(int T, int d, int f) {
+  if (T <= 0 || d <= 0 || f <= 0) return 0;
+  return round_up(static_cast<size_t>(T) * d * 2, 256) + round_up(static_cast<size_t>(T) * f * 2, 256);
+}
+
+twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                      const uint16_t* Wd, int T, int d, int f, const twell_t* tw, uint16_t* y,
+                                      int32_t* ovf_rows, int32_t* n_ovf, void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, y, ovf_rows, n_ovf, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_hybrid_workspace_bytes(T, d, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* xo = static_cast<uint16_t*>(workspace);
+  uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                             round_up(static_cast<size_t>(T) * d * 2, 256));
+  TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
+  route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s));
+  return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
+}
+
+twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                      const uint16_t* Wd, int T, int d, int f, const int32_t* rows,
+                                      const int32_t* n_rows, uint16_t* y, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, rows, n_rows, y, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_hybrid_workspace_bytes(T, d, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  uint16_t* xo = static_cast<uint16_t*>(workspace);
+  uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                             round_up(static_cast<size_t>(T) * d * 2, 256));
+  return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, rows, n_rows, y, xo, ho, dev_status,
+                         static_cast<cudaStream_t>(stream), sms);
+}
+
+size_t twell_dense_workspace_bytes(int T, int d, int f) {
+  (void)d;
+  if (T <= 0 || f <= 0) return 0;
+  return round_up(static_cast<size_t>(T) * f * 2, 256);
+}
+
+twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                     const uint16_t* Wd, int T, int d, int f, uint16_t* y, void* workspace,
+                                     size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, y, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_dense_workspace_bytes(T, d, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return dense_impl(x, T, nullptr, WgT, WuT, Wd, d, f, static_cast<uint16_t*>(workspace), nullptr, y, T,
+                    dev_status, static_cast<cudaStream_t>(stream), sms);
+}
+
+twell_status twell_unpack(const twell_t* tw, uint16_t* g_dense, int32_t* dev_status, void* stream) {
+  if (tw == nullptr) return TWELL_ERR_NULL;
+  TW_TRY(check_tw(tw, tw->T, tw->f));
+  if (tw->T < 0 || tw->f < 128 || tw->f % 128 != 0 || tw->f > 32767) return TWELL_ERR_SHAPE;
+  if (tw->T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({g_dense, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  const int nT = tw->f / 128;
+  const long long warps = static_cast<long long>(tw->T) * nT;
+  const long long blocks = (warps + 7) / 8;
+  if (blocks > 0x7fffffffLL) return TWELL_ERR_SHAPE;
+  unpack_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      tw->counts, tw->idx, tw->vals, tw->T, nT, tw->W, tw->f, g_dense, dev_status);
+  return cuda_ok(cudaGetLastError());
+}
+
+twell_status twell_status_reset(int32_t* dev_status, void* stream) {
+  if (dev_status == nullptr) return TWELL_ERR_NULL;
+  return cuda_ok(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)));
+}
+
+twell_status twell_status_get(const int32_t* dev_status, void* stream, int32_t* host_out) {
+  if (dev_status == nullptr || host_out == nullptr) return TWELL_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  TW_TRY(cuda_ok(cudaMemcpyAsync(host_out, dev_status, sizeof(int32_t), cudaMemcpyDeviceToHost, s)));
+  return cuda_ok(cudaStreamSynchronize(s));
+}
+
+const char* twell_status_str(int status) {
+  switch (status) {
+    case TWELL_OK: return "ok";
+    case TWELL_ERR_NULL: return "a required pointer is NULL";
+    case TWELL_ERR_SHAPE: return "a size is out of range or the TwELL descriptor does not match";
+    case TWELL_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case TWELL_ERR_WORKSPACE: return "workspace missing or too small";
+    case TWELL_ERR_CUDA: return "a CUDA call failed";
+    case TWELL_ERR_DEVICE: return "the current device is not compute capability 10.0 (B200)";
+    case TWELL_ERR_OVERFLOW: return "a row had more nonzeros in a tile than the ELL width (non-hybrid forward)";
+    case TWELL_ERR_INDEX: return "a stored column or row index was out of range";
+    case TWELL_ERR_TIMEOUT: return "a bounded on-chip wait gave up";
+    default: return "unknown status";
+  }
+}
+
+const char* twell_version(void) { return "twell-b200 0.1"; }
+
+}  // extern "C"

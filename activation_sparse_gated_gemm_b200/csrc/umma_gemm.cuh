@@ -1,0 +1,372 @@
+// Persistent tcgen05 GEMM for sm_100a: C[M,N] = A[M,K] . B[N,K]^T with bf16
+// operands and an fp32 accumulator in tensor memory, and three epilogues:
+//
+//   kModeTwell  -- the gate GEMM z = x . Wg. The epilogue applies ReLU and packs
+//                  each 128-column tile of every row into Tile-wise ELLPACK
+//                  (count, first W (column, bf16 value) pairs in ascending
+//                  column order) straight from the accumulator, so the format
+//                  is assembled at the end of the GEMM's own pass with no
+//                  separate launch and no extra trip through memory
+//                  (intellectnews.ru "Sakana AI и NVIDIA ... TwELL", section
+//                  "Формат TwELL вместо классической sparse-упаковки";
+//                  gate.com post 20977915, paragraph on TwELL).
+//   kModeGateUp -- z and u = x . Wu in one MMA (B = 128 rows of Wg stacked on
+//                  the same 128 rows of Wu); the epilogue stores
+//                  h = ReLU(z) * u as bf16. The dense layer's first half.
+//   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
+//                  epilogue stores bf16 rows, optionally scattered through a
+//                  row map (the dense branch of the hybrid route).
+//
+// Structure: one CTA per SM walks output tiles of 128 x 256 (x 128 h-columns
+// for kModeGateUp). Warp 0 issues TMA loads into a 4-stage shared-memory ring,
+// warp 1 issues tcgen05.mma (M=128, N=256, K=16) into one of two 256-column
+// TMEM accumulators, warps 2-5 drain the other accumulator with tcgen05.ld, so
+// the epilogue of tile i overlaps the MMAs of tile i+1. No cluster, no
+// multicast: every CTA loads its own operand tiles.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace twell {
+
+enum GemmMode : int { kModeTwell = 0, kModeGateUp = 1, kModeDown = 2 };
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;  // 64 bf16 = 128 bytes = one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kAStageBytes = kBM * kBK * 2;  // 16 KB
+constexpr int kBStageBytes = kBN * kBK * 2;  // 32 KB
+constexpr int kEpiPitch = 33;                // floats per row of the epilogue transpose buffer
+constexpr int kEpiBytes = 4 * 32 * kEpiPitch * 4;
+constexpr int kGemmThreads = 192;
+constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
+
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kStages * kAStageBytes;
+constexpr int kOffEpi = kOffB + kStages * kBStageBytes;
+constexpr int kOffBar = kOffEpi + kEpiBytes;
+constexpr int kNumBars = 2 * kStages + 4 + 1;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kGemmSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
+
+struct GemmParams {
+  int M;             // rows of A (an upper bound when M_dev is set)
+  const int* M_dev;  // optional device-side row count, clamped to [0, M]
+  int N;             // output columns: f (TwELL), f (gate-up, h columns), d (down)
+  int K;             // reduction length, a multiple of 64
+  // kModeTwell outputs
+  int16_t* counts;
+  int16_t* idx;
+  uint16_t* vals;
+  uint8_t* row_ovf;
+  int nT;
+  int W;
+  // kModeGateUp / kModeDown output (bf16, leading dimension ldo)
+  uint16_t* out;
+  int ldo;
+  const int* row_map;  // kModeDown: output row of each A row, or null
+  int out_rows;        // valid range of output rows
+  int* dev_status;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = bars;                     // [kStages] TMA -> MMA
+  uint64_t* empty = bars + kStages;          // [kStages] MMA -> TMA
+  uint64_t* tfull = bars + 2 * kStages;      // [2] MMA -> epilogue
+  uint64_t* tempty = bars + 2 * kStages + 2; // [2] epilogue -> MMA
+  uint64_t* drain = bars + 2 * kStages + 4;  // abort path: MMAs retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  int M = p.M;
+  if (p.M_dev != nullptr) M = min(max(*p.M_dev, 0), p.M);
+  constexpr int kTileN = (MODE == kModeGateUp) ? 128 : kBN;  // output columns per tile
+  const int num_m = (M + kBM - 1) / kBM;
+  const int num_n = (p.N + kTileN - 1) / kTileN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = p.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (MODE == kModeGateUp) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t issued = 0, issued_par = 0;  // per stage: a load is outstanding / its phase parity
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile / num_n;
+        const int n_blk = tile - m_blk * num_n;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = smem + kOffA + s * kAStageBytes;
+          uint8_t* b_dst = smem + kOffB + s * kBStageBytes;
+          mbar_arrive_expect_tx(&full[s], kAStageBytes + kBStageBytes);
+          tma_load_2d(a_dst, &tmA, &full[s], kb * kBK, m_blk * kBM);
+          if (MODE == kModeTwell) {
+            tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * kBN);
+          } else if (MODE == kModeGateUp) {
+            tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * 128);
+            tma_load_2d(b_dst + kBStageBytes / 2, &tmB1, &full[s], kb * kBK, n_blk * 128);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              tma_load_2d(b_dst + i * (kBStageBytes / 4), &tmB0, &full[s], n_blk * kBN + i * 64, kb * kBK);
+          }
+          issued |= 1u << s;
+          issued_par = (issued_par & ~(1u << s)) | (ph << s);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        raise_status(p.dev_status, kDevTimeout);
+      }
+      if (*abort_flag) {
+        // Let every load still in flight land before the CTA's shared memory goes away.
+        for (int t = 0; t < kStages; ++t)
+          if (issued & (1u << t)) mbar_wait(&full[t], (issued_par >> t) & 1u, nullptr, kDrainTimeoutNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc = umma_idesc_bf16(kBM, kBN, MODE == kModeDown ? 1 : 0);
+      int s = 0;
+      uint32_t ph = 0;
+      int buf = 0;
+      uint32_t tph = 0;
+      bool ok = true, any_mma = false;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[buf], tph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + kOffA + s * kAStageBytes);
+          const uint32_t b_addr = smem_u32(smem + kOffB + s * kBStageBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // K-major, 128-byte swizzle: 8-row groups 1024 bytes apart; a K step of
+            // 16 bf16 is 32 bytes inside the swizzle row.
+            const uint64_t adesc = umma_smem_desc(a_addr + k * 32, 16, 1024);
+            uint64_t bdesc;
+            if (MODE == kModeDown) {
+              // N-major, 128-byte swizzle: 64-column slabs 8 KB apart (LBO), 8-row
+              // K groups 1 KB apart (SBO); a K step of 16 rows is 2 KB.
+              bdesc = umma_smem_desc(b_addr + k * 2048, kBStageBytes / 4, 1024);
+            } else {
+              bdesc = umma_smem_desc(b_addr + k * 32, 16, 1024);
+            }
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+            any_mma = true;
+          }
+          umma_commit(&empty[s]);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[buf]);
+        if (++buf == 2) {
+          buf = 0;
+          tph ^= 1u;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        raise_status(p.dev_status, kDevTimeout);
+      }
+      if (*abort_flag && any_mma) {
+        umma_commit(drain);
+        mbar_wait(drain, 0, nullptr, kDrainTimeoutNs);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
+    float* ebuf = reinterpret_cast<float*>(smem + kOffEpi) + (warp - 2) * 32 * kEpiPitch;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int buf = 0;
+    uint32_t tph = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const bool got = mbar_wait(&tfull[buf], tph, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        *abort_flag = 1;
+        if (lane == 0) raise_status(p.dev_status, kDevTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int m_blk = tile / num_n;
+      const int n_blk = tile - m_blk * num_n;
+      const uint32_t t_row = tmem_base + static_cast<uint32_t>(buf * kBN) + (static_cast<uint32_t>(q * 32) << 16);
+      const int row_base = m_blk * kBM + q * 32;
+      const int my_row = row_base + lane;
+
+      if (MODE == kModeTwell) {
+#pragma unroll 1
+        for (int sub = 0; sub < 2; ++sub) {
+          const int c = n_blk * 2 + sub;  // TwELL column tile
+          int cnt = 0;                    // running count of my_row in tile c
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(sub * 128 + ch * 32), r);
+            tmem_wait_ld();
+            if (sub == 1 && ch == 3) {
+              tc_fence_before();
+              mbar_arrive(&tempty[buf]);
+            }
+            if (c >= p.nT) continue;
+            // Transpose the 32x32 block through shared memory so that each row
+            // can be compacted with one ballot across its 32 columns.
+            uint32_t mine = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float v = __uint_as_float(r[i]);
+              ebuf[lane * kEpiPitch + i] = v;
+              mine |= (v > 0.0f ? 1u : 0u) << i;
+            }
+            const int before = cnt;
+            cnt += __popc(mine);
+            __syncwarp();
+            const int col = c * 128 + ch * 32 + lane;
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr) {
+              const float v = ebuf[rr * kEpiPitch + lane];
+              const bool act = v > 0.0f;
+              const uint32_t mask = __ballot_sync(0xffffffffu, act);
+              const int base = __shfl_sync(0xffffffffu, before, rr);
+              const int pos = base + __popc(mask & lt_mask);
+              const int row = row_base + rr;
+              if (act && pos < p.W && row < M) {
+                const size_t off = (static_cast<size_t>(row) * p.nT + c) * p.W + pos;
+                p.idx[off] = static_cast<int16_t>(col);
+                p.vals[off] = f32_to_bf16_bits(v);
+              }
+            }
+            __syncwarp();
+          }
+          if (c < p.nT && my_row < M) {
+            p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
+            if (cnt > p.W) p.row_ovf[my_row] = 1;
+          }
+        }
+      } else if (MODE == kModeGateUp) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t zr[32], ur[32];
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), zr);
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + ch * 32), ur);
+          tmem_wait_ld();
+          if (ch == 3) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int col = n_blk * 128 + ch * 32;
+          if (my_row < M && col < p.N) {
+            uint32_t hv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = fmaxf(__uint_as_float(zr[2 * i]), 0.0f) * __uint_as_float(ur[2 * i]);
+              const float h1 = fmaxf(__uint_as_float(zr[2 * i + 1]), 0.0f) * __uint_as_float(ur[2 * i + 1]);
+              hv[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(my_row) * p.ldo + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2], hv[4 * v + 3]);
+          }
+        }
+      } else {
+        int orow = my_row;
+        bool valid = my_row < M;
+        if (valid && p.row_map != nullptr) {
+          orow = p.row_map[my_row];
+          if (orow < 0 || orow >= p.out_rows) {
+            valid = false;
+            raise_status(p.dev_status, kDevIndex);
+          }
+        }
+#pragma unroll 1
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), r);
+          tmem_wait_ld();
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int col = n_blk * kBN + ch * 32;
+          if (valid && col < p.N) {
+            uint32_t yv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) yv[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(orow) * p.ldo + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(yv[4 * v], yv[4 * v + 1], yv[4 * v + 2], yv[4 * v + 3]);
+          }
+        }
+      }
+      if (++buf == 2) {
+        buf = 0;
+        tph ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace twell

@@ -1,0 +1,241 @@
+"""ctypes binding of libtwell.so (include/twell.h). Argument marshalling only:
+torch supplies device memory and the stream, every step runs in the library's
+CUDA kernels. Loading fails loudly when the library is missing; there is no
+fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtwell.so")
+
+TWELL_OK = 0
+TWELL_ERR_NULL = 1
+TWELL_ERR_SHAPE = 2
+TWELL_ERR_ALIGN = 3
+TWELL_ERR_WORKSPACE = 4
+TWELL_ERR_CUDA = 5
+TWELL_ERR_DEVICE = 6
+TWELL_ERR_OVERFLOW = 16
+TWELL_ERR_INDEX = 17
+TWELL_ERR_TIMEOUT = 18
+
+EXPORTED = (
+    "twell_gate_pack", "twell_sparse_ffn", "twell_ffn_forward", "twell_route",
+    "twell_hybrid_workspace_bytes", "twell_dense_rows_forward", "twell_ffn_hybrid_forward", "twell_dense_workspace_bytes",
+    "twell_dense_ffn_forward", "twell_unpack", "twell_status_reset", "twell_status_get",
+    "twell_status_str", "twell_version",
+)
+
+
+class TwellError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: status {status} ({msg})")
+        self.status = status
+
+
+class twell_t(ctypes.Structure):
+    _fields_ = [
+        ("counts", ctypes.c_void_p),
+        ("idx", ctypes.c_void_p),
+        ("vals", ctypes.c_void_p),
+        ("row_ovf", ctypes.c_void_p),
+        ("T", ctypes.c_int32),
+        ("f", ctypes.c_int32),
+        ("tile", ctypes.c_int32),
+        ("W", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library once and declare every entry point's signature."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m activation_sparse_gated_gemm_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    tw = ctypes.POINTER(twell_t)
+    sig = {
+        "twell_gate_pack": ([vp, vp, i32, i32, i32, tw, vp, vp], i32),
+        "twell_sparse_ffn": ([vp, vp, vp, i32, i32, i32, tw, i32, vp, vp, vp], i32),
+        "twell_ffn_forward": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp], i32),
+        "twell_route": ([tw, vp, vp, vp], i32),
+        "twell_hybrid_workspace_bytes": ([i32, i32, i32], sz),
+        "twell_dense_rows_forward": ([vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp], i32),
+        "twell_ffn_hybrid_forward": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
+        "twell_dense_workspace_bytes": ([i32, i32, i32], sz),
+        "twell_dense_ffn_forward": ([vp, vp, vp, vp, i32, i32, i32, vp, vp, sz, vp, vp], i32),
+        "twell_unpack": ([tw, vp, vp, vp], i32),
+        "twell_status_reset": ([vp, vp], i32),
+        "twell_status_get": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
+        "twell_status_str": ([i32], ctypes.c_char_p),
+        "twell_version": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def status_str(status: int) -> str:
+    return load().twell_status_str(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != TWELL_OK:
+        raise TwellError(fn, status, status_str(status))
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _bf16(name: str, t: torch.Tensor, shape: tuple) -> None:
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+        raise ValueError(f"{name} must be a contiguous CUDA bfloat16 tensor of shape {shape}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+class Twell:
+    """Device buffers of one TwELL-packed gate activation (see twell.h)."""
+
+    def __init__(self, T: int, f: int, W: int, device="cuda", tile: int = 128):
+        nT = f // tile
+        self.T, self.f, self.W, self.tile, self.nT = T, f, W, tile, nT
+        self.counts = torch.empty((T, nT), dtype=torch.int16, device=device)
+        self.idx = torch.empty((T, nT, W), dtype=torch.int16, device=device)
+        self.vals = torch.empty((T, nT, W), dtype=torch.bfloat16, device=device)
+        self.row_ovf = torch.empty((T,), dtype=torch.uint8, device=device)
+        self.desc = twell_t(self.counts.data_ptr(), self.idx.data_ptr(), self.vals.data_ptr(),
+                            self.row_ovf.data_ptr(), T, f, tile, W)
+
+    def ref(self):
+        return ctypes.byref(self.desc)
+
+
+def new_status(device="cuda") -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def status_reset(dev_status: torch.Tensor, stream=None) -> None:
+    _check("twell_status_reset", load().twell_status_reset(_ptr(dev_status), _stream(stream)))
+
+
+def status_get(dev_status: torch.Tensor, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check("twell_status_get", load().twell_status_get(_ptr(dev_status), _stream(stream), ctypes.byref(out)))
+    return int(out.value)
+
+
+def gate_pack(x, WgT, tw: Twell, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    _bf16("x", x, (T, d))
+    _bf16("WgT", WgT, (f, d))
+    _check("twell_gate_pack", load().twell_gate_pack(_ptr(x), _ptr(WgT), T, d, f, tw.ref(),
+                                                     _ptr(dev_status), _stream(stream)))
+
+
+def sparse_ffn(x, WuT, Wd, tw: Twell, y, skip_overflow_rows: bool, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = WuT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)), ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_sparse_ffn", load().twell_sparse_ffn(_ptr(x), _ptr(WuT), _ptr(Wd), T, d, f, tw.ref(),
+                                                       int(bool(skip_overflow_rows)), _ptr(y),
+                                                       _ptr(dev_status), _stream(stream)))
+
+
+def ffn_forward(x, WgT, WuT, Wd, tw: Twell, y, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_ffn_forward", load().twell_ffn_forward(_ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f,
+                                                         tw.ref(), _ptr(y), _ptr(dev_status),
+                                                         _stream(stream)))
+
+
+def route(tw: Twell, ovf_rows, n_ovf, stream=None) -> None:
+    _check("twell_route", load().twell_route(tw.ref(), _ptr(ovf_rows), _ptr(n_ovf), _stream(stream)))
+
+
+def hybrid_workspace_bytes(T: int, d: int, f: int) -> int:
+    return int(load().twell_hybrid_workspace_bytes(T, d, f))
+
+
+def dense_workspace_bytes(T: int, d: int, f: int) -> int:
+    return int(load().twell_dense_workspace_bytes(T, d, f))
+
+
+def ffn_hybrid_forward(x, WgT, WuT, Wd, tw: Twell, y, ovf_rows, n_ovf, workspace, dev_status,
+                       stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_ffn_hybrid_forward", load().twell_ffn_hybrid_forward(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f, tw.ref(), _ptr(y), _ptr(ovf_rows), _ptr(n_ovf),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def dense_rows_forward(x, WgT, WuT, Wd, rows, n_rows, y, workspace, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_dense_rows_forward", load().twell_dense_rows_forward(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f, _ptr(rows), _ptr(n_rows), _ptr(y),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def dense_ffn_forward(x, WgT, WuT, Wd, y, workspace, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_dense_ffn_forward", load().twell_dense_ffn_forward(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f, _ptr(y), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def unpack(tw: Twell, g_dense, dev_status, stream=None) -> None:
+    _bf16("g_dense", g_dense, (tw.T, tw.f))
+    _check("twell_unpack", load().twell_unpack(tw.ref(), _ptr(g_dense), _ptr(dev_status), _stream(stream)))
+
+
+def to_device_bf16(bits, device="cuda") -> torch.Tensor:
+    """Upload a uint16 numpy array of bf16 bit patterns as a bfloat16 tensor."""
+    import numpy as np
+
+    a = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return a.view(torch.bfloat16).to(device)
+
+
+def bf16_bits(t: torch.Tensor):
+    """bfloat16 tensor -> uint16 numpy array of its bit patterns."""
+    import numpy as np
+
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)

@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the TwELL sparse ReLU-gated FFN forward pass on B200.
+
+One step = one pass of the whole hybrid forward over one batch of synthetic
+tokens: gate GEMM with the TwELL pack in its epilogue, routing, the fused
+sparse up/down step for the rows that fit, and the dense branch for the rows
+that overflow. Inputs are resident in HBM when the timed region starts; the
+L2 is flushed (a 256 MiB write) between steps, outside the timed events.
+
+Prints one JSON line (rank 0). Also measured in the same run: the library's
+own dense FFN at the same shape (speedup denominator), the same metric end to
+end through the C ABI with host buffers, and the CPU oracle on a bounded
+sample of the workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 0.5b] [--impl twell|reference]
+  python bench.py --sweep            # density x batch sweep, one JSON line per point
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from activation_sparse_gated_gemm_b200 import synth  # noqa: E402
+
+METRIC = "sparse gated-FFN tokens/s"
+FLUSH_BYTES = 256 << 20
+FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM (4 sub-partitions x 32)
+DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                 "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        p["source"] = "measured"
+        return p
+    except (OSError, ValueError):
+        return dict(DEFAULT_PEAKS)
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML every
+    ~10 ms in a background thread (read-only queries)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 -- clocks are reported as unavailable
+            self.max_mhz = None
+
+    def _run(self):
+        nv, h = self._nv, self._h
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.time(), sm, reasons))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        mask = 0
+        for _, _, r in self.samples:
+            mask |= r
+        names = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(s for _, s, _ in self.samples)),
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- helpers
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "activation_sparse_gated_gemm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources and this workload; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            t = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    return t.get("kernels", {}).get(kernel)
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+
+def cpu_oracle_rate(cfg, L, sample_rows: int, max_seconds: float = 20.0) -> dict:
+    """The oracle as it stands (hybrid forward: fp64 gate, pack, route,
+    per-token sparse step, dense rows) on the first rows of the workload."""
+    from oracle import twell_oracle as O
+
+    n = min(sample_rows, cfg.T)
+    done, t0 = 0, time.perf_counter()
+    while done < n and time.perf_counter() - t0 < max_seconds:
+        chunk = min(128, n - done)
+        rows = slice(done, done + chunk)
+        O.hybrid_ffn(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], cfg.tile, cfg.W)
+        done += chunk
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {done} of {cfg.T} tokens of the {cfg.name} layer, fp64 numpy oracle "
+                      f"(gate, pack, route, sparse step, dense rows), {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def algorithmic(cfg, n_ovf: int, nnz_stored: int, union_cols: int) -> dict:
+    T, d, f = cfg.T, cfg.d, cfg.f
+    nT = f // cfg.tile
+    gate_flops = 2.0 * T * d * f
+    dense_branch_flops = 6.0 * n_ovf * d * f
+    alg_bytes = (2.0 * d * f                  # Wg
+                 + 4.0 * d * union_cols       # active Wu columns and Wd rows
+                 + 4.0 * T * d                # x read, y written
+                 + 2 * 4.0 * nnz_stored       # TwELL nonzeros written and read (2 B idx + 2 B value)
+                 + 2 * 2.0 * T * nT)          # counts written and read
+    sparse_flops = 4.0 * d * nnz_stored       # up and down for every stored slot (non-overflow rows)
+    return {"gate_flops": gate_flops, "dense_branch_flops": dense_branch_flops, "alg_bytes": alg_bytes,
+            "sparse_flops": sparse_flops}
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+
+    from activation_sparse_gated_gemm_b200 import twell as tl
+
+    tl.load()
+    dev = torch.device("cuda", local)
+    cfg = synth.CONFIGS[args.config]
+    L = synth.make_layer(cfg, seed=args.seed)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    x = tl.to_device_bf16(L["x"], dev)
+    WgT = tl.to_device_bf16(L["WgT"], dev)
+    WuT = tl.to_device_bf16(L["WuT"], dev)
+    Wd = tl.to_device_bf16(L["Wd"], dev)
+    tw = tl.Twell(T, f, W, device=dev)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    ovf_rows = torch.empty((T,), dtype=torch.int32, device=dev)
+    n_ovf = torch.zeros((1,), dtype=torch.int32, device=dev)
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device=dev)
+    ws_dense = torch.empty(tl.dense_workspace_bytes(T, d, f), dtype=torch.uint8, device=dev)
+    y_dense = torch.empty_like(y)
+    st = tl.new_status(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def stages(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tl.gate_pack(x, WgT, tw, st)
+        if ev is not None:
+            ev[1].record(stream)
+        tl.route(tw, ovf_rows, n_ovf)
+        if ev is not None:
+            ev[2].record(stream)
+        tl.sparse_ffn(x, WuT, Wd, tw, y, True, st)
+        if ev is not None:
+            ev[3].record(stream)
+        tl.dense_rows_forward(x, WgT, WuT, Wd, ovf_rows, n_ovf, y, ws, st)
+        if ev is not None:
+            ev[4].record(stream)
+
+    K, Wm = args.steps, args.warmup
+    for _ in range(Wm):
+        flush.zero_()
+        stages()
+    torch.cuda.synchronize(dev)
+    if tl.status_get(st) != 0:
+        raise RuntimeError(f"device status {tl.status_get(st)} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for k in range(K):
+            flush.zero_()
+            stages(evs[k])
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)] for k in range(K)])
+    step_ms_local = float(per.sum(axis=1).mean())
+    step_ms = max_over_ranks(step_ms_local, world)
+    stage_ms = per.mean(axis=0)
+
+    # stats of this batch (for the algorithmic byte and FLOP counts)
+    counts = tw.counts.to(torch.int64)
+    n_ovf_h = int(n_ovf.item())
+    ovf_mask = tw.row_ovf.bool()
+    stored = torch.clamp(counts, max=W)
+    nnz_stored = int(stored[~ovf_mask].sum())
+    g = torch.empty((T, f), dtype=torch.bfloat16, device=dev)
+    tl.unpack(tw, g, st)
+    keep = ~ovf_mask
+    act = (g[keep] != 0).any(dim=0)
+    union_cols = int(act.sum())
+    del g
+
+    # dense baseline at the same shape
+    for _ in range(Wm):
+        flush.zero_()
+        tl.dense_ffn_forward(x, WgT, WuT, Wd, y_dense, ws_dense, st)
+    dense_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    for k in range(K):
+        flush.zero_()
+        dense_ev[k][0].record(stream)
+        tl.dense_ffn_forward(x, WgT, WuT, Wd, y_dense, ws_dense, st)
+        dense_ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    dense_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dense_ev])), world)
+
+    # end to end through the C ABI with host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    for _ in range(max(1, Wm // 2)):
+        x.copy_(x_host, non_blocking=True)
+        tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st)
+        y_host.copy_(y, non_blocking=True)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        flush.zero_()
+        e2e_ev[k][0].record(stream)
+        x.copy_(x_host, non_blocking=True)
+        tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st)
+        y_host.copy_(y, non_blocking=True)
+        e2e_ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in e2e_ev])), world)
+    status = tl.status_get(st)
+    if status != 0:
+        raise RuntimeError(f"device status {status} ({tl.status_str(status)})")
+
+    peaks = load_peaks()
+    alg = algorithmic(cfg, n_ovf_h, nnz_stored, union_cols)
+    hbm = peaks["hbm_gbs"] * 1e9
+    tc = peaks["bf16_tflops"] * 1e12
+    t_tc = (alg["gate_flops"] + alg["dense_branch_flops"]) / tc
+    t_hbm = alg["alg_bytes"] / hbm
+    t_roof = max(t_tc, t_hbm)
+    clocks = sampler.summary()
+    fp32_peak = (torch.cuda.get_device_properties(dev).multi_processor_count * FP32_LANES_PER_SM * 2
+                 * (clocks["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6)
+
+    names = ["gate_pack", "route", "sparse_ffn", "dense_rows"]
+    kern = {
+        "gate_pack": {"bound": "tensor", "work": alg["gate_flops"], "peak": tc, "unit": "TFLOP/s", "scale": 1e12},
+        "sparse_ffn": {"bound": "alu", "work": alg["sparse_flops"], "peak": fp32_peak, "unit": "TFLOP/s",
+                       "scale": 1e12},
+        "dense_rows": {"bound": "tensor", "work": alg["dense_branch_flops"], "peak": tc, "unit": "TFLOP/s",
+                       "scale": 1e12},
+    }
+    dom = max(("gate_pack", "sparse_ffn", "dense_rows"), key=lambda n: stage_ms[names.index(n)])
+    kd = kern[dom]
+    ms = float(stage_ms[names.index(dom)])
+    achieved = kd["work"] / (ms * 1e-3) / kd["scale"]
+    peak = kd["peak"] / kd["scale"]
+    traffic = measured_traffic(dom)
+
+    res = {
+        "metric": METRIC,
+        "value": world * T / (step_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded generator; no dataset or trained weights)",
+        "config": {"workload": f"{cfg.name}-like FFN layer forward, hybrid TwELL", "tokens": T, "d_model": d,
+                   "d_ff": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
+                   "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "roofline": {"kernel": dom, "bound": kd["bound"], "achieved": achieved, "peak": peak, "unit": kd["unit"],
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": ("fp32 FMA lanes x 2 x max SM clock" if kd["bound"] == "alu"
+                                     else f"{peaks['source']} bf16 burst")},
+        "path_roofline": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6, "t_roof_us": t_roof * 1e6,
+                          "frac": t_roof / (step_ms * 1e-3),
+                          "frac_gate_only": (alg["gate_flops"] / tc) / (step_ms * 1e-3),
+                          "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TF/s"},
+        "stages_ms": {n: float(v) for n, v in zip(names, stage_ms)},
+        "dense_ffn_ms": dense_ms,
+        "speedup_vs_own_dense": dense_ms / step_ms,
+        "batch_stats": {"n_ovf": n_ovf_h, "nnz_stored": nnz_stored, "union_cols": union_cols,
+                        "mean_density": float(counts.sum()) / (T * f)},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
+        "gpu_launches": 6 * K,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_oracle_rate(cfg, L, args.cpu_sample)
+    return res
+
+
+# ---------------------------------------------------------------- reference arm
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, on the host cores, on bounded samples of the
+    same workload; same metric and unit as the GPU arm."""
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS[args.config]
+    L = synth.make_layer(cfg, seed=args.seed)
+    sample = max(1, min(cfg.T, args.cpu_sample // 4))
+    from oracle import twell_oracle as O
+
+    def step():
+        O.hybrid_ffn(L["x"][:sample], L["WgT"], L["WuT"], L["Wd"], cfg.tile, cfg.W)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = sample / dt
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
+        "config": {"workload": f"{cfg.name}-like FFN layer forward, hybrid TwELL", "tokens": cfg.T,
+                   "d_model": cfg.d, "d_ff": cfg.f, "tile": cfg.tile, "ell_width": cfg.W,
+                   "density": cfg.density, "dead_frac": cfg.dead_frac},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{sample} of {cfg.T} tokens per step (fp64 numpy oracle)"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="twell", choices=["twell", "reference"])
+    ap.add_argument("--config", default="0.5b", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-sample", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    world, rank, local = dist_setup(args)
+    try:
+        res = run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,193 @@
+/*
+ * twell.h -- C ABI of the TwELL sparse ReLU-gated FFN forward pass (B200, sm_100a).
+ *
+ * The layer is y = (ReLU(x Wg) * (x Wu)) Wd. Hidden units whose gate is not
+ * strictly positive are exact zeros and are skipped: the gate GEMM packs its
+ * ReLU output into Tile-wise ELLPACK (TwELL) in its own epilogue, with no
+ * separate pack launch and no extra pass over memory, and a fused kernel then
+ * computes the up and down projections only for the stored hidden units,
+ * keeping the hidden activations on chip. Rows whose nonzeros do not fit the
+ * ELL width go to a dense branch.
+ *
+ * Sources: intellectnews.ru, "Sakana AI и NVIDIA ... TwELL" -- sections
+ * "Формат TwELL вместо классической sparse-упаковки" (format, packed at the
+ * end of the producing pass), "Слитые CUDA-ядра для инференса и гибрид для
+ * обучения" (fused inference kernel; hybrid sparse/dense rows) and
+ * "Минимальные изменения в рецепте обучения" (ReLU gate gives exact zeros);
+ * gate.com post 20977915, paragraph on TwELL (tiles packed locally by each
+ * compute unit).
+ *
+ * Conventions for every entry point:
+ *   - bf16 values travel as uint16_t bit patterns.
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no memory and keeps no per-call state. It is safe to call from
+ *     several host threads on distinct buffers.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are stream-ordered and never synchronise the host.
+ *   - Argument errors are returned synchronously and nothing is launched.
+ *     Conditions found on the device (ELL overflow in the non-hybrid forward,
+ *     an out-of-range stored index, a bounded wait that gave up) are raised
+ *     into the caller's int32 `dev_status` with an atomic max; `dev_status`
+ *     is sticky until the caller resets it (twell_status_reset).
+ *   - Every pointer must be 16-byte aligned.
+ *
+ * Shapes: T tokens (T >= 0; T == 0 is a no-op), d = d_model, f = d_ff.
+ *   d % 64 == 0, 64 <= d <= 4096; f % 128 == 0, 128 <= f <= 32767;
+ *   tile == 128; W % 8 == 0, 8 <= W <= 128.
+ *
+ * Layouts (row-major):
+ *   x   [T][d]   bf16 activations
+ *   WgT [f][d]   gate weight, transposed (row j = column j of Wg; this is the
+ *                weight of an nn.Linear(d, f))
+ *   WuT [f][d]   up weight, transposed likewise
+ *   Wd  [f][d]   down weight (row j multiplies hidden unit j)
+ *   y   [T][d]   bf16 output
+ */
+#ifndef TWELL_H
+#define TWELL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum twell_status {
+  TWELL_OK = 0,
+  TWELL_ERR_NULL = 1,        /* a required pointer is NULL */
+  TWELL_ERR_SHAPE = 2,       /* a size is outside the ranges above, or tw does not match */
+  TWELL_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  TWELL_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the size query */
+  TWELL_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed (launch, tensor map) */
+  TWELL_ERR_DEVICE = 6,      /* the current device is not compute capability 10.0 */
+  /* device-side codes, raised into dev_status */
+  TWELL_ERR_OVERFLOW = 16,   /* a row of the non-hybrid forward had a tile count > W */
+  TWELL_ERR_INDEX = 17,      /* a stored column index was outside [0, f) */
+  TWELL_ERR_TIMEOUT = 18     /* a bounded on-chip wait gave up; outputs are undefined */
+} twell_status;
+
+/*
+ * TwELL buffers (Tile-wise ELLPACK of ReLU(x Wg)), all caller-owned device memory.
+ * The columns are cut into nT = f / tile tiles. For row t and tile c:
+ *   counts[t*nT + c]          true number of strictly positive gate values in
+ *                             the tile (not capped at W)
+ *   idx [(t*nT + c)*W + s]    global column index j (0..f-1) of the s-th
+ *                             positive value in ascending column order
+ *   vals[(t*nT + c)*W + s]    bf16 (nearest-even) of ReLU(z[t, j])
+ * for s < min(count, W). Slots from min(count, W) on are unspecified.
+ *   row_ovf[t]                1 iff some tile of row t has count > W, else 0.
+ */
+typedef struct twell_t {
+  int16_t* counts;   /* [T][nT]    */
+  int16_t* idx;      /* [T][nT][W] */
+  uint16_t* vals;    /* [T][nT][W] bf16 bits */
+  uint8_t* row_ovf;  /* [T]        */
+  int32_t T, f, tile, W;
+} twell_t;
+
+/*
+ * Gate GEMM with the TwELL pack in its epilogue (steps: z = x Wg on the tensor
+ * cores, ReLU, per-row per-tile compaction; source: the format section above).
+ * Writes tw->counts, tw->idx, tw->vals, tw->row_ovf. tw->T, tw->f must equal
+ * T, f; tw->tile must be 128.
+ */
+twell_status twell_gate_pack(const uint16_t* x, const uint16_t* WgT, int T, int d, int f,
+                             const twell_t* tw, int32_t* dev_status, void* stream);
+
+/*
+ * Fused sparse step alone, on an already packed tw: for each stored slot
+ * (j, g) of row t, u_j = x_t . Wu[:, j], h_j = g * u_j, y_t += h_j Wd[j, :]
+ * with fp32 accumulation; h never leaves the chip (source: the fused-kernel
+ * section above). Rows with row_ovf set are skipped (y rows left untouched)
+ * when skip_overflow_rows != 0; otherwise they use their first W slots, their
+ * y is undefined and dev_status is raised to TWELL_ERR_OVERFLOW.
+ */
+twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd,
+                              int T, int d, int f, const twell_t* tw, int skip_overflow_rows,
+                              uint16_t* y, int32_t* dev_status, void* stream);
+
+/*
+ * Whole non-hybrid forward: twell_gate_pack, then twell_sparse_ffn without
+ * skipping. If any row overflows, dev_status becomes TWELL_ERR_OVERFLOW and
+ * the y of the overflowing rows is undefined (other rows are correct).
+ */
+twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                               const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                               uint16_t* y, int32_t* dev_status, void* stream);
+
+/*
+ * Routing step of the hybrid route (source: the hybrid paragraph of the
+ * fused-kernel section above): ovf_rows[0..n_ovf) = rows with row_ovf set,
+ * in ascending order; *n_ovf (device int32) = their number. ovf_rows has T
+ * entries of room.
+ */
+twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream);
+
+/* Bytes of workspace needed by twell_ffn_hybrid_forward and
+ * twell_dense_rows_forward (worst case: every row overflows). */
+size_t twell_hybrid_workspace_bytes(int T, int d, int f);
+
+/*
+ * Dense branch of the hybrid route alone (source: the hybrid paragraph of the
+ * fused-kernel section above): for i < *n_rows (device int32, <= T), row
+ * r = rows[i] of y is set to the dense gated FFN of x[r] -- gate recomputed,
+ * ReLU(x Wg) * (x Wu) on the tensor cores, then times Wd. The rows are
+ * gathered into `workspace`, which also holds their hidden activations (size:
+ * twell_hybrid_workspace_bytes). Rows not listed are untouched. A listed row
+ * outside [0, T) is skipped and raises TWELL_ERR_INDEX.
+ */
+twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                      const uint16_t* Wd, int T, int d, int f, const int32_t* rows,
+                                      const int32_t* n_rows, uint16_t* y, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Whole hybrid forward = twell_gate_pack, twell_route, twell_sparse_ffn with
+ * overflowing rows skipped, and twell_dense_rows_forward on ovf_rows. Every
+ * row of y is written. `workspace` holds the gathered overflow rows and their
+ * hidden activations.
+ */
+twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                      const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                                      uint16_t* y, int32_t* ovf_rows, int32_t* n_ovf,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, void* stream);
+
+/* Bytes of workspace needed by twell_dense_ffn_forward (the [T][f] bf16 hidden
+ * activations). */
+size_t twell_dense_workspace_bytes(int T, int d, int f);
+
+/*
+ * Dense ReLU-gated FFN on the tensor cores, no sparsity: one GEMM against
+ * [Wg | Wu] with ReLU(z) * u in its epilogue (h stored as bf16 in workspace),
+ * then h Wd. This is the library's own dense baseline for the same layer.
+ */
+twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                     const uint16_t* Wd, int T, int d, int f, uint16_t* y,
+                                     void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream);
+
+/*
+ * TwELL -> dense bf16 g[T][f]: zeros everywhere except the stored slots
+ * (slots below min(count, W); overflowing rows unpack only what was stored).
+ */
+twell_status twell_unpack(const twell_t* tw, uint16_t* g_dense, int32_t* dev_status, void* stream);
+
+/* Zero dev_status (stream-ordered). */
+twell_status twell_status_reset(int32_t* dev_status, void* stream);
+
+/* Synchronise `stream` and copy *dev_status to *host_out (blocks the host). */
+twell_status twell_status_get(const int32_t* dev_status, void* stream, int32_t* host_out);
+
+/* Static description of a status code. */
+const char* twell_status_str(int status);
+
+/* Library version string. */
+const char* twell_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TWELL_H */

@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function the header declares, and rejects bad arguments synchronously
+before touching the device. No call here launches anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from activation_sparse_gated_gemm_b200 import build as tb
+from activation_sparse_gated_gemm_b200 import twell as tl
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "twell.h")
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails its checks first
+MIS = 0x10008   # misaligned
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tb.build()
+    return tl.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(twell_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_library_agree(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(tl.EXPORTED)
+    assert lib.twell_version().decode().startswith("twell-b200")
+
+
+def tw_desc(T=64, f=512, W=16, tile=128, ptr=FAKE):
+    return tl.twell_t(ptr, ptr, ptr, ptr, T, f, tile, W)
+
+
+def call_pack(lib, T=64, d=128, f=512, tw=None, x=FAKE, w=FAKE, st=FAKE):
+    tw = tw or tw_desc(T, f)
+    return lib.twell_gate_pack(x, w, T, d, f, ctypes.byref(tw), st, None)
+
+
+def test_shape_errors(lib):
+    assert call_pack(lib, T=-1, tw=tw_desc(T=-1)) == tl.TWELL_ERR_SHAPE
+    assert call_pack(lib, d=100) == tl.TWELL_ERR_SHAPE        # d % 64
+    assert call_pack(lib, d=8192) == tl.TWELL_ERR_SHAPE       # d > 4096
+    assert call_pack(lib, f=500, tw=tw_desc(f=500)) == tl.TWELL_ERR_SHAPE
+    assert call_pack(lib, f=32768, tw=tw_desc(f=32768)) == tl.TWELL_ERR_SHAPE
+    assert call_pack(lib, tw=tw_desc(T=65)) == tl.TWELL_ERR_SHAPE    # descriptor mismatch
+    assert call_pack(lib, tw=tw_desc(W=12)) == tl.TWELL_ERR_SHAPE    # W % 8
+    assert call_pack(lib, tw=tw_desc(W=136)) == tl.TWELL_ERR_SHAPE   # W > 128
+    assert call_pack(lib, tw=tw_desc(tile=64)) == tl.TWELL_ERR_SHAPE
+
+
+def test_null_and_alignment_errors(lib):
+    assert call_pack(lib, x=None) == tl.TWELL_ERR_NULL
+    assert call_pack(lib, st=None) == tl.TWELL_ERR_NULL
+    assert lib.twell_gate_pack(FAKE, FAKE, 64, 128, 512, None, FAKE, None) == tl.TWELL_ERR_NULL
+    assert call_pack(lib, x=MIS) == tl.TWELL_ERR_ALIGN
+    assert call_pack(lib, tw=tw_desc(ptr=MIS)) == tl.TWELL_ERR_ALIGN
+    assert call_pack(lib, tw=tw_desc(ptr=0)) == tl.TWELL_ERR_NULL
+
+
+def test_zero_tokens_returns_without_launching(lib):
+    tw = tw_desc(T=0)
+    assert lib.twell_gate_pack(None, None, 0, 128, 512, ctypes.byref(tw), None, None) == tl.TWELL_OK
+    assert lib.twell_ffn_forward(None, None, None, None, 0, 128, 512, ctypes.byref(tw), None, None,
+                                 None) == tl.TWELL_OK
+
+
+def test_workspace_queries_and_errors(lib):
+    T, d, f = 1000, 1536, 4096
+    hyb = lib.twell_hybrid_workspace_bytes(T, d, f)
+    den = lib.twell_dense_workspace_bytes(T, d, f)
+    assert hyb >= T * (d + f) * 2 and hyb % 256 == 0
+    assert den >= T * f * 2 and den % 256 == 0
+    assert lib.twell_hybrid_workspace_bytes(0, d, f) == 0
+    tw = tw_desc(T, f, 32)
+    r = lib.twell_ffn_hybrid_forward(FAKE, FAKE, FAKE, FAKE, T, d, f, ctypes.byref(tw), FAKE, FAKE, FAKE,
+                                     FAKE, hyb - 1, FAKE, None)
+    assert r == tl.TWELL_ERR_WORKSPACE
+    r = lib.twell_dense_ffn_forward(FAKE, FAKE, FAKE, FAKE, T, d, f, FAKE, None, den, FAKE, None)
+    assert r == tl.TWELL_ERR_WORKSPACE
+    r = lib.twell_dense_rows_forward(FAKE, FAKE, FAKE, FAKE, T, d, f, FAKE, FAKE, FAKE, MIS, hyb, FAKE, None)
+    assert r == tl.TWELL_ERR_ALIGN
+
+
+def test_status_strings(lib):
+    for code in (0, 1, 2, 3, 4, 5, 6, 16, 17, 18):
+        s = tl.status_str(code)
+        assert s and s != "unknown status"
+    assert tl.status_str(99) == "unknown status"
