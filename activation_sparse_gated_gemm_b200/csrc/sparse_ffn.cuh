@@ -3,7 +3,7 @@
 //       u_j = x_t . Wu[:, j]          (fp32, reduced across the warp)
 //       h_j = g * u_j                 (kept in a register, never stored)
 //       y_t += h_j * Wd[j, :]         (fp32 accumulators in registers)
-// then y_t is rounded to bf16 once (intellectnews.ru "Sakana AI и NVIDIA ...
+// then y_t is stored in fp32 (intellectnews.ru "Sakana AI и NVIDIA ...
 // TwELL", section "Слитые CUDA-ядра для инференса и гибрид для обучения":
 // several FFN steps in one pass, intermediates not written to global memory).
 //
@@ -24,7 +24,7 @@ struct SparseParams {
   const int16_t* idx;
   const uint16_t* vals;
   const uint8_t* row_ovf;
-  uint16_t* y;
+  float* y;
   int T, d, f, nT, W;
   int skip_ovf;
   int* dev_status;
@@ -144,12 +144,9 @@ __global__ void __launch_bounds__(kSparseWarps * 32) sparse_ffn_warp_kernel(cons
   for (int i = 0; i < NCH; ++i) {
     const int k0 = (i * 32 + lane) * 8;
     if (k0 < d) {
-      uint4 o;
-      o.x = pack_bf16x2(y[i][0], y[i][1]);
-      o.y = pack_bf16x2(y[i][2], y[i][3]);
-      o.z = pack_bf16x2(y[i][4], y[i][5]);
-      o.w = pack_bf16x2(y[i][6], y[i][7]);
-      *reinterpret_cast<uint4*>(p.y + static_cast<size_t>(t) * d + k0) = o;
+      float4* dst = reinterpret_cast<float4*>(p.y + static_cast<size_t>(t) * d + k0);
+      dst[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+      dst[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
     }
   }
 }

@@ -166,7 +166,7 @@ twell_status launch_sparse_n(const SparseParams& p, cudaStream_t s) {
 }
 
 twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
-                         const twell_t* tw, int skip, uint16_t* y, int32_t* dev_status, cudaStream_t s) {
+                         const twell_t* tw, int skip, float* y, int32_t* dev_status, cudaStream_t s) {
   SparseParams p{};
   p.x = x;
   p.WuT = WuT;
@@ -205,13 +205,15 @@ twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t*
 }
 
 // Dense gated FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu)
-// into h_buf [M][f], then out[row_map[i]] = h[i] Wd (row_map null: identity).
+// into h_buf, then out[row_map[i]] = h[i] Wd (row_map null: identity). With split, h_buf is
+// [M][2f] holding bf16(h) and the bf16 remainder, and the down GEMM runs K = 2f.
 twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const uint16_t* WgT, const uint16_t* WuT,
-                        const uint16_t* Wd, int d, int f, uint16_t* h_buf, const int* row_map, uint16_t* y,
-                        int y_rows, int32_t* dev_status, cudaStream_t s, int sms) {
+                        const uint16_t* Wd, int d, int f, uint16_t* h_buf, bool split, const int* row_map,
+                        float* y, int y_rows, int32_t* dev_status, cudaStream_t s, int sms) {
+  const int hk = split ? 2 * f : f;
   CUtensorMap ma, mg, mu, mh, md;
   if (!make_map(&ma, a_rows, d, M, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, 128) ||
-      !make_map(&mu, WuT, d, f, kBK, 128) || !make_map(&mh, h_buf, f, M, kBK, kBM) ||
+      !make_map(&mu, WuT, d, f, kBK, 128) || !make_map(&mh, h_buf, hk, M, kBK, kBM) ||
       !make_map(&md, Wd, d, f, 64, kBK))
     return TWELL_ERR_CUDA;
   GemmParams p1{};
@@ -220,7 +222,8 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
   p1.N = f;
   p1.K = d;
   p1.out = h_buf;
-  p1.ldo = f;
+  p1.ldo = hk;
+  p1.h_split = split ? 1 : 0;
   p1.dev_status = dev_status;
   const int g1 = M_dev ? sms : gemm_grid(M, f, 128, sms);
   TW_TRY(launch_gemm<kModeGateUp>(ma, mg, mu, p1, g1, s));
@@ -228,8 +231,9 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
   p2.M = M;
   p2.M_dev = M_dev;
   p2.N = d;
-  p2.K = f;
-  p2.out = y;
+  p2.K = hk;
+  p2.k_wrap = split ? f : 0;
+  p2.out_f32 = y;
   p2.ldo = d;
   p2.row_map = row_map;
   p2.out_rows = y_rows;
@@ -242,11 +246,11 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Dense branch: gather x[rows[i]] into xo, dense gated FFN into ho, scatter to y.
 twell_status dense_rows_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
-                             int T, int d, int f, const int32_t* rows, const int32_t* n_rows, uint16_t* y,
+                             int T, int d, int f, const int32_t* rows, const int32_t* n_rows, float* y,
                              uint16_t* xo, uint16_t* ho, int32_t* dev_status, cudaStream_t s, int sms) {
   gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, rows, n_rows, T, xo, dev_status);
   TW_TRY(cuda_ok(cudaGetLastError()));
-  return dense_impl(xo, T, n_rows, WgT, WuT, Wd, d, f, ho, rows, y, T, dev_status, s, sms);
+  return dense_impl(xo, T, n_rows, WgT, WuT, Wd, d, f, ho, true, rows, y, T, dev_status, s, sms);
 }
 
 }  // namespace
@@ -267,7 +271,7 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* WgT, int T, int 
 }
 
 twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
-                              const twell_t* tw, int skip_overflow_rows, uint16_t* y, int32_t* dev_status,
+                              const twell_t* tw, int skip_overflow_rows, float* y, int32_t* dev_status,
                               void* stream) {
   TW_TRY(check_shape(T, d, f));
   TW_TRY(check_tw(tw, T, f));
@@ -279,7 +283,7 @@ twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint
 }
 
 twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
-                               int T, int d, int f, const twell_t* tw, uint16_t* y, int32_t* dev_status,
+                               int T, int d, int f, const twell_t* tw, float* y, int32_t* dev_status,
                                void* stream) {
   TW_TRY(check_shape(T, d, f));
   TW_TRY(check_tw(tw, T, f));
@@ -304,11 +308,11 @@ twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, v
 
 size_t twell_hybrid_workspace_bytes(int T, int d, int f) {
   if (T <= 0 || d <= 0 || f <= 0) return 0;
-  return round_up(static_cast<size_t>(T) * d * 2, 256) + round_up(static_cast<size_t>(T) * f * 2, 256);
+  return round_up(static_cast<size_t>(T) * d * 2, 256) + round_up(static_cast<size_t>(T) * f * 4, 256);
 }
 
 twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
-                                      const uint16_t* Wd, int T, int d, int f, const twell_t* tw, uint16_t* y,
+                                      const uint16_t* Wd, int T, int d, int f, const twell_t* tw, float* y,
                                       int32_t* ovf_rows, int32_t* n_ovf, void* workspace, size_t workspace_bytes,
                                       int32_t* dev_status, void* stream) {
   TW_TRY(check_shape(T, d, f));
@@ -332,7 +336,7 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
 
 twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                       const uint16_t* Wd, int T, int d, int f, const int32_t* rows,
-                                      const int32_t* n_rows, uint16_t* y, void* workspace,
+                                      const int32_t* n_rows, float* y, void* workspace,
                                       size_t workspace_bytes, int32_t* dev_status, void* stream) {
   TW_TRY(check_shape(T, d, f));
   if (T == 0) return TWELL_OK;
@@ -355,7 +359,7 @@ size_t twell_dense_workspace_bytes(int T, int d, int f) {
 }
 
 twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
-                                     const uint16_t* Wd, int T, int d, int f, uint16_t* y, void* workspace,
+                                     const uint16_t* Wd, int T, int d, int f, float* y, void* workspace,
                                      size_t workspace_bytes, int32_t* dev_status, void* stream) {
   TW_TRY(check_shape(T, d, f));
   if (T == 0) return TWELL_OK;
@@ -364,7 +368,7 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
   if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  return dense_impl(x, T, nullptr, WgT, WuT, Wd, d, f, static_cast<uint16_t*>(workspace), nullptr, y, T,
+  return dense_impl(x, T, nullptr, WgT, WuT, Wd, d, f, static_cast<uint16_t*>(workspace), false, nullptr, y, T,
                     dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 

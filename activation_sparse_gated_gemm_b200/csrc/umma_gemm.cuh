@@ -12,10 +12,13 @@
 //                  gate.com post 20977915, paragraph on TwELL).
 //   kModeGateUp -- z and u = x . Wu in one MMA (B = 128 rows of Wg stacked on
 //                  the same 128 rows of Wu); the epilogue stores
-//                  h = ReLU(z) * u as bf16. The dense layer's first half.
+//                  h = ReLU(z) * u as bf16, and optionally the bf16 remainder
+//                  h - bf16(h) beside it. The dense layer's first half.
 //   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
-//                  epilogue stores bf16 rows, optionally scattered through a
-//                  row map (the dense branch of the hybrid route).
+//                  epilogue stores fp32 rows, optionally scattered through a
+//                  row map (the dense branch of the hybrid route). With the
+//                  remainder stored, K runs over [h | h - bf16(h)] against
+//                  [Wd ; Wd], which removes the bf16 rounding of h to ~2^-16.
 //
 // Structure: one CTA per SM walks output tiles of 128 x 256 (x 128 h-columns
 // for kModeGateUp). Warp 0 issues TMA loads into a 4-stage shared-memory ring,
@@ -62,11 +65,17 @@ struct GemmParams {
   uint8_t* row_ovf;
   int nT;
   int W;
-  // kModeGateUp / kModeDown output (bf16, leading dimension ldo)
+  // kModeGateUp output (bf16) / kModeDown output (fp32), leading dimension ldo
   uint16_t* out;
+  float* out_f32;
   int ldo;
   const int* row_map;  // kModeDown: output row of each A row, or null
   int out_rows;        // valid range of output rows
+  // kModeGateUp: also store h_lo = bf16(h - bf16(h)) at column N + c (ldo = 2N).
+  int h_split;
+  // kModeDown: B rows are read at k mod k_wrap (k_wrap > 0), so K = 2 * k_wrap
+  // runs [h_hi | h_lo] against [Wd ; Wd].
+  int k_wrap;
   int* dev_status;
 };
 
@@ -145,9 +154,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * 128);
             tma_load_2d(b_dst + kBStageBytes / 2, &tmB1, &full[s], kb * kBK, n_blk * 128);
           } else {
+            const int kb_row = p.k_wrap > 0 ? (kb * kBK) % p.k_wrap : kb * kBK;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              tma_load_2d(b_dst + i * (kBStageBytes / 4), &tmB0, &full[s], n_blk * kBN + i * 64, kb * kBK);
+              tma_load_2d(b_dst + i * (kBStageBytes / 4), &tmB0, &full[s], n_blk * kBN + i * 64, kb_row);
           }
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -312,16 +322,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int col = n_blk * 128 + ch * 32;
           if (my_row < M && col < p.N) {
-            uint32_t hv[16];
+            uint32_t hv[16], lv[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float h0 = fmaxf(__uint_as_float(zr[2 * i]), 0.0f) * __uint_as_float(ur[2 * i]);
               const float h1 = fmaxf(__uint_as_float(zr[2 * i + 1]), 0.0f) * __uint_as_float(ur[2 * i + 1]);
               hv[i] = pack_bf16x2(h0, h1);
+              // remainder of the bf16 rounding, itself rounded to bf16
+              lv[i] = pack_bf16x2(h0 - __uint_as_float(hv[i] << 16), h1 - __uint_as_float(hv[i] & 0xffff0000u));
             }
             uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(my_row) * p.ldo + col);
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2], hv[4 * v + 3]);
+            if (p.h_split) {
+              uint4* dlo = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(my_row) * p.ldo + p.N + col);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) dlo[v] = make_uint4(lv[4 * v], lv[4 * v + 1], lv[4 * v + 2], lv[4 * v + 3]);
+            }
           }
         }
       } else {
@@ -345,12 +362,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int col = n_blk * kBN + ch * 32;
           if (valid && col < p.N) {
-            uint32_t yv[16];
+            uint4* dst = reinterpret_cast<uint4*>(p.out_f32 + static_cast<size_t>(orow) * p.ldo + col);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) yv[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(orow) * p.ldo + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(yv[4 * v], yv[4 * v + 1], yv[4 * v + 2], yv[4 * v + 3]);
+            for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
           }
         }
       }

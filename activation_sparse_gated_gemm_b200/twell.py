@@ -108,10 +108,17 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _bf16(name: str, t: torch.Tensor, shape: tuple) -> None:
-    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
-        raise ValueError(f"{name} must be a contiguous CUDA bfloat16 tensor of shape {shape}, "
+def _dev(name: str, t: torch.Tensor, shape: tuple, dtype) -> None:
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor of shape {shape}, "
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _bf16(name: str, t: torch.Tensor, shape: tuple) -> None:
+    if name == "y":
+        _dev(name, t, shape, torch.float32)
+    else:
+        _dev(name, t, shape, torch.bfloat16)
 
 
 class Twell:

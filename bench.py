@@ -218,7 +218,7 @@ def algorithmic(cfg, n_ovf: int, nnz_stored: int, union_cols: int) -> dict:
     dense_branch_flops = 6.0 * n_ovf * d * f
     alg_bytes = (2.0 * d * f                  # Wg
                  + 4.0 * d * union_cols       # active Wu columns and Wd rows
-                 + 4.0 * T * d                # x read, y written
+                 + 6.0 * T * d                # x read (bf16), y written (fp32)
                  + 2 * 4.0 * nnz_stored       # TwELL nonzeros written and read (2 B idx + 2 B value)
                  + 2 * 2.0 * T * nT)          # counts written and read
     sparse_flops = 4.0 * d * nnz_stored       # up and down for every stored slot (non-overflow rows)
@@ -241,7 +241,7 @@ def run_gpu(args, world, rank, local):
     WuT = tl.to_device_bf16(L["WuT"], dev)
     Wd = tl.to_device_bf16(L["Wd"], dev)
     tw = tl.Twell(T, f, W, device=dev)
-    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((T, d), dtype=torch.float32, device=dev)
     ovf_rows = torch.empty((T,), dtype=torch.int32, device=dev)
     n_ovf = torch.zeros((1,), dtype=torch.int32, device=dev)
     ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device=dev)
@@ -319,7 +319,7 @@ def run_gpu(args, world, rank, local):
 
     # end to end through the C ABI with host buffers
     x_host = x.cpu().pin_memory()
-    y_host = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    y_host = torch.empty((T, d), dtype=torch.float32).pin_memory()
     for _ in range(max(1, Wm // 2)):
         x.copy_(x_host, non_blocking=True)
         tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st)
@@ -397,7 +397,7 @@ def run_gpu(args, world, rank, local):
         "batch_stats": {"n_ovf": n_ovf_h, "nnz_stored": nnz_stored, "union_cols": union_cols,
                         "mean_density": float(counts.sum()) / (T * f)},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
+                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4},
         "gpu_launches": 6 * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }

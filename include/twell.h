@@ -41,7 +41,9 @@
  *                weight of an nn.Linear(d, f))
  *   WuT [f][d]   up weight, transposed likewise
  *   Wd  [f][d]   down weight (row j multiplies hidden unit j)
- *   y   [T][d]   bf16 output
+ *   y   [T][d]   fp32 output (accumulated in fp32 and stored without a final
+ *                rounding to bf16; the hidden activations of the dense paths
+ *                are held as bf16)
  */
 #ifndef TWELL_H
 #define TWELL_H
@@ -105,7 +107,7 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* WgT, int T, int 
  */
 twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd,
                               int T, int d, int f, const twell_t* tw, int skip_overflow_rows,
-                              uint16_t* y, int32_t* dev_status, void* stream);
+                              float* y, int32_t* dev_status, void* stream);
 
 /*
  * Whole non-hybrid forward: twell_gate_pack, then twell_sparse_ffn without
@@ -114,7 +116,7 @@ twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint
  */
 twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
-                               uint16_t* y, int32_t* dev_status, void* stream);
+                               float* y, int32_t* dev_status, void* stream);
 
 /*
  * Routing step of the hybrid route (source: the hybrid paragraph of the
@@ -132,14 +134,17 @@ size_t twell_hybrid_workspace_bytes(int T, int d, int f);
  * Dense branch of the hybrid route alone (source: the hybrid paragraph of the
  * fused-kernel section above): for i < *n_rows (device int32, <= T), row
  * r = rows[i] of y is set to the dense gated FFN of x[r] -- gate recomputed,
- * ReLU(x Wg) * (x Wu) on the tensor cores, then times Wd. The rows are
- * gathered into `workspace`, which also holds their hidden activations (size:
+ * h = ReLU(x Wg) * (x Wu) on the tensor cores, then h Wd. h is kept as a pair
+ * of bf16 values (bf16(h) and the bf16 of the remainder), so the rounding of
+ * the hidden activations costs ~2^-16 relative instead of 2^-8; rows routed
+ * here have many active units and large outputs. The rows are gathered into
+ * `workspace`, which also holds their hidden activations (size:
  * twell_hybrid_workspace_bytes). Rows not listed are untouched. A listed row
  * outside [0, T) is skipped and raises TWELL_ERR_INDEX.
  */
 twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                       const uint16_t* Wd, int T, int d, int f, const int32_t* rows,
-                                      const int32_t* n_rows, uint16_t* y, void* workspace,
+                                      const int32_t* n_rows, float* y, void* workspace,
                                       size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
@@ -150,7 +155,7 @@ twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, co
  */
 twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                       const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
-                                      uint16_t* y, int32_t* ovf_rows, int32_t* n_ovf,
+                                      float* y, int32_t* ovf_rows, int32_t* n_ovf,
                                       void* workspace, size_t workspace_bytes,
                                       int32_t* dev_status, void* stream);
 
@@ -160,11 +165,13 @@ size_t twell_dense_workspace_bytes(int T, int d, int f);
 
 /*
  * Dense ReLU-gated FFN on the tensor cores, no sparsity: one GEMM against
- * [Wg | Wu] with ReLU(z) * u in its epilogue (h stored as bf16 in workspace),
- * then h Wd. This is the library's own dense baseline for the same layer.
+ * [Wg | Wu] with ReLU(z) * u in its epilogue (h stored once as bf16 in
+ * workspace, as a standard bf16 layer does), then h Wd. This is the library's
+ * own dense baseline for the same layer; its error is that of one bf16
+ * rounding of h, |y - y_exact| <= 2^-8 sum_j |h_j Wd[j, :]| plus fp32 sums.
  */
 twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
-                                     const uint16_t* Wd, int T, int d, int f, uint16_t* y,
+                                     const uint16_t* Wd, int T, int d, int f, float* y,
                                      void* workspace, size_t workspace_bytes,
                                      int32_t* dev_status, void* stream);
 

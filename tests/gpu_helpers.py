@@ -59,9 +59,21 @@ def assert_y_close(y_gpu: np.ndarray, y_ref: np.ndarray, what: str = "y") -> flo
 
 
 def y_to_f64(y: torch.Tensor) -> np.ndarray:
-    return O.bf16_bits_to_f64(tl.bf16_bits(y))
+    return y.detach().double().cpu().numpy()
 
 
 def oracle_pack_rows(L: dict, rows, tile: int, W: int) -> dict:
     z = O.gate_preactivation(L["x"][rows], L["WgT"])
     return O.twell_pack(z, tile, W)
+
+
+def assert_dense_bf16_hidden_bound(y_gpu: np.ndarray, L: dict) -> None:
+    """A dense layer that stores h once as bf16 has |y - y_exact| <= 2^-8 *
+    sum_j |h_j Wd[j, k]| (one nearest rounding of each h_j to 8 significant
+    bits); 2^-7 leaves room for the fp32 sums."""
+    x = O.bf16_bits_to_f64(L["x"])
+    h = np.maximum(x @ O.bf16_bits_to_f64(L["WgT"]).T, 0) * (x @ O.bf16_bits_to_f64(L["WuT"]).T)
+    wd = O.bf16_bits_to_f64(L["Wd"])
+    y = h @ wd
+    bound = np.abs(h) @ np.abs(wd) * 2.0**-7 + 1e-6
+    assert np.all(np.abs(y_gpu - y) <= bound), float((np.abs(y_gpu - y) / bound).max())

@@ -1,0 +1,67 @@
+"""Parity at the full layer sizes, in the launch configuration bench.py times
+(the whole hybrid forward). Counts, overflow flags and routing are compared
+bit-exactly over every row (the fp64 oracle gate is computed in row chunks);
+the stored slots and y are compared on sampled rows, overflow rows included."""
+
+import numpy as np
+import pytest
+import torch
+
+from activation_sparse_gated_gemm_b200 import synth
+from activation_sparse_gated_gemm_b200 import twell as tl
+from oracle import twell_oracle as O
+from tests.gpu_helpers import assert_twell_equal, assert_y_close, upload
+
+pytestmark = pytest.mark.gpu
+
+CHUNK = 2048
+
+
+@pytest.mark.parametrize("name", ["0.5b", "1.5b", "2b"])
+def test_full_size_hybrid_forward(name):
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    cfg = synth.CONFIGS[name]
+    L = synth.make_layer(cfg, seed=0)
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    assert tl.status_get(st) == 0
+    counts = tw.counts.cpu().numpy()
+    row_ovf = tw.row_ovf.cpu().numpy()
+    idx = tw.idx.cpu().numpy()
+    vals = tl.bf16_bits(tw.vals)
+    yg = y.double().cpu().numpy()
+    assert np.isfinite(yg).all()
+
+    rng = np.random.default_rng(1)
+    sample = np.sort(rng.choice(T, size=256, replace=False))
+    all_counts = np.empty_like(counts)
+    for r0 in range(0, T, CHUNK):
+        rows = np.arange(r0, min(T, r0 + CHUNK))
+        ref = O.twell_pack(O.gate_preactivation(L["x"][rows], L["WgT"]), cfg.tile, W)
+        all_counts[rows] = ref["counts"]
+        assert np.array_equal(counts[rows], ref["counts"]), f"counts differ in rows {r0}.."
+        assert np.array_equal(row_ovf[rows], ref["row_ovf"])
+        sel = sample[(sample >= rows[0]) & (sample <= rows[-1])]
+        if sel.size:
+            got = {"counts": counts[sel], "row_ovf": row_ovf[sel], "idx": idx[sel], "vals": vals[sel]}
+            want = {k: ref[k][sel - r0] for k in ("counts", "row_ovf", "idx", "vals")}
+            assert_twell_equal(got, want, W)
+    ovf_ref = O.route_rows(all_counts, W)
+    n = int(n_ovf.item())
+    assert n == len(ovf_ref)
+    assert np.array_equal(ovf_rows[:n].cpu().numpy(), ovf_ref)
+    if name == "2b":
+        heavy = np.nonzero(L["p_t"] >= cfg.heavy_lo)[0]
+        assert set(heavy.tolist()) <= set(ovf_ref.tolist())
+
+    check = np.unique(np.concatenate([sample, ovf_ref[:64]]))
+    y_ref = O.gated_ffn(L["x"][check], L["WgT"], L["WuT"], L["Wd"])
+    assert_y_close(yg[check], y_ref)

@@ -9,8 +9,8 @@ import torch
 from activation_sparse_gated_gemm_b200 import synth
 from activation_sparse_gated_gemm_b200 import twell as tl
 from oracle import twell_oracle as O
-from tests.gpu_helpers import (assert_twell_equal, assert_y_close, oracle_pack_rows, run_pack,
-                               twell_to_host, upload, y_to_f64)
+from tests.gpu_helpers import (assert_dense_bf16_hidden_bound, assert_twell_equal, assert_y_close,
+                               oracle_pack_rows, run_pack, twell_to_host, upload, y_to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,7 +72,7 @@ def test_ffn_forward_non_hybrid(cfg, layers):
     L = layers[cfg.name]
     dev = upload(L)
     tw = tl.Twell(cfg.T, cfg.f, cfg.W)
-    y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device="cuda")
     st = tl.new_status()
     tl.ffn_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, st)
     status = tl.status_get(st)
@@ -89,7 +89,7 @@ def test_hybrid_forward(cfg, layers):
     L = layers[cfg.name]
     dev = upload(L)
     tw = tl.Twell(cfg.T, cfg.f, cfg.W)
-    y = torch.full((cfg.T, cfg.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((cfg.T, cfg.d), float("nan"), dtype=torch.float32, device="cuda")
     ovf_rows = torch.full((cfg.T,), -7, dtype=torch.int32, device="cuda")
     n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
     ws = torch.empty(tl.hybrid_workspace_bytes(cfg.T, cfg.d, cfg.f), dtype=torch.uint8, device="cuda")
@@ -121,7 +121,7 @@ def test_sparse_step_on_oracle_packed_input(cfg, layers):
     tw.idx.copy_(torch.from_numpy(want["idx"]))
     tw.vals.copy_(torch.from_numpy(want["vals"].view(np.int16)).view(torch.bfloat16))
     tw.row_ovf.copy_(torch.from_numpy(want["row_ovf"]))
-    sentinel = torch.full((cfg.T, cfg.d), 3.0, dtype=torch.bfloat16, device="cuda")
+    sentinel = torch.full((cfg.T, cfg.d), 3.0, dtype=torch.float32, device="cuda")
     y = sentinel.clone()
     st = tl.new_status()
     tl.sparse_ffn(dev["x"], dev["WuT"], dev["Wd"], tw, y, True, st)
@@ -137,28 +137,28 @@ def test_sparse_step_on_oracle_packed_input(cfg, layers):
 def test_dense_ffn(cfg, layers):
     L = layers[cfg.name]
     dev = upload(L)
-    y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device="cuda")
     ws = torch.empty(tl.dense_workspace_bytes(cfg.T, cfg.d, cfg.f), dtype=torch.uint8, device="cuda")
     st = tl.new_status()
     tl.dense_ffn_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], y, ws, st)
     assert tl.status_get(st) == 0
-    assert_y_close(y_to_f64(y), O.gated_ffn(L["x"], L["WgT"], L["WuT"], L["Wd"]))
+    assert_dense_bf16_hidden_bound(y_to_f64(y), L)
 
 
 def test_dense_ffn_unquantised_inputs():
-    """Plain N(0,1) bf16 inputs (no grid): the tensor-core GEMMs still meet
-    the tolerance against fp64."""
+    """Plain N(0,1) bf16 inputs (no grid): the tensor-core GEMMs stay within
+    the bound of one bf16 rounding of h against fp64."""
     rng = np.random.default_rng(0)
     T, d, f = 384, 512, 1280
     mk = lambda *s, sc=1.0: synth.f32_to_bf16_bits((rng.standard_normal(s) * sc).astype(np.float32))
     L = {"x": mk(T, d), "WgT": mk(f, d, sc=d**-0.5), "WuT": mk(f, d, sc=d**-0.5), "Wd": mk(f, d, sc=f**-0.5)}
     dev = upload(L)
-    y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
     ws = torch.empty(tl.dense_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
     st = tl.new_status()
     tl.dense_ffn_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], y, ws, st)
     assert tl.status_get(st) == 0
-    assert_y_close(y_to_f64(y), O.gated_ffn(L["x"], L["WgT"], L["WuT"], L["Wd"]))
+    assert_dense_bf16_hidden_bound(y_to_f64(y), L)
 
 
 def test_all_negative_gate_gives_empty_pack_and_zero_output(layers):
@@ -169,7 +169,7 @@ def test_all_negative_gate_gives_empty_pack_and_zero_output(layers):
     L["WgT"] = synth.f32_to_bf16_bits(wg.astype(np.float32))
     dev = upload(L)
     tw = tl.Twell(cfg.T, cfg.f, cfg.W)
-    y = torch.full((cfg.T, cfg.d), 5.0, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((cfg.T, cfg.d), 5.0, dtype=torch.float32, device="cuda")
     st = tl.new_status()
     tl.ffn_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, st)
     assert tl.status_get(st) == 0
@@ -185,7 +185,7 @@ def test_all_positive_gate_full_width_equals_dense(layers):
     L["WgT"] = synth.f32_to_bf16_bits(wg.astype(np.float32))
     dev = upload(L)
     tw = tl.Twell(cfg.T, cfg.f, cfg.W)
-    y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device="cuda")
     st = tl.new_status()
     tl.ffn_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, st)
     assert tl.status_get(st) == 0
@@ -197,7 +197,7 @@ def test_zero_tokens_is_a_noop():
     x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
     w = torch.zeros((256, 128), dtype=torch.bfloat16, device="cuda")
     tw = tl.Twell(0, 256, 16)
-    y = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((0, 128), dtype=torch.float32, device="cuda")
     st = tl.new_status()
     tl.ffn_forward(x, w, w, w, tw, y, st)
     assert tl.status_get(st) == 0
@@ -208,7 +208,7 @@ def test_overflow_status_is_sticky_and_resettable(layers):
     L = layers[cfg.name]
     dev = upload(L)
     tw = tl.Twell(cfg.T, cfg.f, cfg.W)
-    y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device="cuda")
     st = tl.new_status()
     tl.ffn_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, st)
     assert tl.status_get(st) == tl.TWELL_ERR_OVERFLOW
@@ -227,7 +227,7 @@ def test_out_of_range_index_is_reported_not_read(layers):
     torch.cuda.synchronize()
     row = int(torch.nonzero(tw.counts[:, 0] > 0)[0, 0])
     tw.idx[row, 0, 0] = 32000  # beyond f
-    y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device="cuda")
     st = tl.new_status()
     tl.sparse_ffn(dev["x"], dev["WuT"], dev["Wd"], tw, y, True, st)
     assert tl.status_get(st) == tl.TWELL_ERR_INDEX
