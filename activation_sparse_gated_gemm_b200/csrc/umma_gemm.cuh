@@ -45,10 +45,12 @@ constexpr int kEpiBytes = 4 * 32 * kEpiPitch * 4;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
 
+constexpr int kStageSlotBytes = 32;  // per epilogue thread: 8 staged (idx, value) slots
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kAStageBytes;
 constexpr int kOffEpi = kOffB + kStages * kBStageBytes;
-constexpr int kOffBar = kOffEpi + kEpiBytes;
+constexpr int kOffSlots = kOffEpi + kEpiBytes;
+constexpr int kOffBar = kOffSlots + 128 * kStageSlotBytes;
 constexpr int kNumBars = 2 * kStages + 4 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kGemmSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
@@ -243,7 +245,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
     float* ebuf = reinterpret_cast<float*>(smem + kOffEpi) + (warp - 2) * 32 * kEpiPitch;
-    const uint32_t lt_mask = (1u << lane) - 1u;
     int buf = 0;
     uint32_t tph = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -261,50 +262,68 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int my_row = row_base + lane;
 
       if (MODE == kModeTwell) {
+        // Each thread owns one row (its TMEM lane). Per 32-column chunk it
+        // builds the mask of strictly positive values, then walks only the set
+        // bits in ascending column order, appending (column, bf16 value) to its
+        // row's slot list. Slots go through an 8-entry staging buffer in shared
+        // memory and leave as 16-byte stores.
+        float* vrow = ebuf + lane * kEpiPitch;
+        uint8_t* stg = smem + kOffSlots + (threadIdx.x - 64) * kStageSlotBytes;
+        uint16_t* stg_idx = reinterpret_cast<uint16_t*>(stg);
+        uint16_t* stg_val = reinterpret_cast<uint16_t*>(stg + 16);
+        const bool row_ok = my_row < M;
 #pragma unroll 1
         for (int sub = 0; sub < 2; ++sub) {
           const int c = n_blk * 2 + sub;  // TwELL column tile
-          int cnt = 0;                    // running count of my_row in tile c
+          const bool tile_ok = row_ok && c < p.nT;
+          const size_t slot0 = (static_cast<size_t>(my_row) * p.nT + c) * p.W;
+          int cnt = 0;  // nonzeros of my_row in tile c so far (not capped)
 #pragma unroll 1
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t r[32];
+            __syncwarp();
             tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(sub * 128 + ch * 32), r);
             tmem_wait_ld();
             if (sub == 1 && ch == 3) {
               tc_fence_before();
               mbar_arrive(&tempty[buf]);
             }
-            if (c >= p.nT) continue;
-            // Transpose the 32x32 block through shared memory so that each row
-            // can be compacted with one ballot across its 32 columns.
-            uint32_t mine = 0;
+            if (!tile_ok) continue;
+            uint32_t mask = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float v = __uint_as_float(r[i]);
-              ebuf[lane * kEpiPitch + i] = v;
-              mine |= (v > 0.0f ? 1u : 0u) << i;
-            }
-            const int before = cnt;
-            cnt += __popc(mine);
-            __syncwarp();
-            const int col = c * 128 + ch * 32 + lane;
-#pragma unroll 4
-            for (int rr = 0; rr < 32; ++rr) {
-              const float v = ebuf[rr * kEpiPitch + lane];
-              const bool act = v > 0.0f;
-              const uint32_t mask = __ballot_sync(0xffffffffu, act);
-              const int base = __shfl_sync(0xffffffffu, before, rr);
-              const int pos = base + __popc(mask & lt_mask);
-              const int row = row_base + rr;
-              if (act && pos < p.W && row < M) {
-                const size_t off = (static_cast<size_t>(row) * p.nT + c) * p.W + pos;
-                p.idx[off] = static_cast<int16_t>(col);
-                p.vals[off] = f32_to_bf16_bits(v);
+            for (int i = 0; i < 32; ++i) mask |= (static_cast<int32_t>(r[i]) > 0 ? 1u : 0u) << i;
+            if (mask == 0) continue;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) vrow[i] = __uint_as_float(r[i]);
+            const int col0 = c * 128 + ch * 32;
+            while (mask != 0) {
+              const int i = __ffs(mask) - 1;
+              mask &= mask - 1u;
+              if (cnt < p.W) {
+                const int k = cnt & 7;
+                stg_idx[k] = static_cast<uint16_t>(col0 + i);
+                stg_val[k] = f32_to_bf16_bits(vrow[i]);
+                if (k == 7) {
+                  const size_t off = slot0 + (cnt - 7);
+                  *reinterpret_cast<uint4*>(p.idx + off) = *reinterpret_cast<const uint4*>(stg_idx);
+                  *reinterpret_cast<uint4*>(p.vals + off) = *reinterpret_cast<const uint4*>(stg_val);
+                }
               }
+              ++cnt;
             }
-            __syncwarp();
           }
-          if (c < p.nT && my_row < M) {
+          if (tile_ok) {
+            const int n = min(cnt, p.W);
+            if (n & 7) {
+              // Last partial group of 8: pad with (-1, 0) and store it whole.
+              for (int k = n & 7; k < 8; ++k) {
+                stg_idx[k] = 0xFFFFu;
+                stg_val[k] = 0;
+              }
+              const size_t off = slot0 + (n & ~7);
+              *reinterpret_cast<uint4*>(p.idx + off) = *reinterpret_cast<const uint4*>(stg_idx);
+              *reinterpret_cast<uint4*>(p.vals + off) = *reinterpret_cast<const uint4*>(stg_val);
+            }
             p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
             if (cnt > p.W) p.row_ovf[my_row] = 1;
           }
@@ -313,6 +332,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t zr[32], ur[32];
+          __syncwarp();
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), zr);
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + ch * 32), ur);
           tmem_wait_ld();
@@ -354,6 +374,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
         for (int ch = 0; ch < kBN / 32; ++ch) {
           uint32_t r[32];
+          __syncwarp();
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), r);
           tmem_wait_ld();
           if (ch == kBN / 32 - 1) {
