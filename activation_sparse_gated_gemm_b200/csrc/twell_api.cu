@@ -420,3 +420,59 @@ const char* twell_status_str(int status) {
 const char* twell_version(void) { return "twell-b200 0.1"; }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation variant
+//
+// Some callers cannot hand the library a workspace: code that runs where
+// device allocation is not allowed or not wanted (inside a framework that owns
+// every byte of device memory through its own pool, a real-time loop that must
+// not call the allocator, or a plugin whose host gives it only its inputs and
+// outputs). For them the hybrid forward can run on a scratch area that lives in
+// the library itself: a fixed array in device memory, created when the module
+// is loaded on a device and held until the process exits.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // == TWELL_NOALLOC_SCRATCH_BYTES
+
+// Device-side scratch shared by every call of twell_ffn_hybrid_forward_noalloc
+// on a device. In host code this name is only a handle: its device address is
+// obtained once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices];
+std::once_flag g_noalloc_once[kMaxDevices];
+cudaError_t g_noalloc_err[kMaxDevices];
+
+// Device address of the scratch for the current device `dev`, looked up on the
+// first call made with that device current.
+void* noalloc_scratch(int dev) {
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = (g_noalloc_err[dev] == cudaSuccess) ? p : nullptr;
+  });
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" twell_status twell_ffn_hybrid_forward_noalloc(const uint16_t* x, const uint16_t* WgT,
+                                                         const uint16_t* WuT, const uint16_t* Wd, int T, int d,
+                                                         int f, const twell_t* tw, float* y, int32_t* ovf_rows,
+                                                         int32_t* n_ovf, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, y, ovf_rows, n_ovf, dev_status}));
+  const size_t need = twell_hybrid_workspace_bytes(T, d, f);
+  if (need > kNoAllocScratchBytes) return TWELL_ERR_WORKSPACE;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  void* ws = noalloc_scratch(dev);
+  if (ws == nullptr) {
+    (void)cudaGetLastError();
+    return TWELL_ERR_CUDA;
+  }
+  return twell_ffn_hybrid_forward(x, WgT, WuT, Wd, T, d, f, tw, y, ovf_rows, n_ovf, ws, need, dev_status, stream);
+}

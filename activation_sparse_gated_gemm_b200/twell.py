@@ -28,8 +28,9 @@ EXPORTED = (
     "twell_gate_pack", "twell_sparse_ffn", "twell_ffn_forward", "twell_route",
     "twell_hybrid_workspace_bytes", "twell_dense_rows_forward", "twell_ffn_hybrid_forward", "twell_dense_workspace_bytes",
     "twell_dense_ffn_forward", "twell_unpack", "twell_status_reset", "twell_status_get",
-    "twell_status_str", "twell_version",
+    "twell_status_str", "twell_version", "twell_ffn_hybrid_forward_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class TwellError(RuntimeError):
@@ -76,6 +77,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_dense_workspace_bytes": ([i32, i32, i32], sz),
         "twell_dense_ffn_forward": ([vp, vp, vp, vp, i32, i32, i32, vp, vp, sz, vp, vp], i32),
         "twell_unpack": ([tw, vp, vp, vp], i32),
+        "twell_ffn_hybrid_forward_noalloc": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp], i32),
         "twell_status_reset": ([vp, vp], i32),
         "twell_status_get": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "twell_status_str": ([i32], ctypes.c_char_p),
@@ -204,6 +206,20 @@ def ffn_hybrid_forward(x, WgT, WuT, Wd, tw: Twell, y, ovf_rows, n_ovf, workspace
     _check("twell_ffn_hybrid_forward", load().twell_ffn_hybrid_forward(
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f, tw.ref(), _ptr(y), _ptr(ovf_rows), _ptr(n_ovf),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def ffn_hybrid_forward_noalloc(x, WgT, WuT, Wd, tw: Twell, y, ovf_rows, n_ovf, dev_status,
+                               stream=None) -> None:
+    """Hybrid forward on the library's built-in device scratch, for callers
+    that cannot allocate a workspace (see twell_ffn_hybrid_forward_noalloc)."""
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_ffn_hybrid_forward_noalloc", load().twell_ffn_hybrid_forward_noalloc(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f, tw.ref(), _ptr(y), _ptr(ovf_rows), _ptr(n_ovf),
+        _ptr(dev_status), _stream(stream)))
 
 
 def dense_rows_forward(x, WgT, WuT, Wd, rows, n_rows, y, workspace, dev_status, stream=None) -> None:

@@ -159,6 +159,35 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
                                       void* workspace, size_t workspace_bytes,
                                       int32_t* dev_status, void* stream);
 
+/*
+ * Hybrid forward without a caller-provided workspace (the paper has no
+ * counterpart; this is a convenience of this library).
+ *
+ * For callers that cannot allocate device memory for a workspace -- code that
+ * runs inside a framework that owns all device memory through its own pool,
+ * a loop that must never reach the allocator, or a plugin whose host passes it
+ * only inputs and outputs. Same arguments and results as
+ * twell_ffn_hybrid_forward minus the workspace: the gathered overflow rows and
+ * their hidden activations go to a scratch array compiled into the library
+ * (TWELL_NOALLOC_SCRATCH_BYTES of device memory, held on every device that
+ * loads the library until the process exits). The call itself allocates
+ * nothing.
+ *   - Size limit: twell_hybrid_workspace_bytes(T, d, f) must not exceed
+ *     TWELL_NOALLOC_SCRATCH_BYTES, i.e. roughly T * (2d + 4f) bytes; larger
+ *     calls return TWELL_ERR_WORKSPACE and launch nothing.
+ *   - The first call on a device looks up the scratch address for that device
+ *     (with it current); make that first call before any stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the last
+ *     call's contents (nothing in it needs to start at zero). Calls whose work
+ *     overlaps on the GPU -- on different streams, or from several host
+ *     threads -- race on it; serialise them.
+ */
+#define TWELL_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+twell_status twell_ffn_hybrid_forward_noalloc(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                              const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                                              float* y, int32_t* ovf_rows, int32_t* n_ovf,
+                                              int32_t* dev_status, void* stream);
+
 /* Bytes of workspace needed by twell_dense_ffn_forward (the [T][f] bf16 hidden
  * activations). */
 size_t twell_dense_workspace_bytes(int T, int d, int f);
