@@ -8,8 +8,7 @@
 // several FFN steps in one pass, intermediates not written to global memory).
 //
 // Lane l owns the 8-element chunks l, l+32, l+64, ... of the d axis, so every
-// gather of a weight row is a run of fully coalesced 16-byte loads. x_t and
-// y_t live in registers for the whole row.
+// gather of a weight row is a run of fully coalesced 16-byte loads.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,14 +29,23 @@ struct SparseParams {
   int* dev_status;
 };
 
-constexpr int kSparseWarps = 8;
+// Warps per block of the sparse kernel: 12 while a token's x and y chunks fit
+// the register budget of 12 warps per SM (d <= 1536), 8 above.
+constexpr int sparse_warps_for(int nch) { return nch <= 6 ? 12 : 8; }
 
+// Read-only 16-byte load through the non-coherent path. Left as an ordinary
+// (non-volatile) operation so the compiler may issue it as early as its
+// address is known.
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+#ifdef TWELL_LDG_VOLATILE
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
+#else
+  return __ldg(reinterpret_cast<const uint4*>(p));
+#endif
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -55,100 +63,221 @@ __device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc)
   return acc;
 }
 
+// y[2k], y[2k+1] += h * (w_lo, w_hi) with one packed fp32x2 fma per pair.
+__device__ __forceinline__ void ffma2(float& y0, float& y1, float h, uint32_t w) {
+  asm("{\n\t.reg .b64 yy, hh, ww;\n\t"
+      "mov.b64 yy, {%0, %1};\n\t"
+      "mov.b64 hh, {%2, %2};\n\t"
+      "mov.b64 ww, {%3, %4};\n\t"
+      "fma.rn.f32x2 yy, hh, ww, yy;\n\t"
+      "mov.b64 {%0, %1}, yy;\n\t}"
+      : "+f"(y0), "+f"(y1)
+      : "f"(h), "f"(__uint_as_float(w << 16)), "f"(__uint_as_float(w & 0xffff0000u)));
+}
 __device__ __forceinline__ void axpy8(float (&y)[8], float h, const uint4& w) {
-  y[0] = fmaf(h, bf16lo(w.x), y[0]);
-  y[1] = fmaf(h, bf16hi(w.x), y[1]);
-  y[2] = fmaf(h, bf16lo(w.y), y[2]);
-  y[3] = fmaf(h, bf16hi(w.y), y[3]);
-  y[4] = fmaf(h, bf16lo(w.z), y[4]);
-  y[5] = fmaf(h, bf16hi(w.z), y[5]);
-  y[6] = fmaf(h, bf16lo(w.w), y[6]);
-  y[7] = fmaf(h, bf16hi(w.w), y[7]);
+  ffma2(y[0], y[1], h, w.x);
+  ffma2(y[2], y[3], h, w.y);
+  ffma2(y[4], y[5], h, w.z);
+  ffma2(y[6], y[7], h, w.w);
+}
+
+// acc += sum over 8 bf16 pairs of a_i * b_i, each product exact and added with
+// one rounding (mixed-precision fma with bf16 sources and an fp32 addend).
+__device__ __forceinline__ void mixdot8(const uint4& a, const uint4& b, float& acc0, float& acc1) {
+  asm("{\n\t.reg .b16 a0, a1, a2, a3, a4, a5, a6, a7, b0, b1, b2, b3, b4, b5, b6, b7;\n\t"
+      "mov.b32 {a0, a1}, %2; mov.b32 {a2, a3}, %3; mov.b32 {a4, a5}, %4; mov.b32 {a6, a7}, %5;\n\t"
+      "mov.b32 {b0, b1}, %6; mov.b32 {b2, b3}, %7; mov.b32 {b4, b5}, %8; mov.b32 {b6, b7}, %9;\n\t"
+      "fma.rn.f32.bf16 %0, a0, b0, %0; fma.rn.f32.bf16 %1, a1, b1, %1;\n\t"
+      "fma.rn.f32.bf16 %0, a2, b2, %0; fma.rn.f32.bf16 %1, a3, b3, %1;\n\t"
+      "fma.rn.f32.bf16 %0, a4, b4, %0; fma.rn.f32.bf16 %1, a5, b5, %1;\n\t"
+      "fma.rn.f32.bf16 %0, a6, b6, %0; fma.rn.f32.bf16 %1, a7, b7, %1;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
 }
 
 template <int NCH>
-__global__ void __launch_bounds__(kSparseWarps * 32) sparse_ffn_warp_kernel(const SparseParams p) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kSparseWarps + (threadIdx.x >> 5);
-  if (t >= p.T) return;
-  if (p.skip_ovf && p.row_ovf[t]) return;
-  const int d = p.d;
-
-  uint4 xr[NCH];
+__device__ __forceinline__ void load_row(uint4 (&w)[NCH], const uint16_t* row, int lane, int d) {
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int k0 = (i * 32 + lane) * 8;
-    xr[i] = (k0 < d) ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
+    w[i] = (k0 < d) ? ldg_nc_v4(row + k0) : make_uint4(0, 0, 0, 0);
   }
-  float y[NCH][8];
-#pragma unroll
-  for (int i = 0; i < NCH; ++i)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[i][e] = 0.0f;
+}
 
+// Stored slots of one token, flattened: entry = column index | bf16 value << 16.
+constexpr int kListCap = 1024;  // entries per warp; a group of kListCap / W tiles always fits
+
+__device__ __forceinline__ float entry_g(uint32_t e) { return __uint_as_float(e & 0xffff0000u); }
+__device__ __forceinline__ int entry_j(uint32_t e) { return static_cast<int>(e & 0xffffu); }
+
+// Persistent blocks, one per SM, each walking a contiguous range of tokens
+// with its warps drawing tokens from a shared counter. Per token, x_t is parked in shared memory and y_t (fp32) stays in
+// registers. The token's stored slots are first copied, tile group by tile
+// group, into a flat list in shared memory (counts of 32 tiles per load, a warp
+// prefix sum for the offsets, 16-byte slot loads), so no dependent load chain
+// is paid per tile. The list is then consumed in batches of 32 entries in two
+// passes: every u_j = x_t . Wu[:, j] (lane s keeps h_s = g_s * u_s), then every
+// y_t += h_s * Wd[j_s, :]. In both passes two weight rows alternate, so the
+// gather of entry s+1 is in flight while entry s is computed.
+template <int NCH, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const SparseParams p) {
+  extern __shared__ uint4 smem_dyn[];  // xs: [WARPS][NCH * 32] uint4, then lists
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int d = p.d;
+  uint4* xs = smem_dyn + warp * NCH * 32;
+  uint32_t* list = reinterpret_cast<uint32_t*>(smem_dyn + WARPS * NCH * 32) + warp * kListCap;
+  const int group_tiles = max(1, kListCap / p.W);
   bool overflow = false, bad_index = false;
-  const int16_t* cnt_row = p.counts + static_cast<size_t>(t) * p.nT;
+  // Block b owns the contiguous tokens [t_begin, t_end); its warps take them
+  // one at a time from a shared counter, so a warp that drew light tokens
+  // keeps working while another finishes a heavy one.
+  __shared__ int next_token;
+  const int t_begin = static_cast<int>(static_cast<long long>(p.T) * blockIdx.x / gridDim.x);
+  const int t_end = static_cast<int>(static_cast<long long>(p.T) * (blockIdx.x + 1) / gridDim.x);
+  if (threadIdx.x == 0) next_token = t_begin;
+  __syncthreads();
 #pragma unroll 1
-  for (int c = 0; c < p.nT; ++c) {
-    const int cnt = cnt_row[c];
-    if (cnt > p.W) overflow = true;
-    const int n = min(max(cnt, 0), p.W);
-    const size_t slot0 = (static_cast<size_t>(t) * p.nT + c) * p.W;
-#pragma unroll 1
-    for (int s0 = 0; s0 < n; s0 += 32) {
-      int my_j = 0;
-      float my_g = 0.0f;
-      if (s0 + lane < n) {
-        my_j = p.idx[slot0 + s0 + lane];
-        my_g = __uint_as_float(static_cast<uint32_t>(p.vals[slot0 + s0 + lane]) << 16);
-      }
-      const int ns = min(32, n - s0);
-#pragma unroll 1
-      for (int s = 0; s < ns; ++s) {
-        const int j = __shfl_sync(0xffffffffu, my_j, s);
-        const float g = __shfl_sync(0xffffffffu, my_g, s);
-        if (static_cast<unsigned>(j) >= static_cast<unsigned>(p.f)) {
-          bad_index = true;
-          continue;
-        }
-        const uint16_t* wu = p.WuT + static_cast<size_t>(j) * d;
-        const uint16_t* wd = p.Wd + static_cast<size_t>(j) * d;
-        uint4 a[NCH], b[NCH];
+  for (;;) {
+    int t = 0;
+    if (lane == 0) t = atomicAdd(&next_token, 1);
+    t = __shfl_sync(0xffffffffu, t, 0);
+    if (t >= t_end) break;
+    if (p.skip_ovf && p.row_ovf[t]) continue;
+    __syncwarp();
 #pragma unroll
-        for (int i = 0; i < NCH; ++i) {
-          const int k0 = (i * 32 + lane) * 8;
-          if (k0 < d) {
-            a[i] = ldg_nc_v4(wu + k0);
-            b[i] = ldg_nc_v4(wd + k0);
-          } else {
-            a[i] = make_uint4(0, 0, 0, 0);
-            b[i] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < NCH; ++i) {
+      const int k0 = (i * 32 + lane) * 8;
+      xs[i * 32 + lane] = (k0 < d) ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
+    }
+    float y[NCH][8];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[i][e] = 0.0f;
+
+#pragma unroll 1
+    for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
+      const int c1 = min(p.nT, c0 + group_tiles);
+      // ---- flatten the slots of tiles [c0, c1) into list[0, total)
+      int total = 0;
+#pragma unroll 1
+      for (int cb = c0; cb < c1; cb += 32) {
+        const int c = cb + lane;
+        int n = 0;
+        if (c < c1) {
+          const int cnt = p.counts[static_cast<size_t>(t) * p.nT + c];
+          if (cnt > p.W) overflow = true;
+          n = min(max(cnt, 0), p.W);
+        }
+        int incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int off = total + incl - n;
+        total += __shfl_sync(0xffffffffu, incl, 31);
+        const size_t base = (static_cast<size_t>(t) * p.nT + c) * p.W;
+        for (int k = 0; k < n; k += 8) {
+          // 8 slots at a time; slots past n are read but not used (k + 8 <= W)
+          const uint4 iv = ldg_nc_v4(p.idx + base + k);
+          const uint4 vv = ldg_nc_v4(p.vals + base + k);
+          const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
+          const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (k + e < n) {
+              const uint32_t jj = (e & 1) ? (iw[e >> 1] >> 16) : (iw[e >> 1] & 0xffffu);
+              const uint32_t gg = (e & 1) ? (vw[e >> 1] & 0xffff0000u) : (vw[e >> 1] << 16);
+              uint32_t ent = jj | gg;
+              if (static_cast<int>(static_cast<int16_t>(jj)) < 0 || static_cast<int>(jj) >= p.f) {
+                bad_index = true;
+                ent = 0;  // column 0 with value 0: contributes nothing
+              }
+              list[off + k + e] = ent;
+            }
           }
         }
-        float acc = 0.0f;
+      }
+      __syncwarp();
+      // ---- consume the list
+#pragma unroll 1
+      for (int s0 = 0; s0 < total; s0 += 32) {
+        const int ns = min(32, total - s0);
+        const uint32_t my_e = (lane < ns) ? list[s0 + lane] : 0u;
+        const int my_j = entry_j(my_e);
+        const float my_g = entry_g(my_e);
+        // pass 1: up projections
+        float my_h = 0.0f;
+        uint4 wa[NCH], wb[NCH];
+        load_row<NCH>(wa, p.WuT + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
+#pragma unroll 1
+        for (int s = 0; s < ns; s += 2) {
+          if (s + 1 < ns)
+            load_row<NCH>(wb, p.WuT + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 1)) * d, lane, d);
+          {
+            float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
-        for (int i = 0; i < NCH; ++i) acc = dot8(xr[i], a[i], acc);
+            for (int i = 0; i < NCH; i += 2) {
+              mixdot8(xs[i * 32 + lane], wa[i], a0, a1);
+              if (i + 1 < NCH) mixdot8(xs[(i + 1) * 32 + lane], wa[i + 1], a2, a3);
+            }
+            float acc = (a0 + a1) + (a2 + a3);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        const float h = g * acc;
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == s) my_h = my_g * acc;
+          }
+          if (s + 1 < ns) {
+            if (s + 2 < ns)
+              load_row<NCH>(wa, p.WuT + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 2)) * d, lane, d);
+            float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
-        for (int i = 0; i < NCH; ++i) axpy8(y[i], h, b[i]);
+            for (int i = 0; i < NCH; i += 2) {
+              mixdot8(xs[i * 32 + lane], wb[i], a0, a1);
+              if (i + 1 < NCH) mixdot8(xs[(i + 1) * 32 + lane], wb[i + 1], a2, a3);
+            }
+            float acc = (a0 + a1) + (a2 + a3);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == s + 1) my_h = my_g * acc;
+          }
+        }
+        // pass 2: down projection, h never leaves the registers
+        load_row<NCH>(wa, p.Wd + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
+#pragma unroll 1
+        for (int s = 0; s < ns; s += 2) {
+          if (s + 1 < ns)
+            load_row<NCH>(wb, p.Wd + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 1)) * d, lane, d);
+          {
+            const float h = __shfl_sync(0xffffffffu, my_h, s);
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) axpy8(y[i], h, wa[i]);
+          }
+          if (s + 1 < ns) {
+            if (s + 2 < ns)
+              load_row<NCH>(wa, p.Wd + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 2)) * d, lane, d);
+            const float h = __shfl_sync(0xffffffffu, my_h, s + 1);
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) axpy8(y[i], h, wb[i]);
+          }
+        }
+      }
+      __syncwarp();
+    }
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int k0 = (i * 32 + lane) * 8;
+      if (k0 < d) {
+        float4* dst = reinterpret_cast<float4*>(p.y + static_cast<size_t>(t) * d + k0);
+        dst[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+        dst[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
       }
     }
   }
-  if (lane == 0) {
-    if (overflow && !p.skip_ovf) raise_status(p.dev_status, kDevOverflow);
-    if (bad_index) raise_status(p.dev_status, kDevIndex);
-  }
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    const int k0 = (i * 32 + lane) * 8;
-    if (k0 < d) {
-      float4* dst = reinterpret_cast<float4*>(p.y + static_cast<size_t>(t) * d + k0);
-      dst[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
-      dst[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
-    }
-  }
+  // each lane saw the counts of its own tiles
+  if (__any_sync(0xffffffffu, overflow) && lane == 0 && !p.skip_ovf) raise_status(p.dev_status, kDevOverflow);
+  if (__any_sync(0xffffffffu, bad_index) && lane == 0) raise_status(p.dev_status, kDevIndex);
 }
 
 // ---------------------------------------------------------------- routing

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -159,14 +160,20 @@ twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d
 }
 
 template <int NCH>
-twell_status launch_sparse_n(const SparseParams& p, cudaStream_t s) {
-  const int blocks = (p.T + kSparseWarps - 1) / kSparseWarps;
-  sparse_ffn_warp_kernel<NCH><<<blocks, kSparseWarps * 32, 0, s>>>(p);
+twell_status launch_sparse_n(const SparseParams& p, int sms, cudaStream_t s) {
+  constexpr int kWarps = sparse_warps_for(NCH);
+  // persistent warps: one resident block per SM
+  const int blocks = std::min((p.T + kWarps - 1) / kWarps, sms);
+  const size_t smem = static_cast<size_t>(kWarps) * (NCH * 32 * sizeof(uint4) + kListCap * sizeof(uint32_t));
+  auto kern = sparse_ffn_warp_kernel<NCH, kWarps>;
+  if (smem > 48 * 1024)
+    TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
+  kern<<<blocks, kWarps * 32, smem, s>>>(p);
   return cuda_ok(cudaGetLastError());
 }
 
 twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
-                         const twell_t* tw, int skip, float* y, int32_t* dev_status, cudaStream_t s) {
+                         const twell_t* tw, int skip, float* y, int32_t* dev_status, cudaStream_t s, int sms) {
   SparseParams p{};
   p.x = x;
   p.WuT = WuT;
@@ -184,22 +191,22 @@ twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t*
   p.skip_ovf = skip ? 1 : 0;
   p.dev_status = dev_status;
   switch ((d + 255) / 256) {
-    case 1: return launch_sparse_n<1>(p, s);
-    case 2: return launch_sparse_n<2>(p, s);
-    case 3: return launch_sparse_n<3>(p, s);
-    case 4: return launch_sparse_n<4>(p, s);
-    case 5: return launch_sparse_n<5>(p, s);
-    case 6: return launch_sparse_n<6>(p, s);
-    case 7: return launch_sparse_n<7>(p, s);
-    case 8: return launch_sparse_n<8>(p, s);
-    case 9: return launch_sparse_n<9>(p, s);
-    case 10: return launch_sparse_n<10>(p, s);
-    case 11: return launch_sparse_n<11>(p, s);
-    case 12: return launch_sparse_n<12>(p, s);
-    case 13: return launch_sparse_n<13>(p, s);
-    case 14: return launch_sparse_n<14>(p, s);
-    case 15: return launch_sparse_n<15>(p, s);
-    case 16: return launch_sparse_n<16>(p, s);
+    case 1: return launch_sparse_n<1>(p, sms, s);
+    case 2: return launch_sparse_n<2>(p, sms, s);
+    case 3: return launch_sparse_n<3>(p, sms, s);
+    case 4: return launch_sparse_n<4>(p, sms, s);
+    case 5: return launch_sparse_n<5>(p, sms, s);
+    case 6: return launch_sparse_n<6>(p, sms, s);
+    case 7: return launch_sparse_n<7>(p, sms, s);
+    case 8: return launch_sparse_n<8>(p, sms, s);
+    case 9: return launch_sparse_n<9>(p, sms, s);
+    case 10: return launch_sparse_n<10>(p, sms, s);
+    case 11: return launch_sparse_n<11>(p, sms, s);
+    case 12: return launch_sparse_n<12>(p, sms, s);
+    case 13: return launch_sparse_n<13>(p, sms, s);
+    case 14: return launch_sparse_n<14>(p, sms, s);
+    case 15: return launch_sparse_n<15>(p, sms, s);
+    case 16: return launch_sparse_n<16>(p, sms, s);
     default: return TWELL_ERR_SHAPE;
   }
 }
@@ -279,7 +286,7 @@ twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint
   TW_TRY(check_ptrs({x, WuT, Wd, y, dev_status}));
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  return sparse_impl(x, WuT, Wd, T, d, f, tw, skip_overflow_rows, y, dev_status, static_cast<cudaStream_t>(stream));
+  return sparse_impl(x, WuT, Wd, T, d, f, tw, skip_overflow_rows, y, dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 
 twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
@@ -293,7 +300,7 @@ twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uin
   TW_TRY(current_device(&dev, &sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
-  return sparse_impl(x, WuT, Wd, T, d, f, tw, 0, y, dev_status, s);
+  return sparse_impl(x, WuT, Wd, T, d, f, tw, 0, y, dev_status, s, sms);
 }
 
 twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream) {
@@ -330,7 +337,7 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
   TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
   route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s));
+  TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
 }
 
