@@ -36,32 +36,10 @@ constexpr int sparse_warps_for(int nch) { return nch <= 6 ? 12 : 8; }
 // Read-only 16-byte load through the non-coherent path. Left as an ordinary
 // (non-volatile) operation so the compiler may issue it as early as its
 // address is known.
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-#ifdef TWELL_LDG_VOLATILE
-  uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-#else
-  return __ldg(reinterpret_cast<const uint4*>(p));
-#endif
-}
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc) {
-  acc = fmaf(bf16lo(a.x), bf16lo(b.x), acc);
-  acc = fmaf(bf16hi(a.x), bf16hi(b.x), acc);
-  acc = fmaf(bf16lo(a.y), bf16lo(b.y), acc);
-  acc = fmaf(bf16hi(a.y), bf16hi(b.y), acc);
-  acc = fmaf(bf16lo(a.z), bf16lo(b.z), acc);
-  acc = fmaf(bf16hi(a.z), bf16hi(b.z), acc);
-  acc = fmaf(bf16lo(a.w), bf16lo(b.w), acc);
-  acc = fmaf(bf16hi(a.w), bf16hi(b.w), acc);
-  return acc;
-}
 
 // y[2k], y[2k+1] += h * (w_lo, w_hi) with one packed fp32x2 fma per pair.
 __device__ __forceinline__ void ffma2(float& y0, float& y1, float h, uint32_t w) {
