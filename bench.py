@@ -190,7 +190,7 @@ def blas_threads() -> int:
 # ---------------------------------------------------------------- CPU oracle
 
 
-def cpu_oracle_rate(cfg, L, sample_rows: int, max_seconds: float = 20.0) -> dict:
+def cpu_oracle_rate(cfg, L, sample_rows: int, max_seconds: float = 25.0) -> dict:
     """The oracle as it stands (hybrid forward: fp64 gate, pack, route,
     per-token sparse step, dense rows) on the first rows of the workload."""
     from oracle import twell_oracle as O
@@ -416,7 +416,7 @@ def run_reference(args, world, rank):
         return None
     cfg = synth.CONFIGS[args.config]
     L = synth.make_layer(cfg, seed=args.seed)
-    sample = max(1, min(cfg.T, args.cpu_sample // 4))
+    sample = max(1, min(cfg.T, args.cpu_sample // 16))
     from oracle import twell_oracle as O
 
     def step():
@@ -443,6 +443,70 @@ def run_reference(args, world, rank):
     }
 
 
+def run_sweep(args) -> None:
+    """Density x batch sweep (d=2048, f=8192): one JSON line per point with the
+    hybrid forward's time, the dense FFN's time and the path roofline."""
+    import torch
+
+    from activation_sparse_gated_gemm_b200 import twell as tl
+
+    tl.load()
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    Ts = [int(v) for v in args.sweep_T.split(",")] if args.sweep_T else list(synth.SWEEP_T)
+    Ps = [float(v) for v in args.sweep_p.split(",")] if args.sweep_p else list(synth.SWEEP_P)
+    for T in Ts:
+        for pden in Ps:
+            cfg = synth.sweep_config(T, pden)
+            L = synth.make_layer(cfg, seed=args.seed)
+            x, WgT, WuT, Wd = (tl.to_device_bf16(L[k], dev) for k in ("x", "WgT", "WuT", "Wd"))
+            tw = tl.Twell(T, cfg.f, cfg.W, device=dev)
+            y = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
+            ovf_rows = torch.empty((T,), dtype=torch.int32, device=dev)
+            n_ovf = torch.zeros((1,), dtype=torch.int32, device=dev)
+            ws = torch.empty(tl.hybrid_workspace_bytes(T, cfg.d, cfg.f), dtype=torch.uint8, device=dev)
+            wsd = torch.empty(tl.dense_workspace_bytes(T, cfg.d, cfg.f), dtype=torch.uint8, device=dev)
+            st = tl.new_status(dev)
+
+            def timed(fn, k):
+                ts = []
+                for _ in range(args.warmup):
+                    flush.zero_()
+                    fn()
+                for _ in range(k):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    fn()
+                    b.record()
+                    torch.cuda.synchronize(dev)
+                    ts.append(a.elapsed_time(b))
+                return float(np.median(ts))
+
+            ms = timed(lambda: tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st), args.steps)
+            ms_dense = timed(lambda: tl.dense_ffn_forward(x, WgT, WuT, Wd, y, wsd, st), args.steps)
+            status = tl.status_get(st)
+            counts = tw.counts.to(torch.int64)
+            n_o = int(n_ovf.item())
+            nnz = int(torch.clamp(counts, max=cfg.W)[~tw.row_ovf.bool()].sum())
+            g = torch.empty((T, cfg.f), dtype=torch.bfloat16, device=dev)
+            tl.unpack(tw, g, st)
+            union = int((g[~tw.row_ovf.bool()] != 0).any(dim=0).sum())
+            del g
+            alg = algorithmic(cfg, n_o, nnz, union)
+            t_roof = max((alg["gate_flops"] + alg["dense_branch_flops"]) / (peaks["bf16_tflops"] * 1e12),
+                         alg["alg_bytes"] / (peaks["hbm_gbs"] * 1e9))
+            print(json.dumps({"sweep": True, "T": T, "density": pden, "W": cfg.W, "d": cfg.d, "f": cfg.f,
+                              "ms": ms, "tokens_per_s": T / (ms * 1e-3), "dense_ms": ms_dense,
+                              "speedup_vs_own_dense": ms_dense / ms, "roofline_frac": t_roof / (ms * 1e-3),
+                              "t_roof_us": t_roof * 1e6, "n_ovf": n_o,
+                              "measured_density": float(counts.sum()) / (T * cfg.f), "status": status}),
+                  flush=True)
+            del x, WgT, WuT, Wd, tw, y, ws, wsd
+            torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -451,11 +515,17 @@ def main(argv=None):
     ap.add_argument("--impl", default="twell", choices=["twell", "reference"])
     ap.add_argument("--config", default="0.5b", choices=sorted(synth.CONFIGS))
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-sample", type=int, default=1024)
+    ap.add_argument("--cpu-sample", type=int, default=12288)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="density x batch sweep, one JSON line per point")
+    ap.add_argument("--sweep-T", default="", help="comma-separated token counts (default: the full sweep)")
+    ap.add_argument("--sweep-p", default="", help="comma-separated densities (default: the full sweep)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.sweep:
+        run_sweep(args)
+        return 0
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
