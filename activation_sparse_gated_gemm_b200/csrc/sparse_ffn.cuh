@@ -97,7 +97,11 @@ __device__ __forceinline__ int entry_j(uint32_t e) { return static_cast<int>(e &
 // passes: every u_j = x_t . Wu[:, j] (lane s keeps h_s = g_s * u_s), then every
 // y_t += h_s * Wd[j_s, :]. In both passes two weight rows alternate, so the
 // gather of entry s+1 is in flight while entry s is computed.
-template <int NCH, int WARPS>
+//
+// DOWN_ONLY: the stored values already are the hidden activations h (the up
+// projection ran on the tensor cores); only the second pass runs and x is not
+// read.
+template <int NCH, int WARPS, bool DOWN_ONLY>
 __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const SparseParams p) {
   extern __shared__ uint4 smem_dyn[];  // xs: [WARPS][NCH * 32] uint4, then lists
   const int lane = threadIdx.x & 31;
@@ -123,10 +127,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
     if (t >= t_end) break;
     if (p.skip_ovf && p.row_ovf[t]) continue;
     __syncwarp();
+    if (!DOWN_ONLY) {
 #pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int k0 = (i * 32 + lane) * 8;
-      xs[i * 32 + lane] = (k0 < d) ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < NCH; ++i) {
+        const int k0 = (i * 32 + lane) * 8;
+        xs[i * 32 + lane] = (k0 < d) ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
+      }
     }
     float y[NCH][8];
 #pragma unroll
@@ -187,11 +193,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
         const int my_j = entry_j(my_e);
         const float my_g = entry_g(my_e);
         // pass 1: up projections
-        float my_h = 0.0f;
+        float my_h = DOWN_ONLY ? my_g : 0.0f;
         uint4 wa[NCH], wb[NCH];
-        load_row<NCH>(wa, p.WuT + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
+        if (!DOWN_ONLY)
+          load_row<NCH>(wa, p.WuT + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
 #pragma unroll 1
-        for (int s = 0; s < ns; s += 2) {
+        for (int s = 0; s < (DOWN_ONLY ? 0 : ns); s += 2) {
           if (s + 1 < ns)
             load_row<NCH>(wb, p.WuT + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 1)) * d, lane, d);
           {

@@ -159,21 +159,66 @@ twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d
   return launch_gemm<kModeTwell>(ma, mb, mb, p, gemm_grid(T, f, kBN, sms), s);
 }
 
-template <int NCH>
+// Gate and up GEMM in one pass; TwELL of the gate pattern holding h = z * u.
+twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, int T, int d, int f,
+                               const twell_t* tw, int32_t* dev_status, cudaStream_t s, int sms) {
+  TW_TRY(cuda_ok(cudaMemsetAsync(tw->row_ovf, 0, static_cast<size_t>(T), s)));
+  CUtensorMap ma, mg, mu;
+  if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128))
+    return TWELL_ERR_CUDA;
+  GemmParams p{};
+  p.M = T;
+  p.N = f;
+  p.K = d;
+  p.counts = tw->counts;
+  p.idx = tw->idx;
+  p.vals = tw->vals;
+  p.row_ovf = tw->row_ovf;
+  p.nT = f / 128;
+  p.W = tw->W;
+  p.dev_status = dev_status;
+  return launch_gemm<kModeTwellHidden>(ma, mg, mu, p, gemm_grid(T, f, 128, sms), s);
+}
+
+template <int NCH, bool DOWN_ONLY>
 twell_status launch_sparse_n(const SparseParams& p, int sms, cudaStream_t s) {
   constexpr int kWarps = sparse_warps_for(NCH);
   // persistent warps: one resident block per SM
   const int blocks = std::min((p.T + kWarps - 1) / kWarps, sms);
   const size_t smem = static_cast<size_t>(kWarps) * (NCH * 32 * sizeof(uint4) + kListCap * sizeof(uint32_t));
-  auto kern = sparse_ffn_warp_kernel<NCH, kWarps>;
+  auto kern = sparse_ffn_warp_kernel<NCH, kWarps, DOWN_ONLY>;
   if (smem > 48 * 1024)
     TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
   kern<<<blocks, kWarps * 32, smem, s>>>(p);
   return cuda_ok(cudaGetLastError());
 }
 
+template <bool DOWN_ONLY>
+twell_status sparse_launch(const SparseParams& p, int d, int sms, cudaStream_t s) {
+  switch ((d + 255) / 256) {
+    case 1: return launch_sparse_n<1, DOWN_ONLY>(p, sms, s);
+    case 2: return launch_sparse_n<2, DOWN_ONLY>(p, sms, s);
+    case 3: return launch_sparse_n<3, DOWN_ONLY>(p, sms, s);
+    case 4: return launch_sparse_n<4, DOWN_ONLY>(p, sms, s);
+    case 5: return launch_sparse_n<5, DOWN_ONLY>(p, sms, s);
+    case 6: return launch_sparse_n<6, DOWN_ONLY>(p, sms, s);
+    case 7: return launch_sparse_n<7, DOWN_ONLY>(p, sms, s);
+    case 8: return launch_sparse_n<8, DOWN_ONLY>(p, sms, s);
+    case 9: return launch_sparse_n<9, DOWN_ONLY>(p, sms, s);
+    case 10: return launch_sparse_n<10, DOWN_ONLY>(p, sms, s);
+    case 11: return launch_sparse_n<11, DOWN_ONLY>(p, sms, s);
+    case 12: return launch_sparse_n<12, DOWN_ONLY>(p, sms, s);
+    case 13: return launch_sparse_n<13, DOWN_ONLY>(p, sms, s);
+    case 14: return launch_sparse_n<14, DOWN_ONLY>(p, sms, s);
+    case 15: return launch_sparse_n<15, DOWN_ONLY>(p, sms, s);
+    case 16: return launch_sparse_n<16, DOWN_ONLY>(p, sms, s);
+    default: return TWELL_ERR_SHAPE;
+  }
+}
+
 twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
-                         const twell_t* tw, int skip, float* y, int32_t* dev_status, cudaStream_t s, int sms) {
+                         const twell_t* tw, int skip, float* y, int32_t* dev_status, cudaStream_t s, int sms,
+                         bool down_only = false) {
   SparseParams p{};
   p.x = x;
   p.WuT = WuT;
@@ -190,25 +235,7 @@ twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t*
   p.W = tw->W;
   p.skip_ovf = skip ? 1 : 0;
   p.dev_status = dev_status;
-  switch ((d + 255) / 256) {
-    case 1: return launch_sparse_n<1>(p, sms, s);
-    case 2: return launch_sparse_n<2>(p, sms, s);
-    case 3: return launch_sparse_n<3>(p, sms, s);
-    case 4: return launch_sparse_n<4>(p, sms, s);
-    case 5: return launch_sparse_n<5>(p, sms, s);
-    case 6: return launch_sparse_n<6>(p, sms, s);
-    case 7: return launch_sparse_n<7>(p, sms, s);
-    case 8: return launch_sparse_n<8>(p, sms, s);
-    case 9: return launch_sparse_n<9>(p, sms, s);
-    case 10: return launch_sparse_n<10>(p, sms, s);
-    case 11: return launch_sparse_n<11>(p, sms, s);
-    case 12: return launch_sparse_n<12>(p, sms, s);
-    case 13: return launch_sparse_n<13>(p, sms, s);
-    case 14: return launch_sparse_n<14>(p, sms, s);
-    case 15: return launch_sparse_n<15>(p, sms, s);
-    case 16: return launch_sparse_n<16>(p, sms, s);
-    default: return TWELL_ERR_SHAPE;
-  }
+  return down_only ? sparse_launch<true>(p, d, sms, s) : sparse_launch<false>(p, d, sms, s);
 }
 
 // Dense gated FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu)
@@ -301,6 +328,52 @@ twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uin
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
   return sparse_impl(x, WuT, Wd, T, d, f, tw, 0, y, dev_status, s, sms);
+}
+
+twell_status twell_gate_up_pack(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, int T, int d, int f,
+                                const twell_t* tw, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, static_cast<cudaStream_t>(stream), sms);
+}
+
+twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip_overflow_rows,
+                               float* y, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({Wd, y, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, skip_overflow_rows, y, dev_status,
+                     static_cast<cudaStream_t>(stream), sms, true);
+}
+
+twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                            const uint16_t* Wd, int T, int d, int f, const twell_t* tw, float* y,
+                                            int32_t* ovf_rows, int32_t* n_ovf, void* workspace,
+                                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, y, ovf_rows, n_ovf, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_hybrid_workspace_bytes(T, d, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* xo = static_cast<uint16_t*>(workspace);
+  uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                             round_up(static_cast<size_t>(T) * d * 2, 256));
+  TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms));
+  route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  TW_TRY(sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, 1, y, dev_status, s, sms, true));
+  return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
 }
 
 twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream) {

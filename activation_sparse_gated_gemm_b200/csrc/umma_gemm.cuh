@@ -14,6 +14,10 @@
 //                  the same 128 rows of Wu); the epilogue stores
 //                  h = ReLU(z) * u as bf16, and optionally the bf16 remainder
 //                  h - bf16(h) beside it. The dense layer's first half.
+//   kModeTwellHidden -- z and u as in kModeGateUp; the epilogue packs the
+//                  positions where z > 0 into TwELL exactly as kModeTwell does,
+//                  but stores h = z * u there instead of z (the up projection
+//                  then runs on the tensor cores, densely).
 //   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
 //                  epilogue stores fp32 rows, optionally scattered through a
 //                  row map (the dense branch of the hybrid route). With the
@@ -32,7 +36,7 @@
 
 namespace twell {
 
-enum GemmMode : int { kModeTwell = 0, kModeGateUp = 1, kModeDown = 2 };
+enum GemmMode : int { kModeTwell = 0, kModeGateUp = 1, kModeDown = 2, kModeTwellHidden = 3 };
 
 constexpr int kBM = 128;
 constexpr int kBN = 256;
@@ -81,6 +85,42 @@ struct GemmParams {
   int* dev_status;
 };
 
+// Appends the set bits of `mask` (column col0 + i, value vrow[i]) to one row's
+// slot list of a TwELL tile in ascending column order, staging 8 slots at a
+// time in shared memory and storing each full group with 16-byte stores.
+__device__ __forceinline__ void twell_append(uint32_t mask, const float* vrow, int col0, int& cnt, int W,
+                                             uint16_t* stg_idx, uint16_t* stg_val, int16_t* gidx,
+                                             uint16_t* gval) {
+  while (mask != 0) {
+    const int i = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    if (cnt < W) {
+      const int k = cnt & 7;
+      stg_idx[k] = static_cast<uint16_t>(col0 + i);
+      stg_val[k] = f32_to_bf16_bits(vrow[i]);
+      if (k == 7) {
+        *reinterpret_cast<uint4*>(gidx + (cnt - 7)) = *reinterpret_cast<const uint4*>(stg_idx);
+        *reinterpret_cast<uint4*>(gval + (cnt - 7)) = *reinterpret_cast<const uint4*>(stg_val);
+      }
+    }
+    ++cnt;
+  }
+}
+
+// Stores the last partial group of a row's slot list, padded with (-1, 0).
+__device__ __forceinline__ void twell_close(int cnt, int W, uint16_t* stg_idx, uint16_t* stg_val, int16_t* gidx,
+                                            uint16_t* gval) {
+  const int n = min(cnt, W);
+  if (n & 7) {
+    for (int k = n & 7; k < 8; ++k) {
+      stg_idx[k] = 0xFFFFu;
+      stg_val[k] = 0;
+    }
+    *reinterpret_cast<uint4*>(gidx + (n & ~7)) = *reinterpret_cast<const uint4*>(stg_idx);
+    *reinterpret_cast<uint4*>(gval + (n & ~7)) = *reinterpret_cast<const uint4*>(stg_val);
+  }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -101,7 +141,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   int M = p.M;
   if (p.M_dev != nullptr) M = min(max(*p.M_dev, 0), p.M);
-  constexpr int kTileN = (MODE == kModeGateUp) ? 128 : kBN;  // output columns per tile
+  constexpr bool kStacked = (MODE == kModeGateUp || MODE == kModeTwellHidden);  // B = [Wg rows; Wu rows]
+  constexpr int kTileN = kStacked ? 128 : kBN;  // output columns per tile
   const int num_m = (M + kBM - 1) / kBM;
   const int num_n = (p.N + kTileN - 1) / kTileN;
   const int num_tiles = num_m * num_n;
@@ -123,7 +164,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
-    if (MODE == kModeGateUp) tma_prefetch_desc(&tmB1);
+    if (kStacked) tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -152,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(a_dst, &tmA, &full[s], kb * kBK, m_blk * kBM);
           if (MODE == kModeTwell) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * kBN);
-          } else if (MODE == kModeGateUp) {
+          } else if (kStacked) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * 128);
             tma_load_2d(b_dst + kBStageBytes / 2, &tmB1, &full[s], kb * kBK, n_blk * 128);
           } else {
@@ -295,38 +336,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (mask == 0) continue;
 #pragma unroll
             for (int i = 0; i < 32; ++i) vrow[i] = __uint_as_float(r[i]);
-            const int col0 = c * 128 + ch * 32;
-            while (mask != 0) {
-              const int i = __ffs(mask) - 1;
-              mask &= mask - 1u;
-              if (cnt < p.W) {
-                const int k = cnt & 7;
-                stg_idx[k] = static_cast<uint16_t>(col0 + i);
-                stg_val[k] = f32_to_bf16_bits(vrow[i]);
-                if (k == 7) {
-                  const size_t off = slot0 + (cnt - 7);
-                  *reinterpret_cast<uint4*>(p.idx + off) = *reinterpret_cast<const uint4*>(stg_idx);
-                  *reinterpret_cast<uint4*>(p.vals + off) = *reinterpret_cast<const uint4*>(stg_val);
-                }
-              }
-              ++cnt;
-            }
+            twell_append(mask, vrow, c * 128 + ch * 32, cnt, p.W, stg_idx, stg_val, p.idx + slot0,
+                         p.vals + slot0);
           }
           if (tile_ok) {
-            const int n = min(cnt, p.W);
-            if (n & 7) {
-              // Last partial group of 8: pad with (-1, 0) and store it whole.
-              for (int k = n & 7; k < 8; ++k) {
-                stg_idx[k] = 0xFFFFu;
-                stg_val[k] = 0;
-              }
-              const size_t off = slot0 + (n & ~7);
-              *reinterpret_cast<uint4*>(p.idx + off) = *reinterpret_cast<const uint4*>(stg_idx);
-              *reinterpret_cast<uint4*>(p.vals + off) = *reinterpret_cast<const uint4*>(stg_val);
-            }
+            twell_close(cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
             p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
             if (cnt > p.W) p.row_ovf[my_row] = 1;
           }
+        }
+      } else if (MODE == kModeTwellHidden) {
+        // Same pattern as above from z (columns 0..127 of the accumulator),
+        // value h = z * u with u in columns 128..255.
+        float* vrow = ebuf + lane * kEpiPitch;
+        uint8_t* stg = smem + kOffSlots + (threadIdx.x - 64) * kStageSlotBytes;
+        uint16_t* stg_idx = reinterpret_cast<uint16_t*>(stg);
+        uint16_t* stg_val = reinterpret_cast<uint16_t*>(stg + 16);
+        const int c = n_blk;  // the 128 hidden units of this tile are TwELL tile c
+        const bool tile_ok = my_row < M && c < p.nT;
+        const size_t slot0 = (static_cast<size_t>(my_row) * p.nT + c) * p.W;
+        int cnt = 0;
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t zr[32], ur[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), zr);
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + ch * 32), ur);
+          tmem_wait_ld();
+          if (ch == 3) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          if (!tile_ok) continue;
+          uint32_t mask = 0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mask |= (static_cast<int32_t>(zr[i]) > 0 ? 1u : 0u) << i;
+          if (mask == 0) continue;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) vrow[i] = __uint_as_float(zr[i]) * __uint_as_float(ur[i]);
+          twell_append(mask, vrow, c * 128 + ch * 32, cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
+        }
+        if (tile_ok) {
+          twell_close(cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
+          p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
+          if (cnt > p.W) p.row_ovf[my_row] = 1;
         }
       } else if (MODE == kModeGateUp) {
 #pragma unroll 1

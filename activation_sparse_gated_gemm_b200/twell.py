@@ -29,6 +29,7 @@ EXPORTED = (
     "twell_hybrid_workspace_bytes", "twell_dense_rows_forward", "twell_ffn_hybrid_forward", "twell_dense_workspace_bytes",
     "twell_dense_ffn_forward", "twell_unpack", "twell_status_reset", "twell_status_get",
     "twell_status_str", "twell_version", "twell_ffn_hybrid_forward_noalloc",
+    "twell_gate_up_pack", "twell_sparse_down", "twell_ffn_hybrid_forward_tc_up",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -71,6 +72,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_sparse_ffn": ([vp, vp, vp, i32, i32, i32, tw, i32, vp, vp, vp], i32),
         "twell_ffn_forward": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp], i32),
         "twell_route": ([tw, vp, vp, vp], i32),
+        "twell_gate_up_pack": ([vp, vp, vp, i32, i32, i32, tw, vp, vp], i32),
+        "twell_sparse_down": ([vp, i32, i32, i32, tw, i32, vp, vp, vp], i32),
+        "twell_ffn_hybrid_forward_tc_up": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_hybrid_workspace_bytes": ([i32, i32, i32], sz),
         "twell_dense_rows_forward": ([vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_ffn_hybrid_forward": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
@@ -182,6 +186,36 @@ def ffn_forward(x, WgT, WuT, Wd, tw: Twell, y, dev_status, stream=None) -> None:
     _check("twell_ffn_forward", load().twell_ffn_forward(_ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f,
                                                          tw.ref(), _ptr(y), _ptr(dev_status),
                                                          _stream(stream)))
+
+
+def gate_up_pack(x, WgT, WuT, tw: Twell, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d))):
+        _bf16(n, t, s)
+    _check("twell_gate_up_pack", load().twell_gate_up_pack(_ptr(x), _ptr(WgT), _ptr(WuT), T, d, f, tw.ref(),
+                                                           _ptr(dev_status), _stream(stream)))
+
+
+def sparse_down(Wd, tw: Twell, y, skip_overflow_rows: bool, dev_status, stream=None) -> None:
+    f, d = Wd.shape
+    T = tw.T
+    _bf16("Wd", Wd, (f, d))
+    _bf16("y", y, (T, d))
+    _check("twell_sparse_down", load().twell_sparse_down(_ptr(Wd), T, d, f, tw.ref(), int(bool(skip_overflow_rows)),
+                                                         _ptr(y), _ptr(dev_status), _stream(stream)))
+
+
+def ffn_hybrid_forward_tc_up(x, WgT, WuT, Wd, tw: Twell, y, ovf_rows, n_ovf, workspace, dev_status,
+                             stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_ffn_hybrid_forward_tc_up", load().twell_ffn_hybrid_forward_tc_up(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f, tw.ref(), _ptr(y), _ptr(ovf_rows), _ptr(n_ovf),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
 
 
 def route(tw: Twell, ovf_rows, n_ovf, stream=None) -> None:

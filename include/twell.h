@@ -119,6 +119,36 @@ twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uin
                                float* y, int32_t* dev_status, void* stream);
 
 /*
+ * Variant for mid densities, where the dense up projection on the tensor
+ * cores costs less than gathering Wu rows on the CUDA cores (not on the
+ * pages; the pages' kernels target H100). One GEMM forms z = x Wg and
+ * u = x Wu together ([Wg; Wu] stacked in each MMA); its epilogue packs the
+ * positions where z > 0 exactly as twell_gate_pack does (same counts, indices
+ * and overflow flags) but stores h_j = bf16(ReLU(z_j) * u_j) in `vals`.
+ */
+twell_status twell_gate_up_pack(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, int T, int d,
+                                int f, const twell_t* tw, int32_t* dev_status, void* stream);
+
+/*
+ * Down projection from a TwELL holding hidden activations (twell_gate_up_pack):
+ * y_t = sum over stored slots (j, h) of h * Wd[j, :], fp32 accumulation, fp32
+ * y. Overflow handling as in twell_sparse_ffn.
+ */
+twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                               int skip_overflow_rows, float* y, int32_t* dev_status, void* stream);
+
+/*
+ * Hybrid forward of the tensor-core-up variant = twell_gate_up_pack,
+ * twell_route, twell_sparse_down with overflowing rows skipped, and
+ * twell_dense_rows_forward on ovf_rows. Same arguments and workspace as
+ * twell_ffn_hybrid_forward.
+ */
+twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                            const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                                            float* y, int32_t* ovf_rows, int32_t* n_ovf, void* workspace,
+                                            size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * Routing step of the hybrid route (source: the hybrid paragraph of the
  * fused-kernel section above): ovf_rows[0..n_ovf) = rows with row_ovf set,
  * in ascending order; *n_ovf (device int32) = their number. ovf_rows has T

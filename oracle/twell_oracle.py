@@ -47,6 +47,9 @@ __all__ = [
     "twell_unpack",
     "sparse_ffn_from_twell",
     "hybrid_ffn",
+    "twell_pack_hidden",
+    "sparse_down_from_twell",
+    "hybrid_ffn_up_dense",
 ]
 
 
@@ -196,3 +199,56 @@ def hybrid_ffn(x_bits, WgT_bits, WuT_bits, Wd_bits, tile: int, W: int) -> dict:
     if ovf.size:
         y[ovf] = gated_ffn(np.asarray(x_bits)[ovf], WgT_bits, WuT_bits, Wd_bits)
     return {"y": y, "twell": tw, "ovf_rows": ovf, "z": z}
+
+
+# ---------------------------------------------------------------------------
+# Variant with the up projection on the tensor cores: the gate GEMM also forms
+# u = x . Wu, and the packed values are the hidden activations h = ReLU(z) * u
+# at the same positions; the sparse step is then the down projection alone.
+# The positions, counts and routing are those of twell_pack(z).
+
+
+def twell_pack_hidden(z: np.ndarray, u: np.ndarray, tile: int, W: int) -> dict:
+    """TwELL of the pattern of ReLU(z) holding bf16(ReLU(z) * u) as values."""
+    tw = twell_pack(z, tile, W)
+    T, nT, _ = tw["idx"].shape
+    n = np.minimum(tw["counts"].astype(np.int64), W)
+    live = np.arange(W)[None, None, :] < n[:, :, None]
+    t, c, s = np.nonzero(live)
+    j = tw["idx"][t, c, s].astype(np.int64)
+    tw["vals"][t, c, s] = f64_to_bf16_bits(np.maximum(z[t, j], 0.0) * u[t, j])
+    return tw
+
+
+def sparse_down_from_twell(tw: dict, Wd_bits, rows=None) -> np.ndarray:
+    """y_t = sum over stored slots (j, h) of h * Wd[j, :], in float64."""
+    counts, idx, vals = tw["counts"], tw["idx"], tw["vals"]
+    T, nT, W = idx.shape
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    Wd = bf16_bits_to_f64(Wd_bits)
+    y = np.zeros((len(rows), Wd.shape[1]))
+    for r, t in enumerate(rows):
+        n = np.minimum(counts[t].astype(np.int64), W)
+        js = np.concatenate([idx[t, c, : n[c]] for c in range(nT)]).astype(np.int64)
+        if js.size:
+            hs = bf16_bits_to_f64(np.concatenate([vals[t, c, : n[c]] for c in range(nT)]))
+            y[r] = hs @ Wd[js]
+    return y
+
+
+def hybrid_ffn_up_dense(x_bits, WgT_bits, WuT_bits, Wd_bits, tile: int, W: int) -> dict:
+    """Hybrid forward of the tensor-core-up variant: rows that fit use the
+    stored bf16 hidden values, overflow rows the dense layer."""
+    x = bf16_bits_to_f64(x_bits)
+    z = x @ bf16_bits_to_f64(WgT_bits).T
+    u = x @ bf16_bits_to_f64(WuT_bits).T
+    tw = twell_pack_hidden(z, u, tile, W)
+    ovf = route_rows(tw["counts"], W)
+    T = z.shape[0]
+    keep = np.setdiff1d(np.arange(T), ovf)
+    y = np.zeros((T, np.asarray(Wd_bits).shape[1]))
+    if keep.size:
+        y[keep] = sparse_down_from_twell(tw, Wd_bits, rows=keep)
+    if ovf.size:
+        y[ovf] = gated_ffn(np.asarray(x_bits)[ovf], WgT_bits, WuT_bits, Wd_bits)
+    return {"y": y, "twell": tw, "ovf_rows": ovf}

@@ -9,8 +9,8 @@ import torch
 from activation_sparse_gated_gemm_b200 import synth
 from activation_sparse_gated_gemm_b200 import twell as tl
 from oracle import twell_oracle as O
-from tests.gpu_helpers import (assert_dense_bf16_hidden_bound, assert_twell_equal, assert_y_close,
-                               oracle_pack_rows, run_pack, twell_to_host, upload, y_to_f64)
+from tests.gpu_helpers import (assert_dense_bf16_hidden_bound, assert_twell_equal, assert_within_stored_value_bound,
+                               assert_y_close, oracle_pack_rows, run_pack, twell_to_host, upload, y_to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -80,8 +80,9 @@ def test_ffn_forward_non_hybrid(cfg, layers):
     n_ovf = int(want["row_ovf"].sum())
     assert status == (tl.TWELL_ERR_OVERFLOW if n_ovf else 0)
     keep = np.nonzero(want["row_ovf"] == 0)[0]
-    y_ref = O.gated_ffn(L["x"][keep], L["WgT"], L["WuT"], L["Wd"])
+    y_ref = O.sparse_ffn_from_twell(want, L["x"], L["WuT"], L["Wd"], rows=keep)
     assert_y_close(y_to_f64(y)[keep], y_ref)
+    assert_within_stored_value_bound(y_to_f64(y)[keep], L, keep)
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=IDS)
@@ -101,12 +102,14 @@ def test_hybrid_forward(cfg, layers):
     assert n == len(out["ovf_rows"])
     assert np.array_equal(ovf_rows[:n].cpu().numpy(), out["ovf_rows"])
     assert_twell_equal(twell_to_host(tw), out["twell"], cfg.W)
-    y_dense = O.gated_ffn(L["x"], L["WgT"], L["WuT"], L["Wd"])
     yg = y_to_f64(y)
     assert np.isfinite(yg).all()
-    assert_y_close(yg, y_dense)
+    assert_y_close(yg, out["y"])
+    keep = np.setdiff1d(np.arange(cfg.T), out["ovf_rows"])
+    assert_within_stored_value_bound(yg[keep], L, keep)
     if n:
-        assert_y_close(yg[out["ovf_rows"]], y_dense[out["ovf_rows"]], "dense-branch rows")
+        y_dense = O.gated_ffn(L["x"][out["ovf_rows"]], L["WgT"], L["WuT"], L["Wd"])
+        assert_y_close(yg[out["ovf_rows"]], y_dense, "dense-branch rows")
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=IDS)
@@ -231,3 +234,73 @@ def test_out_of_range_index_is_reported_not_read(layers):
     st = tl.new_status()
     tl.sparse_ffn(dev["x"], dev["WuT"], dev["Wd"], tw, y, True, st)
     assert tl.status_get(st) == tl.TWELL_ERR_INDEX
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core-up variant: the gate GEMM also forms u, TwELL holds h = z * u
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_gate_up_pack_pattern_bit_exact_and_hidden_values(cfg, layers):
+    L = layers[cfg.name]
+    dev = upload(L)
+    tw = tl.Twell(cfg.T, cfg.f, cfg.W)
+    st = tl.new_status()
+    tl.gate_up_pack(dev["x"], dev["WgT"], dev["WuT"], tw, st)
+    assert tl.status_get(st) == 0
+    x = O.bf16_bits_to_f64(L["x"])
+    z = x @ O.bf16_bits_to_f64(L["WgT"]).T
+    u = x @ O.bf16_bits_to_f64(L["WuT"]).T
+    want = O.twell_pack_hidden(z, u, cfg.tile, cfg.W)
+    got = twell_to_host(tw)
+    assert np.array_equal(got["counts"], want["counts"])
+    assert np.array_equal(got["row_ovf"], want["row_ovf"])
+    n = np.minimum(want["counts"].astype(np.int64), cfg.W)
+    live = np.arange(cfg.W)[None, None, :] < n[:, :, None]
+    assert np.array_equal(got["idx"][live], want["idx"][live])
+    # u comes from fp32 tensor-core sums, so bf16(z * u) may differ by one ulp
+    hv, wv = O.bf16_bits_to_f64(got["vals"][live]), O.bf16_bits_to_f64(want["vals"][live])
+    assert np.all(np.abs(hv - wv) <= 2.0**-7 * np.abs(wv) + 1e-30)
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_hybrid_forward_tensor_core_up(cfg, layers):
+    L = layers[cfg.name]
+    dev = upload(L)
+    tw = tl.Twell(cfg.T, cfg.f, cfg.W)
+    y = torch.full((cfg.T, cfg.d), float("nan"), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.full((cfg.T,), -7, dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(cfg.T, cfg.d, cfg.f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward_tc_up(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    assert tl.status_get(st) == 0
+    out = O.hybrid_ffn_up_dense(L["x"], L["WgT"], L["WuT"], L["Wd"], cfg.tile, cfg.W)
+    n = int(n_ovf.item())
+    assert n == len(out["ovf_rows"])
+    assert np.array_equal(ovf_rows[:n].cpu().numpy(), out["ovf_rows"])
+    yg = y_to_f64(y)
+    assert np.isfinite(yg).all()
+    assert_y_close(yg, out["y"])
+    keep = np.setdiff1d(np.arange(cfg.T), out["ovf_rows"])
+    assert_within_stored_value_bound(yg[keep], L, keep, stored="h")
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_sparse_down_on_oracle_packed_input(cfg, layers):
+    L = layers[cfg.name]
+    dev = upload(L)
+    x = O.bf16_bits_to_f64(L["x"])
+    want = O.twell_pack_hidden(x @ O.bf16_bits_to_f64(L["WgT"]).T, x @ O.bf16_bits_to_f64(L["WuT"]).T,
+                               cfg.tile, cfg.W)
+    tw = tl.Twell(cfg.T, cfg.f, cfg.W)
+    tw.counts.copy_(torch.from_numpy(want["counts"]))
+    tw.idx.copy_(torch.from_numpy(want["idx"]))
+    tw.vals.copy_(torch.from_numpy(want["vals"].view(np.int16)).view(torch.bfloat16))
+    tw.row_ovf.copy_(torch.from_numpy(want["row_ovf"]))
+    y = torch.full((cfg.T, cfg.d), 3.0, dtype=torch.float32, device="cuda")
+    st = tl.new_status()
+    tl.sparse_down(dev["Wd"], tw, y, True, st)
+    assert tl.status_get(st) == 0
+    keep = np.nonzero(want["row_ovf"] == 0)[0]
+    assert_y_close(y_to_f64(y)[keep], O.sparse_down_from_twell(want, L["Wd"], rows=keep))

@@ -373,3 +373,49 @@ def test_generator_density_and_determinism():
     z = O.gate_preactivation(L["x"], L["WgT"])
     assert not np.any(z[:, L["dead"]] > 0)
     assert abs((z > 0).mean() - MID.density) < 0.01
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core-up variant: same pattern, hidden values, down projection alone
+
+
+def test_hidden_pack_keeps_the_gate_pattern_and_stores_h():
+    L = synth.make_layer(MID, seed=2)
+    x = O.bf16_bits_to_f64(L["x"])
+    z = x @ O.bf16_bits_to_f64(L["WgT"]).T
+    u = x @ O.bf16_bits_to_f64(L["WuT"]).T
+    tg = O.twell_pack(z, MID.tile, MID.W)
+    th = O.twell_pack_hidden(z, u, MID.tile, MID.W)
+    assert np.array_equal(tg["counts"], th["counts"]) and np.array_equal(tg["idx"], th["idx"])
+    assert np.array_equal(tg["row_ovf"], th["row_ovf"])
+    t, c = np.nonzero(tg["counts"] > 0)
+    t, c = t[:200], c[:200]
+    j = tg["idx"][t, c, 0].astype(np.int64)
+    want = torch_bf16_bits((z[t, j] * u[t, j]).astype(np.float32))  # z > 0 at stored slots
+    assert np.array_equal(th["vals"][t, c, 0], want)
+
+
+def test_down_only_equals_dense_when_hidden_is_bf16_exact():
+    rng = np.random.default_rng(12)
+    T, d, f = 16, 4, 256  # |z|, |u| <= 4, so h = z * u is an integer <= 16: exact in bf16
+    x = bits_of_exact(rng.integers(-1, 2, size=(T, d)).astype(np.float64))
+    WgT = bits_of_exact(rng.integers(-1, 2, size=(f, d)).astype(np.float64))
+    WuT = bits_of_exact(rng.integers(-1, 2, size=(f, d)).astype(np.float64))
+    Wd = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    xf = O.bf16_bits_to_f64(x)
+    z, u = xf @ O.bf16_bits_to_f64(WgT).T, xf @ O.bf16_bits_to_f64(WuT).T
+    th = O.twell_pack_hidden(z, u, 128, 128)
+    yd = O.gated_ffn(x, WgT, WuT, Wd)
+    np.testing.assert_allclose(O.sparse_down_from_twell(th, Wd), yd, rtol=1e-12, atol=1e-12 * np.abs(yd).max())
+
+
+def test_up_dense_hybrid_within_one_rounding_of_dense():
+    L = synth.make_layer(HEAVY, seed=0)
+    out = O.hybrid_ffn_up_dense(L["x"], L["WgT"], L["WuT"], L["Wd"], HEAVY.tile, HEAVY.W)
+    ref = O.hybrid_ffn(L["x"], L["WgT"], L["WuT"], L["Wd"], HEAVY.tile, HEAVY.W)
+    assert np.array_equal(out["ovf_rows"], ref["ovf_rows"])
+    x = O.bf16_bits_to_f64(L["x"])
+    h = np.maximum(x @ O.bf16_bits_to_f64(L["WgT"]).T, 0) * (x @ O.bf16_bits_to_f64(L["WuT"]).T)
+    wd = O.bf16_bits_to_f64(L["Wd"])
+    bound = np.abs(h) @ np.abs(wd) * 2.0**-8 + 1e-12
+    assert np.all(np.abs(out["y"] - h @ wd) <= bound)
