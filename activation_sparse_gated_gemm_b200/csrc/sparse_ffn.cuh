@@ -29,9 +29,12 @@ struct SparseParams {
   int* dev_status;
 };
 
-// Warps per block of the sparse kernel: 12 while a token's x and y chunks fit
-// the register budget of 12 warps per SM (d <= 1536), 8 above.
-constexpr int sparse_warps_for(int nch) { return nch <= 6 ? 12 : 8; }
+// Warps per block of the sparse kernel, as many as the register budget of one
+// block per SM allows: the up+down kernel holds x chunks, y and two weight
+// rows; the down-only kernel needs no x.
+constexpr int sparse_warps_for(int nch, bool down_only) {
+  return down_only ? (nch <= 6 ? 16 : (nch <= 9 ? 12 : 8)) : (nch <= 6 ? 12 : 8);
+}
 
 // Read-only 16-byte load through the non-coherent path. Left as an ordinary
 // (non-volatile) operation so the compiler may issue it as early as its
@@ -342,3 +345,4 @@ __global__ void __launch_bounds__(256) unpack_kernel(const int16_t* counts, cons
 }
 
 }  // namespace twell
+

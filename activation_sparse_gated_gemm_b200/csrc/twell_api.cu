@@ -182,7 +182,7 @@ twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uin
 
 template <int NCH, bool DOWN_ONLY>
 twell_status launch_sparse_n(const SparseParams& p, int sms, cudaStream_t s) {
-  constexpr int kWarps = sparse_warps_for(NCH);
+  constexpr int kWarps = sparse_warps_for(NCH, DOWN_ONLY);
   // persistent warps: one resident block per SM
   const int blocks = std::min((p.T + kWarps - 1) / kWarps, sms);
   const size_t smem = static_cast<size_t>(kWarps) * (NCH * 32 * sizeof(uint4) + kListCap * sizeof(uint32_t));
@@ -236,6 +236,12 @@ twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t*
   p.skip_ovf = skip ? 1 : 0;
   p.dev_status = dev_status;
   return down_only ? sparse_launch<true>(p, d, sms, s) : sparse_launch<false>(p, d, sms, s);
+}
+
+// Down projection from a TwELL of hidden activations (per-token gathers of Wd rows).
+twell_status down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip, float* y,
+                       int32_t* dev_status, cudaStream_t s, int sms) {
+  return sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, skip, y, dev_status, s, sms, true);
 }
 
 // Dense gated FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu)
@@ -349,8 +355,7 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
   TW_TRY(check_ptrs({Wd, y, dev_status}));
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  return sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, skip_overflow_rows, y, dev_status,
-                     static_cast<cudaStream_t>(stream), sms, true);
+  return down_impl(Wd, T, d, f, tw, skip_overflow_rows, y, dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 
 twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
@@ -372,7 +377,7 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
   TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms));
   route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, 1, y, dev_status, s, sms, true));
+  TW_TRY(down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
 }
 
