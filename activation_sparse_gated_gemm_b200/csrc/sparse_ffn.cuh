@@ -303,9 +303,11 @@ __global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int
   if (threadIdx.x == 0) *n_ovf = base;
 }
 
-// out[i, :] = x[rows[i], :] for i < *n_rows (clamped to T, the room in rows and out).
+// out[i, :] = x[rows[i], :] for i < *n_rows (clamped to T, the room in rows and
+// out); when y_zero is given, also y_zero[rows[i], :] = 0 (the dense branch may
+// add split partial sums into those rows).
 __global__ void gather_rows_kernel(const uint16_t* x, int d, const int* rows, const int* n_rows, int T,
-                                   uint16_t* out, int* dev_status) {
+                                   uint16_t* out, float* y_zero, int* dev_status) {
   const int n = min(max(*n_rows, 0), T);
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
     const int r = rows[i];
@@ -316,6 +318,10 @@ __global__ void gather_rows_kernel(const uint16_t* x, int d, const int* rows, co
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * d);
     uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(i) * d);
     for (int k = threadIdx.x; k < d / 8; k += blockDim.x) dst[k] = src[k];
+    if (y_zero != nullptr) {
+      float4* yz = reinterpret_cast<float4*>(y_zero + static_cast<size_t>(r) * d);
+      for (int k = threadIdx.x; k < d / 4; k += blockDim.x) yz[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 }
 

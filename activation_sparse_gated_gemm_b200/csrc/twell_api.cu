@@ -277,6 +277,9 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
   p2.ldo = d;
   p2.row_map = row_map;
   p2.out_rows = y_rows;
+  // the routed rows of y were zeroed by the gather; the full-batch dense
+  // baseline stores without splitting
+  p2.k_splits_max = row_map != nullptr ? 32 : 1;
   p2.dev_status = dev_status;
   const int g2 = M_dev ? sms : gemm_grid(M, d, kBN, sms);
   return launch_gemm<kModeDown>(mh, md, md, p2, g2, s);
@@ -288,7 +291,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 twell_status dense_rows_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
                              int T, int d, int f, const int32_t* rows, const int32_t* n_rows, float* y,
                              uint16_t* xo, uint16_t* ho, int32_t* dev_status, cudaStream_t s, int sms) {
-  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, rows, n_rows, T, xo, dev_status);
+  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, rows, n_rows, T, xo, y, dev_status);
   TW_TRY(cuda_ok(cudaGetLastError()));
   return dense_impl(xo, T, n_rows, WgT, WuT, Wd, d, f, ho, true, rows, y, T, dev_status, s, sms);
 }

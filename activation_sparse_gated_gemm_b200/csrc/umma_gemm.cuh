@@ -82,8 +82,17 @@ struct GemmParams {
   // kModeDown: B rows are read at k mod k_wrap (k_wrap > 0), so K = 2 * k_wrap
   // runs [h_hi | h_lo] against [Wd ; Wd].
   int k_wrap;
+  // kModeDown: when the output tiles do not fill the grid, K is cut into up to
+  // this many splits whose partial sums are added into out_f32 (which must
+  // hold zeros in the rows written); 0 or 1 disables splitting.
+  int k_splits_max;
   int* dev_status;
 };
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
 
 // Appends the set bits of `mask` (column col0 + i, value vrow[i]) to one row's
 // slot list of a TwELL tile in ascending column order, staging 8 slots at a
@@ -145,8 +154,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   constexpr int kTileN = kStacked ? 128 : kBN;  // output columns per tile
   const int num_m = (M + kBM - 1) / kBM;
   const int num_n = (p.N + kTileN - 1) / kTileN;
-  const int num_tiles = num_m * num_n;
   const int num_kb = p.K / kBK;
+  // K splits (kModeDown only): as many as keep every CTA busy, none empty.
+  int kb_per = num_kb, k_splits = 1;
+  if (MODE == kModeDown && p.k_splits_max > 1 && num_m * num_n > 0) {
+    int want = min(p.k_splits_max, max(1, static_cast<int>(gridDim.x) / (num_m * num_n)));
+    want = min(want, num_kb);
+    kb_per = (num_kb + want - 1) / want;
+    k_splits = (num_kb + kb_per - 1) / kb_per;
+  }
+  const int num_tiles = num_m * num_n * k_splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -180,9 +197,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued = 0, issued_par = 0;  // per stage: a load is outstanding / its phase parity
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile / num_n;
-        const int n_blk = tile - m_blk * num_n;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int mn = tile / k_splits;
+        const int ks = tile - mn * k_splits;
+        const int m_blk = mn / num_n;
+        const int n_blk = mn - m_blk * num_n;
+        const int kb_end = min(num_kb, (ks + 1) * kb_per);
+        for (int kb = ks * kb_per; kb < kb_end; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -236,7 +256,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int ks = tile % k_splits;
+        const int kb_begin = ks * kb_per, kb_end = min(num_kb, (ks + 1) * kb_per);
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
             break;
@@ -257,7 +279,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             } else {
               bdesc = umma_smem_desc(b_addr + k * 32, 16, 1024);
             }
-            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (kb != kb_begin || k != 0) ? 1u : 0u);
             any_mma = true;
           }
           umma_commit(&empty[s]);
@@ -296,8 +318,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m_blk = tile / num_n;
-      const int n_blk = tile - m_blk * num_n;
+      const int mn = tile / k_splits;
+      const int m_blk = mn / num_n;
+      const int n_blk = mn - m_blk * num_n;
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(buf * kBN) + (static_cast<uint32_t>(q * 32) << 16);
       const int row_base = m_blk * kBM + q * 32;
       const int my_row = row_base + lane;
@@ -436,9 +459,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int col = n_blk * kBN + ch * 32;
           if (valid && col < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out_f32 + static_cast<size_t>(orow) * p.ldo + col);
+            float* dst = p.out_f32 + static_cast<size_t>(orow) * p.ldo + col;
+            if (k_splits > 1) {
 #pragma unroll
-            for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+              for (int v = 0; v < 8; ++v)
+                red_add_v4(dst + 4 * v, __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            } else {
+              uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+              for (int v = 0; v < 8; ++v) d4[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            }
           }
         }
       }
