@@ -26,6 +26,10 @@ struct SparseParams {
   float* y;
   int T, d, f, nT, W;
   int skip_ovf;
+  // Column tiles per work unit. A unit of all nT tiles stores y_t; smaller
+  // units (used when T is small, to spread one token over several warps) add
+  // their partial y_t into y, which must then hold zeros.
+  int unit_tiles;
   int* dev_status;
 };
 
@@ -117,17 +121,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
   // Block b owns the contiguous tokens [t_begin, t_end); its warps take them
   // one at a time from a shared counter, so a warp that drew light tokens
   // keeps working while another finishes a heavy one.
-  __shared__ int next_token;
-  const int t_begin = static_cast<int>(static_cast<long long>(p.T) * blockIdx.x / gridDim.x);
-  const int t_end = static_cast<int>(static_cast<long long>(p.T) * (blockIdx.x + 1) / gridDim.x);
-  if (threadIdx.x == 0) next_token = t_begin;
+  __shared__ int next_unit;
+  const int units_per_token = (p.nT + p.unit_tiles - 1) / p.unit_tiles;
+  const bool partial = units_per_token > 1;
+  const long long n_units = static_cast<long long>(p.T) * units_per_token;
+  const int u_begin = static_cast<int>(n_units * blockIdx.x / gridDim.x);
+  const int u_end = static_cast<int>(n_units * (blockIdx.x + 1) / gridDim.x);
+  if (threadIdx.x == 0) next_unit = u_begin;
   __syncthreads();
 #pragma unroll 1
   for (;;) {
-    int t = 0;
-    if (lane == 0) t = atomicAdd(&next_token, 1);
-    t = __shfl_sync(0xffffffffu, t, 0);
-    if (t >= t_end) break;
+    int u = 0;
+    if (lane == 0) u = atomicAdd(&next_unit, 1);
+    u = __shfl_sync(0xffffffffu, u, 0);
+    if (u >= u_end) break;
+    const int t = u / units_per_token;
+    const int c_first = (u - t * units_per_token) * p.unit_tiles;
+    const int c_last = min(p.nT, c_first + p.unit_tiles);
     if (p.skip_ovf && p.row_ovf[t]) continue;
     __syncwarp();
     if (!DOWN_ONLY) {
@@ -144,8 +154,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
       for (int e = 0; e < 8; ++e) y[i][e] = 0.0f;
 
 #pragma unroll 1
-    for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
-      const int c1 = min(p.nT, c0 + group_tiles);
+    for (int c0 = c_first; c0 < c_last; c0 += group_tiles) {
+      const int c1 = min(c_last, c0 + group_tiles);
       // ---- flatten the slots of tiles [c0, c1) into list[0, total)
       int total = 0;
 #pragma unroll 1
@@ -257,15 +267,30 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
     for (int i = 0; i < NCH; ++i) {
       const int k0 = (i * 32 + lane) * 8;
       if (k0 < d) {
-        float4* dst = reinterpret_cast<float4*>(p.y + static_cast<size_t>(t) * d + k0);
-        dst[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
-        dst[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
+        float* dst = p.y + static_cast<size_t>(t) * d + k0;
+        if (partial) {
+          red_add_v4(dst, y[i][0], y[i][1], y[i][2], y[i][3]);
+          red_add_v4(dst + 4, y[i][4], y[i][5], y[i][6], y[i][7]);
+        } else {
+          reinterpret_cast<float4*>(dst)[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+          reinterpret_cast<float4*>(dst)[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
+        }
       }
     }
   }
   // each lane saw the counts of its own tiles
   if (__any_sync(0xffffffffu, overflow) && lane == 0 && !p.skip_ovf) raise_status(p.dev_status, kDevOverflow);
   if (__any_sync(0xffffffffu, bad_index) && lane == 0) raise_status(p.dev_status, kDevIndex);
+}
+
+// y[t, :] = 0 for the rows the sparse step will write (all rows, or those
+// without the overflow flag when overflow rows are skipped).
+__global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf, int skip_ovf) {
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    if (skip_ovf && row_ovf[t]) continue;
+    float4* row = reinterpret_cast<float4*>(y + static_cast<size_t>(t) * d);
+    for (int k = threadIdx.x; k < d / 4; k += blockDim.x) row[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 // ---------------------------------------------------------------- routing

@@ -181,10 +181,24 @@ twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uin
 }
 
 template <int NCH, bool DOWN_ONLY>
-twell_status launch_sparse_n(const SparseParams& p, int sms, cudaStream_t s) {
+twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s) {
   constexpr int kWarps = sparse_warps_for(NCH, DOWN_ONLY);
-  // persistent warps: one resident block per SM
-  const int blocks = std::min((p.T + kWarps - 1) / kWarps, sms);
+  // With fewer tokens than resident warps, a token's column tiles are spread
+  // over several warps whose partial sums are added into a zeroed y (rows that
+  // the sparse step skips are rewritten by the dense branch afterwards).
+  const long long warps_resident = static_cast<long long>(kWarps) * sms;
+  p.unit_tiles = p.nT;
+  if (static_cast<long long>(p.T) * 2 < warps_resident) {
+    const long long want_units = warps_resident;  // about one unit per resident warp
+    const long long per_token = std::max(1LL, std::min<long long>(p.nT, want_units / std::max(1, p.T)));
+    p.unit_tiles = static_cast<int>((p.nT + per_token - 1) / per_token);
+    if (p.unit_tiles < p.nT) {
+      zero_rows_kernel<<<std::min(p.T, 4 * sms), 256, 0, s>>>(p.y, p.T, p.d, p.row_ovf, p.skip_ovf);
+      TW_TRY(cuda_ok(cudaGetLastError()));
+    }
+  }
+  const long long units = static_cast<long long>(p.T) * ((p.nT + p.unit_tiles - 1) / p.unit_tiles);
+  const int blocks = static_cast<int>(std::min<long long>((units + kWarps - 1) / kWarps, sms));
   const size_t smem = static_cast<size_t>(kWarps) * (NCH * 32 * sizeof(uint4) + kListCap * sizeof(uint32_t));
   auto kern = sparse_ffn_warp_kernel<NCH, kWarps, DOWN_ONLY>;
   if (smem > 48 * 1024)
@@ -195,6 +209,7 @@ twell_status launch_sparse_n(const SparseParams& p, int sms, cudaStream_t s) {
 
 template <bool DOWN_ONLY>
 twell_status sparse_launch(const SparseParams& p, int d, int sms, cudaStream_t s) {
+  // (the launcher decides how a token's column tiles are split over warps)
   switch ((d + 255) / 256) {
     case 1: return launch_sparse_n<1, DOWN_ONLY>(p, sms, s);
     case 2: return launch_sparse_n<2, DOWN_ONLY>(p, sms, s);
@@ -277,9 +292,16 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
   p2.ldo = d;
   p2.row_map = row_map;
   p2.out_rows = y_rows;
-  // the routed rows of y were zeroed by the gather; the full-batch dense
-  // baseline stores without splitting
-  p2.k_splits_max = row_map != nullptr ? 32 : 1;
+  // The routed rows of y were zeroed by the gather. The full-batch dense
+  // baseline splits K only when its output tiles cannot fill the GPU, after
+  // zeroing y.
+  p2.k_splits_max = 1;
+  if (row_map != nullptr) {
+    p2.k_splits_max = 32;
+  } else if (static_cast<long long>((M + kBM - 1) / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms) {
+    TW_TRY(cuda_ok(cudaMemsetAsync(y, 0, static_cast<size_t>(M) * d * sizeof(float), s)));
+    p2.k_splits_max = 32;
+  }
   p2.dev_status = dev_status;
   const int g2 = M_dev ? sms : gemm_grid(M, d, kBN, sms);
   return launch_gemm<kModeDown>(mh, md, md, p2, g2, s);

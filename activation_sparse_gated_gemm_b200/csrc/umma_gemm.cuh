@@ -89,10 +89,6 @@ struct GemmParams {
   int* dev_status;
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 // Appends the set bits of `mask` (column col0 + i, value vrow[i]) to one row's
 // slot list of a TwELL tile in ascending column order, staging 8 slots at a

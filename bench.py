@@ -169,15 +169,27 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's value (replicas finish when the last one does)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, local_ms: float, world: int, device: str = "cuda") -> tuple:
+    """Whole-job tokens/s of `world` independent replicas: all ranks' tokens
+    over the slowest rank's step time. Returns (tokens/s, max ms)."""
+    ms = max_over_ranks(local_ms, world, device)
+    return job_rate(tokens_per_rank, world, ms), ms
+
+
+def job_rate(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    return world * tokens_per_rank / (max_ms * 1e-3)
 
 
 def blas_threads() -> int:
@@ -383,7 +395,7 @@ def run_gpu(args, world, rank, local):
 
     res = {
         "metric": METRIC,
-        "value": world * T / (step_ms * 1e-3),
+        "value": job_rate(T, world, step_ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -413,7 +425,7 @@ def run_gpu(args, world, rank, local):
         "speedup_vs_own_dense": dense_ms / step_ms,
         "batch_stats": {"n_ovf": n_ovf_h, "nnz_stored": nnz_stored, "union_cols": union_cols,
                         "mean_density": float(counts.sum()) / (T * f)},
-        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4},
         "gpu_launches": 6 * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
@@ -501,7 +513,11 @@ def run_sweep(args) -> None:
                     ts.append(a.elapsed_time(b))
                 return float(np.median(ts))
 
-            ms = timed(lambda: tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st), args.steps)
+            ms_gate = timed(lambda: tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st),
+                            args.steps)
+            ms_tc = timed(lambda: tl.ffn_hybrid_forward_tc_up(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st),
+                          args.steps)
+            ms, form = (ms_gate, "gate") if ms_gate <= ms_tc else (ms_tc, "tc_up")
             ms_dense = timed(lambda: tl.dense_ffn_forward(x, WgT, WuT, Wd, y, wsd, st), args.steps)
             status = tl.status_get(st)
             counts = tw.counts.to(torch.int64)
@@ -515,7 +531,8 @@ def run_sweep(args) -> None:
             t_roof = max((alg["gate_flops"] + alg["dense_branch_flops"]) / (peaks["bf16_tflops"] * 1e12),
                          alg["alg_bytes"] / (peaks["hbm_gbs"] * 1e9))
             print(json.dumps({"sweep": True, "T": T, "density": pden, "W": cfg.W, "d": cfg.d, "f": cfg.f,
-                              "ms": ms, "tokens_per_s": T / (ms * 1e-3), "dense_ms": ms_dense,
+                              "ms": ms, "form": form, "ms_gate_form": ms_gate, "ms_tc_up_form": ms_tc,
+                              "tokens_per_s": T / (ms * 1e-3), "dense_ms": ms_dense,
                               "speedup_vs_own_dense": ms_dense / ms, "roofline_frac": t_roof / (ms * 1e-3),
                               "t_roof_us": t_roof * 1e6, "n_ovf": n_o,
                               "measured_density": float(counts.sum()) / (T * cfg.f), "status": status}),
