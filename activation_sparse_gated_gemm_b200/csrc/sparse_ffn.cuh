@@ -80,6 +80,19 @@ __device__ __forceinline__ void mixdot8(const uint4& a, const uint4& b, float& a
       : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
 }
 
+// y[0..8) += h * w[0..8) with h and w in bf16: mixed-precision fma (exact
+// bf16 x bf16 product, one fp32 rounding), no unpacking of w.
+__device__ __forceinline__ void axpy8_bf16(float (&y)[8], uint16_t h, const uint4& w) {
+  asm("{\n\t.reg .b16 w0, w1, w2, w3, w4, w5, w6, w7;\n\t"
+      "mov.b32 {w0, w1}, %9; mov.b32 {w2, w3}, %10; mov.b32 {w4, w5}, %11; mov.b32 {w6, w7}, %12;\n\t"
+      "fma.rn.f32.bf16 %0, %8, w0, %0; fma.rn.f32.bf16 %1, %8, w1, %1;\n\t"
+      "fma.rn.f32.bf16 %2, %8, w2, %2; fma.rn.f32.bf16 %3, %8, w3, %3;\n\t"
+      "fma.rn.f32.bf16 %4, %8, w4, %4; fma.rn.f32.bf16 %5, %8, w5, %5;\n\t"
+      "fma.rn.f32.bf16 %6, %8, w6, %6; fma.rn.f32.bf16 %7, %8, w7, %7;\n\t}"
+      : "+f"(y[0]), "+f"(y[1]), "+f"(y[2]), "+f"(y[3]), "+f"(y[4]), "+f"(y[5]), "+f"(y[6]), "+f"(y[7])
+      : "h"(h), "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w));
+}
+
 template <int NCH>
 __device__ __forceinline__ void load_row(uint4 (&w)[NCH], const uint16_t* row, int lane, int d) {
 #pragma unroll
@@ -241,13 +254,20 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
             if (lane == s + 1) my_h = my_g * acc;
           }
         }
-        // pass 2: down projection, h never leaves the registers
+        // pass 2: down projection, h never leaves the registers. When the
+        // stored value already is h (a bf16), the mixed-precision fma takes it
+        // and the bf16 weights directly.
+        const uint32_t my_hb = my_e >> 16;
         load_row<NCH>(wa, p.Wd + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
 #pragma unroll 1
         for (int s = 0; s < ns; s += 2) {
           if (s + 1 < ns)
             load_row<NCH>(wb, p.Wd + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 1)) * d, lane, d);
-          {
+          if (DOWN_ONLY) {
+            const uint16_t hb = static_cast<uint16_t>(__shfl_sync(0xffffffffu, my_hb, s));
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) axpy8_bf16(y[i], hb, wa[i]);
+          } else {
             const float h = __shfl_sync(0xffffffffu, my_h, s);
 #pragma unroll
             for (int i = 0; i < NCH; ++i) axpy8(y[i], h, wa[i]);
@@ -255,9 +275,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
           if (s + 1 < ns) {
             if (s + 2 < ns)
               load_row<NCH>(wa, p.Wd + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 2)) * d, lane, d);
-            const float h = __shfl_sync(0xffffffffu, my_h, s + 1);
+            if (DOWN_ONLY) {
+              const uint16_t hb = static_cast<uint16_t>(__shfl_sync(0xffffffffu, my_hb, s + 1));
 #pragma unroll
-            for (int i = 0; i < NCH; ++i) axpy8(y[i], h, wb[i]);
+              for (int i = 0; i < NCH; ++i) axpy8_bf16(y[i], hb, wb[i]);
+            } else {
+              const float h = __shfl_sync(0xffffffffu, my_h, s + 1);
+#pragma unroll
+              for (int i = 0; i < NCH; ++i) axpy8(y[i], h, wb[i]);
+            }
           }
         }
       }
