@@ -322,32 +322,56 @@ __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf,
 // ---------------------------------------------------------------- routing
 
 // Ascending list of the rows whose overflow flag is set, and its length. One
-// block of 1024 threads scans the flags in order, so the list is deterministic.
+// block of 1024 threads; per round each thread owns 16 consecutive flags
+// (read with one 16-byte load when they are in range), counts its own, and a
+// block-wide scan gives every thread the position of its first flagged row,
+// so the list comes out in ascending order.
 __global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf) {
   __shared__ int warp_off[32];
   __shared__ int total_s;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const bool vec_ok = (reinterpret_cast<uintptr_t>(row_ovf) & 15u) == 0;
   int base = 0;
-  for (int start = 0; start < T; start += 1024) {
-    const int t = start + threadIdx.x;
-    const int flag = (t < T && row_ovf[t] != 0) ? 1 : 0;
-    const uint32_t m = __ballot_sync(0xffffffffu, flag);
-    if (lane == 0) warp_off[warp] = __popc(m);
+  for (int start = 0; start < T; start += 1024 * 16) {
+    const int t0 = start + threadIdx.x * 16;
+    uint32_t bits = 0;  // bit k: row t0 + k is flagged
+    if (vec_ok && t0 + 16 <= T) {
+      const uint4 v = *reinterpret_cast<const uint4*>(row_ovf + t0);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 16; ++k) bits |= ((w[k >> 2] >> (8 * (k & 3))) & 0xffu ? 1u : 0u) << k;
+    } else {
+      for (int k = 0; k < 16; ++k)
+        if (t0 + k < T && row_ovf[t0 + k] != 0) bits |= 1u << k;
+    }
+    const int mine = __popc(bits);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) warp_off[warp] = incl;
     __syncthreads();
     if (warp == 0) {
       const int v = warp_off[lane];
-      int incl = v;
+      int wi = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
+        const int u = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += u;
       }
-      warp_off[lane] = incl - v;
-      if (lane == 31) total_s = incl;
+      warp_off[lane] = wi - v;
+      if (lane == 31) total_s = wi;
     }
     __syncthreads();
-    if (flag) ovf_rows[base + warp_off[warp] + __popc(m & ((1u << lane) - 1u))] = t;
+    int pos = base + warp_off[warp] + incl - mine;
+    while (bits != 0) {
+      const int k = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      ovf_rows[pos++] = t0 + k;
+    }
     base += total_s;
     __syncthreads();
   }

@@ -129,7 +129,7 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kernel: str):
+def measured_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel sources and this workload; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -138,7 +138,7 @@ def measured_traffic(kernel: str):
             t = json.load(fh)
     except (OSError, ValueError):
         return None
-    if t.get("source_hash") != kernel_source_hash():
+    if t.get("source_hash") != kernel_source_hash() or t.get("workload") != workload:
         return None
     return t.get("kernels", {}).get(kernel)
 
@@ -391,7 +391,7 @@ def run_gpu(args, world, rank, local):
     ms = float(stage_ms[names.index(dom)])
     achieved = kd["work"] / (ms * 1e-3) / kd["scale"]
     peak = kd["peak"] / kd["scale"]
-    traffic = measured_traffic(dom)
+    traffic = measured_traffic(dom, cfg.name)
 
     res = {
         "metric": METRIC,
