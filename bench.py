@@ -407,8 +407,8 @@ def run_gpu(args, world, rank, local):
         "dtype": "bf16",
         "data": "synthetic (seeded generator; no dataset or trained weights)",
         "config": {"workload": f"{cfg.name}-like FFN layer forward, hybrid TwELL", "variant": chosen,
-                   "tokens": T, "d_model": d,
-                   "d_ff": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
+                   "tokens": T, "d": d,
+                   "f": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
                    "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "roofline": {"kernel": dom, "bound": kd["bound"], "achieved": achieved, "peak": peak, "unit": kd["unit"],
@@ -464,7 +464,7 @@ def run_reference(args, world, rank):
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
         "config": {"workload": f"{cfg.name}-like FFN layer forward, hybrid TwELL", "tokens": cfg.T,
-                   "d_model": cfg.d, "d_ff": cfg.f, "tile": cfg.tile, "ell_width": cfg.W,
+                   "d": cfg.d, "f": cfg.f, "tile": cfg.tile, "ell_width": cfg.W,
                    "density": cfg.density, "dead_frac": cfg.dead_frac},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": f"{sample} of {cfg.T} tokens per step (fp64 numpy oracle)"},

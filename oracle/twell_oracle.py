@@ -16,7 +16,7 @@ Sources (three news pages about one release; cited by page and section):
 * [P2] gate.com post 20977915 -- paragraph on the TwELL format (tiles packed
   locally by each compute unit).
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 
 * a hidden unit is active iff its gate pre-activation is strictly positive;
 * TwELL keeps, per row and per 128-column tile, the true nonzero count and the
