@@ -50,6 +50,8 @@ __all__ = [
     "twell_pack_hidden",
     "sparse_down_from_twell",
     "hybrid_ffn_up_dense",
+    "relu_ffn",
+    "hybrid_relu_ffn",
 ]
 
 
@@ -251,4 +253,36 @@ def hybrid_ffn_up_dense(x_bits, WgT_bits, WuT_bits, Wd_bits, tile: int, W: int) 
         y[keep] = sparse_down_from_twell(tw, Wd_bits, rows=keep)
     if ovf.size:
         y[ovf] = gated_ffn(np.asarray(x_bits)[ovf], WgT_bits, WuT_bits, Wd_bits)
+    return {"y": y, "twell": tw, "ovf_rows": ovf}
+
+
+# ---------------------------------------------------------------------------
+# Non-gated variant y = ReLU(x . W1) . W2 [P1, "Ограничения и открытые
+# вопросы": the method also applies to the non-gated FFN, with a smaller
+# gain]. The pack is twell_pack of z = x . W1 and the stored values are the
+# hidden activations themselves, so the sparse step is the down projection
+# alone (sparse_down_from_twell); overflow rows take the dense layer.
+
+
+def relu_ffn(x_bits, W1T_bits, W2_bits) -> np.ndarray:
+    """Dense non-gated ReLU FFN in float64. W1T is W1 transposed ([f, d]);
+    W2 is [f, d] (row j is hidden unit j's output vector)."""
+    x = bf16_bits_to_f64(x_bits)
+    h = np.maximum(x @ bf16_bits_to_f64(W1T_bits).T, 0.0)
+    return h @ bf16_bits_to_f64(W2_bits)
+
+
+def hybrid_relu_ffn(x_bits, W1T_bits, W2_bits, tile: int, W: int) -> dict:
+    """Hybrid forward of the non-gated layer: rows whose tiles fit use the
+    stored bf16 ReLU outputs, overflow rows the dense layer."""
+    z = gate_preactivation(x_bits, W1T_bits)
+    tw = twell_pack(z, tile, W)
+    ovf = route_rows(tw["counts"], W)
+    T = z.shape[0]
+    keep = np.setdiff1d(np.arange(T), ovf)
+    y = np.zeros((T, np.asarray(W2_bits).shape[1]))
+    if keep.size:
+        y[keep] = sparse_down_from_twell(tw, W2_bits, rows=keep)
+    if ovf.size:
+        y[ovf] = relu_ffn(np.asarray(x_bits)[ovf], W1T_bits, W2_bits)
     return {"y": y, "twell": tw, "ovf_rows": ovf}

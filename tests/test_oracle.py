@@ -419,3 +419,100 @@ def test_up_dense_hybrid_within_one_rounding_of_dense():
     wd = O.bf16_bits_to_f64(L["Wd"])
     bound = np.abs(h) @ np.abs(wd) * 2.0**-8 + 1e-12
     assert np.all(np.abs(out["y"] - h @ wd) <= bound)
+
+
+# ---------------------------------------------------------------------------
+# Non-gated variant y = ReLU(x W1) W2
+
+
+def test_relu_ffn_exact_rational_bruteforce():
+    rng = np.random.default_rng(21)
+    T, d, f = 3, 6, 10
+    x = torch_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    W1T = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    W2 = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    F = lambda b: [[Fraction(float(v)) for v in row] for row in O.bf16_bits_to_f64(b)]
+    xf, af, bf = F(x), F(W1T), F(W2)
+    y = O.relu_ffn(x, W1T, W2)
+    for t in range(T):
+        for k in range(d):
+            acc = Fraction(0)
+            for j in range(f):
+                zj = sum(xf[t][i] * af[j][i] for i in range(d))
+                acc += max(zj, Fraction(0)) * bf[j][k]
+            assert abs(y[t, k] - float(acc)) <= 1e-12 * max(1.0, abs(float(acc)))
+
+
+def test_relu_ffn_permutation_closed_form():
+    """Permutation weights: y[pc(j)] = ReLU(x[pa(j)]); a transposed operand
+    applies the inverse permutation and fails."""
+    rng = np.random.default_rng(22)
+    n, T = 32, 4
+    pa, pc = rng.permutation(n), rng.permutation(n)
+    eye = np.eye(n)
+    xv = rng.integers(-40, 40, size=(T, n)) / 8.0
+    y = O.relu_ffn(bits_of_exact(xv), bits_of_exact(eye[pa]), bits_of_exact(eye[pc]))
+    want = np.zeros((T, n))
+    for j in range(n):
+        want[:, pc[j]] = np.maximum(xv[:, pa[j]], 0)
+    assert np.array_equal(y, want)
+
+
+def test_relu_ffn_is_the_gated_layer_with_unit_up_projection():
+    """The synthetic x carries a constant 1 in its last feature, so an up
+    projection that selects it gives u == 1 and the gated layer reduces to the
+    non-gated one, exactly."""
+    cfg = synth.CONFIGS["tiny"]
+    L = synth.make_layer(cfg, seed=4)
+    assert np.all(O.bf16_bits_to_f64(L["x"])[:, -1] == 1.0)
+    sel = np.zeros((cfg.f, cfg.d))
+    sel[:, -1] = 1.0
+    assert np.array_equal(O.relu_ffn(L["x"], L["WgT"], L["Wd"]),
+                          O.gated_ffn(L["x"], L["WgT"], bits_of_exact(sel), L["Wd"]))
+
+
+def test_relu_hybrid_exact_when_hidden_is_bf16_exact_and_routes_like_the_gate():
+    rng = np.random.default_rng(23)
+    T, d, f, W = 40, 8, 384, 8
+    # z = (small-integer dot product over 7 features) + x[:, 7] * w1[:, 7]: the
+    # last feature is a bias of -4 (sparse rows) or +4 (five dense rows that
+    # overflow); every z is a small integer, exact in bf16
+    xv = rng.integers(-1, 2, size=(T, d)).astype(np.float64)
+    xv[:, 7] = 1.0
+    xv[:5, 7] = -1.0
+    x = bits_of_exact(xv)
+    w1 = rng.integers(-1, 2, size=(f, d)).astype(np.float64)
+    w1[:, 7] = -4.0
+    W1T = bits_of_exact(w1)
+    W2 = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+    out = O.hybrid_relu_ffn(x, W1T, W2, 128, W)
+    z = O.gate_preactivation(x, W1T)
+    assert np.array_equal(O.bf16_bits_to_f64(O.f64_to_bf16_bits(z)), z)
+    assert np.array_equal(out["ovf_rows"], O.route_rows(O.twell_pack(z, 128, W)["counts"], W))
+    assert set(range(5)) <= set(out["ovf_rows"].tolist()) and len(out["ovf_rows"]) < T // 2
+    keep = np.setdiff1d(np.arange(T), out["ovf_rows"])
+    assert out["twell"]["counts"][keep].sum() > 0  # the sparse branch has work
+    yd = O.relu_ffn(x, W1T, W2)
+    np.testing.assert_allclose(out["y"], yd, rtol=1e-12, atol=1e-12 * np.abs(yd).max())
+
+
+def test_relu_hybrid_within_one_rounding_of_dense_and_special_cases():
+    L = synth.make_layer(HEAVY, seed=1)
+    out = O.hybrid_relu_ffn(L["x"], L["WgT"], L["Wd"], HEAVY.tile, HEAVY.W)
+    z = O.gate_preactivation(L["x"], L["WgT"])
+    g = np.maximum(z, 0)
+    w2 = O.bf16_bits_to_f64(L["Wd"])
+    bound = g @ np.abs(w2) * 2.0**-8 + 1e-12
+    assert np.all(np.abs(out["y"] - g @ w2) <= bound)
+    assert np.array_equal(out["y"][out["ovf_rows"]], (g @ w2)[out["ovf_rows"]])
+    # all-negative pre-activation: y == 0; one active column: y = z_j W2[j]
+    neg = O.bf16_bits_to_f64(L["WgT"]).copy()
+    neg[:, -1] = -64.0
+    assert not np.any(O.hybrid_relu_ffn(L["x"], bits_of_exact(neg), L["Wd"], HEAVY.tile, HEAVY.W)["y"])
+    js = 130
+    neg[js, -1] = 64.0
+    zj = O.bf16_bits_to_f64(L["x"]) @ neg[js]
+    assert np.all(zj > 0)
+    got = O.hybrid_relu_ffn(L["x"], bits_of_exact(neg), L["Wd"], HEAVY.tile, HEAVY.W)["y"]
+    want = O.bf16_bits_to_f64(O.f64_to_bf16_bits(zj))[:, None] * w2[js][None, :]
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
