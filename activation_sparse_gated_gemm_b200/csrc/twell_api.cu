@@ -259,16 +259,19 @@ twell_status down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* t
   return sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, skip, y, dev_status, s, sms, true);
 }
 
-// Dense gated FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu)
-// into h_buf, then out[row_map[i]] = h[i] Wd (row_map null: identity). With split, h_buf is
-// [M][2f] holding bf16(h) and the bf16 remainder, and the down GEMM runs K = 2f.
+// Dense FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu), or
+// h = ReLU(A Wg) for the non-gated layer (WuT null), into h_buf, then
+// out[row_map[i]] = h[i] Wd (row_map null: identity). With split, h_buf is [M][2f] holding
+// bf16(h) and the bf16 remainder, and the down GEMM runs K = 2f.
 twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const uint16_t* WgT, const uint16_t* WuT,
                         const uint16_t* Wd, int d, int f, uint16_t* h_buf, bool split, const int* row_map,
                         float* y, int y_rows, int32_t* dev_status, cudaStream_t s, int sms) {
   const int hk = split ? 2 * f : f;
+  const bool gated = WuT != nullptr;
+  const int tile_n = gated ? 128 : kBN;  // h columns per output tile of the first GEMM
   CUtensorMap ma, mg, mu, mh, md;
-  if (!make_map(&ma, a_rows, d, M, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, 128) ||
-      !make_map(&mu, WuT, d, f, kBK, 128) || !make_map(&mh, h_buf, hk, M, kBK, kBM) ||
+  if (!make_map(&ma, a_rows, d, M, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, tile_n) ||
+      (gated && !make_map(&mu, WuT, d, f, kBK, 128)) || !make_map(&mh, h_buf, hk, M, kBK, kBM) ||
       !make_map(&md, Wd, d, f, 64, kBK))
     return TWELL_ERR_CUDA;
   GemmParams p1{};
@@ -280,8 +283,12 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
   p1.ldo = hk;
   p1.h_split = split ? 1 : 0;
   p1.dev_status = dev_status;
-  const int g1 = M_dev ? sms : gemm_grid(M, f, 128, sms);
-  TW_TRY(launch_gemm<kModeGateUp>(ma, mg, mu, p1, g1, s));
+  const int g1 = M_dev ? sms : gemm_grid(M, f, tile_n, sms);
+  if (gated) {
+    TW_TRY(launch_gemm<kModeGateUp>(ma, mg, mu, p1, g1, s));
+  } else {
+    TW_TRY(launch_gemm<kModeRelu>(ma, mg, mg, p1, g1, s));
+  }
   GemmParams p2{};
   p2.M = M;
   p2.M_dev = M_dev;
@@ -303,13 +310,15 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
     p2.k_splits_max = 32;
   }
   p2.dev_status = dev_status;
-  const int g2 = M_dev ? sms : gemm_grid(M, d, kBN, sms);
+  // a split K needs the whole grid: the kernel derives the splits from it
+  const int g2 = (M_dev != nullptr || p2.k_splits_max > 1) ? sms : gemm_grid(M, d, kBN, sms);
   return launch_gemm<kModeDown>(mh, md, md, p2, g2, s);
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Dense branch: gather x[rows[i]] into xo, dense gated FFN into ho, scatter to y.
+// Dense branch: gather x[rows[i]] into xo, dense FFN (gated, or non-gated when WuT is
+// null) into ho, scatter to y.
 twell_status dense_rows_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
                              int T, int d, int f, const int32_t* rows, const int32_t* n_rows, float* y,
                              uint16_t* xo, uint16_t* ho, int32_t* dev_status, cudaStream_t s, int sms) {
@@ -479,6 +488,63 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
   return dense_impl(x, T, nullptr, WgT, WuT, Wd, d, f, static_cast<uint16_t*>(workspace), false, nullptr, y, T,
+                    dev_status, static_cast<cudaStream_t>(stream), sms);
+}
+
+twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2, int T, int d,
+                                           int f, const twell_t* tw, float* y, int32_t* ovf_rows, int32_t* n_ovf,
+                                           void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                           void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, W1T, W2, y, ovf_rows, n_ovf, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_hybrid_workspace_bytes(T, d, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* xo = static_cast<uint16_t*>(workspace);
+  uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                             round_up(static_cast<size_t>(T) * d * 2, 256));
+  // The pack of ReLU(x W1) holds the hidden activations themselves, so the
+  // sparse step is the down projection alone.
+  TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms));
+  route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  TW_TRY(down_impl(W2, T, d, f, tw, 1, y, dev_status, s, sms));
+  return dense_rows_impl(x, W1T, nullptr, W2, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
+}
+
+twell_status twell_relu_dense_rows_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2, int T, int d,
+                                          int f, const int32_t* rows, const int32_t* n_rows, float* y,
+                                          void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                          void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, W1T, W2, rows, n_rows, y, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_hybrid_workspace_bytes(T, d, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  uint16_t* xo = static_cast<uint16_t*>(workspace);
+  uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                             round_up(static_cast<size_t>(T) * d * 2, 256));
+  return dense_rows_impl(x, W1T, nullptr, W2, T, d, f, rows, n_rows, y, xo, ho, dev_status,
+                         static_cast<cudaStream_t>(stream), sms);
+}
+
+twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2, int T, int d,
+                                          int f, float* y, void* workspace, size_t workspace_bytes,
+                                          int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, W1T, W2, y, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_dense_workspace_bytes(T, d, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return dense_impl(x, T, nullptr, W1T, nullptr, W2, d, f, static_cast<uint16_t*>(workspace), false, nullptr, y, T,
                     dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 

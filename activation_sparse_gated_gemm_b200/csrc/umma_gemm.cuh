@@ -18,6 +18,9 @@
 //                  positions where z > 0 into TwELL exactly as kModeTwell does,
 //                  but stores h = z * u there instead of z (the up projection
 //                  then runs on the tensor cores, densely).
+//   kModeRelu   -- h = ReLU(x . W1) stored as bf16 (and optionally the bf16
+//                  remainder, as in kModeGateUp): the first half of the dense
+//                  non-gated layer.
 //   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
 //                  epilogue stores fp32 rows, optionally scattered through a
 //                  row map (the dense branch of the hybrid route). With the
@@ -26,17 +29,18 @@
 //
 // Structure: one CTA per SM walks output tiles of 128 x 256 (x 128 h-columns
 // for kModeGateUp). Warp 0 issues TMA loads into a 4-stage shared-memory ring,
-// warp 1 issues tcgen05.mma (M=128, N=256, K=16) into one of two 256-column
-// TMEM accumulators, warps 2-5 drain the other accumulator with tcgen05.ld, so
-// the epilogue of tile i overlaps the MMAs of tile i+1. No cluster, no
-// multicast: every CTA loads its own operand tiles.
+// warp 1 issues tcgen05.mma (M=128, N=256, K=16) into two 256-column TMEM
+// accumulators in turn, and each accumulator has its own group of four
+// epilogue warps (2-5 and 6-9) that drains it with tcgen05.ld, so the
+// epilogues of tiles i and i+1 overlap each other and the MMAs of tile i+2.
+// No cluster, no multicast: every CTA loads its own operand tiles.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace twell {
 
-enum GemmMode : int { kModeTwell = 0, kModeGateUp = 1, kModeDown = 2, kModeTwellHidden = 3 };
+enum GemmMode : int { kModeTwell = 0, kModeGateUp = 1, kModeDown = 2, kModeTwellHidden = 3, kModeRelu = 4 };
 
 constexpr int kBM = 128;
 constexpr int kBN = 256;
@@ -44,9 +48,11 @@ constexpr int kBK = 64;  // 64 bf16 = 128 bytes = one 128-byte swizzle row
 constexpr int kStages = 4;
 constexpr int kAStageBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBStageBytes = kBN * kBK * 2;  // 32 KB
-constexpr int kEpiPitch = 33;                // floats per row of the epilogue transpose buffer
-constexpr int kEpiBytes = 4 * 32 * kEpiPitch * 4;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;                 // two groups of four, one per TMEM accumulator
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kEpiPitch = 17;                // 32-bit words per row of the bf16 value buffer (16 pairs + pad)
+constexpr int kEpiBytes = kEpiWarps * 32 * kEpiPitch * 4;
+constexpr int kGemmThreads = 64 + kEpiThreads;
 constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
 
 constexpr int kStageSlotBytes = 32;  // per epilogue thread: 8 staged (idx, value) slots
@@ -54,10 +60,11 @@ constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kAStageBytes;
 constexpr int kOffEpi = kOffB + kStages * kBStageBytes;
 constexpr int kOffSlots = kOffEpi + kEpiBytes;
-constexpr int kOffBar = kOffSlots + 128 * kStageSlotBytes;
+constexpr int kOffBar = kOffSlots + kEpiThreads * kStageSlotBytes;
 constexpr int kNumBars = 2 * kStages + 4 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kGemmSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
+static_assert(kGemmSmemBytes <= 232448, "GEMM shared memory exceeds the 227 KB per-CTA limit");
 
 struct GemmParams {
   int M;             // rows of A (an upper bound when M_dev is set)
@@ -71,13 +78,13 @@ struct GemmParams {
   uint8_t* row_ovf;
   int nT;
   int W;
-  // kModeGateUp output (bf16) / kModeDown output (fp32), leading dimension ldo
+  // kModeGateUp / kModeRelu output (bf16) / kModeDown output (fp32), leading dimension ldo
   uint16_t* out;
   float* out_f32;
   int ldo;
   const int* row_map;  // kModeDown: output row of each A row, or null
   int out_rows;        // valid range of output rows
-  // kModeGateUp: also store h_lo = bf16(h - bf16(h)) at column N + c (ldo = 2N).
+  // kModeGateUp / kModeRelu: also store h_lo = bf16(h - bf16(h)) at column N + c (ldo = 2N).
   int h_split;
   // kModeDown: B rows are read at k mod k_wrap (k_wrap > 0), so K = 2 * k_wrap
   // runs [h_hi | h_lo] against [Wd ; Wd].
@@ -90,10 +97,10 @@ struct GemmParams {
 };
 
 
-// Appends the set bits of `mask` (column col0 + i, value vrow[i]) to one row's
-// slot list of a TwELL tile in ascending column order, staging 8 slots at a
-// time in shared memory and storing each full group with 16-byte stores.
-__device__ __forceinline__ void twell_append(uint32_t mask, const float* vrow, int col0, int& cnt, int W,
+// Appends the set bits of `mask` (column col0 + i, bf16 value vrow[i]) to one
+// row's slot list of a TwELL tile in ascending column order, staging 8 slots
+// at a time in shared memory and storing each full group with 16-byte stores.
+__device__ __forceinline__ void twell_append(uint32_t mask, const uint16_t* vrow, int col0, int& cnt, int W,
                                              uint16_t* stg_idx, uint16_t* stg_val, int16_t* gidx,
                                              uint16_t* gval) {
   while (mask != 0) {
@@ -102,7 +109,7 @@ __device__ __forceinline__ void twell_append(uint32_t mask, const float* vrow, i
     if (cnt < W) {
       const int k = cnt & 7;
       stg_idx[k] = static_cast<uint16_t>(col0 + i);
-      stg_val[k] = f32_to_bf16_bits(vrow[i]);
+      stg_val[k] = vrow[i];
       if (k == 7) {
         *reinterpret_cast<uint4*>(gidx + (cnt - 7)) = *reinterpret_cast<const uint4*>(stg_idx);
         *reinterpret_cast<uint4*>(gval + (cnt - 7)) = *reinterpret_cast<const uint4*>(stg_val);
@@ -123,6 +130,25 @@ __device__ __forceinline__ void twell_close(int cnt, int W, uint16_t* stg_idx, u
     }
     *reinterpret_cast<uint4*>(gidx + (n & ~7)) = *reinterpret_cast<const uint4*>(stg_idx);
     *reinterpret_cast<uint4*>(gval + (n & ~7)) = *reinterpret_cast<const uint4*>(stg_val);
+  }
+}
+
+// Stores 32 hidden values of one row as bf16 at row_out[col ..], and with
+// `split` the remainder h - bf16(h), itself rounded to bf16, at row_out[N + col ..].
+__device__ __forceinline__ void store_h32(const float (&h)[32], uint16_t* row_out, int col, int N, bool split) {
+  uint32_t hv[16], lv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    hv[i] = pack_bf16x2(h[2 * i], h[2 * i + 1]);
+    lv[i] = pack_bf16x2(h[2 * i] - __uint_as_float(hv[i] << 16), h[2 * i + 1] - __uint_as_float(hv[i] & 0xffff0000u));
+  }
+  uint4* dst = reinterpret_cast<uint4*>(row_out + col);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2], hv[4 * v + 3]);
+  if (split) {
+    uint4* dlo = reinterpret_cast<uint4*>(row_out + N + col);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) dlo[v] = make_uint4(lv[4 * v], lv[4 * v + 1], lv[4 * v + 2], lv[4 * v + 3]);
   }
 }
 
@@ -160,6 +186,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     k_splits = (num_kb + kb_per - 1) / kb_per;
   }
   const int num_tiles = num_m * num_n * k_splits;
+  // A CTA without a tile leaves before any setup (uniform for the whole CTA).
+  if (static_cast<int>(blockIdx.x) >= num_tiles) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -207,7 +235,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* b_dst = smem + kOffB + s * kBStageBytes;
           mbar_arrive_expect_tx(&full[s], kAStageBytes + kBStageBytes);
           tma_load_2d(a_dst, &tmA, &full[s], kb * kBK, m_blk * kBM);
-          if (MODE == kModeTwell) {
+          if (MODE == kModeTwell || MODE == kModeRelu) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * kBN);
           } else if (kStacked) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * 128);
@@ -301,12 +329,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    // Two groups of four warps: group g drains accumulator g, i.e. every other
+    // tile of this CTA, so two tiles' epilogues run side by side while the
+    // MMAs of the next tile proceed.
     const int q = warp & 3;  // TMEM lanes 32q..32q+31 are reachable from this warp
-    float* ebuf = reinterpret_cast<float*>(smem + kOffEpi) + (warp - 2) * 32 * kEpiPitch;
-    int buf = 0;
+    const int buf = (warp - 2) >> 2;
+    uint32_t* ebuf = reinterpret_cast<uint32_t*>(smem + kOffEpi) + (warp - 2) * 32 * kEpiPitch;
     uint32_t tph = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x + buf * gridDim.x; tile < num_tiles; tile += 2 * gridDim.x) {
       const bool got = mbar_wait(&tfull[buf], tph, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         *abort_flag = 1;
@@ -327,7 +358,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // bits in ascending column order, appending (column, bf16 value) to its
         // row's slot list. Slots go through an 8-entry staging buffer in shared
         // memory and leave as 16-byte stores.
-        float* vrow = ebuf + lane * kEpiPitch;
+        uint32_t* vrow = ebuf + lane * kEpiPitch;
         uint8_t* stg = smem + kOffSlots + (threadIdx.x - 64) * kStageSlotBytes;
         uint16_t* stg_idx = reinterpret_cast<uint16_t*>(stg);
         uint16_t* stg_val = reinterpret_cast<uint16_t*>(stg + 16);
@@ -354,9 +385,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i < 32; ++i) mask |= (static_cast<int32_t>(r[i]) > 0 ? 1u : 0u) << i;
             if (mask == 0) continue;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) vrow[i] = __uint_as_float(r[i]);
-            twell_append(mask, vrow, c * 128 + ch * 32, cnt, p.W, stg_idx, stg_val, p.idx + slot0,
-                         p.vals + slot0);
+            for (int i = 0; i < 16; ++i) vrow[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            twell_append(mask, reinterpret_cast<const uint16_t*>(vrow), c * 128 + ch * 32, cnt, p.W, stg_idx,
+                         stg_val, p.idx + slot0, p.vals + slot0);
           }
           if (tile_ok) {
             twell_close(cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
@@ -367,7 +398,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else if (MODE == kModeTwellHidden) {
         // Same pattern as above from z (columns 0..127 of the accumulator),
         // value h = z * u with u in columns 128..255.
-        float* vrow = ebuf + lane * kEpiPitch;
+        uint32_t* vrow = ebuf + lane * kEpiPitch;
         uint8_t* stg = smem + kOffSlots + (threadIdx.x - 64) * kStageSlotBytes;
         uint16_t* stg_idx = reinterpret_cast<uint16_t*>(stg);
         uint16_t* stg_val = reinterpret_cast<uint16_t*>(stg + 16);
@@ -392,8 +423,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int i = 0; i < 32; ++i) mask |= (static_cast<int32_t>(zr[i]) > 0 ? 1u : 0u) << i;
           if (mask == 0) continue;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) vrow[i] = __uint_as_float(zr[i]) * __uint_as_float(ur[i]);
-          twell_append(mask, vrow, c * 128 + ch * 32, cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
+          for (int i = 0; i < 16; ++i)
+            vrow[i] = pack_bf16x2(__uint_as_float(zr[2 * i]) * __uint_as_float(ur[2 * i]),
+                                  __uint_as_float(zr[2 * i + 1]) * __uint_as_float(ur[2 * i + 1]));
+          twell_append(mask, reinterpret_cast<const uint16_t*>(vrow), c * 128 + ch * 32, cnt, p.W, stg_idx,
+                       stg_val, p.idx + slot0, p.vals + slot0);
         }
         if (tile_ok) {
           twell_close(cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
@@ -414,23 +448,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int col = n_blk * 128 + ch * 32;
           if (my_row < M && col < p.N) {
-            uint32_t hv[16], lv[16];
+            float h[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = fmaxf(__uint_as_float(zr[2 * i]), 0.0f) * __uint_as_float(ur[2 * i]);
-              const float h1 = fmaxf(__uint_as_float(zr[2 * i + 1]), 0.0f) * __uint_as_float(ur[2 * i + 1]);
-              hv[i] = pack_bf16x2(h0, h1);
-              // remainder of the bf16 rounding, itself rounded to bf16
-              lv[i] = pack_bf16x2(h0 - __uint_as_float(hv[i] << 16), h1 - __uint_as_float(hv[i] & 0xffff0000u));
-            }
-            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(my_row) * p.ldo + col);
+            for (int i = 0; i < 32; ++i) h[i] = fmaxf(__uint_as_float(zr[i]), 0.0f) * __uint_as_float(ur[i]);
+            store_h32(h, p.out + static_cast<size_t>(my_row) * p.ldo, col, p.N, p.h_split != 0);
+          }
+        }
+      } else if (MODE == kModeRelu) {
+#pragma unroll 1
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), r);
+          tmem_wait_ld();
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int col = n_blk * kBN + ch * 32;
+          if (my_row < M && col < p.N) {
+            float h[32];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2], hv[4 * v + 3]);
-            if (p.h_split) {
-              uint4* dlo = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(my_row) * p.ldo + p.N + col);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) dlo[v] = make_uint4(lv[4 * v], lv[4 * v + 1], lv[4 * v + 2], lv[4 * v + 3]);
-            }
+            for (int i = 0; i < 32; ++i) h[i] = fmaxf(__uint_as_float(r[i]), 0.0f);
+            store_h32(h, p.out + static_cast<size_t>(my_row) * p.ldo, col, p.N, p.h_split != 0);
           }
         }
       } else {
@@ -469,10 +509,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (++buf == 2) {
-        buf = 0;
-        tph ^= 1u;
-      }
+      tph ^= 1u;
     }
   }
 

@@ -30,6 +30,7 @@ EXPORTED = (
     "twell_dense_ffn_forward", "twell_unpack", "twell_status_reset", "twell_status_get",
     "twell_status_str", "twell_version", "twell_ffn_hybrid_forward_noalloc",
     "twell_gate_up_pack", "twell_sparse_down", "twell_ffn_hybrid_forward_tc_up",
+    "twell_relu_ffn_hybrid_forward", "twell_relu_dense_rows_forward", "twell_relu_dense_ffn_forward",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -80,6 +81,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_ffn_hybrid_forward": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_dense_workspace_bytes": ([i32, i32, i32], sz),
         "twell_dense_ffn_forward": ([vp, vp, vp, vp, i32, i32, i32, vp, vp, sz, vp, vp], i32),
+        "twell_relu_ffn_hybrid_forward": ([vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
+        "twell_relu_dense_rows_forward": ([vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp], i32),
+        "twell_relu_dense_ffn_forward": ([vp, vp, vp, i32, i32, i32, vp, vp, sz, vp, vp], i32),
         "twell_unpack": ([tw, vp, vp, vp], i32),
         "twell_ffn_hybrid_forward_noalloc": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp], i32),
         "twell_status_reset": ([vp, vp], i32),
@@ -275,6 +279,38 @@ def dense_ffn_forward(x, WgT, WuT, Wd, y, workspace, dev_status, stream=None) ->
         _bf16(n, t, s)
     _check("twell_dense_ffn_forward", load().twell_dense_ffn_forward(
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), T, d, f, _ptr(y), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def relu_ffn_hybrid_forward(x, W1T, W2, tw: Twell, y, ovf_rows, n_ovf, workspace, dev_status,
+                            stream=None) -> None:
+    """Non-gated layer y = ReLU(x W1) W2, hybrid forward (W1T = W1 transposed, [f, d])."""
+    T, d = x.shape
+    f = W1T.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("W1T", W1T, (f, d)), ("W2", W2, (f, d)), ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_relu_ffn_hybrid_forward", load().twell_relu_ffn_hybrid_forward(
+        _ptr(x), _ptr(W1T), _ptr(W2), T, d, f, tw.ref(), _ptr(y), _ptr(ovf_rows), _ptr(n_ovf),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def relu_dense_rows_forward(x, W1T, W2, rows, n_rows, y, workspace, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = W1T.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("W1T", W1T, (f, d)), ("W2", W2, (f, d)), ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_relu_dense_rows_forward", load().twell_relu_dense_rows_forward(
+        _ptr(x), _ptr(W1T), _ptr(W2), T, d, f, _ptr(rows), _ptr(n_rows), _ptr(y),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def relu_dense_ffn_forward(x, W1T, W2, y, workspace, dev_status, stream=None) -> None:
+    T, d = x.shape
+    f = W1T.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("W1T", W1T, (f, d)), ("W2", W2, (f, d)), ("y", y, (T, d))):
+        _bf16(n, t, s)
+    _check("twell_relu_dense_ffn_forward", load().twell_relu_dense_ffn_forward(
+        _ptr(x), _ptr(W1T), _ptr(W2), T, d, f, _ptr(y), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
 
 

@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 from activation_sparse_gated_gemm_b200 import synth  # noqa: E402
 
 METRIC = "sparse gated-FFN tokens/s"
+METRIC_RELU = "sparse non-gated ReLU-FFN tokens/s"
 FLUSH_BYTES = 256 << 20
 FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM (4 sub-partitions x 32)
 DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
@@ -205,38 +206,47 @@ def blas_threads() -> int:
 # ---------------------------------------------------------------- CPU oracle
 
 
-def cpu_oracle_rate(cfg, L, sample_rows: int, max_seconds: float = 25.0) -> dict:
-    """The oracle as it stands (hybrid forward: fp64 gate, pack, route,
-    per-token sparse step, dense rows) on the first rows of the workload."""
+def oracle_step(cfg, L, rows, layer: str) -> None:
+    """One hybrid forward of the oracle as it stands on the given rows."""
     from oracle import twell_oracle as O
 
+    if layer == "relu":
+        O.hybrid_relu_ffn(L["x"][rows], L["WgT"], L["Wd"], cfg.tile, cfg.W)
+    else:
+        O.hybrid_ffn(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], cfg.tile, cfg.W)
+
+
+def cpu_oracle_rate(cfg, L, sample_rows: int, layer: str = "gated", max_seconds: float = 25.0) -> dict:
+    """The oracle as it stands (hybrid forward: fp64 gate, pack, route,
+    per-token sparse step, dense rows) on the first rows of the workload."""
     n = min(sample_rows, cfg.T)
     done, t0 = 0, time.perf_counter()
     while done < n and time.perf_counter() - t0 < max_seconds:
         chunk = min(128, n - done)
-        rows = slice(done, done + chunk)
-        O.hybrid_ffn(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], cfg.tile, cfg.W)
+        oracle_step(cfg, L, slice(done, done + chunk), layer)
         done += chunk
     dt = time.perf_counter() - t0
     return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {done} of {cfg.T} tokens of the {cfg.name} layer, fp64 numpy oracle "
+            "sample": f"first {done} of {cfg.T} tokens of the {cfg.name} {layer} layer, fp64 numpy oracle "
                       f"(gate, pack, route, sparse step, dense rows), {dt:.1f} s"}
 
 
 # ---------------------------------------------------------------- GPU arm
 
 
-def algorithmic(cfg, n_ovf: int, nnz_stored: int, union_cols: int) -> dict:
+def algorithmic(cfg, n_ovf: int, nnz_stored: int, union_cols: int, layer: str = "gated") -> dict:
     T, d, f = cfg.T, cfg.d, cfg.f
     nT = f // cfg.tile
+    mats = 2 if layer == "relu" else 3         # weight matrices of the layer
     gate_flops = 2.0 * T * d * f
-    dense_branch_flops = 6.0 * n_ovf * d * f
-    alg_bytes = (2.0 * d * f                  # Wg
-                 + 4.0 * d * union_cols       # active Wu columns and Wd rows
+    dense_branch_flops = 2.0 * mats * n_ovf * d * f
+    alg_bytes = (2.0 * d * f                  # Wg (W1)
+                 + 2.0 * (mats - 1) * d * union_cols  # active Wu columns and Wd rows (W2 rows)
                  + 6.0 * T * d                # x read (bf16), y written (fp32)
                  + 2 * 4.0 * nnz_stored       # TwELL nonzeros written and read (2 B idx + 2 B value)
                  + 2 * 2.0 * T * nT)          # counts written and read
-    sparse_flops = 4.0 * d * nnz_stored       # up and down for every stored slot (non-overflow rows)
+    # up and down for every stored slot (non-overflow rows); down only without the up matrix
+    sparse_flops = 2.0 * (mats - 1) * d * nnz_stored
     return {"gate_flops": gate_flops, "dense_branch_flops": dense_branch_flops, "alg_bytes": alg_bytes,
             "sparse_flops": sparse_flops}
 
@@ -270,6 +280,10 @@ def run_gpu(args, world, rank, local):
     # fused sparse up+down step; "tc_up" forms u on the tensor cores with the
     # gate and packs h, leaving only the down projection sparse.
     def stage_fns(variant):
+        if variant == "relu":  # the non-gated layer ReLU(x W1) W2 with W1 = Wg, W2 = Wd
+            return [lambda: tl.gate_pack(x, WgT, tw, st), lambda: tl.route(tw, ovf_rows, n_ovf),
+                    lambda: tl.sparse_down(Wd, tw, y, True, st),
+                    lambda: tl.relu_dense_rows_forward(x, WgT, Wd, ovf_rows, n_ovf, y, ws, st)]
         pack = ((lambda: tl.gate_pack(x, WgT, tw, st)) if variant == "gate"
                 else (lambda: tl.gate_up_pack(x, WgT, WuT, tw, st)))
         sparse = ((lambda: tl.sparse_ffn(x, WuT, Wd, tw, y, True, st)) if variant == "gate"
@@ -303,7 +317,11 @@ def run_gpu(args, world, rank, local):
         per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)] for k in range(K)])
         return max_over_ranks(float(per.sum(axis=1).mean()), world), per.mean(axis=0)
 
-    variants = ["gate", "tc_up"] if args.variant == "auto" else [args.variant]
+    layer = "relu" if args.layer == "relu" else "gated"
+    if layer == "relu":
+        variants = ["relu"]
+    else:
+        variants = ["gate", "tc_up"] if args.variant == "auto" else [args.variant]
     results = {v: run_variant(v) for v in variants} if len(variants) > 1 else {}
     chosen = min(results, key=lambda v: results[v][0]) if results else variants[0]
     # the reported measurement: the chosen form, timed again with the clocks sampled
@@ -326,15 +344,21 @@ def run_gpu(args, world, rank, local):
     del g
 
     # dense baseline at the same shape
+    def dense():
+        if layer == "relu":
+            tl.relu_dense_ffn_forward(x, WgT, Wd, y_dense, ws_dense, st)
+        else:
+            tl.dense_ffn_forward(x, WgT, WuT, Wd, y_dense, ws_dense, st)
+
     for _ in range(Wm):
         flush.zero_()
-        tl.dense_ffn_forward(x, WgT, WuT, Wd, y_dense, ws_dense, st)
+        dense()
     dense_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     barrier(world)
     for k in range(K):
         flush.zero_()
         dense_ev[k][0].record(stream)
-        tl.dense_ffn_forward(x, WgT, WuT, Wd, y_dense, ws_dense, st)
+        dense()
         dense_ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
     dense_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dense_ev])), world)
@@ -342,7 +366,11 @@ def run_gpu(args, world, rank, local):
     # end to end through the C ABI with host buffers
     x_host = x.cpu().pin_memory()
     y_host = torch.empty((T, d), dtype=torch.float32).pin_memory()
-    hybrid = tl.ffn_hybrid_forward if chosen == "gate" else tl.ffn_hybrid_forward_tc_up
+    if layer == "relu":
+        def hybrid(x, WgT, WuT, Wd, *rest):
+            tl.relu_ffn_hybrid_forward(x, WgT, Wd, *rest)
+    else:
+        hybrid = tl.ffn_hybrid_forward if chosen == "gate" else tl.ffn_hybrid_forward_tc_up
     for _ in range(max(1, Wm // 2)):
         x.copy_(x_host, non_blocking=True)
         hybrid(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st)
@@ -364,7 +392,7 @@ def run_gpu(args, world, rank, local):
         raise RuntimeError(f"device status {status} ({tl.status_str(status)})")
 
     peaks = load_peaks()
-    alg = algorithmic(cfg, n_ovf_h, nnz_stored, union_cols)
+    alg = algorithmic(cfg, n_ovf_h, nnz_stored, union_cols, layer)
     hbm = peaks["hbm_gbs"] * 1e9
     tc = peaks["bf16_tflops"] * 1e12
     t_tc = (alg["gate_flops"] + alg["dense_branch_flops"]) / tc
@@ -374,7 +402,10 @@ def run_gpu(args, world, rank, local):
     fp32_peak = (torch.cuda.get_device_properties(dev).multi_processor_count * FP32_LANES_PER_SM * 2
                  * (clocks["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6)
 
-    if chosen == "gate":
+    if chosen == "relu":
+        names = ["gate_pack", "route", "sparse_down", "dense_rows"]
+        pack_flops, sparse_flops = alg["gate_flops"], alg["sparse_flops"]
+    elif chosen == "gate":
         names = ["gate_pack", "route", "sparse_ffn", "dense_rows"]
         pack_flops, sparse_flops = alg["gate_flops"], alg["sparse_flops"]
     else:
@@ -394,7 +425,7 @@ def run_gpu(args, world, rank, local):
     traffic = measured_traffic(dom, cfg.name)
 
     res = {
-        "metric": METRIC,
+        "metric": METRIC_RELU if layer == "relu" else METRIC,
         "value": job_rate(T, world, step_ms),
         "unit": "tokens/s",
         "n_gpus": world,
@@ -406,7 +437,9 @@ def run_gpu(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded generator; no dataset or trained weights)",
-        "config": {"workload": f"{cfg.name}-like FFN layer forward, hybrid TwELL", "variant": chosen,
+        "config": {"workload": (f"{cfg.name}-like non-gated ReLU FFN layer forward (W1 = Wg, W2 = Wd), "
+                                "hybrid TwELL" if layer == "relu" else
+                                f"{cfg.name}-like FFN layer forward, hybrid TwELL"), "variant": chosen,
                    "tokens": T, "d": d,
                    "f": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
                    "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
@@ -431,7 +464,7 @@ def run_gpu(args, world, rank, local):
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_oracle_rate(cfg, L, args.cpu_sample)
+        res["cpu_baseline"] = cpu_oracle_rate(cfg, L, args.cpu_sample, layer)
     return res
 
 
@@ -446,10 +479,10 @@ def run_reference(args, world, rank):
     cfg = synth.CONFIGS[args.config]
     L = synth.make_layer(cfg, seed=args.seed)
     sample = max(1, min(cfg.T, args.cpu_sample // 16))
-    from oracle import twell_oracle as O
+    layer = "relu" if args.layer == "relu" else "gated"
 
     def step():
-        O.hybrid_ffn(L["x"][:sample], L["WgT"], L["WuT"], L["Wd"], cfg.tile, cfg.W)
+        oracle_step(cfg, L, slice(0, sample), layer)
 
     for _ in range(args.warmup):
         step()
@@ -460,10 +493,13 @@ def run_reference(args, world, rank):
     v = sample / dt
     return {
         "impl": "reference",
-        "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_RELU if layer == "relu" else METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
-        "config": {"workload": f"{cfg.name}-like FFN layer forward, hybrid TwELL", "tokens": cfg.T,
+        "config": {"workload": (f"{cfg.name}-like non-gated ReLU FFN layer forward (W1 = Wg, W2 = Wd), "
+                                "hybrid TwELL" if layer == "relu" else
+                                f"{cfg.name}-like FFN layer forward, hybrid TwELL"), "tokens": cfg.T,
                    "d": cfg.d, "f": cfg.f, "tile": cfg.tile, "ell_width": cfg.W,
                    "density": cfg.density, "dead_frac": cfg.dead_frac},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
@@ -499,18 +535,33 @@ def run_sweep(args) -> None:
             st = tl.new_status(dev)
 
             def timed(fn, k):
-                ts = []
+                """Median device time of fn; replayed from a CUDA graph when the
+                calls capture (they are stream-ordered and never sync), so
+                small batches are not measured as launch gaps."""
                 for _ in range(args.warmup):
                     flush.zero_()
                     fn()
+                torch.cuda.synchronize(dev)
+                run = fn
+                if not args.sweep_eager:
+                    try:
+                        graph = torch.cuda.CUDAGraph()
+                        with torch.cuda.graph(graph):
+                            fn()
+                        run = graph.replay
+                    except Exception:  # noqa: BLE001 -- measured eagerly instead
+                        torch.cuda.synchronize(dev)
+                        run = fn
+                ts = []
                 for _ in range(k):
                     flush.zero_()
                     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     a.record()
-                    fn()
+                    run()
                     b.record()
                     torch.cuda.synchronize(dev)
                     ts.append(a.elapsed_time(b))
+                timed.graph = run is not fn
                 return float(np.median(ts))
 
             ms_gate = timed(lambda: tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st),
@@ -535,7 +586,8 @@ def run_sweep(args) -> None:
                               "tokens_per_s": T / (ms * 1e-3), "dense_ms": ms_dense,
                               "speedup_vs_own_dense": ms_dense / ms, "roofline_frac": t_roof / (ms * 1e-3),
                               "t_roof_us": t_roof * 1e6, "n_ovf": n_o,
-                              "measured_density": float(counts.sum()) / (T * cfg.f), "status": status}),
+                              "measured_density": float(counts.sum()) / (T * cfg.f), "status": status,
+                              "cuda_graph": bool(getattr(timed, "graph", False))}),
                   flush=True)
             del x, WgT, WuT, Wd, tw, y, ws, wsd
             torch.cuda.empty_cache()
@@ -553,9 +605,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", default="auto", choices=["auto", "gate", "tc_up"],
                     help="hybrid form: gate (sparse up+down) or tc_up (up on tensor cores); auto times both")
+    ap.add_argument("--layer", default="gated", choices=["gated", "relu"],
+                    help="gated: (ReLU(x Wg) * x Wu) Wd; relu: the non-gated ReLU(x W1) W2")
     ap.add_argument("--sweep", action="store_true", help="density x batch sweep, one JSON line per point")
     ap.add_argument("--sweep-T", default="", help="comma-separated token counts (default: the full sweep)")
     ap.add_argument("--sweep-p", default="", help="comma-separated densities (default: the full sweep)")
+    ap.add_argument("--sweep-eager", action="store_true", help="time sweep points without CUDA graphs")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -235,6 +235,48 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
                                      int32_t* dev_status, void* stream);
 
 /*
+ * Non-gated ReLU FFN, y = ReLU(x W1) W2, hybrid forward. The pages note the
+ * method also applies to the non-gated layer, with a smaller gain
+ * (intellectnews.ru, "Sakana AI и NVIDIA: TwELL ...", section "Ограничения и
+ * открытые вопросы").
+ *   x [T][d] bf16, W1T [f][d] bf16 (W1 transposed), W2 [f][d] bf16 (row j is
+ *   hidden unit j's output vector), y [T][d] fp32: all device pointers,
+ *   caller-owned, 16-byte aligned. Shapes and the TwELL buffers as for
+ *   twell_ffn_hybrid_forward; workspace of twell_hybrid_workspace_bytes(T, d, f).
+ * Steps: the pack of ReLU(x W1) (its stored values are the hidden activations
+ * themselves), routing, the sparse down projection over the stored slots for
+ * rows that fit, and the dense layer on the tensor cores for overflow rows
+ * (hidden values kept as bf16 plus bf16 remainder, as in the gated dense
+ * branch). Errors as for twell_ffn_hybrid_forward.
+ */
+twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2,
+                                           int T, int d, int f, const twell_t* tw, float* y,
+                                           int32_t* ovf_rows, int32_t* n_ovf, void* workspace,
+                                           size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * The dense branch of twell_relu_ffn_hybrid_forward on its own: for i <
+ * *n_rows, y[rows[i]] = ReLU(x[rows[i]] W1) W2 (rows and n_rows device
+ * int32, as twell_route writes them; rows outside [0, T) raise
+ * TWELL_ERR_INDEX and are skipped). Workspace and errors as for
+ * twell_dense_rows_forward.
+ */
+twell_status twell_relu_dense_rows_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2,
+                                          int T, int d, int f, const int32_t* rows, const int32_t* n_rows,
+                                          float* y, void* workspace, size_t workspace_bytes,
+                                          int32_t* dev_status, void* stream);
+
+/*
+ * Dense non-gated ReLU FFN on the tensor cores (h = ReLU(x W1) stored once as
+ * bf16 in a workspace of twell_dense_workspace_bytes(T, d, f), then h W2): the
+ * library's own baseline for the non-gated layer; error bound as for
+ * twell_dense_ffn_forward.
+ */
+twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2,
+                                          int T, int d, int f, float* y, void* workspace,
+                                          size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * TwELL -> dense bf16 g[T][f]: zeros everywhere except the stored slots
  * (slots below min(count, W); overflowing rows unpack only what was stored).
  */
