@@ -52,6 +52,8 @@ __all__ = [
     "hybrid_ffn_up_dense",
     "relu_ffn",
     "hybrid_relu_ffn",
+    "column_activity",
+    "compact_layer",
 ]
 
 
@@ -286,3 +288,39 @@ def hybrid_relu_ffn(x_bits, W1T_bits, W2_bits, tile: int, W: int) -> dict:
     if ovf.size:
         y[ovf] = relu_ffn(np.asarray(x_bits)[ovf], W1T_bits, W2_bits)
     return {"y": y, "twell": tw, "ovf_rows": ovf}
+
+
+# ---------------------------------------------------------------------------
+# Dead-column compaction [P1, "Ограничения и открытые вопросы": under the
+# chosen L1 setting some hidden units die, i.e. are never active]. A profile
+# marks the hidden units that are active for at least one token; the others
+# are dropped from Wg, Wu and Wd. The kept units keep their order, and the
+# compacted width is padded up to a whole number of tiles with all-zero rows,
+# whose gate pre-activation is exactly 0 and so never active.
+
+
+def column_activity(z: np.ndarray) -> np.ndarray:
+    """active[j] = True iff z[t, j] > 0 for some row t (strictly positive)."""
+    return np.any(np.asarray(z) > 0, axis=0)
+
+
+def compact_layer(WgT_bits, WuT_bits, Wd_bits, active: np.ndarray, tile: int) -> dict:
+    """Keep the rows j of WgT, WuT and Wd with active[j], in ascending j.
+    Returns the compacted matrices ([f_c, d], f_c = the kept count rounded up
+    to a multiple of tile, at least one tile; padding rows are zero), col_map
+    (original index of each compacted row, -1 for padding) and f_live."""
+    live = np.nonzero(np.asarray(active))[0]
+    f_live = int(live.size)
+    f_c = max(tile, -(-f_live // tile) * tile)
+    out = {"f_live": f_live, "f_c": f_c}
+    col_map = np.full(f_c, -1, dtype=np.int32)
+    col_map[:f_live] = live
+    out["col_map"] = col_map
+    for name, m in (("WgT", WgT_bits), ("WuT", WuT_bits), ("Wd", Wd_bits)):
+        if m is None:
+            continue
+        m = np.asarray(m)
+        c = np.zeros((f_c, m.shape[1]), dtype=m.dtype)
+        c[:f_live] = m[live]
+        out[name] = c
+    return out

@@ -516,3 +516,65 @@ def test_relu_hybrid_within_one_rounding_of_dense_and_special_cases():
     got = O.hybrid_relu_ffn(L["x"], bits_of_exact(neg), L["Wd"], HEAVY.tile, HEAVY.W)["y"]
     want = O.bf16_bits_to_f64(O.f64_to_bf16_bits(zj))[:, None] * w2[js][None, :]
     np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Dead-column compaction
+
+
+def test_column_activity_bruteforce():
+    rng = np.random.default_rng(31)
+    z = rng.integers(-3, 2, size=(7, 300)).astype(np.float64)
+    z[:, 5] = 0.0  # zero is not active
+    z[3, 6] = 0.5  # one token suffices
+    want = np.array([any(z[t, j] > 0 for t in range(z.shape[0])) for j in range(z.shape[1])])
+    got = O.column_activity(z)
+    assert np.array_equal(got, want)
+    assert not got[5] and got[6]
+
+
+def test_compaction_keeps_the_layer_on_the_profile_batch():
+    """Dropping units that are never active on a batch changes nothing on that
+    batch: y (gated and non-gated) is the same up to fp64 rounding, and the
+    packs agree as sets of (row, original column, value)."""
+    cfg = synth.LayerConfig("dead", T=96, d=128, f=1024, tile=128, W=128, density=0.05, sigma=0.5,
+                            dead_frac=0.3)
+    L = synth.make_layer(cfg, seed=5)
+    z = O.gate_preactivation(L["x"], L["WgT"])
+    act = O.column_activity(z)
+    c = O.compact_layer(L["WgT"], L["WuT"], L["Wd"], act, cfg.tile)
+    assert c["f_live"] == int(act.sum()) < cfg.f * 0.8
+    assert c["f_c"] % cfg.tile == 0 and c["f_c"] - c["f_live"] < cfg.tile
+    assert np.all(np.diff(c["col_map"][:c["f_live"]]) > 0) and np.all(c["col_map"][c["f_live"]:] == -1)
+    assert not np.any(c["WgT"][c["f_live"]:]) and not np.any(c["Wd"][c["f_live"]:])
+    y0 = O.gated_ffn(L["x"], L["WgT"], L["WuT"], L["Wd"])
+    y1 = O.gated_ffn(L["x"], c["WgT"], c["WuT"], c["Wd"])
+    np.testing.assert_allclose(y1, y0, rtol=1e-12, atol=1e-12 * np.abs(y0).max())
+    r0 = O.relu_ffn(L["x"], L["WgT"], L["Wd"])
+    np.testing.assert_allclose(O.relu_ffn(L["x"], c["WgT"], c["Wd"]), r0, rtol=1e-12, atol=1e-12 * np.abs(r0).max())
+    zc = O.gate_preactivation(L["x"], c["WgT"])
+    assert not np.any(zc[:, c["f_live"]:] > 0)  # padding never activates
+    p0 = O.twell_pack(z, cfg.tile, cfg.tile)
+    p1 = O.twell_pack(zc, cfg.tile, cfg.tile)
+
+    def pairs(p, cmap):
+        out = set()
+        T, nT, W = p["idx"].shape
+        for t in range(T):
+            for ct in range(nT):
+                for s in range(min(int(p["counts"][t, ct]), W)):
+                    j = int(p["idx"][t, ct, s])
+                    out.add((t, int(cmap[j]) if cmap is not None else j, int(p["vals"][t, ct, s])))
+        return out
+
+    assert pairs(p1, c["col_map"]) == pairs(p0, None)
+
+
+def test_compaction_of_a_layer_with_no_dead_units_is_the_identity():
+    rng = np.random.default_rng(32)
+    f, d = 256, 64
+    m = rng.integers(0, 1 << 16, size=(f, d)).astype(np.uint16)
+    c = O.compact_layer(m, m, m, np.ones(f, dtype=bool), 128)
+    assert c["f_c"] == f and np.array_equal(c["WgT"], m) and np.array_equal(c["col_map"], np.arange(f))
+    e = O.compact_layer(m, None, m, np.zeros(f, dtype=bool), 128)
+    assert e["f_live"] == 0 and e["f_c"] == 128 and not np.any(e["WgT"]) and "WuT" not in e
