@@ -54,6 +54,8 @@ __all__ = [
     "hybrid_relu_ffn",
     "column_activity",
     "compact_layer",
+    "gated_ffn_backward",
+    "hybrid_ffn_backward",
 ]
 
 
@@ -323,4 +325,75 @@ def compact_layer(WgT_bits, WuT_bits, Wd_bits, active: np.ndarray, tile: int) ->
         c = np.zeros((f_c, m.shape[1]), dtype=m.dtype)
         c[:f_live] = m[live]
         out[name] = c
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Backward pass through the hybrid format [P1, "Слитые CUDA-ядра для инференса
+# и гибрид для обучения": in training, rows that are sparse enough use the
+# compact sparse format, rows with many active units take a dense branch].
+# The gradients of y = (ReLU(x Wg) * (x Wu)) Wd for an upstream gradient dy:
+#   dh = dy Wd^T, du = dh * g, dz = dh * u * [z > 0] (g = ReLU(z), h = g * u),
+#   dWd = h^T dy, dWu^T = du^T x, dWg^T = dz^T x, dx = dz Wg^T + du Wu^T.
+# Every term vanishes where z <= 0, so the sparse rows need only their stored
+# units. The ReLU derivative at z == 0 is 0 (active iff z > 0).
+
+
+def gated_ffn_backward(x_bits, WgT_bits, WuT_bits, Wd_bits, dy_bits) -> dict:
+    """Dense gradients in float64: dx [T, d], dWgT, dWuT, dWd [f, d]."""
+    x = bf16_bits_to_f64(x_bits)
+    WgT = bf16_bits_to_f64(WgT_bits)
+    WuT = bf16_bits_to_f64(WuT_bits)
+    Wd = bf16_bits_to_f64(Wd_bits)
+    dy = bf16_bits_to_f64(dy_bits)
+    z = x @ WgT.T
+    u = x @ WuT.T
+    act = z > 0
+    g = np.where(act, z, 0.0)
+    dh = dy @ Wd.T
+    du = dh * g
+    dz = np.where(act, dh * u, 0.0)
+    return {"dx": dz @ WgT + du @ WuT, "dWgT": dz.T @ x, "dWuT": du.T @ x, "dWd": (g * u).T @ dy}
+
+
+def hybrid_ffn_backward(x_bits, WgT_bits, WuT_bits, Wd_bits, dy_bits, tile: int, W: int) -> dict:
+    """The method's backward: the gate pack and routing of the forward; for a
+    row that fits, each stored slot (j, g) with g the stored bf16 value gives
+    u_j = x_t . Wu[:, j], dh_j = dy_t . Wd[j, :], h_j = g u_j, du_j = dh_j g,
+    dz_j = dh_j u_j; overflow rows take the dense gradients. dx is per row;
+    the weight gradients sum both kinds of rows."""
+    x = bf16_bits_to_f64(x_bits)
+    WgT = bf16_bits_to_f64(WgT_bits)
+    WuT = bf16_bits_to_f64(WuT_bits)
+    Wd = bf16_bits_to_f64(Wd_bits)
+    dy = bf16_bits_to_f64(dy_bits)
+    z = x @ WgT.T
+    tw = twell_pack(z, tile, W)
+    ovf = route_rows(tw["counts"], W)
+    T, d = x.shape
+    f = WgT.shape[0]
+    out = {"dx": np.zeros((T, d)), "dWgT": np.zeros((f, d)), "dWuT": np.zeros((f, d)), "dWd": np.zeros((f, d)),
+           "twell": tw, "ovf_rows": ovf}
+    counts, idx, vals = tw["counts"], tw["idx"], tw["vals"]
+    nT = idx.shape[1]
+    is_ovf = np.zeros(T, dtype=bool)
+    is_ovf[ovf] = True
+    for t in np.nonzero(~is_ovf)[0]:
+        n = np.minimum(counts[t].astype(np.int64), W)
+        js = np.concatenate([idx[t, c, : n[c]] for c in range(nT)]).astype(np.int64)
+        if js.size == 0:
+            continue
+        g = bf16_bits_to_f64(np.concatenate([vals[t, c, : n[c]] for c in range(nT)]))
+        u = WuT[js] @ x[t]
+        dh = Wd[js] @ dy[t]
+        du, dz = dh * g, dh * u
+        out["dx"][t] = dz @ WgT[js] + du @ WuT[js]
+        out["dWgT"][js] += dz[:, None] * x[t][None, :]
+        out["dWuT"][js] += du[:, None] * x[t][None, :]
+        out["dWd"][js] += (g * u)[:, None] * dy[t][None, :]
+    if ovf.size:
+        dense = gated_ffn_backward(np.asarray(x_bits)[ovf], WgT_bits, WuT_bits, Wd_bits, np.asarray(dy_bits)[ovf])
+        out["dx"][ovf] = dense["dx"]
+        for k in ("dWgT", "dWuT", "dWd"):
+            out[k] += dense[k]
     return out

@@ -578,3 +578,130 @@ def test_compaction_of_a_layer_with_no_dead_units_is_the_identity():
     assert c["f_c"] == f and np.array_equal(c["WgT"], m) and np.array_equal(c["col_map"], np.arange(f))
     e = O.compact_layer(m, None, m, np.zeros(f, dtype=bool), 128)
     assert e["f_live"] == 0 and e["f_c"] == 128 and not np.any(e["WgT"]) and "WuT" not in e
+
+
+# ---------------------------------------------------------------------------
+# Backward pass
+
+
+def _rand_bf16(rng, shape, scale=1.0):
+    return torch_bf16_bits((scale * rng.standard_normal(shape)).astype(np.float32))
+
+
+def test_backward_matches_finite_differences():
+    """Central differences of L = <dy, y> in float64, along random directions,
+    at a point whose gate pre-activations are far from the ReLU kink."""
+    rng = np.random.default_rng(41)
+    T, d, f = 4, 6, 9
+    x, WgT, WuT, Wd, dy = (_rand_bf16(rng, s) for s in ((T, d), (f, d), (f, d), (f, d), (T, d)))
+    F = O.bf16_bits_to_f64
+    xv, gv, uv, wv, dyv = F(x), F(WgT), F(WuT), F(Wd), F(dy)
+    assert np.abs(xv @ gv.T).min() > 1e-3
+
+    def loss(xv, gv, uv, wv):
+        return float(np.sum(dyv * ((np.maximum(xv @ gv.T, 0) * (xv @ uv.T)) @ wv)))
+
+    grads = O.gated_ffn_backward(x, WgT, WuT, Wd, dy)
+    eps = 1e-6
+    for name, pos in (("dx", 0), ("dWgT", 1), ("dWuT", 2), ("dWd", 3)):
+        for _ in range(3):
+            args = [xv, gv, uv, wv]
+            v = rng.standard_normal(args[pos].shape)
+            plus = list(args)
+            minus = list(args)
+            plus[pos] = args[pos] + eps * v
+            minus[pos] = args[pos] - eps * v
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            an = float(np.sum(grads[name] * v))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_backward_exact_rational_bruteforce():
+    rng = np.random.default_rng(42)
+    T, d, f = 2, 3, 4
+    x, WgT, WuT, Wd, dy = (_rand_bf16(rng, s) for s in ((T, d), (f, d), (f, d), (f, d), (T, d)))
+    F = lambda b: [[Fraction(float(v)) for v in row] for row in O.bf16_bits_to_f64(b)]
+    X, G, U, D, DY = F(x), F(WgT), F(WuT), F(Wd), F(dy)
+    got = O.gated_ffn_backward(x, WgT, WuT, Wd, dy)
+    dx = [[Fraction(0)] * d for _ in range(T)]
+    dG = [[Fraction(0)] * d for _ in range(f)]
+    dU = [[Fraction(0)] * d for _ in range(f)]
+    dD = [[Fraction(0)] * d for _ in range(f)]
+    for t in range(T):
+        for j in range(f):
+            z = sum(X[t][k] * G[j][k] for k in range(d))
+            u = sum(X[t][k] * U[j][k] for k in range(d))
+            if z <= 0:
+                continue
+            dh = sum(DY[t][k] * D[j][k] for k in range(d))
+            for k in range(d):
+                dx[t][k] += dh * u * G[j][k] + dh * z * U[j][k]
+                dG[j][k] += dh * u * X[t][k]
+                dU[j][k] += dh * z * X[t][k]
+                dD[j][k] += z * u * DY[t][k]
+    for name, ref in (("dx", dx), ("dWgT", dG), ("dWuT", dU), ("dWd", dD)):
+        r = np.array([[float(v) for v in row] for row in ref])
+        np.testing.assert_allclose(got[name], r, rtol=1e-12, atol=1e-12 * max(1.0, np.abs(r).max()))
+
+
+def test_backward_special_cases():
+    L = synth.make_layer(synth.CONFIGS["tiny"], seed=6)
+    rng = np.random.default_rng(43)
+    dy = _rand_bf16(rng, (64, 128))
+    zero = O.gated_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], np.zeros_like(dy))
+    assert all(not np.any(zero[k]) for k in ("dx", "dWgT", "dWuT", "dWd"))
+    neg = O.bf16_bits_to_f64(L["WgT"]).copy()
+    neg[:, -1] = -64.0
+    dead = O.gated_ffn_backward(L["x"], bits_of_exact(neg), L["WuT"], L["Wd"], dy)
+    assert all(not np.any(dead[k]) for k in ("dx", "dWgT", "dWuT", "dWd"))
+    # one active unit j: dWd[j] = sum_t z_j u_j dy_t, other rows zero
+    js = 9
+    neg[js, -1] = 64.0
+    one = O.gated_ffn_backward(L["x"], bits_of_exact(neg), L["WuT"], L["Wd"], dy)
+    xf = O.bf16_bits_to_f64(L["x"])
+    zj = xf @ neg[js]
+    uj = xf @ O.bf16_bits_to_f64(L["WuT"])[js]
+    assert np.all(zj > 0)
+    np.testing.assert_allclose(one["dWd"][js], (zj * uj) @ O.bf16_bits_to_f64(dy), rtol=1e-12, atol=1e-12)
+    assert not np.any(np.delete(one["dWd"], js, axis=0))
+
+
+def test_hybrid_backward_exact_when_gate_is_bf16_exact():
+    rng = np.random.default_rng(44)
+    T, d, f, W = 40, 8, 384, 8
+    xv = rng.integers(-1, 2, size=(T, d)).astype(np.float64)
+    xv[:, 7] = 1.0
+    xv[:5, 7] = -1.0  # five dense rows that overflow
+    w1 = rng.integers(-1, 2, size=(f, d)).astype(np.float64)
+    w1[:, 7] = -4.0
+    x, WgT = bits_of_exact(xv), bits_of_exact(w1)
+    WuT, Wd, dy = _rand_bf16(rng, (f, d)), _rand_bf16(rng, (f, d)), _rand_bf16(rng, (T, d))
+    out = O.hybrid_ffn_backward(x, WgT, WuT, Wd, dy, 128, W)
+    assert set(range(5)) <= set(out["ovf_rows"].tolist()) and len(out["ovf_rows"]) < T // 2
+    ref = O.gated_ffn_backward(x, WgT, WuT, Wd, dy)
+    for k in ("dx", "dWgT", "dWuT", "dWd"):
+        np.testing.assert_allclose(out[k], ref[k], rtol=1e-12, atol=1e-12 * np.abs(ref[k]).max())
+
+
+def test_hybrid_backward_within_one_rounding_of_dense():
+    """Sparse rows use the stored bf16 gate g: h = g u and du = dh g move by at
+    most 2^-8 relative per term; dz = dh u does not involve g."""
+    L = synth.make_layer(HEAVY, seed=2)
+    rng = np.random.default_rng(45)
+    dy = _rand_bf16(rng, (HEAVY.T, HEAVY.d))
+    out = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, HEAVY.tile, HEAVY.W)
+    ref = O.gated_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy)
+    F = O.bf16_bits_to_f64
+    x, WgT, WuT, Wd, dyv = F(L["x"]), F(L["WgT"]), F(L["WuT"]), F(L["Wd"]), F(dy)
+    z = x @ WgT.T
+    g = np.maximum(z, 0)
+    u = x @ WuT.T
+    dh = dyv @ Wd.T
+    du = np.abs(dh * g)
+    tiny = 1e-12
+    assert np.all(np.abs(out["dx"] - ref["dx"]) <= 2.0**-8 * (du @ np.abs(WuT)) + tiny)
+    assert np.all(np.abs(out["dWuT"] - ref["dWuT"]) <= 2.0**-8 * (du.T @ np.abs(x)) + tiny)
+    assert np.all(np.abs(out["dWd"] - ref["dWd"]) <= 2.0**-8 * (np.abs(g * u).T @ np.abs(dyv)) + tiny)
+    np.testing.assert_allclose(out["dWgT"], ref["dWgT"], rtol=1e-10, atol=1e-10 * np.abs(ref["dWgT"]).max())
+    assert np.array_equal(out["dx"][out["ovf_rows"]], ref["dx"][out["ovf_rows"]])
+    assert np.abs(out["dWd"] - ref["dWd"]).max() > 0  # the rounding is visible
