@@ -425,5 +425,79 @@ __global__ void __launch_bounds__(256) unpack_kernel(const int16_t* counts, cons
   if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(dev_status, kDevIndex);
 }
 
-}  // namespace twell
+// ---------------------------------------------------------------- compaction
 
+// One block of 1024 threads (f / 32 <= 1024 bitmap words): col_map[0..f_live)
+// = the set bits of `active` in ascending order, col_map[f_live..f) = -1,
+// *f_live = their number.
+__global__ void __launch_bounds__(1024) compact_columns_kernel(const uint32_t* __restrict__ active, int f,
+                                                                int32_t* __restrict__ col_map,
+                                                                int32_t* __restrict__ f_live) {
+  __shared__ int warp_sums[32];
+  __shared__ int s_total;
+  const int nwords = (f + 31) / 32;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  uint32_t bits = tid < nwords ? active[tid] : 0u;
+  if (tid == nwords - 1 && (f & 31)) bits &= (1u << (f & 31)) - 1u;
+  const int n = __popc(bits);
+  int incl = n;  // inclusive scan of the popcounts within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {  // warp totals -> exclusive prefixes
+    const int w = warp_sums[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += v;
+    }
+    warp_sums[lane] = wi - w;
+  }
+  __syncthreads();
+  int pos = warp_sums[wid] + incl - n;
+  if (tid == 1023) s_total = warp_sums[31] + incl;
+  while (bits != 0) {
+    const int b = __ffs(bits) - 1;
+    bits &= bits - 1u;
+    col_map[pos++] = tid * 32 + b;
+  }
+  __syncthreads();
+  for (int i = s_total + tid; i < f; i += 1024) col_map[i] = -1;
+  if (tid == 0) *f_live = s_total;
+}
+
+// out[i] = W[col_map[i]] for i < min(*f_live, f_out), zero rows after; one
+// warp per row, 16-byte copies (d % 64 == 0). Map entries outside [0, f)
+// raise TWELL_ERR_INDEX and give a zero row.
+__global__ void gather_weight_rows_kernel(const uint16_t* __restrict__ W, int f, int d,
+                                          const int32_t* __restrict__ col_map, const int32_t* __restrict__ f_live,
+                                          int f_out, uint16_t* __restrict__ out, int* dev_status) {
+  const int n_live = min(max(*f_live, 0), f_out);
+  const int lane = threadIdx.x & 31;
+  const int vecs = d / 8;  // uint4 per row
+  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < f_out;
+       row += (gridDim.x * blockDim.x) >> 5) {
+    int src = -1;
+    if (row < n_live) {
+      src = col_map[row];
+      if (src < 0 || src >= f) {
+        if (lane == 0) raise_status(dev_status, kDevIndex);
+        src = -1;
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(row) * d);
+    if (src < 0) {
+      for (int v = lane; v < vecs; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+    } else {
+      const uint4* s4 = reinterpret_cast<const uint4*>(W + static_cast<size_t>(src) * d);
+      for (int v = lane; v < vecs; v += 32) dst[v] = __ldg(s4 + v);
+    }
+  }
+}
+
+}  // namespace twell

@@ -548,6 +548,50 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
                     dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 
+twell_status twell_column_activity(const uint16_t* x, const uint16_t* WgT, int T, int d, int f,
+                                   uint32_t* active_bits, int accumulate, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_ptrs({active_bits, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!accumulate) TW_TRY(cuda_ok(cudaMemsetAsync(active_bits, 0, static_cast<size_t>(f / 32) * 4, s)));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT}));
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mb, WgT, d, f, kBK, kBN)) return TWELL_ERR_CUDA;
+  GemmParams p{};
+  p.M = T;
+  p.N = f;
+  p.K = d;
+  p.active = active_bits;
+  p.dev_status = dev_status;
+  return launch_gemm<kModeActivity>(ma, mb, mb, p, gemm_grid(T, f, kBN, sms), s);
+}
+
+twell_status twell_compact_columns(const uint32_t* active_bits, int f, int32_t* col_map, int32_t* f_live,
+                                   void* stream) {
+  if (f < 128 || f % 128 != 0 || f > 32767) return TWELL_ERR_SHAPE;
+  TW_TRY(check_ptrs({active_bits, col_map, f_live}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  compact_columns_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(active_bits, f, col_map, f_live);
+  return cuda_ok(cudaGetLastError());
+}
+
+twell_status twell_gather_rows(const uint16_t* W, int f, int d, const int32_t* col_map, const int32_t* f_live,
+                               int f_out, uint16_t* W_out, int32_t* dev_status, void* stream) {
+  if (f < 128 || f % 128 != 0 || f > 32767 || d < 64 || d % 64 != 0 || d > 4096 || f_out < 1 || f_out > f)
+    return TWELL_ERR_SHAPE;
+  TW_TRY(check_ptrs({W, col_map, f_live, W_out, dev_status}));
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  const int blocks = std::min((f_out + 7) / 8, 4 * sms);
+  gather_weight_rows_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, f, d, col_map, f_live, f_out,
+                                                                                  W_out, dev_status);
+  return cuda_ok(cudaGetLastError());
+}
+
 twell_status twell_unpack(const twell_t* tw, uint16_t* g_dense, int32_t* dev_status, void* stream) {
   if (tw == nullptr) return TWELL_ERR_NULL;
   TW_TRY(check_tw(tw, tw->T, tw->f));

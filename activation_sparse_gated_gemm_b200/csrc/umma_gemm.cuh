@@ -21,6 +21,10 @@
 //   kModeRelu   -- h = ReLU(x . W1) stored as bf16 (and optionally the bf16
 //                  remainder, as in kModeGateUp): the first half of the dense
 //                  non-gated layer.
+//   kModeActivity -- the gate GEMM z = x . Wg with an epilogue that only marks
+//                  the columns where some row has z > 0 (a bitmap, one bit per
+//                  hidden unit, OR-ed in with one atomic per warp and 32
+//                  columns): the profile that finds dead hidden units.
 //   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
 //                  epilogue stores fp32 rows, optionally scattered through a
 //                  row map (the dense branch of the hybrid route). With the
@@ -40,7 +44,14 @@
 
 namespace twell {
 
-enum GemmMode : int { kModeTwell = 0, kModeGateUp = 1, kModeDown = 2, kModeTwellHidden = 3, kModeRelu = 4 };
+enum GemmMode : int {
+  kModeTwell = 0,
+  kModeGateUp = 1,
+  kModeDown = 2,
+  kModeTwellHidden = 3,
+  kModeRelu = 4,
+  kModeActivity = 5
+};
 
 constexpr int kBM = 128;
 constexpr int kBN = 256;
@@ -82,6 +93,7 @@ struct GemmParams {
   uint16_t* out;
   float* out_f32;
   int ldo;
+  uint32_t* active;    // kModeActivity: column bitmap, OR-ed into
   const int* row_map;  // kModeDown: output row of each A row, or null
   int out_rows;        // valid range of output rows
   // kModeGateUp / kModeRelu: also store h_lo = bf16(h - bf16(h)) at column N + c (ldo = 2N).
@@ -235,7 +247,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* b_dst = smem + kOffB + s * kBStageBytes;
           mbar_arrive_expect_tx(&full[s], kAStageBytes + kBStageBytes);
           tma_load_2d(a_dst, &tmA, &full[s], kb * kBK, m_blk * kBM);
-          if (MODE == kModeTwell || MODE == kModeRelu) {
+          if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * kBN);
           } else if (kStacked) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * 128);
@@ -453,6 +465,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i < 32; ++i) h[i] = fmaxf(__uint_as_float(zr[i]), 0.0f) * __uint_as_float(ur[i]);
             store_h32(h, p.out + static_cast<size_t>(my_row) * p.ldo, col, p.N, p.h_split != 0);
           }
+        }
+      } else if (MODE == kModeActivity) {
+#pragma unroll 1
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), r);
+          tmem_wait_ld();
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int col = n_blk * kBN + ch * 32;
+          uint32_t mask = 0;
+          if (my_row < M) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mask |= (static_cast<int32_t>(r[i]) > 0 ? 1u : 0u) << i;
+          }
+          mask = __reduce_or_sync(0xffffffffu, mask);
+          if (lane == 0 && mask != 0 && col < p.N) atomicOr(p.active + col / 32, mask);
         }
       } else if (MODE == kModeRelu) {
 #pragma unroll 1

@@ -31,6 +31,7 @@ EXPORTED = (
     "twell_status_str", "twell_version", "twell_ffn_hybrid_forward_noalloc",
     "twell_gate_up_pack", "twell_sparse_down", "twell_ffn_hybrid_forward_tc_up",
     "twell_relu_ffn_hybrid_forward", "twell_relu_dense_rows_forward", "twell_relu_dense_ffn_forward",
+    "twell_column_activity", "twell_compact_columns", "twell_gather_rows",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -84,6 +85,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_relu_ffn_hybrid_forward": ([vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_relu_dense_rows_forward": ([vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_relu_dense_ffn_forward": ([vp, vp, vp, i32, i32, i32, vp, vp, sz, vp, vp], i32),
+        "twell_column_activity": ([vp, vp, i32, i32, i32, vp, i32, vp, vp], i32),
+        "twell_compact_columns": ([vp, i32, vp, vp, vp], i32),
+        "twell_gather_rows": ([vp, i32, i32, vp, vp, i32, vp, vp, vp], i32),
         "twell_unpack": ([tw, vp, vp, vp], i32),
         "twell_ffn_hybrid_forward_noalloc": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp], i32),
         "twell_status_reset": ([vp, vp], i32),
@@ -312,6 +316,60 @@ def relu_dense_ffn_forward(x, W1T, W2, y, workspace, dev_status, stream=None) ->
     _check("twell_relu_dense_ffn_forward", load().twell_relu_dense_ffn_forward(
         _ptr(x), _ptr(W1T), _ptr(W2), T, d, f, _ptr(y), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def column_activity(x, WgT, active_bits, accumulate: bool, dev_status, stream=None) -> None:
+    """Bit j of active_bits ([f // 32] int32 tensor) := some row of x has x . Wg[:, j] > 0
+    (OR-ed into the existing bits when accumulate)."""
+    T, d = x.shape
+    f = WgT.shape[0]
+    _bf16("x", x, (T, d))
+    _bf16("WgT", WgT, (f, d))
+    _dev("active_bits", active_bits, (f // 32,), torch.int32)
+    _check("twell_column_activity", load().twell_column_activity(
+        _ptr(x), _ptr(WgT), T, d, f, _ptr(active_bits), int(bool(accumulate)), _ptr(dev_status), _stream(stream)))
+
+
+def compact_columns(active_bits, f: int, col_map, f_live, stream=None) -> None:
+    _dev("active_bits", active_bits, (f // 32,), torch.int32)
+    _dev("col_map", col_map, (f,), torch.int32)
+    _dev("f_live", f_live, (1,), torch.int32)
+    _check("twell_compact_columns", load().twell_compact_columns(
+        _ptr(active_bits), f, _ptr(col_map), _ptr(f_live), _stream(stream)))
+
+
+def gather_rows(W, col_map, f_live, W_out, dev_status, stream=None) -> None:
+    f, d = W.shape
+    f_out = W_out.shape[0]
+    _bf16("W", W, (f, d))
+    _bf16("W_out", W_out, (f_out, d))
+    _dev("col_map", col_map, (f,), torch.int32)
+    _check("twell_gather_rows", load().twell_gather_rows(
+        _ptr(W), f, d, _ptr(col_map), _ptr(f_live), f_out, _ptr(W_out), _ptr(dev_status), _stream(stream)))
+
+
+def compact_layer(x_profile, weights, dev_status, tile: int = 128, stream=None) -> dict:
+    """Drop the hidden units that no row of x_profile activates: returns the
+    gathered weights (same keys as `weights`, e.g. WgT/WuT/Wd, each [f_c, d]),
+    col_map (original unit of each kept row, -1 for padding), f_live and f_c
+    (f_live rounded up to a whole tile). The gate weight is weights["WgT"].
+    Reads f_live back to the host once (a one-time model transformation)."""
+    WgT = weights["WgT"]
+    f = WgT.shape[0]
+    dev = WgT.device
+    bits = torch.empty((f // 32,), dtype=torch.int32, device=dev)
+    col_map = torch.empty((f,), dtype=torch.int32, device=dev)
+    f_live = torch.zeros((1,), dtype=torch.int32, device=dev)
+    column_activity(x_profile, WgT, bits, False, dev_status, stream)
+    compact_columns(bits, f, col_map, f_live, stream)
+    n = int(f_live.item())
+    f_c = max(tile, -(-n // tile) * tile)
+    out = {"col_map": col_map[:f_c].clone(), "f_live": n, "f_c": f_c, "active_bits": bits}
+    for k, W in weights.items():
+        Wc = torch.empty((f_c, W.shape[1]), dtype=W.dtype, device=dev)
+        gather_rows(W, col_map, f_live, Wc, dev_status, stream)
+        out[k] = Wc
+    return out
 
 
 def unpack(tw: Twell, g_dense, dev_status, stream=None) -> None:

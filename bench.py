@@ -19,6 +19,7 @@ sample of the workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -260,11 +261,20 @@ def run_gpu(args, world, rank, local):
     dev = torch.device("cuda", local)
     cfg = synth.CONFIGS[args.config]
     L = synth.make_layer(cfg, seed=args.seed)
-    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
     x = tl.to_device_bf16(L["x"], dev)
     WgT = tl.to_device_bf16(L["WgT"], dev)
     WuT = tl.to_device_bf16(L["WuT"], dev)
     Wd = tl.to_device_bf16(L["Wd"], dev)
+    compact_info = None
+    if args.compact:
+        # drop the hidden units that the batch never activates (a one-time model
+        # transformation, outside the timed region); the layer then has f_c units
+        c = tl.compact_layer(x, {"WgT": WgT, "WuT": WuT, "Wd": Wd}, tl.new_status(dev))
+        WgT, WuT, Wd = c["WgT"], c["WuT"], c["Wd"]
+        compact_info = {"f_orig": cfg.f, "f_live": c["f_live"], "f_c": c["f_c"],
+                        "profile": "the timed batch itself"}
+        cfg = dataclasses.replace(cfg, f=c["f_c"])
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
     tw = tl.Twell(T, f, W, device=dev)
     y = torch.empty((T, d), dtype=torch.float32, device=dev)
     ovf_rows = torch.empty((T,), dtype=torch.int32, device=dev)
@@ -439,7 +449,9 @@ def run_gpu(args, world, rank, local):
         "data": "synthetic (seeded generator; no dataset or trained weights)",
         "config": {"workload": (f"{cfg.name}-like non-gated ReLU FFN layer forward (W1 = Wg, W2 = Wd), "
                                 "hybrid TwELL" if layer == "relu" else
-                                f"{cfg.name}-like FFN layer forward, hybrid TwELL"), "variant": chosen,
+                                f"{cfg.name}-like FFN layer forward, hybrid TwELL")
+                               + (f", dead units dropped (f {compact_info['f_orig']} -> {cfg.f})"
+                                  if compact_info else ""), "variant": chosen, "compaction": compact_info,
                    "tokens": T, "d": d,
                    "f": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
                    "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
@@ -607,6 +619,8 @@ def main(argv=None):
                     help="hybrid form: gate (sparse up+down) or tc_up (up on tensor cores); auto times both")
     ap.add_argument("--layer", default="gated", choices=["gated", "relu"],
                     help="gated: (ReLU(x Wg) * x Wu) Wd; relu: the non-gated ReLU(x W1) W2")
+    ap.add_argument("--compact", action="store_true",
+                    help="drop the hidden units the batch never activates before timing")
     ap.add_argument("--sweep", action="store_true", help="density x batch sweep, one JSON line per point")
     ap.add_argument("--sweep-T", default="", help="comma-separated token counts (default: the full sweep)")
     ap.add_argument("--sweep-p", default="", help="comma-separated densities (default: the full sweep)")

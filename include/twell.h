@@ -277,6 +277,42 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
                                           size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * Dead hidden units (intellectnews.ru, "Sakana AI и NVIDIA: TwELL ...",
+ * section "Ограничения и открытые вопросы": under the chosen L1 setting some
+ * units die, i.e. are never active). Three calls compact a layer to the units
+ * a profile batch activates:
+ *
+ * twell_column_activity: the gate GEMM z = x Wg on the tensor cores with an
+ * epilogue that sets bit j of active_bits ([f / 32] uint32, device) iff
+ * z[t, j] > 0 for some row t. accumulate == 0 clears the bitmap first;
+ * accumulate != 0 ORs this batch into it (a profile over several batches).
+ * T == 0 only clears (or keeps) the bitmap. Shapes as for twell_gate_pack.
+ */
+twell_status twell_column_activity(const uint16_t* x, const uint16_t* WgT, int T, int d, int f,
+                                   uint32_t* active_bits, int accumulate, int32_t* dev_status,
+                                   void* stream);
+
+/*
+ * twell_compact_columns: col_map[0 .. f_live) = the indices j with bit j of
+ * active_bits set, ascending; col_map[f_live .. f) = -1; *f_live (device
+ * int32) = their number. col_map is [f] int32 device memory. One block.
+ */
+twell_status twell_compact_columns(const uint32_t* active_bits, int f, int32_t* col_map, int32_t* f_live,
+                                   void* stream);
+
+/*
+ * twell_gather_rows: W_out[i, :] = W[col_map[i], :] for i < min(*f_live,
+ * f_out) and zero rows for the rest, W [f][d] and W_out [f_out][d] bf16
+ * (1 <= f_out <= f). Applied to WgT, WuT and Wd with f_out = f_live rounded
+ * up to a multiple of 128 (the caller reads *f_live), it gives the compacted
+ * layer: its zero gate rows have z = 0 and are never active, so on the
+ * profile batch the layer computes the same y with f_out hidden units. A map
+ * entry outside [0, f) raises TWELL_ERR_INDEX and gives a zero row.
+ */
+twell_status twell_gather_rows(const uint16_t* W, int f, int d, const int32_t* col_map, const int32_t* f_live,
+                               int f_out, uint16_t* W_out, int32_t* dev_status, void* stream);
+
+/*
  * TwELL -> dense bf16 g[T][f]: zeros everywhere except the stored slots
  * (slots below min(count, W); overflowing rows unpack only what was stored).
  */

@@ -97,3 +97,17 @@ def test_status_strings(lib):
         s = tl.status_str(code)
         assert s and s != "unknown status"
     assert tl.status_str(99) == "unknown status"
+
+
+def test_compaction_argument_errors(lib):
+    # shapes are checked before anything else
+    assert lib.twell_column_activity(FAKE, FAKE, 64, 100, 512, FAKE, 0, FAKE, None) == tl.TWELL_ERR_SHAPE
+    assert lib.twell_compact_columns(FAKE, 500, FAKE, FAKE, None) == tl.TWELL_ERR_SHAPE
+    assert lib.twell_compact_columns(FAKE, 32768, FAKE, FAKE, None) == tl.TWELL_ERR_SHAPE
+    assert lib.twell_gather_rows(FAKE, 512, 128, FAKE, FAKE, 513, FAKE, FAKE, None) == tl.TWELL_ERR_SHAPE
+    assert lib.twell_gather_rows(FAKE, 512, 128, FAKE, FAKE, 0, FAKE, FAKE, None) == tl.TWELL_ERR_SHAPE
+    assert lib.twell_gather_rows(FAKE, 512, 96, FAKE, FAKE, 128, FAKE, FAKE, None) == tl.TWELL_ERR_SHAPE
+    # then pointers
+    assert lib.twell_column_activity(FAKE, FAKE, 64, 128, 512, None, 0, FAKE, None) == tl.TWELL_ERR_NULL
+    assert lib.twell_compact_columns(FAKE, 512, None, FAKE, None) == tl.TWELL_ERR_NULL
+    assert lib.twell_gather_rows(FAKE, 512, 128, MIS, FAKE, 128, FAKE, FAKE, None) == tl.TWELL_ERR_ALIGN
