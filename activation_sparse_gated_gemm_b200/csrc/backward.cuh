@@ -1,0 +1,396 @@
+// Backward pass of the TwELL gated FFN through the hybrid format
+// (intellectnews.ru "Sakana AI и NVIDIA ... TwELL", section "Слитые CUDA-ядра
+// для инференса и гибрид для обучения": in training, rows that are sparse
+// enough use the compact format, rows with many active units a dense branch).
+//
+// With g = ReLU(z), h = g * u and an upstream gradient dy:
+//   dh_j = dy . Wd[j, :], du_j = dh_j g_j, dz_j = dh_j u_j   (only where z_j > 0)
+//   dx   = sum_j dz_j Wg[:, j] + du_j Wu[:, j]
+//   dWd[j, :] = sum_t h_tj dy_t, dWu[:, j] = sum_t du_tj x_t, dWg[:, j] = sum_t dz_tj x_t
+//
+// Two passes over the stored units:
+//   1. per token (one warp per token, like the forward's fused kernel): u_j and
+//      dh_j by two dot products per stored unit, then dx_t by two row axpys;
+//      the per-unit scalars (h, du, dz) are written beside the slots;
+//   2. per hidden unit: the slots are sorted by column (count, scan, scatter)
+//      and one warp per (unit, 256-wide slice of d) sums h dy_t, du x_t, dz x_t
+//      over the unit's tokens into the three weight-gradient rows.
+// Rows that overflow the ELL width are packed again at the full tile width
+// (nothing dropped) from the gathered rows, and go through the same two
+// passes with their gate recomputed in fp32 instead of the stored bf16 value.
+#pragma once
+
+#include "sparse_ffn.cuh"
+
+namespace twell {
+
+struct BwdParams {
+  const uint16_t* x;   // [rows][d] bf16: the tokens, or the gathered overflow rows
+  const uint16_t* dy;  // [rows][d] bf16 upstream gradient, same rows
+  const uint16_t* WgT;
+  const uint16_t* WuT;
+  const uint16_t* Wd;
+  const int16_t* counts;  // TwELL of these rows
+  const int16_t* idx;
+  const uint16_t* vals;
+  const uint8_t* row_ovf;
+  int rows;             // rows of this pass (an upper bound when rows_dev is set)
+  const int* rows_dev;  // device row count, or null
+  const int* row_map;   // dx row of each pass row, or null for the identity
+  int d, f, nT, W;
+  int skip_ovf;     // skip rows whose overflow flag is set
+  int recompute_g;  // g_j = max(0, x_t . Wg[:, j]) in fp32 instead of the stored bf16
+  float* dx;        // [dx_rows][d] fp32
+  int dx_rows;
+  float* s_h;  // per stored slot [rows][nT][W]: h, du, dz (fp32)
+  float* s_du;
+  float* s_dz;
+  int* dev_status;
+};
+
+constexpr int kBwdWarps = 8;
+
+// One warp per token of the pass. Shared memory per warp: x_t and dy_t
+// (NCH * 32 uint4 each), the flattened slot list (column | bf16 g << 16) and
+// the slot position of every list entry inside the row's [nT][W] block.
+template <int NCH>
+__global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_token_kernel(const BwdParams p) {
+  extern __shared__ uint4 bwd_smem[];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int d = p.d;
+  uint4* xs = bwd_smem + warp * 2 * NCH * 32;
+  uint4* ds = xs + NCH * 32;
+  uint32_t* list = reinterpret_cast<uint32_t*>(bwd_smem + kBwdWarps * 2 * NCH * 32) + warp * kListCap;
+  uint16_t* lpos =
+      reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + kBwdWarps * 2 * NCH * 32) +
+                                  kBwdWarps * kListCap) +
+      warp * kListCap;
+  const int group_tiles = max(1, kListCap / p.W);
+  int rows = p.rows;
+  if (p.rows_dev != nullptr) rows = min(max(*p.rows_dev, 0), rows);
+  bool bad_index = false;
+  const int gw = blockIdx.x * kBwdWarps + warp;
+  const int nw = gridDim.x * kBwdWarps;
+#pragma unroll 1
+  for (int t = gw; t < rows; t += nw) {
+    if (p.skip_ovf && p.row_ovf[t]) continue;
+    int r = t;
+    if (p.row_map != nullptr) {
+      r = p.row_map[t];
+      if (r < 0 || r >= p.dx_rows) {
+        bad_index = true;
+        continue;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int k0 = (i * 32 + lane) * 8;
+      const bool in = k0 < d;
+      xs[i * 32 + lane] = in ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
+      ds[i * 32 + lane] = in ? ldg_nc_v4(p.dy + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
+    }
+    float acc[NCH][8];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
+    const size_t slot_row = static_cast<size_t>(t) * p.nT * p.W;
+
+#pragma unroll 1
+    for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
+      const int c1 = min(p.nT, c0 + group_tiles);
+      // ---- flatten the stored slots of tiles [c0, c1)
+      int total = 0;
+#pragma unroll 1
+      for (int cb = c0; cb < c1; cb += 32) {
+        const int c = cb + lane;
+        int n = 0;
+        if (c < c1) n = min(max(static_cast<int>(p.counts[static_cast<size_t>(t) * p.nT + c]), 0), p.W);
+        int incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int off = total + incl - n;
+        total += __shfl_sync(0xffffffffu, incl, 31);
+        const size_t base = (static_cast<size_t>(t) * p.nT + c) * p.W;
+        for (int k = 0; k < n; ++k) {
+          const int jj = p.idx[base + k];
+          uint32_t ent = static_cast<uint32_t>(jj) | (static_cast<uint32_t>(p.vals[base + k]) << 16);
+          uint16_t pos = static_cast<uint16_t>(c * p.W + k);  // < 2^15: nT * W <= 255 * 128
+          if (jj < 0 || jj >= p.f) {
+            bad_index = true;
+            ent = 0;         // read column 0 ...
+            pos |= 0x8000u;  // ... but contribute nothing and store nothing
+          }
+          list[off + k] = ent;
+          lpos[off + k] = pos;
+        }
+      }
+      __syncwarp();
+      // ---- consume in batches of 32 entries
+#pragma unroll 1
+      for (int s0 = 0; s0 < total; s0 += 32) {
+        const int ns = min(32, total - s0);
+        const uint32_t my_e = lane < ns ? list[s0 + lane] : 0u;
+        const int my_j = entry_j(my_e);
+        float my_g = entry_g(my_e), my_u = 0.0f, my_dh = 0.0f;
+        // pass 1: u_j = x . Wu[:, j], dh_j = dy . Wd[j, :] (and z_j when recomputed)
+#pragma unroll 1
+        for (int s = 0; s < ns; ++s) {
+          const int j = __shfl_sync(0xffffffffu, my_j, s);
+          const uint16_t* wu = p.WuT + static_cast<size_t>(j) * d;
+          const uint16_t* wd = p.Wd + static_cast<size_t>(j) * d;
+          const uint16_t* wg = p.WgT + static_cast<size_t>(j) * d;
+          float au0 = 0.f, au1 = 0.f, ah0 = 0.f, ah1 = 0.f, az0 = 0.f, az1 = 0.f;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const int k0 = (i * 32 + lane) * 8;
+            if (k0 < d) {
+              mixdot8(xs[i * 32 + lane], ldg_nc_v4(wu + k0), au0, au1);
+              mixdot8(ds[i * 32 + lane], ldg_nc_v4(wd + k0), ah0, ah1);
+              if (p.recompute_g) mixdot8(xs[i * 32 + lane], ldg_nc_v4(wg + k0), az0, az1);
+            }
+          }
+          float au = au0 + au1, ah = ah0 + ah1, az = az0 + az1;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            au += __shfl_xor_sync(0xffffffffu, au, o);
+            ah += __shfl_xor_sync(0xffffffffu, ah, o);
+            if (p.recompute_g) az += __shfl_xor_sync(0xffffffffu, az, o);
+          }
+          if (lane == s) {
+            my_u = au;
+            my_dh = ah;
+            if (p.recompute_g) my_g = fmaxf(az, 0.0f);
+          }
+        }
+        const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
+        const bool valid = (my_pos & 0x8000u) == 0;
+        const float my_du = valid ? my_dh * my_g : 0.0f;
+        const float my_dz = valid ? my_dh * my_u : 0.0f;
+        if (valid) {
+          const size_t slot = slot_row + my_pos;
+          p.s_h[slot] = my_g * my_u;
+          p.s_du[slot] = my_du;
+          p.s_dz[slot] = my_dz;
+        }
+        // pass 2: dx_t += dz_j Wg[:, j] + du_j Wu[:, j]
+#pragma unroll 1
+        for (int s = 0; s < ns; ++s) {
+          const int j = __shfl_sync(0xffffffffu, my_j, s);
+          const float dz = __shfl_sync(0xffffffffu, my_dz, s);
+          const float du = __shfl_sync(0xffffffffu, my_du, s);
+          const uint16_t* wg = p.WgT + static_cast<size_t>(j) * d;
+          const uint16_t* wu = p.WuT + static_cast<size_t>(j) * d;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const int k0 = (i * 32 + lane) * 8;
+            if (k0 < d) {
+              axpy8(acc[i], dz, ldg_nc_v4(wg + k0));
+              axpy8(acc[i], du, ldg_nc_v4(wu + k0));
+            }
+          }
+        }
+      }
+      __syncwarp();
+    }
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int k0 = (i * 32 + lane) * 8;
+      if (k0 < d) {
+        float4* dst = reinterpret_cast<float4*>(p.dx + static_cast<size_t>(r) * d + k0);
+        dst[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        dst[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, bad_index) && lane == 0) raise_status(p.dev_status, kDevIndex);
+}
+
+// ---------------------------------------------------------------- by column
+
+// The stored slots of one pass, as the column sort sees them.
+struct SlotSource {
+  const int16_t* counts;
+  const int16_t* idx;
+  const uint8_t* row_ovf;  // rows with the flag set are skipped when skip_ovf
+  int rows;
+  const int* rows_dev;
+  int nT, W, f;
+  int skip_ovf;
+  uint32_t tag;  // bit 31 of each list entry: which pass the slot belongs to
+};
+
+__device__ __forceinline__ int source_rows(const SlotSource& s) {
+  return s.rows_dev != nullptr ? min(max(*s.rows_dev, 0), s.rows) : s.rows;
+}
+
+// SCATTER == false: colcnt[j] += number of slots with column j.
+// SCATTER == true: each slot is written to list[colptr[j] + cursor[j]++] as
+// tag | slot index (the order inside a column is that of the atomics).
+template <bool SCATTER>
+__global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colptr, uint32_t* list) {
+  const int lane = threadIdx.x & 31;
+  const int rows = source_rows(src);
+  const long long pairs = static_cast<long long>(rows) * src.nT;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < pairs;
+       w += nw) {
+    const int t = static_cast<int>(w / src.nT);
+    if (src.skip_ovf && src.row_ovf[t]) continue;
+    const int n = min(max(static_cast<int>(src.counts[w]), 0), src.W);
+    for (int k = lane; k < n; k += 32) {
+      const size_t slot = static_cast<size_t>(w) * src.W + k;
+      const int j = src.idx[slot];
+      if (j < 0 || j >= src.f) continue;
+      if (SCATTER) {
+        const int pos = colptr[j] + atomicAdd(colcnt + j, 1);
+        list[pos] = src.tag | static_cast<uint32_t>(slot);
+      } else {
+        atomicAdd(colcnt + j, 1);
+      }
+    }
+  }
+}
+
+// colptr[j] = sum of colcnt[0..j) for j <= f, and colcnt is reset to zero (it
+// then serves as the scatter cursor). One block of 1024 threads.
+__global__ void __launch_bounds__(1024) bwd_column_scan_kernel(int* colcnt, int f, int* colptr) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < f; base += 1024) {
+    const int j = base + tid;
+    const int v = j < f ? colcnt[j] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      const int w = warp_sums[lane];
+      int wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += u;
+      }
+      warp_sums[lane] = wi - w;
+    }
+    __syncthreads();
+    const int excl = carry + warp_sums[wid] + incl - v;
+    if (j < f) {
+      colptr[j] = excl;
+      colcnt[j] = 0;
+    }
+    __syncthreads();
+    if (tid == 1023) carry = excl + v;
+    __syncthreads();
+  }
+  if (tid == 0) colptr[f] = carry;
+}
+
+struct WgradParams {
+  const uint32_t* list;
+  const int* colptr;
+  // pass 0 (rows that fit) and pass 1 (overflow rows), selected by bit 31
+  const uint16_t* x0;
+  const uint16_t* dy0;
+  const float* h0;
+  const float* du0;
+  const float* dz0;
+  int slots_per_row0;  // nT * W of the pass
+  const uint16_t* x1;
+  const uint16_t* dy1;
+  const float* h1;
+  const float* du1;
+  const float* dz1;
+  int slots_per_row1;
+  int f, d;
+  float* dWgT;  // [f][d] fp32, fully written
+  float* dWuT;
+  float* dWd;
+};
+
+// One warp per (hidden unit j, 256-wide slice of d): lane l owns 8 consecutive
+// elements of the slice; the unit's slots are read 32 at a time (lane e
+// fetches entry e's scalars and row), then broadcast one by one.
+__global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
+  const int lane = threadIdx.x & 31;
+  const int slices = (p.d + 255) / 256;
+  const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (w >= static_cast<long long>(p.f) * slices) return;
+  const int j = static_cast<int>(w / slices);
+  const int k0 = static_cast<int>(w - static_cast<long long>(j) * slices) * 256 + lane * 8;
+  const bool mine = k0 < p.d;
+  float ag[8], au[8], ad[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ag[e] = au[e] = ad[e] = 0.0f;
+  const int e0 = p.colptr[j], e1 = p.colptr[j + 1];
+#pragma unroll 1
+  for (int b = e0; b < e1; b += 32) {
+    const int nb = min(32, e1 - b);
+    const uint16_t* xr = nullptr;
+    const uint16_t* dr = nullptr;
+    float vh = 0.f, vu = 0.f, vz = 0.f;
+    if (lane < nb) {
+      const uint32_t ent = p.list[b + lane];
+      const size_t slot = ent & 0x7fffffffu;
+      if (ent >> 31) {
+        const size_t row = slot / static_cast<size_t>(p.slots_per_row1);
+        xr = p.x1 + row * p.d;
+        dr = p.dy1 + row * p.d;
+        vh = p.h1[slot];
+        vu = p.du1[slot];
+        vz = p.dz1[slot];
+      } else {
+        const size_t row = slot / static_cast<size_t>(p.slots_per_row0);
+        xr = p.x0 + row * p.d;
+        dr = p.dy0 + row * p.d;
+        vh = p.h0[slot];
+        vu = p.du0[slot];
+        vz = p.dz0[slot];
+      }
+    }
+#pragma unroll 1
+    for (int s = 0; s < nb; ++s) {
+      const uint16_t* xs = reinterpret_cast<const uint16_t*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(xr), s));
+      const uint16_t* dsr = reinterpret_cast<const uint16_t*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dr), s));
+      const float h = __shfl_sync(0xffffffffu, vh, s);
+      const float du = __shfl_sync(0xffffffffu, vu, s);
+      const float dz = __shfl_sync(0xffffffffu, vz, s);
+      if (mine) {
+        const uint4 xv = ldg_nc_v4(xs + k0);
+        const uint4 dv = ldg_nc_v4(dsr + k0);
+        axpy8(ad, h, dv);
+        axpy8(au, du, xv);
+        axpy8(ag, dz, xv);
+      }
+    }
+  }
+  if (mine) {
+    const size_t o = static_cast<size_t>(j) * p.d + k0;
+    float4* g4 = reinterpret_cast<float4*>(p.dWgT + o);
+    float4* u4 = reinterpret_cast<float4*>(p.dWuT + o);
+    float4* d4 = reinterpret_cast<float4*>(p.dWd + o);
+    g4[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
+    g4[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
+    u4[0] = make_float4(au[0], au[1], au[2], au[3]);
+    u4[1] = make_float4(au[4], au[5], au[6], au[7]);
+    d4[0] = make_float4(ad[0], ad[1], ad[2], ad[3]);
+    d4[1] = make_float4(ad[4], ad[5], ad[6], ad[7]);
+  }
+}
+
+}  // namespace twell

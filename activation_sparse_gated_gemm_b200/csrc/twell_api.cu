@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "twell.h"
+#include "backward.cuh"
 #include "sparse_ffn.cuh"
 #include "umma_gemm.cuh"
 
@@ -141,12 +142,13 @@ int gemm_grid(int M, int N, int tile_n, int sms) {
 }
 
 twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
-                            int32_t* dev_status, cudaStream_t s, int sms) {
+                            int32_t* dev_status, cudaStream_t s, int sms, const int* M_dev = nullptr) {
   TW_TRY(cuda_ok(cudaMemsetAsync(tw->row_ovf, 0, static_cast<size_t>(T), s)));
   CUtensorMap ma, mb;
   if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mb, WgT, d, f, kBK, kBN)) return TWELL_ERR_CUDA;
   GemmParams p{};
   p.M = T;
+  p.M_dev = M_dev;
   p.N = f;
   p.K = d;
   p.counts = tw->counts;
@@ -156,7 +158,7 @@ twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d
   p.nT = f / 128;
   p.W = tw->W;
   p.dev_status = dev_status;
-  return launch_gemm<kModeTwell>(ma, mb, mb, p, gemm_grid(T, f, kBN, sms), s);
+  return launch_gemm<kModeTwell>(ma, mb, mb, p, M_dev ? sms : gemm_grid(T, f, kBN, sms), s);
 }
 
 // Gate and up GEMM in one pass; TwELL of the gate pattern holding h = z * u.
@@ -325,6 +327,178 @@ twell_status dense_rows_impl(const uint16_t* x, const uint16_t* WgT, const uint1
   gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, rows, n_rows, T, xo, y, dev_status);
   TW_TRY(cuda_ok(cudaGetLastError()));
   return dense_impl(xo, T, n_rows, WgT, WuT, Wd, d, f, ho, true, rows, y, T, dev_status, s, sms);
+}
+
+// ------------------------------------------------------------------ backward
+
+// Workspace of the hybrid backward, carved in this order (each piece 256-byte
+// aligned): per-slot h, du, dz of the rows that fit ([T][nT][W] fp32 each);
+// the gathered overflow rows of x and dy ([T][d] bf16 each); their full-width
+// TwELL (counts, idx, vals, flags) and per-slot h, du, dz ([T][nT][128]); the
+// column counts/cursors ([f]), column offsets ([f + 1]) and the column-sorted
+// slot list (one uint32 per slot of both passes).
+struct BwdWorkspace {
+  float *h0, *du0, *dz0;
+  uint16_t *xo, *dyo;
+  int16_t *c1, *i1;
+  uint16_t* v1;
+  uint8_t* r1;
+  float *h1, *du1, *dz1;
+  int *colcnt, *colptr;
+  uint32_t* list;
+  size_t bytes;
+};
+
+BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
+  const size_t nT = static_cast<size_t>(f) / 128;
+  const size_t s0 = static_cast<size_t>(T) * nT * W, s1 = static_cast<size_t>(T) * nT * 128;
+  BwdWorkspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += round_up(bytes, 256);
+    return p;
+  };
+  w.h0 = reinterpret_cast<float*>(take(s0 * 4));
+  w.du0 = reinterpret_cast<float*>(take(s0 * 4));
+  w.dz0 = reinterpret_cast<float*>(take(s0 * 4));
+  w.xo = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * d * 2));
+  w.dyo = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * d * 2));
+  w.c1 = reinterpret_cast<int16_t*>(take(static_cast<size_t>(T) * nT * 2));
+  w.i1 = reinterpret_cast<int16_t*>(take(s1 * 2));
+  w.v1 = reinterpret_cast<uint16_t*>(take(s1 * 2));
+  w.r1 = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(T)));
+  w.h1 = reinterpret_cast<float*>(take(s1 * 4));
+  w.du1 = reinterpret_cast<float*>(take(s1 * 4));
+  w.dz1 = reinterpret_cast<float*>(take(s1 * 4));
+  w.colcnt = reinterpret_cast<int*>(take(static_cast<size_t>(f) * 4));
+  w.colptr = reinterpret_cast<int*>(take((static_cast<size_t>(f) + 1) * 4));
+  w.list = reinterpret_cast<uint32_t*>(take((s0 + s1) * 4));
+  w.bytes = off;
+  return w;
+}
+
+template <int NCH>
+twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(kBwdWarps) * (2 * NCH * 32 * sizeof(uint4) + kListCap * 6);
+  auto kern = bwd_token_kernel<NCH>;
+  if (smem > 48 * 1024)
+    TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
+  const long long want = (static_cast<long long>(p.rows) + kBwdWarps - 1) / kBwdWarps;
+  const int blocks = static_cast<int>(std::max(1LL, std::min<long long>(want, sms)));
+  kern<<<blocks, kBwdWarps * 32, smem, s>>>(p);
+  return cuda_ok(cudaGetLastError());
+}
+
+twell_status launch_bwd_token(const BwdParams& p, int sms, cudaStream_t s) {
+  switch ((p.d + 255) / 256) {
+    case 1: return launch_bwd_token_n<1>(p, sms, s);
+    case 2: return launch_bwd_token_n<2>(p, sms, s);
+    case 3: return launch_bwd_token_n<3>(p, sms, s);
+    case 4: return launch_bwd_token_n<4>(p, sms, s);
+    case 5: return launch_bwd_token_n<5>(p, sms, s);
+    case 6: return launch_bwd_token_n<6>(p, sms, s);
+    case 7: return launch_bwd_token_n<7>(p, sms, s);
+    case 8: return launch_bwd_token_n<8>(p, sms, s);
+    case 9: return launch_bwd_token_n<9>(p, sms, s);
+    case 10: return launch_bwd_token_n<10>(p, sms, s);
+    case 11: return launch_bwd_token_n<11>(p, sms, s);
+    case 12: return launch_bwd_token_n<12>(p, sms, s);
+    case 13: return launch_bwd_token_n<13>(p, sms, s);
+    case 14: return launch_bwd_token_n<14>(p, sms, s);
+    case 15: return launch_bwd_token_n<15>(p, sms, s);
+    case 16: return launch_bwd_token_n<16>(p, sms, s);
+    default: return TWELL_ERR_SHAPE;
+  }
+}
+
+twell_status backward_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
+                           const uint16_t* dy, int T, int d, int f, const twell_t* tw, const int32_t* ovf_rows,
+                           const int32_t* n_ovf, float* dx, float* dWgT, float* dWuT, float* dWd, char* ws,
+                           int32_t* dev_status, cudaStream_t s, int sms) {
+  const int nT = f / 128;
+  BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
+  // 1. rows that fit: per-token pass over their stored slots
+  BwdParams p0{};
+  p0.x = x;
+  p0.dy = dy;
+  p0.WgT = WgT;
+  p0.WuT = WuT;
+  p0.Wd = Wd;
+  p0.counts = tw->counts;
+  p0.idx = tw->idx;
+  p0.vals = tw->vals;
+  p0.row_ovf = tw->row_ovf;
+  p0.rows = T;
+  p0.d = d;
+  p0.f = f;
+  p0.nT = nT;
+  p0.W = tw->W;
+  p0.skip_ovf = 1;
+  p0.dx = dx;
+  p0.dx_rows = T;
+  p0.s_h = w.h0;
+  p0.s_du = w.du0;
+  p0.s_dz = w.dz0;
+  p0.dev_status = dev_status;
+  TW_TRY(launch_bwd_token(p0, sms, s));
+  // 2. overflow rows: gather x and dy, pack again at the full tile width, same pass
+  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, ovf_rows, n_ovf, T, w.xo, nullptr, dev_status);
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(dy, d, ovf_rows, n_ovf, T, w.dyo, nullptr, dev_status);
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  const twell_t tw1{w.c1, w.i1, w.v1, w.r1, T, f, 128, 128};
+  TW_TRY(gate_pack_impl(w.xo, WgT, T, d, f, &tw1, dev_status, s, sms, n_ovf));
+  BwdParams p1 = p0;
+  p1.x = w.xo;
+  p1.dy = w.dyo;
+  p1.counts = w.c1;
+  p1.idx = w.i1;
+  p1.vals = w.v1;
+  p1.row_ovf = w.r1;
+  p1.rows_dev = n_ovf;
+  p1.row_map = ovf_rows;
+  p1.W = 128;
+  p1.skip_ovf = 0;
+  p1.recompute_g = 1;
+  p1.s_h = w.h1;
+  p1.s_du = w.du1;
+  p1.s_dz = w.dz1;
+  TW_TRY(launch_bwd_token(p1, sms, s));
+  // 3. weight gradients: sort both passes' slots by column, then sum per column
+  SlotSource a{tw->counts, tw->idx, tw->row_ovf, T, nullptr, nT, tw->W, f, 1, 0u};
+  SlotSource b{w.c1, w.i1, w.r1, T, n_ovf, nT, 128, f, 0, 0x80000000u};
+  TW_TRY(cuda_ok(cudaMemsetAsync(w.colcnt, 0, static_cast<size_t>(f) * 4, s)));
+  const int cblocks = 4 * sms;
+  bwd_columns_kernel<false><<<cblocks, 256, 0, s>>>(a, w.colcnt, w.colptr, w.list);
+  bwd_columns_kernel<false><<<cblocks, 256, 0, s>>>(b, w.colcnt, w.colptr, w.list);
+  bwd_column_scan_kernel<<<1, 1024, 0, s>>>(w.colcnt, f, w.colptr);
+  bwd_columns_kernel<true><<<cblocks, 256, 0, s>>>(a, w.colcnt, w.colptr, w.list);
+  bwd_columns_kernel<true><<<cblocks, 256, 0, s>>>(b, w.colcnt, w.colptr, w.list);
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  WgradParams g{};
+  g.list = w.list;
+  g.colptr = w.colptr;
+  g.x0 = x;
+  g.dy0 = dy;
+  g.h0 = w.h0;
+  g.du0 = w.du0;
+  g.dz0 = w.dz0;
+  g.slots_per_row0 = nT * tw->W;
+  g.x1 = w.xo;
+  g.dy1 = w.dyo;
+  g.h1 = w.h1;
+  g.du1 = w.du1;
+  g.dz1 = w.dz1;
+  g.slots_per_row1 = nT * 128;
+  g.f = f;
+  g.d = d;
+  g.dWgT = dWgT;
+  g.dWuT = dWuT;
+  g.dWd = dWd;
+  const long long warps = static_cast<long long>(f) * ((d + 255) / 256);
+  bwd_wgrad_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(g);
+  return cuda_ok(cudaGetLastError());
 }
 
 }  // namespace
@@ -546,6 +720,38 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
   TW_TRY(current_device(&dev, &sms));
   return dense_impl(x, T, nullptr, W1T, nullptr, W2, d, f, static_cast<uint16_t*>(workspace), false, nullptr, y, T,
                     dev_status, static_cast<cudaStream_t>(stream), sms);
+}
+
+size_t twell_backward_workspace_bytes(int T, int d, int f, int W) {
+  if (T <= 0 || d <= 0 || f < 128 || W <= 0) return 0;
+  return bwd_carve(nullptr, T, d, f, W).bytes;
+}
+
+twell_status twell_ffn_hybrid_backward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                       const uint16_t* Wd, const uint16_t* dy, int T, int d, int f,
+                                       const twell_t* tw, const int32_t* ovf_rows, const int32_t* n_ovf, float* dx,
+                                       float* dWgT, float* dWuT, float* dWd, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  // slot indices of both passes are kept in 31 bits
+  if (static_cast<long long>(T) * (f / 128) * 128 >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  TW_TRY(check_ptrs({dWgT, dWuT, dWd, dev_status}));
+  if (T == 0) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = static_cast<size_t>(f) * d * sizeof(float);
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWgT, 0, n, s)));
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWuT, 0, n, s)));
+    return cuda_ok(cudaMemsetAsync(dWd, 0, n, s));
+  }
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, dy, ovf_rows, n_ovf, dx}));
+  if (workspace == nullptr || workspace_bytes < twell_backward_workspace_bytes(T, d, f, tw->W))
+    return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return backward_impl(x, WgT, WuT, Wd, dy, T, d, f, tw, ovf_rows, n_ovf, dx, dWgT, dWuT, dWd,
+                       static_cast<char*>(workspace), dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 
 twell_status twell_column_activity(const uint16_t* x, const uint16_t* WgT, int T, int d, int f,

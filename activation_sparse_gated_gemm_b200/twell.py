@@ -32,6 +32,7 @@ EXPORTED = (
     "twell_gate_up_pack", "twell_sparse_down", "twell_ffn_hybrid_forward_tc_up",
     "twell_relu_ffn_hybrid_forward", "twell_relu_dense_rows_forward", "twell_relu_dense_ffn_forward",
     "twell_column_activity", "twell_compact_columns", "twell_gather_rows",
+    "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -85,6 +86,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_relu_ffn_hybrid_forward": ([vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_relu_dense_rows_forward": ([vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_relu_dense_ffn_forward": ([vp, vp, vp, i32, i32, i32, vp, vp, sz, vp, vp], i32),
+        "twell_backward_workspace_bytes": ([i32, i32, i32, i32], sz),
+        "twell_ffn_hybrid_backward": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp],
+                                      i32),
         "twell_column_activity": ([vp, vp, i32, i32, i32, vp, i32, vp, vp], i32),
         "twell_compact_columns": ([vp, i32, vp, vp, vp], i32),
         "twell_gather_rows": ([vp, i32, i32, vp, vp, i32, vp, vp, vp], i32),
@@ -316,6 +320,27 @@ def relu_dense_ffn_forward(x, W1T, W2, y, workspace, dev_status, stream=None) ->
     _check("twell_relu_dense_ffn_forward", load().twell_relu_dense_ffn_forward(
         _ptr(x), _ptr(W1T), _ptr(W2), T, d, f, _ptr(y), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def backward_workspace_bytes(T: int, d: int, f: int, W: int) -> int:
+    return int(load().twell_backward_workspace_bytes(T, d, f, W))
+
+
+def ffn_hybrid_backward(x, WgT, WuT, Wd, dy, tw: Twell, ovf_rows, n_ovf, dx, dWgT, dWuT, dWd, workspace,
+                        dev_status, stream=None) -> None:
+    """Gradients of the hybrid forward (gate form) for upstream gradient dy:
+    dx [T, d] and dWgT, dWuT, dWd [f, d], all fp32 (see twell_ffn_hybrid_backward)."""
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("dy", dy, (T, d))):
+        _bf16(n, t, s)
+    for n, t, s in (("dx", dx, (T, d)), ("dWgT", dWgT, (f, d)), ("dWuT", dWuT, (f, d)), ("dWd", dWd, (f, d))):
+        _dev(n, t, s, torch.float32)
+    _check("twell_ffn_hybrid_backward", load().twell_ffn_hybrid_backward(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), _ptr(dy), T, d, f, tw.ref(), _ptr(ovf_rows), _ptr(n_ovf),
+        _ptr(dx), _ptr(dWgT), _ptr(dWuT), _ptr(dWd), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(dev_status), _stream(stream)))
 
 
 def column_activity(x, WgT, active_bits, accumulate: bool, dev_status, stream=None) -> None:

@@ -277,6 +277,35 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
                                           size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * Backward pass through the hybrid format (intellectnews.ru, "Sakana AI и
+ * NVIDIA: TwELL ...", section "Слитые CUDA-ядра для инференса и гибрид для
+ * обучения": in training, rows that are sparse enough use the compact format
+ * and rows with many active units a dense branch). For y = (ReLU(x Wg) *
+ * (x Wu)) Wd and an upstream gradient dy [T][d] (bf16):
+ *   dh_j = dy . Wd[j, :], du_j = dh_j g_j, dz_j = dh_j u_j where z_j > 0
+ *   dx [T][d] = dz Wg^T + du Wu^T           (fp32)
+ *   dWgT [f][d] = dz^T x, dWuT [f][d] = du^T x, dWd [f][d] = h^T dy   (fp32,
+ *   overwritten; the layouts of WgT, WuT and Wd)
+ * tw, ovf_rows and n_ovf are the outputs of twell_ffn_hybrid_forward on the
+ * same x (the gate form: tw's values are the bf16 gate). Rows that fit use
+ * their stored slots with the stored bf16 gate g (h = g u), so the result is
+ * the method's, within one bf16 rounding per term of the exact gradients;
+ * overflow rows are packed again at the full tile width from the gathered
+ * rows and use the gate recomputed in fp32. The weight gradients are summed
+ * per hidden unit over a column sort of the slots; the order of the terms
+ * inside a column is not fixed, so the fp32 sums are not bit-reproducible.
+ * workspace: twell_backward_workspace_bytes(T, d, f, tw->W) bytes (worst case:
+ * every row overflows). T == 0 zeroes the weight gradients. Errors as for
+ * twell_ffn_hybrid_forward; T * (f / 128) * 128 must stay below 2^31.
+ */
+size_t twell_backward_workspace_bytes(int T, int d, int f, int W);
+twell_status twell_ffn_hybrid_backward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                       const uint16_t* Wd, const uint16_t* dy, int T, int d, int f,
+                                       const twell_t* tw, const int32_t* ovf_rows, const int32_t* n_ovf,
+                                       float* dx, float* dWgT, float* dWuT, float* dWd, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * Dead hidden units (intellectnews.ru, "Sakana AI и NVIDIA: TwELL ...",
  * section "Ограничения и открытые вопросы": under the chosen L1 setting some
  * units die, i.e. are never active). Three calls compact a layer to the units

@@ -56,6 +56,7 @@ __all__ = [
     "compact_layer",
     "gated_ffn_backward",
     "hybrid_ffn_backward",
+    "hybrid_backward_weight_rows",
 ]
 
 
@@ -397,3 +398,23 @@ def hybrid_ffn_backward(x_bits, WgT_bits, WuT_bits, Wd_bits, dy_bits, tile: int,
         for k in ("dWgT", "dWuT", "dWd"):
             out[k] += dense[k]
     return out
+
+
+def hybrid_backward_weight_rows(x_bits, WgT_bits, WuT_bits, Wd_bits, dy_bits, ovf_rows, cols) -> dict:
+    """Rows `cols` of the hybrid backward's weight gradients, given the routing
+    (ovf_rows) of the whole batch: a row that fits stores every active unit,
+    with the bf16 gate, and an overflow row uses the exact gate. Needs only the
+    gate, up and down columns `cols`, so it scales to full-size batches."""
+    cols = np.asarray(cols)
+    x = bf16_bits_to_f64(x_bits)
+    dy = bf16_bits_to_f64(dy_bits)
+    z = x @ bf16_bits_to_f64(np.asarray(WgT_bits)[cols]).T
+    u = x @ bf16_bits_to_f64(np.asarray(WuT_bits)[cols]).T
+    dh = dy @ bf16_bits_to_f64(np.asarray(Wd_bits)[cols]).T
+    act = z > 0
+    g = np.where(act, bf16_bits_to_f64(f64_to_bf16_bits(np.where(act, z, 0.0))), 0.0)
+    ovf = np.asarray(ovf_rows, dtype=np.int64)
+    g[ovf] = np.where(act[ovf], z[ovf], 0.0)
+    du = dh * g
+    dz = np.where(act, dh * u, 0.0)
+    return {"dWgT": dz.T @ x, "dWuT": du.T @ x, "dWd": (g * u).T @ dy}

@@ -1,0 +1,105 @@
+"""GPU parity of the backward pass through the hybrid format against the CPU
+oracle. The forward (gate form) provides the pack and the routing; each
+gradient (dx, dWgT, dWuT, dWd) must satisfy max|g - g_ref| <= 2e-2 * rms(g_ref)
+against the oracle's result of the method. The kernels sum in fp32 what the
+oracle sums in fp64 from the same bf16 values, so a much tighter 1e-3 * rms is
+also required."""
+
+import numpy as np
+import pytest
+import torch
+
+from activation_sparse_gated_gemm_b200 import synth
+from activation_sparse_gated_gemm_b200 import twell as tl
+from oracle import twell_oracle as O
+from tests.gpu_helpers import upload
+from tests.test_gpu_parity import IDS, SMALL
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ("dx", "dWgT", "dWuT", "dWd")
+TIGHT = 1e-3
+CONTRACT = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    tl.load()
+
+
+def make_dy(T: int, d: int, seed: int) -> np.ndarray:
+    """Seeded upstream gradient, N(0, 1) rounded to bf16."""
+    rng = np.random.default_rng(1000 + seed)
+    return O.f64_to_bf16_bits(rng.standard_normal((T, d)))
+
+
+def forward_backward(L, cfg, dy_bits):
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.empty((T,), dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    dy = tl.to_device_bf16(dy_bits)
+    g = {k: torch.full((T if k == "dx" else f, d), float("nan"), dtype=torch.float32, device="cuda")
+         for k in GRADS}
+    wsb = torch.empty(tl.backward_workspace_bytes(T, d, f, W), dtype=torch.uint8, device="cuda")
+    tl.ffn_hybrid_backward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], dy, tw, ovf_rows, n_ovf,
+                           g["dx"], g["dWgT"], g["dWuT"], g["dWd"], wsb, st)
+    assert tl.status_get(st) == 0
+    n = int(n_ovf.item())
+    return {k: v.double().cpu().numpy() for k, v in g.items()}, ovf_rows[:n].cpu().numpy()
+
+
+def assert_grad_close(got: np.ndarray, ref: np.ndarray, name: str) -> None:
+    assert np.isfinite(got).all(), name
+    rms = float(np.sqrt(np.mean(ref**2)))
+    err = float(np.abs(got - ref).max())
+    assert err <= CONTRACT * rms, f"{name}: {err:.3e} > {CONTRACT} * rms {rms:.3e}"
+    assert err <= TIGHT * rms, f"{name}: {err:.3e} > {TIGHT} * rms {rms:.3e}"
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_hybrid_backward(cfg):
+    L = synth.make_layer(cfg, seed=0)
+    dy = make_dy(cfg.T, cfg.d, 0)
+    got, ovf = forward_backward(L, cfg, dy)
+    ref = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, cfg.tile, cfg.W)
+    assert np.array_equal(ovf, ref["ovf_rows"])
+    for k in GRADS:
+        assert_grad_close(got[k], ref[k], k)
+
+
+def test_backward_of_an_all_negative_gate_is_zero():
+    cfg = SMALL[1]
+    L = dict(synth.make_layer(cfg, seed=0))
+    neg = O.bf16_bits_to_f64(L["WgT"]).copy()
+    neg[:, -1] = -64.0
+    L["WgT"] = O.f64_to_bf16_bits(neg)
+    got, ovf = forward_backward(L, cfg, make_dy(cfg.T, cfg.d, 1))
+    assert ovf.size == 0
+    for k in GRADS:
+        assert not np.any(got[k]), k
+
+
+@pytest.mark.parametrize("name", ["0.5b", "2b"])
+def test_full_size_hybrid_backward(name):
+    """Full layer size: dx on sampled rows and on overflow rows, the weight
+    gradients on sampled hidden units (oracle restricted to those units)."""
+    cfg = synth.CONFIGS[name]
+    L = synth.make_layer(cfg, seed=0)
+    dy = make_dy(cfg.T, cfg.d, 2)
+    got, ovf = forward_backward(L, cfg, dy)
+    rng = np.random.default_rng(3)
+    rows = np.union1d(np.sort(rng.choice(cfg.T, size=128, replace=False)), ovf[:32])
+    ref_rows = O.hybrid_ffn_backward(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], dy[rows], cfg.tile, cfg.W)
+    assert_grad_close(got["dx"][rows], ref_rows["dx"], "dx")
+    cols = np.sort(rng.choice(cfg.f, size=48, replace=False))
+    ref_cols = O.hybrid_backward_weight_rows(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, ovf, cols)
+    for k in ("dWgT", "dWuT", "dWd"):
+        assert_grad_close(got[k][cols], ref_cols[k], k)

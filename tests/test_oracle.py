@@ -705,3 +705,15 @@ def test_hybrid_backward_within_one_rounding_of_dense():
     np.testing.assert_allclose(out["dWgT"], ref["dWgT"], rtol=1e-10, atol=1e-10 * np.abs(ref["dWgT"]).max())
     assert np.array_equal(out["dx"][out["ovf_rows"]], ref["dx"][out["ovf_rows"]])
     assert np.abs(out["dWd"] - ref["dWd"]).max() > 0  # the rounding is visible
+
+
+def test_backward_weight_rows_agree_with_the_full_hybrid_backward():
+    L = synth.make_layer(HEAVY, seed=3)
+    rng = np.random.default_rng(46)
+    dy = _rand_bf16(rng, (HEAVY.T, HEAVY.d))
+    full = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, HEAVY.tile, HEAVY.W)
+    assert len(full["ovf_rows"]) > 0
+    cols = np.sort(rng.choice(HEAVY.f, size=40, replace=False))
+    part = O.hybrid_backward_weight_rows(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, full["ovf_rows"], cols)
+    for k in ("dWgT", "dWuT", "dWd"):
+        np.testing.assert_allclose(part[k], full[k][cols], rtol=1e-11, atol=1e-11 * np.abs(full[k]).max())
