@@ -48,32 +48,110 @@ struct BwdParams {
   int* dev_status;
 };
 
-constexpr int kBwdWarps = 8;
+// Warps per block of the per-token pass: x_t, dy_t (shared memory), dx_t and
+// two weight rows (registers) per warp.
+constexpr int bwd_warps_for(int nch) { return nch <= 3 ? 12 : 8; }
+
+// For the entries s < ns of a batch (column my_j on lane s): lane s receives
+// <src, M[j_s, :]>, src being a row parked in shared memory. Two row buffers
+// alternate so the gather of entry s + 1 is in flight while entry s is reduced.
+template <int NCH>
+__device__ __forceinline__ float bwd_dot_pass(const uint4* src, const uint16_t* M, int my_j, int ns, int lane,
+                                              int d) {
+  float mine = 0.0f;
+  uint4 wa[NCH], wb[NCH];
+  load_row<NCH>(wa, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
+#pragma unroll 1
+  for (int s = 0; s < ns; s += 2) {
+    if (s + 1 < ns) load_row<NCH>(wb, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 1)) * d, lane, d);
+    {
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int i = 0; i < NCH; i += 2) {
+        mixdot8(src[i * 32 + lane], wa[i], a0, a1);
+        if (i + 1 < NCH) mixdot8(src[(i + 1) * 32 + lane], wa[i + 1], a2, a3);
+      }
+      float acc = (a0 + a1) + (a2 + a3);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == s) mine = acc;
+    }
+    if (s + 1 < ns) {
+      if (s + 2 < ns)
+        load_row<NCH>(wa, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 2)) * d, lane, d);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int i = 0; i < NCH; i += 2) {
+        mixdot8(src[i * 32 + lane], wb[i], a0, a1);
+        if (i + 1 < NCH) mixdot8(src[(i + 1) * 32 + lane], wb[i + 1], a2, a3);
+      }
+      float acc = (a0 + a1) + (a2 + a3);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == s + 1) mine = acc;
+    }
+  }
+  return mine;
+}
+
+// acc += c_s * M[j_s, :] for the entries s < ns (c_s on lane s), with the same
+// two-buffer gather.
+template <int NCH>
+__device__ __forceinline__ void bwd_axpy_pass(float (&acc)[NCH][8], const uint16_t* M, int my_j, float my_c, int ns,
+                                              int lane, int d) {
+  uint4 wa[NCH], wb[NCH];
+  load_row<NCH>(wa, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
+#pragma unroll 1
+  for (int s = 0; s < ns; s += 2) {
+    if (s + 1 < ns) load_row<NCH>(wb, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 1)) * d, lane, d);
+    const float c0 = __shfl_sync(0xffffffffu, my_c, s);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) axpy8(acc[i], c0, wa[i]);
+    if (s + 1 < ns) {
+      if (s + 2 < ns)
+        load_row<NCH>(wa, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 2)) * d, lane, d);
+      const float c1 = __shfl_sync(0xffffffffu, my_c, s + 1);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) axpy8(acc[i], c1, wb[i]);
+    }
+  }
+}
 
 // One warp per token of the pass. Shared memory per warp: x_t and dy_t
 // (NCH * 32 uint4 each), the flattened slot list (column | bf16 g << 16) and
 // the slot position of every list entry inside the row's [nT][W] block.
-template <int NCH>
-__global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_token_kernel(const BwdParams p) {
+//
+// RECOMPUTE: the gate is recomputed in fp32 (overflow rows, packed again at
+// the full tile width) instead of taken from the stored bf16 value.
+template <int NCH, int WARPS, bool RECOMPUTE>
+__global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParams p) {
   extern __shared__ uint4 bwd_smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int d = p.d;
   uint4* xs = bwd_smem + warp * 2 * NCH * 32;
   uint4* ds = xs + NCH * 32;
-  uint32_t* list = reinterpret_cast<uint32_t*>(bwd_smem + kBwdWarps * 2 * NCH * 32) + warp * kListCap;
-  uint16_t* lpos =
-      reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + kBwdWarps * 2 * NCH * 32) +
-                                  kBwdWarps * kListCap) +
-      warp * kListCap;
+  uint32_t* list = reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) + warp * kListCap;
+  uint16_t* lpos = reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) +
+                                               WARPS * kListCap) +
+                   warp * kListCap;
   const int group_tiles = max(1, kListCap / p.W);
   int rows = p.rows;
   if (p.rows_dev != nullptr) rows = min(max(*p.rows_dev, 0), rows);
   bool bad_index = false;
-  const int gw = blockIdx.x * kBwdWarps + warp;
-  const int nw = gridDim.x * kBwdWarps;
+  // tokens are handed out one at a time from a per-block counter over the
+  // block's contiguous share of the rows
+  __shared__ int next_row;
+  const int r_begin = static_cast<int>(static_cast<long long>(rows) * blockIdx.x / gridDim.x);
+  const int r_end = static_cast<int>(static_cast<long long>(rows) * (blockIdx.x + 1) / gridDim.x);
+  if (threadIdx.x == 0) next_row = r_begin;
+  __syncthreads();
 #pragma unroll 1
-  for (int t = gw; t < rows; t += nw) {
+  for (;;) {
+    int t = 0;
+    if (lane == 0) t = atomicAdd(&next_row, 1);
+    t = __shfl_sync(0xffffffffu, t, 0);
+    if (t >= r_end) break;
     if (p.skip_ovf && p.row_ovf[t]) continue;
     int r = t;
     if (p.row_map != nullptr) {
@@ -101,7 +179,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_token_kernel(const BwdP
 #pragma unroll 1
     for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
       const int c1 = min(p.nT, c0 + group_tiles);
-      // ---- flatten the stored slots of tiles [c0, c1)
+      // ---- flatten the stored slots of tiles [c0, c1), 8 slots per 16-byte load
       int total = 0;
 #pragma unroll 1
       for (int cb = c0; cb < c1; cb += 32) {
@@ -117,17 +195,28 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_token_kernel(const BwdP
         const int off = total + incl - n;
         total += __shfl_sync(0xffffffffu, incl, 31);
         const size_t base = (static_cast<size_t>(t) * p.nT + c) * p.W;
-        for (int k = 0; k < n; ++k) {
-          const int jj = p.idx[base + k];
-          uint32_t ent = static_cast<uint32_t>(jj) | (static_cast<uint32_t>(p.vals[base + k]) << 16);
-          uint16_t pos = static_cast<uint16_t>(c * p.W + k);  // < 2^15: nT * W <= 255 * 128
-          if (jj < 0 || jj >= p.f) {
-            bad_index = true;
-            ent = 0;         // read column 0 ...
-            pos |= 0x8000u;  // ... but contribute nothing and store nothing
+        for (int k = 0; k < n; k += 8) {
+          // slots past n are read but not used (k + 8 <= W)
+          const uint4 iv = ldg_nc_v4(p.idx + base + k);
+          const uint4 vv = ldg_nc_v4(p.vals + base + k);
+          const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
+          const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (k + e < n) {
+              const uint32_t jj = (e & 1) ? (iw[e >> 1] >> 16) : (iw[e >> 1] & 0xffffu);
+              const uint32_t gg = (e & 1) ? (vw[e >> 1] & 0xffff0000u) : (vw[e >> 1] << 16);
+              uint32_t ent = jj | gg;
+              uint16_t pos = static_cast<uint16_t>(c * p.W + k + e);  // < 2^15: nT * W <= 255 * 128
+              if (static_cast<int>(static_cast<int16_t>(jj)) < 0 || static_cast<int>(jj) >= p.f) {
+                bad_index = true;
+                ent = 0;         // read column 0 ...
+                pos |= 0x8000u;  // ... but contribute nothing and store nothing
+              }
+              list[off + k + e] = ent;
+              lpos[off + k + e] = pos;
+            }
           }
-          list[off + k] = ent;
-          lpos[off + k] = pos;
         }
       }
       __syncwarp();
@@ -137,39 +226,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_token_kernel(const BwdP
         const int ns = min(32, total - s0);
         const uint32_t my_e = lane < ns ? list[s0 + lane] : 0u;
         const int my_j = entry_j(my_e);
-        float my_g = entry_g(my_e), my_u = 0.0f, my_dh = 0.0f;
-        // pass 1: u_j = x . Wu[:, j], dh_j = dy . Wd[j, :] (and z_j when recomputed)
-#pragma unroll 1
-        for (int s = 0; s < ns; ++s) {
-          const int j = __shfl_sync(0xffffffffu, my_j, s);
-          const uint16_t* wu = p.WuT + static_cast<size_t>(j) * d;
-          const uint16_t* wd = p.Wd + static_cast<size_t>(j) * d;
-          const uint16_t* wg = p.WgT + static_cast<size_t>(j) * d;
-          float au0 = 0.f, au1 = 0.f, ah0 = 0.f, ah1 = 0.f, az0 = 0.f, az1 = 0.f;
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            const int k0 = (i * 32 + lane) * 8;
-            if (k0 < d) {
-              mixdot8(xs[i * 32 + lane], ldg_nc_v4(wu + k0), au0, au1);
-              mixdot8(ds[i * 32 + lane], ldg_nc_v4(wd + k0), ah0, ah1);
-              if (p.recompute_g) mixdot8(xs[i * 32 + lane], ldg_nc_v4(wg + k0), az0, az1);
-            }
-          }
-          float au = au0 + au1, ah = ah0 + ah1, az = az0 + az1;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            au += __shfl_xor_sync(0xffffffffu, au, o);
-            ah += __shfl_xor_sync(0xffffffffu, ah, o);
-            if (p.recompute_g) az += __shfl_xor_sync(0xffffffffu, az, o);
-          }
-          if (lane == s) {
-            my_u = au;
-            my_dh = ah;
-            if (p.recompute_g) my_g = fmaxf(az, 0.0f);
-          }
-        }
         const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
         const bool valid = (my_pos & 0x8000u) == 0;
+        // u_j = x . Wu[:, j], dh_j = dy . Wd[j, :] (and z_j when recomputed)
+        const float my_u = bwd_dot_pass<NCH>(xs, p.WuT, my_j, ns, lane, d);
+        const float my_dh = bwd_dot_pass<NCH>(ds, p.Wd, my_j, ns, lane, d);
+        float my_g = entry_g(my_e);
+        if (RECOMPUTE) my_g = fmaxf(bwd_dot_pass<NCH>(xs, p.WgT, my_j, ns, lane, d), 0.0f);
         const float my_du = valid ? my_dh * my_g : 0.0f;
         const float my_dz = valid ? my_dh * my_u : 0.0f;
         if (valid) {
@@ -178,23 +241,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_token_kernel(const BwdP
           p.s_du[slot] = my_du;
           p.s_dz[slot] = my_dz;
         }
-        // pass 2: dx_t += dz_j Wg[:, j] + du_j Wu[:, j]
-#pragma unroll 1
-        for (int s = 0; s < ns; ++s) {
-          const int j = __shfl_sync(0xffffffffu, my_j, s);
-          const float dz = __shfl_sync(0xffffffffu, my_dz, s);
-          const float du = __shfl_sync(0xffffffffu, my_du, s);
-          const uint16_t* wg = p.WgT + static_cast<size_t>(j) * d;
-          const uint16_t* wu = p.WuT + static_cast<size_t>(j) * d;
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            const int k0 = (i * 32 + lane) * 8;
-            if (k0 < d) {
-              axpy8(acc[i], dz, ldg_nc_v4(wg + k0));
-              axpy8(acc[i], du, ldg_nc_v4(wu + k0));
-            }
-          }
-        }
+        // dx_t += dz_j Wg[:, j] + du_j Wu[:, j]
+        bwd_axpy_pass<NCH>(acc, p.WgT, my_j, my_dz, ns, lane, d);
+        bwd_axpy_pass<NCH>(acc, p.WuT, my_j, my_du, ns, lane, d);
       }
       __syncwarp();
     }

@@ -380,13 +380,14 @@ BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
 
 template <int NCH>
 twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(kBwdWarps) * (2 * NCH * 32 * sizeof(uint4) + kListCap * 6);
-  auto kern = bwd_token_kernel<NCH>;
+  constexpr int kWarps = bwd_warps_for(NCH);
+  const size_t smem = static_cast<size_t>(kWarps) * (2 * NCH * 32 * sizeof(uint4) + kListCap * 6);
+  auto kern = p.recompute_g ? bwd_token_kernel<NCH, kWarps, true> : bwd_token_kernel<NCH, kWarps, false>;
   if (smem > 48 * 1024)
     TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
-  const long long want = (static_cast<long long>(p.rows) + kBwdWarps - 1) / kBwdWarps;
+  const long long want = (static_cast<long long>(p.rows) + kWarps - 1) / kWarps;
   const int blocks = static_cast<int>(std::max(1LL, std::min<long long>(want, sms)));
-  kern<<<blocks, kBwdWarps * 32, smem, s>>>(p);
+  kern<<<blocks, kWarps * 32, smem, s>>>(p);
   return cuda_ok(cudaGetLastError());
 }
 
@@ -412,10 +413,11 @@ twell_status launch_bwd_token(const BwdParams& p, int sms, cudaStream_t s) {
   }
 }
 
-twell_status backward_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
-                           const uint16_t* dy, int T, int d, int f, const twell_t* tw, const int32_t* ovf_rows,
-                           const int32_t* n_ovf, float* dx, float* dWgT, float* dWuT, float* dWd, char* ws,
-                           int32_t* dev_status, cudaStream_t s, int sms) {
+// dx, and the per-slot scalars of both passes in the workspace.
+twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
+                              const uint16_t* dy, int T, int d, int f, const twell_t* tw, const int32_t* ovf_rows,
+                              const int32_t* n_ovf, float* dx, char* ws, int32_t* dev_status, cudaStream_t s,
+                              int sms) {
   const int nT = f / 128;
   BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
   // 1. rows that fit: per-token pass over their stored slots
@@ -464,7 +466,15 @@ twell_status backward_impl(const uint16_t* x, const uint16_t* WgT, const uint16_
   p1.s_h = w.h1;
   p1.s_du = w.du1;
   p1.s_dz = w.dz1;
-  TW_TRY(launch_bwd_token(p1, sms, s));
+  return launch_bwd_token(p1, sms, s);
+}
+
+// Weight gradients from the workspace filled by backward_dx_impl.
+twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int d, int f, const twell_t* tw,
+                              const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd, char* ws, cudaStream_t s,
+                              int sms) {
+  const int nT = f / 128;
+  BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
   // 3. weight gradients: sort both passes' slots by column, then sum per column
   SlotSource a{tw->counts, tw->idx, tw->row_ovf, T, nullptr, nT, tw->W, f, 1, 0u};
   SlotSource b{w.c1, w.i1, w.r1, T, n_ovf, nT, 128, f, 0, 0x80000000u};
@@ -750,8 +760,53 @@ twell_status twell_ffn_hybrid_backward(const uint16_t* x, const uint16_t* WgT, c
   if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  return backward_impl(x, WgT, WuT, Wd, dy, T, d, f, tw, ovf_rows, n_ovf, dx, dWgT, dWuT, dWd,
-                       static_cast<char*>(workspace), dev_status, static_cast<cudaStream_t>(stream), sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  TW_TRY(backward_dx_impl(x, WgT, WuT, Wd, dy, T, d, f, tw, ovf_rows, n_ovf, dx, ws, dev_status, s, sms));
+  return backward_dw_impl(x, dy, T, d, f, tw, n_ovf, dWgT, dWuT, dWd, ws, s, sms);
+}
+
+twell_status twell_ffn_hybrid_backward_dx(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                          const uint16_t* Wd, const uint16_t* dy, int T, int d, int f,
+                                          const twell_t* tw, const int32_t* ovf_rows, const int32_t* n_ovf,
+                                          float* dx, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                          void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (static_cast<long long>(T) * (f / 128) * 128 >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, dy, ovf_rows, n_ovf, dx, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_backward_workspace_bytes(T, d, f, tw->W))
+    return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return backward_dx_impl(x, WgT, WuT, Wd, dy, T, d, f, tw, ovf_rows, n_ovf, dx, static_cast<char*>(workspace),
+                          dev_status, static_cast<cudaStream_t>(stream), sms);
+}
+
+twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy, int T, int d, int f,
+                                          const twell_t* tw, const int32_t* n_ovf, float* dWgT, float* dWuT,
+                                          float* dWd, void* workspace, size_t workspace_bytes, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (static_cast<long long>(T) * (f / 128) * 128 >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  TW_TRY(check_ptrs({dWgT, dWuT, dWd}));
+  if (T == 0) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = static_cast<size_t>(f) * d * sizeof(float);
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWgT, 0, n, s)));
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWuT, 0, n, s)));
+    return cuda_ok(cudaMemsetAsync(dWd, 0, n, s));
+  }
+  TW_TRY(check_ptrs({x, dy, n_ovf}));
+  if (workspace == nullptr || workspace_bytes < twell_backward_workspace_bytes(T, d, f, tw->W))
+    return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return backward_dw_impl(x, dy, T, d, f, tw, n_ovf, dWgT, dWuT, dWd, static_cast<char*>(workspace),
+                          static_cast<cudaStream_t>(stream), sms);
 }
 
 twell_status twell_column_activity(const uint16_t* x, const uint16_t* WgT, int T, int d, int f,

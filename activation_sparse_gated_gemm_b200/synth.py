@@ -212,3 +212,10 @@ def _inv_cdf_vec(q: np.ndarray) -> np.ndarray:
     from scipy.special import ndtri
 
     return ndtri(q)
+
+
+def make_dy(T: int, d: int, seed: int = 0) -> np.ndarray:
+    """Seeded upstream gradient for the backward pass, [T, d]: N(0, 1) drawn
+    in fp32 and rounded to bf16 (uint16 bit patterns)."""
+    rng = np.random.default_rng(1000 + seed)
+    return f32_to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))

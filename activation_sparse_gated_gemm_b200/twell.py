@@ -32,7 +32,8 @@ EXPORTED = (
     "twell_gate_up_pack", "twell_sparse_down", "twell_ffn_hybrid_forward_tc_up",
     "twell_relu_ffn_hybrid_forward", "twell_relu_dense_rows_forward", "twell_relu_dense_ffn_forward",
     "twell_column_activity", "twell_compact_columns", "twell_gather_rows",
-    "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward",
+    "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward", "twell_ffn_hybrid_backward_dx",
+    "twell_ffn_hybrid_backward_dw",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -89,6 +90,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_backward_workspace_bytes": ([i32, i32, i32, i32], sz),
         "twell_ffn_hybrid_backward": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp],
                                       i32),
+        "twell_ffn_hybrid_backward_dx": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
+        "twell_ffn_hybrid_backward_dw": ([vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, sz, vp], i32),
         "twell_column_activity": ([vp, vp, i32, i32, i32, vp, i32, vp, vp], i32),
         "twell_compact_columns": ([vp, i32, vp, vp, vp], i32),
         "twell_gather_rows": ([vp, i32, i32, vp, vp, i32, vp, vp, vp], i32),
@@ -341,6 +344,31 @@ def ffn_hybrid_backward(x, WgT, WuT, Wd, dy, tw: Twell, ovf_rows, n_ovf, dx, dWg
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), _ptr(dy), T, d, f, tw.ref(), _ptr(ovf_rows), _ptr(n_ovf),
         _ptr(dx), _ptr(dWgT), _ptr(dWuT), _ptr(dWd), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _ptr(dev_status), _stream(stream)))
+
+
+def ffn_hybrid_backward_dx(x, WgT, WuT, Wd, dy, tw: Twell, ovf_rows, n_ovf, dx, workspace, dev_status,
+                           stream=None) -> None:
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("dy", dy, (T, d))):
+        _bf16(n, t, s)
+    _dev("dx", dx, (T, d), torch.float32)
+    _check("twell_ffn_hybrid_backward_dx", load().twell_ffn_hybrid_backward_dx(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), _ptr(dy), T, d, f, tw.ref(), _ptr(ovf_rows), _ptr(n_ovf),
+        _ptr(dx), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def ffn_hybrid_backward_dw(x, dy, tw: Twell, n_ovf, dWgT, dWuT, dWd, workspace, stream=None) -> None:
+    T, d = x.shape
+    f = tw.f
+    _bf16("x", x, (T, d))
+    _bf16("dy", dy, (T, d))
+    for n, t in (("dWgT", dWgT), ("dWuT", dWuT), ("dWd", dWd)):
+        _dev(n, t, (f, d), torch.float32)
+    _check("twell_ffn_hybrid_backward_dw", load().twell_ffn_hybrid_backward_dw(
+        _ptr(x), _ptr(dy), T, d, f, tw.ref(), _ptr(n_ovf), _ptr(dWgT), _ptr(dWuT), _ptr(dWd), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def column_activity(x, WgT, active_bits, accumulate: bool, dev_status, stream=None) -> None:

@@ -37,6 +37,7 @@ from activation_sparse_gated_gemm_b200 import synth  # noqa: E402
 
 METRIC = "sparse gated-FFN tokens/s"
 METRIC_RELU = "sparse non-gated ReLU-FFN tokens/s"
+METRIC_BWD = "sparse gated-FFN backward tokens/s"
 FLUSH_BYTES = 256 << 20
 FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM (4 sub-partitions x 32)
 DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
@@ -207,29 +208,34 @@ def blas_threads() -> int:
 # ---------------------------------------------------------------- CPU oracle
 
 
-def oracle_step(cfg, L, rows, layer: str) -> None:
-    """One hybrid forward of the oracle as it stands on the given rows."""
+def oracle_step(cfg, L, rows, layer: str, dy=None) -> None:
+    """One hybrid forward (or backward, given dy) of the oracle as it stands on the given rows."""
     from oracle import twell_oracle as O
 
-    if layer == "relu":
+    if dy is not None:
+        O.hybrid_ffn_backward(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], dy[rows], cfg.tile, cfg.W)
+    elif layer == "relu":
         O.hybrid_relu_ffn(L["x"][rows], L["WgT"], L["Wd"], cfg.tile, cfg.W)
     else:
         O.hybrid_ffn(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], cfg.tile, cfg.W)
 
 
-def cpu_oracle_rate(cfg, L, sample_rows: int, layer: str = "gated", max_seconds: float = 25.0) -> dict:
+def cpu_oracle_rate(cfg, L, sample_rows: int, layer: str = "gated", max_seconds: float = 25.0,
+                    dy=None) -> dict:
     """The oracle as it stands (hybrid forward: fp64 gate, pack, route,
-    per-token sparse step, dense rows) on the first rows of the workload."""
+    per-token sparse step, dense rows; or the hybrid backward when dy is given)
+    on the first rows of the workload."""
     n = min(sample_rows, cfg.T)
     done, t0 = 0, time.perf_counter()
     while done < n and time.perf_counter() - t0 < max_seconds:
         chunk = min(128, n - done)
-        oracle_step(cfg, L, slice(done, done + chunk), layer)
+        oracle_step(cfg, L, slice(done, done + chunk), layer, dy)
         done += chunk
     dt = time.perf_counter() - t0
+    what = "hybrid backward" if dy is not None else "gate, pack, route, sparse step, dense rows"
     return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"first {done} of {cfg.T} tokens of the {cfg.name} {layer} layer, fp64 numpy oracle "
-                      f"(gate, pack, route, sparse step, dense rows), {dt:.1f} s"}
+                      f"({what}), {dt:.1f} s"}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -480,6 +486,149 @@ def run_gpu(args, world, rank, local):
     return res
 
 
+def run_gpu_backward(args, world, rank, local):
+    """The backward pass through the hybrid format: dx (per-token sparse pass,
+    overflow rows repacked at full width) then the weight gradients (column
+    sort, per-unit sums). The forward that produces the pack and the routing
+    runs once before timing: its outputs are the backward's inputs."""
+    import torch
+
+    from activation_sparse_gated_gemm_b200 import twell as tl
+
+    tl.load()
+    dev = torch.device("cuda", local)
+    cfg = synth.CONFIGS[args.config]
+    L = synth.make_layer(cfg, seed=args.seed)
+    dy_bits = synth.make_dy(cfg.T, cfg.d, args.seed)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    x = tl.to_device_bf16(L["x"], dev)
+    WgT = tl.to_device_bf16(L["WgT"], dev)
+    WuT = tl.to_device_bf16(L["WuT"], dev)
+    Wd = tl.to_device_bf16(L["Wd"], dev)
+    dy = tl.to_device_bf16(dy_bits, dev)
+    tw = tl.Twell(T, f, W, device=dev)
+    y = torch.empty((T, d), dtype=torch.float32, device=dev)
+    ovf_rows = torch.empty((T,), dtype=torch.int32, device=dev)
+    n_ovf = torch.zeros((1,), dtype=torch.int32, device=dev)
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device=dev)
+    st = tl.new_status(dev)
+    tl.ffn_hybrid_forward(x, WgT, WuT, Wd, tw, y, ovf_rows, n_ovf, ws, st)
+    del ws
+    dx = torch.empty((T, d), dtype=torch.float32, device=dev)
+    dW = [torch.empty((f, d), dtype=torch.float32, device=dev) for _ in range(3)]
+    wsb = torch.empty(tl.backward_workspace_bytes(T, d, f, W), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    K, Wm = args.steps, args.warmup
+
+    def stage_dx():
+        tl.ffn_hybrid_backward_dx(x, WgT, WuT, Wd, dy, tw, ovf_rows, n_ovf, dx, wsb, st)
+
+    def stage_dw():
+        tl.ffn_hybrid_backward_dw(x, dy, tw, n_ovf, dW[0], dW[1], dW[2], wsb)
+
+    for _ in range(Wm):
+        flush.zero_()
+        stage_dx()
+        stage_dw()
+    torch.cuda.synchronize(dev)
+    if tl.status_get(st) != 0:
+        raise RuntimeError(f"device status {tl.status_get(st)} after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for k in range(K):
+            flush.zero_()
+            evs[k][0].record(stream)
+            stage_dx()
+            evs[k][1].record(stream)
+            stage_dw()
+            evs[k][2].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(2)] for k in range(K)])
+    stage_ms = per.mean(axis=0)
+    step_ms = max_over_ranks(float(per.sum(axis=1).mean()), world)
+
+    # e2e through the C ABI: dy from pinned host memory in, dx and the weight gradients out
+    dy_host = dy.cpu().pin_memory()
+    dx_host = torch.empty((T, d), dtype=torch.float32).pin_memory()
+    dW_host = [torch.empty((f, d), dtype=torch.float32).pin_memory() for _ in range(3)]
+
+    def e2e_step():
+        dy.copy_(dy_host, non_blocking=True)
+        tl.ffn_hybrid_backward(x, WgT, WuT, Wd, dy, tw, ovf_rows, n_ovf, dx, dW[0], dW[1], dW[2], wsb, st)
+        dx_host.copy_(dx, non_blocking=True)
+        for h, g in zip(dW_host, dW):
+            h.copy_(g, non_blocking=True)
+
+    for _ in range(max(1, Wm // 2)):
+        e2e_step()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for k in range(K):
+        flush.zero_()
+        e2e_ev[k][0].record(stream)
+        e2e_step()
+        e2e_ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in e2e_ev])), world)
+    status = tl.status_get(st)
+    if status != 0:
+        raise RuntimeError(f"device status {status} ({tl.status_str(status)})")
+
+    counts = tw.counts.to(torch.int64)
+    ovf_mask = tw.row_ovf.bool()
+    n_ovf_h = int(n_ovf.item())
+    nnz_fit = int(torch.clamp(counts, max=W)[~ovf_mask].sum())
+    nnz_ovf = int(counts[ovf_mask].sum())  # true counts: every active unit of an overflow row
+    flops_dx = 8.0 * d * nnz_fit + 10.0 * d * nnz_ovf  # u, dh (and z) dots, two axpys per unit
+    flops_dw = 6.0 * d * (nnz_fit + nnz_ovf)           # three axpys per unit
+    clocks = sampler.summary()
+    peaks = load_peaks()
+    fp32_peak = (torch.cuda.get_device_properties(dev).multi_processor_count * FP32_LANES_PER_SM * 2
+                 * (clocks["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6)
+    names = ["backward_dx", "backward_dw"]
+    work = {"backward_dx": flops_dx, "backward_dw": flops_dw}
+    dom = names[int(np.argmax(stage_ms))]
+    ms = float(stage_ms[names.index(dom)])
+    achieved = work[dom] / (ms * 1e-3) / 1e12
+    res = {
+        "metric": METRIC_BWD,
+        "value": job_rate(T, world, step_ms),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded generator; no dataset or trained weights)",
+        "config": {"workload": f"{cfg.name}-like FFN layer backward through the hybrid TwELL format",
+                   "tokens": T, "d": d, "f": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
+                   "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "roofline": {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": fp32_peak / 1e12,
+                     "unit": "TFLOP/s", "frac": achieved / (fp32_peak / 1e12), "traffic": None,
+                     "peak_source": "fp32 FMA lanes x 2 x max SM clock"},
+        "stages_ms": {n: float(v) for n, v in zip(names, stage_ms)},
+        "batch_stats": {"n_ovf": n_ovf_h, "nnz_fit_rows": nnz_fit, "nnz_overflow_rows": nnz_ovf},
+        "dense_backward_ms": None,
+        "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
+        "gpu_launches": 11 * K,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_oracle_rate(cfg, L, max(128, args.cpu_sample // 8), "gated", dy=dy_bits)
+    return res
+
+
 # ---------------------------------------------------------------- reference arm
 
 
@@ -492,9 +641,13 @@ def run_reference(args, world, rank):
     L = synth.make_layer(cfg, seed=args.seed)
     sample = max(1, min(cfg.T, args.cpu_sample // 16))
     layer = "relu" if args.layer == "relu" else "gated"
+    backward = args.pass_ == "backward"
+    dy = synth.make_dy(cfg.T, cfg.d, args.seed) if backward else None
+    if backward:
+        sample = max(1, sample // 4)
 
     def step():
-        oracle_step(cfg, L, slice(0, sample), layer)
+        oracle_step(cfg, L, slice(0, sample), layer, dy)
 
     for _ in range(args.warmup):
         step()
@@ -505,11 +658,14 @@ def run_reference(args, world, rank):
     v = sample / dt
     return {
         "impl": "reference",
-        "metric": METRIC_RELU if layer == "relu" else METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC_BWD if backward else (METRIC_RELU if layer == "relu" else METRIC), "value": v,
+        "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
-        "config": {"workload": (f"{cfg.name}-like non-gated ReLU FFN layer forward (W1 = Wg, W2 = Wd), "
+        "config": {"workload": (f"{cfg.name}-like FFN layer backward through the hybrid TwELL format"
+                                if backward else
+                                f"{cfg.name}-like non-gated ReLU FFN layer forward (W1 = Wg, W2 = Wd), "
                                 "hybrid TwELL" if layer == "relu" else
                                 f"{cfg.name}-like FFN layer forward, hybrid TwELL"), "tokens": cfg.T,
                    "d": cfg.d, "f": cfg.f, "tile": cfg.tile, "ell_width": cfg.W,
@@ -619,6 +775,8 @@ def main(argv=None):
                     help="hybrid form: gate (sparse up+down) or tc_up (up on tensor cores); auto times both")
     ap.add_argument("--layer", default="gated", choices=["gated", "relu"],
                     help="gated: (ReLU(x Wg) * x Wu) Wd; relu: the non-gated ReLU(x W1) W2")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
+                    help="forward (the default) or the backward pass through the hybrid format")
     ap.add_argument("--compact", action="store_true",
                     help="drop the hidden units the batch never activates before timing")
     ap.add_argument("--sweep", action="store_true", help="density x batch sweep, one JSON line per point")
@@ -641,7 +799,7 @@ def main(argv=None):
 
     world, rank, local = dist_setup(args)
     try:
-        res = run_gpu(args, world, rank, local)
+        res = (run_gpu_backward if args.pass_ == "backward" else run_gpu)(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

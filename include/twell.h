@@ -306,6 +306,23 @@ twell_status twell_ffn_hybrid_backward(const uint16_t* x, const uint16_t* WgT, c
                                        size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * The two halves of twell_ffn_hybrid_backward, for callers that want dx early
+ * (to go on with the previous layer's backward while the weight gradients are
+ * summed, e.g. on another stream ordered after this one). _dx writes dx and
+ * leaves per-slot scalars in the workspace; _dw reads them and writes the
+ * weight gradients, and must see the same workspace, x, dy, tw and n_ovf,
+ * stream-ordered after _dx with nothing in between that writes them.
+ */
+twell_status twell_ffn_hybrid_backward_dx(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                          const uint16_t* Wd, const uint16_t* dy, int T, int d, int f,
+                                          const twell_t* tw, const int32_t* ovf_rows, const int32_t* n_ovf,
+                                          float* dx, void* workspace, size_t workspace_bytes,
+                                          int32_t* dev_status, void* stream);
+twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy, int T, int d, int f,
+                                          const twell_t* tw, const int32_t* n_ovf, float* dWgT, float* dWuT,
+                                          float* dWd, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dead hidden units (intellectnews.ru, "Sakana AI и NVIDIA: TwELL ...",
  * section "Ограничения и открытые вопросы": under the chosen L1 setting some
  * units die, i.e. are never active). Three calls compact a layer to the units

@@ -30,9 +30,7 @@ def _lib():
 
 
 def make_dy(T: int, d: int, seed: int) -> np.ndarray:
-    """Seeded upstream gradient, N(0, 1) rounded to bf16."""
-    rng = np.random.default_rng(1000 + seed)
-    return O.f64_to_bf16_bits(rng.standard_normal((T, d)))
+    return synth.make_dy(T, d, seed)
 
 
 def forward_backward(L, cfg, dy_bits):
@@ -103,3 +101,31 @@ def test_full_size_hybrid_backward(name):
     ref_cols = O.hybrid_backward_weight_rows(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, ovf, cols)
     for k in ("dWgT", "dWuT", "dWd"):
         assert_grad_close(got[k][cols], ref_cols[k], k)
+
+
+def test_split_backward_matches_the_oracle():
+    """dx first, weight gradients afterwards, through the two-call form."""
+    cfg = SMALL[4]  # heavy tokens: both passes have work
+    L = synth.make_layer(cfg, seed=0)
+    dy_bits = make_dy(cfg.T, cfg.d, 4)
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.empty((T,), dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    dy = tl.to_device_bf16(dy_bits)
+    dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    dW = [torch.empty((f, d), dtype=torch.float32, device="cuda") for _ in range(3)]
+    wsb = torch.empty(tl.backward_workspace_bytes(T, d, f, W), dtype=torch.uint8, device="cuda")
+    tl.ffn_hybrid_backward_dx(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], dy, tw, ovf_rows, n_ovf, dx, wsb, st)
+    tl.ffn_hybrid_backward_dw(dev["x"], dy, tw, n_ovf, dW[0], dW[1], dW[2], wsb)
+    assert tl.status_get(st) == 0
+    ref = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy_bits, cfg.tile, cfg.W)
+    assert int(n_ovf.item()) > 0
+    assert_grad_close(dx.double().cpu().numpy(), ref["dx"], "dx")
+    for k, t in zip(("dWgT", "dWuT", "dWd"), dW):
+        assert_grad_close(t.double().cpu().numpy(), ref[k], k)
