@@ -326,7 +326,13 @@ __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf,
 // (read with one 16-byte load when they are in range), counts its own, and a
 // block-wide scan gives every thread the position of its first flagged row,
 // so the list comes out in ascending order.
-__global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf) {
+//
+// With xo given (small batches), the same block then gathers the listed rows
+// of x into xo and zeroes them in y_zero, which saves the separate gather
+// launch of the dense branch.
+__global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf,
+                                                     const uint16_t* x = nullptr, int d = 0, uint16_t* xo = nullptr,
+                                                     float* y_zero = nullptr) {
   __shared__ int warp_off[32];
   __shared__ int total_s;
   const int lane = threadIdx.x & 31;
@@ -376,6 +382,18 @@ __global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int
     __syncthreads();
   }
   if (threadIdx.x == 0) *n_ovf = base;
+  if (xo == nullptr) return;
+  __syncthreads();  // the list written above is read back by the whole block
+  const int vecs = d / 8;
+  for (int e = threadIdx.x; e < base * vecs; e += 1024) {
+    const int i = e / vecs, k = e - i * vecs;
+    const int r = ovf_rows[i];
+    reinterpret_cast<uint4*>(xo + static_cast<size_t>(i) * d)[k] =
+        reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * d)[k];
+    float4* yz = reinterpret_cast<float4*>(y_zero + static_cast<size_t>(r) * d);
+    yz[2 * k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    yz[2 * k + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 // out[i, :] = x[rows[i], :] for i < *n_rows (clamped to T, the room in rows and
@@ -497,6 +515,83 @@ __global__ void gather_weight_rows_kernel(const uint16_t* __restrict__ W, int f,
       const uint4* s4 = reinterpret_cast<const uint4*>(W + static_cast<size_t>(src) * d);
       for (int v = lane; v < vecs; v += 32) dst[v] = __ldg(s4 + v);
     }
+  }
+}
+
+// ---------------------------------------------------------------- small batches
+
+// TwELL pack from fp32 gate pre-activations z [T][f] (the split-K gate GEMM of
+// a small batch): one warp per (row, tile), lane l holding columns 4l..4l+3 of
+// the tile; the positive ones are placed in ascending column order by a warp
+// prefix sum of the per-lane counts. Same output as the GEMM epilogue: the
+// true count, the first W (column, bf16 value) slots, the overflow flag (set
+// only; row_ovf must start at zero). When y_zero is given, its T x d entries
+// are zeroed first (for the sparse step's split-unit partial sums).
+__global__ void __launch_bounds__(256) pack_f32_kernel(const float* __restrict__ z, int T, int f, int W,
+                                                       int16_t* __restrict__ counts, int16_t* __restrict__ idx,
+                                                       uint16_t* __restrict__ vals, uint8_t* __restrict__ row_ovf,
+                                                       float* __restrict__ y_zero, int d) {
+  if (y_zero != nullptr) {
+    const size_t n4 = static_cast<size_t>(T) * d / 4;
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+      reinterpret_cast<float4*>(y_zero)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int nT = f / 128;
+  const int lane = threadIdx.x & 31;
+  const long long pairs = static_cast<long long>(T) * nT;
+  for (long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); w < pairs;
+       w += static_cast<long long>(gridDim.x) * 8) {
+    const int t = static_cast<int>(w / nT);
+    const int c = static_cast<int>(w - static_cast<long long>(t) * nT);
+    const float4 v = reinterpret_cast<const float4*>(z + static_cast<size_t>(t) * f + c * 128)[lane];
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m |= (vv[k] > 0.0f ? 1u : 0u) << k;
+    const int n = __popc(m);
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int s = incl - n;
+    const size_t slot0 = static_cast<size_t>(w) * W;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if ((m >> k) & 1u) {
+        if (s < W) {
+          idx[slot0 + s] = static_cast<int16_t>(c * 128 + 4 * lane + k);
+          vals[slot0 + s] = f32_to_bf16_bits(vv[k]);
+        }
+        ++s;
+      }
+    }
+    if (lane == 0) {
+      counts[w] = static_cast<int16_t>(total);
+      if (total > W) row_ovf[t] = 1;
+    }
+  }
+}
+
+// h [T][f] = bf16(ReLU(z) * u) from zu [T][2f] = [z | u] in fp32 (the first
+// half of the dense layer for a small batch), or bf16(ReLU(z)) from z [T][f]
+// when not gated.
+__global__ void h_from_zu_kernel(const float* __restrict__ zu, int T, int f, int gated, uint16_t* __restrict__ h) {
+  const size_t per_row = static_cast<size_t>(f) / 4;
+  const size_t n = static_cast<size_t>(T) * per_row;
+  const size_t ldz = gated ? 2 * static_cast<size_t>(f) : static_cast<size_t>(f);
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t t = i / per_row, q = i - t * per_row;
+    const float4 z = reinterpret_cast<const float4*>(zu + t * ldz)[q];
+    const float4 u = gated ? reinterpret_cast<const float4*>(zu + t * ldz + f)[q] : make_float4(1.f, 1.f, 1.f, 1.f);
+    uint2 o;
+    o.x = pack_bf16x2(fmaxf(z.x, 0.f) * u.x, fmaxf(z.y, 0.f) * u.y);
+    o.y = pack_bf16x2(fmaxf(z.z, 0.f) * u.z, fmaxf(z.w, 0.f) * u.w);
+    reinterpret_cast<uint2*>(h + t * f)[q] = o;
   }
 }
 

@@ -182,8 +182,16 @@ twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uin
   return launch_gemm<kModeTwellHidden>(ma, mg, mu, p, gemm_grid(T, f, 128, sms), s);
 }
 
+// Whether the sparse step spreads tokens over several warps (with partial
+// sums added into a zeroed y): when the batch has fewer tokens than twice the
+// resident warps.
+bool sparse_splits_units(int T, int d, bool down_only, int sms) {
+  const int nch = (d + 255) / 256;
+  return static_cast<long long>(T) * 2 < static_cast<long long>(sparse_warps_for(nch, down_only)) * sms;
+}
+
 template <int NCH, bool DOWN_ONLY>
-twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s) {
+twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s, bool y_zeroed) {
   constexpr int kWarps = sparse_warps_for(NCH, DOWN_ONLY);
   // With fewer tokens than resident warps, a token's column tiles are spread
   // over several warps whose partial sums are added into a zeroed y (rows that
@@ -194,7 +202,7 @@ twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s) {
     const long long want_units = warps_resident;  // about one unit per resident warp
     const long long per_token = std::max(1LL, std::min<long long>(p.nT, want_units / std::max(1, p.T)));
     p.unit_tiles = static_cast<int>((p.nT + per_token - 1) / per_token);
-    if (p.unit_tiles < p.nT) {
+    if (p.unit_tiles < p.nT && !y_zeroed) {
       zero_rows_kernel<<<std::min(p.T, 4 * sms), 256, 0, s>>>(p.y, p.T, p.d, p.row_ovf, p.skip_ovf);
       TW_TRY(cuda_ok(cudaGetLastError()));
     }
@@ -210,32 +218,32 @@ twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s) {
 }
 
 template <bool DOWN_ONLY>
-twell_status sparse_launch(const SparseParams& p, int d, int sms, cudaStream_t s) {
+twell_status sparse_launch(const SparseParams& p, int d, int sms, cudaStream_t s, bool y_zeroed) {
   // (the launcher decides how a token's column tiles are split over warps)
   switch ((d + 255) / 256) {
-    case 1: return launch_sparse_n<1, DOWN_ONLY>(p, sms, s);
-    case 2: return launch_sparse_n<2, DOWN_ONLY>(p, sms, s);
-    case 3: return launch_sparse_n<3, DOWN_ONLY>(p, sms, s);
-    case 4: return launch_sparse_n<4, DOWN_ONLY>(p, sms, s);
-    case 5: return launch_sparse_n<5, DOWN_ONLY>(p, sms, s);
-    case 6: return launch_sparse_n<6, DOWN_ONLY>(p, sms, s);
-    case 7: return launch_sparse_n<7, DOWN_ONLY>(p, sms, s);
-    case 8: return launch_sparse_n<8, DOWN_ONLY>(p, sms, s);
-    case 9: return launch_sparse_n<9, DOWN_ONLY>(p, sms, s);
-    case 10: return launch_sparse_n<10, DOWN_ONLY>(p, sms, s);
-    case 11: return launch_sparse_n<11, DOWN_ONLY>(p, sms, s);
-    case 12: return launch_sparse_n<12, DOWN_ONLY>(p, sms, s);
-    case 13: return launch_sparse_n<13, DOWN_ONLY>(p, sms, s);
-    case 14: return launch_sparse_n<14, DOWN_ONLY>(p, sms, s);
-    case 15: return launch_sparse_n<15, DOWN_ONLY>(p, sms, s);
-    case 16: return launch_sparse_n<16, DOWN_ONLY>(p, sms, s);
+    case 1: return launch_sparse_n<1, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 2: return launch_sparse_n<2, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 3: return launch_sparse_n<3, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 4: return launch_sparse_n<4, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 5: return launch_sparse_n<5, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 6: return launch_sparse_n<6, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 7: return launch_sparse_n<7, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 8: return launch_sparse_n<8, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 9: return launch_sparse_n<9, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 10: return launch_sparse_n<10, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 11: return launch_sparse_n<11, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 12: return launch_sparse_n<12, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 13: return launch_sparse_n<13, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 14: return launch_sparse_n<14, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 15: return launch_sparse_n<15, DOWN_ONLY>(p, sms, s, y_zeroed);
+    case 16: return launch_sparse_n<16, DOWN_ONLY>(p, sms, s, y_zeroed);
     default: return TWELL_ERR_SHAPE;
   }
 }
 
 twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
                          const twell_t* tw, int skip, float* y, int32_t* dev_status, cudaStream_t s, int sms,
-                         bool down_only = false) {
+                         bool down_only = false, bool y_zeroed = false) {
   SparseParams p{};
   p.x = x;
   p.WuT = WuT;
@@ -252,7 +260,7 @@ twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t*
   p.W = tw->W;
   p.skip_ovf = skip ? 1 : 0;
   p.dev_status = dev_status;
-  return down_only ? sparse_launch<true>(p, d, sms, s) : sparse_launch<false>(p, d, sms, s);
+  return down_only ? sparse_launch<true>(p, d, sms, s, y_zeroed) : sparse_launch<false>(p, d, sms, s, y_zeroed);
 }
 
 // Down projection from a TwELL of hidden activations (per-token gathers of Wd rows).
@@ -260,6 +268,10 @@ twell_status down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* t
                        int32_t* dev_status, cudaStream_t s, int sms) {
   return sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, skip, y, dev_status, s, sms, true);
 }
+
+twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, const uint16_t* Wd, int d, int f,
+                             bool split, const int* row_map, float* y, int y_rows, int32_t* dev_status,
+                             cudaStream_t s, int sms);
 
 // Dense FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu), or
 // h = ReLU(A Wg) for the non-gated layer (WuT null), into h_buf, then
@@ -271,10 +283,9 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
   const int hk = split ? 2 * f : f;
   const bool gated = WuT != nullptr;
   const int tile_n = gated ? 128 : kBN;  // h columns per output tile of the first GEMM
-  CUtensorMap ma, mg, mu, mh, md;
+  CUtensorMap ma, mg, mu;
   if (!make_map(&ma, a_rows, d, M, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, tile_n) ||
-      (gated && !make_map(&mu, WuT, d, f, kBK, 128)) || !make_map(&mh, h_buf, hk, M, kBK, kBM) ||
-      !make_map(&md, Wd, d, f, 64, kBK))
+      (gated && !make_map(&mu, WuT, d, f, kBK, 128)))
     return TWELL_ERR_CUDA;
   GemmParams p1{};
   p1.M = M;
@@ -291,6 +302,17 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
   } else {
     TW_TRY(launch_gemm<kModeRelu>(ma, mg, mg, p1, g1, s));
   }
+  return dense_down_impl(h_buf, M, M_dev, Wd, d, f, split, row_map, y, y_rows, dev_status, s, sms);
+}
+
+// Second half of the dense layer: out[row_map[i]] = h[i] Wd (row_map null: identity), h_buf
+// [M][f] bf16, or [M][2f] (h and its bf16 remainder) with split.
+twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, const uint16_t* Wd, int d, int f,
+                             bool split, const int* row_map, float* y, int y_rows, int32_t* dev_status,
+                             cudaStream_t s, int sms) {
+  const int hk = split ? 2 * f : f;
+  CUtensorMap mh, md;
+  if (!make_map(&mh, h_buf, hk, M, kBK, kBM) || !make_map(&md, Wd, d, f, 64, kBK)) return TWELL_ERR_CUDA;
   GemmParams p2{};
   p2.M = M;
   p2.M_dev = M_dev;
@@ -318,6 +340,50 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ small batches
+
+// Batches up to this many tokens whose gate GEMM has too few output tiles to
+// fill the GPU take the small-batch path: the gate GEMM splits K over the whole
+// grid into fp32 pre-activations, and a separate kernel packs them.
+constexpr int kSmallT = 512;
+
+bool small_batch(int T, int N, int tile_n, int sms) {
+  const long long tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((N + tile_n - 1) / tile_n);
+  return T <= kSmallT && tiles * 2 <= sms;
+}
+
+// C[M][ldo] += A[M][K] B[N][K]^T in fp32 with K split over the whole grid; C's
+// first N columns of rows < M must hold zeros.
+twell_status f32_gemm_impl(const uint16_t* A, int M, const uint16_t* B, int N, int K, float* C, int ldo,
+                           int32_t* dev_status, cudaStream_t s, int sms) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, K, M, kBK, kBM) || !make_map(&mb, B, K, N, kBK, kBN)) return TWELL_ERR_CUDA;
+  GemmParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.out_f32 = C;
+  p.ldo = ldo;
+  p.out_rows = M;
+  p.k_splits_max = 32;
+  p.dev_status = dev_status;
+  return launch_gemm<kModeF32>(ma, mb, mb, p, sms, s);
+}
+
+// The gate pack of a small batch: split-K gate GEMM into zbuf ([T][f] fp32,
+// caller's scratch), then one warp per (row, tile) packs it; y is zeroed on
+// the way when y_zero is given.
+twell_status small_gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
+                                  float* zbuf, float* y_zero, int32_t* dev_status, cudaStream_t s, int sms) {
+  TW_TRY(cuda_ok(cudaMemsetAsync(tw->row_ovf, 0, static_cast<size_t>(T), s)));
+  TW_TRY(cuda_ok(cudaMemsetAsync(zbuf, 0, static_cast<size_t>(T) * f * sizeof(float), s)));
+  TW_TRY(f32_gemm_impl(x, T, WgT, f, d, zbuf, f, dev_status, s, sms));
+  const long long warps = static_cast<long long>(T) * (f / 128);
+  const int blocks = static_cast<int>(std::min<long long>((warps + 7) / 8, 4LL * sms));
+  pack_f32_kernel<<<blocks, 256, 0, s>>>(zbuf, T, f, tw->W, tw->counts, tw->idx, tw->vals, tw->row_ovf, y_zero, d);
+  return cuda_ok(cudaGetLastError());
+}
 
 // Dense branch: gather x[rows[i]] into xo, dense FFN (gated, or non-gated when WuT is
 // null) into ho, scatter to y.
@@ -630,6 +696,16 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
   uint16_t* xo = static_cast<uint16_t*>(workspace);
   uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
                                              round_up(static_cast<size_t>(T) * d * 2, 256));
+  if (small_batch(T, f, kBN, sms)) {
+    // the h region of the dense branch is free until that branch runs
+    const bool zero_y = sparse_splits_units(T, d, false, sms);
+    TW_TRY(small_gate_pack_impl(x, WgT, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
+                                dev_status, s, sms));
+    route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y);
+    TW_TRY(cuda_ok(cudaGetLastError()));
+    TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms, false, zero_y));
+    return dense_impl(xo, T, n_ovf, WgT, WuT, Wd, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
+  }
   TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
   route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
   TW_TRY(cuda_ok(cudaGetLastError()));
@@ -658,7 +734,9 @@ twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, co
 size_t twell_dense_workspace_bytes(int T, int d, int f) {
   (void)d;
   if (T <= 0 || f <= 0) return 0;
-  return round_up(static_cast<size_t>(T) * f * 2, 256);
+  // h [T][f] bf16, and for small batches the fp32 pre-activations [T][2f]
+  const size_t small = T <= kSmallT ? round_up(static_cast<size_t>(T) * f * 8, 256) : 0;
+  return round_up(static_cast<size_t>(T) * f * 2, 256) + small;
 }
 
 twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
@@ -671,8 +749,21 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
   if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  return dense_impl(x, T, nullptr, WgT, WuT, Wd, d, f, static_cast<uint16_t*>(workspace), false, nullptr, y, T,
-                    dev_status, static_cast<cudaStream_t>(stream), sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* h = static_cast<uint16_t*>(workspace);
+  if (small_batch(T, f, 128, sms)) {
+    // z and u with K split over the whole grid, then h = bf16(ReLU(z) * u)
+    float* zu = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(T) * f * 2, 256));
+    TW_TRY(cuda_ok(cudaMemsetAsync(zu, 0, static_cast<size_t>(T) * f * 8, s)));
+    TW_TRY(f32_gemm_impl(x, T, WgT, f, d, zu, 2 * f, dev_status, s, sms));
+    TW_TRY(f32_gemm_impl(x, T, WuT, f, d, zu + f, 2 * f, dev_status, s, sms));
+    const size_t n4 = static_cast<size_t>(T) * f / 4;
+    h_from_zu_kernel<<<static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 4 * static_cast<size_t>(sms))), 256, 0,
+                       s>>>(zu, T, f, 1, h);
+    TW_TRY(cuda_ok(cudaGetLastError()));
+    return dense_down_impl(h, T, nullptr, Wd, d, f, false, nullptr, y, T, dev_status, s, sms);
+  }
+  return dense_impl(x, T, nullptr, WgT, WuT, Wd, d, f, h, false, nullptr, y, T, dev_status, s, sms);
 }
 
 twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2, int T, int d,
@@ -693,6 +784,15 @@ twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1
                                              round_up(static_cast<size_t>(T) * d * 2, 256));
   // The pack of ReLU(x W1) holds the hidden activations themselves, so the
   // sparse step is the down projection alone.
+  if (small_batch(T, f, kBN, sms)) {
+    const bool zero_y = sparse_splits_units(T, d, true, sms);
+    TW_TRY(small_gate_pack_impl(x, W1T, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
+                                dev_status, s, sms));
+    route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y);
+    TW_TRY(cuda_ok(cudaGetLastError()));
+    TW_TRY(sparse_impl(nullptr, nullptr, W2, T, d, f, tw, 1, y, dev_status, s, sms, true, zero_y));
+    return dense_impl(xo, T, n_ovf, W1T, nullptr, W2, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
+  }
   TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms));
   route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
   TW_TRY(cuda_ok(cudaGetLastError()));
@@ -728,8 +828,19 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
   if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  return dense_impl(x, T, nullptr, W1T, nullptr, W2, d, f, static_cast<uint16_t*>(workspace), false, nullptr, y, T,
-                    dev_status, static_cast<cudaStream_t>(stream), sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* h = static_cast<uint16_t*>(workspace);
+  if (small_batch(T, f, kBN, sms)) {
+    float* z = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(T) * f * 2, 256));
+    TW_TRY(cuda_ok(cudaMemsetAsync(z, 0, static_cast<size_t>(T) * f * 4, s)));
+    TW_TRY(f32_gemm_impl(x, T, W1T, f, d, z, f, dev_status, s, sms));
+    const size_t n4 = static_cast<size_t>(T) * f / 4;
+    h_from_zu_kernel<<<static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 4 * static_cast<size_t>(sms))), 256, 0,
+                       s>>>(z, T, f, 0, h);
+    TW_TRY(cuda_ok(cudaGetLastError()));
+    return dense_down_impl(h, T, nullptr, W2, d, f, false, nullptr, y, T, dev_status, s, sms);
+  }
+  return dense_impl(x, T, nullptr, W1T, nullptr, W2, d, f, h, false, nullptr, y, T, dev_status, s, sms);
 }
 
 size_t twell_backward_workspace_bytes(int T, int d, int f, int W) {

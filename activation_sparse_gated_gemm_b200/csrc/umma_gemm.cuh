@@ -25,6 +25,11 @@
 //                  the columns where some row has z > 0 (a bitmap, one bit per
 //                  hidden unit, OR-ed in with one atomic per warp and 32
 //                  columns): the profile that finds dead hidden units.
+//   kModeF32    -- plain C = A . B^T (B K-major, like the gate GEMM) stored as
+//                  fp32, with K split over the grid when the output tiles
+//                  cannot fill it (partial sums added into zeroed rows): the
+//                  gate (or up) pre-activations of a small batch, packed or
+//                  combined by a separate kernel.
 //   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
 //                  epilogue stores fp32 rows, optionally scattered through a
 //                  row map (the dense branch of the hybrid route). With the
@@ -50,7 +55,8 @@ enum GemmMode : int {
   kModeDown = 2,
   kModeTwellHidden = 3,
   kModeRelu = 4,
-  kModeActivity = 5
+  kModeActivity = 5,
+  kModeF32 = 6
 };
 
 constexpr int kBM = 128;
@@ -101,7 +107,7 @@ struct GemmParams {
   // kModeDown: B rows are read at k mod k_wrap (k_wrap > 0), so K = 2 * k_wrap
   // runs [h_hi | h_lo] against [Wd ; Wd].
   int k_wrap;
-  // kModeDown: when the output tiles do not fill the grid, K is cut into up to
+  // kModeDown / kModeF32: when the output tiles do not fill the grid, K is cut into up to
   // this many splits whose partial sums are added into out_f32 (which must
   // hold zeros in the rows written); 0 or 1 disables splitting.
   int k_splits_max;
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int num_kb = p.K / kBK;
   // K splits (kModeDown only): as many as keep every CTA busy, none empty.
   int kb_per = num_kb, k_splits = 1;
-  if (MODE == kModeDown && p.k_splits_max > 1 && num_m * num_n > 0) {
+  if ((MODE == kModeDown || MODE == kModeF32) && p.k_splits_max > 1 && num_m * num_n > 0) {
     int want = min(p.k_splits_max, max(1, static_cast<int>(gridDim.x) / (num_m * num_n)));
     want = min(want, num_kb);
     kb_per = (num_kb + want - 1) / want;
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* b_dst = smem + kOffB + s * kBStageBytes;
           mbar_arrive_expect_tx(&full[s], kAStageBytes + kBStageBytes);
           tma_load_2d(a_dst, &tmA, &full[s], kb * kBK, m_blk * kBM);
-          if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity) {
+          if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity || MODE == kModeF32) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * kBN);
           } else if (kStacked) {
             tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * 128);
@@ -505,7 +511,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             store_h32(h, p.out + static_cast<size_t>(my_row) * p.ldo, col, p.N, p.h_split != 0);
           }
         }
-      } else {
+      } else {  // kModeDown, kModeF32: fp32 rows (through the row map when given)
         int orow = my_row;
         bool valid = my_row < M;
         if (valid && p.row_map != nullptr) {

@@ -157,7 +157,10 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
 twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream);
 
 /* Bytes of workspace needed by twell_ffn_hybrid_forward and
- * twell_dense_rows_forward (worst case: every row overflows). */
+ * twell_dense_rows_forward (worst case: every row overflows). For small
+ * batches the hybrid forward also uses the hidden-activation part of it for the
+ * fp32 gate pre-activations of its split-K gate GEMM, before the dense branch
+ * runs. */
 size_t twell_hybrid_workspace_bytes(int T, int d, int f);
 
 /*
@@ -218,8 +221,10 @@ twell_status twell_ffn_hybrid_forward_noalloc(const uint16_t* x, const uint16_t*
                                               float* y, int32_t* ovf_rows, int32_t* n_ovf,
                                               int32_t* dev_status, void* stream);
 
-/* Bytes of workspace needed by twell_dense_ffn_forward (the [T][f] bf16 hidden
- * activations). */
+/* Bytes of workspace needed by twell_dense_ffn_forward and
+ * twell_relu_dense_ffn_forward: the [T][f] bf16 hidden activations, and for
+ * T <= 512 room for the fp32 pre-activations ([T][2f]) of the small-batch path,
+ * whose first GEMMs split K over the whole GPU. */
 size_t twell_dense_workspace_bytes(int T, int d, int f);
 
 /*
