@@ -8,16 +8,16 @@
 //   dx   = sum_j dz_j Wg[:, j] + du_j Wu[:, j]
 //   dWd[j, :] = sum_t h_tj dy_t, dWu[:, j] = sum_t du_tj x_t, dWg[:, j] = sum_t dz_tj x_t
 //
-// Two passes over the stored units:
+// Rows that fit the ELL width take two passes over their stored units:
 //   1. per token (one warp per token, like the forward's fused kernel): u_j and
 //      dh_j by two dot products per stored unit, then dx_t by two row axpys;
 //      the per-unit scalars (h, du, dz) are written beside the slots;
 //   2. per hidden unit: the slots are sorted by column (count, scan, scatter)
 //      and one warp per (unit, 256-wide slice of d) sums h dy_t, du x_t, dz x_t
 //      over the unit's tokens into the three weight-gradient rows.
-// Rows that overflow the ELL width are packed again at the full tile width
-// (nothing dropped) from the gathered rows, and go through the same two
-// passes with their gate recomputed in fp32 instead of the stored bf16 value.
+// Rows that overflow take the dense branch on the tensor cores (the GEMM
+// modes kModeZU, kModeBwdDh and kModeDown), which adds their share to the
+// weight gradients afterwards.
 #pragma once
 
 #include "sparse_ffn.cuh"
@@ -25,23 +25,18 @@
 namespace twell {
 
 struct BwdParams {
-  const uint16_t* x;   // [rows][d] bf16: the tokens, or the gathered overflow rows
-  const uint16_t* dy;  // [rows][d] bf16 upstream gradient, same rows
+  const uint16_t* x;   // [rows][d] bf16
+  const uint16_t* dy;  // [rows][d] bf16 upstream gradient
   const uint16_t* WgT;
   const uint16_t* WuT;
   const uint16_t* Wd;
-  const int16_t* counts;  // TwELL of these rows
+  const int16_t* counts;  // TwELL of these rows (the forward's gate pack)
   const int16_t* idx;
   const uint16_t* vals;
-  const uint8_t* row_ovf;
-  int rows;             // rows of this pass (an upper bound when rows_dev is set)
-  const int* rows_dev;  // device row count, or null
-  const int* row_map;   // dx row of each pass row, or null for the identity
+  const uint8_t* row_ovf;  // rows with the flag set are skipped
+  int rows;
   int d, f, nT, W;
-  int skip_ovf;     // skip rows whose overflow flag is set
-  int recompute_g;  // g_j = max(0, x_t . Wg[:, j]) in fp32 instead of the stored bf16
-  float* dx;        // [dx_rows][d] fp32
-  int dx_rows;
+  float* dx;   // [rows][d] fp32
   float* s_h;  // per stored slot [rows][nT][W]: h, du, dz (fp32)
   float* s_du;
   float* s_dz;
@@ -117,13 +112,10 @@ __device__ __forceinline__ void bwd_axpy_pass(float (&acc)[NCH][8], const uint16
   }
 }
 
-// One warp per token of the pass. Shared memory per warp: x_t and dy_t
+// One warp per token that fits. Shared memory per warp: x_t and dy_t
 // (NCH * 32 uint4 each), the flattened slot list (column | bf16 g << 16) and
 // the slot position of every list entry inside the row's [nT][W] block.
-//
-// RECOMPUTE: the gate is recomputed in fp32 (overflow rows, packed again at
-// the full tile width) instead of taken from the stored bf16 value.
-template <int NCH, int WARPS, bool RECOMPUTE>
+template <int NCH, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParams p) {
   extern __shared__ uint4 bwd_smem[];
   const int lane = threadIdx.x & 31;
@@ -136,8 +128,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
                                                WARPS * kListCap) +
                    warp * kListCap;
   const int group_tiles = max(1, kListCap / p.W);
-  int rows = p.rows;
-  if (p.rows_dev != nullptr) rows = min(max(*p.rows_dev, 0), rows);
+  const int rows = p.rows;
   bool bad_index = false;
   // tokens are handed out one at a time from a per-block counter over the
   // block's contiguous share of the rows
@@ -152,15 +143,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
     if (lane == 0) t = atomicAdd(&next_row, 1);
     t = __shfl_sync(0xffffffffu, t, 0);
     if (t >= r_end) break;
-    if (p.skip_ovf && p.row_ovf[t]) continue;
-    int r = t;
-    if (p.row_map != nullptr) {
-      r = p.row_map[t];
-      if (r < 0 || r >= p.dx_rows) {
-        bad_index = true;
-        continue;
-      }
-    }
+    if (p.row_ovf[t]) continue;
     __syncwarp();
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
@@ -228,11 +211,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
         const int my_j = entry_j(my_e);
         const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
         const bool valid = (my_pos & 0x8000u) == 0;
-        // u_j = x . Wu[:, j], dh_j = dy . Wd[j, :] (and z_j when recomputed)
+        // u_j = x . Wu[:, j], dh_j = dy . Wd[j, :]
         const float my_u = bwd_dot_pass<NCH>(xs, p.WuT, my_j, ns, lane, d);
         const float my_dh = bwd_dot_pass<NCH>(ds, p.Wd, my_j, ns, lane, d);
-        float my_g = entry_g(my_e);
-        if (RECOMPUTE) my_g = fmaxf(bwd_dot_pass<NCH>(xs, p.WgT, my_j, ns, lane, d), 0.0f);
+        const float my_g = entry_g(my_e);
         const float my_du = valid ? my_dh * my_g : 0.0f;
         const float my_dz = valid ? my_dh * my_u : 0.0f;
         if (valid) {
@@ -251,7 +233,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
     for (int i = 0; i < NCH; ++i) {
       const int k0 = (i * 32 + lane) * 8;
       if (k0 < d) {
-        float4* dst = reinterpret_cast<float4*>(p.dx + static_cast<size_t>(r) * d + k0);
+        float4* dst = reinterpret_cast<float4*>(p.dx + static_cast<size_t>(t) * d + k0);
         dst[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         dst[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
       }
@@ -349,21 +331,14 @@ __global__ void __launch_bounds__(1024) bwd_column_scan_kernel(int* colcnt, int 
 }
 
 struct WgradParams {
-  const uint32_t* list;
+  const uint32_t* list;  // slot indices sorted by column
   const int* colptr;
-  // pass 0 (rows that fit) and pass 1 (overflow rows), selected by bit 31
   const uint16_t* x0;
   const uint16_t* dy0;
-  const float* h0;
+  const float* h0;  // per-slot scalars of the rows that fit
   const float* du0;
   const float* dz0;
-  int slots_per_row0;  // nT * W of the pass
-  const uint16_t* x1;
-  const uint16_t* dy1;
-  const float* h1;
-  const float* du1;
-  const float* dz1;
-  int slots_per_row1;
+  int slots_per_row0;  // nT * W
   int f, d;
   float* dWgT;  // [f][d] fp32, fully written
   float* dWuT;
@@ -392,23 +367,13 @@ __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
     const uint16_t* dr = nullptr;
     float vh = 0.f, vu = 0.f, vz = 0.f;
     if (lane < nb) {
-      const uint32_t ent = p.list[b + lane];
-      const size_t slot = ent & 0x7fffffffu;
-      if (ent >> 31) {
-        const size_t row = slot / static_cast<size_t>(p.slots_per_row1);
-        xr = p.x1 + row * p.d;
-        dr = p.dy1 + row * p.d;
-        vh = p.h1[slot];
-        vu = p.du1[slot];
-        vz = p.dz1[slot];
-      } else {
-        const size_t row = slot / static_cast<size_t>(p.slots_per_row0);
-        xr = p.x0 + row * p.d;
-        dr = p.dy0 + row * p.d;
-        vh = p.h0[slot];
-        vu = p.du0[slot];
-        vz = p.dz0[slot];
-      }
+      const size_t slot = p.list[b + lane] & 0x7fffffffu;
+      const size_t row = slot / static_cast<size_t>(p.slots_per_row0);
+      xr = p.x0 + row * p.d;
+      dr = p.dy0 + row * p.d;
+      vh = p.h0[slot];
+      vu = p.du0[slot];
+      vz = p.dz0[slot];
     }
 #pragma unroll 1
     for (int s = 0; s < nb; ++s) {

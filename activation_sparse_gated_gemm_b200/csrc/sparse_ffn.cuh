@@ -398,10 +398,19 @@ __global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int
 
 // out[i, :] = x[rows[i], :] for i < *n_rows (clamped to T, the room in rows and
 // out); when y_zero is given, also y_zero[rows[i], :] = 0 (the dense branch may
-// add split partial sums into those rows).
+// add split partial sums into those rows). With pad_rows > 0 (the room in out,
+// at least T), rows from n up to the next multiple of 64 are zeroed, so a
+// GEMM whose K runs over out's rows in blocks of 64 reads zeros past n.
 __global__ void gather_rows_kernel(const uint16_t* x, int d, const int* rows, const int* n_rows, int T,
-                                   uint16_t* out, float* y_zero, int* dev_status) {
+                                   uint16_t* out, float* y_zero, int* dev_status, int pad_rows = 0) {
   const int n = min(max(*n_rows, 0), T);
+  if (pad_rows > 0) {
+    const int pad_end = min((n + 63) / 64 * 64, pad_rows);
+    for (int i = n + blockIdx.x; i < pad_end; i += gridDim.x) {
+      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(i) * d);
+      for (int k = threadIdx.x; k < d / 8; k += blockDim.x) dst[k] = make_uint4(0, 0, 0, 0);
+    }
+  }
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
     const int r = rows[i];
     if (r < 0 || r >= T) {

@@ -399,25 +399,26 @@ twell_status dense_rows_impl(const uint16_t* x, const uint16_t* WgT, const uint1
 
 // Workspace of the hybrid backward, carved in this order (each piece 256-byte
 // aligned): per-slot h, du, dz of the rows that fit ([T][nT][W] fp32 each);
-// the gathered overflow rows of x and dy ([T][d] bf16 each); their full-width
-// TwELL (counts, idx, vals, flags) and per-slot h, du, dz ([T][nT][128]); the
-// column counts/cursors ([f]), column offsets ([f + 1]) and the column-sorted
-// slot list (one uint32 per slot of both passes).
+// for the overflow rows, the gathered rows of x and dy ([Tp][d] bf16 each, Tp =
+// T rounded up to 64), their [z | u] ([T][2f] fp32), [dz | du | dz_lo | du_lo]
+// ([T][4f] bf16) and the three transposed blocks dz, du, h ([f][2 Tp] bf16
+// each); the column counts/cursors ([f]), column offsets ([f + 1]) and the
+// column-sorted slot list (one uint32 per slot of the rows that fit).
 struct BwdWorkspace {
   float *h0, *du0, *dz0;
   uint16_t *xo, *dyo;
-  int16_t *c1, *i1;
-  uint16_t* v1;
-  uint8_t* r1;
-  float *h1, *du1, *dz1;
+  float* zu;
+  uint16_t *a2, *tT;
   int *colcnt, *colptr;
   uint32_t* list;
+  int t_pad;
   size_t bytes;
 };
 
 BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
   const size_t nT = static_cast<size_t>(f) / 128;
-  const size_t s0 = static_cast<size_t>(T) * nT * W, s1 = static_cast<size_t>(T) * nT * 128;
+  const size_t s0 = static_cast<size_t>(T) * nT * W;
+  const size_t tp = round_up(static_cast<size_t>(T), 64);
   BwdWorkspace w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -428,18 +429,15 @@ BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
   w.h0 = reinterpret_cast<float*>(take(s0 * 4));
   w.du0 = reinterpret_cast<float*>(take(s0 * 4));
   w.dz0 = reinterpret_cast<float*>(take(s0 * 4));
-  w.xo = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * d * 2));
-  w.dyo = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * d * 2));
-  w.c1 = reinterpret_cast<int16_t*>(take(static_cast<size_t>(T) * nT * 2));
-  w.i1 = reinterpret_cast<int16_t*>(take(s1 * 2));
-  w.v1 = reinterpret_cast<uint16_t*>(take(s1 * 2));
-  w.r1 = reinterpret_cast<uint8_t*>(take(static_cast<size_t>(T)));
-  w.h1 = reinterpret_cast<float*>(take(s1 * 4));
-  w.du1 = reinterpret_cast<float*>(take(s1 * 4));
-  w.dz1 = reinterpret_cast<float*>(take(s1 * 4));
+  w.xo = reinterpret_cast<uint16_t*>(take(tp * d * 2));
+  w.dyo = reinterpret_cast<uint16_t*>(take(tp * d * 2));
+  w.zu = reinterpret_cast<float*>(take(static_cast<size_t>(T) * f * 8));
+  w.a2 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * f * 8));
+  w.tT = reinterpret_cast<uint16_t*>(take(3 * static_cast<size_t>(f) * 2 * tp * 2));
   w.colcnt = reinterpret_cast<int*>(take(static_cast<size_t>(f) * 4));
   w.colptr = reinterpret_cast<int*>(take((static_cast<size_t>(f) + 1) * 4));
-  w.list = reinterpret_cast<uint32_t*>(take((s0 + s1) * 4));
+  w.list = reinterpret_cast<uint32_t*>(take(s0 * 4));
+  w.t_pad = static_cast<int>(tp);
   w.bytes = off;
   return w;
 }
@@ -448,7 +446,7 @@ template <int NCH>
 twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
   constexpr int kWarps = bwd_warps_for(NCH);
   const size_t smem = static_cast<size_t>(kWarps) * (2 * NCH * 32 * sizeof(uint4) + kListCap * 6);
-  auto kern = p.recompute_g ? bwd_token_kernel<NCH, kWarps, true> : bwd_token_kernel<NCH, kWarps, false>;
+  auto kern = bwd_token_kernel<NCH, kWarps>;
   if (smem > 48 * 1024)
     TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
   const long long want = (static_cast<long long>(p.rows) + kWarps - 1) / kWarps;
@@ -502,37 +500,59 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   p0.f = f;
   p0.nT = nT;
   p0.W = tw->W;
-  p0.skip_ovf = 1;
   p0.dx = dx;
-  p0.dx_rows = T;
   p0.s_h = w.h0;
   p0.s_du = w.du0;
   p0.s_dz = w.dz0;
   p0.dev_status = dev_status;
   TW_TRY(launch_bwd_token(p0, sms, s));
-  // 2. overflow rows: gather x and dy, pack again at the full tile width, same pass
-  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, ovf_rows, n_ovf, T, w.xo, nullptr, dev_status);
+  // 2. overflow rows, dense on the tensor cores: gather x and dy (zero the dx
+  // rows and the padding rows up to a multiple of 64), recompute [z | u], then
+  // dh = dy Wd^T with dz, du, h in its epilogue, then dx = [dz | du] [Wg; Wu]^T
+  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, ovf_rows, n_ovf, T, w.xo, dx, dev_status, w.t_pad);
   TW_TRY(cuda_ok(cudaGetLastError()));
-  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(dy, d, ovf_rows, n_ovf, T, w.dyo, nullptr, dev_status);
+  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(dy, d, ovf_rows, n_ovf, T, w.dyo, nullptr, dev_status, w.t_pad);
   TW_TRY(cuda_ok(cudaGetLastError()));
-  const twell_t tw1{w.c1, w.i1, w.v1, w.r1, T, f, 128, 128};
-  TW_TRY(gate_pack_impl(w.xo, WgT, T, d, f, &tw1, dev_status, s, sms, n_ovf));
-  BwdParams p1 = p0;
-  p1.x = w.xo;
-  p1.dy = w.dyo;
-  p1.counts = w.c1;
-  p1.idx = w.i1;
-  p1.vals = w.v1;
-  p1.row_ovf = w.r1;
-  p1.rows_dev = n_ovf;
-  p1.row_map = ovf_rows;
-  p1.W = 128;
-  p1.skip_ovf = 0;
-  p1.recompute_g = 1;
-  p1.s_h = w.h1;
-  p1.s_du = w.du1;
-  p1.s_dz = w.dz1;
-  return launch_bwd_token(p1, sms, s);
+  CUtensorMap mx, mdy, mg, mu, mwd, ma2, mgT, muT;
+  if (!make_map(&mx, w.xo, d, T, kBK, kBM) || !make_map(&mdy, w.dyo, d, T, kBK, kBM) ||
+      !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128) ||
+      !make_map(&mwd, Wd, d, f, kBK, kBN) || !make_map(&ma2, w.a2, 4 * f, T, kBK, kBM) ||
+      !make_map(&mgT, WgT, d, f, 64, kBK) || !make_map(&muT, WuT, d, f, 64, kBK))
+    return TWELL_ERR_CUDA;
+  GemmParams q1{};
+  q1.M = T;
+  q1.M_dev = n_ovf;
+  q1.N = f;
+  q1.K = d;
+  q1.out_f32 = w.zu;
+  q1.ldo = 2 * f;
+  q1.dev_status = dev_status;
+  TW_TRY(launch_gemm<kModeZU>(mx, mg, mu, q1, sms, s));
+  GemmParams q2{};
+  q2.M = T;
+  q2.M_dev = n_ovf;
+  q2.N = f;
+  q2.K = d;
+  q2.zu = w.zu;
+  q2.a2 = w.a2;
+  q2.tT = w.tT;
+  q2.t_pad = w.t_pad;
+  q2.dev_status = dev_status;
+  TW_TRY(launch_gemm<kModeBwdDh>(mdy, mwd, mwd, q2, sms, s));
+  GemmParams q3{};
+  q3.M = T;
+  q3.M_dev = n_ovf;
+  q3.N = d;
+  q3.K = 4 * f;
+  q3.k_wrap = 2 * f;
+  q3.k_split_b = f;
+  q3.out_f32 = dx;
+  q3.ldo = d;
+  q3.row_map = ovf_rows;
+  q3.out_rows = T;
+  q3.k_splits_max = 32;  // the gather zeroed these dx rows
+  q3.dev_status = dev_status;
+  return launch_gemm<kModeDown>(ma2, mgT, muT, q3, sms, s);
 }
 
 // Weight gradients from the workspace filled by backward_dx_impl.
@@ -541,16 +561,14 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
                               int sms) {
   const int nT = f / 128;
   BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
-  // 3. weight gradients: sort both passes' slots by column, then sum per column
+  // 3. weight gradients of the rows that fit: sort their slots by column, then
+  // sum per column (every row of dW is written)
   SlotSource a{tw->counts, tw->idx, tw->row_ovf, T, nullptr, nT, tw->W, f, 1, 0u};
-  SlotSource b{w.c1, w.i1, w.r1, T, n_ovf, nT, 128, f, 0, 0x80000000u};
   TW_TRY(cuda_ok(cudaMemsetAsync(w.colcnt, 0, static_cast<size_t>(f) * 4, s)));
   const int cblocks = 4 * sms;
   bwd_columns_kernel<false><<<cblocks, 256, 0, s>>>(a, w.colcnt, w.colptr, w.list);
-  bwd_columns_kernel<false><<<cblocks, 256, 0, s>>>(b, w.colcnt, w.colptr, w.list);
   bwd_column_scan_kernel<<<1, 1024, 0, s>>>(w.colcnt, f, w.colptr);
   bwd_columns_kernel<true><<<cblocks, 256, 0, s>>>(a, w.colcnt, w.colptr, w.list);
-  bwd_columns_kernel<true><<<cblocks, 256, 0, s>>>(b, w.colcnt, w.colptr, w.list);
   TW_TRY(cuda_ok(cudaGetLastError()));
   WgradParams g{};
   g.list = w.list;
@@ -561,12 +579,6 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
   g.du0 = w.du0;
   g.dz0 = w.dz0;
   g.slots_per_row0 = nT * tw->W;
-  g.x1 = w.xo;
-  g.dy1 = w.dyo;
-  g.h1 = w.h1;
-  g.du1 = w.du1;
-  g.dz1 = w.dz1;
-  g.slots_per_row1 = nT * 128;
   g.f = f;
   g.d = d;
   g.dWgT = dWgT;
@@ -574,7 +586,33 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
   g.dWd = dWd;
   const long long warps = static_cast<long long>(f) * ((d + 255) / 256);
   bwd_wgrad_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(g);
-  return cuda_ok(cudaGetLastError());
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  // 4. the overflow rows' share, on the tensor cores: dWgT += dz^T x,
+  // dWuT += du^T x, dWd += h^T dy over the gathered rows (K = their tokens, as
+  // bf16 value and remainder halves)
+  const size_t tblock = static_cast<size_t>(f) * 2 * w.t_pad;
+  const uint16_t* aT[3] = {w.tT, w.tT + tblock, w.tT + 2 * tblock};
+  const uint16_t* bT[3] = {w.xo, w.xo, w.dyo};
+  float* outs[3] = {dWgT, dWuT, dWd};
+  for (int i = 0; i < 3; ++i) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, aT[i], 2 * w.t_pad, f, kBK, kBM) || !make_map(&mb, bT[i], d, w.t_pad, 64, kBK))
+      return TWELL_ERR_CUDA;
+    GemmParams q{};
+    q.M = f;
+    q.N = d;
+    q.K = 2 * w.t_pad;
+    q.k_wrap = w.t_pad;
+    q.k_dev = n_ovf;
+    q.k_half = w.t_pad;
+    q.accumulate = 1;
+    q.k_splits_max = 32;
+    q.out_f32 = outs[i];
+    q.ldo = d;
+    q.dev_status = nullptr;
+    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, sms, s));
+  }
+  return TWELL_OK;
 }
 
 }  // namespace
@@ -855,8 +893,8 @@ twell_status twell_ffn_hybrid_backward(const uint16_t* x, const uint16_t* WgT, c
                                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
   TW_TRY(check_shape(T, d, f));
   TW_TRY(check_tw(tw, T, f));
-  // slot indices of both passes are kept in 31 bits
-  if (static_cast<long long>(T) * (f / 128) * 128 >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  // slot indices are kept in 31 bits
+  if (static_cast<long long>(T) * (f / 128) * tw->W >= (1LL << 31)) return TWELL_ERR_SHAPE;
   TW_TRY(check_ptrs({dWgT, dWuT, dWd, dev_status}));
   if (T == 0) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -884,7 +922,7 @@ twell_status twell_ffn_hybrid_backward_dx(const uint16_t* x, const uint16_t* WgT
                                           void* stream) {
   TW_TRY(check_shape(T, d, f));
   TW_TRY(check_tw(tw, T, f));
-  if (static_cast<long long>(T) * (f / 128) * 128 >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  if (static_cast<long long>(T) * (f / 128) * tw->W >= (1LL << 31)) return TWELL_ERR_SHAPE;
   if (T == 0) return TWELL_OK;
   TW_TRY(check_ptrs({x, WgT, WuT, Wd, dy, ovf_rows, n_ovf, dx, dev_status}));
   if (workspace == nullptr || workspace_bytes < twell_backward_workspace_bytes(T, d, f, tw->W))
@@ -901,7 +939,7 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
                                           float* dWd, void* workspace, size_t workspace_bytes, void* stream) {
   TW_TRY(check_shape(T, d, f));
   TW_TRY(check_tw(tw, T, f));
-  if (static_cast<long long>(T) * (f / 128) * 128 >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  if (static_cast<long long>(T) * (f / 128) * tw->W >= (1LL << 31)) return TWELL_ERR_SHAPE;
   TW_TRY(check_ptrs({dWgT, dWuT, dWd}));
   if (T == 0) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -30,6 +30,15 @@
 //                  cannot fill it (partial sums added into zeroed rows): the
 //                  gate (or up) pre-activations of a small batch, packed or
 //                  combined by a separate kernel.
+//   kModeZU     -- z and u as in kModeGateUp, both stored as fp32 ([z | u]
+//                  rows): the dense backward's recomputed forward.
+//   kModeBwdDh  -- dh = dy . Wd^T (B = Wd, K-major) with the backward's
+//                  elementwise step in the epilogue: from the stored z and u,
+//                  dz = dh u [z > 0], du = dh ReLU(z), h = ReLU(z) u, each kept
+//                  as bf16 plus bf16 remainder, written row-major as
+//                  [dz | du | dz_lo | du_lo] (the A operand of dx) and
+//                  transposed, unit-major over tokens (the A operands of the
+//                  weight gradients).
 //   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
 //                  epilogue stores fp32 rows, optionally scattered through a
 //                  row map (the dense branch of the hybrid route). With the
@@ -56,7 +65,9 @@ enum GemmMode : int {
   kModeTwellHidden = 3,
   kModeRelu = 4,
   kModeActivity = 5,
-  kModeF32 = 6
+  kModeF32 = 6,
+  kModeZU = 7,
+  kModeBwdDh = 8
 };
 
 constexpr int kBM = 128;
@@ -100,6 +111,23 @@ struct GemmParams {
   float* out_f32;
   int ldo;
   uint32_t* active;    // kModeActivity: column bitmap, OR-ed into
+  // kModeBwdDh: zu = [z | u] rows ([M][2N] fp32); a2 = [M][4N] bf16 rows
+  // [dz | du | dz_lo | du_lo]; tT = three [N][2 t_pad] bf16 blocks (dz, du, h),
+  // unit-major, tokens [0, t_pad) holding bf16(v) and [t_pad, 2 t_pad) the
+  // remainder; rows in [M, t_pad) of the tile are written as zeros.
+  const float* zu;
+  uint16_t* a2;
+  uint16_t* tT;
+  int t_pad;
+  // kModeDown: B rows at or past k_split_b (after k_wrap) come from tmB1, at
+  // row - k_split_b (two matrices stacked along K without copying them).
+  int k_split_b;
+  // kModeDown: with k_dev set, K holds two halves of k_half rows each and only
+  // the first *k_dev rows (rounded up to 64) of each half are summed.
+  const int* k_dev;
+  int k_half;
+  // kModeDown / kModeF32: add into out_f32 even when K is not split.
+  int accumulate;
   const int* row_map;  // kModeDown: output row of each A row, or null
   int out_rows;        // valid range of output rows
   // kModeGateUp / kModeRelu: also store h_lo = bf16(h - bf16(h)) at column N + c (ldo = 2N).
@@ -190,20 +218,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   int M = p.M;
   if (p.M_dev != nullptr) M = min(max(*p.M_dev, 0), p.M);
-  constexpr bool kStacked = (MODE == kModeGateUp || MODE == kModeTwellHidden);  // B = [Wg rows; Wu rows]
+  constexpr bool kStacked = (MODE == kModeGateUp || MODE == kModeTwellHidden || MODE == kModeZU);  // B = [Wg; Wu]
   constexpr int kTileN = kStacked ? 128 : kBN;  // output columns per tile
   const int num_m = (M + kBM - 1) / kBM;
   const int num_n = (p.N + kTileN - 1) / kTileN;
-  const int num_kb = p.K / kBK;
-  // K splits (kModeDown only): as many as keep every CTA busy, none empty.
+  int num_kb = p.K / kBK;
+  // compact K (kModeDown with k_dev): blocks [0, nkb_half) of each half
+  int nkb_half = 0;
+  if (MODE == kModeDown && p.k_dev != nullptr) {
+    nkb_half = (min(max(*p.k_dev, 0), p.k_half) + kBK - 1) / kBK;
+    num_kb = 2 * nkb_half;
+  }
+  // K splits (kModeDown / kModeF32): as many as keep every CTA busy, none empty.
   int kb_per = num_kb, k_splits = 1;
-  if ((MODE == kModeDown || MODE == kModeF32) && p.k_splits_max > 1 && num_m * num_n > 0) {
+  if ((MODE == kModeDown || MODE == kModeF32) && p.k_splits_max > 1 && num_m * num_n > 0 && num_kb > 0) {
     int want = min(p.k_splits_max, max(1, static_cast<int>(gridDim.x) / (num_m * num_n)));
     want = min(want, num_kb);
     kb_per = (num_kb + want - 1) / want;
     k_splits = (num_kb + kb_per - 1) / kb_per;
   }
-  const int num_tiles = num_m * num_n * k_splits;
+  // no K block at all (an empty compact K): nothing to compute or store
+  const int num_tiles = num_kb > 0 ? num_m * num_n * k_splits : 0;
   // A CTA without a tile leaves before any setup (uniform for the whole CTA).
   if (static_cast<int>(blockIdx.x) >= num_tiles) return;
 
@@ -251,18 +286,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t* a_dst = smem + kOffA + s * kAStageBytes;
           uint8_t* b_dst = smem + kOffB + s * kBStageBytes;
+          // the K block's position in A (and B): compact K skips the empty
+          // tail of each half
+          const int kc = (nkb_half > 0 && kb >= nkb_half) ? p.k_half / kBK + (kb - nkb_half) : kb;
           mbar_arrive_expect_tx(&full[s], kAStageBytes + kBStageBytes);
-          tma_load_2d(a_dst, &tmA, &full[s], kb * kBK, m_blk * kBM);
-          if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity || MODE == kModeF32) {
-            tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * kBN);
+          tma_load_2d(a_dst, &tmA, &full[s], kc * kBK, m_blk * kBM);
+          if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity || MODE == kModeF32 ||
+              MODE == kModeBwdDh) {
+            tma_load_2d(b_dst, &tmB0, &full[s], kc * kBK, n_blk * kBN);
           } else if (kStacked) {
-            tma_load_2d(b_dst, &tmB0, &full[s], kb * kBK, n_blk * 128);
-            tma_load_2d(b_dst + kBStageBytes / 2, &tmB1, &full[s], kb * kBK, n_blk * 128);
+            tma_load_2d(b_dst, &tmB0, &full[s], kc * kBK, n_blk * 128);
+            tma_load_2d(b_dst + kBStageBytes / 2, &tmB1, &full[s], kc * kBK, n_blk * 128);
           } else {
-            const int kb_row = p.k_wrap > 0 ? (kb * kBK) % p.k_wrap : kb * kBK;
+            int kb_row = p.k_wrap > 0 ? (kc * kBK) % p.k_wrap : kc * kBK;
+            const CUtensorMap* bm = &tmB0;
+            if (p.k_split_b > 0 && kb_row >= p.k_split_b) {
+              bm = &tmB1;
+              kb_row -= p.k_split_b;
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              tma_load_2d(b_dst + i * (kBStageBytes / 4), &tmB0, &full[s], n_blk * kBN + i * 64, kb_row);
+              tma_load_2d(b_dst + i * (kBStageBytes / 4), bm, &full[s], n_blk * kBN + i * 64, kb_row);
           }
           issued |= 1u << s;
           issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -472,6 +516,110 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             store_h32(h, p.out + static_cast<size_t>(my_row) * p.ldo, col, p.N, p.h_split != 0);
           }
         }
+      } else if (MODE == kModeZU) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t zr[32], ur[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), zr);
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + ch * 32), ur);
+          tmem_wait_ld();
+          if (ch == 3) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int col = n_blk * 128 + ch * 32;
+          if (my_row < M && col < p.N) {
+            uint4* dz4 = reinterpret_cast<uint4*>(p.out_f32 + static_cast<size_t>(my_row) * p.ldo + col);
+            uint4* du4 = reinterpret_cast<uint4*>(p.out_f32 + static_cast<size_t>(my_row) * p.ldo + p.N + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              dz4[v] = make_uint4(zr[4 * v], zr[4 * v + 1], zr[4 * v + 2], zr[4 * v + 3]);
+              du4[v] = make_uint4(ur[4 * v], ur[4 * v + 1], ur[4 * v + 2], ur[4 * v + 3]);
+            }
+          }
+        }
+      } else if (MODE == kModeBwdDh) {
+        const size_t tstride = 2 * static_cast<size_t>(p.t_pad);  // one unit's row in a transposed block
+        const size_t tblock = static_cast<size_t>(p.N) * tstride;
+#pragma unroll 1
+        for (int ch = 0; ch < kBN / 32; ++ch) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), r);
+          tmem_wait_ld();
+          if (ch == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int col = n_blk * kBN + ch * 32;
+          if (col >= p.N || my_row >= p.t_pad) continue;
+          if (my_row < M) {
+            const float4* z4 = reinterpret_cast<const float4*>(p.zu + static_cast<size_t>(my_row) * 2 * p.N + col);
+            const float4* u4 = reinterpret_cast<const float4*>(p.zu + static_cast<size_t>(my_row) * 2 * p.N + p.N + col);
+            uint32_t dzh[16], duh[16], dzl[16], dul[16];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 zq = z4[q], uq = u4[q];
+              const float zz[4] = {zq.x, zq.y, zq.z, zq.w};
+              const float uu[4] = {uq.x, uq.y, uq.z, uq.w};
+              float vz[4], vu[4], vh[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float dh = __uint_as_float(r[4 * q + e]);
+                const float g = fmaxf(zz[e], 0.0f);
+                vz[e] = zz[e] > 0.0f ? dh * uu[e] : 0.0f;
+                vu[e] = dh * g;
+                vh[e] = g * uu[e];
+              }
+#pragma unroll
+              for (int e = 0; e < 4; e += 2) {
+                const int k = 2 * q + e / 2;
+                dzh[k] = pack_bf16x2(vz[e], vz[e + 1]);
+                duh[k] = pack_bf16x2(vu[e], vu[e + 1]);
+                dzl[k] = pack_bf16x2(vz[e] - __uint_as_float(dzh[k] << 16), vz[e + 1] - __uint_as_float(dzh[k] & 0xffff0000u));
+                dul[k] = pack_bf16x2(vu[e] - __uint_as_float(duh[k] << 16), vu[e + 1] - __uint_as_float(duh[k] & 0xffff0000u));
+              }
+              // transposed: unit j = col + 4q + e, token my_row (32 lanes = 32 consecutive tokens)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const size_t o = static_cast<size_t>(col + 4 * q + e) * tstride + my_row;
+                const uint16_t zh = f32_to_bf16_bits(vz[e]);
+                const uint16_t uh = f32_to_bf16_bits(vu[e]);
+                const uint16_t hh = f32_to_bf16_bits(vh[e]);
+                p.tT[o] = zh;
+                p.tT[o + p.t_pad] = f32_to_bf16_bits(vz[e] - __uint_as_float(static_cast<uint32_t>(zh) << 16));
+                p.tT[tblock + o] = uh;
+                p.tT[tblock + o + p.t_pad] = f32_to_bf16_bits(vu[e] - __uint_as_float(static_cast<uint32_t>(uh) << 16));
+                p.tT[2 * tblock + o] = hh;
+                p.tT[2 * tblock + o + p.t_pad] =
+                    f32_to_bf16_bits(vh[e] - __uint_as_float(static_cast<uint32_t>(hh) << 16));
+              }
+            }
+            uint16_t* arow = p.a2 + static_cast<size_t>(my_row) * 4 * p.N;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              reinterpret_cast<uint4*>(arow + col)[v] = make_uint4(dzh[4 * v], dzh[4 * v + 1], dzh[4 * v + 2], dzh[4 * v + 3]);
+              reinterpret_cast<uint4*>(arow + p.N + col)[v] =
+                  make_uint4(duh[4 * v], duh[4 * v + 1], duh[4 * v + 2], duh[4 * v + 3]);
+              reinterpret_cast<uint4*>(arow + 2 * p.N + col)[v] =
+                  make_uint4(dzl[4 * v], dzl[4 * v + 1], dzl[4 * v + 2], dzl[4 * v + 3]);
+              reinterpret_cast<uint4*>(arow + 3 * p.N + col)[v] =
+                  make_uint4(dul[4 * v], dul[4 * v + 1], dul[4 * v + 2], dul[4 * v + 3]);
+            }
+          } else {
+            // padding tokens of the transposed blocks must read as zeros
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i) {
+              const size_t o = static_cast<size_t>(col + i) * tstride + my_row;
+#pragma unroll
+              for (int b = 0; b < 3; ++b) {
+                p.tT[b * tblock + o] = 0;
+                p.tT[b * tblock + o + p.t_pad] = 0;
+              }
+            }
+          }
+        }
       } else if (MODE == kModeActivity) {
 #pragma unroll 1
         for (int ch = 0; ch < kBN / 32; ++ch) {
@@ -534,7 +682,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int col = n_blk * kBN + ch * 32;
           if (valid && col < p.N) {
             float* dst = p.out_f32 + static_cast<size_t>(orow) * p.ldo + col;
-            if (k_splits > 1) {
+            if (k_splits > 1 || p.accumulate) {
 #pragma unroll
               for (int v = 0; v < 8; ++v)
                 red_add_v4(dst + 4 * v, __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),

@@ -487,9 +487,10 @@ def run_gpu(args, world, rank, local):
 
 
 def run_gpu_backward(args, world, rank, local):
-    """The backward pass through the hybrid format: dx (per-token sparse pass,
-    overflow rows repacked at full width) then the weight gradients (column
-    sort, per-unit sums). The forward that produces the pack and the routing
+    """The backward pass through the hybrid format: dx (per-token sparse pass
+    for the rows that fit, tensor-core dense branch for overflow rows) then the
+    weight gradients (column sort and per-unit sums, plus the dense branch's
+    share). The forward that produces the pack and the routing
     runs once before timing: its outputs are the backward's inputs."""
     import torch
 
@@ -585,8 +586,10 @@ def run_gpu_backward(args, world, rank, local):
     n_ovf_h = int(n_ovf.item())
     nnz_fit = int(torch.clamp(counts, max=W)[~ovf_mask].sum())
     nnz_ovf = int(counts[ovf_mask].sum())  # true counts: every active unit of an overflow row
-    flops_dx = 8.0 * d * nnz_fit + 10.0 * d * nnz_ovf  # u, dh (and z) dots, two axpys per unit
-    flops_dw = 6.0 * d * (nnz_fit + nnz_ovf)           # three axpys per unit
+    # CUDA-core work of the rows that fit (the overflow rows' dense branch runs
+    # on the tensor cores: 12 n_ovf d f FLOPs, reported beside it)
+    flops_dx = 8.0 * d * nnz_fit  # u and dh dots, two axpys per stored unit
+    flops_dw = 6.0 * d * nnz_fit  # three axpys per stored unit
     clocks = sampler.summary()
     peaks = load_peaks()
     fp32_peak = (torch.cuda.get_device_properties(dev).multi_processor_count * FP32_LANES_PER_SM * 2
@@ -617,11 +620,12 @@ def run_gpu_backward(args, world, rank, local):
                      "unit": "TFLOP/s", "frac": achieved / (fp32_peak / 1e12), "traffic": None,
                      "peak_source": "fp32 FMA lanes x 2 x max SM clock"},
         "stages_ms": {n: float(v) for n, v in zip(names, stage_ms)},
-        "batch_stats": {"n_ovf": n_ovf_h, "nnz_fit_rows": nnz_fit, "nnz_overflow_rows": nnz_ovf},
+        "batch_stats": {"n_ovf": n_ovf_h, "nnz_fit_rows": nnz_fit, "nnz_overflow_rows": nnz_ovf,
+                        "dense_branch_gflop": 12.0 * n_ovf_h * d * f / 1e9},
         "dense_backward_ms": None,
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
-        "gpu_launches": 11 * K,
+        "gpu_launches": 13 * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -295,13 +295,15 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
  * same x (the gate form: tw's values are the bf16 gate). Rows that fit use
  * their stored slots with the stored bf16 gate g (h = g u), so the result is
  * the method's, within one bf16 rounding per term of the exact gradients;
- * overflow rows are packed again at the full tile width from the gathered
- * rows and use the gate recomputed in fp32. The weight gradients are summed
- * per hidden unit over a column sort of the slots; the order of the terms
- * inside a column is not fixed, so the fp32 sums are not bit-reproducible.
+ * their weight gradients are summed per hidden unit over a column sort of the
+ * slots (the order of the terms inside a column is not fixed, so the fp32 sums
+ * are not bit-reproducible). Overflow rows take the dense branch on the tensor
+ * cores: [z | u] recomputed, dh = dy Wd^T with dz, du, h formed in its
+ * epilogue (kept as bf16 plus bf16 remainder), dx = [dz | du] [Wg; Wu]^T, and
+ * their share of the weight gradients added by three GEMMs over their tokens.
  * workspace: twell_backward_workspace_bytes(T, d, f, tw->W) bytes (worst case:
  * every row overflows). T == 0 zeroes the weight gradients. Errors as for
- * twell_ffn_hybrid_forward; T * (f / 128) * 128 must stay below 2^31.
+ * twell_ffn_hybrid_forward; T * (f / 128) * W must stay below 2^31.
  */
 size_t twell_backward_workspace_bytes(int T, int d, int f, int W);
 twell_status twell_ffn_hybrid_backward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,

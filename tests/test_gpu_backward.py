@@ -1,9 +1,11 @@
 """GPU parity of the backward pass through the hybrid format against the CPU
 oracle. The forward (gate form) provides the pack and the routing; each
 gradient (dx, dWgT, dWuT, dWd) must satisfy max|g - g_ref| <= 2e-2 * rms(g_ref)
-against the oracle's result of the method. The kernels sum in fp32 what the
-oracle sums in fp64 from the same bf16 values, so a much tighter 1e-3 * rms is
-also required."""
+against the oracle's result of the method. Rows that fit are summed in fp32
+from the same bf16 values the oracle sums in fp64, so a much tighter
+1e-3 * rms is also required; the overflow rows' dense branch holds dz, du and
+h as bf16 value plus bf16 remainder (relative error <= 2^-16 per term), so
+their share may in addition move by 2^-15 * sum |term|."""
 
 import numpy as np
 import pytest
@@ -54,12 +56,37 @@ def forward_backward(L, cfg, dy_bits):
     return {k: v.double().cpu().numpy() for k, v in g.items()}, ovf_rows[:n].cpu().numpy()
 
 
-def assert_grad_close(got: np.ndarray, ref: np.ndarray, name: str) -> None:
+def assert_grad_close(got: np.ndarray, ref: np.ndarray, name: str, pair_bound=None) -> None:
     assert np.isfinite(got).all(), name
     rms = float(np.sqrt(np.mean(ref**2)))
-    err = float(np.abs(got - ref).max())
-    assert err <= CONTRACT * rms, f"{name}: {err:.3e} > {CONTRACT} * rms {rms:.3e}"
-    assert err <= TIGHT * rms, f"{name}: {err:.3e} > {TIGHT} * rms {rms:.3e}"
+    err = np.abs(got - ref)
+    assert err.max() <= CONTRACT * rms, f"{name}: {err.max():.3e} > {CONTRACT} * rms {rms:.3e}"
+    tight = TIGHT * rms + (0.0 if pair_bound is None else pair_bound)
+    assert np.all(err <= tight), f"{name}: {float((err / tight).max()):.3f} x the tight bound"
+
+
+def dense_branch_bounds(L, dy_bits, ovf, rows=None, cols=None) -> dict:
+    """2^-15 * sum |term| of the overflow rows' share: per sampled row of dx
+    (zero for rows that fit) and per sampled unit of the weight gradients."""
+    F = O.bf16_bits_to_f64
+    x, dyv = F(L["x"][ovf]), F(dy_bits[ovf])
+    WgT, WuT, Wd = F(L["WgT"]), F(L["WuT"]), F(L["Wd"])
+    sel = slice(None) if cols is None else cols
+    z, u = x @ WgT[sel].T, x @ WuT[sel].T
+    g = np.maximum(z, 0)
+    dh = dyv @ Wd[sel].T
+    dz, du, h = np.abs(np.where(z > 0, dh * u, 0)), np.abs(dh * g), np.abs(g * u)
+    k = 2.0**-15
+    out = {"dWgT": k * dz.T @ np.abs(x), "dWuT": k * du.T @ np.abs(x), "dWd": k * h.T @ np.abs(dyv)}
+    if rows is not None:
+        bx = np.zeros((len(rows), x.shape[1]))
+        pos = {int(r): i for i, r in enumerate(ovf)}
+        for i, r in enumerate(rows):
+            if int(r) in pos:
+                q = pos[int(r)]
+                bx[i] = k * (dz[q] @ np.abs(WgT) + du[q] @ np.abs(WuT))
+        out["dx"] = bx
+    return out
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=IDS)
@@ -69,8 +96,9 @@ def test_hybrid_backward(cfg):
     got, ovf = forward_backward(L, cfg, dy)
     ref = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, cfg.tile, cfg.W)
     assert np.array_equal(ovf, ref["ovf_rows"])
+    b = dense_branch_bounds(L, dy, ovf, rows=np.arange(cfg.T)) if ovf.size else {}
     for k in GRADS:
-        assert_grad_close(got[k], ref[k], k)
+        assert_grad_close(got[k], ref[k], k, b.get(k))
 
 
 def test_backward_of_an_all_negative_gate_is_zero():
@@ -96,11 +124,14 @@ def test_full_size_hybrid_backward(name):
     rng = np.random.default_rng(3)
     rows = np.union1d(np.sort(rng.choice(cfg.T, size=128, replace=False)), ovf[:32])
     ref_rows = O.hybrid_ffn_backward(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], dy[rows], cfg.tile, cfg.W)
-    assert_grad_close(got["dx"][rows], ref_rows["dx"], "dx")
+    ovf_in = np.intersect1d(rows, ovf)  # the sampled rows that took the dense branch
+    bx = dense_branch_bounds(L, dy, ovf_in, rows=rows) if ovf_in.size else {}
+    assert_grad_close(got["dx"][rows], ref_rows["dx"], "dx", bx.get("dx"))
     cols = np.sort(rng.choice(cfg.f, size=48, replace=False))
     ref_cols = O.hybrid_backward_weight_rows(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, ovf, cols)
+    bw = dense_branch_bounds(L, dy, ovf, cols=cols) if ovf.size else {}
     for k in ("dWgT", "dWuT", "dWd"):
-        assert_grad_close(got[k][cols], ref_cols[k], k)
+        assert_grad_close(got[k][cols], ref_cols[k], k, bw.get(k))
 
 
 def test_split_backward_matches_the_oracle():
@@ -126,6 +157,7 @@ def test_split_backward_matches_the_oracle():
     assert tl.status_get(st) == 0
     ref = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy_bits, cfg.tile, cfg.W)
     assert int(n_ovf.item()) > 0
-    assert_grad_close(dx.double().cpu().numpy(), ref["dx"], "dx")
+    b = dense_branch_bounds(L, dy_bits, ref["ovf_rows"], rows=np.arange(T))
+    assert_grad_close(dx.double().cpu().numpy(), ref["dx"], "dx", b["dx"])
     for k, t in zip(("dWgT", "dWuT", "dWd"), dW):
-        assert_grad_close(t.double().cpu().numpy(), ref[k], k)
+        assert_grad_close(t.double().cpu().numpy(), ref[k], k, b[k])
