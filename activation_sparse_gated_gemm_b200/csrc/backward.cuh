@@ -45,7 +45,26 @@ struct BwdParams {
 
 // Warps per block of the per-token pass: x_t, dy_t (shared memory), dx_t and
 // two weight rows (registers) per warp.
-constexpr int bwd_warps_for(int nch) { return nch <= 3 ? 12 : 8; }
+constexpr int bwd_warps_for(int nch) { return nch <= 3 ? 12 : (nch <= 10 ? 8 : 5); }
+// From this many 256-element chunks of d on, dx_t waits in shared memory while
+// the dot passes run (registers hold either dx_t or the dot passes' rows).
+constexpr int kBwdAccSmemNch = 7;
+
+// Bytes of dynamic shared memory per block of the per-token pass.
+constexpr size_t bwd_smem_bytes(int nch) {
+  return static_cast<size_t>(bwd_warps_for(nch)) *
+         (2 * nch * 32 * 16 + kListCap * 6 + (nch >= kBwdAccSmemNch ? nch * 32 * 32 : 0));
+}
+
+// 16-byte shared-memory load that the compiler keeps inside its loop (x_t and
+// dy_t are reread per entry instead of being held in registers across it).
+__device__ __forceinline__ uint4 lds_v4(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
 
 // For the entries s < ns of a batch (column my_j on lane s): lane s receives
 // <src, M[j_s, :]>, src being a row parked in shared memory. Two row buffers
@@ -63,8 +82,8 @@ __device__ __forceinline__ float bwd_dot_pass(const uint4* src, const uint16_t* 
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
       for (int i = 0; i < NCH; i += 2) {
-        mixdot8(src[i * 32 + lane], wa[i], a0, a1);
-        if (i + 1 < NCH) mixdot8(src[(i + 1) * 32 + lane], wa[i + 1], a2, a3);
+        mixdot8(lds_v4(src + i * 32 + lane), wa[i], a0, a1);
+        if (i + 1 < NCH) mixdot8(lds_v4(src + (i + 1) * 32 + lane), wa[i + 1], a2, a3);
       }
       float acc = (a0 + a1) + (a2 + a3);
 #pragma unroll
@@ -77,8 +96,8 @@ __device__ __forceinline__ float bwd_dot_pass(const uint4* src, const uint16_t* 
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
       for (int i = 0; i < NCH; i += 2) {
-        mixdot8(src[i * 32 + lane], wb[i], a0, a1);
-        if (i + 1 < NCH) mixdot8(src[(i + 1) * 32 + lane], wb[i + 1], a2, a3);
+        mixdot8(lds_v4(src + i * 32 + lane), wb[i], a0, a1);
+        if (i + 1 < NCH) mixdot8(lds_v4(src + (i + 1) * 32 + lane), wb[i + 1], a2, a3);
       }
       float acc = (a0 + a1) + (a2 + a3);
 #pragma unroll
@@ -127,6 +146,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
   uint16_t* lpos = reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) +
                                                WARPS * kListCap) +
                    warp * kListCap;
+  constexpr bool kAccSmem = NCH >= kBwdAccSmemNch;
+  // dx_t parked between batches: [NCH][32 lanes] float4 pairs, after the lists
+  float4* acc_s = reinterpret_cast<float4*>(reinterpret_cast<uint16_t*>(
+                      reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) + WARPS * kListCap) +
+                                            WARPS * kListCap) +
+                  warp * NCH * 32 * 2;
   const int group_tiles = max(1, kListCap / p.W);
   const int rows = p.rows;
   bool bad_index = false;
@@ -157,6 +182,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
     for (int i = 0; i < NCH; ++i)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
+    if (kAccSmem) {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        acc_s[(i * 32 + lane) * 2] = make_float4(0.f, 0.f, 0.f, 0.f);
+        acc_s[(i * 32 + lane) * 2 + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
     const size_t slot_row = static_cast<size_t>(t) * p.nT * p.W;
 
 #pragma unroll 1
@@ -211,9 +243,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
         const int my_j = entry_j(my_e);
         const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
         const bool valid = (my_pos & 0x8000u) == 0;
-        // u_j = x . Wu[:, j], dh_j = dy . Wd[j, :]
+        // u_j = x . Wu[:, j], dh_j = dy . Wd[j, :]. The empty asm statements
+        // with a memory clobber keep each pass's first gather from being
+        // started inside the previous pass, which would hold a third row of
+        // registers live.
         const float my_u = bwd_dot_pass<NCH>(xs, p.WuT, my_j, ns, lane, d);
+        asm volatile("" ::: "memory");
         const float my_dh = bwd_dot_pass<NCH>(ds, p.Wd, my_j, ns, lane, d);
+        asm volatile("" ::: "memory");
         const float my_g = entry_g(my_e);
         const float my_du = valid ? my_dh * my_g : 0.0f;
         const float my_dz = valid ? my_dh * my_u : 0.0f;
@@ -224,8 +261,25 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
           p.s_dz[slot] = my_dz;
         }
         // dx_t += dz_j Wg[:, j] + du_j Wu[:, j]
+        if (kAccSmem) {
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const float4 a = acc_s[(i * 32 + lane) * 2], b = acc_s[(i * 32 + lane) * 2 + 1];
+            acc[i][0] = a.x, acc[i][1] = a.y, acc[i][2] = a.z, acc[i][3] = a.w;
+            acc[i][4] = b.x, acc[i][5] = b.y, acc[i][6] = b.z, acc[i][7] = b.w;
+          }
+        }
         bwd_axpy_pass<NCH>(acc, p.WgT, my_j, my_dz, ns, lane, d);
+        asm volatile("" ::: "memory");
         bwd_axpy_pass<NCH>(acc, p.WuT, my_j, my_du, ns, lane, d);
+        if (kAccSmem) {
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            acc_s[(i * 32 + lane) * 2] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+            acc_s[(i * 32 + lane) * 2 + 1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+          }
+        }
+        asm volatile("" ::: "memory");
       }
       __syncwarp();
     }
@@ -234,8 +288,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
       const int k0 = (i * 32 + lane) * 8;
       if (k0 < d) {
         float4* dst = reinterpret_cast<float4*>(p.dx + static_cast<size_t>(t) * d + k0);
-        dst[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-        dst[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+        if (kAccSmem) {
+          dst[0] = acc_s[(i * 32 + lane) * 2];
+          dst[1] = acc_s[(i * 32 + lane) * 2 + 1];
+        } else {
+          dst[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+          dst[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+        }
       }
     }
   }

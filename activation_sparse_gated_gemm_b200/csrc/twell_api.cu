@@ -445,7 +445,7 @@ BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
 template <int NCH>
 twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
   constexpr int kWarps = bwd_warps_for(NCH);
-  const size_t smem = static_cast<size_t>(kWarps) * (2 * NCH * 32 * sizeof(uint4) + kListCap * 6);
+  const size_t smem = bwd_smem_bytes(NCH);
   auto kern = bwd_token_kernel<NCH, kWarps>;
   if (smem > 48 * 1024)
     TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
@@ -537,6 +537,7 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   q2.a2 = w.a2;
   q2.tT = w.tT;
   q2.t_pad = w.t_pad;
+  q2.h_split = 1;
   q2.dev_status = dev_status;
   TW_TRY(launch_gemm<kModeBwdDh>(mdy, mwd, mwd, q2, sms, s));
   GemmParams q3{};
@@ -956,6 +957,104 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
   TW_TRY(current_device(&dev, &sms));
   return backward_dw_impl(x, dy, T, d, f, tw, n_ovf, dWgT, dWuT, dWd, static_cast<char*>(workspace),
                           static_cast<cudaStream_t>(stream), sms);
+}
+
+size_t twell_dense_backward_workspace_bytes(int T, int d, int f) {
+  (void)d;
+  if (T <= 0 || f <= 0) return 0;
+  const size_t tp = round_up(static_cast<size_t>(T), 64);
+  return round_up(static_cast<size_t>(T) * f * 8, 256)        // [z | u] fp32
+         + round_up(static_cast<size_t>(T) * f * 4, 256)      // [dz | du] bf16
+         + round_up(3 * static_cast<size_t>(f) * tp * 2, 256);  // dz, du, h unit-major bf16
+}
+
+twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                      const uint16_t* Wd, const uint16_t* dy, int T, int d, int f, float* dx,
+                                      float* dWgT, float* dWuT, float* dWd, void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_ptrs({dWgT, dWuT, dWd, dev_status}));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    const size_t n = static_cast<size_t>(f) * d * sizeof(float);
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWgT, 0, n, s)));
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWuT, 0, n, s)));
+    return cuda_ok(cudaMemsetAsync(dWd, 0, n, s));
+  }
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, dy, dx}));
+  if (workspace == nullptr || workspace_bytes < twell_dense_backward_workspace_bytes(T, d, f))
+    return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  char* ws = static_cast<char*>(workspace);
+  const int tp = static_cast<int>(round_up(static_cast<size_t>(T), 64));
+  float* zu = reinterpret_cast<float*>(ws);
+  uint16_t* a2 = reinterpret_cast<uint16_t*>(ws + round_up(static_cast<size_t>(T) * f * 8, 256));
+  uint16_t* tT = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(a2) + round_up(static_cast<size_t>(T) * f * 4, 256));
+  CUtensorMap mx, mdy, mg, mu, mwd, ma2, mgT, muT;
+  if (!make_map(&mx, x, d, T, kBK, kBM) || !make_map(&mdy, dy, d, T, kBK, kBM) ||
+      !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128) ||
+      !make_map(&mwd, Wd, d, f, kBK, kBN) || !make_map(&ma2, a2, 2 * f, T, kBK, kBM) ||
+      !make_map(&mgT, WgT, d, f, 64, kBK) || !make_map(&muT, WuT, d, f, 64, kBK))
+    return TWELL_ERR_CUDA;
+  // [z | u] = x [Wg | Wu]; dh = dy Wd^T with dz, du, h (bf16) in the epilogue
+  GemmParams q1{};
+  q1.M = T;
+  q1.N = f;
+  q1.K = d;
+  q1.out_f32 = zu;
+  q1.ldo = 2 * f;
+  q1.dev_status = dev_status;
+  TW_TRY(launch_gemm<kModeZU>(mx, mg, mu, q1, gemm_grid(T, f, 128, sms), s));
+  GemmParams q2{};
+  q2.M = T;
+  q2.N = f;
+  q2.K = d;
+  q2.zu = zu;
+  q2.a2 = a2;
+  q2.tT = tT;
+  q2.t_pad = tp;
+  q2.h_split = 0;
+  q2.dev_status = dev_status;
+  TW_TRY(launch_gemm<kModeBwdDh>(mdy, mwd, mwd, q2, gemm_grid(T, f, kBN, sms), s));
+  // dx = [dz | du] [Wg; Wu]^T: K split (into a zeroed dx) only when the tiles cannot fill the GPU
+  GemmParams q3{};
+  q3.M = T;
+  q3.N = d;
+  q3.K = 2 * f;
+  q3.k_split_b = f;
+  q3.out_f32 = dx;
+  q3.ldo = d;
+  q3.k_splits_max = 1;
+  q3.dev_status = dev_status;
+  if (static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms) {
+    TW_TRY(cuda_ok(cudaMemsetAsync(dx, 0, static_cast<size_t>(T) * d * sizeof(float), s)));
+    q3.k_splits_max = 32;
+  }
+  TW_TRY(launch_gemm<kModeDown>(ma2, mgT, muT, q3, q3.k_splits_max > 1 ? sms : gemm_grid(T, d, kBN, sms), s));
+  // dWgT = dz^T x, dWuT = du^T x, dWd = h^T dy (K = the tokens; rows of x and
+  // dy past T are read as zeros by the tensor maps)
+  const size_t tblock = static_cast<size_t>(f) * tp;
+  const uint16_t* aT[3] = {tT, tT + tblock, tT + 2 * tblock};
+  const uint16_t* bT[3] = {x, x, dy};
+  float* outs[3] = {dWgT, dWuT, dWd};
+  const bool split = static_cast<long long>(f / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms;
+  for (int i = 0; i < 3; ++i) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, aT[i], tp, f, kBK, kBM) || !make_map(&mb, bT[i], d, T, 64, kBK)) return TWELL_ERR_CUDA;
+    GemmParams q{};
+    q.M = f;
+    q.N = d;
+    q.K = tp;
+    q.out_f32 = outs[i];
+    q.ldo = d;
+    q.k_splits_max = split ? 32 : 1;
+    q.dev_status = dev_status;
+    if (split) TW_TRY(cuda_ok(cudaMemsetAsync(outs[i], 0, static_cast<size_t>(f) * d * sizeof(float), s)));
+    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, split ? sms : gemm_grid(f, d, kBN, sms), s));
+  }
+  return TWELL_OK;
 }
 
 twell_status twell_column_activity(const uint16_t* x, const uint16_t* WgT, int T, int d, int f,

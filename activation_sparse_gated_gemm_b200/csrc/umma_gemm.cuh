@@ -114,7 +114,9 @@ struct GemmParams {
   // kModeBwdDh: zu = [z | u] rows ([M][2N] fp32); a2 = [M][4N] bf16 rows
   // [dz | du | dz_lo | du_lo]; tT = three [N][2 t_pad] bf16 blocks (dz, du, h),
   // unit-major, tokens [0, t_pad) holding bf16(v) and [t_pad, 2 t_pad) the
-  // remainder; rows in [M, t_pad) of the tile are written as zeros.
+  // remainder; rows in [M, t_pad) of the tile are written as zeros. With
+  // h_split == 0 only the bf16 values are kept: a2 = [M][2N] rows [dz | du],
+  // tT = three [N][t_pad] blocks.
   const float* zu;
   uint16_t* a2;
   uint16_t* tT;
@@ -540,7 +542,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else if (MODE == kModeBwdDh) {
-        const size_t tstride = 2 * static_cast<size_t>(p.t_pad);  // one unit's row in a transposed block
+        const bool pair = p.h_split != 0;
+        const size_t tstride = (pair ? 2 : 1) * static_cast<size_t>(p.t_pad);  // one unit's row, transposed
         const size_t tblock = static_cast<size_t>(p.N) * tstride;
 #pragma unroll 1
         for (int ch = 0; ch < kBN / 32; ++ch) {
@@ -588,24 +591,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const uint16_t uh = f32_to_bf16_bits(vu[e]);
                 const uint16_t hh = f32_to_bf16_bits(vh[e]);
                 p.tT[o] = zh;
-                p.tT[o + p.t_pad] = f32_to_bf16_bits(vz[e] - __uint_as_float(static_cast<uint32_t>(zh) << 16));
                 p.tT[tblock + o] = uh;
-                p.tT[tblock + o + p.t_pad] = f32_to_bf16_bits(vu[e] - __uint_as_float(static_cast<uint32_t>(uh) << 16));
                 p.tT[2 * tblock + o] = hh;
-                p.tT[2 * tblock + o + p.t_pad] =
-                    f32_to_bf16_bits(vh[e] - __uint_as_float(static_cast<uint32_t>(hh) << 16));
+                if (pair) {
+                  p.tT[o + p.t_pad] = f32_to_bf16_bits(vz[e] - __uint_as_float(static_cast<uint32_t>(zh) << 16));
+                  p.tT[tblock + o + p.t_pad] =
+                      f32_to_bf16_bits(vu[e] - __uint_as_float(static_cast<uint32_t>(uh) << 16));
+                  p.tT[2 * tblock + o + p.t_pad] =
+                      f32_to_bf16_bits(vh[e] - __uint_as_float(static_cast<uint32_t>(hh) << 16));
+                }
               }
             }
-            uint16_t* arow = p.a2 + static_cast<size_t>(my_row) * 4 * p.N;
+            uint16_t* arow = p.a2 + static_cast<size_t>(my_row) * (pair ? 4 : 2) * p.N;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               reinterpret_cast<uint4*>(arow + col)[v] = make_uint4(dzh[4 * v], dzh[4 * v + 1], dzh[4 * v + 2], dzh[4 * v + 3]);
               reinterpret_cast<uint4*>(arow + p.N + col)[v] =
                   make_uint4(duh[4 * v], duh[4 * v + 1], duh[4 * v + 2], duh[4 * v + 3]);
-              reinterpret_cast<uint4*>(arow + 2 * p.N + col)[v] =
-                  make_uint4(dzl[4 * v], dzl[4 * v + 1], dzl[4 * v + 2], dzl[4 * v + 3]);
-              reinterpret_cast<uint4*>(arow + 3 * p.N + col)[v] =
-                  make_uint4(dul[4 * v], dul[4 * v + 1], dul[4 * v + 2], dul[4 * v + 3]);
+              if (pair) {
+                reinterpret_cast<uint4*>(arow + 2 * p.N + col)[v] =
+                    make_uint4(dzl[4 * v], dzl[4 * v + 1], dzl[4 * v + 2], dzl[4 * v + 3]);
+                reinterpret_cast<uint4*>(arow + 3 * p.N + col)[v] =
+                    make_uint4(dul[4 * v], dul[4 * v + 1], dul[4 * v + 2], dul[4 * v + 3]);
+              }
             }
           } else {
             // padding tokens of the transposed blocks must read as zeros
@@ -615,7 +623,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int b = 0; b < 3; ++b) {
                 p.tT[b * tblock + o] = 0;
-                p.tT[b * tblock + o + p.t_pad] = 0;
+                if (pair) p.tT[b * tblock + o + p.t_pad] = 0;
               }
             }
           }

@@ -33,7 +33,7 @@ EXPORTED = (
     "twell_relu_ffn_hybrid_forward", "twell_relu_dense_rows_forward", "twell_relu_dense_ffn_forward",
     "twell_column_activity", "twell_compact_columns", "twell_gather_rows",
     "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward", "twell_ffn_hybrid_backward_dx",
-    "twell_ffn_hybrid_backward_dw",
+    "twell_ffn_hybrid_backward_dw", "twell_dense_backward_workspace_bytes", "twell_dense_ffn_backward",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -92,6 +92,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                       i32),
         "twell_ffn_hybrid_backward_dx": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_ffn_hybrid_backward_dw": ([vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, sz, vp], i32),
+        "twell_dense_backward_workspace_bytes": ([i32, i32, i32], sz),
+        "twell_dense_ffn_backward": ([vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_column_activity": ([vp, vp, i32, i32, i32, vp, i32, vp, vp], i32),
         "twell_compact_columns": ([vp, i32, vp, vp, vp], i32),
         "twell_gather_rows": ([vp, i32, i32, vp, vp, i32, vp, vp, vp], i32),
@@ -369,6 +371,24 @@ def ffn_hybrid_backward_dw(x, dy, tw: Twell, n_ovf, dWgT, dWuT, dWd, workspace, 
     _check("twell_ffn_hybrid_backward_dw", load().twell_ffn_hybrid_backward_dw(
         _ptr(x), _ptr(dy), T, d, f, tw.ref(), _ptr(n_ovf), _ptr(dWgT), _ptr(dWuT), _ptr(dWd), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dense_backward_workspace_bytes(T: int, d: int, f: int) -> int:
+    return int(load().twell_dense_backward_workspace_bytes(T, d, f))
+
+
+def dense_ffn_backward(x, WgT, WuT, Wd, dy, dx, dWgT, dWuT, dWd, workspace, dev_status, stream=None) -> None:
+    """The library's dense backward (tensor cores, bf16 dz/du/h): the baseline of the hybrid backward."""
+    T, d = x.shape
+    f = WgT.shape[0]
+    for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
+                    ("dy", dy, (T, d))):
+        _bf16(n, t, s)
+    for n, t, s in (("dx", dx, (T, d)), ("dWgT", dWgT, (f, d)), ("dWuT", dWuT, (f, d)), ("dWd", dWd, (f, d))):
+        _dev(n, t, s, torch.float32)
+    _check("twell_dense_ffn_backward", load().twell_dense_ffn_backward(
+        _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), _ptr(dy), T, d, f, _ptr(dx), _ptr(dWgT), _ptr(dWuT), _ptr(dWd),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
 
 
 def column_activity(x, WgT, active_bits, accumulate: bool, dev_status, stream=None) -> None:

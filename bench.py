@@ -553,6 +553,28 @@ def run_gpu_backward(args, world, rank, local):
     stage_ms = per.mean(axis=0)
     step_ms = max_over_ranks(float(per.sum(axis=1).mean()), world)
 
+    # the library's dense backward at the same shape (tensor cores, bf16 dz/du/h)
+    wsd = torch.empty(tl.dense_backward_workspace_bytes(T, d, f), dtype=torch.uint8, device=dev)
+    dxd = torch.empty_like(dx)
+    dWdn = [torch.empty_like(g) for g in dW]
+
+    def dense_bwd():
+        tl.dense_ffn_backward(x, WgT, WuT, Wd, dy, dxd, dWdn[0], dWdn[1], dWdn[2], wsd, st)
+
+    for _ in range(Wm):
+        flush.zero_()
+        dense_bwd()
+    dense_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    for k in range(K):
+        flush.zero_()
+        dense_ev[k][0].record(stream)
+        dense_bwd()
+        dense_ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    dense_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dense_ev])), world)
+    del wsd, dxd, dWdn
+
     # e2e through the C ABI: dy from pinned host memory in, dx and the weight gradients out
     dy_host = dy.cpu().pin_memory()
     dx_host = torch.empty((T, d), dtype=torch.float32).pin_memory()
@@ -622,7 +644,8 @@ def run_gpu_backward(args, world, rank, local):
         "stages_ms": {n: float(v) for n, v in zip(names, stage_ms)},
         "batch_stats": {"n_ovf": n_ovf_h, "nnz_fit_rows": nnz_fit, "nnz_overflow_rows": nnz_ovf,
                         "dense_branch_gflop": 12.0 * n_ovf_h * d * f / 1e9},
-        "dense_backward_ms": None,
+        "dense_backward_ms": dense_ms,
+        "speedup_vs_own_dense": dense_ms / step_ms,
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
         "gpu_launches": 13 * K,

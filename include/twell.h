@@ -330,6 +330,22 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
                                           float* dWd, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Dense backward of the gated layer on the tensor cores, no sparsity: the
+ * library's own baseline for twell_ffn_hybrid_backward. [z | u] = x [Wg | Wu]
+ * (fp32), dh = dy Wd^T with dz = dh u [z > 0], du = dh ReLU(z), h = ReLU(z) u
+ * formed in that GEMM's epilogue and stored once as bf16 (as a standard bf16
+ * layer does), then dx = [dz | du] [Wg; Wu]^T and dWgT = dz^T x, dWuT = du^T x,
+ * dWd = h^T dy (fp32, overwritten). Its error is that of one bf16 rounding of
+ * dz, du and h: at most 2^-8 of the summed magnitudes of the terms, plus fp32
+ * sums. Workspace: twell_dense_backward_workspace_bytes(T, d, f).
+ */
+size_t twell_dense_backward_workspace_bytes(int T, int d, int f);
+twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                      const uint16_t* Wd, const uint16_t* dy, int T, int d, int f, float* dx,
+                                      float* dWgT, float* dWuT, float* dWd, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * Dead hidden units (intellectnews.ru, "Sakana AI и NVIDIA: TwELL ...",
  * section "Ограничения и открытые вопросы": under the chosen L1 setting some
  * units die, i.e. are never active). Three calls compact a layer to the units

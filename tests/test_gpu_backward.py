@@ -65,9 +65,10 @@ def assert_grad_close(got: np.ndarray, ref: np.ndarray, name: str, pair_bound=No
     assert np.all(err <= tight), f"{name}: {float((err / tight).max()):.3f} x the tight bound"
 
 
-def dense_branch_bounds(L, dy_bits, ovf, rows=None, cols=None) -> dict:
-    """2^-15 * sum |term| of the overflow rows' share: per sampled row of dx
-    (zero for rows that fit) and per sampled unit of the weight gradients."""
+def dense_branch_bounds(L, dy_bits, ovf, rows=None, cols=None, k=2.0**-15) -> dict:
+    """k * sum |term| of the rows `ovf` (by default 2^-15, the bf16 value and
+    remainder pair's error): per sampled row of dx (zero for other rows) and
+    per sampled unit of the weight gradients."""
     F = O.bf16_bits_to_f64
     x, dyv = F(L["x"][ovf]), F(dy_bits[ovf])
     WgT, WuT, Wd = F(L["WgT"]), F(L["WuT"]), F(L["Wd"])
@@ -76,7 +77,6 @@ def dense_branch_bounds(L, dy_bits, ovf, rows=None, cols=None) -> dict:
     g = np.maximum(z, 0)
     dh = dyv @ Wd[sel].T
     dz, du, h = np.abs(np.where(z > 0, dh * u, 0)), np.abs(dh * g), np.abs(g * u)
-    k = 2.0**-15
     out = {"dWgT": k * dz.T @ np.abs(x), "dWuT": k * du.T @ np.abs(x), "dWd": k * h.T @ np.abs(dyv)}
     if rows is not None:
         bx = np.zeros((len(rows), x.shape[1]))
@@ -161,3 +161,30 @@ def test_split_backward_matches_the_oracle():
     assert_grad_close(dx.double().cpu().numpy(), ref["dx"], "dx", b["dx"])
     for k, t in zip(("dWgT", "dWuT", "dWd"), dW):
         assert_grad_close(t.double().cpu().numpy(), ref[k], k, b[k])
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_dense_backward_baseline(cfg):
+    """The library's dense backward (one bf16 rounding of dz, du, h) against
+    the exact gradients: within 2^-7 of the summed term magnitudes (2^-8 for
+    the rounding, the rest for fp32 sums)."""
+    L = synth.make_layer(cfg, seed=0)
+    dy_bits = make_dy(cfg.T, cfg.d, 5)
+    dev = upload(L)
+    T, d, f = cfg.T, cfg.d, cfg.f
+    dy = tl.to_device_bf16(dy_bits)
+    g = {k: torch.full((T if k == "dx" else f, d), float("nan"), dtype=torch.float32, device="cuda")
+         for k in GRADS}
+    ws = torch.empty(tl.dense_backward_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.dense_ffn_backward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], dy, g["dx"], g["dWgT"], g["dWuT"], g["dWd"],
+                          ws, st)
+    assert tl.status_get(st) == 0
+    ref = O.gated_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy_bits)
+    b = dense_branch_bounds(L, dy_bits, np.arange(T), rows=np.arange(T), k=2.0**-7)
+    for k in GRADS:
+        got = g[k].double().cpu().numpy()
+        assert np.isfinite(got).all(), k
+        err = np.abs(got - ref[k])
+        bound = b[k] + 1e-6 * float(np.sqrt(np.mean(ref[k] ** 2)))
+        assert np.all(err <= bound), (k, float((err / bound).max()))
