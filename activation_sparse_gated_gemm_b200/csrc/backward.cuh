@@ -136,6 +136,8 @@ __device__ __forceinline__ void bwd_axpy_pass(float (&acc)[NCH][8], const uint16
 // the slot position of every list entry inside the row's [nT][W] block.
 template <int NCH, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
   extern __shared__ uint4 bwd_smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -324,6 +326,8 @@ __device__ __forceinline__ int source_rows(const SlotSource& s) {
 // tag | slot index (the order inside a column is that of the atomics).
 template <bool SCATTER>
 __global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colptr, uint32_t* list) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int rows = source_rows(src);
   const long long pairs = static_cast<long long>(rows) * src.nT;
@@ -350,6 +354,8 @@ __global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colpt
 // colptr[j] = sum of colcnt[0..j) for j <= f, and colcnt is reset to zero (it
 // then serves as the scatter cursor). One block of 1024 threads.
 __global__ void __launch_bounds__(1024) bwd_column_scan_kernel(int* colcnt, int f, int* colptr) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int warp_sums[32];
   __shared__ int carry;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -408,6 +414,8 @@ struct WgradParams {
 // elements of the slice; the unit's slots are read 32 at a time (lane e
 // fetches entry e's scalars and row), then broadcast one by one.
 __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int slices = (p.d + 255) / 256;
   const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);

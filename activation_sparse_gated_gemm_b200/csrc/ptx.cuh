@@ -191,6 +191,18 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// ---------------------------------------------------------------- dependent launch
+
+// Programmatic dependent launch. Every kernel of the library first lets the
+// next kernel in the stream start launching (its blocks then run their own
+// setup while this grid finishes), and waits for the previous kernel to have
+// completed, with its memory visible, before touching anything that kernel
+// may read or write. Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {

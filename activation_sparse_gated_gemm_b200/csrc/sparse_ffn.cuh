@@ -123,6 +123,8 @@ __device__ __forceinline__ int entry_j(uint32_t e) { return static_cast<int>(e &
 // read.
 template <int NCH, int WARPS, bool DOWN_ONLY>
 __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const SparseParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
   extern __shared__ uint4 smem_dyn[];  // xs: [WARPS][NCH * 32] uint4, then lists
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -312,6 +314,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
 // y[t, :] = 0 for the rows the sparse step will write (all rows, or those
 // without the overflow flag when overflow rows are skipped).
 __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf, int skip_ovf) {
+  griddep_launch_dependents();
+  griddep_wait();
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     if (skip_ovf && row_ovf[t]) continue;
     float4* row = reinterpret_cast<float4*>(y + static_cast<size_t>(t) * d);
@@ -333,6 +337,8 @@ __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf,
 __global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf,
                                                      const uint16_t* x = nullptr, int d = 0, uint16_t* xo = nullptr,
                                                      float* y_zero = nullptr) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int warp_off[32];
   __shared__ int total_s;
   const int lane = threadIdx.x & 31;
@@ -403,6 +409,8 @@ __global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int
 // GEMM whose K runs over out's rows in blocks of 64 reads zeros past n.
 __global__ void gather_rows_kernel(const uint16_t* x, int d, const int* rows, const int* n_rows, int T,
                                    uint16_t* out, float* y_zero, int* dev_status, int pad_rows = 0) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int n = min(max(*n_rows, 0), T);
   if (pad_rows > 0) {
     const int pad_end = min((n + 63) / 64 * 64, pad_rows);
@@ -431,6 +439,8 @@ __global__ void gather_rows_kernel(const uint16_t* x, int d, const int* rows, co
 // as zeros, then scatters the stored slots.
 __global__ void __launch_bounds__(256) unpack_kernel(const int16_t* counts, const int16_t* idx, const uint16_t* vals,
                                                      int T, int nT, int W, int f, uint16_t* g, int* dev_status) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const long long wid = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (wid >= static_cast<long long>(T) * nT) return;
@@ -460,6 +470,8 @@ __global__ void __launch_bounds__(256) unpack_kernel(const int16_t* counts, cons
 __global__ void __launch_bounds__(1024) compact_columns_kernel(const uint32_t* __restrict__ active, int f,
                                                                 int32_t* __restrict__ col_map,
                                                                 int32_t* __restrict__ f_live) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int warp_sums[32];
   __shared__ int s_total;
   const int nwords = (f + 31) / 32;
@@ -504,6 +516,8 @@ __global__ void __launch_bounds__(1024) compact_columns_kernel(const uint32_t* _
 __global__ void gather_weight_rows_kernel(const uint16_t* __restrict__ W, int f, int d,
                                           const int32_t* __restrict__ col_map, const int32_t* __restrict__ f_live,
                                           int f_out, uint16_t* __restrict__ out, int* dev_status) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int n_live = min(max(*f_live, 0), f_out);
   const int lane = threadIdx.x & 31;
   const int vecs = d / 8;  // uint4 per row
@@ -540,6 +554,8 @@ __global__ void __launch_bounds__(256) pack_f32_kernel(const float* __restrict__
                                                        int16_t* __restrict__ counts, int16_t* __restrict__ idx,
                                                        uint16_t* __restrict__ vals, uint8_t* __restrict__ row_ovf,
                                                        float* __restrict__ y_zero, int d) {
+  griddep_launch_dependents();
+  griddep_wait();
   if (y_zero != nullptr) {
     const size_t n4 = static_cast<size_t>(T) * d / 4;
     for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
@@ -589,6 +605,8 @@ __global__ void __launch_bounds__(256) pack_f32_kernel(const float* __restrict__
 // half of the dense layer for a small batch), or bf16(ReLU(z)) from z [T][f]
 // when not gated.
 __global__ void h_from_zu_kernel(const float* __restrict__ zu, int T, int f, int gated, uint16_t* __restrict__ h) {
+  griddep_launch_dependents();
+  griddep_wait();
   const size_t per_row = static_cast<size_t>(f) / 4;
   const size_t n = static_cast<size_t>(T) * per_row;
   const size_t ldz = gated ? 2 * static_cast<size_t>(f) : static_cast<size_t>(f);
@@ -601,6 +619,33 @@ __global__ void h_from_zu_kernel(const float* __restrict__ zu, int T, int f, int
     o.x = pack_bf16x2(fmaxf(z.x, 0.f) * u.x, fmaxf(z.y, 0.f) * u.y);
     o.y = pack_bf16x2(fmaxf(z.z, 0.f) * u.z, fmaxf(z.w, 0.f) * u.w);
     reinterpret_cast<uint2*>(h + t * f)[q] = o;
+  }
+}
+
+// ---------------------------------------------------------------- zeroing
+
+// Up to three byte ranges set to zero by one launch (in place of memsets,
+// which would interrupt the chain of dependent launches).
+struct ZeroRanges {
+  void* p[3];
+  size_t n[3];
+};
+
+__global__ void zero_ranges_kernel(ZeroRanges r) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t nth = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (int k = 0; k < 3; ++k) {
+    uint8_t* b = static_cast<uint8_t*>(r.p[k]);
+    const size_t n = r.n[k];
+    if (b == nullptr || n == 0) continue;
+    const size_t head = min(n, (16 - (reinterpret_cast<uintptr_t>(b) & 15)) & 15);
+    const size_t body = (n - head) / 16;
+    for (size_t i = tid; i < head; i += nth) b[i] = 0;
+    uint4* b4 = reinterpret_cast<uint4*>(b + head);
+    for (size_t i = tid; i < body; i += nth) b4[i] = make_uint4(0, 0, 0, 0);
+    for (size_t i = head + body * 16 + tid; i < n; i += nth) b[i] = 0;
   }
 }
 

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "twell.h"
 #include "backward.cuh"
@@ -127,12 +128,39 @@ twell_status cuda_ok(cudaError_t e) {
 
 // ------------------------------------------------------------------ launches
 
+// Every kernel is launched as a programmatic dependent of the previous work in
+// the stream: its blocks may start (and run their private setup) while that
+// work finishes; each kernel waits for it before touching shared data.
+template <typename... KArgs, typename... Args>
+twell_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_ok(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
+}
+
+// Zero up to three device byte ranges with one dependent launch.
+twell_status zero_async(cudaStream_t s, int sms, void* p0, size_t n0, void* p1 = nullptr, size_t n1 = 0,
+                        void* p2 = nullptr, size_t n2 = 0) {
+  ZeroRanges r{{p0, p1, p2}, {n0, n1, n2}};
+  const size_t most = std::max(n0, std::max(n1, n2)) / 16 + 1;
+  const int blocks = static_cast<int>(std::min<size_t>((most + 255) / 256, 2 * static_cast<size_t>(sms)));
+  return launch(zero_ranges_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, s, r);
+}
+
 template <int MODE>
 twell_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, const GemmParams& p,
                          int grid, cudaStream_t s) {
   auto kern = umma_gemm_kernel<MODE>;
   TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes)));
-  kern<<<grid, kGemmThreads, kGemmSmemBytes, s>>>(a, b0, b1, p);
+  TW_TRY(launch(kern, dim3(grid), dim3(kGemmThreads), kGemmSmemBytes, s, a, b0, b1, p));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -143,7 +171,7 @@ int gemm_grid(int M, int N, int tile_n, int sms) {
 
 twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
                             int32_t* dev_status, cudaStream_t s, int sms, const int* M_dev = nullptr) {
-  TW_TRY(cuda_ok(cudaMemsetAsync(tw->row_ovf, 0, static_cast<size_t>(T), s)));
+  TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
   CUtensorMap ma, mb;
   if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mb, WgT, d, f, kBK, kBN)) return TWELL_ERR_CUDA;
   GemmParams p{};
@@ -164,7 +192,7 @@ twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d
 // Gate and up GEMM in one pass; TwELL of the gate pattern holding h = z * u.
 twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, int T, int d, int f,
                                const twell_t* tw, int32_t* dev_status, cudaStream_t s, int sms) {
-  TW_TRY(cuda_ok(cudaMemsetAsync(tw->row_ovf, 0, static_cast<size_t>(T), s)));
+  TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
   CUtensorMap ma, mg, mu;
   if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128))
     return TWELL_ERR_CUDA;
@@ -203,7 +231,7 @@ twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s, bool y_zer
     const long long per_token = std::max(1LL, std::min<long long>(p.nT, want_units / std::max(1, p.T)));
     p.unit_tiles = static_cast<int>((p.nT + per_token - 1) / per_token);
     if (p.unit_tiles < p.nT && !y_zeroed) {
-      zero_rows_kernel<<<std::min(p.T, 4 * sms), 256, 0, s>>>(p.y, p.T, p.d, p.row_ovf, p.skip_ovf);
+      TW_TRY(launch(zero_rows_kernel, dim3(std::min(p.T, 4 * sms)), dim3(256), 0, s, p.y, p.T, p.d, p.row_ovf, p.skip_ovf));
       TW_TRY(cuda_ok(cudaGetLastError()));
     }
   }
@@ -213,7 +241,7 @@ twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s, bool y_zer
   auto kern = sparse_ffn_warp_kernel<NCH, kWarps, DOWN_ONLY>;
   if (smem > 48 * 1024)
     TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
-  kern<<<blocks, kWarps * 32, smem, s>>>(p);
+  TW_TRY(launch(kern, dim3(blocks), dim3(kWarps * 32), smem, s, p));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -330,7 +358,7 @@ twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, con
   if (row_map != nullptr) {
     p2.k_splits_max = 32;
   } else if (static_cast<long long>((M + kBM - 1) / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms) {
-    TW_TRY(cuda_ok(cudaMemsetAsync(y, 0, static_cast<size_t>(M) * d * sizeof(float), s)));
+    TW_TRY(zero_async(s, sms, y, static_cast<size_t>(M) * d * sizeof(float)));
     p2.k_splits_max = 32;
   }
   p2.dev_status = dev_status;
@@ -376,12 +404,11 @@ twell_status f32_gemm_impl(const uint16_t* A, int M, const uint16_t* B, int N, i
 // the way when y_zero is given.
 twell_status small_gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
                                   float* zbuf, float* y_zero, int32_t* dev_status, cudaStream_t s, int sms) {
-  TW_TRY(cuda_ok(cudaMemsetAsync(tw->row_ovf, 0, static_cast<size_t>(T), s)));
-  TW_TRY(cuda_ok(cudaMemsetAsync(zbuf, 0, static_cast<size_t>(T) * f * sizeof(float), s)));
+  TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), zbuf, static_cast<size_t>(T) * f * sizeof(float)));
   TW_TRY(f32_gemm_impl(x, T, WgT, f, d, zbuf, f, dev_status, s, sms));
   const long long warps = static_cast<long long>(T) * (f / 128);
   const int blocks = static_cast<int>(std::min<long long>((warps + 7) / 8, 4LL * sms));
-  pack_f32_kernel<<<blocks, 256, 0, s>>>(zbuf, T, f, tw->W, tw->counts, tw->idx, tw->vals, tw->row_ovf, y_zero, d);
+  TW_TRY(launch(pack_f32_kernel, dim3(blocks), dim3(256), 0, s, zbuf, T, f, tw->W, tw->counts, tw->idx, tw->vals, tw->row_ovf, y_zero, d));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -390,7 +417,7 @@ twell_status small_gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T,
 twell_status dense_rows_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
                              int T, int d, int f, const int32_t* rows, const int32_t* n_rows, float* y,
                              uint16_t* xo, uint16_t* ho, int32_t* dev_status, cudaStream_t s, int sms) {
-  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, rows, n_rows, T, xo, y, dev_status);
+  TW_TRY(launch(gather_rows_kernel, dim3(sms * 2), dim3(256), 0, s, x, d, rows, n_rows, T, xo, y, dev_status, 0));
   TW_TRY(cuda_ok(cudaGetLastError()));
   return dense_impl(xo, T, n_rows, WgT, WuT, Wd, d, f, ho, true, rows, y, T, dev_status, s, sms);
 }
@@ -451,7 +478,7 @@ twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
     TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
   const long long want = (static_cast<long long>(p.rows) + kWarps - 1) / kWarps;
   const int blocks = static_cast<int>(std::max(1LL, std::min<long long>(want, sms)));
-  kern<<<blocks, kWarps * 32, smem, s>>>(p);
+  TW_TRY(launch(kern, dim3(blocks), dim3(kWarps * 32), smem, s, p));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -509,9 +536,9 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   // 2. overflow rows, dense on the tensor cores: gather x and dy (zero the dx
   // rows and the padding rows up to a multiple of 64), recompute [z | u], then
   // dh = dy Wd^T with dz, du, h in its epilogue, then dx = [dz | du] [Wg; Wu]^T
-  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(x, d, ovf_rows, n_ovf, T, w.xo, dx, dev_status, w.t_pad);
+  TW_TRY(launch(gather_rows_kernel, dim3(sms * 2), dim3(256), 0, s, x, d, ovf_rows, n_ovf, T, w.xo, dx, dev_status, w.t_pad));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  gather_rows_kernel<<<sms * 2, 256, 0, s>>>(dy, d, ovf_rows, n_ovf, T, w.dyo, nullptr, dev_status, w.t_pad);
+  TW_TRY(launch(gather_rows_kernel, dim3(sms * 2), dim3(256), 0, s, dy, d, ovf_rows, n_ovf, T, w.dyo, nullptr, dev_status, w.t_pad));
   TW_TRY(cuda_ok(cudaGetLastError()));
   CUtensorMap mx, mdy, mg, mu, mwd, ma2, mgT, muT;
   if (!make_map(&mx, w.xo, d, T, kBK, kBM) || !make_map(&mdy, w.dyo, d, T, kBK, kBM) ||
@@ -565,11 +592,11 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
   // 3. weight gradients of the rows that fit: sort their slots by column, then
   // sum per column (every row of dW is written)
   SlotSource a{tw->counts, tw->idx, tw->row_ovf, T, nullptr, nT, tw->W, f, 1, 0u};
-  TW_TRY(cuda_ok(cudaMemsetAsync(w.colcnt, 0, static_cast<size_t>(f) * 4, s)));
+  TW_TRY(zero_async(s, sms, w.colcnt, static_cast<size_t>(f) * 4));
   const int cblocks = 4 * sms;
-  bwd_columns_kernel<false><<<cblocks, 256, 0, s>>>(a, w.colcnt, w.colptr, w.list);
-  bwd_column_scan_kernel<<<1, 1024, 0, s>>>(w.colcnt, f, w.colptr);
-  bwd_columns_kernel<true><<<cblocks, 256, 0, s>>>(a, w.colcnt, w.colptr, w.list);
+  TW_TRY(launch(bwd_columns_kernel<false>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
+  TW_TRY(launch(bwd_column_scan_kernel, dim3(1), dim3(1024), 0, s, w.colcnt, f, w.colptr));
+  TW_TRY(launch(bwd_columns_kernel<true>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
   TW_TRY(cuda_ok(cudaGetLastError()));
   WgradParams g{};
   g.list = w.list;
@@ -586,7 +613,7 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
   g.dWuT = dWuT;
   g.dWd = dWd;
   const long long warps = static_cast<long long>(f) * ((d + 255) / 256);
-  bwd_wgrad_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(g);
+  TW_TRY(launch(bwd_wgrad_kernel, dim3(static_cast<unsigned>((warps + 7) / 8)), dim3(256), 0, s, g));
   TW_TRY(cuda_ok(cudaGetLastError()));
   // 4. the overflow rows' share, on the tensor cores: dWgT += dz^T x,
   // dWuT += du^T x, dWd += h^T dy over the gathered rows (K = their tokens, as
@@ -698,7 +725,7 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
   uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
                                              round_up(static_cast<size_t>(T) * d * 2, 256));
   TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms));
-  route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
@@ -710,7 +737,7 @@ twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, v
   TW_TRY(check_ptrs({ovf_rows, n_ovf}));
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  route_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(tw->row_ovf, tw->T, ovf_rows, n_ovf);
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream), tw->row_ovf, tw->T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -740,13 +767,13 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
     const bool zero_y = sparse_splits_units(T, d, false, sms);
     TW_TRY(small_gate_pack_impl(x, WgT, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
                                 dev_status, s, sms));
-    route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y);
+    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y));
     TW_TRY(cuda_ok(cudaGetLastError()));
     TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms, false, zero_y));
     return dense_impl(xo, T, n_ovf, WgT, WuT, Wd, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
   TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
-  route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
@@ -793,12 +820,11 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
   if (small_batch(T, f, 128, sms)) {
     // z and u with K split over the whole grid, then h = bf16(ReLU(z) * u)
     float* zu = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(T) * f * 2, 256));
-    TW_TRY(cuda_ok(cudaMemsetAsync(zu, 0, static_cast<size_t>(T) * f * 8, s)));
+    TW_TRY(zero_async(s, sms, zu, static_cast<size_t>(T) * f * 8));
     TW_TRY(f32_gemm_impl(x, T, WgT, f, d, zu, 2 * f, dev_status, s, sms));
     TW_TRY(f32_gemm_impl(x, T, WuT, f, d, zu + f, 2 * f, dev_status, s, sms));
     const size_t n4 = static_cast<size_t>(T) * f / 4;
-    h_from_zu_kernel<<<static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 4 * static_cast<size_t>(sms))), 256, 0,
-                       s>>>(zu, T, f, 1, h);
+    TW_TRY(launch(h_from_zu_kernel, dim3(static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 4 * static_cast<size_t>(sms)))), dim3(256), 0, s, zu, T, f, 1, h));
     TW_TRY(cuda_ok(cudaGetLastError()));
     return dense_down_impl(h, T, nullptr, Wd, d, f, false, nullptr, y, T, dev_status, s, sms);
   }
@@ -827,13 +853,13 @@ twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1
     const bool zero_y = sparse_splits_units(T, d, true, sms);
     TW_TRY(small_gate_pack_impl(x, W1T, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
                                 dev_status, s, sms));
-    route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y);
+    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y));
     TW_TRY(cuda_ok(cudaGetLastError()));
     TW_TRY(sparse_impl(nullptr, nullptr, W2, T, d, f, tw, 1, y, dev_status, s, sms, true, zero_y));
     return dense_impl(xo, T, n_ovf, W1T, nullptr, W2, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
   TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms));
-  route_kernel<<<1, 1024, 0, s>>>(tw->row_ovf, T, ovf_rows, n_ovf);
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(down_impl(W2, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, W1T, nullptr, W2, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
@@ -871,11 +897,10 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
   uint16_t* h = static_cast<uint16_t*>(workspace);
   if (small_batch(T, f, kBN, sms)) {
     float* z = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(T) * f * 2, 256));
-    TW_TRY(cuda_ok(cudaMemsetAsync(z, 0, static_cast<size_t>(T) * f * 4, s)));
+    TW_TRY(zero_async(s, sms, z, static_cast<size_t>(T) * f * 4));
     TW_TRY(f32_gemm_impl(x, T, W1T, f, d, z, f, dev_status, s, sms));
     const size_t n4 = static_cast<size_t>(T) * f / 4;
-    h_from_zu_kernel<<<static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 4 * static_cast<size_t>(sms))), 256, 0,
-                       s>>>(z, T, f, 0, h);
+    TW_TRY(launch(h_from_zu_kernel, dim3(static_cast<unsigned>(std::min<size_t>((n4 + 255) / 256, 4 * static_cast<size_t>(sms)))), dim3(256), 0, s, z, T, f, 0, h));
     TW_TRY(cuda_ok(cudaGetLastError()));
     return dense_down_impl(h, T, nullptr, W2, d, f, false, nullptr, y, T, dev_status, s, sms);
   }
@@ -1029,7 +1054,7 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
   q3.k_splits_max = 1;
   q3.dev_status = dev_status;
   if (static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms) {
-    TW_TRY(cuda_ok(cudaMemsetAsync(dx, 0, static_cast<size_t>(T) * d * sizeof(float), s)));
+    TW_TRY(zero_async(s, sms, dx, static_cast<size_t>(T) * d * sizeof(float)));
     q3.k_splits_max = 32;
   }
   TW_TRY(launch_gemm<kModeDown>(ma2, mgT, muT, q3, q3.k_splits_max > 1 ? sms : gemm_grid(T, d, kBN, sms), s));
@@ -1051,7 +1076,7 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
     q.ldo = d;
     q.k_splits_max = split ? 32 : 1;
     q.dev_status = dev_status;
-    if (split) TW_TRY(cuda_ok(cudaMemsetAsync(outs[i], 0, static_cast<size_t>(f) * d * sizeof(float), s)));
+    if (split) TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
     TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, split ? sms : gemm_grid(f, d, kBN, sms), s));
   }
   return TWELL_OK;
@@ -1064,7 +1089,7 @@ twell_status twell_column_activity(const uint16_t* x, const uint16_t* WgT, int T
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (!accumulate) TW_TRY(cuda_ok(cudaMemsetAsync(active_bits, 0, static_cast<size_t>(f / 32) * 4, s)));
+  if (!accumulate) TW_TRY(zero_async(s, sms, active_bits, static_cast<size_t>(f / 32) * 4));
   if (T == 0) return TWELL_OK;
   TW_TRY(check_ptrs({x, WgT}));
   CUtensorMap ma, mb;
@@ -1084,7 +1109,7 @@ twell_status twell_compact_columns(const uint32_t* active_bits, int f, int32_t* 
   TW_TRY(check_ptrs({active_bits, col_map, f_live}));
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  compact_columns_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(active_bits, f, col_map, f_live);
+  TW_TRY(launch(compact_columns_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream), active_bits, f, col_map, f_live));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -1096,8 +1121,8 @@ twell_status twell_gather_rows(const uint16_t* W, int f, int d, const int32_t* c
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
   const int blocks = std::min((f_out + 7) / 8, 4 * sms);
-  gather_weight_rows_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(W, f, d, col_map, f_live, f_out,
-                                                                                  W_out, dev_status);
+  TW_TRY(launch(gather_weight_rows_kernel, dim3(blocks), dim3(256), 0, static_cast<cudaStream_t>(stream), W, f, d, col_map, f_live, f_out,
+                                                                                  W_out, dev_status));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -1113,8 +1138,8 @@ twell_status twell_unpack(const twell_t* tw, uint16_t* g_dense, int32_t* dev_sta
   const long long warps = static_cast<long long>(tw->T) * nT;
   const long long blocks = (warps + 7) / 8;
   if (blocks > 0x7fffffffLL) return TWELL_ERR_SHAPE;
-  unpack_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      tw->counts, tw->idx, tw->vals, tw->T, nT, tw->W, tw->f, g_dense, dev_status);
+  TW_TRY(launch(unpack_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, static_cast<cudaStream_t>(stream), 
+      tw->counts, tw->idx, tw->vals, tw->T, nT, tw->W, tw->f, g_dense, dev_status));
   return cuda_ok(cudaGetLastError());
 }
 

@@ -217,33 +217,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  int M = p.M;
-  if (p.M_dev != nullptr) M = min(max(*p.M_dev, 0), p.M);
   constexpr bool kStacked = (MODE == kModeGateUp || MODE == kModeTwellHidden || MODE == kModeZU);  // B = [Wg; Wu]
   constexpr int kTileN = kStacked ? 128 : kBN;  // output columns per tile
-  const int num_m = (M + kBM - 1) / kBM;
-  const int num_n = (p.N + kTileN - 1) / kTileN;
-  int num_kb = p.K / kBK;
-  // compact K (kModeDown with k_dev): blocks [0, nkb_half) of each half
-  int nkb_half = 0;
-  if (MODE == kModeDown && p.k_dev != nullptr) {
-    nkb_half = (min(max(*p.k_dev, 0), p.k_half) + kBK - 1) / kBK;
-    num_kb = 2 * nkb_half;
-  }
-  // K splits (kModeDown / kModeF32): as many as keep every CTA busy, none empty.
-  int kb_per = num_kb, k_splits = 1;
-  if ((MODE == kModeDown || MODE == kModeF32) && p.k_splits_max > 1 && num_m * num_n > 0 && num_kb > 0) {
-    int want = min(p.k_splits_max, max(1, static_cast<int>(gridDim.x) / (num_m * num_n)));
-    want = min(want, num_kb);
-    kb_per = (num_kb + want - 1) / want;
-    k_splits = (num_kb + kb_per - 1) / kb_per;
-  }
-  // no K block at all (an empty compact K): nothing to compute or store
-  const int num_tiles = num_kb > 0 ? num_m * num_n * k_splits : 0;
-  // A CTA without a tile leaves before any setup (uniform for the whole CTA).
-  if (static_cast<int>(blockIdx.x) >= num_tiles) return;
 
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -266,6 +243,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Everything above is private to this CTA; what follows reads the previous
+  // kernels' outputs (device-side row counts included).
+  griddep_wait();
+  int M = p.M;
+  if (p.M_dev != nullptr) M = min(max(*p.M_dev, 0), p.M);
+  const int num_m = (M + kBM - 1) / kBM;
+  const int num_n = (p.N + kTileN - 1) / kTileN;
+  int num_kb = p.K / kBK;
+  // compact K (kModeDown with k_dev): blocks [0, nkb_half) of each half
+  int nkb_half = 0;
+  if (MODE == kModeDown && p.k_dev != nullptr) {
+    nkb_half = (min(max(*p.k_dev, 0), p.k_half) + kBK - 1) / kBK;
+    num_kb = 2 * nkb_half;
+  }
+  // K splits (kModeDown / kModeF32): as many as keep every CTA busy, none empty.
+  int kb_per = num_kb, k_splits = 1;
+  if ((MODE == kModeDown || MODE == kModeF32) && p.k_splits_max > 1 && num_m * num_n > 0 && num_kb > 0) {
+    int want = min(p.k_splits_max, max(1, static_cast<int>(gridDim.x) / (num_m * num_n)));
+    want = min(want, num_kb);
+    kb_per = (num_kb + want - 1) / want;
+    k_splits = (num_kb + kb_per - 1) / kb_per;
+  }
+  // no K block at all (an empty compact K): nothing to compute or store
+  const int num_tiles = num_kb > 0 ? num_m * num_n * k_splits : 0;
+
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
