@@ -11,10 +11,11 @@
 // Rows that fit the ELL width take two passes over their stored units:
 //   1. per token (one warp per token, like the forward's fused kernel): u_j and
 //      dh_j by two dot products per stored unit, then dx_t by two row axpys;
-//      the per-unit scalars (h, du, dz) are written beside the slots;
-//   2. per hidden unit: the slots are sorted by column (count, scan, scatter)
-//      and one warp per (unit, 256-wide slice of d) sums h dy_t, du x_t, dz x_t
-//      over the unit's tokens into the three weight-gradient rows.
+//      each slot's record {h, du, dz, token} is written beside the slots;
+//   2. per hidden unit: the records are sorted by column (count, scan, scatter
+//      of whole 16-byte records) and one warp per (unit, 256-wide slice of d)
+//      reads its unit's records in order and sums h dy_t, du x_t, dz x_t into
+//      the three weight-gradient rows.
 // Rows that overflow take the dense branch on the tensor cores (the GEMM
 // modes kModeZU, kModeBwdDh and kModeDown), which adds their share to the
 // weight gradients afterwards.
@@ -36,10 +37,8 @@ struct BwdParams {
   const uint8_t* row_ovf;  // rows with the flag set are skipped
   int rows;
   int d, f, nT, W;
-  float* dx;   // [rows][d] fp32
-  float* s_h;  // per stored slot [rows][nT][W]: h, du, dz (fp32)
-  float* s_du;
-  float* s_dz;
+  float* dx;      // [rows][d] fp32
+  float4* s_rec;  // per stored slot [rows][nT][W]: {h, du, dz, token (int bits)}
   int* dev_status;
 };
 
@@ -256,12 +255,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
         const float my_g = entry_g(my_e);
         const float my_du = valid ? my_dh * my_g : 0.0f;
         const float my_dz = valid ? my_dh * my_u : 0.0f;
-        if (valid) {
-          const size_t slot = slot_row + my_pos;
-          p.s_h[slot] = my_g * my_u;
-          p.s_du[slot] = my_du;
-          p.s_dz[slot] = my_dz;
-        }
+        if (valid) p.s_rec[slot_row + my_pos] = make_float4(my_g * my_u, my_du, my_dz, __int_as_float(t));
         // dx_t += dz_j Wg[:, j] + du_j Wu[:, j]
         if (kAccSmem) {
 #pragma unroll
@@ -309,12 +303,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
 struct SlotSource {
   const int16_t* counts;
   const int16_t* idx;
+  const float4* rec;  // the slots' records (read by the scatter)
   const uint8_t* row_ovf;  // rows with the flag set are skipped when skip_ovf
   int rows;
   const int* rows_dev;
   int nT, W, f;
   int skip_ovf;
-  uint32_t tag;  // bit 31 of each list entry: which pass the slot belongs to
 };
 
 __device__ __forceinline__ int source_rows(const SlotSource& s) {
@@ -322,10 +316,10 @@ __device__ __forceinline__ int source_rows(const SlotSource& s) {
 }
 
 // SCATTER == false: colcnt[j] += number of slots with column j.
-// SCATTER == true: each slot is written to list[colptr[j] + cursor[j]++] as
-// tag | slot index (the order inside a column is that of the atomics).
+// SCATTER == true: each slot's record is copied to list[colptr[j] +
+// cursor[j]++] (the order inside a column is that of the atomics).
 template <bool SCATTER>
-__global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colptr, uint32_t* list) {
+__global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colptr, float4* list) {
   griddep_launch_dependents();
   griddep_wait();
   const int lane = threadIdx.x & 31;
@@ -343,7 +337,7 @@ __global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colpt
       if (j < 0 || j >= src.f) continue;
       if (SCATTER) {
         const int pos = colptr[j] + atomicAdd(colcnt + j, 1);
-        list[pos] = src.tag | static_cast<uint32_t>(slot);
+        list[pos] = src.rec[slot];
       } else {
         atomicAdd(colcnt + j, 1);
       }
@@ -396,14 +390,10 @@ __global__ void __launch_bounds__(1024) bwd_column_scan_kernel(int* colcnt, int 
 }
 
 struct WgradParams {
-  const uint32_t* list;  // slot indices sorted by column
+  const float4* list;  // slot records {h, du, dz, token} sorted by column
   const int* colptr;
   const uint16_t* x0;
   const uint16_t* dy0;
-  const float* h0;  // per-slot scalars of the rows that fit
-  const float* du0;
-  const float* dz0;
-  int slots_per_row0;  // nT * W
   int f, d;
   float* dWgT;  // [f][d] fp32, fully written
   float* dWuT;
@@ -434,13 +424,13 @@ __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
     const uint16_t* dr = nullptr;
     float vh = 0.f, vu = 0.f, vz = 0.f;
     if (lane < nb) {
-      const size_t slot = p.list[b + lane] & 0x7fffffffu;
-      const size_t row = slot / static_cast<size_t>(p.slots_per_row0);
+      const float4 rec = p.list[b + lane];
+      const size_t row = static_cast<size_t>(__float_as_int(rec.w));
       xr = p.x0 + row * p.d;
       dr = p.dy0 + row * p.d;
-      vh = p.h0[slot];
-      vu = p.du0[slot];
-      vz = p.dz0[slot];
+      vh = rec.x;
+      vu = rec.y;
+      vz = rec.z;
     }
 #pragma unroll 1
     for (int s = 0; s < nb; ++s) {

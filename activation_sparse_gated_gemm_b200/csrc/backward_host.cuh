@@ -1,0 +1,218 @@
+// Host side of the backward pass through the hybrid format: the workspace
+// layout and the launch sequences of its two halves (dx, then the weight
+// gradients). Included by twell_api.cu inside its internal namespace, after
+// the forward's helpers it reuses (launch, zero_async, make_map, gather).
+#pragma once
+
+// Workspace of the hybrid backward, carved in this order (each piece 256-byte
+// aligned): per-slot records {h, du, dz, token} of the rows that fit
+// ([T][nT][W] float4); for the overflow rows, the gathered rows of x and dy
+// ([Tp][d] bf16 each, Tp = T rounded up to 64), their [z | u] ([T][2f] fp32),
+// [dz | du | dz_lo | du_lo] ([T][4f] bf16) and the three transposed blocks dz,
+// du, h ([f][2 Tp] bf16 each); the column counts/cursors ([f]), column
+// offsets ([f + 1]) and the column-sorted records (one float4 per slot of the
+// rows that fit).
+struct BwdWorkspace {
+  float4* rec;
+  uint16_t *xo, *dyo;
+  float* zu;
+  uint16_t *a2, *tT;
+  int *colcnt, *colptr;
+  float4* list;
+  int t_pad;
+  size_t bytes;
+};
+
+BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
+  const size_t nT = static_cast<size_t>(f) / 128;
+  const size_t s0 = static_cast<size_t>(T) * nT * W;
+  const size_t tp = round_up(static_cast<size_t>(T), 64);
+  BwdWorkspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += round_up(bytes, 256);
+    return p;
+  };
+  w.rec = reinterpret_cast<float4*>(take(s0 * 16));
+  w.xo = reinterpret_cast<uint16_t*>(take(tp * d * 2));
+  w.dyo = reinterpret_cast<uint16_t*>(take(tp * d * 2));
+  w.zu = reinterpret_cast<float*>(take(static_cast<size_t>(T) * f * 8));
+  w.a2 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * f * 8));
+  w.tT = reinterpret_cast<uint16_t*>(take(3 * static_cast<size_t>(f) * 2 * tp * 2));
+  w.colcnt = reinterpret_cast<int*>(take(static_cast<size_t>(f) * 4));
+  w.colptr = reinterpret_cast<int*>(take((static_cast<size_t>(f) + 1) * 4));
+  w.list = reinterpret_cast<float4*>(take(s0 * 16));
+  w.t_pad = static_cast<int>(tp);
+  w.bytes = off;
+  return w;
+}
+
+template <int NCH>
+twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
+  constexpr int kWarps = bwd_warps_for(NCH);
+  const size_t smem = bwd_smem_bytes(NCH);
+  auto kern = bwd_token_kernel<NCH, kWarps>;
+  if (smem > 48 * 1024)
+    TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
+  const long long want = (static_cast<long long>(p.rows) + kWarps - 1) / kWarps;
+  const int blocks = static_cast<int>(std::max(1LL, std::min<long long>(want, sms)));
+  TW_TRY(launch(kern, dim3(blocks), dim3(kWarps * 32), smem, s, p));
+  return cuda_ok(cudaGetLastError());
+}
+
+twell_status launch_bwd_token(const BwdParams& p, int sms, cudaStream_t s) {
+  switch ((p.d + 255) / 256) {
+    case 1: return launch_bwd_token_n<1>(p, sms, s);
+    case 2: return launch_bwd_token_n<2>(p, sms, s);
+    case 3: return launch_bwd_token_n<3>(p, sms, s);
+    case 4: return launch_bwd_token_n<4>(p, sms, s);
+    case 5: return launch_bwd_token_n<5>(p, sms, s);
+    case 6: return launch_bwd_token_n<6>(p, sms, s);
+    case 7: return launch_bwd_token_n<7>(p, sms, s);
+    case 8: return launch_bwd_token_n<8>(p, sms, s);
+    case 9: return launch_bwd_token_n<9>(p, sms, s);
+    case 10: return launch_bwd_token_n<10>(p, sms, s);
+    case 11: return launch_bwd_token_n<11>(p, sms, s);
+    case 12: return launch_bwd_token_n<12>(p, sms, s);
+    case 13: return launch_bwd_token_n<13>(p, sms, s);
+    case 14: return launch_bwd_token_n<14>(p, sms, s);
+    case 15: return launch_bwd_token_n<15>(p, sms, s);
+    case 16: return launch_bwd_token_n<16>(p, sms, s);
+    default: return TWELL_ERR_SHAPE;
+  }
+}
+
+// dx, and the per-slot scalars of both passes in the workspace.
+twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
+                              const uint16_t* dy, int T, int d, int f, const twell_t* tw, const int32_t* ovf_rows,
+                              const int32_t* n_ovf, float* dx, char* ws, int32_t* dev_status, cudaStream_t s,
+                              int sms) {
+  const int nT = f / 128;
+  BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
+  // 1. rows that fit: per-token pass over their stored slots
+  BwdParams p0{};
+  p0.x = x;
+  p0.dy = dy;
+  p0.WgT = WgT;
+  p0.WuT = WuT;
+  p0.Wd = Wd;
+  p0.counts = tw->counts;
+  p0.idx = tw->idx;
+  p0.vals = tw->vals;
+  p0.row_ovf = tw->row_ovf;
+  p0.rows = T;
+  p0.d = d;
+  p0.f = f;
+  p0.nT = nT;
+  p0.W = tw->W;
+  p0.dx = dx;
+  p0.s_rec = w.rec;
+  p0.dev_status = dev_status;
+  TW_TRY(launch_bwd_token(p0, sms, s));
+  // 2. overflow rows, dense on the tensor cores: gather x and dy (zero the dx
+  // rows and the padding rows up to a multiple of 64), recompute [z | u], then
+  // dh = dy Wd^T with dz, du, h in its epilogue, then dx = [dz | du] [Wg; Wu]^T
+  TW_TRY(launch(gather_rows_kernel, dim3(sms * 2), dim3(256), 0, s, x, d, ovf_rows, n_ovf, T, w.xo, dx, dev_status, w.t_pad));
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  TW_TRY(launch(gather_rows_kernel, dim3(sms * 2), dim3(256), 0, s, dy, d, ovf_rows, n_ovf, T, w.dyo, nullptr, dev_status, w.t_pad));
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  CUtensorMap mx, mdy, mg, mu, mwd, ma2, mgT, muT;
+  if (!make_map(&mx, w.xo, d, T, kBK, kBM) || !make_map(&mdy, w.dyo, d, T, kBK, kBM) ||
+      !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128) ||
+      !make_map(&mwd, Wd, d, f, kBK, kBN) || !make_map(&ma2, w.a2, 4 * f, T, kBK, kBM) ||
+      !make_map(&mgT, WgT, d, f, 64, kBK) || !make_map(&muT, WuT, d, f, 64, kBK))
+    return TWELL_ERR_CUDA;
+  GemmParams q1{};
+  q1.M = T;
+  q1.M_dev = n_ovf;
+  q1.N = f;
+  q1.K = d;
+  q1.out_f32 = w.zu;
+  q1.ldo = 2 * f;
+  q1.dev_status = dev_status;
+  TW_TRY(launch_gemm<kModeZU>(mx, mg, mu, q1, sms, s));
+  GemmParams q2{};
+  q2.M = T;
+  q2.M_dev = n_ovf;
+  q2.N = f;
+  q2.K = d;
+  q2.zu = w.zu;
+  q2.a2 = w.a2;
+  q2.tT = w.tT;
+  q2.t_pad = w.t_pad;
+  q2.h_split = 1;
+  q2.dev_status = dev_status;
+  TW_TRY(launch_gemm<kModeBwdDh>(mdy, mwd, mwd, q2, sms, s));
+  GemmParams q3{};
+  q3.M = T;
+  q3.M_dev = n_ovf;
+  q3.N = d;
+  q3.K = 4 * f;
+  q3.k_wrap = 2 * f;
+  q3.k_split_b = f;
+  q3.out_f32 = dx;
+  q3.ldo = d;
+  q3.row_map = ovf_rows;
+  q3.out_rows = T;
+  q3.k_splits_max = 32;  // the gather zeroed these dx rows
+  q3.dev_status = dev_status;
+  return launch_gemm<kModeDown>(ma2, mgT, muT, q3, sms, s);
+}
+
+// Weight gradients from the workspace filled by backward_dx_impl.
+twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int d, int f, const twell_t* tw,
+                              const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd, char* ws, cudaStream_t s,
+                              int sms) {
+  const int nT = f / 128;
+  BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
+  // 3. weight gradients of the rows that fit: sort their slots by column, then
+  // sum per column (every row of dW is written)
+  SlotSource a{tw->counts, tw->idx, w.rec, tw->row_ovf, T, nullptr, nT, tw->W, f, 1};
+  TW_TRY(zero_async(s, sms, w.colcnt, static_cast<size_t>(f) * 4));
+  const int cblocks = 4 * sms;
+  TW_TRY(launch(bwd_columns_kernel<false>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
+  TW_TRY(launch(bwd_column_scan_kernel, dim3(1), dim3(1024), 0, s, w.colcnt, f, w.colptr));
+  TW_TRY(launch(bwd_columns_kernel<true>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  WgradParams g{};
+  g.list = w.list;
+  g.colptr = w.colptr;
+  g.x0 = x;
+  g.dy0 = dy;
+  g.f = f;
+  g.d = d;
+  g.dWgT = dWgT;
+  g.dWuT = dWuT;
+  g.dWd = dWd;
+  const long long warps = static_cast<long long>(f) * ((d + 255) / 256);
+  TW_TRY(launch(bwd_wgrad_kernel, dim3(static_cast<unsigned>((warps + 7) / 8)), dim3(256), 0, s, g));
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  // 4. the overflow rows' share, on the tensor cores: dWgT += dz^T x,
+  // dWuT += du^T x, dWd += h^T dy over the gathered rows (K = their tokens, as
+  // bf16 value and remainder halves)
+  const size_t tblock = static_cast<size_t>(f) * 2 * w.t_pad;
+  const uint16_t* aT[3] = {w.tT, w.tT + tblock, w.tT + 2 * tblock};
+  const uint16_t* bT[3] = {w.xo, w.xo, w.dyo};
+  float* outs[3] = {dWgT, dWuT, dWd};
+  for (int i = 0; i < 3; ++i) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, aT[i], 2 * w.t_pad, f, kBK, kBM) || !make_map(&mb, bT[i], d, w.t_pad, 64, kBK))
+      return TWELL_ERR_CUDA;
+    GemmParams q{};
+    q.M = f;
+    q.N = d;
+    q.K = 2 * w.t_pad;
+    q.k_wrap = w.t_pad;
+    q.k_dev = n_ovf;
+    q.k_half = w.t_pad;
+    q.accumulate = 1;
+    q.k_splits_max = 32;
+    q.out_f32 = outs[i];
+    q.ldo = d;
+    q.dev_status = nullptr;
+    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, sms, s));
+  }
+  return TWELL_OK;
+}
+
