@@ -8,10 +8,13 @@
 //   dx   = sum_j dz_j Wg[:, j] + du_j Wu[:, j]
 //   dWd[j, :] = sum_t h_tj dy_t, dWu[:, j] = sum_t du_tj x_t, dWg[:, j] = sum_t dz_tj x_t
 //
-// Rows that fit the ELL width take two passes over their stored units:
+// Rows that fit the ELL width take three passes over their stored units:
 //   1. per token (one warp per token, like the forward's fused kernel): u_j and
-//      dh_j by two dot products per stored unit, then dx_t by two row axpys;
-//      each slot's record {h, du, dz, token} is written beside the slots;
+//      dh_j by two dot products per stored unit; each slot's record
+//      {h, du, dz, token} is written beside the slots;
+//   1b. per token again: dx_t by two row axpys with du_j, dz_j from the records
+//      (split from pass 1 so that neither pass holds both dx_t and the dot
+//      passes' rows, which lets each run twice the warps);
 //   2. per hidden unit: the records are sorted by column (count, scan, scatter
 //      of whole 16-byte records) and one warp per (unit, 256-wide slice of d)
 //      reads its unit's records in order and sums h dy_t, du x_t, dz x_t into
@@ -42,18 +45,19 @@ struct BwdParams {
   int* dev_status;
 };
 
-// Warps per block of the per-token pass: x_t, dy_t (shared memory), dx_t and
-// two weight rows (registers) per warp.
-constexpr int bwd_warps_for(int nch) { return nch <= 3 ? 12 : (nch <= 10 ? 8 : 5); }
-// From this many 256-element chunks of d on, dx_t waits in shared memory while
-// the dot passes run (registers hold either dx_t or the dot passes' rows).
-constexpr int kBwdAccSmemNch = 7;
-
-// Bytes of dynamic shared memory per block of the per-token pass.
-constexpr size_t bwd_smem_bytes(int nch) {
-  return static_cast<size_t>(bwd_warps_for(nch)) *
-         (2 * nch * 32 * 16 + kListCap * 6 + (nch >= kBwdAccSmemNch ? nch * 32 * 32 : 0));
+// Warps per block of the two per-token passes. The dot pass holds x_t and
+// dy_t in shared memory and two weight rows in registers; the dx pass holds
+// dx_t and two weight rows in registers.
+constexpr int bwd_dots_warps(int nch) {
+  // registers (two rows of d per lane and the reductions) cap it before shared memory does
+  return nch <= 6 ? 16 : (nch <= 8 ? 12 : 8);
 }
+constexpr int bwd_dx_warps(int nch) { return nch <= 4 ? 16 : (nch <= 7 ? 12 : 8); }
+
+constexpr size_t bwd_dots_smem_bytes(int nch) {
+  return static_cast<size_t>(bwd_dots_warps(nch)) * (2 * nch * 32 * 16 + kListCap * 6);
+}
+constexpr size_t bwd_dx_smem_bytes(int nch) { return static_cast<size_t>(bwd_dx_warps(nch)) * kListCap * 6; }
 
 // 16-byte shared-memory load that the compiler keeps inside its loop (x_t and
 // dy_t are reread per entry instead of being held in registers across it).
@@ -130,14 +134,71 @@ __device__ __forceinline__ void bwd_axpy_pass(float (&acc)[NCH][8], const uint16
   }
 }
 
-// One warp per token that fits. Shared memory per warp: x_t and dy_t
-// (NCH * 32 uint4 each), the flattened slot list (column | bf16 g << 16) and
-// the slot position of every list entry inside the row's [nT][W] block.
+// Flattens the stored slots of row t, tiles [c0, c1), into list (column |
+// bf16 g << 16) and lpos (the slot's position in the row's [nT][W] block, bit
+// 15 set for an out-of-range column, which is then read as column 0 and must
+// contribute nothing). Returns the number of entries; 8 slots per 16-byte load.
+__device__ __forceinline__ int bwd_build_list(const BwdParams& p, int t, int c0, int c1, uint32_t* list,
+                                              uint16_t* lpos, int lane, bool& bad_index) {
+  int total = 0;
+#pragma unroll 1
+  for (int cb = c0; cb < c1; cb += 32) {
+    const int c = cb + lane;
+    int n = 0;
+    if (c < c1) n = min(max(static_cast<int>(p.counts[static_cast<size_t>(t) * p.nT + c]), 0), p.W);
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int off = total + incl - n;
+    total += __shfl_sync(0xffffffffu, incl, 31);
+    const size_t base = (static_cast<size_t>(t) * p.nT + c) * p.W;
+    for (int k = 0; k < n; k += 8) {
+      // slots past n are read but not used (k + 8 <= W)
+      const uint4 iv = ldg_nc_v4(p.idx + base + k);
+      const uint4 vv = ldg_nc_v4(p.vals + base + k);
+      const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
+      const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (k + e < n) {
+          const uint32_t jj = (e & 1) ? (iw[e >> 1] >> 16) : (iw[e >> 1] & 0xffffu);
+          const uint32_t gg = (e & 1) ? (vw[e >> 1] & 0xffff0000u) : (vw[e >> 1] << 16);
+          uint32_t ent = jj | gg;
+          uint16_t pos = static_cast<uint16_t>(c * p.W + k + e);  // < 2^15: nT * W <= 255 * 128
+          if (static_cast<int>(static_cast<int16_t>(jj)) < 0 || static_cast<int>(jj) >= p.f) {
+            bad_index = true;
+            ent = 0;
+            pos |= 0x8000u;
+          }
+          list[off + k + e] = ent;
+          lpos[off + k + e] = pos;
+        }
+      }
+    }
+  }
+  return total;
+}
+
+// Tokens are handed out one at a time from a per-block counter over the
+// block's contiguous share of the rows.
+__device__ __forceinline__ int bwd_next_row(int* next_row, int lane) {
+  int t = 0;
+  if (lane == 0) t = atomicAdd(next_row, 1);
+  return __shfl_sync(0xffffffffu, t, 0);
+}
+
+// Pass 1, one warp per token that fits: u_j = x_t . Wu[:, j] and
+// dh_j = dy_t . Wd[j, :] for every stored slot (x_t and dy_t parked in shared
+// memory), and the slot's record {h = g u, du = dh g, dz = dh u, t}.
 template <int NCH, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(WARPS * 32, 1) bwd_dots_kernel(const BwdParams p) {
   griddep_launch_dependents();
   griddep_wait();
   extern __shared__ uint4 bwd_smem[];
+  __shared__ int next_row;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int d = p.d;
@@ -147,27 +208,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
   uint16_t* lpos = reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) +
                                                WARPS * kListCap) +
                    warp * kListCap;
-  constexpr bool kAccSmem = NCH >= kBwdAccSmemNch;
-  // dx_t parked between batches: [NCH][32 lanes] float4 pairs, after the lists
-  float4* acc_s = reinterpret_cast<float4*>(reinterpret_cast<uint16_t*>(
-                      reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) + WARPS * kListCap) +
-                                            WARPS * kListCap) +
-                  warp * NCH * 32 * 2;
   const int group_tiles = max(1, kListCap / p.W);
-  const int rows = p.rows;
   bool bad_index = false;
-  // tokens are handed out one at a time from a per-block counter over the
-  // block's contiguous share of the rows
-  __shared__ int next_row;
-  const int r_begin = static_cast<int>(static_cast<long long>(rows) * blockIdx.x / gridDim.x);
-  const int r_end = static_cast<int>(static_cast<long long>(rows) * (blockIdx.x + 1) / gridDim.x);
-  if (threadIdx.x == 0) next_row = r_begin;
+  const int r_end = static_cast<int>(static_cast<long long>(p.rows) * (blockIdx.x + 1) / gridDim.x);
+  if (threadIdx.x == 0) next_row = static_cast<int>(static_cast<long long>(p.rows) * blockIdx.x / gridDim.x);
   __syncthreads();
 #pragma unroll 1
   for (;;) {
-    int t = 0;
-    if (lane == 0) t = atomicAdd(&next_row, 1);
-    t = __shfl_sync(0xffffffffu, t, 0);
+    const int t = bwd_next_row(&next_row, lane);
     if (t >= r_end) break;
     if (p.row_ovf[t]) continue;
     __syncwarp();
@@ -178,119 +226,87 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_token_kernel(const BwdParam
       xs[i * 32 + lane] = in ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
       ds[i * 32 + lane] = in ? ldg_nc_v4(p.dy + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
     }
-    float acc[NCH][8];
-#pragma unroll
-    for (int i = 0; i < NCH; ++i)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
-    if (kAccSmem) {
-#pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        acc_s[(i * 32 + lane) * 2] = make_float4(0.f, 0.f, 0.f, 0.f);
-        acc_s[(i * 32 + lane) * 2 + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
     const size_t slot_row = static_cast<size_t>(t) * p.nT * p.W;
-
 #pragma unroll 1
     for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
-      const int c1 = min(p.nT, c0 + group_tiles);
-      // ---- flatten the stored slots of tiles [c0, c1), 8 slots per 16-byte load
-      int total = 0;
-#pragma unroll 1
-      for (int cb = c0; cb < c1; cb += 32) {
-        const int c = cb + lane;
-        int n = 0;
-        if (c < c1) n = min(max(static_cast<int>(p.counts[static_cast<size_t>(t) * p.nT + c]), 0), p.W);
-        int incl = n;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const int off = total + incl - n;
-        total += __shfl_sync(0xffffffffu, incl, 31);
-        const size_t base = (static_cast<size_t>(t) * p.nT + c) * p.W;
-        for (int k = 0; k < n; k += 8) {
-          // slots past n are read but not used (k + 8 <= W)
-          const uint4 iv = ldg_nc_v4(p.idx + base + k);
-          const uint4 vv = ldg_nc_v4(p.vals + base + k);
-          const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
-          const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (k + e < n) {
-              const uint32_t jj = (e & 1) ? (iw[e >> 1] >> 16) : (iw[e >> 1] & 0xffffu);
-              const uint32_t gg = (e & 1) ? (vw[e >> 1] & 0xffff0000u) : (vw[e >> 1] << 16);
-              uint32_t ent = jj | gg;
-              uint16_t pos = static_cast<uint16_t>(c * p.W + k + e);  // < 2^15: nT * W <= 255 * 128
-              if (static_cast<int>(static_cast<int16_t>(jj)) < 0 || static_cast<int>(jj) >= p.f) {
-                bad_index = true;
-                ent = 0;         // read column 0 ...
-                pos |= 0x8000u;  // ... but contribute nothing and store nothing
-              }
-              list[off + k + e] = ent;
-              lpos[off + k + e] = pos;
-            }
-          }
-        }
-      }
+      const int total = bwd_build_list(p, t, c0, min(p.nT, c0 + group_tiles), list, lpos, lane, bad_index);
       __syncwarp();
-      // ---- consume in batches of 32 entries
 #pragma unroll 1
       for (int s0 = 0; s0 < total; s0 += 32) {
         const int ns = min(32, total - s0);
         const uint32_t my_e = lane < ns ? list[s0 + lane] : 0u;
         const int my_j = entry_j(my_e);
         const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
-        const bool valid = (my_pos & 0x8000u) == 0;
-        // u_j = x . Wu[:, j], dh_j = dy . Wd[j, :]. The empty asm statements
-        // with a memory clobber keep each pass's first gather from being
-        // started inside the previous pass, which would hold a third row of
-        // registers live.
         const float my_u = bwd_dot_pass<NCH>(xs, p.WuT, my_j, ns, lane, d);
-        asm volatile("" ::: "memory");
         const float my_dh = bwd_dot_pass<NCH>(ds, p.Wd, my_j, ns, lane, d);
-        asm volatile("" ::: "memory");
         const float my_g = entry_g(my_e);
-        const float my_du = valid ? my_dh * my_g : 0.0f;
-        const float my_dz = valid ? my_dh * my_u : 0.0f;
-        if (valid) p.s_rec[slot_row + my_pos] = make_float4(my_g * my_u, my_du, my_dz, __int_as_float(t));
-        // dx_t += dz_j Wg[:, j] + du_j Wu[:, j]
-        if (kAccSmem) {
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            const float4 a = acc_s[(i * 32 + lane) * 2], b = acc_s[(i * 32 + lane) * 2 + 1];
-            acc[i][0] = a.x, acc[i][1] = a.y, acc[i][2] = a.z, acc[i][3] = a.w;
-            acc[i][4] = b.x, acc[i][5] = b.y, acc[i][6] = b.z, acc[i][7] = b.w;
-          }
-        }
-        bwd_axpy_pass<NCH>(acc, p.WgT, my_j, my_dz, ns, lane, d);
-        asm volatile("" ::: "memory");
-        bwd_axpy_pass<NCH>(acc, p.WuT, my_j, my_du, ns, lane, d);
-        if (kAccSmem) {
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            acc_s[(i * 32 + lane) * 2] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-            acc_s[(i * 32 + lane) * 2 + 1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-          }
-        }
-        asm volatile("" ::: "memory");
+        if ((my_pos & 0x8000u) == 0)
+          p.s_rec[slot_row + my_pos] = make_float4(my_g * my_u, my_dh * my_g, my_dh * my_u, __int_as_float(t));
       }
       __syncwarp();
+    }
+  }
+  if (__any_sync(0xffffffffu, bad_index) && lane == 0) raise_status(p.dev_status, kDevIndex);
+}
+
+// Pass 2, one warp per token that fits: dx_t = sum over its stored slots of
+// dz_j Wg[:, j] + du_j Wu[:, j], with du_j, dz_j from the slots' records and
+// dx_t in registers (two alternating weight-row buffers, as in the forward).
+template <int NCH, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) bwd_dx_kernel(const BwdParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  extern __shared__ uint4 bwd_smem[];
+  __shared__ int next_row;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int d = p.d;
+  uint32_t* list = reinterpret_cast<uint32_t*>(bwd_smem) + warp * kListCap;
+  uint16_t* lpos = reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem) + WARPS * kListCap) +
+                   warp * kListCap;
+  const int group_tiles = max(1, kListCap / p.W);
+  bool bad_index = false;
+  const int r_end = static_cast<int>(static_cast<long long>(p.rows) * (blockIdx.x + 1) / gridDim.x);
+  if (threadIdx.x == 0) next_row = static_cast<int>(static_cast<long long>(p.rows) * blockIdx.x / gridDim.x);
+  __syncthreads();
+#pragma unroll 1
+  for (;;) {
+    const int t = bwd_next_row(&next_row, lane);
+    if (t >= r_end) break;
+    if (p.row_ovf[t]) continue;
+    float acc[NCH][8];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
+    const size_t slot_row = static_cast<size_t>(t) * p.nT * p.W;
+#pragma unroll 1
+    for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
+      __syncwarp();
+      const int total = bwd_build_list(p, t, c0, min(p.nT, c0 + group_tiles), list, lpos, lane, bad_index);
+      __syncwarp();
+#pragma unroll 1
+      for (int s0 = 0; s0 < total; s0 += 32) {
+        const int ns = min(32, total - s0);
+        const int my_j = lane < ns ? entry_j(list[s0 + lane]) : 0;
+        const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
+        float my_du = 0.0f, my_dz = 0.0f;
+        if ((my_pos & 0x8000u) == 0) {
+          const float4 rec = p.s_rec[slot_row + my_pos];
+          my_du = rec.y;
+          my_dz = rec.z;
+        }
+        bwd_axpy_pass<NCH>(acc, p.WgT, my_j, my_dz, ns, lane, d);
+        bwd_axpy_pass<NCH>(acc, p.WuT, my_j, my_du, ns, lane, d);
+      }
     }
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int k0 = (i * 32 + lane) * 8;
       if (k0 < d) {
         float4* dst = reinterpret_cast<float4*>(p.dx + static_cast<size_t>(t) * d + k0);
-        if (kAccSmem) {
-          dst[0] = acc_s[(i * 32 + lane) * 2];
-          dst[1] = acc_s[(i * 32 + lane) * 2 + 1];
-        } else {
-          dst[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-          dst[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-        }
+        dst[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        dst[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
       }
     }
   }

@@ -48,17 +48,21 @@ BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
   return w;
 }
 
+template <int NCH, int WARPS>
+twell_status launch_bwd_pass(void (*kern)(BwdParams), size_t smem, const BwdParams& p, int sms, cudaStream_t s) {
+  // always opt in: the static shared memory adds to the dynamic size
+  TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
+  const long long want = (static_cast<long long>(p.rows) + WARPS - 1) / WARPS;
+  const int blocks = static_cast<int>(std::max(1LL, std::min<long long>(want, sms)));
+  return launch(kern, dim3(blocks), dim3(WARPS * 32), smem, s, p);
+}
+
+// The per-token passes of the rows that fit: the dot pass (records), then dx.
 template <int NCH>
 twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
-  constexpr int kWarps = bwd_warps_for(NCH);
-  const size_t smem = bwd_smem_bytes(NCH);
-  auto kern = bwd_token_kernel<NCH, kWarps>;
-  if (smem > 48 * 1024)
-    TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
-  const long long want = (static_cast<long long>(p.rows) + kWarps - 1) / kWarps;
-  const int blocks = static_cast<int>(std::max(1LL, std::min<long long>(want, sms)));
-  TW_TRY(launch(kern, dim3(blocks), dim3(kWarps * 32), smem, s, p));
-  return cuda_ok(cudaGetLastError());
+  constexpr int kDots = bwd_dots_warps(NCH), kDx = bwd_dx_warps(NCH);
+  TW_TRY((launch_bwd_pass<NCH, kDots>(bwd_dots_kernel<NCH, kDots>, bwd_dots_smem_bytes(NCH), p, sms, s)));
+  return launch_bwd_pass<NCH, kDx>(bwd_dx_kernel<NCH, kDx>, bwd_dx_smem_bytes(NCH), p, sms, s);
 }
 
 twell_status launch_bwd_token(const BwdParams& p, int sms, cudaStream_t s) {

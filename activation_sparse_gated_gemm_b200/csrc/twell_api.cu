@@ -239,8 +239,8 @@ twell_status launch_sparse_n(SparseParams p, int sms, cudaStream_t s, bool y_zer
   const int blocks = static_cast<int>(std::min<long long>((units + kWarps - 1) / kWarps, sms));
   const size_t smem = static_cast<size_t>(kWarps) * (NCH * 32 * sizeof(uint4) + kListCap * sizeof(uint32_t));
   auto kern = sparse_ffn_warp_kernel<NCH, kWarps, DOWN_ONLY>;
-  if (smem > 48 * 1024)
-    TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
+  // always opt in: the static shared memory adds to the dynamic size
+  TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
   TW_TRY(launch(kern, dim3(blocks), dim3(kWarps * 32), smem, s, p));
   return cuda_ok(cudaGetLastError());
 }
