@@ -462,6 +462,8 @@ def run_gpu(args, world, rank, local):
         "dense_rows": {"bound": "tensor", "work": alg["dense_branch_flops"], "peak": tc, "unit": "TFLOP/s",
                        "scale": 1e12},
     }
+    # weight rows the sparse step gathers: Wu and Wd rows in the gate form, Wd rows otherwise
+    gathered_rows = nnz_stored * (2 if chosen == "gate" else 1)
     dom = max((names[0], names[2], "dense_rows"), key=lambda n: stage_ms[names.index(n)])
     kd = kern[dom]
     ms = float(stage_ms[names.index(dom)])
@@ -494,7 +496,11 @@ def run_gpu(args, world, rank, local):
         "roofline": {"kernel": dom, "bound": kd["bound"], "achieved": achieved, "peak": peak, "unit": kd["unit"],
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": ("fp32 FMA lanes x 2 x max SM clock" if kd["bound"] == "alu"
-                                     else f"{peaks['source']} bf16 burst")},
+                                     else f"{peaks['source']} bf16 burst"),
+                     # the sparse step's real limit: weight rows gathered from L2 (2 bytes x d per
+                     # stored slot and gathered matrix)
+                     "l2_gather_tbs": (gathered_rows * 2.0 * d / (float(stage_ms[names.index(names[2])]) * 1e-3)
+                                       / 1e12)},
         "path_roofline": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6, "t_roof_us": t_roof * 1e6,
                           "frac": t_roof / (step_ms * 1e-3),
                           "frac_gate_only": (alg["gate_flops"] / tc) / (step_ms * 1e-3),
@@ -509,7 +515,8 @@ def run_gpu(args, world, rank, local):
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4,
                 "pipelined": "copy-in, compute and copy-out on three streams, two buffer sets",
                 "l2": "not flushed: each step touches ~0.26 GB, above the 126 MB L2"},
-        "gpu_launches": 6 * K,
+        # per step: zeroing, gate (or gate+up) GEMM, routing, sparse step, row gather, two dense-branch GEMMs
+        "gpu_launches": 7 * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -679,7 +686,9 @@ def run_gpu_backward(args, world, rank, local):
         "speedup_vs_own_dense": dense_ms / step_ms,
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
-        "gpu_launches": 13 * K,
+        # per step: dots and dx passes, two gathers, three dense-branch GEMMs; zeroing, count, scan,
+        # scatter, per-unit sums and three weight-gradient GEMMs
+        "gpu_launches": 15 * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

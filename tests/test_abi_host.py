@@ -111,3 +111,30 @@ def test_compaction_argument_errors(lib):
     assert lib.twell_column_activity(FAKE, FAKE, 64, 128, 512, None, 0, FAKE, None) == tl.TWELL_ERR_NULL
     assert lib.twell_compact_columns(FAKE, 512, None, FAKE, None) == tl.TWELL_ERR_NULL
     assert lib.twell_gather_rows(FAKE, 512, 128, MIS, FAKE, 128, FAKE, FAKE, None) == tl.TWELL_ERR_ALIGN
+
+
+def test_backward_argument_errors(lib):
+    tw = tw_desc()
+    bw = lib.twell_ffn_hybrid_backward
+    args = dict(x=FAKE, g=FAKE, u=FAKE, d=FAKE, dy=FAKE, T=64, dm=128, f=512, ovf=FAKE, n=FAKE, dx=FAKE,
+                a=FAKE, b=FAKE, c=FAKE, ws=FAKE, wsb=1 << 30, st=FAKE)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return bw(a["x"], a["g"], a["u"], a["d"], a["dy"], a["T"], a["dm"], a["f"], ctypes.byref(tw), a["ovf"], a["n"],
+                  a["dx"], a["a"], a["b"], a["c"], a["ws"], a["wsb"], a["st"], None)
+
+    assert call(dm=100) == tl.TWELL_ERR_SHAPE
+    assert call(f=500) == tl.TWELL_ERR_SHAPE
+    assert call(dy=None) == tl.TWELL_ERR_NULL
+    assert call(a=None) == tl.TWELL_ERR_NULL
+    assert call(dx=MIS) == tl.TWELL_ERR_ALIGN
+    assert call(ws=None) == tl.TWELL_ERR_WORKSPACE
+    assert call(wsb=16) == tl.TWELL_ERR_WORKSPACE
+    need = lib.twell_backward_workspace_bytes(64, 128, 512, 16)
+    assert need > 0 and lib.twell_backward_workspace_bytes(0, 128, 512, 16) == 0
+    assert lib.twell_dense_backward_workspace_bytes(64, 128, 512) > 0
+    assert lib.twell_dense_ffn_backward(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 128, 512, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+                                        FAKE, None) == tl.TWELL_ERR_WORKSPACE
+    assert lib.twell_relu_ffn_hybrid_forward(FAKE, FAKE, None, 64, 128, 512, ctypes.byref(tw), FAKE, FAKE, FAKE, FAKE,
+                                             1 << 30, FAKE, None) == tl.TWELL_ERR_NULL
