@@ -433,36 +433,25 @@ __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) ag[e] = au[e] = ad[e] = 0.0f;
   const int e0 = p.colptr[j], e1 = p.colptr[j + 1];
+  // a batch of 32 records staged in shared memory, read back by broadcast
+  __shared__ float4 srec_all[8][32];
+  float4* srec = srec_all[threadIdx.x >> 5];
 #pragma unroll 1
   for (int b = e0; b < e1; b += 32) {
     const int nb = min(32, e1 - b);
-    const uint16_t* xr = nullptr;
-    const uint16_t* dr = nullptr;
-    float vh = 0.f, vu = 0.f, vz = 0.f;
-    if (lane < nb) {
-      const float4 rec = p.list[b + lane];
-      const size_t row = static_cast<size_t>(__float_as_int(rec.w));
-      xr = p.x0 + row * p.d;
-      dr = p.dy0 + row * p.d;
-      vh = rec.x;
-      vu = rec.y;
-      vz = rec.z;
-    }
-#pragma unroll 1
+    __syncwarp();
+    if (lane < nb) srec[lane] = p.list[b + lane];
+    __syncwarp();
+#pragma unroll 2
     for (int s = 0; s < nb; ++s) {
-      const uint16_t* xs = reinterpret_cast<const uint16_t*>(
-          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(xr), s));
-      const uint16_t* dsr = reinterpret_cast<const uint16_t*>(
-          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dr), s));
-      const float h = __shfl_sync(0xffffffffu, vh, s);
-      const float du = __shfl_sync(0xffffffffu, vu, s);
-      const float dz = __shfl_sync(0xffffffffu, vz, s);
+      const float4 rec = srec[s];
       if (mine) {
-        const uint4 xv = ldg_nc_v4(xs + k0);
-        const uint4 dv = ldg_nc_v4(dsr + k0);
-        axpy8(ad, h, dv);
-        axpy8(au, du, xv);
-        axpy8(ag, dz, xv);
+        const size_t off = static_cast<size_t>(__float_as_int(rec.w)) * p.d + k0;
+        const uint4 xv = ldg_nc_v4(p.x0 + off);
+        const uint4 dv = ldg_nc_v4(p.dy0 + off);
+        axpy8(ad, rec.x, dv);
+        axpy8(au, rec.y, xv);
+        axpy8(ag, rec.z, xv);
       }
     }
   }
