@@ -462,6 +462,7 @@ def run_gpu(args, world, rank, local):
         "dense_rows": {"bound": "tensor", "work": alg["dense_branch_flops"], "peak": tc, "unit": "TFLOP/s",
                        "scale": 1e12},
     }
+    sparse_flops_path = alg["sparse_flops"] if chosen in ("gate", "relu") else alg["sparse_flops"] / 2
     # weight rows the sparse step gathers: Wu and Wd rows in the gate form, Wd rows otherwise
     gathered_rows = nnz_stored * (2 if chosen == "gate" else 1)
     dom = max((names[0], names[2], "dense_rows"), key=lambda n: stage_ms[names.index(n)])
@@ -503,6 +504,9 @@ def run_gpu(args, world, rank, local):
                                        / 1e12)},
         "path_roofline": {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6, "t_roof_us": t_roof * 1e6,
                           "frac": t_roof / (step_ms * 1e-3),
+                          # the method's own second bound: the sparse step's FLOPs on the CUDA cores
+                          "t_simt_us": sparse_flops_path / fp32_peak * 1e6,
+                          "frac_with_simt": max(t_roof, sparse_flops_path / fp32_peak) / (step_ms * 1e-3),
                           "frac_gate_only": (alg["gate_flops"] / tc) / (step_ms * 1e-3),
                           "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TF/s"},
         "stages_ms": {n: float(v) for n, v in zip(names, stage_ms)},
@@ -759,6 +763,8 @@ def run_sweep(args) -> None:
     for T in Ts:
         for pden in Ps:
             cfg = synth.sweep_config(T, pden)
+            if args.sweep_w:
+                cfg = dataclasses.replace(cfg, W=args.sweep_w)
             L = synth.make_layer(cfg, seed=args.seed)
             x, WgT, WuT, Wd = (tl.to_device_bf16(L[k], dev) for k in ("x", "WgT", "WuT", "Wd"))
             tw = tl.Twell(T, cfg.f, cfg.W, device=dev)
@@ -850,6 +856,9 @@ def main(argv=None):
     ap.add_argument("--sweep-T", default="", help="comma-separated token counts (default: the full sweep)")
     ap.add_argument("--sweep-p", default="", help="comma-separated densities (default: the full sweep)")
     ap.add_argument("--sweep-eager", action="store_true", help="time sweep points without CUDA graphs")
+    ap.add_argument("--sweep-w", type=int, default=0,
+                    help="ELL width for every sweep point (0: the smallest that stores the pure sparse path); "
+                         "a fixed W such as 32 measures the hybrid route, dense branch included")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -304,3 +304,38 @@ def test_sparse_down_on_oracle_packed_input(cfg, layers):
     assert tl.status_get(st) == 0
     keep = np.nonzero(want["row_ovf"] == 0)[0]
     assert_y_close(y_to_f64(y)[keep], O.sparse_down_from_twell(want, L["Wd"], rows=keep))
+
+
+def test_gate_pack_unquantised_inputs():
+    """Plain N(0,1) bf16 inputs (no exact grid): the tensor cores' fp32 sums
+    may differ from fp64 in the last bits, so the pack is compared where the
+    sign of z is decided: tiles whose every |z| exceeds 2^-10 * sum|x w| match
+    exactly in counts and indices (values within one bf16 step); elsewhere the
+    count may move by at most the number of undecided entries. The excluded
+    count is reported."""
+    rng = np.random.default_rng(7)
+    T, d, f, W = 256, 512, 1024, 128
+    mk = lambda *s, sc=1.0: synth.f32_to_bf16_bits((rng.standard_normal(s) * sc).astype(np.float32))
+    L = {"x": mk(T, d), "WgT": mk(f, d, sc=d**-0.5)}
+    dev = upload(dict(L, WuT=L["WgT"], Wd=L["WgT"]))
+    tw = tl.Twell(T, f, W)
+    st = tl.new_status()
+    tl.gate_pack(dev["x"], dev["WgT"], tw, st)
+    assert tl.status_get(st) == 0
+    got = twell_to_host(tw)
+    x, w = O.bf16_bits_to_f64(L["x"]), O.bf16_bits_to_f64(L["WgT"])
+    z = x @ w.T
+    margin = 2.0**-10 * (np.abs(x) @ np.abs(w).T)
+    undecided = np.abs(z) <= margin
+    ref = O.twell_pack(z, 128, W)
+    nT = f // 128
+    und_tiles = undecided.reshape(T, nT, 128).sum(axis=2)
+    clean = und_tiles == 0
+    print(f"undecided entries: {int(undecided.sum())} of {T * f}; tiles excluded: {int((~clean).sum())}")
+    assert np.array_equal(got["counts"][clean], ref["counts"][clean])
+    assert np.all(np.abs(got["counts"].astype(int) - ref["counts"].astype(int)) <= und_tiles)
+    for t, c in zip(*np.nonzero(clean)):
+        n = int(ref["counts"][t, c])
+        assert np.array_equal(got["idx"][t, c, :n], ref["idx"][t, c, :n])
+        gv, rv = O.bf16_bits_to_f64(got["vals"][t, c, :n]), O.bf16_bits_to_f64(ref["vals"][t, c, :n])
+        assert np.all(np.abs(gv - rv) <= 2.0**-7 * np.abs(rv))
