@@ -717,3 +717,41 @@ def test_backward_weight_rows_agree_with_the_full_hybrid_backward():
     part = O.hybrid_backward_weight_rows(L["x"], L["WgT"], L["WuT"], L["Wd"], dy, full["ovf_rows"], cols)
     for k in ("dWgT", "dWuT", "dWd"):
         np.testing.assert_allclose(part[k], full[k][cols], rtol=1e-11, atol=1e-11 * np.abs(full[k]).max())
+
+
+def test_tiny_layers_bruteforce_over_1000_seeds():
+    """Tiny layers (T <= 8, d <= 16, f = 256) for seeds 0..999: the gate from
+    small-integer x and Wg (exact), the pack against plain loops (bf16 values
+    from torch's rounding, computed once per case), the routing predicate, and
+    for the rows that fit the sparse step against the dense layer."""
+    tile = 128
+    for seed in range(1000):
+        rng = np.random.default_rng(seed)
+        T, d, f = int(rng.integers(1, 9)), int(rng.integers(1, 17)), 256
+        W = (1, 2, 8, 16, 128)[seed % 5]
+        x = rng.integers(-3, 4, size=(T, d)).astype(np.float64)
+        wg = rng.integers(-3, 4, size=(f, d)).astype(np.float64)
+        shift = rng.integers(-6, 3)  # moves the density from nearly empty to nearly full
+        wg[:, 0] += shift
+        z = x @ wg.T
+        tw = O.twell_pack(z, tile, W)
+        zb = torch_bf16_bits(z.astype(np.float32)).astype(np.int64)
+        for t in range(T):
+            for c in range(f // tile):
+                n = 0
+                for k in range(tile):
+                    j = c * tile + k
+                    if z[t, j] > 0:
+                        if n < W:
+                            assert tw["idx"][t, c, n] == j and int(tw["vals"][t, c, n]) == zb[t, j], (seed, t, j)
+                        n += 1
+                assert tw["counts"][t, c] == n, (seed, t, c)
+        assert np.array_equal(tw["row_ovf"], (tw["counts"] > W).any(axis=1).astype(np.uint8))
+        keep = np.nonzero(tw["row_ovf"] == 0)[0]
+        if keep.size and seed % 10 == 0:  # the sparse step on a tenth of the cases
+            xb, wgb = bits_of_exact(x), bits_of_exact(wg)
+            wu = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+            wd = torch_bf16_bits(rng.standard_normal((f, d)).astype(np.float32))
+            ys = O.sparse_ffn_from_twell(tw, xb, wu, wd, rows=keep)
+            yd = O.gated_ffn(xb[keep], wgb, wu, wd)
+            np.testing.assert_allclose(ys, yd, rtol=1e-12, atol=1e-12 * max(1.0, np.abs(yd).max()))
