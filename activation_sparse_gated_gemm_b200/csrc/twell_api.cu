@@ -385,9 +385,12 @@ bool small_batch(int T, int N, int tile_n, int sms) {
 // first N columns of rows < M must hold zeros.
 twell_status f32_gemm_impl(const uint16_t* A, int M, const uint16_t* B, int N, int K, float* C, int ldo,
                            int32_t* dev_status, cudaStream_t s, int sms) {
+  // a batch of fewer than 128 rows loads only its rows of A
+  const int a_rows = std::min(kBM, (M + 7) / 8 * 8);
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, K, M, kBK, kBM) || !make_map(&mb, B, K, N, kBK, kBN)) return TWELL_ERR_CUDA;
+  if (!make_map(&ma, A, K, M, kBK, a_rows) || !make_map(&mb, B, K, N, kBK, kBN)) return TWELL_ERR_CUDA;
   GemmParams p{};
+  p.a_box_rows = a_rows;
   p.M = M;
   p.N = N;
   p.K = K;

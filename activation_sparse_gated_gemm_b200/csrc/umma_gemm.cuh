@@ -130,6 +130,10 @@ struct GemmParams {
   int k_half;
   // kModeDown / kModeF32: add into out_f32 even when K is not split.
   int accumulate;
+  // Rows of A per TMA box (0: all 128). A small batch loads only its rows (a
+  // multiple of 8); the A rows past them in shared memory hold stale data that
+  // only reaches accumulator rows the epilogue never stores.
+  int a_box_rows;
   const int* row_map;  // kModeDown: output row of each A row, or null
   int out_rows;        // valid range of output rows
   // kModeGateUp / kModeRelu: also store h_lo = bf16(h - bf16(h)) at column N + c (ldo = 2N).
@@ -293,7 +297,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // the K block's position in A (and B): compact K skips the empty
           // tail of each half
           const int kc = (nkb_half > 0 && kb >= nkb_half) ? p.k_half / kBK + (kb - nkb_half) : kb;
-          mbar_arrive_expect_tx(&full[s], kAStageBytes + kBStageBytes);
+          mbar_arrive_expect_tx(&full[s], (p.a_box_rows > 0 ? p.a_box_rows * kBK * 2 : kAStageBytes) + kBStageBytes);
           tma_load_2d(a_dst, &tmA, &full[s], kc * kBK, m_blk * kBM);
           if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity || MODE == kModeF32 ||
               MODE == kModeBwdDh) {
