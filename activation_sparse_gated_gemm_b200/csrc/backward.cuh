@@ -469,4 +469,40 @@ __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
   }
 }
 
+// Tensor-core form of the weight gradients: the records of the rows that fit,
+// scattered into three unit-major blocks dense[b][j][2 t_pad] (b = dz, du, h):
+// bf16(v) at token t and the bf16 remainder v - bf16(v) at t_pad + t, zeros
+// elsewhere. Three GEMMs over [tokens | tokens] against [x; x] (or dy) then
+// give dWg, dWu, dWd with ~2^-16 relative error per term. One warp per
+// (row, tile); rows that overflow are skipped.
+__global__ void bwd_scatter_dense_kernel(SlotSource src, int t_pad, uint16_t* __restrict__ dense) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const long long pairs = static_cast<long long>(src.rows) * src.nT;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const size_t row = 2 * static_cast<size_t>(t_pad);
+  const size_t block = static_cast<size_t>(src.f) * row;
+  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < pairs;
+       w += nw) {
+    const int t = static_cast<int>(w / src.nT);
+    if (src.row_ovf[t]) continue;
+    const int n = min(max(static_cast<int>(src.counts[w]), 0), src.W);
+    for (int k = lane; k < n; k += 32) {
+      const size_t slot = static_cast<size_t>(w) * src.W + k;
+      const int j = src.idx[slot];
+      if (j < 0 || j >= src.f) continue;
+      const float4 rec = src.rec[slot];
+      const size_t o = static_cast<size_t>(j) * row + t;
+      const float v[3] = {rec.z, rec.y, rec.x};  // dz, du, h
+#pragma unroll
+      for (int b = 0; b < 3; ++b) {
+        const uint16_t hi = f32_to_bf16_bits(v[b]);
+        dense[b * block + o] = hi;
+        dense[b * block + o + t_pad] = f32_to_bf16_bits(v[b] - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+      }
+    }
+  }
+}
+
 }  // namespace twell

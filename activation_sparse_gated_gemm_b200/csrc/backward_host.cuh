@@ -11,7 +11,9 @@
 // [dz | du | dz_lo | du_lo] ([T][4f] bf16) and the three transposed blocks dz,
 // du, h ([f][2 Tp] bf16 each); the column counts/cursors ([f]), column
 // offsets ([f + 1]) and the column-sorted records (one float4 per slot of the
-// rows that fit).
+// rows that fit); for the tensor-core form of the weight gradients, the rows
+// that fit as dense unit-major dz, du, h ([3][f][2 Tp] bf16, value and
+// remainder).
 struct BwdWorkspace {
   float4* rec;
   uint16_t *xo, *dyo;
@@ -19,6 +21,7 @@ struct BwdWorkspace {
   uint16_t *a2, *tT;
   int *colcnt, *colptr;
   float4* list;
+  uint16_t* dense;  // tensor-core form: dz, du, h of the rows that fit, [3][f][2 Tp] bf16 (value, remainder)
   int t_pad;
   size_t bytes;
 };
@@ -43,6 +46,7 @@ BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
   w.colcnt = reinterpret_cast<int*>(take(static_cast<size_t>(f) * 4));
   w.colptr = reinterpret_cast<int*>(take((static_cast<size_t>(f) + 1) * 4));
   w.list = reinterpret_cast<float4*>(take(s0 * 16));
+  w.dense = reinterpret_cast<uint16_t*>(take(3 * static_cast<size_t>(f) * 2 * tp * 2));
   w.t_pad = static_cast<int>(tp);
   w.bytes = off;
   return w;
@@ -164,6 +168,9 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   return launch_gemm<kModeDown>(ma2, mgT, muT, q3, sms, s);
 }
 
+twell_status backward_dw_overflow(int d, int f, const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd,
+                                  const BwdWorkspace& w, cudaStream_t s, int sms);
+
 // Weight gradients from the workspace filled by backward_dx_impl.
 twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int d, int f, const twell_t* tw,
                               const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd, char* ws, cudaStream_t s,
@@ -192,9 +199,14 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
   const long long warps = static_cast<long long>(f) * ((d + 255) / 256);
   TW_TRY(launch(bwd_wgrad_kernel, dim3(static_cast<unsigned>((warps + 7) / 8)), dim3(256), 0, s, g));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  // 4. the overflow rows' share, on the tensor cores: dWgT += dz^T x,
-  // dWuT += du^T x, dWd += h^T dy over the gathered rows (K = their tokens, as
-  // bf16 value and remainder halves)
+  return backward_dw_overflow(d, f, n_ovf, dWgT, dWuT, dWd, w, s, sms);
+}
+
+// The overflow rows' share of the weight gradients, on the tensor cores:
+// dWgT += dz^T x, dWuT += du^T x, dWd += h^T dy over the gathered rows (K =
+// their tokens, as bf16 value and remainder halves).
+twell_status backward_dw_overflow(int d, int f, const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd,
+                                  const BwdWorkspace& w, cudaStream_t s, int sms) {
   const size_t tblock = static_cast<size_t>(f) * 2 * w.t_pad;
   const uint16_t* aT[3] = {w.tT, w.tT + tblock, w.tT + 2 * tblock};
   const uint16_t* bT[3] = {w.xo, w.xo, w.dyo};
@@ -220,3 +232,37 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
   return TWELL_OK;
 }
 
+// Tensor-core form of the weight gradients from the workspace filled by
+// backward_dx_impl: the rows that fit are scattered densely (bf16 value and
+// remainder) by unit and token, three GEMMs over all tokens give their share,
+// then the overflow rows' GEMMs add theirs.
+twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, int d, int f, const twell_t* tw,
+                                 const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd, char* ws,
+                                 cudaStream_t s, int sms) {
+  const int nT = f / 128;
+  BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
+  const size_t block = static_cast<size_t>(f) * 2 * w.t_pad;
+  TW_TRY(zero_async(s, sms, w.dense, 3 * block * 2));
+  SlotSource a{tw->counts, tw->idx, w.rec, tw->row_ovf, T, nullptr, nT, tw->W, f, 1};
+  TW_TRY(launch(bwd_scatter_dense_kernel, dim3(4 * sms), dim3(256), 0, s, a, w.t_pad, w.dense));
+  // K runs over all tokens; rows of x and dy past T read as zeros
+  const bool split = static_cast<long long>(f / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms;
+  const uint16_t* bT[3] = {x, x, dy};
+  float* outs[3] = {dWgT, dWuT, dWd};
+  for (int i = 0; i < 3; ++i) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, w.dense + i * block, 2 * w.t_pad, f, kBK, kBM) || !make_map(&mb, bT[i], d, T, 64, kBK))
+      return TWELL_ERR_CUDA;
+    GemmParams q{};
+    q.M = f;
+    q.N = d;
+    q.K = 2 * w.t_pad;
+    q.k_wrap = w.t_pad;  // [value | remainder] halves against the same rows of x (or dy)
+    q.out_f32 = outs[i];
+    q.ldo = d;
+    q.k_splits_max = split ? 32 : 1;
+    if (split) TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
+    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, split ? sms : gemm_grid(f, d, kBN, sms), s));
+  }
+  return backward_dw_overflow(d, f, n_ovf, dWgT, dWuT, dWd, w, s, sms);
+}

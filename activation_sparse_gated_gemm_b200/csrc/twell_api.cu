@@ -768,6 +768,30 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
                           static_cast<cudaStream_t>(stream), sms);
 }
 
+twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* dy, int T, int d, int f,
+                                             const twell_t* tw, const int32_t* n_ovf, float* dWgT, float* dWuT,
+                                             float* dWd, void* workspace, size_t workspace_bytes, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (static_cast<long long>(T) * (f / 128) * tw->W >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  TW_TRY(check_ptrs({dWgT, dWuT, dWd}));
+  if (T == 0) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = static_cast<size_t>(f) * d * sizeof(float);
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWgT, 0, n, s)));
+    TW_TRY(cuda_ok(cudaMemsetAsync(dWuT, 0, n, s)));
+    return cuda_ok(cudaMemsetAsync(dWd, 0, n, s));
+  }
+  TW_TRY(check_ptrs({x, dy, n_ovf}));
+  if (workspace == nullptr || workspace_bytes < twell_backward_workspace_bytes(T, d, f, tw->W))
+    return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return backward_dw_tc_impl(x, dy, T, d, f, tw, n_ovf, dWgT, dWuT, dWd, static_cast<char*>(workspace),
+                             static_cast<cudaStream_t>(stream), sms);
+}
+
 size_t twell_dense_backward_workspace_bytes(int T, int d, int f) {
   (void)d;
   if (T <= 0 || f <= 0) return 0;

@@ -34,6 +34,7 @@ EXPORTED = (
     "twell_column_activity", "twell_compact_columns", "twell_gather_rows",
     "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward", "twell_ffn_hybrid_backward_dx",
     "twell_ffn_hybrid_backward_dw", "twell_dense_backward_workspace_bytes", "twell_dense_ffn_backward",
+    "twell_ffn_hybrid_backward_dw_tc",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -92,6 +93,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                       i32),
         "twell_ffn_hybrid_backward_dx": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_ffn_hybrid_backward_dw": ([vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, sz, vp], i32),
+        "twell_ffn_hybrid_backward_dw_tc": ([vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, sz, vp], i32),
         "twell_dense_backward_workspace_bytes": ([i32, i32, i32], sz),
         "twell_dense_ffn_backward": ([vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_column_activity": ([vp, vp, i32, i32, i32, vp, i32, vp, vp], i32),
@@ -361,14 +363,18 @@ def ffn_hybrid_backward_dx(x, WgT, WuT, Wd, dy, tw: Twell, ovf_rows, n_ovf, dx, 
         _ptr(dx), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
 
 
-def ffn_hybrid_backward_dw(x, dy, tw: Twell, n_ovf, dWgT, dWuT, dWd, workspace, stream=None) -> None:
+def ffn_hybrid_backward_dw(x, dy, tw: Twell, n_ovf, dWgT, dWuT, dWd, workspace, stream=None,
+                           tensor_cores: bool = False) -> None:
+    """Weight gradients after ffn_hybrid_backward_dx: per-unit sums on the CUDA
+    cores, or (tensor_cores) the dense-scatter form on the tensor cores."""
     T, d = x.shape
     f = tw.f
     _bf16("x", x, (T, d))
     _bf16("dy", dy, (T, d))
     for n, t in (("dWgT", dWgT), ("dWuT", dWuT), ("dWd", dWd)):
         _dev(n, t, (f, d), torch.float32)
-    _check("twell_ffn_hybrid_backward_dw", load().twell_ffn_hybrid_backward_dw(
+    name = "twell_ffn_hybrid_backward_dw_tc" if tensor_cores else "twell_ffn_hybrid_backward_dw"
+    _check(name, getattr(load(), name)(
         _ptr(x), _ptr(dy), T, d, f, tw.ref(), _ptr(n_ovf), _ptr(dWgT), _ptr(dWuT), _ptr(dWd), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 

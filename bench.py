@@ -567,8 +567,32 @@ def run_gpu_backward(args, world, rank, local):
     def stage_dx():
         tl.ffn_hybrid_backward_dx(x, WgT, WuT, Wd, dy, tw, ovf_rows, n_ovf, dx, wsb, st)
 
-    def stage_dw():
-        tl.ffn_hybrid_backward_dw(x, dy, tw, n_ovf, dW[0], dW[1], dW[2], wsb)
+    def make_dw(tensor_cores):
+        return lambda: tl.ffn_hybrid_backward_dw(x, dy, tw, n_ovf, dW[0], dW[1], dW[2], wsb,
+                                                 tensor_cores=tensor_cores)
+
+    # the two forms of the weight gradients (per-unit sums on the CUDA cores, or
+    # the dense scatter and GEMMs on the tensor cores), timed after a dx pass;
+    # the faster is the one the step uses
+    dw_forms = {}
+    stage_dx()
+    for name, tc in (("cuda_cores", False), ("tensor_cores", True)):
+        fn = make_dw(tc)
+        for _ in range(Wm):
+            flush.zero_()
+            fn()
+        ts = []
+        for _ in range(max(3, K // 4)):
+            flush.zero_()
+            a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_ev.record(stream)
+            fn()
+            b_ev.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a_ev.elapsed_time(b_ev))
+        dw_forms[name] = max_over_ranks(float(np.median(ts)), world)
+    dw_form = min(dw_forms, key=dw_forms.get)
+    stage_dw = make_dw(dw_form == "tensor_cores")
 
     for _ in range(Wm):
         flush.zero_()
@@ -624,7 +648,8 @@ def run_gpu_backward(args, world, rank, local):
 
     def e2e_step():
         dy.copy_(dy_host, non_blocking=True)
-        tl.ffn_hybrid_backward(x, WgT, WuT, Wd, dy, tw, ovf_rows, n_ovf, dx, dW[0], dW[1], dW[2], wsb, st)
+        stage_dx()
+        stage_dw()
         dx_host.copy_(dx, non_blocking=True)
         for h, g in zip(dW_host, dW):
             h.copy_(g, non_blocking=True)
@@ -660,6 +685,12 @@ def run_gpu_backward(args, world, rank, local):
                  * (clocks["sm_max_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6)
     names = ["backward_dx", "backward_dw"]
     work = {"backward_dx": flops_dx, "backward_dw": flops_dw}
+    bound = {"backward_dx": "alu", "backward_dw": "alu"}
+    peak_tf = {"backward_dx": fp32_peak / 1e12, "backward_dw": fp32_peak / 1e12}
+    if dw_form == "tensor_cores":  # three GEMMs over all tokens (plus the overflow rows' ones)
+        work["backward_dw"] = 6.0 * T * d * f
+        bound["backward_dw"] = "tensor"
+        peak_tf["backward_dw"] = peaks["bf16_tflops"]
     dom = names[int(np.argmax(stage_ms))]
     ms = float(stage_ms[names.index(dom)])
     achieved = work[dom] / (ms * 1e-3) / 1e12
@@ -680,10 +711,13 @@ def run_gpu_backward(args, world, rank, local):
                    "tokens": T, "d": d, "f": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
                    "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
-        "roofline": {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": fp32_peak / 1e12,
-                     "unit": "TFLOP/s", "frac": achieved / (fp32_peak / 1e12), "traffic": None,
-                     "peak_source": "fp32 FMA lanes x 2 x max SM clock"},
+        "roofline": {"kernel": dom, "bound": bound[dom], "achieved": achieved, "peak": peak_tf[dom],
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf[dom], "traffic": None,
+                     "peak_source": ("fp32 FMA lanes x 2 x max SM clock" if bound[dom] == "alu"
+                                     else f"{peaks['source']} bf16 burst")},
         "stages_ms": {n: float(v) for n, v in zip(names, stage_ms)},
+        "weight_gradient_forms_ms": dw_forms,
+        "weight_gradient_form": dw_form,
         "batch_stats": {"n_ovf": n_ovf_h, "nnz_fit_rows": nnz_fit, "nnz_overflow_rows": nnz_ovf,
                         "dense_branch_gflop": 12.0 * n_ovf_h * d * f / 1e9},
         "dense_backward_ms": dense_ms,

@@ -330,6 +330,20 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
                                           float* dWd, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Tensor-core form of twell_ffn_hybrid_backward_dw (same arguments, same
+ * workspace, called after twell_ffn_hybrid_backward_dx). At densities where
+ * every unit is active for many tokens of a batch, the weight gradients are a
+ * dense contraction over the tokens: the rows that fit scatter their dz, du
+ * and h (as bf16 value plus bf16 remainder) by unit and token into dense
+ * blocks, three tcgen05 GEMMs over all tokens form their share, and the
+ * overflow rows' GEMMs add theirs. The extra error is ~2^-16 of each term; the
+ * sums are in fp32 in a fixed order.
+ */
+twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* dy, int T, int d, int f,
+                                             const twell_t* tw, const int32_t* n_ovf, float* dWgT, float* dWuT,
+                                             float* dWd, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dense backward of the gated layer on the tensor cores, no sparsity: the
  * library's own baseline for twell_ffn_hybrid_backward. [z | u] = x [Wg | Wu]
  * (fp32), dh = dy Wd^T with dz = dh u [z > 0], du = dh ReLU(z), h = ReLU(z) u

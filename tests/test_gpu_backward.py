@@ -188,3 +188,38 @@ def test_dense_backward_baseline(cfg):
         err = np.abs(got - ref[k])
         bound = b[k] + 1e-6 * float(np.sqrt(np.mean(ref[k] ** 2)))
         assert np.all(err <= bound), (k, float((err / bound).max()))
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_tensor_core_weight_gradients(cfg):
+    """The tensor-core form of the weight gradients (dz, du, h of the rows that
+    fit as bf16 value plus remainder, GEMMs over the tokens) against the
+    oracle: within the contract and within 2^-15 of the summed term magnitudes
+    on top of the tight check."""
+    L = synth.make_layer(cfg, seed=0)
+    dy_bits = make_dy(cfg.T, cfg.d, 6)
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.empty((T,), dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    dy = tl.to_device_bf16(dy_bits)
+    dx = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    dW = [torch.full((f, d), float("nan"), dtype=torch.float32, device="cuda") for _ in range(3)]
+    wsb = torch.empty(tl.backward_workspace_bytes(T, d, f, W), dtype=torch.uint8, device="cuda")
+    tl.ffn_hybrid_backward_dx(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], dy, tw, ovf_rows, n_ovf, dx, wsb, st)
+    tl.ffn_hybrid_backward_dw(dev["x"], dy, tw, n_ovf, dW[0], dW[1], dW[2], wsb, tensor_cores=True)
+    assert tl.status_get(st) == 0
+    ref = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy_bits, cfg.tile, cfg.W)
+    b = dense_branch_bounds(L, dy_bits, np.arange(T))
+    for k, t in zip(("dWgT", "dWuT", "dWd"), dW):
+        got = t.double().cpu().numpy()
+        assert np.isfinite(got).all(), k
+        rms = float(np.sqrt(np.mean(ref[k] ** 2)))
+        err = np.abs(got - ref[k])
+        assert err.max() <= CONTRACT * rms, (k, float(err.max()), rms)
+        assert np.all(err <= b[k] + TIGHT * rms), k
