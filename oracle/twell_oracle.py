@@ -28,9 +28,10 @@ Readings taken where the pages are silent:
   overflow rows, in ascending order, go to the dense branch;
 * the dense branch recomputes the gate for its rows.
 
-Pinned by ``tests/test_oracle.py`` (closed forms, exact rational brute force,
-library rounding, hand-written fixtures in ``tests/golden``, invariants).
-Parity unpinned: nothing on the pages gives a numeric worked example.
+Every function here is pinned by ``tests/test_oracle.py`` (closed forms,
+exact rational brute force, finite differences, library rounding, hand-derived
+fixtures in ``tests/golden``, invariants). The pages print no numeric worked
+example, so no pin uses values printed on the pages.
 """
 
 from __future__ import annotations
