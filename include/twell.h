@@ -138,6 +138,32 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
                                int skip_overflow_rows, float* y, int32_t* dev_status, void* stream);
 
 /*
+ * The same down projection, staged through shared memory (same source; the
+ * staging is this library's, not the pages'). An alternative to
+ * twell_sparse_down, which the hybrid forwards use: on B200 at the 0.5B-2B
+ * layer shapes this form is 1.7-3.4x slower (its per-slot instruction count,
+ * not memory, bounds it). The tokens
+ * are cut into groups of G (120..240, chosen from T, d and the SM count);
+ * per group and per 128-column slice of d, Wd is copied into shared memory
+ * in chunks of 256 rows and each stored slot of the group's tokens reads its
+ * row piece there instead of gathering the whole row from L2. y as for
+ * twell_sparse_down (fp32 sums in another order); rows skipped by
+ * skip_overflow_rows are left untouched.
+ * Requires d >= 128 (TWELL_ERR_SHAPE otherwise). workspace: device memory of
+ * at least twell_sparse_down_staged_workspace_bytes(T, d, f, W) bytes,
+ * 16-byte aligned, caller-owned, overwritten (the per-group token order, the
+ * per-chunk slot lists). A stored index outside its own column tile raises
+ * TWELL_ERR_INDEX and adds nothing. Three kernel launches.
+ */
+twell_status twell_sparse_down_staged(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                                      int skip_overflow_rows, float* y, void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, void* stream);
+
+/* Workspace bytes of twell_sparse_down_staged (about T * f * W / 32, the
+ * slot lists at full ELL width, plus small tables). */
+size_t twell_sparse_down_staged_workspace_bytes(int T, int d, int f, int W);
+
+/*
  * Hybrid forward of the tensor-core-up variant = twell_gate_up_pack,
  * twell_route, twell_sparse_down with overflowing rows skipped, and
  * twell_dense_rows_forward on ovf_rows. Same arguments and workspace as
