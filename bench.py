@@ -299,15 +299,25 @@ def run_gpu(args, world, rank, local):
     # The two forms of the hybrid forward: "gate" packs ReLU(z) and runs the
     # fused sparse up+down step; "tc_up" forms u on the tensor cores with the
     # gate and packs h, leaving only the down projection sparse.
+    # --down staged: the down projection of the tc_up and non-gated forms
+    # through the shared-memory-staged alternative (its lists in a workspace of
+    # its own), to measure it against the per-token kernel the library uses
+    ws_staged = (torch.empty(tl.sparse_down_staged_workspace_bytes(T, d, f, W), dtype=torch.uint8, device=dev)
+                 if args.down == "staged" else None)
+
+    def down():
+        if ws_staged is not None:
+            tl.sparse_down_staged(Wd, tw, y, True, ws_staged, st)
+        else:
+            tl.sparse_down(Wd, tw, y, True, st)
+
     def stage_fns(variant):
         if variant == "relu":  # the non-gated layer ReLU(x W1) W2 with W1 = Wg, W2 = Wd
-            return [lambda: tl.gate_pack(x, WgT, tw, st), lambda: tl.route(tw, ovf_rows, n_ovf),
-                    lambda: tl.sparse_down(Wd, tw, y, True, st),
+            return [lambda: tl.gate_pack(x, WgT, tw, st), lambda: tl.route(tw, ovf_rows, n_ovf), down,
                     lambda: tl.relu_dense_rows_forward(x, WgT, Wd, ovf_rows, n_ovf, y, ws, st)]
         pack = ((lambda: tl.gate_pack(x, WgT, tw, st)) if variant == "gate"
                 else (lambda: tl.gate_up_pack(x, WgT, WuT, tw, st)))
-        sparse = ((lambda: tl.sparse_ffn(x, WuT, Wd, tw, y, True, st)) if variant == "gate"
-                  else (lambda: tl.sparse_down(Wd, tw, y, True, st)))
+        sparse = (lambda: tl.sparse_ffn(x, WuT, Wd, tw, y, True, st)) if variant == "gate" else down
         return [pack, lambda: tl.route(tw, ovf_rows, n_ovf), sparse,
                 lambda: tl.dense_rows_forward(x, WgT, WuT, Wd, ovf_rows, n_ovf, y, ws, st)]
 
@@ -518,9 +528,13 @@ def run_gpu(args, world, rank, local):
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4,
                 "pipelined": "copy-in, compute and copy-out on three streams, two buffer sets",
+                "path": "the library's hybrid forward of the chosen form (per-token down projection)",
                 "l2": "not flushed: each step touches ~0.26 GB, above the 126 MB L2"},
         # per step: zeroing, gate (or gate+up) GEMM, routing, sparse step, row gather, two dense-branch GEMMs
-        "gpu_launches": 7 * K,
+        # (the staged down projection adds its two planning kernels)
+        "gpu_launches": (9 if ws_staged is not None and chosen != "gate" else 7) * K,
+        "down_projection": ("fused up+down per token" if chosen == "gate" else
+                            "staged through shared memory" if ws_staged is not None else "per token"),
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -884,6 +898,9 @@ def main(argv=None):
                     help="gated: (ReLU(x Wg) * x Wu) Wd; relu: the non-gated ReLU(x W1) W2")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
                     help="forward (the default) or the backward pass through the hybrid format")
+    ap.add_argument("--down", default="per_token", choices=["per_token", "staged"],
+                    help="down projection of the tc_up and non-gated forms (the library's hybrid forwards use "
+                         "per_token)")
     ap.add_argument("--compact", action="store_true",
                     help="drop the hidden units the batch never activates before timing")
     ap.add_argument("--sweep", action="store_true", help="density x batch sweep, one JSON line per point")
