@@ -406,6 +406,7 @@ size_t staged_bytes_bound(int T, int d, int f, int W) {
 twell_status staged_down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip, float* y,
                               void* ws, int32_t* dev_status, cudaStream_t s, int sms) {
   const StagedPlan pl = staged_plan(T, d, f, tw->W, sms);
+  if (pl.ngroups > 65535) return TWELL_ERR_SHAPE;  // the list kernel's grid has one row per token group
   StagedParams p{};
   p.counts = tw->counts;
   p.idx = tw->idx;

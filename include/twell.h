@@ -149,7 +149,8 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
  * row piece there instead of gathering the whole row from L2. y as for
  * twell_sparse_down (fp32 sums in another order); rows skipped by
  * skip_overflow_rows are left untouched.
- * Requires d >= 128 (TWELL_ERR_SHAPE otherwise). workspace: device memory of
+ * Requires d >= 128 and at most 65535 token groups (T up to about 7.8 M;
+ * TWELL_ERR_SHAPE otherwise). workspace: device memory of
  * at least twell_sparse_down_staged_workspace_bytes(T, d, f, W) bytes,
  * 16-byte aligned, caller-owned, overwritten (the per-group token order, the
  * per-chunk slot lists). A stored index outside its own column tile raises
