@@ -9,9 +9,11 @@
 //   dWd[j, :] = sum_t h_tj dy_t, dWu[:, j] = sum_t du_tj x_t, dWg[:, j] = sum_t dz_tj x_t
 //
 // Rows that fit the ELL width take three passes over their stored units:
-//   1. per token (one warp per token, like the forward's fused kernel): u_j and
-//      dh_j by two dot products per stored unit; each slot's record
-//      {h, du, dz, token} is written beside the slots;
+//   0. dh = dy . Wd^T for every token on the tensor cores (a plain dense
+//      contraction, [T][f] fp32): cheaper than gathering a row of Wd per slot;
+//   1. per token (one warp per token, like the forward's fused kernel): u_j by
+//      a dot product per stored unit, dh_j read from row t of dh; each slot's
+//      record {h, du, dz, token} is written beside the slots;
 //   1b. per token again: dx_t by two row axpys with du_j, dz_j from the records
 //      (split from pass 1 so that neither pass holds both dx_t and the dot
 //      passes' rows, which lets each run twice the warps);
@@ -30,10 +32,9 @@ namespace twell {
 
 struct BwdParams {
   const uint16_t* x;   // [rows][d] bf16
-  const uint16_t* dy;  // [rows][d] bf16 upstream gradient
   const uint16_t* WgT;
   const uint16_t* WuT;
-  const uint16_t* Wd;
+  const float* dh;        // [rows][f] fp32: dy . Wd^T
   const int16_t* counts;  // TwELL of these rows (the forward's gate pack)
   const int16_t* idx;
   const uint16_t* vals;
@@ -45,9 +46,9 @@ struct BwdParams {
   int* dev_status;
 };
 
-// Warps per block of the two per-token passes. The dot pass holds x_t and
-// dy_t in shared memory and two weight rows in registers; the dx pass holds
-// dx_t and two weight rows in registers.
+// Warps per block of the two per-token passes. The dot pass holds x_t in
+// shared memory and two weight rows in registers; the dx pass holds dx_t and
+// two weight rows in registers.
 constexpr int bwd_dots_warps(int nch) {
   // registers (two rows of d per lane and the reductions) cap it before shared memory does
   return nch <= 6 ? 16 : (nch <= 8 ? 12 : 8);
@@ -55,12 +56,12 @@ constexpr int bwd_dots_warps(int nch) {
 constexpr int bwd_dx_warps(int nch) { return nch <= 4 ? 16 : (nch <= 7 ? 12 : 8); }
 
 constexpr size_t bwd_dots_smem_bytes(int nch) {
-  return static_cast<size_t>(bwd_dots_warps(nch)) * (2 * nch * 32 * 16 + kListCap * 6);
+  return static_cast<size_t>(bwd_dots_warps(nch)) * (nch * 32 * 16 + kListCap * 6);
 }
 constexpr size_t bwd_dx_smem_bytes(int nch) { return static_cast<size_t>(bwd_dx_warps(nch)) * kListCap * 6; }
 
-// 16-byte shared-memory load that the compiler keeps inside its loop (x_t and
-// dy_t are reread per entry instead of being held in registers across it).
+// 16-byte shared-memory load that the compiler keeps inside its loop (x_t is
+// reread per entry instead of being held in registers across it).
 __device__ __forceinline__ uint4 lds_v4(const uint4* p) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -202,10 +203,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dots_kernel(const BwdParams
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int d = p.d;
-  uint4* xs = bwd_smem + warp * 2 * NCH * 32;
-  uint4* ds = xs + NCH * 32;
-  uint32_t* list = reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) + warp * kListCap;
-  uint16_t* lpos = reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + WARPS * 2 * NCH * 32) +
+  uint4* xs = bwd_smem + warp * NCH * 32;
+  uint32_t* list = reinterpret_cast<uint32_t*>(bwd_smem + WARPS * NCH * 32) + warp * kListCap;
+  uint16_t* lpos = reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + WARPS * NCH * 32) +
                                                WARPS * kListCap) +
                    warp * kListCap;
   const int group_tiles = max(1, kListCap / p.W);
@@ -224,8 +224,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dots_kernel(const BwdParams
       const int k0 = (i * 32 + lane) * 8;
       const bool in = k0 < d;
       xs[i * 32 + lane] = in ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
-      ds[i * 32 + lane] = in ? ldg_nc_v4(p.dy + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
     }
+    const float* dh_row = p.dh + static_cast<size_t>(t) * p.f;
     const size_t slot_row = static_cast<size_t>(t) * p.nT * p.W;
 #pragma unroll 1
     for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
@@ -238,7 +238,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dots_kernel(const BwdParams
         const int my_j = entry_j(my_e);
         const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
         const float my_u = bwd_dot_pass<NCH>(xs, p.WuT, my_j, ns, lane, d);
-        const float my_dh = bwd_dot_pass<NCH>(ds, p.Wd, my_j, ns, lane, d);
+        // my_j is a checked column (0 for an entry that was out of range)
+        const float my_dh = lane < ns ? __ldg(dh_row + my_j) : 0.0f;
         const float my_g = entry_g(my_e);
         if ((my_pos & 0x8000u) == 0)
           p.s_rec[slot_row + my_pos] = make_float4(my_g * my_u, my_dh * my_g, my_dh * my_u, __int_as_float(t));

@@ -7,7 +7,8 @@
 // Workspace of the hybrid backward, carved in this order (each piece 256-byte
 // aligned): per-slot records {h, du, dz, token} of the rows that fit
 // ([T][nT][W] float4); for the overflow rows, the gathered rows of x and dy
-// ([Tp][d] bf16 each, Tp = T rounded up to 64), their [z | u] ([T][2f] fp32),
+// ([Tp][d] bf16 each, Tp = T rounded up to 64), their [z | u] ([T][2f] fp32;
+// before that, dh = dy . Wd^T of every token, [T][f] fp32),
 // [dz | du | dz_lo | du_lo] ([T][4f] bf16) and the three transposed blocks dz,
 // du, h ([f][2 Tp] bf16 each); the column counts/cursors ([f]), column
 // offsets ([f + 1]) and the column-sorted records (one float4 per slot of the
@@ -98,13 +99,19 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
                               int sms) {
   const int nT = f / 128;
   BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
+  // 0. dh = dy . Wd^T for every token, fp32 [T][f], in the [z | u] region
+  // (free until the overflow rows' dense branch below). K is split over the
+  // grid, with partial sums added into zeroed rows, when the output tiles
+  // cannot fill it.
+  const long long dh_tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((f + kBN - 1) / kBN);
+  if (dh_tiles < sms) TW_TRY(zero_async(s, sms, w.zu, static_cast<size_t>(T) * f * sizeof(float)));
+  TW_TRY(f32_gemm_impl(dy, T, Wd, f, d, w.zu, f, dev_status, s, sms));
   // 1. rows that fit: per-token pass over their stored slots
   BwdParams p0{};
   p0.x = x;
-  p0.dy = dy;
   p0.WgT = WgT;
   p0.WuT = WuT;
-  p0.Wd = Wd;
+  p0.dh = w.zu;
   p0.counts = tw->counts;
   p0.idx = tw->idx;
   p0.vals = tw->vals;

@@ -738,9 +738,9 @@ def run_gpu_backward(args, world, rank, local):
         "speedup_vs_own_dense": dense_ms / step_ms,
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
-        # per step: dots and dx passes, two gathers, three dense-branch GEMMs; zeroing, count, scan,
-        # scatter, per-unit sums and three weight-gradient GEMMs
-        "gpu_launches": 15 * K,
+        # per step: the dh GEMM, dots and dx passes, two gathers, three dense-branch GEMMs; zeroing, count,
+        # scan, scatter, per-unit sums and three weight-gradient GEMMs
+        "gpu_launches": 16 * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
