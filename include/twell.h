@@ -319,7 +319,8 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
  *   dWgT [f][d] = dz^T x, dWuT [f][d] = du^T x, dWd [f][d] = h^T dy   (fp32,
  *   overwritten; the layouts of WgT, WuT and Wd)
  * tw, ovf_rows and n_ovf are the outputs of twell_ffn_hybrid_forward on the
- * same x (the gate form: tw's values are the bf16 gate). Rows that fit use
+ * same x (the gate form: tw's values are the bf16 gate). dh is formed for
+ * every token by one tensor-core GEMM (dy Wd^T, fp32 sums). Rows that fit use
  * their stored slots with the stored bf16 gate g (h = g u), so the result is
  * the method's, within one bf16 rounding per term of the exact gradients;
  * their weight gradients are summed per hidden unit over a column sort of the
