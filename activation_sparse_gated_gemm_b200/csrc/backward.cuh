@@ -506,4 +506,39 @@ __global__ void bwd_scatter_dense_kernel(SlotSource src, int t_pad, uint16_t* __
   }
 }
 
+// Tensor-core form of dx: the records of the rows that fit, scattered into
+// token-major rows a2[t][4f] = [dz | du | dz_lo | du_lo] (bf16 value, then the
+// bf16 remainder v - bf16(v); zeros elsewhere, rows that overflow left zero),
+// the layout of the overflow rows' dense branch, so that one GEMM against
+// [Wg; Wu] (read twice along K) gives dx for every token. One warp per
+// (row, tile).
+__global__ void bwd_scatter_rows_kernel(SlotSource src, uint16_t* __restrict__ a2) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const long long pairs = static_cast<long long>(src.rows) * src.nT;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const size_t f = static_cast<size_t>(src.f);
+  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < pairs;
+       w += nw) {
+    const int t = static_cast<int>(w / src.nT);
+    if (src.row_ovf[t]) continue;
+    const int n = min(max(static_cast<int>(src.counts[w]), 0), src.W);
+    uint16_t* row = a2 + static_cast<size_t>(t) * 4 * f;
+    for (int k = lane; k < n; k += 32) {
+      const size_t slot = static_cast<size_t>(w) * src.W + k;
+      const int j = src.idx[slot];
+      if (j < 0 || j >= src.f) continue;
+      const float4 rec = src.rec[slot];
+      const float v[2] = {rec.z, rec.y};  // dz, du
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const uint16_t hi = f32_to_bf16_bits(v[b]);
+        row[b * f + j] = hi;
+        row[(2 + b) * f + j] = f32_to_bf16_bits(v[b] - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+      }
+    }
+  }
+}
+
 }  // namespace twell

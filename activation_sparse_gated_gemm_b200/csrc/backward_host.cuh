@@ -62,41 +62,45 @@ twell_status launch_bwd_pass(void (*kern)(BwdParams), size_t smem, const BwdPara
   return launch(kern, dim3(blocks), dim3(WARPS * 32), smem, s, p);
 }
 
-// The per-token passes of the rows that fit: the dot pass (records), then dx.
+// The per-token passes of the rows that fit: the dot pass (records), then dx
+// (unless the tensor cores form dx).
 template <int NCH>
-twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s) {
+twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s, bool with_dx) {
   constexpr int kDots = bwd_dots_warps(NCH), kDx = bwd_dx_warps(NCH);
   TW_TRY((launch_bwd_pass<NCH, kDots>(bwd_dots_kernel<NCH, kDots>, bwd_dots_smem_bytes(NCH), p, sms, s)));
+  if (!with_dx) return TWELL_OK;
   return launch_bwd_pass<NCH, kDx>(bwd_dx_kernel<NCH, kDx>, bwd_dx_smem_bytes(NCH), p, sms, s);
 }
 
-twell_status launch_bwd_token(const BwdParams& p, int sms, cudaStream_t s) {
+twell_status launch_bwd_token(const BwdParams& p, int sms, cudaStream_t s, bool with_dx) {
   switch ((p.d + 255) / 256) {
-    case 1: return launch_bwd_token_n<1>(p, sms, s);
-    case 2: return launch_bwd_token_n<2>(p, sms, s);
-    case 3: return launch_bwd_token_n<3>(p, sms, s);
-    case 4: return launch_bwd_token_n<4>(p, sms, s);
-    case 5: return launch_bwd_token_n<5>(p, sms, s);
-    case 6: return launch_bwd_token_n<6>(p, sms, s);
-    case 7: return launch_bwd_token_n<7>(p, sms, s);
-    case 8: return launch_bwd_token_n<8>(p, sms, s);
-    case 9: return launch_bwd_token_n<9>(p, sms, s);
-    case 10: return launch_bwd_token_n<10>(p, sms, s);
-    case 11: return launch_bwd_token_n<11>(p, sms, s);
-    case 12: return launch_bwd_token_n<12>(p, sms, s);
-    case 13: return launch_bwd_token_n<13>(p, sms, s);
-    case 14: return launch_bwd_token_n<14>(p, sms, s);
-    case 15: return launch_bwd_token_n<15>(p, sms, s);
-    case 16: return launch_bwd_token_n<16>(p, sms, s);
+    case 1: return launch_bwd_token_n<1>(p, sms, s, with_dx);
+    case 2: return launch_bwd_token_n<2>(p, sms, s, with_dx);
+    case 3: return launch_bwd_token_n<3>(p, sms, s, with_dx);
+    case 4: return launch_bwd_token_n<4>(p, sms, s, with_dx);
+    case 5: return launch_bwd_token_n<5>(p, sms, s, with_dx);
+    case 6: return launch_bwd_token_n<6>(p, sms, s, with_dx);
+    case 7: return launch_bwd_token_n<7>(p, sms, s, with_dx);
+    case 8: return launch_bwd_token_n<8>(p, sms, s, with_dx);
+    case 9: return launch_bwd_token_n<9>(p, sms, s, with_dx);
+    case 10: return launch_bwd_token_n<10>(p, sms, s, with_dx);
+    case 11: return launch_bwd_token_n<11>(p, sms, s, with_dx);
+    case 12: return launch_bwd_token_n<12>(p, sms, s, with_dx);
+    case 13: return launch_bwd_token_n<13>(p, sms, s, with_dx);
+    case 14: return launch_bwd_token_n<14>(p, sms, s, with_dx);
+    case 15: return launch_bwd_token_n<15>(p, sms, s, with_dx);
+    case 16: return launch_bwd_token_n<16>(p, sms, s, with_dx);
     default: return TWELL_ERR_SHAPE;
   }
 }
 
-// dx, and the per-slot scalars of both passes in the workspace.
+// dx, and the per-slot scalars of both passes in the workspace. tc_dx: the
+// rows that fit get dx from one tensor-core GEMM over their scattered dz, du
+// instead of the per-token axpy pass.
 twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
                               const uint16_t* dy, int T, int d, int f, const twell_t* tw, const int32_t* ovf_rows,
                               const int32_t* n_ovf, float* dx, char* ws, int32_t* dev_status, cudaStream_t s,
-                              int sms) {
+                              int sms, bool tc_dx = false) {
   const int nT = f / 128;
   BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
   // 0. dh = dy . Wd^T for every token, fp32 [T][f], in the [z | u] region
@@ -124,7 +128,37 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   p0.dx = dx;
   p0.s_rec = w.rec;
   p0.dev_status = dev_status;
-  TW_TRY(launch_bwd_token(p0, sms, s));
+  TW_TRY(launch_bwd_token(p0, sms, s, !tc_dx));
+  if (tc_dx) {
+    // 1b. dx of every token = [dz | du | dz_lo | du_lo] [Wg; Wu; Wg; Wu]^T on
+    // the tensor cores, the rows that fit scattered token-major into the
+    // [z | u] region (dh there is no longer needed), overflow rows left zero
+    // (their dx is rewritten below). K is split over the grid, with partial
+    // sums added into zeroed rows, when the output tiles cannot fill it.
+    uint16_t* a2all = reinterpret_cast<uint16_t*>(w.zu);
+    const long long dx_tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN);
+    if (dx_tiles < sms)
+      TW_TRY(zero_async(s, sms, a2all, static_cast<size_t>(T) * 4 * f * 2, dx, static_cast<size_t>(T) * d * 4));
+    else
+      TW_TRY(zero_async(s, sms, a2all, static_cast<size_t>(T) * 4 * f * 2));
+    SlotSource src{tw->counts, tw->idx, w.rec, tw->row_ovf, T, nullptr, nT, tw->W, f, 1};
+    TW_TRY(launch(bwd_scatter_rows_kernel, dim3(4 * sms), dim3(256), 0, s, src, a2all));
+    CUtensorMap ma, mgT, muT;
+    if (!make_map(&ma, a2all, 4 * f, T, kBK, kBM) || !make_map(&mgT, WgT, d, f, 64, kBK) ||
+        !make_map(&muT, WuT, d, f, 64, kBK))
+      return TWELL_ERR_CUDA;
+    GemmParams q{};
+    q.M = T;
+    q.N = d;
+    q.K = 4 * f;
+    q.k_wrap = 2 * f;
+    q.k_split_b = f;
+    q.out_f32 = dx;
+    q.ldo = d;
+    q.k_splits_max = 32;
+    q.dev_status = dev_status;
+    TW_TRY(launch_gemm<kModeDown>(ma, mgT, muT, q, dx_tiles < sms ? sms : gemm_grid(T, d, kBN, sms), s));
+  }
   // 2. overflow rows, dense on the tensor cores: gather x and dy (zero the dx
   // rows and the padding rows up to a multiple of 64), recompute [z | u], then
   // dh = dy Wd^T with dz, du, h in its epilogue, then dx = [dz | du] [Wg; Wu]^T

@@ -870,6 +870,25 @@ twell_status twell_ffn_hybrid_backward_dx(const uint16_t* x, const uint16_t* WgT
                           dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 
+twell_status twell_ffn_hybrid_backward_dx_tc(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                             const uint16_t* Wd, const uint16_t* dy, int T, int d, int f,
+                                             const twell_t* tw, const int32_t* ovf_rows, const int32_t* n_ovf,
+                                             float* dx, void* workspace, size_t workspace_bytes,
+                                             int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (static_cast<long long>(T) * (f / 128) * tw->W >= (1LL << 31)) return TWELL_ERR_SHAPE;
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({x, WgT, WuT, Wd, dy, ovf_rows, n_ovf, dx, dev_status}));
+  if (workspace == nullptr || workspace_bytes < twell_backward_workspace_bytes(T, d, f, tw->W))
+    return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return backward_dx_impl(x, WgT, WuT, Wd, dy, T, d, f, tw, ovf_rows, n_ovf, dx, static_cast<char*>(workspace),
+                          dev_status, static_cast<cudaStream_t>(stream), sms, true);
+}
+
 twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy, int T, int d, int f,
                                           const twell_t* tw, const int32_t* n_ovf, float* dWgT, float* dWuT,
                                           float* dWd, void* workspace, size_t workspace_bytes, void* stream) {

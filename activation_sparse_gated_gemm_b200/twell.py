@@ -35,6 +35,7 @@ EXPORTED = (
     "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward", "twell_ffn_hybrid_backward_dx",
     "twell_ffn_hybrid_backward_dw", "twell_dense_backward_workspace_bytes", "twell_dense_ffn_backward",
     "twell_ffn_hybrid_backward_dw_tc", "twell_sparse_down_staged", "twell_sparse_down_staged_workspace_bytes",
+    "twell_ffn_hybrid_backward_dx_tc",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -94,6 +95,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_ffn_hybrid_backward": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp],
                                       i32),
         "twell_ffn_hybrid_backward_dx": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
+        "twell_ffn_hybrid_backward_dx_tc": ([vp, vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp],
+                                            i32),
         "twell_ffn_hybrid_backward_dw": ([vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, sz, vp], i32),
         "twell_ffn_hybrid_backward_dw_tc": ([vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, vp, sz, vp], i32),
         "twell_dense_backward_workspace_bytes": ([i32, i32, i32], sz),
@@ -369,14 +372,17 @@ def ffn_hybrid_backward(x, WgT, WuT, Wd, dy, tw: Twell, ovf_rows, n_ovf, dx, dWg
 
 
 def ffn_hybrid_backward_dx(x, WgT, WuT, Wd, dy, tw: Twell, ovf_rows, n_ovf, dx, workspace, dev_status,
-                           stream=None) -> None:
+                           stream=None, tensor_cores: bool = False) -> None:
+    """dx and the per-slot records: the rows that fit by per-token axpys on the
+    CUDA cores, or (tensor_cores) by one GEMM over their scattered dz, du."""
     T, d = x.shape
     f = WgT.shape[0]
     for n, t, s in (("x", x, (T, d)), ("WgT", WgT, (f, d)), ("WuT", WuT, (f, d)), ("Wd", Wd, (f, d)),
                     ("dy", dy, (T, d))):
         _bf16(n, t, s)
     _dev("dx", dx, (T, d), torch.float32)
-    _check("twell_ffn_hybrid_backward_dx", load().twell_ffn_hybrid_backward_dx(
+    name = "twell_ffn_hybrid_backward_dx_tc" if tensor_cores else "twell_ffn_hybrid_backward_dx"
+    _check(name, getattr(load(), name)(
         _ptr(x), _ptr(WgT), _ptr(WuT), _ptr(Wd), _ptr(dy), T, d, f, tw.ref(), _ptr(ovf_rows), _ptr(n_ovf),
         _ptr(dx), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
 

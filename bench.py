@@ -578,8 +578,34 @@ def run_gpu_backward(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     K, Wm = args.steps, args.warmup
 
-    def stage_dx():
-        tl.ffn_hybrid_backward_dx(x, WgT, WuT, Wd, dy, tw, ovf_rows, n_ovf, dx, wsb, st)
+    def make_dx(tensor_cores):
+        return lambda: tl.ffn_hybrid_backward_dx(x, WgT, WuT, Wd, dy, tw, ovf_rows, n_ovf, dx, wsb, st,
+                                                 tensor_cores=tensor_cores)
+
+    def time_forms(make):
+        out = {}
+        for name, tc in (("cuda_cores", False), ("tensor_cores", True)):
+            fn = make(tc)
+            for _ in range(Wm):
+                flush.zero_()
+                fn()
+            ts = []
+            for _ in range(max(3, K // 4)):
+                flush.zero_()
+                a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a_ev.record(stream)
+                fn()
+                b_ev.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(a_ev.elapsed_time(b_ev))
+            out[name] = max_over_ranks(float(np.median(ts)), world)
+        return out
+
+    # the two forms of dx (per-token axpys on the CUDA cores, or the scattered
+    # dz, du through one tensor-core GEMM); the faster is the one the step uses
+    dx_forms = time_forms(make_dx)
+    dx_form = min(dx_forms, key=dx_forms.get)
+    stage_dx = make_dx(dx_form == "tensor_cores")
 
     def make_dw(tensor_cores):
         return lambda: tl.ffn_hybrid_backward_dw(x, dy, tw, n_ovf, dW[0], dW[1], dW[2], wsb,
@@ -588,23 +614,8 @@ def run_gpu_backward(args, world, rank, local):
     # the two forms of the weight gradients (per-unit sums on the CUDA cores, or
     # the dense scatter and GEMMs on the tensor cores), timed after a dx pass;
     # the faster is the one the step uses
-    dw_forms = {}
     stage_dx()
-    for name, tc in (("cuda_cores", False), ("tensor_cores", True)):
-        fn = make_dw(tc)
-        for _ in range(Wm):
-            flush.zero_()
-            fn()
-        ts = []
-        for _ in range(max(3, K // 4)):
-            flush.zero_()
-            a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a_ev.record(stream)
-            fn()
-            b_ev.record(stream)
-            torch.cuda.synchronize(dev)
-            ts.append(a_ev.elapsed_time(b_ev))
-        dw_forms[name] = max_over_ranks(float(np.median(ts)), world)
+    dw_forms = time_forms(make_dw)
     dw_form = min(dw_forms, key=dw_forms.get)
     stage_dw = make_dw(dw_form == "tensor_cores")
 
@@ -691,7 +702,7 @@ def run_gpu_backward(args, world, rank, local):
     nnz_ovf = int(counts[ovf_mask].sum())  # true counts: every active unit of an overflow row
     # CUDA-core work of the rows that fit (the overflow rows' dense branch runs
     # on the tensor cores: 12 n_ovf d f FLOPs, reported beside it)
-    flops_dx = 8.0 * d * nnz_fit  # u and dh dots, two axpys per stored unit
+    flops_dx = 8.0 * d * nnz_fit  # u and dh per stored unit (dh from the dense GEMM), two axpys
     flops_dw = 6.0 * d * nnz_fit  # three axpys per stored unit
     clocks = sampler.summary()
     peaks = load_peaks()
@@ -701,6 +712,10 @@ def run_gpu_backward(args, world, rank, local):
     work = {"backward_dx": flops_dx, "backward_dw": flops_dw}
     bound = {"backward_dx": "alu", "backward_dw": "alu"}
     peak_tf = {"backward_dx": fp32_peak / 1e12, "backward_dw": fp32_peak / 1e12}
+    if dx_form == "tensor_cores":  # one GEMM over all tokens, K = 4 f (values and remainders)
+        work["backward_dx"] = 8.0 * T * d * f
+        bound["backward_dx"] = "tensor"
+        peak_tf["backward_dx"] = peaks["bf16_tflops"]
     if dw_form == "tensor_cores":  # three GEMMs over all tokens (plus the overflow rows' ones)
         work["backward_dw"] = 6.0 * T * d * f
         bound["backward_dw"] = "tensor"
@@ -730,6 +745,8 @@ def run_gpu_backward(args, world, rank, local):
                      "peak_source": ("fp32 FMA lanes x 2 x max SM clock" if bound[dom] == "alu"
                                      else f"{peaks['source']} bf16 burst")},
         "stages_ms": {n: float(v) for n, v in zip(names, stage_ms)},
+        "dx_forms_ms": dx_forms,
+        "dx_form": dx_form,
         "weight_gradient_forms_ms": dw_forms,
         "weight_gradient_form": dw_form,
         "batch_stats": {"n_ovf": n_ovf_h, "nnz_fit_rows": nnz_fit, "nnz_overflow_rows": nnz_ovf,
@@ -738,9 +755,10 @@ def run_gpu_backward(args, world, rank, local):
         "speedup_vs_own_dense": dense_ms / step_ms,
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
-        # per step: the dh GEMM, dots and dx passes, two gathers, three dense-branch GEMMs; zeroing, count,
-        # scan, scatter, per-unit sums and three weight-gradient GEMMs
-        "gpu_launches": 16 * K,
+        # per step: the dh GEMM, the dots pass and the dx pass (tensor-core form: zeroing, scatter and the dx
+        # GEMM), two gathers and three dense-branch GEMMs; five launches of either weight-gradient form and
+        # the overflow rows' three weight-gradient GEMMs
+        "gpu_launches": (18 if dx_form == "tensor_cores" else 16) * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

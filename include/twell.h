@@ -372,6 +372,23 @@ twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* 
                                              float* dWd, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Tensor-core form of twell_ffn_hybrid_backward_dx (same arguments, same
+ * workspace; twell_ffn_hybrid_backward_dw or _dw_tc may follow it). The rows
+ * that fit still form u and their per-slot records on the CUDA cores, but
+ * their dx comes from one tcgen05 GEMM: their dz and du are scattered by
+ * token into dense rows [dz | du | dz_lo | du_lo] (bf16 value plus bf16
+ * remainder, zeros elsewhere) and multiplied by [Wg; Wu] read twice along K,
+ * the layout the overflow rows' dense branch uses. Pays where the rows hold
+ * many stored units (the GEMM's cost does not fall with density); the extra
+ * error is ~2^-16 of each term.
+ */
+twell_status twell_ffn_hybrid_backward_dx_tc(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
+                                             const uint16_t* Wd, const uint16_t* dy, int T, int d, int f,
+                                             const twell_t* tw, const int32_t* ovf_rows, const int32_t* n_ovf,
+                                             float* dx, void* workspace, size_t workspace_bytes,
+                                             int32_t* dev_status, void* stream);
+
+/*
  * Dense backward of the gated layer on the tensor cores, no sparsity: the
  * library's own baseline for twell_ffn_hybrid_backward. [z | u] = x [Wg | Wu]
  * (fp32), dh = dy Wd^T with dz = dh u [z > 0], du = dh ReLU(z), h = ReLU(z) u

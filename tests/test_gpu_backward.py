@@ -223,3 +223,68 @@ def test_tensor_core_weight_gradients(cfg):
         err = np.abs(got - ref[k])
         assert err.max() <= CONTRACT * rms, (k, float(err.max()), rms)
         assert np.all(err <= b[k] + TIGHT * rms), k
+
+
+def _forward_for_backward(L, cfg):
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.empty((T,), dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    return dev, tw, ovf_rows, n_ovf, st
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_tensor_core_dx(cfg):
+    """The tensor-core form of dx (dz, du of the rows that fit as bf16 value
+    plus remainder, one GEMM against [Wg; Wu]) against the oracle: within the
+    contract and within 2^-15 of the summed term magnitudes on top of the
+    tight check; the weight gradients that follow it are unchanged."""
+    L = synth.make_layer(cfg, seed=0)
+    dy_bits = make_dy(cfg.T, cfg.d, 7)
+    dev, tw, ovf_rows, n_ovf, st = _forward_for_backward(L, cfg)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    dy = tl.to_device_bf16(dy_bits)
+    dx = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    dW = [torch.full((f, d), float("nan"), dtype=torch.float32, device="cuda") for _ in range(3)]
+    wsb = torch.empty(tl.backward_workspace_bytes(T, d, f, W), dtype=torch.uint8, device="cuda")
+    tl.ffn_hybrid_backward_dx(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], dy, tw, ovf_rows, n_ovf, dx, wsb, st,
+                              tensor_cores=True)
+    tl.ffn_hybrid_backward_dw(dev["x"], dy, tw, n_ovf, dW[0], dW[1], dW[2], wsb)
+    assert tl.status_get(st) == 0
+    ref = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy_bits, cfg.tile, cfg.W)
+    n = int(n_ovf.item())
+    assert np.array_equal(ovf_rows[:n].cpu().numpy(), ref["ovf_rows"])
+    b = dense_branch_bounds(L, dy_bits, np.arange(T), rows=np.arange(T))
+    assert_grad_close(dx.double().cpu().numpy(), ref["dx"], "dx", b["dx"])
+    ovf = ref["ovf_rows"]
+    bw = dense_branch_bounds(L, dy_bits, ovf) if ovf.size else {}
+    for k, t in zip(("dWgT", "dWuT", "dWd"), dW):
+        assert_grad_close(t.double().cpu().numpy(), ref[k], k, bw.get(k))
+
+
+def test_full_size_tensor_core_dx():
+    """The tensor-core form of dx at the 0.5B size: sampled rows, overflow rows among them."""
+    cfg = synth.CONFIGS["0.5b"]
+    L = synth.make_layer(cfg, seed=0)
+    dy_bits = make_dy(cfg.T, cfg.d, 8)
+    dev, tw, ovf_rows, n_ovf, st = _forward_for_backward(L, cfg)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    dy = tl.to_device_bf16(dy_bits)
+    dx = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    wsb = torch.empty(tl.backward_workspace_bytes(T, d, f, W), dtype=torch.uint8, device="cuda")
+    tl.ffn_hybrid_backward_dx(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], dy, tw, ovf_rows, n_ovf, dx, wsb, st,
+                              tensor_cores=True)
+    assert tl.status_get(st) == 0
+    got = dx.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    ovf = ovf_rows[:int(n_ovf.item())].cpu().numpy()
+    rng = np.random.default_rng(9)
+    rows = np.union1d(np.sort(rng.choice(T, size=128, replace=False)), ovf[:32])
+    ref = O.hybrid_ffn_backward(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], dy_bits[rows], cfg.tile, cfg.W)
+    b = dense_branch_bounds(L, dy_bits, rows, rows=rows)
+    assert_grad_close(got[rows], ref["dx"], "dx", b["dx"])
