@@ -15,7 +15,6 @@
 #include "twell.h"
 #include "backward.cuh"
 #include "sparse_ffn.cuh"
-#include "staged_down.cuh"
 #include "umma_gemm.cuh"
 
 namespace {
@@ -353,93 +352,6 @@ twell_status dense_impl(const uint16_t* a_rows, int M, const int* M_dev, const u
 
 // Second half of the dense layer: out[row_map[i]] = h[i] Wd (row_map null: identity), h_buf
 // [M][f] bf16, or [M][2f] (h and its bf16 remainder) with split.
-// ------------------------------------------------------------------ staged down projection
-
-// Token-group size and workspace carve of the staged down projection. The
-// group size G (a multiple of the 15 consumer warps, 120 to 240) is the one whose units
-// (groups x 128-column slices) fill the last wave of a persistent grid best;
-// a smaller group re-reads Wd into shared memory more often, which the score
-// charges at about 8% for half the size.
-struct StagedPlan {
-  int G = 0, tpw = 0, ngroups = 0, nC = 0, nsl = 0;
-  size_t off_offs = 0, off_list = 0, bytes = 0;
-};
-
-StagedPlan staged_plan_for(int T, int d, int f, int W, int G) {
-  StagedPlan pl;
-  const int nT = f / 128;
-  pl.G = G;
-  pl.tpw = G / kStgWarps;
-  pl.ngroups = (T + G - 1) / G;
-  pl.nC = (nT + kStgTiles - 1) / kStgTiles;
-  pl.nsl = (d + kStgCols - 1) / kStgCols;
-  pl.off_offs = round_up(static_cast<size_t>(pl.ngroups) * G * 4, 256);
-  pl.off_list = pl.off_offs + round_up(static_cast<size_t>(pl.ngroups) * pl.nC * (G + 1) * 4, 256);
-  pl.bytes = pl.off_list + round_up(static_cast<size_t>(T) * nT * W * 4, 256);
-  return pl;
-}
-
-StagedPlan staged_plan(int T, int d, int f, int W, int sms) {
-  int best_g = kStgMaxG;
-  double best = -1.0;
-  const int nsl = (d + kStgCols - 1) / kStgCols;
-  for (int G = kStgMaxG; G >= kStgMaxG / 2; G -= kStgWarps) {
-    const long long units = static_cast<long long>((T + G - 1) / G) * nsl;
-    const long long waves = (units + sms - 1) / sms;
-    const double eff = static_cast<double>(units) / static_cast<double>(waves * sms);
-    const double score = eff * (1.0 - 0.08 * (kStgMaxG - G) / (kStgMaxG / 2));
-    if (score > best + 1e-9) {
-      best = score;
-      best_g = G;
-    }
-  }
-  return staged_plan_for(T, d, f, W, best_g);
-}
-
-// The workspace that covers every group size the plan may pick.
-size_t staged_bytes_bound(int T, int d, int f, int W) {
-  size_t b = 0;
-  for (int G = kStgMaxG; G >= kStgMaxG / 2; G -= kStgWarps) b = std::max(b, staged_plan_for(T, d, f, W, G).bytes);
-  return b;
-}
-
-twell_status staged_down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip, float* y,
-                              void* ws, int32_t* dev_status, cudaStream_t s, int sms) {
-  const StagedPlan pl = staged_plan(T, d, f, tw->W, sms);
-  if (pl.ngroups > 65535) return TWELL_ERR_SHAPE;  // the list kernel's grid has one row per token group
-  StagedParams p{};
-  p.counts = tw->counts;
-  p.idx = tw->idx;
-  p.vals = tw->vals;
-  p.row_ovf = tw->row_ovf;
-  p.y = y;
-  char* w = static_cast<char*>(ws);
-  p.pos_tok = reinterpret_cast<int*>(w);
-  p.offs = reinterpret_cast<int*>(w + pl.off_offs);
-  p.list = reinterpret_cast<uint32_t*>(w + pl.off_list);
-  p.T = T;
-  p.d = d;
-  p.f = f;
-  p.nT = f / 128;
-  p.W = tw->W;
-  p.G = pl.G;
-  p.tpw = pl.tpw;
-  p.ngroups = pl.ngroups;
-  p.nC = pl.nC;
-  p.nsl = pl.nsl;
-  p.skip_ovf = skip ? 1 : 0;
-  p.dev_status = dev_status;
-  CUtensorMap map;
-  if (!make_map_plain(&map, Wd, d, f, kStgCols, kStgRows)) return TWELL_ERR_CUDA;
-  TW_TRY(launch(staged_order_kernel, dim3(pl.ngroups), dim3(256), 0, s, p));
-  TW_TRY(launch(staged_lists_kernel, dim3(pl.nC, pl.ngroups), dim3(256), 0, s, p));
-  auto kern = staged_down_kernel;
-  TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStgSmemBytes)));
-  const int units = pl.ngroups * pl.nsl;
-  TW_TRY(launch(kern, dim3(std::min(units, sms)), dim3(kStgThreads), kStgSmemBytes, s, map, p));
-  return cuda_ok(cudaGetLastError());
-}
-
 twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, const uint16_t* Wd, int d, int f,
                              bool split, const int* row_map, float* y, int y_rows, int32_t* dev_status,
                              cudaStream_t s, int sms) {
@@ -594,28 +506,6 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
   return down_impl(Wd, T, d, f, tw, skip_overflow_rows, y, dev_status, static_cast<cudaStream_t>(stream), sms);
-}
-
-size_t twell_sparse_down_staged_workspace_bytes(int T, int d, int f, int W) {
-  if (T <= 0 || d <= 0 || f < 128 || W <= 0) return 0;
-  return staged_bytes_bound(T, d, f, W);
-}
-
-twell_status twell_sparse_down_staged(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
-                                      int skip_overflow_rows, float* y, void* workspace, size_t workspace_bytes,
-                                      int32_t* dev_status, void* stream) {
-  TW_TRY(check_shape(T, d, f));
-  if (d < kStgCols) return TWELL_ERR_SHAPE;
-  TW_TRY(check_tw(tw, T, f));
-  if (T == 0) return TWELL_OK;
-  TW_TRY(check_ptrs({Wd, y, dev_status}));
-  if (workspace == nullptr || workspace_bytes < twell_sparse_down_staged_workspace_bytes(T, d, f, tw->W))
-    return TWELL_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
-  int dev, sms;
-  TW_TRY(current_device(&dev, &sms));
-  return staged_down_impl(Wd, T, d, f, tw, skip_overflow_rows, y, workspace, dev_status,
-                          static_cast<cudaStream_t>(stream), sms);
 }
 
 twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
@@ -1147,19 +1037,22 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // == TWELL_NOALLOC_S
 // obtained once per device with cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-void* g_noalloc_ptr[kMaxDevices];
-std::once_flag g_noalloc_once[kMaxDevices];
-cudaError_t g_noalloc_err[kMaxDevices];
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
 
-// Device address of the scratch for the current device `dev`, looked up on the
-// first call made with that device current.
+// Device address of the scratch for the current device `dev`. It is looked up
+// with that device current on the first call that succeeds in doing so and
+// kept from then on; a failed lookup is not kept, so the next call tries
+// again. (Two threads making their first calls at once may both look it up;
+// they get the same address.)
 void* noalloc_scratch(int dev) {
-  std::call_once(g_noalloc_once[dev], [dev] {
-    void* p = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    g_noalloc_ptr[dev] = (g_noalloc_err[dev] == cudaSuccess) ? p : nullptr;
-  });
-  return g_noalloc_ptr[dev];
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p != nullptr) return p;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  return p;
 }
 
 }  // namespace
@@ -1177,9 +1070,6 @@ extern "C" twell_status twell_ffn_hybrid_forward_noalloc(const uint16_t* x, cons
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
   void* ws = noalloc_scratch(dev);
-  if (ws == nullptr) {
-    (void)cudaGetLastError();
-    return TWELL_ERR_CUDA;
-  }
+  if (ws == nullptr) return TWELL_ERR_CUDA;
   return twell_ffn_hybrid_forward(x, WgT, WuT, Wd, T, d, f, tw, y, ovf_rows, n_ovf, ws, need, dev_status, stream);
 }

@@ -34,8 +34,7 @@ EXPORTED = (
     "twell_column_activity", "twell_compact_columns", "twell_gather_rows",
     "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward", "twell_ffn_hybrid_backward_dx",
     "twell_ffn_hybrid_backward_dw", "twell_dense_backward_workspace_bytes", "twell_dense_ffn_backward",
-    "twell_ffn_hybrid_backward_dw_tc", "twell_sparse_down_staged", "twell_sparse_down_staged_workspace_bytes",
-    "twell_ffn_hybrid_backward_dx_tc",
+    "twell_ffn_hybrid_backward_dw_tc", "twell_ffn_hybrid_backward_dx_tc",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -80,8 +79,6 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_route": ([tw, vp, vp, vp], i32),
         "twell_gate_up_pack": ([vp, vp, vp, i32, i32, i32, tw, vp, vp], i32),
         "twell_sparse_down": ([vp, i32, i32, i32, tw, i32, vp, vp, vp], i32),
-        "twell_sparse_down_staged": ([vp, i32, i32, i32, tw, i32, vp, vp, sz, vp, vp], i32),
-        "twell_sparse_down_staged_workspace_bytes": ([i32, i32, i32, i32], sz),
         "twell_ffn_hybrid_forward_tc_up": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_hybrid_workspace_bytes": ([i32, i32, i32], sz),
         "twell_dense_rows_forward": ([vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp], i32),
@@ -228,22 +225,6 @@ def sparse_down(Wd, tw: Twell, y, skip_overflow_rows: bool, dev_status, stream=N
     _bf16("y", y, (T, d))
     _check("twell_sparse_down", load().twell_sparse_down(_ptr(Wd), T, d, f, tw.ref(), int(bool(skip_overflow_rows)),
                                                          _ptr(y), _ptr(dev_status), _stream(stream)))
-
-
-def sparse_down_staged(Wd, tw: Twell, y, skip_overflow_rows: bool, workspace, dev_status, stream=None) -> None:
-    """The down projection staged through shared memory (d >= 128); workspace of
-    sparse_down_staged_workspace_bytes(T, d, f, W) bytes."""
-    f, d = Wd.shape
-    T = tw.T
-    _bf16("Wd", Wd, (f, d))
-    _bf16("y", y, (T, d))
-    _check("twell_sparse_down_staged", load().twell_sparse_down_staged(
-        _ptr(Wd), T, d, f, tw.ref(), int(bool(skip_overflow_rows)), _ptr(y), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
-
-
-def sparse_down_staged_workspace_bytes(T: int, d: int, f: int, W: int) -> int:
-    return int(load().twell_sparse_down_staged_workspace_bytes(T, d, f, W))
 
 
 def ffn_hybrid_forward_tc_up(x, WgT, WuT, Wd, tw: Twell, y, ovf_rows, n_ovf, workspace, dev_status,

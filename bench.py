@@ -122,9 +122,10 @@ class ClockSampler:
 # ---------------------------------------------------------------- helpers
 
 
-# Sources of the forward kernels whose DRAM traffic profiles/traffic.json records
-# (the backward kernels live in their own header and do not change them).
-FORWARD_SOURCES = ("ptx.cuh", "sparse_ffn.cuh", "twell_api.cu", "umma_gemm.cuh")
+# Device code of the forward kernels whose DRAM traffic profiles/traffic.json
+# records (host code and the backward kernels, in other files, do not change
+# them): a record taken on other sources is not reported.
+FORWARD_SOURCES = ("ptx.cuh", "sparse_ffn.cuh", "umma_gemm.cuh")
 
 
 def kernel_source_hash() -> str:
@@ -148,6 +149,43 @@ def measured_traffic(kernel: str, workload: str):
     if t.get("source_hash") != kernel_source_hash() or t.get("workload") != workload:
         return None
     return t.get("kernels", {}).get(kernel)
+
+
+UNIT_BYTES = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+
+
+def record_traffic(csv_path: str, workload: str, kernels: list, command: str) -> dict:
+    """profiles/traffic.json from an ncu raw-page CSV (`ncu -i rep --page raw
+    --csv`): per bench stage, the mean over its captured launches of
+    dram__bytes_read.sum + dram__bytes_write.sum, keyed to the current device
+    sources. kernels: "stage=substring" pairs naming which captured kernel is
+    which stage."""
+    import csv
+
+    with open(csv_path, newline="") as fh:
+        rows = list(csv.reader(fh))
+    head = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    cols, units = rows[head], rows[head + 1]
+    kn = cols.index("Kernel Name")
+    rd, wr = cols.index("dram__bytes_read.sum"), cols.index("dram__bytes_write.sum")
+
+    def val(r, c):
+        return float(r[c].replace(",", "")) * UNIT_BYTES.get(units[c], 1.0)
+
+    out = {}
+    for pair in kernels:
+        stage, sub = pair.split("=", 1)
+        got = [val(r, rd) + val(r, wr) for r in rows[head + 2:] if len(r) > kn and sub in r[kn]]
+        if not got:
+            raise SystemExit(f"no captured launch of {sub!r} in {csv_path}")
+        out[stage] = float(np.mean(got))
+    rec = {"source_hash": kernel_source_hash(), "workload": workload, "command": command,
+           "note": "dram__bytes_read.sum + dram__bytes_write.sum per launch (mean over the captured launches)",
+           "kernels": out}
+    with open(os.path.join(ROOT, "profiles", "traffic.json"), "w") as fh:
+        json.dump(rec, fh, indent=1)
+        fh.write("\n")
+    return rec
 
 
 def dist_setup(args):
@@ -299,17 +337,8 @@ def run_gpu(args, world, rank, local):
     # The two forms of the hybrid forward: "gate" packs ReLU(z) and runs the
     # fused sparse up+down step; "tc_up" forms u on the tensor cores with the
     # gate and packs h, leaving only the down projection sparse.
-    # --down staged: the down projection of the tc_up and non-gated forms
-    # through the shared-memory-staged alternative (its lists in a workspace of
-    # its own), to measure it against the per-token kernel the library uses
-    ws_staged = (torch.empty(tl.sparse_down_staged_workspace_bytes(T, d, f, W), dtype=torch.uint8, device=dev)
-                 if args.down == "staged" else None)
-
     def down():
-        if ws_staged is not None:
-            tl.sparse_down_staged(Wd, tw, y, True, ws_staged, st)
-        else:
-            tl.sparse_down(Wd, tw, y, True, st)
+        tl.sparse_down(Wd, tw, y, True, st)
 
     def stage_fns(variant):
         if variant == "relu":  # the non-gated layer ReLU(x W1) W2 with W1 = Wg, W2 = Wd
@@ -345,7 +374,8 @@ def run_gpu(args, world, rank, local):
             torch.cuda.synchronize(dev)
         barrier(world)
         per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)] for k in range(K)])
-        return max_over_ranks(float(per.sum(axis=1).mean()), world), per.mean(axis=0)
+        # median step (and median per stage) over the K timed steps
+        return max_over_ranks(float(np.median(per.sum(axis=1))), world), np.median(per, axis=0)
 
     layer = "relu" if args.layer == "relu" else "gated"
     if layer == "relu":
@@ -391,7 +421,7 @@ def run_gpu(args, world, rank, local):
         dense()
         dense_ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
-    dense_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dense_ev])), world)
+    dense_ms = max_over_ranks(float(np.median([a.elapsed_time(b) for a, b in dense_ev])), world)
 
     # End to end through the C ABI with host buffers: every step copies its x
     # from pinned host memory, runs the hybrid forward and copies y back to
@@ -528,13 +558,11 @@ def run_gpu(args, world, rank, local):
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4,
                 "pipelined": "copy-in, compute and copy-out on three streams, two buffer sets",
-                "path": "the library's hybrid forward of the chosen form (per-token down projection)",
+                "path": "the library's hybrid forward of the chosen form",
                 "l2": "not flushed: each step touches ~0.26 GB, above the 126 MB L2"},
         # per step: zeroing, gate (or gate+up) GEMM, routing, sparse step, row gather, two dense-branch GEMMs
-        # (the staged down projection adds its two planning kernels)
-        "gpu_launches": (9 if ws_staged is not None and chosen != "gate" else 7) * K,
-        "down_projection": ("fused up+down per token" if chosen == "gate" else
-                            "staged through shared memory" if ws_staged is not None else "per token"),
+        "gpu_launches": 7 * K,
+        "down_projection": "fused up+down per token" if chosen == "gate" else "per token",
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -641,8 +669,8 @@ def run_gpu_backward(args, world, rank, local):
         torch.cuda.synchronize(dev)
     barrier(world)
     per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(2)] for k in range(K)])
-    stage_ms = per.mean(axis=0)
-    step_ms = max_over_ranks(float(per.sum(axis=1).mean()), world)
+    stage_ms = np.median(per, axis=0)
+    step_ms = max_over_ranks(float(np.median(per.sum(axis=1))), world)
 
     # the library's dense backward at the same shape (tensor cores, bf16 dz/du/h)
     wsd = torch.empty(tl.dense_backward_workspace_bytes(T, d, f), dtype=torch.uint8, device=dev)
@@ -663,7 +691,7 @@ def run_gpu_backward(args, world, rank, local):
         dense_bwd()
         dense_ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
-    dense_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in dense_ev])), world)
+    dense_ms = max_over_ranks(float(np.median([a.elapsed_time(b) for a, b in dense_ev])), world)
     del wsd, dxd, dWdn
 
     # e2e through the C ABI: dy from pinned host memory in, dx and the weight gradients out
@@ -690,7 +718,7 @@ def run_gpu_backward(args, world, rank, local):
         e2e_step()
         e2e_ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in e2e_ev])), world)
+    e2e_ms = max_over_ranks(float(np.median([a.elapsed_time(b) for a, b in e2e_ev])), world)
     status = tl.status_get(st)
     if status != 0:
         raise RuntimeError(f"device status {status} ({tl.status_str(status)})")
@@ -906,7 +934,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="twell", choices=["twell", "reference"])
-    ap.add_argument("--config", default="0.5b", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--config", default="2b", choices=sorted(synth.CONFIGS),
+                    help="layer shape (default: the 2B-like hybrid layer, the largest that fits one GPU)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-sample", type=int, default=12288)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -916,9 +945,6 @@ def main(argv=None):
                     help="gated: (ReLU(x Wg) * x Wu) Wd; relu: the non-gated ReLU(x W1) W2")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"],
                     help="forward (the default) or the backward pass through the hybrid format")
-    ap.add_argument("--down", default="per_token", choices=["per_token", "staged"],
-                    help="down projection of the tc_up and non-gated forms (the library's hybrid forwards use "
-                         "per_token)")
     ap.add_argument("--compact", action="store_true",
                     help="drop the hidden units the batch never activates before timing")
     ap.add_argument("--sweep", action="store_true", help="density x batch sweep, one JSON line per point")
@@ -928,7 +954,16 @@ def main(argv=None):
     ap.add_argument("--sweep-w", type=int, default=0,
                     help="ELL width for every sweep point (0: the smallest that stores the pure sparse path); "
                          "a fixed W such as 32 measures the hybrid route, dense branch included")
+    ap.add_argument("--record-traffic", default="",
+                    help="write profiles/traffic.json from this ncu raw-page CSV and exit")
+    ap.add_argument("--record-kernel", action="append", default=[],
+                    help="stage=kernel-name substring, for --record-traffic (repeatable)")
+    ap.add_argument("--record-command", default="", help="the ncu command the CSV came from")
     args = ap.parse_args(argv)
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic, args.config, args.record_kernel,
+                                        args.record_command)))
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.sweep:

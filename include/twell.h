@@ -111,8 +111,13 @@ twell_status twell_sparse_ffn(const uint16_t* x, const uint16_t* WuT, const uint
 
 /*
  * Whole non-hybrid forward: twell_gate_pack, then twell_sparse_ffn without
- * skipping. If any row overflows, dev_status becomes TWELL_ERR_OVERFLOW and
- * the y of the overflowing rows is undefined (other rows are correct).
+ * skipping (source: intellectnews.ru "Sakana AI и NVIDIA ... TwELL", section
+ * "Слитые CUDA-ядра для инференса и гибрид для обучения": at inference the
+ * packed gate output feeds fused kernels that do the rest of the FFN for the
+ * stored units only; section "Формат TwELL вместо классической
+ * sparse-упаковки": the pack is formed at the end of the gate's own pass).
+ * If any row overflows, dev_status becomes TWELL_ERR_OVERFLOW and the y of
+ * the overflowing rows is undefined (other rows are correct).
  */
 twell_status twell_ffn_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
@@ -136,33 +141,6 @@ twell_status twell_gate_up_pack(const uint16_t* x, const uint16_t* WgT, const ui
  */
 twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
                                int skip_overflow_rows, float* y, int32_t* dev_status, void* stream);
-
-/*
- * The same down projection, staged through shared memory (same source; the
- * staging is this library's, not the pages'). An alternative to
- * twell_sparse_down, which the hybrid forwards use: on B200 at the 0.5B-2B
- * layer shapes this form is 1.7-3.4x slower (its per-slot instruction count,
- * not memory, bounds it). The tokens
- * are cut into groups of G (120..240, chosen from T, d and the SM count);
- * per group and per 128-column slice of d, Wd is copied into shared memory
- * in chunks of 256 rows and each stored slot of the group's tokens reads its
- * row piece there instead of gathering the whole row from L2. y as for
- * twell_sparse_down (fp32 sums in another order); rows skipped by
- * skip_overflow_rows are left untouched.
- * Requires d >= 128 and at most 65535 token groups (T up to about 7.8 M;
- * TWELL_ERR_SHAPE otherwise). workspace: device memory of
- * at least twell_sparse_down_staged_workspace_bytes(T, d, f, W) bytes,
- * 16-byte aligned, caller-owned, overwritten (the per-group token order, the
- * per-chunk slot lists). A stored index outside its own column tile raises
- * TWELL_ERR_INDEX and adds nothing. Three kernel launches.
- */
-twell_status twell_sparse_down_staged(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
-                                      int skip_overflow_rows, float* y, void* workspace, size_t workspace_bytes,
-                                      int32_t* dev_status, void* stream);
-
-/* Workspace bytes of twell_sparse_down_staged (about T * f * W / 32, the
- * slot lists at full ELL width, plus small tables). */
-size_t twell_sparse_down_staged_workspace_bytes(int T, int d, int f, int W);
 
 /*
  * Hybrid forward of the tensor-core-up variant = twell_gate_up_pack,
@@ -209,9 +187,13 @@ twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, co
 
 /*
  * Whole hybrid forward = twell_gate_pack, twell_route, twell_sparse_ffn with
- * overflowing rows skipped, and twell_dense_rows_forward on ovf_rows. Every
- * row of y is written. `workspace` holds the gathered overflow rows and their
- * hidden activations.
+ * overflowing rows skipped, and twell_dense_rows_forward on ovf_rows (source:
+ * intellectnews.ru "Sakana AI и NVIDIA ... TwELL", section "Слитые CUDA-ядра
+ * для инференса и гибрид для обучения": rows whose active units do not fit
+ * the sparse format are handled in dense form, the rest sparsely; the pages
+ * describe this split for training and this library applies the same rule to
+ * the forward pass). Every row of y is written. `workspace` holds the gathered
+ * overflow rows and their hidden activations.
  */
 twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                       const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
@@ -236,7 +218,11 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
  *     TWELL_NOALLOC_SCRATCH_BYTES, i.e. roughly T * (2d + 4f) bytes; larger
  *     calls return TWELL_ERR_WORKSPACE and launch nothing.
  *   - The first call on a device looks up the scratch address for that device
- *     (with it current); make that first call before any stream capture.
+ *     (with it current) and keeps it; make that first call before any stream
+ *     capture. A lookup that fails is not kept (the call returns
+ *     TWELL_ERR_CUDA and the next call tries again). The kept address belongs
+ *     to the device's current context: after cudaDeviceReset the library must
+ *     not be called again in that process.
  *   - Every call on a device shares the one scratch array, which keeps the last
  *     call's contents (nothing in it needs to start at zero). Calls whose work
  *     overlaps on the GPU -- on different streams, or from several host
@@ -443,6 +429,10 @@ twell_status twell_gather_rows(const uint16_t* W, int f, int d, const int32_t* c
 /*
  * TwELL -> dense bf16 g[T][f]: zeros everywhere except the stored slots
  * (slots below min(count, W); overflowing rows unpack only what was stored).
+ * The inverse of the packing of intellectnews.ru "Sakana AI и NVIDIA ...
+ * TwELL", section "Формат TwELL вместо классической sparse-упаковки" (per row
+ * and column tile, the nonzero values with their column indices); for tests
+ * and for callers that need the dense hidden activations.
  */
 twell_status twell_unpack(const twell_t* tw, uint16_t* g_dense, int32_t* dev_status, void* stream);
 

@@ -138,28 +138,3 @@ def test_backward_argument_errors(lib):
                                         FAKE, None) == tl.TWELL_ERR_WORKSPACE
     assert lib.twell_relu_ffn_hybrid_forward(FAKE, FAKE, None, 64, 128, 512, ctypes.byref(tw), FAKE, FAKE, FAKE, FAKE,
                                              1 << 30, FAKE, None) == tl.TWELL_ERR_NULL
-
-
-def test_staged_down_argument_errors_and_workspace(lib):
-    T, d, f, W = 1000, 1536, 4096, 32
-    need = lib.twell_sparse_down_staged_workspace_bytes(T, d, f, W)
-    nT = f // 128
-    # the slot lists at full ELL width, plus the per-group tables
-    assert need >= T * nT * W * 4 and need % 256 == 0
-    assert need <= T * nT * W * 4 + 64 * 1024 + (nT // 2) * (T + T // 120 + 260) * 4 + 3 * 256
-    assert lib.twell_sparse_down_staged_workspace_bytes(0, d, f, W) == 0
-    tw = tw_desc(T, f, W)
-    st = lib.twell_sparse_down_staged
-
-    def call(d_=d, y=FAKE, ws=FAKE, wsb=need, desc=tw):
-        return st(FAKE, T, d_, f, ctypes.byref(desc), 1, y, ws, wsb, FAKE, None)
-
-    assert call(d_=64) == tl.TWELL_ERR_SHAPE          # a 128-column slice at least
-    assert call(d_=100) == tl.TWELL_ERR_SHAPE
-    assert call(desc=tw_desc(T + 1, f, W)) == tl.TWELL_ERR_SHAPE
-    assert call(y=None) == tl.TWELL_ERR_NULL
-    assert call(ws=None) == tl.TWELL_ERR_WORKSPACE
-    assert call(wsb=need - 1) == tl.TWELL_ERR_WORKSPACE
-    assert call(ws=MIS) == tl.TWELL_ERR_ALIGN
-    z = tw_desc(0, f, W)
-    assert st(None, 0, d, f, ctypes.byref(z), 1, None, None, 0, None, None) == tl.TWELL_OK

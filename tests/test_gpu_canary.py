@@ -108,19 +108,3 @@ def test_compaction_stays_inside_its_outputs():
     assert tl.status_get(st) == 0
     for k, v in (("bits", bits), ("col_map", col_map), ("f_live", f_live), ("rows", out)):
         v.check(k)
-
-
-def test_staged_down_stays_inside_its_outputs():
-    cfg = next(c for c in SMALL if c.name == "heavy")
-    L = synth.make_layer(cfg, seed=0)
-    dev = upload(L)
-    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
-    tw = tl.Twell(T, f, W)
-    st = tl.new_status()
-    tl.gate_up_pack(dev["x"], dev["WgT"], dev["WuT"], tw, st)
-    y = Guarded((T, d), torch.float32)
-    ws = Guarded((tl.sparse_down_staged_workspace_bytes(T, d, f, W),), torch.uint8)
-    tl.sparse_down_staged(dev["Wd"], tw, y.t, True, ws.t, st)
-    assert tl.status_get(st) == 0
-    y.check("staged down: y")
-    ws.check("staged down: workspace")

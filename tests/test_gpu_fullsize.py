@@ -10,7 +10,7 @@ import torch
 from activation_sparse_gated_gemm_b200 import synth
 from activation_sparse_gated_gemm_b200 import twell as tl
 from oracle import twell_oracle as O
-from tests.gpu_helpers import assert_twell_equal, assert_within_stored_value_bound, assert_y_close, upload
+from tests.gpu_helpers import assert_twell_equal, assert_within_stored_value_bound, assert_y_close, upload, y_to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -72,3 +72,41 @@ def test_full_size_hybrid_forward(name):
     y_ref = np.concatenate([y_keep, O.gated_ffn(L["x"][ovf], L["WgT"], L["WuT"], L["Wd"])])
     assert_y_close(yg[rows], y_ref)
     assert_within_stored_value_bound(yg[keep], L, keep)
+
+
+@pytest.mark.parametrize("name", ["0.5b", "1.5b", "2b"])
+def test_full_size_tensor_core_up_hybrid_forward(name):
+    """The tensor-core-up hybrid forward at the full layer sizes, as bench.py
+    times it: routing over every row, y on sampled rows that fit and on
+    overflow rows."""
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    cfg = synth.CONFIGS[name]
+    L = synth.make_layer(cfg, seed=0)
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward_tc_up(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    assert tl.status_get(st) == 0
+    yg = y_to_f64(y)
+    assert np.isfinite(yg).all()
+    row_ovf = tw.row_ovf.cpu().numpy()
+    n = int(n_ovf.item())
+    ovf = ovf_rows[:n].cpu().numpy()
+    assert np.array_equal(ovf, np.nonzero(row_ovf)[0])
+    rng = np.random.default_rng(3)
+    sample = np.sort(rng.choice(T, size=256, replace=False))
+    keep = sample[row_ovf[sample] == 0]
+    x = O.bf16_bits_to_f64(L["x"][keep])
+    want = O.twell_pack_hidden(x @ O.bf16_bits_to_f64(L["WgT"]).T, x @ O.bf16_bits_to_f64(L["WuT"]).T,
+                               cfg.tile, W)
+    assert np.array_equal(want["row_ovf"], np.zeros(len(keep), np.uint8))
+    y_keep = O.sparse_down_from_twell(want, L["Wd"])
+    rows = np.concatenate([keep, ovf[:64]])
+    y_ref = np.concatenate([y_keep, O.gated_ffn(L["x"][ovf[:64]], L["WgT"], L["WuT"], L["Wd"])])
+    assert_y_close(yg[rows], y_ref)
