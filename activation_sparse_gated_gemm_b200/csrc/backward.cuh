@@ -317,6 +317,49 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dx_kernel(const BwdParams p
 // ---------------------------------------------------------------- by column
 
 // The stored slots of one pass, as the column sort sees them.
+// The records of the rows that fit from dense u = x . Wu^T and dh = dy . Wd^T
+// ([rows][f] fp32 each, from two tensor-core GEMMs) instead of a dot pass per
+// stored slot: one thread per (row, tile) reads its stored slots (j, g) and
+// writes {h = g u_j, du = dh_j g, dz = dh_j u_j, t}. A stored index outside
+// [0, f) raises TWELL_ERR_INDEX and leaves its record unwritten, as the dot
+// pass does.
+__global__ void __launch_bounds__(256) bwd_records_kernel(const BwdParams p, const float* __restrict__ u) {
+  griddep_launch_dependents();
+  griddep_wait();
+  bool bad = false;
+  const long long pairs = static_cast<long long>(p.rows) * p.nT;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < pairs;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / p.nT);
+    if (p.row_ovf[t]) continue;
+    const int n = min(max(static_cast<int>(p.counts[i]), 0), p.W);
+    const size_t base = static_cast<size_t>(i) * p.W;
+    const float* urow = u + static_cast<size_t>(t) * p.f;
+    const float* dhrow = p.dh + static_cast<size_t>(t) * p.f;
+    for (int k = 0; k < n; k += 8) {
+      // 8 slots per 16-byte load; k + 8 <= W since W is a multiple of 8
+      const uint4 iv = ldg_nc_v4(p.idx + base + k);
+      const uint4 vv = ldg_nc_v4(p.vals + base + k);
+      const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
+      const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (k + e < n) {
+          const int j = static_cast<int16_t>((e & 1) ? (iw[e >> 1] >> 16) : (iw[e >> 1] & 0xffffu));
+          const float g = __uint_as_float((e & 1) ? (vw[e >> 1] & 0xffff0000u) : (vw[e >> 1] << 16));
+          if (j < 0 || j >= p.f) {
+            bad = true;
+            continue;
+          }
+          const float uj = __ldg(urow + j), dh = __ldg(dhrow + j);
+          p.s_rec[base + k + e] = make_float4(g * uj, dh * g, dh * uj, __int_as_float(t));
+        }
+      }
+    }
+  }
+  if (bad) raise_status(p.dev_status, kDevIndex);
+}
+
 struct SlotSource {
   const int16_t* counts;
   const int16_t* idx;

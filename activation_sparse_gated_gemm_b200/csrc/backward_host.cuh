@@ -128,7 +128,20 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   p0.dx = dx;
   p0.s_rec = w.rec;
   p0.dev_status = dev_status;
-  TW_TRY(launch_bwd_token(p0, sms, s, !tc_dx));
+  if (tc_dx) {
+    // 1a. the records from dense u = x Wu^T (a second tensor-core GEMM, into the
+    // idle half of the [z | u] region) and dh, in place of the per-slot dot
+    // pass that gathers a Wu row for every stored slot
+    float* ubuf = w.zu + static_cast<size_t>(T) * f;
+    if (dh_tiles < sms) TW_TRY(zero_async(s, sms, ubuf, static_cast<size_t>(T) * f * sizeof(float)));
+    TW_TRY(f32_gemm_impl(x, T, WuT, f, d, ubuf, f, dev_status, s, sms));
+    const long long pairs = static_cast<long long>(T) * nT;
+    const int rb = static_cast<int>(std::min<long long>((pairs + 255) / 256, 8LL * sms));
+    TW_TRY(launch(bwd_records_kernel, dim3(std::max(rb, 1)), dim3(256), 0, s, p0, static_cast<const float*>(ubuf)));
+    TW_TRY(cuda_ok(cudaGetLastError()));
+  } else {
+    TW_TRY(launch_bwd_token(p0, sms, s, true));
+  }
   if (tc_dx) {
     // 1b. dx of every token = [dz | du | dz_lo | du_lo] [Wg; Wu; Wg; Wu]^T on
     // the tensor cores, the rows that fit scattered token-major into the
@@ -205,6 +218,7 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   q3.row_map = ovf_rows;
   q3.out_rows = T;
   q3.k_splits_max = 32;  // the gather zeroed these dx rows
+  q3.split_waves = 1;
   q3.dev_status = dev_status;
   return launch_gemm<kModeDown>(ma2, mgT, muT, q3, sms, s);
 }

@@ -311,6 +311,110 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
   if (__any_sync(0xffffffffu, bad_index) && lane == 0) raise_status(p.dev_status, kDevIndex);
 }
 
+// The sparse step of a batch of at most 8 tokens (d a multiple of 256): one
+// warp per stored slot, so that a token's few slots are all in flight at once
+// instead of queueing behind one another in the warps of its column tiles.
+// Block (b, t) takes slots b*8 + warp, stepping by gridDim.x * 8, of token t
+// (numbered across its tiles by a prefix of the stored counts); a warp loads
+// the slot's Wd row (and, for the gate form, its WuT row, u = x_t . Wu[:, j]
+// and h = g u), adds h Wd[j, :] into the block's copy of y_t in shared memory,
+// and the block adds that copy into y (which holds zeros in the rows written).
+constexpr int kSmallSparseWarps = 8;
+constexpr int kSmallSparseMaxTiles = 256;  // f <= 32767
+
+template <int NCH, bool DOWN_ONLY>
+__global__ void __launch_bounds__(kSmallSparseWarps * 32) sparse_small_kernel(const SparseParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ int pre[kSmallSparseMaxTiles + 1];
+  __shared__ float ys[NCH * 256];  // y_t, element (i*32 + l)*8 + e at i*256 + e*32 + l
+  __shared__ uint4 xs[DOWN_ONLY ? 1 : NCH * 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.y;
+  if (p.skip_ovf && p.row_ovf[t]) return;
+  bool overflow = false, bad_index = false;
+  if (warp == 0) {
+    int run = 0;
+    for (int cb = 0; cb < p.nT; cb += 32) {
+      const int c = cb + lane;
+      int n = 0;
+      if (c < p.nT) {
+        const int cnt = p.counts[static_cast<size_t>(t) * p.nT + c];
+        if (cnt > p.W) overflow = true;
+        n = min(max(cnt, 0), p.W);
+      }
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (c < p.nT) pre[c] = run + incl - n;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) pre[p.nT] = run;
+    if (__any_sync(0xffffffffu, overflow) && lane == 0 && !p.skip_ovf) raise_status(p.dev_status, kDevOverflow);
+  }
+  __syncthreads();
+  const int total = pre[p.nT];
+  if (blockIdx.x * kSmallSparseWarps >= total) return;  // no slot for this block
+  for (int e = threadIdx.x; e < NCH * 256; e += blockDim.x) ys[e] = 0.0f;
+  if (!DOWN_ONLY)
+    for (int e = threadIdx.x; e < NCH * 32; e += blockDim.x)
+      xs[e] = ldg_nc_v4(p.x + static_cast<size_t>(t) * p.d + e * 8);
+  __syncthreads();
+  const int stride = gridDim.x * kSmallSparseWarps;
+#pragma unroll 1
+  for (int s = blockIdx.x * kSmallSparseWarps + warp; s < total; s += stride) {
+    // the tile holding slot s: the last c with pre[c] <= s
+    int lo = 0, hi = p.nT - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= s) lo = mid; else hi = mid - 1;
+    }
+    const size_t at = (static_cast<size_t>(t) * p.nT + lo) * p.W + (s - pre[lo]);
+    const int j = p.idx[at];
+    if (j < 0 || j >= p.f) {
+      bad_index = true;
+      continue;
+    }
+    const uint16_t gb = p.vals[at];
+    uint4 wd[NCH];
+    load_row<NCH>(wd, p.Wd + static_cast<size_t>(j) * p.d, lane, p.d);
+    float h = __uint_as_float(static_cast<uint32_t>(gb) << 16);
+    if (!DOWN_ONLY) {
+      uint4 wu[NCH];
+      load_row<NCH>(wu, p.WuT + static_cast<size_t>(j) * p.d, lane, p.d);
+      float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) mixdot8(xs[i * 32 + lane], wu[i], a0, a1);
+      float u = a0 + a1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+      h *= u;
+    }
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const uint32_t w4[4] = {wd[i].x, wd[i].y, wd[i].z, wd[i].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float w = (e & 1) ? bf16hi(w4[e >> 1]) : bf16lo(w4[e >> 1]);
+        atomicAdd(&ys[i * 256 + e * 32 + lane], h * w);
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, bad_index) && lane == 0) raise_status(p.dev_status, kDevIndex);
+  __syncthreads();
+  // y_t += the block's copy, four columns per thread and step
+  float* yt = p.y + static_cast<size_t>(t) * p.d;
+  for (int q = threadIdx.x; q < NCH * 64; q += blockDim.x) {
+    const int k0 = q * 4;                    // columns k0..k0+3
+    const int i = k0 >> 8, l = (k0 >> 3) & 31, e0 = k0 & 7;
+    red_add_v4(yt + k0, ys[i * 256 + (e0 + 0) * 32 + l], ys[i * 256 + (e0 + 1) * 32 + l],
+               ys[i * 256 + (e0 + 2) * 32 + l], ys[i * 256 + (e0 + 3) * 32 + l]);
+  }
+}
+
 // y[t, :] = 0 for the rows the sparse step will write (all rows, or those
 // without the overflow flag when overflow rows are skipped).
 __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf, int skip_ovf) {
@@ -334,11 +438,24 @@ __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf,
 // With xo given (small batches), the same block then gathers the listed rows
 // of x into xo and zeroes them in y_zero, which saves the separate gather
 // launch of the dense branch.
-__global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf,
+//
+// With counts given (the batches of at most 8 tokens, whose pack writes no
+// flags), the block first sets row_ovf[t] = (some tile of row t counts more
+// than W nonzeros) for every row.
+__global__ void __launch_bounds__(1024) route_kernel(uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf,
                                                      const uint16_t* x = nullptr, int d = 0, uint16_t* xo = nullptr,
-                                                     float* y_zero = nullptr) {
+                                                     float* y_zero = nullptr, const int16_t* counts = nullptr,
+                                                     int nT = 0, int W = 0) {
   griddep_launch_dependents();
   griddep_wait();
+  if (counts != nullptr) {
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+      bool o = false;
+      for (int c = 0; c < nT; ++c) o |= counts[static_cast<size_t>(t) * nT + c] > W;
+      row_ovf[t] = o ? 1 : 0;
+    }
+    __syncthreads();
+  }
   __shared__ int warp_off[32];
   __shared__ int total_s;
   const int lane = threadIdx.x & 31;
@@ -460,6 +577,124 @@ __global__ void __launch_bounds__(256) unpack_kernel(const int16_t* counts, cons
     row[j] = vals[wid * W + s];
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(dev_status, kDevIndex);
+}
+
+// ---------------------------------------------------------------- union of a row tile
+
+// Per tile of 128 rows (one block): the hidden units that the tile's rows that
+// fit (overflow rows skipped when skip_ovf) activate -- the union of their
+// stored columns -- in ascending order, and the tile's hidden values over that
+// union, for the down projection on the tensor cores (kModeUnion):
+//   kb_tile[m]                 K blocks of 64 the tile runs (>= 1)
+//   union_rows[m][0..64 kb)    the union, padded with unit 0
+//   H[128 m + r][0..64 kb)     bf16 hidden value of row r at each union unit, 0 elsewhere
+// (row stride `stride` for both). A stored index outside its own column tile
+// raises TWELL_ERR_INDEX and is left out; a count above W raises
+// TWELL_ERR_OVERFLOW unless overflow rows are skipped.
+struct UnionParams {
+  const int16_t* counts;
+  const int16_t* idx;
+  const uint16_t* vals;
+  const uint8_t* row_ovf;
+  int T, f, nT, W, skip_ovf;
+  int* kb_tile;
+  int* union_rows;
+  uint16_t* H;
+  int stride;
+  int* dev_status;
+};
+
+__global__ void __launch_bounds__(256) union_prep_kernel(const UnionParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ uint32_t bits[1024];  // f <= 32767: at most 1024 words
+  __shared__ int wpre[1024];
+  __shared__ int warp_sum[8];
+  const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwords = p.f / 32;
+  const int t0 = m * 128;
+  for (int w = tid; w < nwords; w += blockDim.x) bits[w] = 0u;
+  __syncthreads();
+  bool bad = false, overflow = false;
+  // 1. the union: one thread per (row, column tile)
+  for (int i = tid; i < 128 * p.nT; i += blockDim.x) {
+    const int r = i / p.nT, c = i - r * p.nT;
+    const int t = t0 + r;
+    if (t >= p.T || (p.skip_ovf && p.row_ovf[t])) continue;
+    const size_t at = static_cast<size_t>(t) * p.nT + c;
+    if (p.counts[at] > p.W) overflow = true;
+    const int n = min(max(static_cast<int>(p.counts[at]), 0), p.W);
+    for (int s = 0; s < n; ++s) {
+      const int j = p.idx[at * p.W + s];
+      if (j < c * 128 || j >= c * 128 + 128) {
+        bad = true;
+        continue;
+      }
+      atomicOr(&bits[j >> 5], 1u << (j & 31));
+    }
+  }
+  __syncthreads();
+  // 2. exclusive prefix of the words' popcounts (each thread a run of words)
+  const int per = (nwords + blockDim.x - 1) / blockDim.x;
+  const int w0 = min(nwords, tid * per), w1 = min(nwords, w0 + per);
+  int mine = 0;
+  for (int w = w0; w < w1; ++w) mine += __popc(bits[w]);
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int before = 0, total = 0;
+  for (int k = 0; k < static_cast<int>(blockDim.x / 32); ++k) {
+    before += k < warp ? warp_sum[k] : 0;
+    total += warp_sum[k];
+  }
+  int run = before + incl - mine;
+  for (int w = w0; w < w1; ++w) {
+    wpre[w] = run;
+    run += __popc(bits[w]);
+  }
+  const int kb = max(1, (total + 63) / 64);
+  const int kpad = kb * 64;
+  if (tid == 0) p.kb_tile[m] = kb;
+  // 3. the union list, padded with unit 0
+  int* ur = p.union_rows + static_cast<size_t>(m) * p.stride;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t b = bits[w];
+    int pos = wpre[w];
+    while (b != 0u) {
+      const int k = __ffs(b) - 1;
+      b &= b - 1u;
+      ur[pos++] = w * 32 + k;
+    }
+  }
+  for (int i = total + tid; i < kpad; i += blockDim.x) ur[i] = 0;
+  // 4. the tile's hidden values over the union: zeros, then the stored slots
+  uint16_t* hb = p.H + static_cast<size_t>(t0) * p.stride;
+  const int vpr = kpad / 8;  // 16-byte vectors per row
+  for (int i = tid; i < 128 * vpr; i += blockDim.x) {
+    const int r = i / vpr, v = i - r * vpr;
+    reinterpret_cast<uint4*>(hb + static_cast<size_t>(r) * p.stride)[v] = make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();  // every zero is written before any value lands on it
+  for (int i = tid; i < 128 * p.nT; i += blockDim.x) {
+    const int r = i / p.nT, c = i - r * p.nT;
+    const int t = t0 + r;
+    if (t >= p.T || (p.skip_ovf && p.row_ovf[t])) continue;
+    const size_t at = static_cast<size_t>(t) * p.nT + c;
+    const int n = min(max(static_cast<int>(p.counts[at]), 0), p.W);
+    for (int s = 0; s < n; ++s) {
+      const int j = p.idx[at * p.W + s];
+      if (j < c * 128 || j >= c * 128 + 128) continue;
+      const int pos = wpre[j >> 5] + __popc(bits[j >> 5] & ((1u << (j & 31)) - 1u));
+      hb[static_cast<size_t>(r) * p.stride + pos] = p.vals[at * p.W + s];
+    }
+  }
+  if (__syncthreads_or(bad) && tid == 0) raise_status(p.dev_status, kDevIndex);
+  if (__syncthreads_or(overflow) && tid == 0 && !p.skip_ovf) raise_status(p.dev_status, kDevOverflow);
 }
 
 // ---------------------------------------------------------------- compaction

@@ -14,6 +14,7 @@
 
 #include "twell.h"
 #include "backward.cuh"
+#include "gemv.cuh"
 #include "sparse_ffn.cuh"
 #include "umma_gemm.cuh"
 
@@ -163,6 +164,27 @@ twell_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, 
   return cuda_ok(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
 }
 
+// The same, with the grid cut into clusters of `cluster` consecutive blocks.
+template <typename... KArgs, typename... Args>
+twell_status launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, int cluster, cudaStream_t s,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cuda_ok(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
+}
+
 // Zero up to three device byte ranges with one dependent launch.
 twell_status zero_async(cudaStream_t s, int sms, void* p0, size_t n0, void* p1 = nullptr, size_t n1 = 0,
                         void* p2 = nullptr, size_t n2 = 0) {
@@ -308,6 +330,58 @@ twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t*
   return down_only ? sparse_launch<true>(p, d, sms, s, y_zeroed) : sparse_launch<false>(p, d, sms, s, y_zeroed);
 }
 
+// The sparse step of a batch of at most 8 tokens with d a multiple of 256: one
+// warp per stored slot (sparse_small_kernel), enough blocks per token for one
+// slot per warp when every tile is full, and about two blocks per SM at most.
+// The rows of y it writes must hold zeros; overflow rows are skipped.
+template <int NCH>
+twell_status sparse_small_n(const SparseParams& p, bool down_only, int sms, cudaStream_t s) {
+  const long long most = (static_cast<long long>(p.nT) * p.W + kSmallSparseWarps - 1) / kSmallSparseWarps;
+  const long long spread = (2LL * sms + p.T - 1) / p.T;
+  const dim3 grid(static_cast<unsigned>(std::max(1LL, std::min(most, spread))), static_cast<unsigned>(p.T));
+  if (down_only) return launch(sparse_small_kernel<NCH, true>, grid, dim3(kSmallSparseWarps * 32), 0, s, p);
+  return launch(sparse_small_kernel<NCH, false>, grid, dim3(kSmallSparseWarps * 32), 0, s, p);
+}
+
+twell_status sparse_small_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
+                               const twell_t* tw, float* y, int32_t* dev_status, cudaStream_t s, int sms,
+                               bool down_only) {
+  SparseParams p{};
+  p.x = x;
+  p.WuT = WuT;
+  p.Wd = Wd;
+  p.counts = tw->counts;
+  p.idx = tw->idx;
+  p.vals = tw->vals;
+  p.row_ovf = tw->row_ovf;
+  p.y = y;
+  p.T = T;
+  p.d = d;
+  p.f = f;
+  p.nT = f / 128;
+  p.W = tw->W;
+  p.skip_ovf = 1;
+  p.dev_status = dev_status;
+  switch (d / 256) {
+    case 1: return sparse_small_n<1>(p, down_only, sms, s);
+    case 2: return sparse_small_n<2>(p, down_only, sms, s);
+    case 3: return sparse_small_n<3>(p, down_only, sms, s);
+    case 4: return sparse_small_n<4>(p, down_only, sms, s);
+    case 5: return sparse_small_n<5>(p, down_only, sms, s);
+    case 6: return sparse_small_n<6>(p, down_only, sms, s);
+    case 7: return sparse_small_n<7>(p, down_only, sms, s);
+    case 8: return sparse_small_n<8>(p, down_only, sms, s);
+    case 9: return sparse_small_n<9>(p, down_only, sms, s);
+    case 10: return sparse_small_n<10>(p, down_only, sms, s);
+    case 11: return sparse_small_n<11>(p, down_only, sms, s);
+    case 12: return sparse_small_n<12>(p, down_only, sms, s);
+    case 13: return sparse_small_n<13>(p, down_only, sms, s);
+    case 14: return sparse_small_n<14>(p, down_only, sms, s);
+    case 15: return sparse_small_n<15>(p, down_only, sms, s);
+    default: return sparse_small_n<16>(p, down_only, sms, s);
+  }
+}
+
 // Down projection from a TwELL of hidden activations (per-token gathers of Wd rows).
 twell_status down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip, float* y,
                        int32_t* dev_status, cudaStream_t s, int sms) {
@@ -317,6 +391,79 @@ twell_status down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* t
 twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, const uint16_t* Wd, int d, int f,
                              bool split, const int* row_map, float* y, int y_rows, int32_t* dev_status,
                              cudaStream_t s, int sms);
+
+// ------------------------------------------------------------------ down projection over tile unions
+
+// Workspace of the union down projection, carved from the hybrid workspace:
+// the tiles' hidden-value blocks (H, [num_m * 128][f] bf16), then the tiles'
+// union lists ([num_m][f] int32) and K block counts ([num_m] int32).
+size_t union_bytes(int T, int f) {
+  const size_t num_m = (static_cast<size_t>(T) + kBM - 1) / kBM;
+  return round_up(num_m * kBM * f * 2, 256) + round_up(num_m * f * 4, 256) + round_up(num_m * 4, 256);
+}
+
+// Whether the hybrid forwards take the union form. Measured on B200 it loses
+// to the per-token kernel at every configured layer (0.5B, 1.5B and 2B), so
+// the forwards keep the per-token kernel; the union form stays an explicit
+// entry point. When enabled it needs output tiles that fill the GPU at least
+// once (below that the per-token kernel spreads a token over several warps).
+constexpr bool kUnionInHybrid = false;
+
+bool union_selected(int T, int d, int f, size_t workspace_bytes, int sms) {
+  const long long tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN);
+  return kUnionInHybrid && tiles >= sms && union_bytes(T, f) <= workspace_bytes;
+}
+
+// y (rows that fit) = per 128-row tile, the tile's hidden values over its
+// union of stored units times those rows of Wd, on the tensor cores.
+twell_status union_down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip, float* y,
+                             void* ws, int32_t* dev_status, cudaStream_t s, int sms) {
+  const int num_m = (T + kBM - 1) / kBM;
+  char* w = static_cast<char*>(ws);
+  UnionParams u{};
+  u.counts = tw->counts;
+  u.idx = tw->idx;
+  u.vals = tw->vals;
+  u.row_ovf = tw->row_ovf;
+  u.T = T;
+  u.f = f;
+  u.nT = f / 128;
+  u.W = tw->W;
+  u.skip_ovf = skip ? 1 : 0;
+  u.H = reinterpret_cast<uint16_t*>(w);
+  u.union_rows = reinterpret_cast<int*>(w + round_up(static_cast<size_t>(num_m) * kBM * f * 2, 256));
+  u.kb_tile = u.union_rows + round_up(static_cast<size_t>(num_m) * f * 4, 256) / 4;
+  u.stride = f;
+  u.dev_status = dev_status;
+  TW_TRY(launch(union_prep_kernel, dim3(num_m), dim3(256), 0, s, u));
+  // A: the H blocks in 128 x 64 boxes; B: Wd rows one at a time (gather4 takes four)
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, u.H, f, static_cast<uint64_t>(num_m) * kBM, kBK, kBM) || !make_map(&mb, Wd, d, f, 64, 1))
+    return TWELL_ERR_CUDA;
+  GemmParams p{};
+  p.M = T;
+  p.N = d;
+  p.K = f;
+  p.out_f32 = y;
+  p.ldo = d;
+  p.out_rows = T;
+  p.k_splits_max = 1;
+  p.kb_tile = u.kb_tile;
+  p.union_rows = u.union_rows;
+  p.union_stride = f;
+  p.dev_status = dev_status;
+  return launch_gemm<kModeUnion>(ma, mb, mb, p, gemm_grid(T, d, kBN, sms), s);
+}
+
+// The down projection of the hybrid forwards whose pack holds the hidden
+// activations (overflow rows skipped): over tile unions on the tensor cores
+// when that fills the GPU and fits the caller's workspace (used only until the
+// dense branch, which runs after), else the per-token kernel.
+twell_status hybrid_down(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, float* y, void* ws,
+                         size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms) {
+  if (union_selected(T, d, f, ws_bytes, sms)) return union_down_impl(Wd, T, d, f, tw, 1, y, ws, dev_status, s, sms);
+  return down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms);
+}
 
 // Dense FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu), or
 // h = ReLU(A Wg) for the non-gated layer (WuT null), into h_buf, then
@@ -374,6 +521,7 @@ twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, con
   p2.k_splits_max = 1;
   if (row_map != nullptr) {
     p2.k_splits_max = 32;
+    p2.split_waves = 1;  // the gather zeroed every routed row
   } else if (static_cast<long long>((M + kBM - 1) / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms) {
     TW_TRY(zero_async(s, sms, y, static_cast<size_t>(M) * d * sizeof(float)));
     p2.k_splits_max = 32;
@@ -386,6 +534,137 @@ twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, con
 
 
 // ------------------------------------------------------------------ small batches
+
+// ------------------------------------------------------------------ batches of <= 8 tokens
+
+// The GEMV path: at most 8 tokens and d a multiple of 256.
+bool gemv_batch(int T, int d) { return T <= kGemvMaxT && d % 256 == 0; }
+
+// Tokens the kernels are compiled for: the batch rounded up to 1, 2, 4 or 8
+// (the branch modes read their row count on the device and take 8).
+int gemv_nt(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : 8; }
+
+template <int MODE, int NT>
+twell_status gemv_first_nt(const GemvParams& p, cudaStream_t s) {
+  auto kern = gemv_first_kernel<MODE, NT>;
+  const size_t smem = static_cast<size_t>(NT) * p.d * 2;
+  TW_TRY(cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))));
+  if (gv_pack(MODE))
+    return launch_cluster(kern, dim3(p.nT * kGemvCluster), dim3(kGemvThreads), smem, kGemvCluster, s, p);
+  return launch(kern, dim3(p.f / kGemvCols), dim3(kGemvThreads), smem, s, p);
+}
+
+template <int MODE>
+twell_status gemv_first(const GemvParams& p, cudaStream_t s) {
+  switch (gv_branch(MODE) ? kGemvMaxT : gemv_nt(p.T)) {
+    case 1: return gemv_first_nt<MODE, 1>(p, s);
+    case 2: return gemv_first_nt<MODE, 2>(p, s);
+    case 4: return gemv_first_nt<MODE, 4>(p, s);
+    default: return gemv_first_nt<MODE, kGemvMaxT>(p, s);
+  }
+}
+
+// The down GEMV's grid: one block per 256 columns of d times row groups, about
+// two blocks per SM in all (one wave), each group a multiple of 8 rows.
+twell_status gemv_down(GemvDownParams p, int nt, cudaStream_t s, int sms) {
+  const int slices = (p.d + kGemvDownCols - 1) / kGemvDownCols;
+  const int groups = std::max(1, (2 * sms + slices - 1) / slices);
+  int rpb = (p.f + groups - 1) / groups;
+  rpb = std::min(kGemvDownMaxRows, std::max(kGemvWarps, (rpb + kGemvWarps - 1) / kGemvWarps * kGemvWarps));
+  p.rows_per_block = rpb;
+  const dim3 grid(static_cast<unsigned>((p.f + rpb - 1) / rpb), static_cast<unsigned>(slices));
+  switch (nt) {
+    case 1: return launch(gemv_down_kernel<1>, grid, dim3(kGemvThreads), 0, s, p);
+    case 2: return launch(gemv_down_kernel<2>, grid, dim3(kGemvThreads), 0, s, p);
+    case 4: return launch(gemv_down_kernel<4>, grid, dim3(kGemvThreads), 0, s, p);
+    default: return launch(gemv_down_kernel<kGemvMaxT>, grid, dim3(kGemvThreads), 0, s, p);
+  }
+}
+
+GemvParams gemv_params(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, int T, int d, int f,
+                       int32_t* dev_status) {
+  GemvParams p{};
+  p.x = x;
+  p.WgT = WgT;
+  p.WuT = WuT;
+  p.T = T;
+  p.d = d;
+  p.f = f;
+  p.nT = f / 128;
+  p.dev_status = dev_status;
+  return p;
+}
+
+// Hybrid forward of a batch of <= 8 tokens: the pack from the GEMV (which also
+// zeroes y), routing with the flags derived from the counts, the sparse step
+// with one warp per stored slot (down only when the pack holds hidden
+// values), and the dense branch as
+// GEMVs over the listed rows with fp32 hidden activations (h_buf: [T][f] fp32).
+// mode: 0 gated (gate pack, fused up+down), 1 gated with hidden values, 2 non-gated.
+twell_status gemv_hybrid(int mode, const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
+                         int T, int d, int f, const twell_t* tw, float* y, int32_t* ovf_rows, int32_t* n_ovf,
+                         float* h_buf, int32_t* dev_status, cudaStream_t s, int sms) {
+  GemvParams p = gemv_params(x, WgT, mode == 1 ? WuT : nullptr, T, d, f, dev_status);
+  p.W = tw->W;
+  p.counts = tw->counts;
+  p.idx = tw->idx;
+  p.vals = tw->vals;
+  p.y_zero = y;
+  if (mode == 1) {
+    TW_TRY(gemv_first<kGvPackHidden>(p, s));
+  } else {
+    TW_TRY(gemv_first<kGvPackGate>(p, s));
+  }
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf,
+                static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr),
+                static_cast<const int16_t*>(tw->counts), f / 128, tw->W));
+  TW_TRY(sparse_small_impl(x, WuT, Wd, T, d, f, tw, y, dev_status, s, sms, mode != 0));
+  // the dense branch over the listed rows, hidden activations in fp32
+  GemvParams b = gemv_params(x, WgT, mode == 2 ? nullptr : WuT, T, d, f, dev_status);
+  b.rows = ovf_rows;
+  b.n_rows = n_ovf;
+  b.h_f32 = h_buf;
+  if (mode == 2) {
+    TW_TRY(gemv_first<kGvBranchRelu>(b, s));
+  } else {
+    TW_TRY(gemv_first<kGvBranchH>(b, s));
+  }
+  GemvDownParams q{};
+  q.h_f32 = h_buf;
+  q.Wd = Wd;
+  q.y = y;
+  q.rows = ovf_rows;
+  q.n_rows = n_ovf;
+  q.T = T;
+  q.d = d;
+  q.f = f;
+  TW_TRY(gemv_down(q, kGemvMaxT, s, sms));
+  return cuda_ok(cudaGetLastError());
+}
+
+// Dense layer of a batch of <= 8 tokens: h (bf16, in h_buf [T][f]) from the
+// GEMV, which also zeroes y, then y += h Wd. gated: ReLU(x Wg) (x Wu), else ReLU(x W1).
+twell_status gemv_dense(bool gated, const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
+                        int T, int d, int f, float* y, uint16_t* h_buf, int32_t* dev_status, cudaStream_t s,
+                        int sms) {
+  GemvParams p = gemv_params(x, WgT, gated ? WuT : nullptr, T, d, f, dev_status);
+  p.h_bf16 = h_buf;
+  p.y_zero = y;
+  if (gated) {
+    TW_TRY(gemv_first<kGvDenseH>(p, s));
+  } else {
+    TW_TRY(gemv_first<kGvDenseRelu>(p, s));
+  }
+  GemvDownParams q{};
+  q.h_bf16 = h_buf;
+  q.Wd = Wd;
+  q.y = y;
+  q.T = T;
+  q.d = d;
+  q.f = f;
+  TW_TRY(gemv_down(q, gemv_nt(T), s, sms));
+  return cuda_ok(cudaGetLastError());
+}
 
 // Batches up to this many tokens whose gate GEMM has too few output tiles to
 // fill the GPU take the small-batch path: the gate GEMM splits K over the whole
@@ -508,6 +787,34 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
   return down_impl(Wd, T, d, f, tw, skip_overflow_rows, y, dev_status, static_cast<cudaStream_t>(stream), sms);
 }
 
+size_t twell_sparse_down_union_workspace_bytes(int T, int d, int f) {
+  (void)d;
+  if (T <= 0 || f < 128) return 0;
+  return union_bytes(T, f);
+}
+
+twell_status twell_sparse_down_union(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                                     int skip_overflow_rows, float* y, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream) {
+  TW_TRY(check_shape(T, d, f));
+  TW_TRY(check_tw(tw, T, f));
+  if (T == 0) return TWELL_OK;
+  TW_TRY(check_ptrs({Wd, y, dev_status}));
+  if (workspace == nullptr || workspace_bytes < union_bytes(T, f)) return TWELL_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return TWELL_ERR_ALIGN;
+  int dev, sms;
+  TW_TRY(current_device(&dev, &sms));
+  return union_down_impl(Wd, T, d, f, tw, skip_overflow_rows, y, workspace, dev_status,
+                         static_cast<cudaStream_t>(stream), sms);
+}
+
+int twell_hybrid_down_is_union(int T, int d, int f, size_t workspace_bytes) {
+  if (check_shape(T, d, f) != TWELL_OK || T == 0) return 0;
+  int dev, sms;
+  if (current_device(&dev, &sms) != TWELL_OK) return 0;
+  return union_selected(T, d, f, workspace_bytes, sms) ? 1 : 0;
+}
+
 twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                             const uint16_t* Wd, int T, int d, int f, const twell_t* tw, float* y,
                                             int32_t* ovf_rows, int32_t* n_ovf, void* workspace,
@@ -524,10 +831,12 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
   uint16_t* xo = static_cast<uint16_t*>(workspace);
   uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
                                              round_up(static_cast<size_t>(T) * d * 2, 256));
+  if (gemv_batch(T, d)) return gemv_hybrid(1, x, WgT, WuT, Wd, T, d, f, tw, y, ovf_rows, n_ovf,
+                                        reinterpret_cast<float*>(ho), dev_status, s, sms);
   TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms));
+  TW_TRY(hybrid_down(Wd, T, d, f, tw, y, workspace, workspace_bytes, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
 }
 
@@ -537,7 +846,7 @@ twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, v
   TW_TRY(check_ptrs({ovf_rows, n_ovf}));
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream), tw->row_ovf, tw->T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream), tw->row_ovf, tw->T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -562,18 +871,20 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
   uint16_t* xo = static_cast<uint16_t*>(workspace);
   uint16_t* ho = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
                                              round_up(static_cast<size_t>(T) * d * 2, 256));
+  if (gemv_batch(T, d)) return gemv_hybrid(0, x, WgT, WuT, Wd, T, d, f, tw, y, ovf_rows, n_ovf,
+                                        reinterpret_cast<float*>(ho), dev_status, s, sms);
   if (small_batch(T, f, kBN, sms)) {
     // the h region of the dense branch is free until that branch runs
     const bool zero_y = sparse_splits_units(T, d, false, sms);
     TW_TRY(small_gate_pack_impl(x, WgT, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
                                 dev_status, s, sms));
-    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y));
+    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y, static_cast<const int16_t*>(nullptr), 0, 0));
     TW_TRY(cuda_ok(cudaGetLastError()));
     TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms, false, zero_y));
     return dense_impl(xo, T, n_ovf, WgT, WuT, Wd, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
   TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
@@ -617,6 +928,7 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
   TW_TRY(current_device(&dev, &sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint16_t* h = static_cast<uint16_t*>(workspace);
+  if (gemv_batch(T, d)) return gemv_dense(true, x, WgT, WuT, Wd, T, d, f, y, h, dev_status, s, sms);
   if (small_batch(T, f, 128, sms)) {
     // z and u with K split over the whole grid, then h = bf16(ReLU(z) * u)
     float* zu = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(T) * f * 2, 256));
@@ -649,19 +961,21 @@ twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1
                                              round_up(static_cast<size_t>(T) * d * 2, 256));
   // The pack of ReLU(x W1) holds the hidden activations themselves, so the
   // sparse step is the down projection alone.
+  if (gemv_batch(T, d)) return gemv_hybrid(2, x, W1T, nullptr, W2, T, d, f, tw, y, ovf_rows, n_ovf,
+                                        reinterpret_cast<float*>(ho), dev_status, s, sms);
   if (small_batch(T, f, kBN, sms)) {
     const bool zero_y = sparse_splits_units(T, d, true, sms);
     TW_TRY(small_gate_pack_impl(x, W1T, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
                                 dev_status, s, sms));
-    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y));
+    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y, static_cast<const int16_t*>(nullptr), 0, 0));
     TW_TRY(cuda_ok(cudaGetLastError()));
     TW_TRY(sparse_impl(nullptr, nullptr, W2, T, d, f, tw, 1, y, dev_status, s, sms, true, zero_y));
     return dense_impl(xo, T, n_ovf, W1T, nullptr, W2, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
   TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(down_impl(W2, T, d, f, tw, 1, y, dev_status, s, sms));
+  TW_TRY(hybrid_down(W2, T, d, f, tw, y, workspace, workspace_bytes, dev_status, s, sms));
   return dense_rows_impl(x, W1T, nullptr, W2, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
 }
 
@@ -695,6 +1009,7 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
   TW_TRY(current_device(&dev, &sms));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint16_t* h = static_cast<uint16_t*>(workspace);
+  if (gemv_batch(T, d)) return gemv_dense(false, x, W1T, nullptr, W2, T, d, f, y, h, dev_status, s, sms);
   if (small_batch(T, f, kBN, sms)) {
     float* z = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(static_cast<size_t>(T) * f * 2, 256));
     TW_TRY(zero_async(s, sms, z, static_cast<size_t>(T) * f * 4));

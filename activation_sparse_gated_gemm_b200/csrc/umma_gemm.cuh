@@ -44,6 +44,13 @@
 //                  row map (the dense branch of the hybrid route). With the
 //                  remainder stored, K runs over [h | h - bf16(h)] against
 //                  [Wd ; Wd], which removes the bf16 rounding of h to ~2^-16.
+//   kModeUnion  -- the down projection of the rows that fit over the hidden
+//                  units their 128-row tile activates: per M tile, K runs over
+//                  that tile's union of stored units only (its own length,
+//                  read on the device), A is the tile's hidden values at those
+//                  units (a block written by union_prep_kernel) and B is the
+//                  union's rows of Wd, gathered four rows per TMA instruction
+//                  (tile::gather4) into the layout kModeDown's boxes give.
 //
 // Structure: one CTA per SM walks output tiles of 128 x 256 (x 128 h-columns
 // for kModeGateUp). Warp 0 issues TMA loads into a 4-stage shared-memory ring,
@@ -67,7 +74,8 @@ enum GemmMode : int {
   kModeActivity = 5,
   kModeF32 = 6,
   kModeZU = 7,
-  kModeBwdDh = 8
+  kModeBwdDh = 8,
+  kModeUnion = 9
 };
 
 constexpr int kBM = 128;
@@ -91,7 +99,7 @@ constexpr int kOffSlots = kOffEpi + kEpiBytes;
 constexpr int kOffBar = kOffSlots + kEpiThreads * kStageSlotBytes;
 constexpr int kNumBars = 2 * kStages + 4 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kGemmSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
+constexpr int kGemmSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024 (misc: TMEM base, abort flag, K splits)
 static_assert(kGemmSmemBytes <= 232448, "GEMM shared memory exceeds the 227 KB per-CTA limit");
 
 struct GemmParams {
@@ -145,6 +153,16 @@ struct GemmParams {
   // this many splits whose partial sums are added into out_f32 (which must
   // hold zeros in the rows written); 0 or 1 disables splitting.
   int k_splits_max;
+  // With split_waves set (the caller zeroes the rows written in every case),
+  // K is also split when the tiles fill the grid but leave its last wave
+  // short.
+  int split_waves;
+  // kModeUnion: K blocks of each M tile (>= 1) and the B rows of each M tile
+  // ([num_m][union_stride] row indices into tmB0's rows, ascending, padded to
+  // a multiple of 64 with a valid row; 16-byte aligned).
+  const int* kb_tile;
+  const int* union_rows;
+  int union_stride;
   int* dev_status;
 };
 
@@ -261,11 +279,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     nkb_half = (min(max(*p.k_dev, 0), p.k_half) + kBK - 1) / kBK;
     num_kb = 2 * nkb_half;
   }
-  // K splits (kModeDown / kModeF32): as many as keep every CTA busy, none empty.
+  // K splits (kModeDown / kModeF32, output zeroed beforehand; when the tiles
+  // fill the grid only with split_waves): the count whose work units
+  // (tiles x splits) finish soonest on the grid, counting the waves of the
+  // slowest CTA in units of a whole-K tile, with 2% per extra split for the
+  // partial sums it adds (e.g. 189 tiles on 148 CTAs: 3 splits, 1.33 waves
+  // instead of 2).
+  // Warp 0 scores the candidate counts, two per lane, and the choice reaches
+  // the other warps through shared memory (the divisions are too slow to run
+  // in every thread of every CTA).
   int kb_per = num_kb, k_splits = 1;
-  if ((MODE == kModeDown || MODE == kModeF32) && p.k_splits_max > 1 && num_m * num_n > 0 && num_kb > 0) {
-    int want = min(p.k_splits_max, max(1, static_cast<int>(gridDim.x) / (num_m * num_n)));
-    want = min(want, num_kb);
+  if ((MODE == kModeDown || MODE == kModeF32) && p.k_splits_max > 1 && num_m * num_n > 0 && num_kb > 0 &&
+      (p.split_waves || num_m * num_n < static_cast<int>(gridDim.x))) {
+    int* split_slot = reinterpret_cast<int*>(smem + kOffMisc + 8);
+    if (warp == 0) {
+      const long long tiles = static_cast<long long>(num_m) * num_n, grid = gridDim.x;
+      const int most = min(min(p.k_splits_max, num_kb), 64);
+      float best = 3.0e38f;
+      int want = 1;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int ks = lane + 1 + 32 * h;
+        if (ks <= most) {
+          const int per = (num_kb + ks - 1) / ks;
+          const int splits = (num_kb + per - 1) / per;
+          const float waves = static_cast<float>((tiles * splits + grid - 1) / grid) * per / num_kb;
+          const float cost = waves * (1.0f + 0.02f * (splits - 1));
+          if (cost < best - 1e-6f) {
+            best = cost;
+            want = ks;
+          }
+        }
+      }
+      // the lowest cost, ties to the fewest splits
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int ow = __shfl_xor_sync(0xffffffffu, want, o);
+        if (ob < best - 1e-6f || (fabsf(ob - best) <= 1e-6f && ow < want)) {
+          best = ob;
+          want = ow;
+        }
+      }
+      if (lane == 0) *split_slot = want;
+    }
+    __syncthreads();
+    const int want = *split_slot;
     kb_per = (num_kb + want - 1) / want;
     k_splits = (num_kb + kb_per - 1) / kb_per;
   }
@@ -286,14 +345,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int ks = tile - mn * k_splits;
         const int m_blk = mn / num_n;
         const int n_blk = mn - m_blk * num_n;
-        const int kb_end = min(num_kb, (ks + 1) * kb_per);
-        for (int kb = ks * kb_per; kb < kb_end; ++kb) {
+        int kb_begin = ks * kb_per, kb_end = min(num_kb, (ks + 1) * kb_per);
+        const int* urows = nullptr;
+        int slabs = 4;
+        if (MODE == kModeUnion) {
+          // this M tile's union length, and the 64-column slabs of B inside d
+          kb_begin = 0;
+          kb_end = min(max(p.kb_tile[m_blk], 0), num_kb);
+          urows = p.union_rows + static_cast<size_t>(m_blk) * p.union_stride;
+          slabs = min(4, (p.N - n_blk * kBN) / 64);
+        }
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
+          int4 rq[16];
+          if (MODE == kModeUnion) {
+            // the K block's 64 rows of B, fetched before the wait
+#pragma unroll
+            for (int q = 0; q < 16; ++q) rq[q] = __ldg(reinterpret_cast<const int4*>(urows + kb * kBK) + q);
+          }
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           uint8_t* a_dst = smem + kOffA + s * kAStageBytes;
           uint8_t* b_dst = smem + kOffB + s * kBStageBytes;
+          if (MODE == kModeUnion) {
+            // A: the tile's hidden values over the union (one TMA box). B: each
+            // 64-column slab gets the K block's 64 rows of Wd four at a time
+            // (tile::gather4 with a one-row box), landing in the same
+            // 128-byte-swizzled N-major layout a 64 x 64 box gives.
+            mbar_arrive_expect_tx(&full[s], kAStageBytes + slabs * (kBStageBytes / 4));
+            tma_load_2d(a_dst, &tmA, &full[s], kb * kBK, m_blk * kBM);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const int lim = p.K - 1;  // a row outside Wd would be a fault in the list: clamped
+              const int r0 = min(max(rq[q].x, 0), lim), r1 = min(max(rq[q].y, 0), lim);
+              const int r2 = min(max(rq[q].z, 0), lim), r3 = min(max(rq[q].w, 0), lim);
+              for (int i = 0; i < slabs; ++i)
+                tma_gather4(b_dst + i * (kBStageBytes / 4) + q * 4 * 128, &tmB0, &full[s], n_blk * kBN + i * 64,
+                            r0, r1, r2, r3);
+            }
+            issued |= 1u << s;
+            issued_par = (issued_par & ~(1u << s)) | (ph << s);
+            if (++s == kStages) {
+              s = 0;
+              ph ^= 1u;
+            }
+            continue;
+          }
           // the K block's position in A (and B): compact K skips the empty
           // tail of each half
           const int kc = (nkb_half > 0 && kb >= nkb_half) ? p.k_half / kBK + (kb - nkb_half) : kb;
@@ -337,7 +435,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      const uint32_t idesc = umma_idesc_bf16(kBM, kBN, MODE == kModeDown ? 1 : 0);
+      const uint32_t idesc = umma_idesc_bf16(kBM, kBN, (MODE == kModeDown || MODE == kModeUnion) ? 1 : 0);
       int s = 0;
       uint32_t ph = 0;
       int buf = 0;
@@ -351,7 +449,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
         const int ks = tile % k_splits;
-        const int kb_begin = ks * kb_per, kb_end = min(num_kb, (ks + 1) * kb_per);
+        int kb_begin = ks * kb_per, kb_end = min(num_kb, (ks + 1) * kb_per);
+        if (MODE == kModeUnion) {
+          kb_begin = 0;
+          kb_end = min(max(p.kb_tile[(tile / k_splits) / num_n], 0), num_kb);
+        }
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
             ok = false;
@@ -366,7 +468,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // 16 bf16 is 32 bytes inside the swizzle row.
             const uint64_t adesc = umma_smem_desc(a_addr + k * 32, 16, 1024);
             uint64_t bdesc;
-            if (MODE == kModeDown) {
+            if (MODE == kModeDown || MODE == kModeUnion) {
               // N-major, 128-byte swizzle: 64-column slabs 8 KB apart (LBO), 8-row
               // K groups 1 KB apart (SBO); a K step of 16 rows is 2 KB.
               bdesc = umma_smem_desc(b_addr + k * 2048, kBStageBytes / 4, 1024);

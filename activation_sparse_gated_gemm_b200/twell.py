@@ -34,7 +34,8 @@ EXPORTED = (
     "twell_column_activity", "twell_compact_columns", "twell_gather_rows",
     "twell_backward_workspace_bytes", "twell_ffn_hybrid_backward", "twell_ffn_hybrid_backward_dx",
     "twell_ffn_hybrid_backward_dw", "twell_dense_backward_workspace_bytes", "twell_dense_ffn_backward",
-    "twell_ffn_hybrid_backward_dw_tc", "twell_ffn_hybrid_backward_dx_tc",
+    "twell_ffn_hybrid_backward_dw_tc", "twell_ffn_hybrid_backward_dx_tc", "twell_sparse_down_union",
+    "twell_sparse_down_union_workspace_bytes", "twell_hybrid_down_is_union",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -79,6 +80,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "twell_route": ([tw, vp, vp, vp], i32),
         "twell_gate_up_pack": ([vp, vp, vp, i32, i32, i32, tw, vp, vp], i32),
         "twell_sparse_down": ([vp, i32, i32, i32, tw, i32, vp, vp, vp], i32),
+        "twell_sparse_down_union": ([vp, i32, i32, i32, tw, i32, vp, vp, sz, vp, vp], i32),
+        "twell_sparse_down_union_workspace_bytes": ([i32, i32, i32], sz),
+        "twell_hybrid_down_is_union": ([i32, i32, i32, sz], i32),
         "twell_ffn_hybrid_forward_tc_up": ([vp, vp, vp, vp, i32, i32, i32, tw, vp, vp, vp, vp, sz, vp, vp], i32),
         "twell_hybrid_workspace_bytes": ([i32, i32, i32], sz),
         "twell_dense_rows_forward": ([vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp], i32),
@@ -225,6 +229,28 @@ def sparse_down(Wd, tw: Twell, y, skip_overflow_rows: bool, dev_status, stream=N
     _bf16("y", y, (T, d))
     _check("twell_sparse_down", load().twell_sparse_down(_ptr(Wd), T, d, f, tw.ref(), int(bool(skip_overflow_rows)),
                                                          _ptr(y), _ptr(dev_status), _stream(stream)))
+
+
+def sparse_down_union(Wd, tw: Twell, y, skip_overflow_rows: bool, workspace, dev_status, stream=None) -> None:
+    """The down projection per 128-row tile over the tile's union of stored
+    units, on the tensor cores; workspace of sparse_down_union_workspace_bytes(T, d, f)."""
+    f, d = Wd.shape
+    T = tw.T
+    _bf16("Wd", Wd, (f, d))
+    _bf16("y", y, (T, d))
+    _check("twell_sparse_down_union", load().twell_sparse_down_union(
+        _ptr(Wd), T, d, f, tw.ref(), int(bool(skip_overflow_rows)), _ptr(y), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream)))
+
+
+def sparse_down_union_workspace_bytes(T: int, d: int, f: int) -> int:
+    return int(load().twell_sparse_down_union_workspace_bytes(T, d, f))
+
+
+def hybrid_down_is_union(T: int, d: int, f: int, workspace_bytes: int) -> bool:
+    """Whether the hybrid forwards whose pack holds hidden activations run the
+    down projection over tile unions at this shape with this much workspace."""
+    return bool(load().twell_hybrid_down_is_union(T, d, f, workspace_bytes))
 
 
 def ffn_hybrid_forward_tc_up(x, WgT, WuT, Wd, tw: Twell, y, ovf_rows, n_ovf, workspace, dev_status,

@@ -165,17 +165,27 @@ def record_traffic(csv_path: str, workload: str, kernels: list, command: str) ->
     with open(csv_path, newline="") as fh:
         rows = list(csv.reader(fh))
     head = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
-    cols, units = rows[head], rows[head + 1]
+    cols = rows[head]
     kn = cols.index("Kernel Name")
-    rd, wr = cols.index("dram__bytes_read.sum"), cols.index("dram__bytes_write.sum")
-
-    def val(r, c):
-        return float(r[c].replace(",", "")) * UNIT_BYTES.get(units[c], 1.0)
-
+    launches = {}  # launch id -> (kernel name, bytes)
+    if "Metric Name" in cols:  # one row per (launch, metric): ncu --metrics ... --csv
+        idc, mn, mu, mv = (cols.index(c) for c in ("ID", "Metric Name", "Metric Unit", "Metric Value"))
+        for r in rows[head + 1:]:
+            if len(r) > mv and r[mn] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+                v = float(r[mv].replace(",", "")) * UNIT_BYTES.get(r[mu], 1.0)
+                name, b = launches.get(r[idc], (r[kn], 0.0))
+                launches[r[idc]] = (name, b + v)
+    else:  # one row per launch: ncu -i rep --page raw --csv (second row: units)
+        units = rows[head + 1]
+        rd, wr = cols.index("dram__bytes_read.sum"), cols.index("dram__bytes_write.sum")
+        for i, r in enumerate(rows[head + 2:]):
+            if len(r) > max(rd, wr):
+                launches[i] = (r[kn], sum(float(r[c].replace(",", "")) * UNIT_BYTES.get(units[c], 1.0)
+                                          for c in (rd, wr)))
     out = {}
     for pair in kernels:
         stage, sub = pair.split("=", 1)
-        got = [val(r, rd) + val(r, wr) for r in rows[head + 2:] if len(r) > kn and sub in r[kn]]
+        got = [b for name, b in launches.values() if sub in name]
         if not got:
             raise SystemExit(f"no captured launch of {sub!r} in {csv_path}")
         out[stage] = float(np.mean(got))
@@ -337,8 +347,16 @@ def run_gpu(args, world, rank, local):
     # The two forms of the hybrid forward: "gate" packs ReLU(z) and runs the
     # fused sparse up+down step; "tc_up" forms u on the tensor cores with the
     # gate and packs h, leaving only the down projection sparse.
+    # the down projection of the tc_up and non-gated forms, as the library's
+    # hybrid forwards run it for this shape (over tile unions on the tensor
+    # cores, its blocks in the hybrid workspace, or per token)
+    down_union = tl.hybrid_down_is_union(T, d, f, ws.numel())
+
     def down():
-        tl.sparse_down(Wd, tw, y, True, st)
+        if down_union:
+            tl.sparse_down_union(Wd, tw, y, True, ws, st)
+        else:
+            tl.sparse_down(Wd, tw, y, True, st)
 
     def stage_fns(variant):
         if variant == "relu":  # the non-gated layer ReLU(x W1) W2 with W1 = Wg, W2 = Wd
@@ -561,8 +579,10 @@ def run_gpu(args, world, rank, local):
                 "path": "the library's hybrid forward of the chosen form",
                 "l2": "not flushed: each step touches ~0.26 GB, above the 126 MB L2"},
         # per step: zeroing, gate (or gate+up) GEMM, routing, sparse step, row gather, two dense-branch GEMMs
-        "gpu_launches": 7 * K,
-        "down_projection": "fused up+down per token" if chosen == "gate" else "per token",
+        # (the down projection over tile unions is two launches: its preparation and its GEMM)
+        "gpu_launches": (8 if down_union and chosen != "gate" else 7) * K,
+        "down_projection": ("fused up+down per token" if chosen == "gate" else
+                            "over tile unions on the tensor cores" if down_union else "per token"),
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -916,11 +936,17 @@ def run_sweep(args) -> None:
             alg = algorithmic(cfg, n_o, nnz, union)
             t_roof = max((alg["gate_flops"] + alg["dense_branch_flops"]) / (peaks["bf16_tflops"] * 1e12),
                          alg["alg_bytes"] / (peaks["hbm_gbs"] * 1e9))
+            # the dense layer's own bound: 6 T d f FLOPs at the tensor peak, or its
+            # three weight matrices, x, y and the bf16 h round trip at the HBM peak
+            dense_bytes = 3 * 2.0 * cfg.d * cfg.f + 6.0 * T * cfg.d + 4.0 * T * cfg.f
+            t_dense_roof = max(6.0 * T * cfg.d * cfg.f / (peaks["bf16_tflops"] * 1e12),
+                               dense_bytes / (peaks["hbm_gbs"] * 1e9))
             print(json.dumps({"sweep": True, "T": T, "density": pden, "W": cfg.W, "d": cfg.d, "f": cfg.f,
                               "ms": ms, "form": form, "ms_gate_form": ms_gate, "ms_tc_up_form": ms_tc,
                               "tokens_per_s": T / (ms * 1e-3), "dense_ms": ms_dense,
                               "speedup_vs_own_dense": ms_dense / ms, "roofline_frac": t_roof / (ms * 1e-3),
-                              "t_roof_us": t_roof * 1e6, "n_ovf": n_o,
+                              "t_roof_us": t_roof * 1e6, "dense_roofline_frac": t_dense_roof / (ms_dense * 1e-3),
+                              "t_dense_roof_us": t_dense_roof * 1e6, "n_ovf": n_o,
                               "measured_density": float(counts.sum()) / (T * cfg.f), "status": status,
                               "cuda_graph": bool(getattr(timed, "graph", False))}),
                   flush=True)

@@ -143,10 +143,51 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
                                int skip_overflow_rows, float* y, int32_t* dev_status, void* stream);
 
 /*
+ * The same down projection per 128-row tile over the tile's union of stored
+ * units, on the tensor cores (same source as twell_sparse_down; the grouping
+ * of rows into tiles and their unions is this library's). For
+ * each tile of 128 rows, the units that its rows that fit have stored (the
+ * union, ascending) are collected, the tile's hidden values over that union
+ * are written as a bf16 block in `workspace`, and y_tile = block . Wd[union, :]
+ * runs on tcgen05 with K = the tile's union (the union's rows of Wd gathered
+ * into shared memory per K block). y as for twell_sparse_down (fp32 sums of
+ * the same exact products, in another order), except that with
+ * skip_overflow_rows != 0 the overflow rows' y is written as zeros (the
+ * dense branch rewrites it) instead of left untouched; with
+ * skip_overflow_rows == 0 they use their first W slots, their y is undefined
+ * and dev_status is raised to TWELL_ERR_OVERFLOW. workspace: at least twell_sparse_down_union_workspace_bytes(T, d, f) bytes,
+ * 16-byte aligned, caller-owned, overwritten. A stored index outside its own
+ * column tile raises TWELL_ERR_INDEX and adds nothing. Two kernel launches.
+ * It pays when the output tiles fill the GPU (twell_hybrid_down_is_union).
+ */
+twell_status twell_sparse_down_union(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
+                                     int skip_overflow_rows, float* y, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream);
+
+/* Workspace bytes of twell_sparse_down_union: about (T + 127) * f * 2 (the
+ * tiles' hidden-value blocks) plus the tiles' union lists. */
+size_t twell_sparse_down_union_workspace_bytes(int T, int d, int f);
+
+/*
+ * 1 if twell_ffn_hybrid_forward_tc_up and twell_relu_ffn_hybrid_forward run
+ * their down projection as twell_sparse_down_union for this shape on the
+ * current device with a workspace of workspace_bytes (its output tiles fill
+ * the GPU and its blocks fit the workspace, which they use only before the
+ * dense branch), 0 if as twell_sparse_down. Invalid shapes give 0.
+ */
+int twell_hybrid_down_is_union(int T, int d, int f, size_t workspace_bytes);
+
+/*
  * Hybrid forward of the tensor-core-up variant = twell_gate_up_pack,
- * twell_route, twell_sparse_down with overflowing rows skipped, and
+ * twell_route, the down projection of the rows that fit, and
  * twell_dense_rows_forward on ovf_rows. Same arguments and workspace as
- * twell_ffn_hybrid_forward.
+ * twell_ffn_hybrid_forward. When the batch's output tiles (128 rows x 256
+ * columns) fill the GPU, the down projection runs per 128-row tile over the
+ * union of the units the tile's rows that fit have stored, on the tensor
+ * cores (the tile's hidden values over its union are written as a bf16 block
+ * in the workspace, the union's rows of Wd are gathered into each K block);
+ * otherwise it is twell_sparse_down. Both sum the same exact products in
+ * fp32, in different orders.
  */
 twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                             const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
@@ -162,10 +203,11 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
 twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream);
 
 /* Bytes of workspace needed by twell_ffn_hybrid_forward and
- * twell_dense_rows_forward (worst case: every row overflows). For small
- * batches the hybrid forward also uses the hidden-activation part of it for the
- * fp32 gate pre-activations of its split-K gate GEMM, before the dense branch
- * runs. */
+ * twell_dense_rows_forward (worst case: every row overflows). For batches of
+ * 9 to 512 tokens the hybrid forward also uses the hidden-activation part of
+ * it for the fp32 gate pre-activations of its split-K gate GEMM, before the
+ * dense branch runs; for batches of at most 8 tokens the dense branch keeps its
+ * hidden activations there in fp32. */
 size_t twell_hybrid_workspace_bytes(int T, int d, int f);
 
 /*
@@ -194,6 +236,13 @@ twell_status twell_dense_rows_forward(const uint16_t* x, const uint16_t* WgT, co
  * describe this split for training and this library applies the same rule to
  * the forward pass). Every row of y is written. `workspace` holds the gathered
  * overflow rows and their hidden activations.
+ * Batches of at most 8 tokens take a CUDA-core path (a weight GEMM tile would
+ * hold 1-8 real rows): the gate is a GEMV whose epilogue makes the pack, four
+ * blocks per column tile exchanging their partial counts through distributed
+ * shared memory; routing derives the overflow flags from the counts; the dense
+ * branch is a pair of GEMVs over the listed rows with fp32 hidden activations.
+ * The same holds for twell_ffn_hybrid_forward_tc_up and
+ * twell_relu_ffn_hybrid_forward.
  */
 twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                       const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
@@ -237,7 +286,8 @@ twell_status twell_ffn_hybrid_forward_noalloc(const uint16_t* x, const uint16_t*
 /* Bytes of workspace needed by twell_dense_ffn_forward and
  * twell_relu_dense_ffn_forward: the [T][f] bf16 hidden activations, and for
  * T <= 512 room for the fp32 pre-activations ([T][2f]) of the small-batch path,
- * whose first GEMMs split K over the whole GPU. */
+ * whose first GEMMs split K over the whole GPU (batches of at most 8 tokens
+ * use two CUDA-core GEMVs instead, h in bf16 as in the GEMM path). */
 size_t twell_dense_workspace_bytes(int T, int d, int f);
 
 /*
@@ -262,8 +312,10 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
  *   caller-owned, 16-byte aligned. Shapes and the TwELL buffers as for
  *   twell_ffn_hybrid_forward; workspace of twell_hybrid_workspace_bytes(T, d, f).
  * Steps: the pack of ReLU(x W1) (its stored values are the hidden activations
- * themselves), routing, the sparse down projection over the stored slots for
- * rows that fit, and the dense layer on the tensor cores for overflow rows
+ * themselves), routing, the down projection of the stored slots for rows that
+ * fit (over tile unions on the tensor cores when the output tiles fill the
+ * GPU, as twell_ffn_hybrid_forward_tc_up does), and the dense layer on the
+ * tensor cores for overflow rows
  * (hidden values kept as bf16 plus bf16 remainder, as in the gated dense
  * branch). Errors as for twell_ffn_hybrid_forward.
  */
@@ -359,14 +411,17 @@ twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* 
 
 /*
  * Tensor-core form of twell_ffn_hybrid_backward_dx (same arguments, same
- * workspace; twell_ffn_hybrid_backward_dw or _dw_tc may follow it). The rows
- * that fit still form u and their per-slot records on the CUDA cores, but
- * their dx comes from one tcgen05 GEMM: their dz and du are scattered by
- * token into dense rows [dz | du | dz_lo | du_lo] (bf16 value plus bf16
- * remainder, zeros elsewhere) and multiplied by [Wg; Wu] read twice along K,
- * the layout the overflow rows' dense branch uses. Pays where the rows hold
- * many stored units (the GEMM's cost does not fall with density); the extra
- * error is ~2^-16 of each term.
+ * workspace; twell_ffn_hybrid_backward_dw or _dw_tc may follow it). Every
+ * dense step runs on the tensor cores: u = x Wu^T for every token is a
+ * tcgen05 GEMM beside dh = dy Wd^T (fp32, in the workspace), so the rows
+ * that fit build their per-slot records {h, du, dz} by reading u_j and dh_j
+ * instead of gathering a Wu row per stored slot; their dx then comes from one
+ * tcgen05 GEMM: their dz and du are scattered by token into dense rows
+ * [dz | du | dz_lo | du_lo] (bf16 value plus bf16 remainder, zeros elsewhere)
+ * and multiplied by [Wg; Wu] read twice along K, the layout the overflow
+ * rows' dense branch uses. Pays where the rows hold many stored units (the
+ * GEMMs' cost does not fall with density); the extra error is ~2^-16 of each
+ * term.
  */
 twell_status twell_ffn_hybrid_backward_dx_tc(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                              const uint16_t* Wd, const uint16_t* dy, int T, int d, int f,

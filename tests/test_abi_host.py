@@ -138,3 +138,30 @@ def test_backward_argument_errors(lib):
                                         FAKE, None) == tl.TWELL_ERR_WORKSPACE
     assert lib.twell_relu_ffn_hybrid_forward(FAKE, FAKE, None, 64, 128, 512, ctypes.byref(tw), FAKE, FAKE, FAKE, FAKE,
                                              1 << 30, FAKE, None) == tl.TWELL_ERR_NULL
+
+
+def test_union_down_argument_errors_and_workspace(lib):
+    T, d, f, W = 1000, 2304, 9216, 24
+    need = lib.twell_sparse_down_union_workspace_bytes(T, d, f)
+    num_m = (T + 127) // 128
+    # the tiles' hidden-value blocks, their union lists and K block counts
+    assert need >= num_m * 128 * f * 2 + num_m * f * 4 + num_m * 4 and need % 256 == 0
+    assert need <= num_m * 128 * f * 2 + num_m * f * 4 + num_m * 4 + 3 * 256
+    assert lib.twell_sparse_down_union_workspace_bytes(0, d, f) == 0
+    tw = tw_desc(T, f, W)
+    un = lib.twell_sparse_down_union
+
+    def call(d_=d, y=FAKE, ws=FAKE, wsb=need, desc=tw):
+        return un(FAKE, T, d_, f, ctypes.byref(desc), 1, y, ws, wsb, FAKE, None)
+
+    assert call(d_=100) == tl.TWELL_ERR_SHAPE
+    assert call(desc=tw_desc(T + 1, f, W)) == tl.TWELL_ERR_SHAPE
+    assert call(y=None) == tl.TWELL_ERR_NULL
+    assert call(ws=None) == tl.TWELL_ERR_WORKSPACE
+    assert call(wsb=need - 1) == tl.TWELL_ERR_WORKSPACE
+    assert call(ws=MIS) == tl.TWELL_ERR_ALIGN
+    z = tw_desc(0, f, W)
+    assert un(None, 0, d, f, ctypes.byref(z), 1, None, None, 0, None, None) == tl.TWELL_OK
+    # the form query answers 0 for invalid shapes and when no device is current
+    assert lib.twell_hybrid_down_is_union(T, 100, f, 1 << 40) == 0
+    assert lib.twell_hybrid_down_is_union(0, d, f, 1 << 40) == 0

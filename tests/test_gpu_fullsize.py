@@ -110,3 +110,90 @@ def test_full_size_tensor_core_up_hybrid_forward(name):
     rows = np.concatenate([keep, ovf[:64]])
     y_ref = np.concatenate([y_keep, O.gated_ffn(L["x"][ovf[:64]], L["WgT"], L["WuT"], L["Wd"])])
     assert_y_close(yg[rows], y_ref)
+
+
+UNION_CASES = [
+    # output tiles >= the SM count (the size the union form is built for)
+    synth.LayerConfig("union_mid", T=2400, d=2048, f=1024, tile=128, W=16, density=0.05, sigma=0.5,
+                      dead_frac=0.03),
+    # ragged T, d = 9 x 256, heavy tokens that overflow
+    synth.LayerConfig("union_heavy", T=2219, d=2304, f=2304, tile=128, W=24, density=0.012, sigma=0.5,
+                      heavy_frac=0.08, heavy_lo=0.25, heavy_hi=0.40),
+]
+
+
+def _union_against_per_token(dev, tw, T, d, f, keep):
+    """The union down projection and the per-token kernel on the same pack:
+    the same exact products summed in another order, so the rows that fit
+    agree to fp32 summation error."""
+    st = tl.new_status()
+    yu = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    wsu = torch.empty(tl.sparse_down_union_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    tl.sparse_down_union(dev["Wd"], tw, yu, True, wsu, st)
+    assert tl.status_get(st) == 0
+    y2 = torch.zeros((T, d), dtype=torch.float32, device="cuda")
+    tl.sparse_down(dev["Wd"], tw, y2, True, st)
+    assert tl.status_get(st) == 0
+    a, b = y_to_f64(yu)[keep], y_to_f64(y2)[keep]
+    assert np.isfinite(a).all()
+    rms = float(np.sqrt(np.mean(b**2)))
+    assert float(np.abs(a - b).max()) <= 1e-5 * rms
+    return a
+
+
+@pytest.mark.parametrize("cfg", UNION_CASES, ids=[c.name for c in UNION_CASES])
+def test_union_down_projection_every_row(cfg):
+    """The tensor-core-up hybrid forward on every row against the oracle's
+    result of the method, then the down projection over the tiles' unions of
+    stored units on its pack: within the stored-value bound of the oracle and
+    within fp32 summation error of the per-token kernel."""
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    L = synth.make_layer(cfg, seed=0)
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.ffn_hybrid_forward_tc_up(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    assert tl.status_get(st) == 0
+    out = O.hybrid_ffn_up_dense(L["x"], L["WgT"], L["WuT"], L["Wd"], cfg.tile, W)
+    n = int(n_ovf.item())
+    assert n == len(out["ovf_rows"])
+    assert np.array_equal(ovf_rows[:n].cpu().numpy(), out["ovf_rows"])
+    yg = y_to_f64(y)
+    assert np.isfinite(yg).all()
+    assert_y_close(yg, out["y"])
+    keep = np.setdiff1d(np.arange(T), out["ovf_rows"])
+    yu = _union_against_per_token(dev, tw, T, d, f, keep)
+    assert_within_stored_value_bound(yu, L, keep, stored="h")
+    assert_y_close(yu, out["y"][keep])
+
+
+def test_union_relu_hybrid_forward():
+    """The non-gated hybrid forward, then the union down projection on its
+    pack (which holds ReLU(x W1) itself)."""
+    cfg = UNION_CASES[1]
+    L = synth.make_layer(cfg, seed=1)
+    dev = upload(L)
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    tw = tl.Twell(T, f, W)
+    y = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    ovf_rows = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    n_ovf = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tl.hybrid_workspace_bytes(T, d, f), dtype=torch.uint8, device="cuda")
+    st = tl.new_status()
+    tl.relu_ffn_hybrid_forward(dev["x"], dev["WgT"], dev["Wd"], tw, y, ovf_rows, n_ovf, ws, st)
+    assert tl.status_get(st) == 0
+    out = O.hybrid_relu_ffn(L["x"], L["WgT"], L["Wd"], cfg.tile, W)
+    n = int(n_ovf.item())
+    assert np.array_equal(ovf_rows[:n].cpu().numpy(), out["ovf_rows"])
+    yg = y_to_f64(y)
+    assert np.isfinite(yg).all()
+    assert_y_close(yg, out["y"])
+    keep = np.setdiff1d(np.arange(T), out["ovf_rows"])
+    yu = _union_against_per_token(dev, tw, T, d, f, keep)
+    assert_y_close(yu, out["y"][keep])
