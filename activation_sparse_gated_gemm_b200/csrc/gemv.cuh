@@ -1,13 +1,14 @@
 // Batches of at most 8 tokens on the CUDA cores. A GEMM tile of 128 rows would
 // hold 1-8 rows of real data, so the tensor cores would stream the weights at
 // a fraction of HBM speed (the split-K tcgen05 path reaches ~30% of DRAM peak at
-// T = 1); here the weights stream through registers exactly once, each lane
-// keeping a ring of eight 16-byte loads per matrix in flight so that every SM
-// has ~64 KB outstanding, and the tokens' x rows wait in shared memory.
+// T = 1); here the weights stream through registers exactly once with many
+// 16-byte loads in flight per SM (32 warps of 512-thread blocks, each lane
+// issuing several loads before using any), and the tokens' x rows wait in
+// shared memory. Kernels are compiled for 1, 2, 4 and 8 tokens.
 //
 // gemv_first_kernel: z = x Wg (and u = x Wu when gated) for 32 columns per
-// block (four per warp, whose weight rows the warp reads as one contiguous
-// stream of 512-byte chunks), then, by mode,
+// block (two per warp, read in rounds of four loads per lane and matrix),
+// then, by mode,
 //  - the TwELL pack of ReLU(z) (or of h = ReLU(z) u) in the same kernel
 //    (intellectnews.ru "Sakana AI и NVIDIA ... TwELL", section "Формат TwELL
 //    вместо классической sparse-упаковки": the format is assembled at the end
@@ -18,9 +19,10 @@
 //  - the hidden activations of the dense layer (bf16, the library's dense
 //    baseline), or, for the rows routed to the dense branch, in fp32.
 // gemv_down_kernel: y[rows] += h Wd, one block per (row group of Wd, 256
-// columns of d), the grid sized to one wave; partial sums added into y.
-// Both need d to be a multiple of 256 (a 512-byte chunk never straddles two
-// weight rows); other shapes take the small-batch GEMM path.
+// columns of d), the grid sized to one wave, each lane keeping a ring of
+// eight row loads in flight; partial sums added into y.
+// Both need d to be a multiple of 256; other shapes take the small-batch GEMM
+// path.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -31,12 +33,13 @@
 namespace twell {
 
 constexpr int kGemvMaxT = 8;      // tokens per batch on this path
-constexpr int kGemvWarps = 8;
+constexpr int kGemvWarps = 16;
 constexpr int kGemvThreads = kGemvWarps * 32;
-constexpr int kGemvCols = 32;     // columns of z per block (4 per warp)
+constexpr int kGemvCols = 32;     // columns of z per block (2 per warp)
 constexpr int kGemvColsPerWarp = kGemvCols / kGemvWarps;
 constexpr int kGemvCluster = 4;   // blocks per 128-column tile in the packing modes
-constexpr int kGemvRing = 8;      // 16-byte loads in flight per lane and matrix
+constexpr int kGemvRound = 4;     // gemv_first: 16-byte loads per lane and matrix issued together
+constexpr int kGemvRing = 8;      // gemv_down: 16-byte loads in flight per lane
 constexpr int kGemvDownCols = 256;
 constexpr int kGemvDownMaxRows = 512;  // rows of Wd per block (their h values sit in shared memory)
 
@@ -92,7 +95,7 @@ __device__ __forceinline__ void gv_dot(float (&acc)[NT], const uint4* xs, int dv
 }
 
 template <int MODE, int NT>
-__global__ void __launch_bounds__(kGemvThreads, 2) gemv_first_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(kGemvThreads, NT <= 2 ? 2 : 1) gemv_first_kernel(const GemvParams p) {
   griddep_launch_dependents();
   griddep_wait();
   extern __shared__ __align__(16) uint8_t gv_smem[];
@@ -129,58 +132,47 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_first_kernel(const GemvP
 
   const int col0 = gv_pack(MODE) ? (blockIdx.x / kGemvCluster) * 128 + (blockIdx.x % kGemvCluster) * kGemvCols
                                  : blockIdx.x * kGemvCols;
-  // The warp's four weight rows are consecutive in WgT (and WuT): one stream of
-  // 512-byte chunks, cpc per row; lane l reads piece l of each chunk.
-  const int cpc = dv / 32;
-  const int nch = kGemvColsPerWarp * cpc;
-  const int jw = col0 + warp * kGemvColsPerWarp;
-  const uint4* gs = reinterpret_cast<const uint4*>(p.WgT + static_cast<size_t>(jw) * d) + lane;
-  const uint4* ust = gv_gated(MODE) ? reinterpret_cast<const uint4*>(p.WuT + static_cast<size_t>(jw) * d) + lane
-                                    : nullptr;
-  uint4 wg[kGemvRing], wu[kGemvRing];
+  // Warp w reads weight rows col0 + 2w and + 2w + 1, each in rounds of four
+  // 16-byte loads per lane and matrix, all issued before any is used.
+#pragma unroll 1
+  for (int k = 0; k < kGemvColsPerWarp; ++k) {
+    const int lc = warp * kGemvColsPerWarp + k;  // local column
+    const int j = col0 + lc;
+    float ag[NT], au[NT];
 #pragma unroll
-  for (int i = 0; i < kGemvRing; ++i) {
-    if (i < nch) {
-      wg[i] = __ldg(gs + i * 32);
-      if (gv_gated(MODE)) wu[i] = __ldg(ust + i * 32);
-    }
-  }
-  float ag[NT], au[NT];
+    for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.0f;
+    const uint4* rg = reinterpret_cast<const uint4*>(p.WgT + static_cast<size_t>(j) * d);
+    const uint4* ru = gv_gated(MODE) ? reinterpret_cast<const uint4*>(p.WuT + static_cast<size_t>(j) * d) : nullptr;
+#pragma unroll 1
+    for (int base = 0; base < dv; base += kGemvRound * 32) {
+      uint4 wg[kGemvRound], wu[kGemvRound];
 #pragma unroll
-  for (int t = 0; t < NT; ++t) ag[t] = au[t] = 0.0f;
-  int lc = 0, kc = 0;  // row within the warp's four, chunk within the row
-  for (int base = 0; base < nch; base += kGemvRing) {
+      for (int i = 0; i < kGemvRound; ++i) {
+        const int v = base + i * 32 + lane;
+        wg[i] = v < dv ? __ldg(rg + v) : make_uint4(0, 0, 0, 0);
+        if (gv_gated(MODE)) wu[i] = v < dv ? __ldg(ru + v) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (int i = 0; i < kGemvRing; ++i) {
-      const int c = base + i;
-      if (c < nch) {
-        const int v = kc * 32 + lane;
-        gv_dot<NT>(ag, xs, dv, v, n, wg[i]);
-        if (gv_gated(MODE)) gv_dot<NT>(au, xs, dv, v, n, wu[i]);
-        if (c + kGemvRing < nch) {
-          wg[i] = __ldg(gs + (c + kGemvRing) * 32);
-          if (gv_gated(MODE)) wu[i] = __ldg(ust + (c + kGemvRing) * 32);
+      for (int i = 0; i < kGemvRound; ++i) {
+        const int v = base + i * 32 + lane;
+        if (v < dv) {
+          gv_dot<NT>(ag, xs, dv, v, n, wg[i]);
+          if (gv_gated(MODE)) gv_dot<NT>(au, xs, dv, v, n, wu[i]);
         }
-        if (++kc == cpc) {
-          // the row is complete: reduce over the lanes
+      }
+    }
 #pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            if (t < n) {
-              float g = ag[t], u = au[t];
+    for (int t = 0; t < NT; ++t) {
+      if (t < n) {
+        float g = ag[t], u = au[t];
 #pragma unroll
-              for (int o = 16; o > 0; o >>= 1) {
-                g += __shfl_xor_sync(0xffffffffu, g, o);
-                if (gv_gated(MODE)) u += __shfl_xor_sync(0xffffffffu, u, o);
-              }
-              if (lane == 0) {
-                zs[t][warp * kGemvColsPerWarp + lc] = g;
-                us[t][warp * kGemvColsPerWarp + lc] = u;
-              }
-            }
-            ag[t] = au[t] = 0.0f;
-          }
-          kc = 0;
-          ++lc;
+        for (int o = 16; o > 0; o >>= 1) {
+          g += __shfl_xor_sync(0xffffffffu, g, o);
+          if (gv_gated(MODE)) u += __shfl_xor_sync(0xffffffffu, u, o);
+        }
+        if (lane == 0) {
+          zs[t][lc] = g;
+          us[t][lc] = u;
         }
       }
     }
@@ -252,7 +244,7 @@ struct GemvDownParams {
 // the slice; the warps' partial sums meet in shared memory (column-major so
 // the lanes' adds hit distinct banks), then are added into y.
 template <int NT>
-__global__ void __launch_bounds__(kGemvThreads, 2) gemv_down_kernel(const GemvDownParams p) {
+__global__ void __launch_bounds__(kGemvThreads, NT <= 2 ? 2 : 1) gemv_down_kernel(const GemvDownParams p) {
   griddep_launch_dependents();
   griddep_wait();
   __shared__ float hs[NT][kGemvDownMaxRows];

@@ -30,6 +30,12 @@ struct SparseParams {
   // units (used when T is small, to spread one token over several warps) add
   // their partial y_t into y, which must then hold zeros.
   int unit_tiles;
+  // sparse_small_kernel only: when route_n is set, block (0, 0) also routes
+  // the batch (T <= 8): route_flags[t] = (some tile of row t counts more than
+  // W), route_rows = the flagged rows ascending, *route_n = their number.
+  uint8_t* route_flags;
+  int* route_rows;
+  int* route_n;
   int* dev_status;
 };
 
@@ -319,6 +325,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
 // the slot's Wd row (and, for the gate form, its WuT row, u = x_t . Wu[:, j]
 // and h = g u), adds h Wd[j, :] into the block's copy of y_t in shared memory,
 // and the block adds that copy into y (which holds zeros in the rows written).
+// A token with a tile above W is left to the dense branch when skip_ovf is
+// set (found from its counts here); block (0, 0) also writes the routing of
+// the batch when asked, which saves the routing launch.
 constexpr int kSmallSparseWarps = 8;
 constexpr int kSmallSparseMaxTiles = 256;  // f <= 32767
 
@@ -327,13 +336,19 @@ __global__ void __launch_bounds__(kSmallSparseWarps * 32) sparse_small_kernel(co
   griddep_launch_dependents();
   griddep_wait();
   __shared__ int pre[kSmallSparseMaxTiles + 1];
+  __shared__ int over_s;
   __shared__ float ys[NCH * 256];  // y_t, element (i*32 + l)*8 + e at i*256 + e*32 + l
   __shared__ uint4 xs[DOWN_ONLY ? 1 : NCH * 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.y;
-  if (p.skip_ovf && p.row_ovf[t]) return;
-  bool overflow = false, bad_index = false;
+  // x_t and the zeroed copy of y_t do not wait for the counts
+  if (!DOWN_ONLY)
+    for (int e = threadIdx.x; e < NCH * 32; e += blockDim.x)
+      xs[e] = ldg_nc_v4(p.x + static_cast<size_t>(t) * p.d + e * 8);
+  for (int e = threadIdx.x; e < NCH * 256; e += blockDim.x) ys[e] = 0.0f;
+  bool bad_index = false;
   if (warp == 0) {
+    bool overflow = false;
     int run = 0;
     for (int cb = 0; cb < p.nT; cb += 32) {
       const int c = cb + lane;
@@ -352,17 +367,30 @@ __global__ void __launch_bounds__(kSmallSparseWarps * 32) sparse_small_kernel(co
       if (c < p.nT) pre[c] = run + incl - n;
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) pre[p.nT] = run;
-    if (__any_sync(0xffffffffu, overflow) && lane == 0 && !p.skip_ovf) raise_status(p.dev_status, kDevOverflow);
+    overflow = __any_sync(0xffffffffu, overflow);
+    if (lane == 0) {
+      pre[p.nT] = run;
+      over_s = overflow ? 1 : 0;
+      if (overflow && !p.skip_ovf) raise_status(p.dev_status, kDevOverflow);
+    }
+  } else if (warp == 1 && p.route_n != nullptr && blockIdx.x == 0 && t == 0) {
+    int n_over = 0;
+    for (int r = 0; r < p.T; ++r) {
+      bool o = false;
+      for (int c = lane; c < p.nT; c += 32) o |= p.counts[static_cast<size_t>(r) * p.nT + c] > p.W;
+      o = __any_sync(0xffffffffu, o);
+      if (lane == 0) {
+        p.route_flags[r] = o ? 1 : 0;
+        if (o) p.route_rows[n_over] = r;
+      }
+      n_over += o ? 1 : 0;
+    }
+    if (lane == 0) *p.route_n = n_over;
   }
   __syncthreads();
+  if (p.skip_ovf && over_s) return;  // the dense branch computes this row
   const int total = pre[p.nT];
   if (blockIdx.x * kSmallSparseWarps >= total) return;  // no slot for this block
-  for (int e = threadIdx.x; e < NCH * 256; e += blockDim.x) ys[e] = 0.0f;
-  if (!DOWN_ONLY)
-    for (int e = threadIdx.x; e < NCH * 32; e += blockDim.x)
-      xs[e] = ldg_nc_v4(p.x + static_cast<size_t>(t) * p.d + e * 8);
-  __syncthreads();
   const int stride = gridDim.x * kSmallSparseWarps;
 #pragma unroll 1
   for (int s = blockIdx.x * kSmallSparseWarps + warp; s < total; s += stride) {
@@ -438,24 +466,10 @@ __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf,
 // With xo given (small batches), the same block then gathers the listed rows
 // of x into xo and zeroes them in y_zero, which saves the separate gather
 // launch of the dense branch.
-//
-// With counts given (the batches of at most 8 tokens, whose pack writes no
-// flags), the block first sets row_ovf[t] = (some tile of row t counts more
-// than W nonzeros) for every row.
-__global__ void __launch_bounds__(1024) route_kernel(uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf,
-                                                     const uint16_t* x = nullptr, int d = 0, uint16_t* xo = nullptr,
-                                                     float* y_zero = nullptr, const int16_t* counts = nullptr,
-                                                     int nT = 0, int W = 0) {
+__global__ void __launch_bounds__(1024) route_kernel(const uint8_t* row_ovf, int T, int* ovf_rows, int* n_ovf,
+                                                     const uint16_t* x, int d, uint16_t* xo, float* y_zero) {
   griddep_launch_dependents();
   griddep_wait();
-  if (counts != nullptr) {
-    for (int t = threadIdx.x; t < T; t += blockDim.x) {
-      bool o = false;
-      for (int c = 0; c < nT; ++c) o |= counts[static_cast<size_t>(t) * nT + c] > W;
-      row_ovf[t] = o ? 1 : 0;
-    }
-    __syncthreads();
-  }
   __shared__ int warp_off[32];
   __shared__ int total_s;
   const int lane = threadIdx.x & 31;

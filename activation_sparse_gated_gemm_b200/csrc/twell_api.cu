@@ -344,8 +344,8 @@ twell_status sparse_small_n(const SparseParams& p, bool down_only, int sms, cuda
 }
 
 twell_status sparse_small_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
-                               const twell_t* tw, float* y, int32_t* dev_status, cudaStream_t s, int sms,
-                               bool down_only) {
+                               const twell_t* tw, float* y, int32_t* ovf_rows, int32_t* n_ovf, int32_t* dev_status,
+                               cudaStream_t s, int sms, bool down_only) {
   SparseParams p{};
   p.x = x;
   p.WuT = WuT;
@@ -361,6 +361,9 @@ twell_status sparse_small_impl(const uint16_t* x, const uint16_t* WuT, const uin
   p.nT = f / 128;
   p.W = tw->W;
   p.skip_ovf = 1;
+  p.route_flags = tw->row_ovf;
+  p.route_rows = ovf_rows;
+  p.route_n = n_ovf;
   p.dev_status = dev_status;
   switch (d / 256) {
     case 1: return sparse_small_n<1>(p, down_only, sms, s);
@@ -596,9 +599,9 @@ GemvParams gemv_params(const uint16_t* x, const uint16_t* WgT, const uint16_t* W
 }
 
 // Hybrid forward of a batch of <= 8 tokens: the pack from the GEMV (which also
-// zeroes y), routing with the flags derived from the counts, the sparse step
-// with one warp per stored slot (down only when the pack holds hidden
-// values), and the dense branch as
+// zeroes y), the sparse step with one warp per stored slot (down only when the
+// pack holds hidden values), which also routes the batch from the counts, and
+// the dense branch as
 // GEMVs over the listed rows with fp32 hidden activations (h_buf: [T][f] fp32).
 // mode: 0 gated (gate pack, fused up+down), 1 gated with hidden values, 2 non-gated.
 twell_status gemv_hybrid(int mode, const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
@@ -615,10 +618,7 @@ twell_status gemv_hybrid(int mode, const uint16_t* x, const uint16_t* WgT, const
   } else {
     TW_TRY(gemv_first<kGvPackGate>(p, s));
   }
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf,
-                static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr),
-                static_cast<const int16_t*>(tw->counts), f / 128, tw->W));
-  TW_TRY(sparse_small_impl(x, WuT, Wd, T, d, f, tw, y, dev_status, s, sms, mode != 0));
+  TW_TRY(sparse_small_impl(x, WuT, Wd, T, d, f, tw, y, ovf_rows, n_ovf, dev_status, s, sms, mode != 0));
   // the dense branch over the listed rows, hidden activations in fp32
   GemvParams b = gemv_params(x, WgT, mode == 2 ? nullptr : WuT, T, d, f, dev_status);
   b.rows = ovf_rows;
@@ -834,7 +834,7 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
   if (gemv_batch(T, d)) return gemv_hybrid(1, x, WgT, WuT, Wd, T, d, f, tw, y, ovf_rows, n_ovf,
                                         reinterpret_cast<float*>(ho), dev_status, s, sms);
   TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(hybrid_down(Wd, T, d, f, tw, y, workspace, workspace_bytes, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
@@ -846,7 +846,7 @@ twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, v
   TW_TRY(check_ptrs({ovf_rows, n_ovf}));
   int dev, sms;
   TW_TRY(current_device(&dev, &sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream), tw->row_ovf, tw->T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream), tw->row_ovf, tw->T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   return cuda_ok(cudaGetLastError());
 }
 
@@ -878,13 +878,13 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
     const bool zero_y = sparse_splits_units(T, d, false, sms);
     TW_TRY(small_gate_pack_impl(x, WgT, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
                                 dev_status, s, sms));
-    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y, static_cast<const int16_t*>(nullptr), 0, 0));
+    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y));
     TW_TRY(cuda_ok(cudaGetLastError()));
     TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms, false, zero_y));
     return dense_impl(xo, T, n_ovf, WgT, WuT, Wd, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
   TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
@@ -967,13 +967,13 @@ twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1
     const bool zero_y = sparse_splits_units(T, d, true, sms);
     TW_TRY(small_gate_pack_impl(x, W1T, T, d, f, tw, reinterpret_cast<float*>(ho), zero_y ? y : nullptr,
                                 dev_status, s, sms));
-    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y, static_cast<const int16_t*>(nullptr), 0, 0));
+    TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, x, d, xo, y));
     TW_TRY(cuda_ok(cudaGetLastError()));
     TW_TRY(sparse_impl(nullptr, nullptr, W2, T, d, f, tw, 1, y, dev_status, s, sms, true, zero_y));
     return dense_impl(xo, T, n_ovf, W1T, nullptr, W2, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
   TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms));
-  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr), static_cast<const int16_t*>(nullptr), 0, 0));
+  TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(hybrid_down(W2, T, d, f, tw, y, workspace, workspace_bytes, dev_status, s, sms));
   return dense_rows_impl(x, W1T, nullptr, W2, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);

@@ -5,7 +5,10 @@ One step = one pass of the whole hybrid forward over one batch of synthetic
 tokens: gate GEMM with the TwELL pack in its epilogue, routing, the fused
 sparse up/down step for the rows that fit, and the dense branch for the rows
 that overflow. Inputs are resident in HBM when the timed region starts; the
-L2 is flushed (a 256 MiB write) between steps, outside the timed events.
+L2 is flushed between steps, outside the timed events: a 256 MiB buffer is
+written and then read back, so the timed work starts from a cold L2 that holds
+no dirty lines (a write alone leaves ~126 MB of the flush's own write-backs to
+the first reads of the timed step).
 
 Prints one JSON line (rank 0). Also measured in the same run: the library's
 own dense FFN at the same shape (speedup denominator), the same metric end to
@@ -39,6 +42,23 @@ METRIC = "sparse gated-FFN tokens/s"
 METRIC_RELU = "sparse non-gated ReLU-FFN tokens/s"
 METRIC_BWD = "sparse gated-FFN backward tokens/s"
 FLUSH_BYTES = 256 << 20
+
+
+def layer_config(args):
+    """The configured layer, at --tokens tokens when given."""
+    cfg = synth.CONFIGS[args.config]
+    if getattr(args, "tokens", 0):
+        cfg = dataclasses.replace(cfg, T=int(args.tokens), name=f"{cfg.name}-T{int(args.tokens)}")
+    return cfg
+
+
+def flush_l2(buf) -> None:
+    """Evict L2: write a buffer larger than L2, then read it back, so the lines
+    left in L2 are clean and the timed work pays no write-back of the flush."""
+    import torch
+
+    buf.zero_()
+    buf.view(torch.int64).sum()
 FP32_LANES_PER_SM = 128  # FP32 FMA lanes per SM (4 sub-partitions x 32)
 DEFAULT_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                  "sm_max_mhz": 1965.0, "source": "fallback"}
@@ -317,7 +337,7 @@ def run_gpu(args, world, rank, local):
 
     tl.load()
     dev = torch.device("cuda", local)
-    cfg = synth.CONFIGS[args.config]
+    cfg = layer_config(args)
     L = synth.make_layer(cfg, seed=args.seed)
     x = tl.to_device_bf16(L["x"], dev)
     WgT = tl.to_device_bf16(L["WgT"], dev)
@@ -372,7 +392,7 @@ def run_gpu(args, world, rank, local):
         fns = stage_fns(variant)
         K, Wm = args.steps, args.warmup
         for _ in range(Wm):
-            flush.zero_()
+            flush_l2(flush)
             for fn in fns:
                 fn()
         torch.cuda.synchronize(dev)
@@ -384,7 +404,7 @@ def run_gpu(args, world, rank, local):
         ctx = sampler if sampler is not None else ClockSampler(None)
         with ctx:
             for k in range(K):
-                flush.zero_()
+                flush_l2(flush)
                 evs[k][0].record(stream)
                 for i, fn in enumerate(fns):
                     fn()
@@ -429,12 +449,12 @@ def run_gpu(args, world, rank, local):
             tl.dense_ffn_forward(x, WgT, WuT, Wd, y_dense, ws_dense, st)
 
     for _ in range(Wm):
-        flush.zero_()
+        flush_l2(flush)
         dense()
     dense_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     barrier(world)
     for k in range(K):
-        flush.zero_()
+        flush_l2(flush)
         dense_ev[k][0].record(stream)
         dense()
         dense_ev[k][1].record(stream)
@@ -550,7 +570,7 @@ def run_gpu(args, world, rank, local):
                                   if compact_info else ""), "variant": chosen, "compaction": compact_info,
                    "tokens": T, "d": d,
                    "f": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
-                   "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
+                   "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB written, then read back so that no dirty line is left; outside events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "roofline": {"kernel": dom, "bound": kd["bound"], "achieved": achieved, "peak": peak, "unit": kd["unit"],
                      "frac": achieved / peak, "traffic": traffic,
@@ -602,7 +622,7 @@ def run_gpu_backward(args, world, rank, local):
 
     tl.load()
     dev = torch.device("cuda", local)
-    cfg = synth.CONFIGS[args.config]
+    cfg = layer_config(args)
     L = synth.make_layer(cfg, seed=args.seed)
     dy_bits = synth.make_dy(cfg.T, cfg.d, args.seed)
     T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
@@ -635,11 +655,11 @@ def run_gpu_backward(args, world, rank, local):
         for name, tc in (("cuda_cores", False), ("tensor_cores", True)):
             fn = make(tc)
             for _ in range(Wm):
-                flush.zero_()
+                flush_l2(flush)
                 fn()
             ts = []
             for _ in range(max(3, K // 4)):
-                flush.zero_()
+                flush_l2(flush)
                 a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a_ev.record(stream)
                 fn()
@@ -668,7 +688,7 @@ def run_gpu_backward(args, world, rank, local):
     stage_dw = make_dw(dw_form == "tensor_cores")
 
     for _ in range(Wm):
-        flush.zero_()
+        flush_l2(flush)
         stage_dx()
         stage_dw()
     torch.cuda.synchronize(dev)
@@ -680,7 +700,7 @@ def run_gpu_backward(args, world, rank, local):
     torch.cuda.synchronize(dev)
     with sampler:
         for k in range(K):
-            flush.zero_()
+            flush_l2(flush)
             evs[k][0].record(stream)
             stage_dx()
             evs[k][1].record(stream)
@@ -701,12 +721,12 @@ def run_gpu_backward(args, world, rank, local):
         tl.dense_ffn_backward(x, WgT, WuT, Wd, dy, dxd, dWdn[0], dWdn[1], dWdn[2], wsd, st)
 
     for _ in range(Wm):
-        flush.zero_()
+        flush_l2(flush)
         dense_bwd()
     dense_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     barrier(world)
     for k in range(K):
-        flush.zero_()
+        flush_l2(flush)
         dense_ev[k][0].record(stream)
         dense_bwd()
         dense_ev[k][1].record(stream)
@@ -733,7 +753,7 @@ def run_gpu_backward(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize(dev)
     for k in range(K):
-        flush.zero_()
+        flush_l2(flush)
         e2e_ev[k][0].record(stream)
         e2e_step()
         e2e_ev[k][1].record(stream)
@@ -786,7 +806,7 @@ def run_gpu_backward(args, world, rank, local):
         "data": "synthetic (seeded generator; no dataset or trained weights)",
         "config": {"workload": f"{cfg.name}-like FFN layer backward through the hybrid TwELL format",
                    "tokens": T, "d": d, "f": f, "tile": cfg.tile, "ell_width": W, "density": cfg.density,
-                   "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB write, outside events)",
+                   "dead_frac": cfg.dead_frac, "l2": "flushed between steps (256 MiB written, then read back so that no dirty line is left; outside events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "roofline": {"kernel": dom, "bound": bound[dom], "achieved": achieved, "peak": peak_tf[dom],
                      "unit": "TFLOP/s", "frac": achieved / peak_tf[dom], "traffic": None,
@@ -822,7 +842,7 @@ def run_reference(args, world, rank):
     same workload; same metric and unit as the GPU arm."""
     if rank != 0:
         return None
-    cfg = synth.CONFIGS[args.config]
+    cfg = layer_config(args)
     L = synth.make_layer(cfg, seed=args.seed)
     sample = max(1, min(cfg.T, args.cpu_sample // 16))
     layer = "relu" if args.layer == "relu" else "gated"
@@ -894,7 +914,7 @@ def run_sweep(args) -> None:
                 calls capture (they are stream-ordered and never sync), so
                 small batches are not measured as launch gaps."""
                 for _ in range(args.warmup):
-                    flush.zero_()
+                    flush_l2(flush)
                     fn()
                 torch.cuda.synchronize(dev)
                 run = fn
@@ -909,7 +929,7 @@ def run_sweep(args) -> None:
                         run = fn
                 ts = []
                 for _ in range(k):
-                    flush.zero_()
+                    flush_l2(flush)
                     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     a.record()
                     run()
@@ -963,6 +983,8 @@ def main(argv=None):
     ap.add_argument("--config", default="2b", choices=sorted(synth.CONFIGS),
                     help="layer shape (default: the 2B-like hybrid layer, the largest that fits one GPU)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the configured layer on this many tokens instead (small cases for profiler captures)")
     ap.add_argument("--cpu-sample", type=int, default=12288)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", default="auto", choices=["auto", "gate", "tc_up"],
