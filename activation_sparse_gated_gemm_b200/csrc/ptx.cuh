@@ -230,6 +230,34 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+// L2 policy for data streamed once (a token's x row, its y row): evicted
+// before anything of normal priority, so the gathered weight rows stay.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ void st_stream_v4(float* addr, float a, float b, float c, float d, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d), "l"(pol)
+               : "memory");
+}
+
+__device__ __forceinline__ void red_add_stream_v4(float* addr, float a, float b, float c, float d, uint64_t pol) {
+  asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d), "l"(pol)
+               : "memory");
+}
+
 __device__ __forceinline__ void raise_status(int* dev_status, int code) {
   if (dev_status != nullptr) atomicMax(dev_status, code);
 }

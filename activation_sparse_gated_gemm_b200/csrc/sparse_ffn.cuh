@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
   uint32_t* list = reinterpret_cast<uint32_t*>(smem_dyn + WARPS * NCH * 32) + warp * kListCap;
   const int group_tiles = max(1, kListCap / p.W);
   bool overflow = false, bad_index = false;
+  // x_t, y_t and the pack pass through once: evict them first, keep the weight rows
+  const uint64_t stream_pol = l2_evict_first_policy();
   // Block b owns the contiguous tokens [t_begin, t_end); its warps take them
   // one at a time from a shared counter, so a warp that drew light tokens
   // keeps working while another finishes a heavy one.
@@ -165,7 +167,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
         const int k0 = (i * 32 + lane) * 8;
-        xs[i * 32 + lane] = (k0 < d) ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
+        xs[i * 32 + lane] = (k0 < d) ? ldg_stream_v4(p.x + static_cast<size_t>(t) * d + k0, stream_pol)
+                                     : make_uint4(0, 0, 0, 0);
       }
     }
     float y[NCH][8];
@@ -199,8 +202,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
         const size_t base = (static_cast<size_t>(t) * p.nT + c) * p.W;
         for (int k = 0; k < n; k += 8) {
           // 8 slots at a time; slots past n are read but not used (k + 8 <= W)
-          const uint4 iv = ldg_nc_v4(p.idx + base + k);
-          const uint4 vv = ldg_nc_v4(p.vals + base + k);
+          const uint4 iv = ldg_stream_v4(p.idx + base + k, stream_pol);
+          const uint4 vv = ldg_stream_v4(p.vals + base + k, stream_pol);
           const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
           const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
@@ -303,11 +306,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
       if (k0 < d) {
         float* dst = p.y + static_cast<size_t>(t) * d + k0;
         if (partial) {
-          red_add_v4(dst, y[i][0], y[i][1], y[i][2], y[i][3]);
-          red_add_v4(dst + 4, y[i][4], y[i][5], y[i][6], y[i][7]);
+          red_add_stream_v4(dst, y[i][0], y[i][1], y[i][2], y[i][3], stream_pol);
+          red_add_stream_v4(dst + 4, y[i][4], y[i][5], y[i][6], y[i][7], stream_pol);
         } else {
-          reinterpret_cast<float4*>(dst)[0] = make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
-          reinterpret_cast<float4*>(dst)[1] = make_float4(y[i][4], y[i][5], y[i][6], y[i][7]);
+          st_stream_v4(dst, y[i][0], y[i][1], y[i][2], y[i][3], stream_pol);
+          st_stream_v4(dst + 4, y[i][4], y[i][5], y[i][6], y[i][7], stream_pol);
         }
       }
     }

@@ -222,6 +222,24 @@ __device__ __forceinline__ void store_h32(const float (&h)[32], uint16_t* row_ou
   }
 }
 
+// Output tiles are visited in groups of group_n consecutive N blocks: inside
+// a group, every M block in turn with its group_n tiles side by side. The CTAs
+// running at once then share the few B tiles of one group, which stay in L2
+// while A streams past (B comes from HBM about once, A once per group); in
+// plain row order every wave would touch all of B, which at the 2B layer's
+// 85 MB of [Wg; Wu] does not stay in L2 (11x the algorithmic DRAM reads).
+constexpr size_t kGroupBBytes = 32u << 20;
+
+__device__ __forceinline__ void tile_mn(int mn, int num_m, int num_n, int group_n, int& m_blk, int& n_blk) {
+  const int per_group = group_n * num_m;
+  const int g = mn / per_group;
+  const int n0 = g * group_n;
+  const int gs = min(group_n, num_n - n0);
+  const int r = mn - g * per_group;
+  m_blk = r / gs;
+  n_blk = n0 + (r - m_blk * gs);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -330,6 +348,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   // no K block at all (an empty compact K): nothing to compute or store
   const int num_tiles = num_kb > 0 ? num_m * num_n * k_splits : 0;
+  // N blocks per group: as many as keep the group's B tiles within kGroupBBytes
+  const size_t b_bytes_n = static_cast<size_t>(kTileN) * (kStacked ? 2 : 1) * static_cast<size_t>(max(num_kb, 1)) * kBK * 2;
+  const size_t fit_n = kGroupBBytes / b_bytes_n;
+  const int group_n = fit_n < 1 ? 1 : (fit_n >= static_cast<size_t>(max(num_n, 1)) ? max(num_n, 1) : static_cast<int>(fit_n));
 
   const uint32_t tmem_base = *tmem_slot;
 
@@ -343,8 +365,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mn = tile / k_splits;
         const int ks = tile - mn * k_splits;
-        const int m_blk = mn / num_n;
-        const int n_blk = mn - m_blk * num_n;
+        int m_blk, n_blk;
+        tile_mn(mn, num_m, num_n, group_n, m_blk, n_blk);
         int kb_begin = ks * kb_per, kb_end = min(num_kb, (ks + 1) * kb_per);
         const int* urows = nullptr;
         int slabs = 4;
@@ -452,7 +474,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int kb_begin = ks * kb_per, kb_end = min(num_kb, (ks + 1) * kb_per);
         if (MODE == kModeUnion) {
           kb_begin = 0;
-          kb_end = min(max(p.kb_tile[(tile / k_splits) / num_n], 0), num_kb);
+          int m_u, n_u;
+          tile_mn(tile / k_splits, num_m, num_n, group_n, m_u, n_u);
+          kb_end = min(max(p.kb_tile[m_u], 0), num_kb);
         }
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag)) {
@@ -518,8 +542,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const int mn = tile / k_splits;
-      const int m_blk = mn / num_n;
-      const int n_blk = mn - m_blk * num_n;
+      int m_blk, n_blk;
+      tile_mn(mn, num_m, num_n, group_n, m_blk, n_blk);
       const uint32_t t_row = tmem_base + static_cast<uint32_t>(buf * kBN) + (static_cast<uint32_t>(q * 32) << 16);
       const int row_base = m_blk * kBM + q * 32;
       const int my_row = row_base + lane;
