@@ -91,12 +91,10 @@ constexpr int kEpiBytes = kEpiWarps * 32 * kEpiPitch * 4;
 constexpr int kGemmThreads = 64 + kEpiThreads;
 constexpr int kTmemCols = 512;  // two 256-column fp32 accumulators
 
-constexpr int kStageSlotBytes = 32;  // per epilogue thread: 8 staged (idx, value) slots
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kAStageBytes;
 constexpr int kOffEpi = kOffB + kStages * kBStageBytes;
-constexpr int kOffSlots = kOffEpi + kEpiBytes;
-constexpr int kOffBar = kOffSlots + kEpiThreads * kStageSlotBytes;
+constexpr int kOffBar = kOffEpi + kEpiBytes;
 constexpr int kNumBars = 2 * kStages + 4 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kGemmSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024 (misc: TMEM base, abort flag, K splits)
@@ -167,39 +165,52 @@ struct GemmParams {
 };
 
 
+// The last eight (column, bf16 value) slots of one row's list, held in
+// registers: a push shifts both 128-bit queues down by one 16-bit entry and
+// enters the new one at the top, so after eight pushes entry k sits at bits
+// 16k..16k+15 and the group leaves as one 16-byte store per array.
+struct SlotQueue {
+  uint32_t i0 = 0, i1 = 0, i2 = 0, i3 = 0, v0 = 0, v1 = 0, v2 = 0, v3 = 0;
+};
+
+__device__ __forceinline__ void q_push(SlotQueue& q, uint32_t idx16, uint32_t val16) {
+  q.i0 = __funnelshift_r(q.i0, q.i1, 16);
+  q.i1 = __funnelshift_r(q.i1, q.i2, 16);
+  q.i2 = __funnelshift_r(q.i2, q.i3, 16);
+  q.i3 = __funnelshift_r(q.i3, idx16, 16);
+  q.v0 = __funnelshift_r(q.v0, q.v1, 16);
+  q.v1 = __funnelshift_r(q.v1, q.v2, 16);
+  q.v2 = __funnelshift_r(q.v2, q.v3, 16);
+  q.v3 = __funnelshift_r(q.v3, val16, 16);
+}
+
+__device__ __forceinline__ void q_store(const SlotQueue& q, int16_t* gidx, uint16_t* gval) {
+  *reinterpret_cast<uint4*>(gidx) = make_uint4(q.i0, q.i1, q.i2, q.i3);
+  *reinterpret_cast<uint4*>(gval) = make_uint4(q.v0, q.v1, q.v2, q.v3);
+}
+
 // Appends the set bits of `mask` (column col0 + i, bf16 value vrow[i]) to one
-// row's slot list of a TwELL tile in ascending column order, staging 8 slots
-// at a time in shared memory and storing each full group with 16-byte stores.
+// row's slot list of a TwELL tile in ascending column order, storing each full
+// group of 8 with 16-byte stores.
 __device__ __forceinline__ void twell_append(uint32_t mask, const uint16_t* vrow, int col0, int& cnt, int W,
-                                             uint16_t* stg_idx, uint16_t* stg_val, int16_t* gidx,
-                                             uint16_t* gval) {
+                                             SlotQueue& q, int16_t* gidx, uint16_t* gval) {
   while (mask != 0) {
     const int i = __ffs(mask) - 1;
     mask &= mask - 1u;
     if (cnt < W) {
-      const int k = cnt & 7;
-      stg_idx[k] = static_cast<uint16_t>(col0 + i);
-      stg_val[k] = vrow[i];
-      if (k == 7) {
-        *reinterpret_cast<uint4*>(gidx + (cnt - 7)) = *reinterpret_cast<const uint4*>(stg_idx);
-        *reinterpret_cast<uint4*>(gval + (cnt - 7)) = *reinterpret_cast<const uint4*>(stg_val);
-      }
+      q_push(q, static_cast<uint32_t>(col0 + i), vrow[i]);
+      if ((cnt & 7) == 7) q_store(q, gidx + (cnt - 7), gval + (cnt - 7));
     }
     ++cnt;
   }
 }
 
 // Stores the last partial group of a row's slot list, padded with (-1, 0).
-__device__ __forceinline__ void twell_close(int cnt, int W, uint16_t* stg_idx, uint16_t* stg_val, int16_t* gidx,
-                                            uint16_t* gval) {
+__device__ __forceinline__ void twell_close(int cnt, int W, SlotQueue& q, int16_t* gidx, uint16_t* gval) {
   const int n = min(cnt, W);
   if (n & 7) {
-    for (int k = n & 7; k < 8; ++k) {
-      stg_idx[k] = 0xFFFFu;
-      stg_val[k] = 0;
-    }
-    *reinterpret_cast<uint4*>(gidx + (n & ~7)) = *reinterpret_cast<const uint4*>(stg_idx);
-    *reinterpret_cast<uint4*>(gval + (n & ~7)) = *reinterpret_cast<const uint4*>(stg_val);
+    for (int k = n & 7; k < 8; ++k) q_push(q, 0xFFFFu, 0u);
+    q_store(q, gidx + (n & ~7), gval + (n & ~7));
   }
 }
 
@@ -555,78 +566,97 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // row's slot list. Slots go through an 8-entry staging buffer in shared
         // memory and leave as 16-byte stores.
         uint32_t* vrow = ebuf + lane * kEpiPitch;
-        uint8_t* stg = smem + kOffSlots + (threadIdx.x - 64) * kStageSlotBytes;
-        uint16_t* stg_idx = reinterpret_cast<uint16_t*>(stg);
-        uint16_t* stg_val = reinterpret_cast<uint16_t*>(stg + 16);
         const bool row_ok = my_row < M;
-#pragma unroll 1
-        for (int sub = 0; sub < 2; ++sub) {
-          const int c = n_blk * 2 + sub;  // TwELL column tile
+        // The 8 chunks of 32 columns (TwELL tiles 2 n_blk and 2 n_blk + 1,
+        // four chunks each) come out of TMEM one ahead of the walk: chunk k + 1
+        // is in flight while chunk k is walked.
+        int cnt = 0;  // nonzeros of my_row in the current tile so far (not capped)
+        SlotQueue q;
+        auto walk = [&](const uint32_t (&r)[32], int k) {
+          const int c = n_blk * 2 + (k >> 2);  // TwELL column tile
           const bool tile_ok = row_ok && c < p.nT;
           const size_t slot0 = (static_cast<size_t>(my_row) * p.nT + c) * p.W;
-          int cnt = 0;  // nonzeros of my_row in tile c so far (not capped)
-#pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t r[32];
-            __syncwarp();
-            tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(sub * 128 + ch * 32), r);
-            tmem_wait_ld();
-            if (sub == 1 && ch == 3) {
-              tc_fence_before();
-              mbar_arrive(&tempty[buf]);
-            }
-            if (!tile_ok) continue;
+          if ((k & 3) == 0) cnt = 0;
+          if (tile_ok) {
             uint32_t mask = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) mask |= (static_cast<int32_t>(r[i]) > 0 ? 1u : 0u) << i;
-            if (mask == 0) continue;
+            if (mask != 0) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) vrow[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            twell_append(mask, reinterpret_cast<const uint16_t*>(vrow), c * 128 + ch * 32, cnt, p.W, stg_idx,
-                         stg_val, p.idx + slot0, p.vals + slot0);
+              for (int i = 0; i < 16; ++i) vrow[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              twell_append(mask, reinterpret_cast<const uint16_t*>(vrow), c * 128 + (k & 3) * 32, cnt, p.W, q,
+                           p.idx + slot0, p.vals + slot0);
+            }
+            if ((k & 3) == 3) {
+              twell_close(cnt, p.W, q, p.idx + slot0, p.vals + slot0);
+              p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
+              if (cnt > p.W) p.row_ovf[my_row] = 1;
+            }
           }
-          if (tile_ok) {
-            twell_close(cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
-            p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
-            if (cnt > p.W) p.row_ovf[my_row] = 1;
+        };
+        uint32_t ra[32], rb[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(t_row, ra);
+#pragma unroll 1
+        for (int k = 0; k < 8; k += 2) {
+          tmem_wait_ld(ra);  // chunk k is in ra
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((k + 1) * 32), rb);
+          walk(ra, k);
+          tmem_wait_ld(rb);  // chunk k + 1 is in rb
+          if (k == 6) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
+          } else {
+            __syncwarp();
+            tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((k + 2) * 32), ra);
           }
+          walk(rb, k + 1);
         }
       } else if (MODE == kModeTwellHidden) {
         // Same pattern as above from z (columns 0..127 of the accumulator),
         // value h = z * u with u in columns 128..255.
         uint32_t* vrow = ebuf + lane * kEpiPitch;
-        uint8_t* stg = smem + kOffSlots + (threadIdx.x - 64) * kStageSlotBytes;
-        uint16_t* stg_idx = reinterpret_cast<uint16_t*>(stg);
-        uint16_t* stg_val = reinterpret_cast<uint16_t*>(stg + 16);
         const int c = n_blk;  // the 128 hidden units of this tile are TwELL tile c
         const bool tile_ok = my_row < M && c < p.nT;
         const size_t slot0 = (static_cast<size_t>(my_row) * p.nT + c) * p.W;
         int cnt = 0;
+        SlotQueue q;
+        // Chunk k's mask and bf16 values go to registers and shared memory
+        // first; then chunk k + 1's loads are issued into the same registers and
+        // the walk of chunk k runs while they are in flight.
+        uint32_t zr[32], ur[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(t_row, zr);
+        tmem_ld_32x32b_x32(t_row + 128u, ur);
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
-          uint32_t zr[32], ur[32];
-          __syncwarp();
-          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), zr);
-          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + ch * 32), ur);
-          tmem_wait_ld();
-          if (ch == 3) {
-            tc_fence_before();
-            mbar_arrive(&tempty[buf]);
-          }
-          if (!tile_ok) continue;
+          tmem_wait_ld(zr);
+          tmem_wait_ld(ur);
           uint32_t mask = 0;
 #pragma unroll
           for (int i = 0; i < 32; ++i) mask |= (static_cast<int32_t>(zr[i]) > 0 ? 1u : 0u) << i;
-          if (mask == 0) continue;
+          if (!tile_ok) mask = 0;
+          if (mask != 0) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            vrow[i] = pack_bf16x2(__uint_as_float(zr[2 * i]) * __uint_as_float(ur[2 * i]),
-                                  __uint_as_float(zr[2 * i + 1]) * __uint_as_float(ur[2 * i + 1]));
-          twell_append(mask, reinterpret_cast<const uint16_t*>(vrow), c * 128 + ch * 32, cnt, p.W, stg_idx,
-                       stg_val, p.idx + slot0, p.vals + slot0);
+            for (int i = 0; i < 16; ++i)
+              vrow[i] = pack_bf16x2(__uint_as_float(zr[2 * i]) * __uint_as_float(ur[2 * i]),
+                                    __uint_as_float(zr[2 * i + 1]) * __uint_as_float(ur[2 * i + 1]));
+          }
+          if (ch == 3) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
+          } else {
+            __syncwarp();
+            tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((ch + 1) * 32), zr);
+            tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + (ch + 1) * 32), ur);
+          }
+          if (mask != 0)
+            twell_append(mask, reinterpret_cast<const uint16_t*>(vrow), c * 128 + ch * 32, cnt, p.W, q,
+                         p.idx + slot0, p.vals + slot0);
         }
         if (tile_ok) {
-          twell_close(cnt, p.W, stg_idx, stg_val, p.idx + slot0, p.vals + slot0);
+          twell_close(cnt, p.W, q, p.idx + slot0, p.vals + slot0);
           p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
           if (cnt > p.W) p.row_ovf[my_row] = 1;
         }
