@@ -446,6 +446,47 @@ __global__ void __launch_bounds__(kSmallSparseWarps * 32) sparse_small_kernel(co
   }
 }
 
+// The dense branch's hidden activations of the overflowing rows in the tiles
+// that did not overflow: all of their nonzeros are in the pack (as bf16 h), so
+// the slot's row of H gets them over zeros, with a zero remainder (the tiles
+// that overflowed were written, exact, by the gate+up GEMM). Slot s holds row
+// slot_row[s]; the slot's row of y is zeroed for the branch's partial sums.
+// One warp per (slot, tile), lane l owning units 4l..4l+3.
+__global__ void __launch_bounds__(256) ovf_fill_kernel(const int16_t* counts, const int16_t* idx, const uint16_t* vals,
+                                                       int nT, int W, int f, const int* slot_row, const int* n_slots,
+                                                       uint16_t* H, float* y, int d) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const long long n = static_cast<long long>(max(*n_slots, 0)) * nT;
+  for (long long u = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); u < n; u += warps) {
+    const int sl = static_cast<int>(u / nT), c = static_cast<int>(u - static_cast<long long>(sl) * nT);
+    const int t = slot_row[sl];
+    if (c == 0) {
+      float4* yr = reinterpret_cast<float4*>(y + static_cast<size_t>(t) * d);
+      for (int k = lane; k < d / 4; k += 32) yr[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const size_t at = static_cast<size_t>(t) * nT + c;
+    const int cnt = counts[at];
+    if (cnt > W) continue;  // written by the gate+up GEMM
+    uint32_t h01 = 0, h23 = 0;
+    for (int k = 0; k < cnt; ++k) {
+      const int j = static_cast<int>(idx[at * W + k]) - c * 128;
+      if ((j >> 2) == lane) {
+        const uint32_t v = vals[at * W + k];
+        if ((j & 3) == 0) h01 |= v;
+        else if ((j & 3) == 1) h01 |= v << 16;
+        else if ((j & 3) == 2) h23 |= v;
+        else h23 |= v << 16;
+      }
+    }
+    uint16_t* hrow = H + static_cast<size_t>(sl) * 2 * f;
+    *reinterpret_cast<uint2*>(hrow + c * 128 + 4 * lane) = make_uint2(h01, h23);
+    *reinterpret_cast<uint2*>(hrow + f + c * 128 + 4 * lane) = make_uint2(0u, 0u);
+  }
+}
+
 // y[t, :] = 0 for the rows the sparse step will write (all rows, or those
 // without the overflow flag when overflow rows are skipped).
 __global__ void zero_rows_kernel(float* y, int T, int d, const uint8_t* row_ovf, int skip_ovf) {

@@ -229,9 +229,17 @@ twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d
 }
 
 // Gate and up GEMM in one pass; TwELL of the gate pattern holding h = z * u.
+// With slot_of_row set, the GEMM also writes the exact h of every overflowing
+// (row, tile) into ovf_h at the row's compact slot (see GemmParams).
 twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, int T, int d, int f,
-                               const twell_t* tw, int32_t* dev_status, cudaStream_t s, int sms) {
-  TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
+                               const twell_t* tw, int32_t* dev_status, cudaStream_t s, int sms,
+                               int* slot_of_row = nullptr, int* slot_row = nullptr, int* ovf_n = nullptr,
+                               uint16_t* ovf_h = nullptr) {
+  if (slot_of_row != nullptr) {
+    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), slot_of_row, static_cast<size_t>(T) * 4, ovf_n, 4));
+  } else {
+    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
+  }
   CUtensorMap ma, mg, mu;
   if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128))
     return TWELL_ERR_CUDA;
@@ -245,6 +253,10 @@ twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uin
   p.row_ovf = tw->row_ovf;
   p.nT = f / 128;
   p.W = tw->W;
+  p.slot_of_row = slot_of_row;
+  p.slot_row = slot_row;
+  p.ovf_n = ovf_n;
+  p.ovf_h = ovf_h;
   p.dev_status = dev_status;
   return launch_gemm<kModeTwellHidden>(ma, mg, mu, p, gemm_grid(T, f, 128, sms), s);
 }
@@ -833,11 +845,23 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
                                              round_up(static_cast<size_t>(T) * d * 2, 256));
   if (gemv_batch(T, d)) return gemv_hybrid(1, x, WgT, WuT, Wd, T, d, f, tw, y, ovf_rows, n_ovf,
                                         reinterpret_cast<float*>(ho), dev_status, s, sms);
-  TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms));
+  // The dense branch takes its hidden activations from the gate+up GEMM (the
+  // overflowing tiles, exact) and the pack (the others): no second gate and up
+  // GEMM over the routed rows. The x-gather region holds the slot tables.
+  int* slot_of_row = reinterpret_cast<int*>(xo);
+  int* slot_row = slot_of_row + T;
+  int* n_slots = slot_row + T;
+  TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms, slot_of_row, slot_row, n_slots, ho));
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(hybrid_down(Wd, T, d, f, tw, y, workspace, workspace_bytes, dev_status, s, sms));
-  return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
+  const long long pairs = static_cast<long long>(T) * (f / 128);
+  TW_TRY(launch(ovf_fill_kernel, dim3(static_cast<unsigned>(std::max(1LL, std::min<long long>((pairs + 7) / 8, 4LL * sms)))),
+                dim3(256), 0, s, static_cast<const int16_t*>(tw->counts), static_cast<const int16_t*>(tw->idx),
+                static_cast<const uint16_t*>(tw->vals), f / 128, tw->W, f, static_cast<const int*>(slot_row),
+                static_cast<const int*>(n_slots), ho, y, d));
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  return dense_down_impl(ho, T, n_slots, Wd, d, f, true, slot_row, y, T, dev_status, s, sms);
 }
 
 twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream) {

@@ -161,6 +161,16 @@ struct GemmParams {
   const int* kb_tile;
   const int* union_rows;
   int union_stride;
+  // kModeTwellHidden, optional (ovf_h set): the dense branch's hidden
+  // activations of the overflowing rows, written here for their overflowing
+  // tiles. A row's first overflowing tile claims a compact slot s (slot_of_row
+  // holds s + 1, 0 while unclaimed, -1 while being claimed; slot_row[s] = the
+  // row; *ovf_n counts the slots) and the tile's exact h goes to row s of
+  // ovf_h ([slots][2 N] bf16: h at column j, h - bf16(h) at N + j).
+  int* slot_of_row;
+  int* slot_row;
+  int* ovf_n;
+  uint16_t* ovf_h;
   int* dev_status;
 };
 
@@ -643,13 +653,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               vrow[i] = pack_bf16x2(__uint_as_float(zr[2 * i]) * __uint_as_float(ur[2 * i]),
                                     __uint_as_float(zr[2 * i + 1]) * __uint_as_float(ur[2 * i + 1]));
           }
-          if (ch == 3) {
-            tc_fence_before();
-            mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
-          } else {
+          if (ch < 3) {
             __syncwarp();
             tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((ch + 1) * 32), zr);
             tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + (ch + 1) * 32), ur);
+          } else if (p.ovf_h == nullptr) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
           }
           if (mask != 0)
             twell_append(mask, reinterpret_cast<const uint16_t*>(vrow), c * 128 + ch * 32, cnt, p.W, q,
@@ -659,6 +669,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           twell_close(cnt, p.W, q, p.idx + slot0, p.vals + slot0);
           p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
           if (cnt > p.W) p.row_ovf[my_row] = 1;
+        }
+        if (p.ovf_h != nullptr) {
+          // An overflowing tile's exact h for the dense branch, read again from
+          // TMEM (the accumulator is released only after this).
+          const bool over = tile_ok && cnt > p.W;
+          if (__any_sync(0xffffffffu, over)) {
+            int sl = 0;
+            if (over) {
+              volatile int* so = p.slot_of_row + my_row;
+              sl = *so;
+              if (sl == 0) {
+                const int old = atomicCAS(p.slot_of_row + my_row, 0, -1);
+                if (old == 0) {
+                  const int sn = atomicAdd(p.ovf_n, 1);
+                  p.slot_row[sn] = my_row;
+                  __threadfence();
+                  atomicExch(p.slot_of_row + my_row, sn + 1);
+                  sl = sn + 1;
+                } else {
+                  sl = old;
+                }
+              }
+              // another tile of this row is claiming: a few instructions away
+              for (int it = 0; sl < 0 && it < (1 << 22); ++it) sl = *so;
+              if (sl <= 0) raise_status(p.dev_status, kDevTimeout);
+            }
+            uint16_t* hrow = sl > 0 ? p.ovf_h + static_cast<size_t>(sl - 1) * 2 * p.N : nullptr;
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+              __syncwarp();
+              tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), zr);
+              tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(128 + ch * 32), ur);
+              tmem_wait_ld(zr);
+              tmem_wait_ld(ur);
+              if (hrow != nullptr) {
+                float h[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) h[i] = fmaxf(__uint_as_float(zr[i]), 0.0f) * __uint_as_float(ur[i]);
+                store_h32(h, hrow, c * 128 + ch * 32, p.N, true);
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
         }
       } else if (MODE == kModeGateUp) {
 #pragma unroll 1

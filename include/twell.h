@@ -178,16 +178,17 @@ size_t twell_sparse_down_union_workspace_bytes(int T, int d, int f);
 int twell_hybrid_down_is_union(int T, int d, int f, size_t workspace_bytes);
 
 /*
- * Hybrid forward of the tensor-core-up variant = twell_gate_up_pack,
- * twell_route, the down projection of the rows that fit, and
- * twell_dense_rows_forward on ovf_rows. Same arguments and workspace as
- * twell_ffn_hybrid_forward. When the batch's output tiles (128 rows x 256
- * columns) fill the GPU, the down projection runs per 128-row tile over the
- * union of the units the tile's rows that fit have stored, on the tensor
- * cores (the tile's hidden values over its union are written as a bf16 block
- * in the workspace, the union's rows of Wd are gathered into each K block);
- * otherwise it is twell_sparse_down. Both sum the same exact products in
- * fp32, in different orders.
+ * Hybrid forward of the tensor-core-up variant: twell_gate_up_pack,
+ * twell_route, twell_sparse_down of the rows that fit (overflow rows
+ * skipped), and the dense branch on ovf_rows. Same arguments and workspace as
+ * twell_ffn_hybrid_forward. The dense branch does not recompute the gate and
+ * up GEMMs: the gate+up GEMM writes each overflowing (row, tile)'s exact
+ * hidden activations h = ReLU(z) u (bf16 value and bf16 remainder) into the
+ * workspace at the row's compact slot, the row's other tiles take their
+ * nonzeros from the pack (bf16 h, every nonzero of a tile that fits is
+ * stored), and one down GEMM adds them times Wd into the zeroed rows of y.
+ * Batches of at most 8 tokens (d a multiple of 256) run the GEMV path of
+ * twell_ffn_hybrid_forward with the hidden values packed.
  */
 twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                             const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
