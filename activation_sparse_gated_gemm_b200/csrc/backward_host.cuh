@@ -150,12 +150,9 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
     // sums added into zeroed rows, when the output tiles cannot fill it.
     uint16_t* a2all = reinterpret_cast<uint16_t*>(w.zu);
     const long long dx_tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN);
-    if (dx_tiles < sms)
-      TW_TRY(zero_async(s, sms, a2all, static_cast<size_t>(T) * 4 * f * 2, dx, static_cast<size_t>(T) * d * 4));
-    else
-      TW_TRY(zero_async(s, sms, a2all, static_cast<size_t>(T) * 4 * f * 2));
+    if (dx_tiles < sms) TW_TRY(zero_async(s, sms, dx, static_cast<size_t>(T) * d * 4));
     SlotSource src{tw->counts, tw->idx, w.rec, tw->row_ovf, T, nullptr, nT, tw->W, f, 1};
-    TW_TRY(launch(bwd_scatter_rows_kernel, dim3(4 * sms), dim3(256), 0, s, src, a2all));
+    TW_TRY(launch(bwd_dense_rows_kernel, dim3(8 * sms), dim3(256), 0, s, src, a2all));
     CUtensorMap ma, mgT, muT;
     if (!make_map(&ma, a2all, 4 * f, T, kBK, kBM) || !make_map(&mgT, WgT, d, f, 64, kBK) ||
         !make_map(&muT, WuT, d, f, 64, kBK))
