@@ -285,18 +285,24 @@ twell_status backward_dw_overflow(int d, int f, const int32_t* n_ovf, float* dWg
 }
 
 // Tensor-core form of the weight gradients from the workspace filled by
-// backward_dx_impl: the rows that fit are scattered densely (bf16 value and
-// remainder) by unit and token, three GEMMs over all tokens give their share,
-// then the overflow rows' GEMMs add theirs.
+// backward_dx_impl: the records of the rows that fit are sorted by column and
+// written densely (bf16 value and remainder) by unit and token, three GEMMs
+// over all tokens give their share, then the overflow rows' GEMMs add theirs.
 twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, int d, int f, const twell_t* tw,
                                  const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd, char* ws,
                                  cudaStream_t s, int sms) {
   const int nT = f / 128;
   BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
   const size_t block = static_cast<size_t>(f) * 2 * w.t_pad;
-  TW_TRY(zero_async(s, sms, w.dense, 3 * block * 2));
   SlotSource a{tw->counts, tw->idx, w.rec, tw->row_ovf, T, nullptr, nT, tw->W, f, 1};
-  TW_TRY(launch(bwd_scatter_dense_kernel, dim3(4 * sms), dim3(256), 0, s, a, w.t_pad, w.dense));
+  TW_TRY(zero_async(s, sms, w.colcnt, static_cast<size_t>(f) * 4));
+  const int cblocks = 4 * sms;
+  TW_TRY(launch(bwd_columns_kernel<false>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
+  TW_TRY(launch(bwd_column_scan_kernel, dim3(1), dim3(1024), 0, s, w.colcnt, f, w.colptr));
+  TW_TRY(launch(bwd_columns_kernel<true>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
+  TW_TRY(launch(bwd_dense_units_kernel, dim3(static_cast<unsigned>(std::min(f, 8 * sms))), dim3(256), 0, s,
+                static_cast<const int*>(w.colptr), static_cast<const float4*>(w.list), f, w.t_pad, w.dense));
+  TW_TRY(cuda_ok(cudaGetLastError()));
   // K runs over all tokens; rows of x and dy past T read as zeros
   const bool split = static_cast<long long>(f / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms;
   const uint16_t* bT[3] = {x, x, dy};
