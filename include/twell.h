@@ -400,9 +400,10 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
  * Tensor-core form of twell_ffn_hybrid_backward_dw (same arguments, same
  * workspace, called after twell_ffn_hybrid_backward_dx). At densities where
  * every unit is active for many tokens of a batch, the weight gradients are a
- * dense contraction over the tokens: the rows that fit scatter their dz, du
- * and h (as bf16 value plus bf16 remainder) by unit and token into dense
- * blocks, three tcgen05 GEMMs over all tokens form their share, and the
+ * dense contraction over the tokens: the records of the rows that fit are
+ * sorted by unit and their dz, du and h written (as bf16 value plus bf16
+ * remainder) by unit and token into dense blocks, one unit's rows at a time;
+ * three tcgen05 GEMMs over all tokens form their share, and the
  * overflow rows' GEMMs add theirs. The extra error is ~2^-16 of each term; the
  * sums are in fp32 in a fixed order.
  */
@@ -417,7 +418,7 @@ twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* 
  * tcgen05 GEMM beside dh = dy Wd^T (fp32, in the workspace), so the rows
  * that fit build their per-slot records {h, du, dz} by reading u_j and dh_j
  * instead of gathering a Wu row per stored slot; their dx then comes from one
- * tcgen05 GEMM: their dz and du are scattered by token into dense rows
+ * tcgen05 GEMM: their dz and du are written by token into dense rows
  * [dz | du | dz_lo | du_lo] (bf16 value plus bf16 remainder, zeros elsewhere)
  * and multiplied by [Wg; Wu] read twice along K, the layout the overflow
  * rows' dense branch uses. Pays where the rows hold many stored units (the
