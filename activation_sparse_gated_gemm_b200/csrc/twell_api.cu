@@ -417,18 +417,6 @@ size_t union_bytes(int T, int f) {
   return round_up(num_m * kBM * f * 2, 256) + round_up(num_m * f * 4, 256) + round_up(num_m * 4, 256);
 }
 
-// Whether the hybrid forwards take the union form. Measured on B200 it loses
-// to the per-token kernel at every configured layer (0.5B, 1.5B and 2B), so
-// the forwards keep the per-token kernel; the union form stays an explicit
-// entry point. When enabled it needs output tiles that fill the GPU at least
-// once (below that the per-token kernel spreads a token over several warps).
-constexpr bool kUnionInHybrid = false;
-
-bool union_selected(int T, int d, int f, size_t workspace_bytes, int sms) {
-  const long long tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN);
-  return kUnionInHybrid && tiles >= sms && union_bytes(T, f) <= workspace_bytes;
-}
-
 // y (rows that fit) = per 128-row tile, the tile's hidden values over its
 // union of stored units times those rows of Wd, on the tensor cores.
 twell_status union_down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip, float* y,
@@ -468,16 +456,6 @@ twell_status union_down_impl(const uint16_t* Wd, int T, int d, int f, const twel
   p.union_stride = f;
   p.dev_status = dev_status;
   return launch_gemm<kModeUnion>(ma, mb, mb, p, gemm_grid(T, d, kBN, sms), s);
-}
-
-// The down projection of the hybrid forwards whose pack holds the hidden
-// activations (overflow rows skipped): over tile unions on the tensor cores
-// when that fills the GPU and fits the caller's workspace (used only until the
-// dense branch, which runs after), else the per-token kernel.
-twell_status hybrid_down(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, float* y, void* ws,
-                         size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms) {
-  if (union_selected(T, d, f, ws_bytes, sms)) return union_down_impl(Wd, T, d, f, tw, 1, y, ws, dev_status, s, sms);
-  return down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms);
 }
 
 // Dense FFN over A rows (x itself, or gathered overflow rows): h = ReLU(A Wg) * (A Wu), or
@@ -820,11 +798,14 @@ twell_status twell_sparse_down_union(const uint16_t* Wd, int T, int d, int f, co
                          static_cast<cudaStream_t>(stream), sms);
 }
 
+// The union form measured slower than the per-token kernel at every
+// configured layer (0.5B, 1.5B and 2B), so the hybrid forwards never take it.
 int twell_hybrid_down_is_union(int T, int d, int f, size_t workspace_bytes) {
-  if (check_shape(T, d, f) != TWELL_OK || T == 0) return 0;
-  int dev, sms;
-  if (current_device(&dev, &sms) != TWELL_OK) return 0;
-  return union_selected(T, d, f, workspace_bytes, sms) ? 1 : 0;
+  (void)T;
+  (void)d;
+  (void)f;
+  (void)workspace_bytes;
+  return 0;
 }
 
 twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
@@ -854,7 +835,7 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
   TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms, slot_of_row, slot_row, n_slots, ho));
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(hybrid_down(Wd, T, d, f, tw, y, workspace, workspace_bytes, dev_status, s, sms));
+  TW_TRY(down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms));
   const long long pairs = static_cast<long long>(T) * (f / 128);
   TW_TRY(launch(ovf_fill_kernel, dim3(static_cast<unsigned>(std::max(1LL, std::min<long long>((pairs + 7) / 8, 4LL * sms)))),
                 dim3(256), 0, s, static_cast<const int16_t*>(tw->counts), static_cast<const int16_t*>(tw->idx),
@@ -999,7 +980,7 @@ twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1
   TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms));
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(hybrid_down(W2, T, d, f, tw, y, workspace, workspace_bytes, dev_status, s, sms));
+  TW_TRY(down_impl(W2, T, d, f, tw, 1, y, dev_status, s, sms));
   return dense_rows_impl(x, W1T, nullptr, W2, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
 }
 

@@ -367,16 +367,11 @@ def run_gpu(args, world, rank, local):
     # The two forms of the hybrid forward: "gate" packs ReLU(z) and runs the
     # fused sparse up+down step; "tc_up" forms u on the tensor cores with the
     # gate and packs h, leaving only the down projection sparse.
-    # the down projection of the tc_up and non-gated forms, as the library's
-    # hybrid forwards run it for this shape (over tile unions on the tensor
-    # cores, its blocks in the hybrid workspace, or per token)
-    down_union = tl.hybrid_down_is_union(T, d, f, ws.numel())
-
+    # the down projection of the tc_up and non-gated forms (per token; the
+    # union form on the tensor cores is an explicit entry point the forwards
+    # do not use)
     def down():
-        if down_union:
-            tl.sparse_down_union(Wd, tw, y, True, ws, st)
-        else:
-            tl.sparse_down(Wd, tw, y, True, st)
+        tl.sparse_down(Wd, tw, y, True, st)
 
     def stage_fns(variant):
         if variant == "relu":  # the non-gated layer ReLU(x W1) W2 with W1 = Wg, W2 = Wd
@@ -620,8 +615,7 @@ def run_gpu(args, world, rank, local):
         # per step: zeroing, gate (or gate+up) GEMM, routing, sparse step, row gather, two dense-branch GEMMs
         # (the down projection over tile unions is two launches: its preparation and its GEMM)
         "gpu_launches": (6 if chosen == "tc_up" else 7) * K,
-        "down_projection": ("fused up+down per token" if chosen == "gate" else
-                            "over tile unions on the tensor cores" if down_union else "per token"),
+        "down_projection": "fused up+down per token" if chosen == "gate" else "per token",
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -150,7 +150,8 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
  * union, ascending) are collected, the tile's hidden values over that union
  * are written as a bf16 block in `workspace`, and y_tile = block . Wd[union, :]
  * runs on tcgen05 with K = the tile's union (the union's rows of Wd gathered
- * into shared memory per K block). y as for twell_sparse_down (fp32 sums of
+ * into shared memory per K block by TMA, four rows per instruction). y as for
+ * twell_sparse_down (fp32 sums of
  * the same exact products, in another order), except that with
  * skip_overflow_rows != 0 the overflow rows' y is written as zeros (the
  * dense branch rewrites it) instead of left untouched; with
@@ -158,7 +159,9 @@ twell_status twell_sparse_down(const uint16_t* Wd, int T, int d, int f, const tw
  * and dev_status is raised to TWELL_ERR_OVERFLOW. workspace: at least twell_sparse_down_union_workspace_bytes(T, d, f) bytes,
  * 16-byte aligned, caller-owned, overwritten. A stored index outside its own
  * column tile raises TWELL_ERR_INDEX and adds nothing. Two kernel launches.
- * It pays when the output tiles fill the GPU (twell_hybrid_down_is_union).
+ * Measured on B200 it is slower than twell_sparse_down at the 0.5B, 1.5B and
+ * 2B layers (the row gather is the wall), so the hybrid forwards do not use
+ * it.
  */
 twell_status twell_sparse_down_union(const uint16_t* Wd, int T, int d, int f, const twell_t* tw,
                                      int skip_overflow_rows, float* y, void* workspace, size_t workspace_bytes,
@@ -169,11 +172,10 @@ twell_status twell_sparse_down_union(const uint16_t* Wd, int T, int d, int f, co
 size_t twell_sparse_down_union_workspace_bytes(int T, int d, int f);
 
 /*
- * 1 if twell_ffn_hybrid_forward_tc_up and twell_relu_ffn_hybrid_forward run
- * their down projection as twell_sparse_down_union for this shape on the
- * current device with a workspace of workspace_bytes (its output tiles fill
- * the GPU and its blocks fit the workspace, which they use only before the
- * dense branch), 0 if as twell_sparse_down. Invalid shapes give 0.
+ * 1 if twell_ffn_hybrid_forward_tc_up and twell_relu_ffn_hybrid_forward would
+ * run their down projection as twell_sparse_down_union for this shape and
+ * workspace, 0 if as twell_sparse_down. Always 0: the union form is an
+ * explicit entry point only (see above).
  */
 int twell_hybrid_down_is_union(int T, int d, int f, size_t workspace_bytes);
 
