@@ -208,9 +208,17 @@ int gemm_grid(int M, int N, int tile_n, int sms) {
   return static_cast<int>(tiles < sms ? (tiles > 0 ? tiles : 1) : sms);
 }
 
+// With slot_of_row set, the GEMM also writes the exact ReLU(z) of every
+// overflowing (row, tile) into ovf_h at the row's compact slot (see GemmParams).
 twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
-                            int32_t* dev_status, cudaStream_t s, int sms, const int* M_dev = nullptr) {
-  TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
+                            int32_t* dev_status, cudaStream_t s, int sms, const int* M_dev = nullptr,
+                            int* slot_of_row = nullptr, int* slot_row = nullptr, int* ovf_n = nullptr,
+                            uint16_t* ovf_h = nullptr) {
+  if (slot_of_row != nullptr) {
+    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), slot_of_row, static_cast<size_t>(T) * 4, ovf_n, 4));
+  } else {
+    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
+  }
   CUtensorMap ma, mb;
   if (!make_map(&ma, x, d, T, kBK, kBM) || !make_map(&mb, WgT, d, f, kBK, kBN)) return TWELL_ERR_CUDA;
   GemmParams p{};
@@ -224,6 +232,10 @@ twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d
   p.row_ovf = tw->row_ovf;
   p.nT = f / 128;
   p.W = tw->W;
+  p.slot_of_row = slot_of_row;
+  p.slot_row = slot_row;
+  p.ovf_n = ovf_n;
+  p.ovf_h = ovf_h;
   p.dev_status = dev_status;
   return launch_gemm<kModeTwell>(ma, mb, mb, p, M_dev ? sms : gemm_grid(T, f, kBN, sms), s);
 }
@@ -808,6 +820,25 @@ int twell_hybrid_down_is_union(int T, int d, int f, size_t workspace_bytes) {
   return 0;
 }
 
+namespace {
+
+// The dense branch over the compact slots that the pack GEMM claimed for the
+// routed rows (their overflowing tiles' exact h already in ho): the other
+// tiles' h from the pack (a bf16 value and a zero remainder), the rows of y
+// zeroed, then y[slot_row[s]] = [h | h_lo][s] [Wd; Wd].
+twell_status slot_branch_impl(const twell_t* tw, const uint16_t* Wd, int T, int d, int f, const int* slot_row,
+                              const int* n_slots, uint16_t* ho, float* y, int32_t* dev_status, cudaStream_t s,
+                              int sms) {
+  const long long pairs = static_cast<long long>(T) * (f / 128);
+  TW_TRY(launch(ovf_fill_kernel, dim3(static_cast<unsigned>(std::max(1LL, std::min<long long>((pairs + 7) / 8, 4LL * sms)))),
+                dim3(256), 0, s, static_cast<const int16_t*>(tw->counts), static_cast<const int16_t*>(tw->idx),
+                static_cast<const uint16_t*>(tw->vals), f / 128, tw->W, f, slot_row, n_slots, ho, y, d));
+  TW_TRY(cuda_ok(cudaGetLastError()));
+  return dense_down_impl(ho, T, n_slots, Wd, d, f, true, slot_row, y, T, dev_status, s, sms);
+}
+
+}  // namespace
+
 twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
                                             const uint16_t* Wd, int T, int d, int f, const twell_t* tw, float* y,
                                             int32_t* ovf_rows, int32_t* n_ovf, void* workspace,
@@ -836,13 +867,7 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms));
-  const long long pairs = static_cast<long long>(T) * (f / 128);
-  TW_TRY(launch(ovf_fill_kernel, dim3(static_cast<unsigned>(std::max(1LL, std::min<long long>((pairs + 7) / 8, 4LL * sms)))),
-                dim3(256), 0, s, static_cast<const int16_t*>(tw->counts), static_cast<const int16_t*>(tw->idx),
-                static_cast<const uint16_t*>(tw->vals), f / 128, tw->W, f, static_cast<const int*>(slot_row),
-                static_cast<const int*>(n_slots), ho, y, d));
-  TW_TRY(cuda_ok(cudaGetLastError()));
-  return dense_down_impl(ho, T, n_slots, Wd, d, f, true, slot_row, y, T, dev_status, s, sms);
+  return slot_branch_impl(tw, Wd, T, d, f, slot_row, n_slots, ho, y, dev_status, s, sms);
 }
 
 twell_status twell_route(const twell_t* tw, int32_t* ovf_rows, int32_t* n_ovf, void* stream) {
@@ -977,11 +1002,18 @@ twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1
     TW_TRY(sparse_impl(nullptr, nullptr, W2, T, d, f, tw, 1, y, dev_status, s, sms, true, zero_y));
     return dense_impl(xo, T, n_ovf, W1T, nullptr, W2, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
-  TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms));
+  // As in the tensor-core-up form, the dense branch takes the routed rows' h
+  // from the pack GEMM (the overflowing tiles, exact) and the pack (the
+  // others) instead of a second GEMM over them; the x-gather region holds the
+  // slot tables.
+  int* slot_of_row = reinterpret_cast<int*>(xo);
+  int* slot_row = slot_of_row + T;
+  int* n_slots = slot_row + T;
+  TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms, nullptr, slot_of_row, slot_row, n_slots, ho));
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
   TW_TRY(down_impl(W2, T, d, f, tw, 1, y, dev_status, s, sms));
-  return dense_rows_impl(x, W1T, nullptr, W2, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
+  return slot_branch_impl(tw, W2, T, d, f, slot_row, n_slots, ho, y, dev_status, s, sms);
 }
 
 twell_status twell_relu_dense_rows_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2, int T, int d,

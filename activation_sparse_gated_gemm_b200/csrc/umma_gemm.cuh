@@ -161,9 +161,9 @@ struct GemmParams {
   const int* kb_tile;
   const int* union_rows;
   int union_stride;
-  // kModeTwellHidden, optional (ovf_h set): the dense branch's hidden
-  // activations of the overflowing rows, written here for their overflowing
-  // tiles. A row's first overflowing tile claims a compact slot s (slot_of_row
+  // kModeTwellHidden and kModeTwell, optional (ovf_h set): the dense branch's
+  // hidden activations of the overflowing rows, written here for their
+  // overflowing tiles (h = ReLU(z) u, or ReLU(z) for the non-gated layer). A row's first overflowing tile claims a compact slot s (slot_of_row
   // holds s + 1, 0 while unclaimed, -1 while being claimed; slot_row[s] = the
   // row; *ovf_n counts the slots) and the tile's exact h goes to row s of
   // ovf_h ([slots][2 N] bf16: h at column j, h - bf16(h) at N + j).
@@ -241,6 +241,32 @@ __device__ __forceinline__ void store_h32(const float (&h)[32], uint16_t* row_ou
 #pragma unroll
     for (int v = 0; v < 4; ++v) dlo[v] = make_uint4(lv[4 * v], lv[4 * v + 1], lv[4 * v + 2], lv[4 * v + 3]);
   }
+}
+
+// The compact dense-branch slot of `row`, claimed by the first of its
+// overflowing tiles to get here: returns s + 1 (see GemmParams::slot_of_row),
+// or 0 after raising a timeout status if another tile's claim never lands.
+__device__ __forceinline__ int claim_ovf_slot(const GemmParams& p, int row) {
+  volatile int* so = p.slot_of_row + row;
+  int sl = *so;
+  if (sl == 0) {
+    const int old = atomicCAS(p.slot_of_row + row, 0, -1);
+    if (old == 0) {
+      const int sn = atomicAdd(p.ovf_n, 1);
+      p.slot_row[sn] = row;
+      __threadfence();
+      atomicExch(p.slot_of_row + row, sn + 1);
+      return sn + 1;
+    }
+    sl = old;
+  }
+  // another tile of this row is claiming: a few instructions away
+  for (int it = 0; sl < 0 && it < (1 << 22); ++it) sl = *so;
+  if (sl <= 0) {
+    raise_status(p.dev_status, kDevTimeout);
+    return 0;
+  }
+  return sl;
 }
 
 // Output tiles are visited in groups of group_n consecutive N blocks: inside
@@ -581,6 +607,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // four chunks each) come out of TMEM one ahead of the walk: chunk k + 1
         // is in flight while chunk k is walked.
         int cnt = 0;  // nonzeros of my_row in the current tile so far (not capped)
+        int over2 = 0;  // bit i: TwELL tile 2 n_blk + i of my_row overflowed
         SlotQueue q;
         auto walk = [&](const uint32_t (&r)[32], int k) {
           const int c = n_blk * 2 + (k >> 2);  // TwELL column tile
@@ -600,7 +627,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if ((k & 3) == 3) {
               twell_close(cnt, p.W, q, p.idx + slot0, p.vals + slot0);
               p.counts[static_cast<size_t>(my_row) * p.nT + c] = static_cast<int16_t>(cnt);
-              if (cnt > p.W) p.row_ovf[my_row] = 1;
+              if (cnt > p.W) {
+                p.row_ovf[my_row] = 1;
+                over2 |= 1 << (k >> 2);
+              }
             }
           }
         };
@@ -614,14 +644,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((k + 1) * 32), rb);
           walk(ra, k);
           tmem_wait_ld(rb);  // chunk k + 1 is in rb
-          if (k == 6) {
-            tc_fence_before();
-            mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
-          } else {
+          if (k < 6) {
             __syncwarp();
             tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>((k + 2) * 32), ra);
+          } else if (p.ovf_h == nullptr) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
           }
           walk(rb, k + 1);
+        }
+        if (p.ovf_h != nullptr) {
+          // The overflowing tiles' exact h = ReLU(z) for the dense branch, read
+          // again from TMEM (the accumulator is released only after this).
+          if (__any_sync(0xffffffffu, over2 != 0)) {
+            const int sl = over2 != 0 ? claim_ovf_slot(p, my_row) : 0;
+            uint16_t* hrow = sl > 0 ? p.ovf_h + static_cast<size_t>(sl - 1) * 2 * p.N : nullptr;
+#pragma unroll 1
+            for (int k = 0; k < 8; ++k) {
+              const bool mine = ((over2 >> (k >> 2)) & 1) != 0;
+              if (!__any_sync(0xffffffffu, mine)) continue;
+              __syncwarp();
+              tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(k * 32), ra);
+              tmem_wait_ld(ra);
+              if (hrow != nullptr && mine) {
+                float h[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) h[i] = fmaxf(__uint_as_float(ra[i]), 0.0f);
+                store_h32(h, hrow, (n_blk * 2 + (k >> 2)) * 128 + (k & 3) * 32, p.N, true);
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[buf]);  // all 256 columns are out of TMEM
         }
       } else if (MODE == kModeTwellHidden) {
         // Same pattern as above from z (columns 0..127 of the accumulator),
@@ -675,26 +729,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // TMEM (the accumulator is released only after this).
           const bool over = tile_ok && cnt > p.W;
           if (__any_sync(0xffffffffu, over)) {
-            int sl = 0;
-            if (over) {
-              volatile int* so = p.slot_of_row + my_row;
-              sl = *so;
-              if (sl == 0) {
-                const int old = atomicCAS(p.slot_of_row + my_row, 0, -1);
-                if (old == 0) {
-                  const int sn = atomicAdd(p.ovf_n, 1);
-                  p.slot_row[sn] = my_row;
-                  __threadfence();
-                  atomicExch(p.slot_of_row + my_row, sn + 1);
-                  sl = sn + 1;
-                } else {
-                  sl = old;
-                }
-              }
-              // another tile of this row is claiming: a few instructions away
-              for (int it = 0; sl < 0 && it < (1 << 22); ++it) sl = *so;
-              if (sl <= 0) raise_status(p.dev_status, kDevTimeout);
-            }
+            const int sl = over ? claim_ovf_slot(p, my_row) : 0;
             uint16_t* hrow = sl > 0 ? p.ovf_h + static_cast<size_t>(sl - 1) * 2 * p.N : nullptr;
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {

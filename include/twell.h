@@ -315,12 +315,15 @@ twell_status twell_dense_ffn_forward(const uint16_t* x, const uint16_t* WgT, con
  *   caller-owned, 16-byte aligned. Shapes and the TwELL buffers as for
  *   twell_ffn_hybrid_forward; workspace of twell_hybrid_workspace_bytes(T, d, f).
  * Steps: the pack of ReLU(x W1) (its stored values are the hidden activations
- * themselves), routing, the down projection of the stored slots for rows that
- * fit (over tile unions on the tensor cores when the output tiles fill the
- * GPU, as twell_ffn_hybrid_forward_tc_up does), and the dense layer on the
- * tensor cores for overflow rows
- * (hidden values kept as bf16 plus bf16 remainder, as in the gated dense
- * branch). Errors as for twell_ffn_hybrid_forward.
+ * themselves), routing, the per-token down projection of the stored slots for
+ * rows that fit (twell_sparse_down), and the dense layer on the tensor cores
+ * for overflow rows (hidden values kept as bf16 plus bf16 remainder, as in
+ * the gated dense branch). Past the small-batch paths the dense branch does
+ * not recompute x W1 over the routed rows: as in
+ * twell_ffn_hybrid_forward_tc_up, the pack GEMM writes each overflowing
+ * (row, tile)'s exact ReLU(z) into the workspace at the row's compact slot and
+ * the row's other tiles take theirs from the pack. Errors as for
+ * twell_ffn_hybrid_forward.
  */
 twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1T, const uint16_t* W2,
                                            int T, int d, int f, const twell_t* tw, float* y,
