@@ -147,7 +147,9 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
     // the tensor cores, the rows that fit scattered token-major into the
     // [z | u] region (dh there is no longer needed), overflow rows left zero
     // (their dx is rewritten below). K is split over the grid, with partial
-    // sums added into zeroed rows, when the output tiles cannot fill it.
+    // sums added into zeroed rows, when the output tiles cannot fill it (a
+    // split that only shortens the last wave measured slower here: the
+    // zeroing and the added partial sums of dx cost more than it saves).
     uint16_t* a2all = reinterpret_cast<uint16_t*>(w.zu);
     const long long dx_tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN);
     if (dx_tiles < sms) TW_TRY(zero_async(s, sms, dx, static_cast<size_t>(T) * d * 4));
@@ -303,8 +305,10 @@ twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, i
   TW_TRY(launch(bwd_dense_units_kernel, dim3(static_cast<unsigned>(std::min(f, 8 * sms))), dim3(256), 0, s,
                 static_cast<const int*>(w.colptr), static_cast<const float4*>(w.list), f, w.t_pad, w.dense));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  // K runs over all tokens; rows of x and dy past T read as zeros
-  const bool split = static_cast<long long>(f / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms;
+  // K runs over all tokens; rows of x and dy past T read as zeros. K is split
+  // whenever that shortens the last wave of output tiles (e.g. 192 tiles on
+  // 148 SMs: three splits, 1.33 waves instead of 2), the partial sums added
+  // into zeroed outputs.
   const uint16_t* bT[3] = {x, x, dy};
   float* outs[3] = {dWgT, dWuT, dWd};
   for (int i = 0; i < 3; ++i) {
@@ -318,9 +322,10 @@ twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, i
     q.k_wrap = w.t_pad;  // [value | remainder] halves against the same rows of x (or dy)
     q.out_f32 = outs[i];
     q.ldo = d;
-    q.k_splits_max = split ? 32 : 1;
-    if (split) TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
-    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, split ? sms : gemm_grid(f, d, kBN, sms), s));
+    q.k_splits_max = 32;
+    q.split_waves = 1;
+    TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
+    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, sms, s));
   }
   return backward_dw_overflow(d, f, n_ovf, dWgT, dWuT, dWd, w, s, sms);
 }

@@ -1254,12 +1254,13 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
   }
   TW_TRY(launch_gemm<kModeDown>(ma2, mgT, muT, q3, q3.k_splits_max > 1 ? sms : gemm_grid(T, d, kBN, sms), s));
   // dWgT = dz^T x, dWuT = du^T x, dWd = h^T dy (K = the tokens; rows of x and
-  // dy past T are read as zeros by the tensor maps)
+  // dy past T are read as zeros by the tensor maps). As in the hybrid's
+  // tensor-core weight gradients, K is split whenever that shortens the last
+  // wave of output tiles, the partial sums added into zeroed outputs.
   const size_t tblock = static_cast<size_t>(f) * tp;
   const uint16_t* aT[3] = {tT, tT + tblock, tT + 2 * tblock};
   const uint16_t* bT[3] = {x, x, dy};
   float* outs[3] = {dWgT, dWuT, dWd};
-  const bool split = static_cast<long long>(f / kBM) * ((d + kBN - 1) / kBN) * 2 <= sms;
   for (int i = 0; i < 3; ++i) {
     CUtensorMap ma, mb;
     if (!make_map(&ma, aT[i], tp, f, kBK, kBM) || !make_map(&mb, bT[i], d, T, 64, kBK)) return TWELL_ERR_CUDA;
@@ -1269,10 +1270,11 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
     q.K = tp;
     q.out_f32 = outs[i];
     q.ldo = d;
-    q.k_splits_max = split ? 32 : 1;
+    q.k_splits_max = 32;
+    q.split_waves = 1;
     q.dev_status = dev_status;
-    if (split) TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
-    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, split ? sms : gemm_grid(f, d, kBN, sms), s));
+    TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
+    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, sms, s));
   }
   return TWELL_OK;
 }

@@ -410,7 +410,9 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
  * remainder) by unit and token into dense blocks, one unit's rows at a time;
  * three tcgen05 GEMMs over all tokens form their share, and the
  * overflow rows' GEMMs add theirs. The extra error is ~2^-16 of each term; the
- * sums are in fp32 in a fixed order.
+ * sums are in fp32, with K (the tokens) split over the GPU where that shortens
+ * the GEMMs' last wave, the partial sums added atomically (so not
+ * bit-reproducible from run to run).
  */
 twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* dy, int T, int d, int f,
                                              const twell_t* tw, const int32_t* n_ovf, float* dWgT, float* dWuT,
