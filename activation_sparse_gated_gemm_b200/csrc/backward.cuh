@@ -513,54 +513,17 @@ __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
   }
 }
 
-// Tensor-core form of the weight gradients: the records of the rows that fit,
-// written into three unit-major blocks dense[b][j][2 t_pad] (b = dz, du, h):
-// bf16(v) at token t and the bf16 remainder v - bf16(v) at t_pad + t, zeros
-// elsewhere. Three GEMMs over [tokens | tokens] against [x; x] (or dy) then
-// give dWg, dWu, dWd with ~2^-16 relative error per term. One block per unit
-// j, from the records sorted by column (colptr, list): the block zeroes the
-// unit's three rows and then writes its records into them while they are in
-// L2 (a memset of the 3 f 2 t_pad block followed by 2-byte stores scattered
-// over all of it took 0.82 ms at the 0.5B layer).
-__global__ void __launch_bounds__(256) bwd_dense_units_kernel(const int* colptr, const float4* list, int f,
-                                                              int t_pad, uint16_t* __restrict__ dense) {
-  griddep_launch_dependents();
-  griddep_wait();
-  const size_t row = 2 * static_cast<size_t>(t_pad);
-  const size_t block = static_cast<size_t>(f) * row;
-  for (int j = blockIdx.x; j < f; j += gridDim.x) {
-#pragma unroll
-    for (int b = 0; b < 3; ++b) {
-      uint4* r = reinterpret_cast<uint4*>(dense + b * block + static_cast<size_t>(j) * row);
-      for (int i = threadIdx.x; i < static_cast<int>(row / 8); i += blockDim.x) r[i] = make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();
-    const int e0 = colptr[j], e1 = colptr[j + 1];
-    for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
-      const float4 rec = list[e];
-      const int t = __float_as_int(rec.w);
-      if (t < 0 || t >= t_pad) continue;
-      const size_t o = static_cast<size_t>(j) * row + t;
-      const float v[3] = {rec.z, rec.y, rec.x};  // dz, du, h
-#pragma unroll
-      for (int b = 0; b < 3; ++b) {
-        const uint16_t hi = f32_to_bf16_bits(v[b]);
-        dense[b * block + o] = hi;
-        dense[b * block + o + t_pad] = f32_to_bf16_bits(v[b] - __uint_as_float(static_cast<uint32_t>(hi) << 16));
-      }
-    }
-    __syncthreads();  // the next unit's zeros go to other rows; keep the block in step
-  }
-}
-
-// Tensor-core form of dx: the records of the rows that fit, written as
-// token-major rows a2[t][4f] = [dz | du | dz_lo | du_lo] (bf16 value, then the
-// bf16 remainder v - bf16(v); zeros where no slot is stored, and for the rows
-// that overflow), the layout of the overflow rows' dense branch, so that one
-// GEMM against [Wg; Wu] (read twice along K) gives dx for every token. One warp
-// per (row, tile), lane l owning units 4l..4l+3: every byte of the block is
+// Tensor-core forms: the records of the rows that fit, written as token-major
+// rows a2[t][4f] = [dz | du | dz_lo | du_lo] (bf16 value, then the bf16
+// remainder v - bf16(v); zeros where no slot is stored, and for the rows that
+// overflow), the layout of the overflow rows' dense branch, so that one GEMM
+// against [Wg; Wu] (read twice along K) gives dx for every token. WITH_H: rows
+// a2[t][6f] that also hold [h | h_lo], from which the weight-gradient GEMMs
+// read dz, du and h with the tokens as K (an MN-major A operand). One warp per
+// (row, tile), lane l owning units 4l..4l+3: every byte of the block is
 // written once with 8-byte stores that a warp makes contiguous (a memset of
 // the block and 2-byte scattered stores into it took 0.27 ms at the 0.5B layer).
+template <bool WITH_H>
 __global__ void __launch_bounds__(256) bwd_dense_rows_kernel(SlotSource src, uint16_t* __restrict__ a2) {
   griddep_launch_dependents();
   griddep_wait();
@@ -572,7 +535,8 @@ __global__ void __launch_bounds__(256) bwd_dense_rows_kernel(SlotSource src, uin
        w += nw) {
     const int t = static_cast<int>(w / src.nT);
     const int c = static_cast<int>(w - static_cast<long long>(t) * src.nT);
-    float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // dz, du of my four units
+    constexpr int kVals = WITH_H ? 3 : 2;
+    float v[3][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // dz, du, h of my four units
     if (!src.row_ovf[t]) {
       const int n = min(max(static_cast<int>(src.counts[w]), 0), src.W);
       for (int k = 0; k < n; ++k) {
@@ -585,18 +549,21 @@ __global__ void __launch_bounds__(256) bwd_dense_rows_kernel(SlotSource src, uin
             if ((j & 3) == e) {
               v[0][e] = rec.z;
               v[1][e] = rec.y;
+              v[2][e] = rec.x;
             }
         }
       }
     }
-    uint16_t* row = a2 + static_cast<size_t>(t) * 4 * f + static_cast<size_t>(c) * 128 + 4 * lane;
+    uint16_t* row = a2 + static_cast<size_t>(t) * (WITH_H ? 6 : 4) * f + static_cast<size_t>(c) * 128 + 4 * lane;
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kVals; ++b) {
       const uint32_t h01 = pack_bf16x2(v[b][0], v[b][1]), h23 = pack_bf16x2(v[b][2], v[b][3]);
       const uint32_t l01 = pack_bf16x2(v[b][0] - __uint_as_float(h01 << 16), v[b][1] - __uint_as_float(h01 & 0xffff0000u));
       const uint32_t l23 = pack_bf16x2(v[b][2] - __uint_as_float(h23 << 16), v[b][3] - __uint_as_float(h23 & 0xffff0000u));
-      *reinterpret_cast<uint2*>(row + b * f) = make_uint2(h01, h23);
-      *reinterpret_cast<uint2*>(row + (2 + b) * f) = make_uint2(l01, l23);
+      // value and remainder columns: dz 0 and 2f, du f and 3f, h 4f and 5f
+      const size_t hi_col = b < 2 ? b * f : 4 * f, lo_col = b < 2 ? (2 + b) * f : 5 * f;
+      *reinterpret_cast<uint2*>(row + hi_col) = make_uint2(h01, h23);
+      *reinterpret_cast<uint2*>(row + lo_col) = make_uint2(l01, l23);
     }
   }
 }

@@ -13,8 +13,8 @@
 // du, h ([f][2 Tp] bf16 each); the column counts/cursors ([f]), column
 // offsets ([f + 1]) and the column-sorted records (one float4 per slot of the
 // rows that fit); for the tensor-core form of the weight gradients, the rows
-// that fit as dense unit-major dz, du, h ([3][f][2 Tp] bf16, value and
-// remainder).
+// that fit as dense token-major [dz | du | dz_lo | du_lo | h | h_lo] ([T][6f]
+// bf16, within a region of 6 f Tp elements).
 struct BwdWorkspace {
   float4* rec;
   uint16_t *xo, *dyo;
@@ -22,7 +22,7 @@ struct BwdWorkspace {
   uint16_t *a2, *tT;
   int *colcnt, *colptr;
   float4* list;
-  uint16_t* dense;  // tensor-core form: dz, du, h of the rows that fit, [3][f][2 Tp] bf16 (value, remainder)
+  uint16_t* dense;  // tensor-core form: the rows that fit, [T][6f] bf16 (dz, du, their remainders, h, its remainder)
   int t_pad;
   size_t bytes;
 };
@@ -154,7 +154,7 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
     const long long dx_tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((d + kBN - 1) / kBN);
     if (dx_tiles < sms) TW_TRY(zero_async(s, sms, dx, static_cast<size_t>(T) * d * 4));
     SlotSource src{tw->counts, tw->idx, w.rec, tw->row_ovf, T, nullptr, nT, tw->W, f, 1};
-    TW_TRY(launch(bwd_dense_rows_kernel, dim3(8 * sms), dim3(256), 0, s, src, a2all));
+    TW_TRY(launch(bwd_dense_rows_kernel<false>, dim3(8 * sms), dim3(256), 0, s, src, a2all));
     CUtensorMap ma, mgT, muT;
     if (!make_map(&ma, a2all, 4 * f, T, kBK, kBM) || !make_map(&mgT, WgT, d, f, 64, kBK) ||
         !make_map(&muT, WuT, d, f, 64, kBK))
@@ -295,31 +295,34 @@ twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, i
                                  cudaStream_t s, int sms) {
   const int nT = f / 128;
   BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
-  const size_t block = static_cast<size_t>(f) * 2 * w.t_pad;
+  // The records of the rows that fit, token-major: [dz | du | dz_lo | du_lo |
+  // h | h_lo] (6 f bf16 per token, in the region of 6 f t_pad elements that
+  // the weight gradients own). The three GEMMs read them as an MN-major A
+  // (units along M, tokens along K), so no transposition by unit is needed.
   SlotSource a{tw->counts, tw->idx, w.rec, tw->row_ovf, T, nullptr, nT, tw->W, f, 1};
-  TW_TRY(zero_async(s, sms, w.colcnt, static_cast<size_t>(f) * 4));
-  const int cblocks = 4 * sms;
-  TW_TRY(launch(bwd_columns_kernel<false>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
-  TW_TRY(launch(bwd_column_scan_kernel, dim3(1), dim3(1024), 0, s, w.colcnt, f, w.colptr));
-  TW_TRY(launch(bwd_columns_kernel<true>, dim3(cblocks), dim3(256), 0, s, a, w.colcnt, w.colptr, w.list));
-  TW_TRY(launch(bwd_dense_units_kernel, dim3(static_cast<unsigned>(std::min(f, 8 * sms))), dim3(256), 0, s,
-                static_cast<const int*>(w.colptr), static_cast<const float4*>(w.list), f, w.t_pad, w.dense));
+  uint16_t* rows = w.dense;
+  TW_TRY(launch(bwd_dense_rows_kernel<true>, dim3(8 * sms), dim3(256), 0, s, a, rows));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  // K runs over all tokens; rows of x and dy past T read as zeros. K is split
-  // whenever that shortens the last wave of output tiles (e.g. 192 tiles on
-  // 148 SMs: three splits, 1.33 waves instead of 2), the partial sums added
-  // into zeroed outputs.
+  CUtensorMap ma;
+  if (!make_map(&ma, rows, 6 * static_cast<uint64_t>(f), T, 64, kBK)) return TWELL_ERR_CUDA;
+  // K runs over the tokens twice (values, then remainders); rows of the block,
+  // x and dy past T read as zeros. K is split whenever that shortens the last
+  // wave of output tiles (e.g. 192 tiles on 148 SMs: three splits, 1.33 waves
+  // instead of 2), the partial sums added into zeroed outputs.
   const uint16_t* bT[3] = {x, x, dy};
   float* outs[3] = {dWgT, dWuT, dWd};
+  const int col_hi[3] = {0, f, 4 * f}, col_lo[3] = {2 * f, 3 * f, 5 * f};
   for (int i = 0; i < 3; ++i) {
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, w.dense + i * block, 2 * w.t_pad, f, kBK, kBM) || !make_map(&mb, bT[i], d, T, 64, kBK))
-      return TWELL_ERR_CUDA;
+    CUtensorMap mb;
+    if (!make_map(&mb, bT[i], d, T, 64, kBK)) return TWELL_ERR_CUDA;
     GemmParams q{};
     q.M = f;
     q.N = d;
     q.K = 2 * w.t_pad;
     q.k_wrap = w.t_pad;  // [value | remainder] halves against the same rows of x (or dy)
+    q.a_mn_major = 1;
+    q.a_col_hi = col_hi[i];
+    q.a_col_lo = col_lo[i];
     q.out_f32 = outs[i];
     q.ldo = d;
     q.k_splits_max = 32;

@@ -140,6 +140,13 @@ struct GemmParams {
   // multiple of 8); the A rows past them in shared memory hold stale data that
   // only reaches accumulator rows the epilogue never stores.
   int a_box_rows;
+  // kModeDown: A stored MN-major, i.e. as [K][...] rows with the M index
+  // contiguous (tmA covers that array; boxes of 64 M columns by 64 K rows).
+  // K block k reads rows k mod k_wrap at columns a_col_hi + m (k < k_wrap, or
+  // k_wrap == 0) or a_col_lo + m (k >= k_wrap): the value and remainder halves
+  // of one token-major block.
+  int a_mn_major;
+  int a_col_hi, a_col_lo;
   const int* row_map;  // kModeDown: output row of each A row, or null
   int out_rows;        // valid range of output rows
   // kModeGateUp / kModeRelu: also store h_lo = bf16(h - bf16(h)) at column N + c (ldo = 2N).
@@ -465,7 +472,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // tail of each half
           const int kc = (nkb_half > 0 && kb >= nkb_half) ? p.k_half / kBK + (kb - nkb_half) : kb;
           mbar_arrive_expect_tx(&full[s], (p.a_box_rows > 0 ? p.a_box_rows * kBK * 2 : kAStageBytes) + kBStageBytes);
-          tma_load_2d(a_dst, &tmA, &full[s], kc * kBK, m_blk * kBM);
+          if (MODE == kModeDown && p.a_mn_major) {
+            // two 64-column slabs of M, each the K block's 64 rows
+            const int kr = kc * kBK;
+            const bool lo = p.k_wrap > 0 && kr >= p.k_wrap;
+            const int col = (lo ? p.a_col_lo : p.a_col_hi) + m_blk * kBM;
+            const int row = p.k_wrap > 0 ? kr % p.k_wrap : kr;
+            tma_load_2d(a_dst, &tmA, &full[s], col, row);
+            tma_load_2d(a_dst + kAStageBytes / 2, &tmA, &full[s], col + 64, row);
+          } else {
+            tma_load_2d(a_dst, &tmA, &full[s], kc * kBK, m_blk * kBM);
+          }
           if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity || MODE == kModeF32 ||
               MODE == kModeBwdDh) {
             tma_load_2d(b_dst, &tmB0, &full[s], kc * kBK, n_blk * kBN);
@@ -504,7 +521,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      const uint32_t idesc = umma_idesc_bf16(kBM, kBN, (MODE == kModeDown || MODE == kModeUnion) ? 1 : 0);
+      const bool a_mn = MODE == kModeDown && p.a_mn_major != 0;
+      const uint32_t idesc = umma_idesc_bf16(kBM, kBN, (MODE == kModeDown || MODE == kModeUnion) ? 1 : 0) |
+                             (a_mn ? (1u << 15) : 0u);  // bit 15: A MN-major
       int s = 0;
       uint32_t ph = 0;
       int buf = 0;
@@ -537,7 +556,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int k = 0; k < kBK / 16; ++k) {
             // K-major, 128-byte swizzle: 8-row groups 1024 bytes apart; a K step of
             // 16 bf16 is 32 bytes inside the swizzle row.
-            const uint64_t adesc = umma_smem_desc(a_addr + k * 32, 16, 1024);
+            // (MN-major A: two 64-wide slabs of M 8 KB apart, laid out like B below)
+            const uint64_t adesc = a_mn ? umma_smem_desc(a_addr + k * 2048, kAStageBytes / 2, 1024)
+                                        : umma_smem_desc(a_addr + k * 32, 16, 1024);
             uint64_t bdesc;
             if (MODE == kModeDown || MODE == kModeUnion) {
               // N-major, 128-byte swizzle: 64-column slabs 8 KB apart (LBO), 8-row

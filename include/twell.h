@@ -406,13 +406,13 @@ twell_status twell_ffn_hybrid_backward_dw(const uint16_t* x, const uint16_t* dy,
  * workspace, called after twell_ffn_hybrid_backward_dx). At densities where
  * every unit is active for many tokens of a batch, the weight gradients are a
  * dense contraction over the tokens: the records of the rows that fit are
- * sorted by unit and their dz, du and h written (as bf16 value plus bf16
- * remainder) by unit and token into dense blocks, one unit's rows at a time;
- * three tcgen05 GEMMs over all tokens form their share, and the
- * overflow rows' GEMMs add theirs. The extra error is ~2^-16 of each term; the
- * sums are in fp32, with K (the tokens) split over the GPU where that shortens
- * the GEMMs' last wave, the partial sums added atomically (so not
- * bit-reproducible from run to run).
+ * written token-major into a dense block [dz | du | h] (each as bf16 value
+ * plus bf16 remainder, zeros where no slot is stored) and three tcgen05 GEMMs
+ * over all tokens, reading that block with the units along M, form their
+ * share; the overflow rows' GEMMs add theirs. The extra error is ~2^-16 of
+ * each term; the sums are in fp32, with K (the tokens) split over the GPU
+ * where that shortens the GEMMs' last wave, the partial sums added atomically
+ * (so not bit-reproducible from run to run).
  */
 twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* dy, int T, int d, int f,
                                              const twell_t* tw, const int32_t* n_ovf, float* dWgT, float* dWuT,
