@@ -9,8 +9,8 @@
 // ([T][nT][W] float4); for the overflow rows, the gathered rows of x and dy
 // ([Tp][d] bf16 each, Tp = T rounded up to 64), their [z | u] ([T][2f] fp32;
 // before that, dh = dy . Wd^T of every token, [T][f] fp32),
-// [dz | du | dz_lo | du_lo] ([T][4f] bf16) and the three transposed blocks dz,
-// du, h ([f][2 Tp] bf16 each); the column counts/cursors ([f]), column
+// [dz | du | dz_lo | du_lo | h | h_lo] ([Tp][6f] bf16); the column
+// counts/cursors ([f]), column
 // offsets ([f + 1]) and the column-sorted records (one float4 per slot of the
 // rows that fit); for the tensor-core form of the weight gradients, the rows
 // that fit as dense token-major [dz | du | dz_lo | du_lo | h | h_lo] ([T][6f]
@@ -19,7 +19,7 @@ struct BwdWorkspace {
   float4* rec;
   uint16_t *xo, *dyo;
   float* zu;
-  uint16_t *a2, *tT;
+  uint16_t* a2;
   int *colcnt, *colptr;
   float4* list;
   uint16_t* dense;  // tensor-core form: the rows that fit, [T][6f] bf16 (dz, du, their remainders, h, its remainder)
@@ -42,8 +42,7 @@ BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
   w.xo = reinterpret_cast<uint16_t*>(take(tp * d * 2));
   w.dyo = reinterpret_cast<uint16_t*>(take(tp * d * 2));
   w.zu = reinterpret_cast<float*>(take(static_cast<size_t>(T) * f * 8));
-  w.a2 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * f * 8));
-  w.tT = reinterpret_cast<uint16_t*>(take(3 * static_cast<size_t>(f) * 2 * tp * 2));
+  w.a2 = reinterpret_cast<uint16_t*>(take(tp * f * 12));
   w.colcnt = reinterpret_cast<int*>(take(static_cast<size_t>(f) * 4));
   w.colptr = reinterpret_cast<int*>(take((static_cast<size_t>(f) + 1) * 4));
   w.list = reinterpret_cast<float4*>(take(s0 * 16));
@@ -181,7 +180,7 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   CUtensorMap mx, mdy, mg, mu, mwd, ma2, mgT, muT;
   if (!make_map(&mx, w.xo, d, T, kBK, kBM) || !make_map(&mdy, w.dyo, d, T, kBK, kBM) ||
       !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128) ||
-      !make_map(&mwd, Wd, d, f, kBK, kBN) || !make_map(&ma2, w.a2, 4 * f, T, kBK, kBM) ||
+      !make_map(&mwd, Wd, d, f, kBK, kBN) || !make_map(&ma2, w.a2, 6 * f, T, kBK, kBM) ||
       !make_map(&mgT, WgT, d, f, 64, kBK) || !make_map(&muT, WuT, d, f, 64, kBK))
     return TWELL_ERR_CUDA;
   GemmParams q1{};
@@ -200,7 +199,6 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   q2.K = d;
   q2.zu = w.zu;
   q2.a2 = w.a2;
-  q2.tT = w.tT;
   q2.t_pad = w.t_pad;
   q2.h_split = 1;
   q2.dev_status = dev_status;
@@ -261,14 +259,18 @@ twell_status backward_dw_impl(const uint16_t* x, const uint16_t* dy, int T, int 
 // their tokens, as bf16 value and remainder halves).
 twell_status backward_dw_overflow(int d, int f, const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd,
                                   const BwdWorkspace& w, cudaStream_t s, int sms) {
-  const size_t tblock = static_cast<size_t>(f) * 2 * w.t_pad;
-  const uint16_t* aT[3] = {w.tT, w.tT + tblock, w.tT + 2 * tblock};
+  // A: the overflow rows' [dz | du | dz_lo | du_lo | h | h_lo] block (token-major,
+  // read MN-major: units along M, the gathered tokens along K, values then
+  // remainders); K sized on the device to the overflow count rounded up to 64
+  // (the padding rows of the block and of xo, dyo hold zeros).
+  CUtensorMap ma;
+  if (!make_map(&ma, w.a2, 6 * static_cast<uint64_t>(f), w.t_pad, 64, kBK)) return TWELL_ERR_CUDA;
   const uint16_t* bT[3] = {w.xo, w.xo, w.dyo};
   float* outs[3] = {dWgT, dWuT, dWd};
+  const int col_hi[3] = {0, f, 4 * f}, col_lo[3] = {2 * f, 3 * f, 5 * f};
   for (int i = 0; i < 3; ++i) {
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, aT[i], 2 * w.t_pad, f, kBK, kBM) || !make_map(&mb, bT[i], d, w.t_pad, 64, kBK))
-      return TWELL_ERR_CUDA;
+    CUtensorMap mb;
+    if (!make_map(&mb, bT[i], d, w.t_pad, 64, kBK)) return TWELL_ERR_CUDA;
     GemmParams q{};
     q.M = f;
     q.N = d;
@@ -276,6 +278,9 @@ twell_status backward_dw_overflow(int d, int f, const int32_t* n_ovf, float* dWg
     q.k_wrap = w.t_pad;
     q.k_dev = n_ovf;
     q.k_half = w.t_pad;
+    q.a_mn_major = 1;
+    q.a_col_hi = col_hi[i];
+    q.a_col_lo = col_lo[i];
     q.accumulate = 1;
     q.k_splits_max = 32;
     q.out_f32 = outs[i];
@@ -287,9 +292,9 @@ twell_status backward_dw_overflow(int d, int f, const int32_t* n_ovf, float* dWg
 }
 
 // Tensor-core form of the weight gradients from the workspace filled by
-// backward_dx_impl: the records of the rows that fit are sorted by column and
-// written densely (bf16 value and remainder) by unit and token, three GEMMs
-// over all tokens give their share, then the overflow rows' GEMMs add theirs.
+// backward_dx_impl: the records of the rows that fit are written densely
+// (bf16 value and remainder) by token, three GEMMs over all tokens give their
+// share, then the overflow rows' GEMMs add theirs.
 twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, int d, int f, const twell_t* tw,
                                  const int32_t* n_ovf, float* dWgT, float* dWuT, float* dWd, char* ws,
                                  cudaStream_t s, int sms) {

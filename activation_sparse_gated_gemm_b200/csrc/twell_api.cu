@@ -1183,9 +1183,8 @@ size_t twell_dense_backward_workspace_bytes(int T, int d, int f) {
   (void)d;
   if (T <= 0 || f <= 0) return 0;
   const size_t tp = round_up(static_cast<size_t>(T), 64);
-  return round_up(static_cast<size_t>(T) * f * 8, 256)        // [z | u] fp32
-         + round_up(static_cast<size_t>(T) * f * 4, 256)      // [dz | du] bf16
-         + round_up(3 * static_cast<size_t>(f) * tp * 2, 256);  // dz, du, h unit-major bf16
+  return round_up(static_cast<size_t>(T) * f * 8, 256)   // [z | u] fp32
+         + round_up(tp * f * 6, 256);                     // [dz | du | h] bf16, token-major
 }
 
 twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
@@ -1211,11 +1210,10 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
   const int tp = static_cast<int>(round_up(static_cast<size_t>(T), 64));
   float* zu = reinterpret_cast<float*>(ws);
   uint16_t* a2 = reinterpret_cast<uint16_t*>(ws + round_up(static_cast<size_t>(T) * f * 8, 256));
-  uint16_t* tT = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(a2) + round_up(static_cast<size_t>(T) * f * 4, 256));
   CUtensorMap mx, mdy, mg, mu, mwd, ma2, mgT, muT;
   if (!make_map(&mx, x, d, T, kBK, kBM) || !make_map(&mdy, dy, d, T, kBK, kBM) ||
       !make_map(&mg, WgT, d, f, kBK, 128) || !make_map(&mu, WuT, d, f, kBK, 128) ||
-      !make_map(&mwd, Wd, d, f, kBK, kBN) || !make_map(&ma2, a2, 2 * f, T, kBK, kBM) ||
+      !make_map(&mwd, Wd, d, f, kBK, kBN) || !make_map(&ma2, a2, 3 * f, T, kBK, kBM) ||
       !make_map(&mgT, WgT, d, f, 64, kBK) || !make_map(&muT, WuT, d, f, 64, kBK))
     return TWELL_ERR_CUDA;
   // [z | u] = x [Wg | Wu]; dh = dy Wd^T with dz, du, h (bf16) in the epilogue
@@ -1233,7 +1231,6 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
   q2.K = d;
   q2.zu = zu;
   q2.a2 = a2;
-  q2.tT = tT;
   q2.t_pad = tp;
   q2.h_split = 0;
   q2.dev_status = dev_status;
@@ -1253,28 +1250,32 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
     q3.k_splits_max = 32;
   }
   TW_TRY(launch_gemm<kModeDown>(ma2, mgT, muT, q3, q3.k_splits_max > 1 ? sms : gemm_grid(T, d, kBN, sms), s));
-  // dWgT = dz^T x, dWuT = du^T x, dWd = h^T dy (K = the tokens; rows of x and
-  // dy past T are read as zeros by the tensor maps). As in the hybrid's
-  // tensor-core weight gradients, K is split whenever that shortens the last
-  // wave of output tiles, the partial sums added into zeroed outputs.
-  const size_t tblock = static_cast<size_t>(f) * tp;
-  const uint16_t* aT[3] = {tT, tT + tblock, tT + 2 * tblock};
+  // dWgT = dz^T x, dWuT = du^T x, dWd = h^T dy: the [dz | du | h] block read
+  // as an MN-major A operand (units along M, tokens along K; its padding rows
+  // hold zeros, and rows of x and dy past T are read as zeros by the tensor
+  // maps). As in the hybrid's tensor-core weight gradients, K is split
+  // whenever that shortens the last wave of output tiles, the partial sums
+  // added into zeroed outputs.
+  CUtensorMap maT;
+  if (!make_map(&maT, a2, 3 * static_cast<uint64_t>(f), tp, 64, kBK)) return TWELL_ERR_CUDA;
   const uint16_t* bT[3] = {x, x, dy};
   float* outs[3] = {dWgT, dWuT, dWd};
   for (int i = 0; i < 3; ++i) {
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, aT[i], tp, f, kBK, kBM) || !make_map(&mb, bT[i], d, T, 64, kBK)) return TWELL_ERR_CUDA;
+    CUtensorMap mb;
+    if (!make_map(&mb, bT[i], d, T, 64, kBK)) return TWELL_ERR_CUDA;
     GemmParams q{};
     q.M = f;
     q.N = d;
     q.K = tp;
+    q.a_mn_major = 1;
+    q.a_col_hi = i * f;
     q.out_f32 = outs[i];
     q.ldo = d;
     q.k_splits_max = 32;
     q.split_waves = 1;
     q.dev_status = dev_status;
     TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
-    TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, sms, s));
+    TW_TRY(launch_gemm<kModeDown>(maT, mb, mb, q, sms, s));
   }
   return TWELL_OK;
 }

@@ -117,15 +117,14 @@ struct GemmParams {
   float* out_f32;
   int ldo;
   uint32_t* active;    // kModeActivity: column bitmap, OR-ed into
-  // kModeBwdDh: zu = [z | u] rows ([M][2N] fp32); a2 = [M][4N] bf16 rows
-  // [dz | du | dz_lo | du_lo]; tT = three [N][2 t_pad] bf16 blocks (dz, du, h),
-  // unit-major, tokens [0, t_pad) holding bf16(v) and [t_pad, 2 t_pad) the
-  // remainder; rows in [M, t_pad) of the tile are written as zeros. With
-  // h_split == 0 only the bf16 values are kept: a2 = [M][2N] rows [dz | du],
-  // tT = three [N][t_pad] blocks.
+  // kModeBwdDh: zu = [z | u] rows ([M][2N] fp32); a2 = [t_pad][6N] bf16 rows
+  // [dz | du | dz_lo | du_lo | h | h_lo] (bf16 value and remainder), rows in
+  // [M, t_pad) of the tile written as zeros. With h_split == 0 only the bf16
+  // values are kept: a2 = [t_pad][3N] rows [dz | du | h]. dx reads the first
+  // 2N (4N) columns along K; the weight gradients read the block as an
+  // MN-major A operand with the tokens along K.
   const float* zu;
   uint16_t* a2;
-  uint16_t* tT;
   int t_pad;
   // kModeDown: B rows at or past k_split_b (after k_wrap) come from tmB1, at
   // row - k_split_b (two matrices stacked along K without copying them).
@@ -815,8 +814,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else if (MODE == kModeBwdDh) {
         const bool pair = p.h_split != 0;
-        const size_t tstride = (pair ? 2 : 1) * static_cast<size_t>(p.t_pad);  // one unit's row, transposed
-        const size_t tblock = static_cast<size_t>(p.N) * tstride;
+        const size_t pitch = (pair ? 6 : 3) * static_cast<size_t>(p.N);
+        // column of each value's bf16 part and (pair) of its remainder
+        const size_t c_hi[3] = {0, static_cast<size_t>(p.N), (pair ? 4 : 2) * static_cast<size_t>(p.N)};
+        const size_t c_lo[3] = {2 * static_cast<size_t>(p.N), 3 * static_cast<size_t>(p.N),
+                                5 * static_cast<size_t>(p.N)};
 #pragma unroll 1
         for (int ch = 0; ch < kBN / 32; ++ch) {
           uint32_t r[32];
@@ -829,75 +831,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const int col = n_blk * kBN + ch * 32;
           if (col >= p.N || my_row >= p.t_pad) continue;
+          uint16_t* arow = p.a2 + static_cast<size_t>(my_row) * pitch + col;
           if (my_row < M) {
             const float4* z4 = reinterpret_cast<const float4*>(p.zu + static_cast<size_t>(my_row) * 2 * p.N + col);
             const float4* u4 = reinterpret_cast<const float4*>(p.zu + static_cast<size_t>(my_row) * 2 * p.N + p.N + col);
-            uint32_t dzh[16], duh[16], dzl[16], dul[16];
+            uint32_t hi[3][16], lo[3][16];  // dz, du, h of the chunk's 32 units, as bf16 pairs
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 zq = z4[q], uq = u4[q];
               const float zz[4] = {zq.x, zq.y, zq.z, zq.w};
               const float uu[4] = {uq.x, uq.y, uq.z, uq.w};
-              float vz[4], vu[4], vh[4];
+              float v[3][4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float dh = __uint_as_float(r[4 * q + e]);
                 const float g = fmaxf(zz[e], 0.0f);
-                vz[e] = zz[e] > 0.0f ? dh * uu[e] : 0.0f;
-                vu[e] = dh * g;
-                vh[e] = g * uu[e];
+                v[0][e] = zz[e] > 0.0f ? dh * uu[e] : 0.0f;  // dz
+                v[1][e] = dh * g;                           // du
+                v[2][e] = g * uu[e];                        // h
               }
 #pragma unroll
-              for (int e = 0; e < 4; e += 2) {
-                const int k = 2 * q + e / 2;
-                dzh[k] = pack_bf16x2(vz[e], vz[e + 1]);
-                duh[k] = pack_bf16x2(vu[e], vu[e + 1]);
-                dzl[k] = pack_bf16x2(vz[e] - __uint_as_float(dzh[k] << 16), vz[e + 1] - __uint_as_float(dzh[k] & 0xffff0000u));
-                dul[k] = pack_bf16x2(vu[e] - __uint_as_float(duh[k] << 16), vu[e + 1] - __uint_as_float(duh[k] & 0xffff0000u));
-              }
-              // transposed: unit j = col + 4q + e, token my_row (32 lanes = 32 consecutive tokens)
+              for (int b = 0; b < 3; ++b)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const size_t o = static_cast<size_t>(col + 4 * q + e) * tstride + my_row;
-                const uint16_t zh = f32_to_bf16_bits(vz[e]);
-                const uint16_t uh = f32_to_bf16_bits(vu[e]);
-                const uint16_t hh = f32_to_bf16_bits(vh[e]);
-                p.tT[o] = zh;
-                p.tT[tblock + o] = uh;
-                p.tT[2 * tblock + o] = hh;
-                if (pair) {
-                  p.tT[o + p.t_pad] = f32_to_bf16_bits(vz[e] - __uint_as_float(static_cast<uint32_t>(zh) << 16));
-                  p.tT[tblock + o + p.t_pad] =
-                      f32_to_bf16_bits(vu[e] - __uint_as_float(static_cast<uint32_t>(uh) << 16));
-                  p.tT[2 * tblock + o + p.t_pad] =
-                      f32_to_bf16_bits(vh[e] - __uint_as_float(static_cast<uint32_t>(hh) << 16));
+                for (int e = 0; e < 4; e += 2) {
+                  const int k = 2 * q + e / 2;
+                  hi[b][k] = pack_bf16x2(v[b][e], v[b][e + 1]);
+                  lo[b][k] = pack_bf16x2(v[b][e] - __uint_as_float(hi[b][k] << 16),
+                                         v[b][e + 1] - __uint_as_float(hi[b][k] & 0xffff0000u));
                 }
-              }
             }
-            uint16_t* arow = p.a2 + static_cast<size_t>(my_row) * (pair ? 4 : 2) * p.N;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              reinterpret_cast<uint4*>(arow + col)[v] = make_uint4(dzh[4 * v], dzh[4 * v + 1], dzh[4 * v + 2], dzh[4 * v + 3]);
-              reinterpret_cast<uint4*>(arow + p.N + col)[v] =
-                  make_uint4(duh[4 * v], duh[4 * v + 1], duh[4 * v + 2], duh[4 * v + 3]);
-              if (pair) {
-                reinterpret_cast<uint4*>(arow + 2 * p.N + col)[v] =
-                    make_uint4(dzl[4 * v], dzl[4 * v + 1], dzl[4 * v + 2], dzl[4 * v + 3]);
-                reinterpret_cast<uint4*>(arow + 3 * p.N + col)[v] =
-                    make_uint4(dul[4 * v], dul[4 * v + 1], dul[4 * v + 2], dul[4 * v + 3]);
+            for (int b = 0; b < 3; ++b)
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                reinterpret_cast<uint4*>(arow + c_hi[b])[v4] =
+                    make_uint4(hi[b][4 * v4], hi[b][4 * v4 + 1], hi[b][4 * v4 + 2], hi[b][4 * v4 + 3]);
+                if (pair)
+                  reinterpret_cast<uint4*>(arow + c_lo[b])[v4] =
+                      make_uint4(lo[b][4 * v4], lo[b][4 * v4 + 1], lo[b][4 * v4 + 2], lo[b][4 * v4 + 3]);
               }
-            }
           } else {
-            // padding tokens of the transposed blocks must read as zeros
-#pragma unroll 4
-            for (int i = 0; i < 32; ++i) {
-              const size_t o = static_cast<size_t>(col + i) * tstride + my_row;
+            // padding tokens: the weight gradients' K runs over whole 64-row blocks
 #pragma unroll
-              for (int b = 0; b < 3; ++b) {
-                p.tT[b * tblock + o] = 0;
-                if (pair) p.tT[b * tblock + o + p.t_pad] = 0;
+            for (int b = 0; b < 3; ++b)
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                reinterpret_cast<uint4*>(arow + c_hi[b])[v4] = make_uint4(0u, 0u, 0u, 0u);
+                if (pair) reinterpret_cast<uint4*>(arow + c_lo[b])[v4] = make_uint4(0u, 0u, 0u, 0u);
               }
-            }
           }
         }
       } else if (MODE == kModeActivity) {
