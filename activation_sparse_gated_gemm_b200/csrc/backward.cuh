@@ -520,14 +520,20 @@ __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
 // against [Wg; Wu] (read twice along K) gives dx for every token. WITH_H: rows
 // a2[t][6f] that also hold [h | h_lo], from which the weight-gradient GEMMs
 // read dz, du and h with the tokens as K (an MN-major A operand). One warp per
-// (row, tile), lane l owning units 4l..4l+3: every byte of the block is
-// written once with 8-byte stores that a warp makes contiguous (a memset of
-// the block and 2-byte scattered stores into it took 0.27 ms at the 0.5B layer).
+// (row, tile): its lanes load the tile's slots side by side and drop their
+// values into the tile's 128 units in shared memory, then lane l writes units
+// 4l..4l+3, so every byte of the block is written once with 8-byte stores that
+// a warp makes contiguous (a memset of the block and 2-byte scattered stores
+// into it took 0.27 ms at the 0.5B layer; a slot-by-slot walk by every lane,
+// 0.22 ms).
 template <bool WITH_H>
 __global__ void __launch_bounds__(256) bwd_dense_rows_kernel(SlotSource src, uint16_t* __restrict__ a2) {
   griddep_launch_dependents();
   griddep_wait();
+  constexpr int kVals = WITH_H ? 3 : 2;
+  __shared__ __align__(16) float tile_vals[8][3][128];  // per warp: dz, du, h of the tile's units
   const int lane = threadIdx.x & 31;
+  float (*tv)[128] = tile_vals[threadIdx.x >> 5];
   const long long pairs = static_cast<long long>(src.rows) * src.nT;
   const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   const size_t f = static_cast<size_t>(src.f);
@@ -535,25 +541,33 @@ __global__ void __launch_bounds__(256) bwd_dense_rows_kernel(SlotSource src, uin
        w += nw) {
     const int t = static_cast<int>(w / src.nT);
     const int c = static_cast<int>(w - static_cast<long long>(t) * src.nT);
-    constexpr int kVals = WITH_H ? 3 : 2;
-    float v[3][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // dz, du, h of my four units
+#pragma unroll
+    for (int b = 0; b < kVals; ++b) *reinterpret_cast<float4*>(&tv[b][4 * lane]) = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncwarp();
     if (!src.row_ovf[t]) {
       const int n = min(max(static_cast<int>(src.counts[w]), 0), src.W);
-      for (int k = 0; k < n; ++k) {
+      for (int k = lane; k < n; k += 32) {
         const size_t slot = static_cast<size_t>(w) * src.W + k;
         const int j = static_cast<int>(src.idx[slot]) - c * 128;
-        if ((j >> 2) == lane && j >= 0) {
+        if (j >= 0 && j < 128) {
           const float4 rec = src.rec[slot];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if ((j & 3) == e) {
-              v[0][e] = rec.z;
-              v[1][e] = rec.y;
-              v[2][e] = rec.x;
-            }
+          tv[0][j] = rec.z;
+          tv[1][j] = rec.y;
+          if (WITH_H) tv[2][j] = rec.x;
         }
       }
     }
+    __syncwarp();
+    float v[3][4];
+#pragma unroll
+    for (int b = 0; b < kVals; ++b) {
+      const float4 q = *reinterpret_cast<const float4*>(&tv[b][4 * lane]);
+      v[b][0] = q.x;
+      v[b][1] = q.y;
+      v[b][2] = q.z;
+      v[b][3] = q.w;
+    }
+    __syncwarp();  // the next pair's zeros overwrite these units
     uint16_t* row = a2 + static_cast<size_t>(t) * (WITH_H ? 6 : 4) * f + static_cast<size_t>(c) * 128 + 4 * lane;
 #pragma unroll
     for (int b = 0; b < kVals; ++b) {

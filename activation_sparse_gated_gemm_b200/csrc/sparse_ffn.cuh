@@ -451,13 +451,17 @@ __global__ void __launch_bounds__(kSmallSparseWarps * 32) sparse_small_kernel(co
 // the slot's row of H gets them over zeros, with a zero remainder (the tiles
 // that overflowed were written, exact, by the gate+up GEMM). Slot s holds row
 // slot_row[s]; the slot's row of y is zeroed for the branch's partial sums.
-// One warp per (slot, tile), lane l owning units 4l..4l+3.
+// One warp per (slot, tile): its lanes load the tile's stored slots side by
+// side into the tile's 128 units in shared memory, then lane l writes units
+// 4l..4l+3.
 __global__ void __launch_bounds__(256) ovf_fill_kernel(const int16_t* counts, const int16_t* idx, const uint16_t* vals,
                                                        int nT, int W, int f, const int* slot_row, const int* n_slots,
                                                        uint16_t* H, float* y, int d) {
   griddep_launch_dependents();
   griddep_wait();
+  __shared__ __align__(16) uint16_t tile_h[8][128];
   const int lane = threadIdx.x & 31;
+  uint16_t* th = tile_h[threadIdx.x >> 5];
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   const long long n = static_cast<long long>(max(*n_slots, 0)) * nT;
   for (long long u = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); u < n; u += warps) {
@@ -469,20 +473,18 @@ __global__ void __launch_bounds__(256) ovf_fill_kernel(const int16_t* counts, co
     }
     const size_t at = static_cast<size_t>(t) * nT + c;
     const int cnt = counts[at];
-    if (cnt > W) continue;  // written by the gate+up GEMM
-    uint32_t h01 = 0, h23 = 0;
-    for (int k = 0; k < cnt; ++k) {
+    if (cnt > W) continue;  // written by the gate+up GEMM (warp-uniform)
+    *reinterpret_cast<uint2*>(th + 4 * lane) = make_uint2(0u, 0u);
+    __syncwarp();
+    for (int k = lane; k < cnt; k += 32) {
       const int j = static_cast<int>(idx[at * W + k]) - c * 128;
-      if ((j >> 2) == lane) {
-        const uint32_t v = vals[at * W + k];
-        if ((j & 3) == 0) h01 |= v;
-        else if ((j & 3) == 1) h01 |= v << 16;
-        else if ((j & 3) == 2) h23 |= v;
-        else h23 |= v << 16;
-      }
+      if (j >= 0 && j < 128) th[j] = vals[at * W + k];
     }
+    __syncwarp();
+    const uint2 h = *reinterpret_cast<const uint2*>(th + 4 * lane);
+    __syncwarp();  // the next pair's zeros overwrite these units
     uint16_t* hrow = H + static_cast<size_t>(sl) * 2 * f;
-    *reinterpret_cast<uint2*>(hrow + c * 128 + 4 * lane) = make_uint2(h01, h23);
+    *reinterpret_cast<uint2*>(hrow + c * 128 + 4 * lane) = h;
     *reinterpret_cast<uint2*>(hrow + f + c * 128 + 4 * lane) = make_uint2(0u, 0u);
   }
 }
