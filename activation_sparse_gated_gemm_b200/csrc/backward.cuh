@@ -11,12 +11,11 @@
 // Rows that fit the ELL width take three passes over their stored units:
 //   0. dh = dy . Wd^T for every token on the tensor cores (a plain dense
 //      contraction, [T][f] fp32): cheaper than gathering a row of Wd per slot;
-//   1. per token (one warp per token, like the forward's fused kernel): u_j by
-//      a dot product per stored unit, dh_j read from row t of dh; each slot's
-//      record {h, du, dz, token} is written beside the slots;
-//   1b. per token again: dx_t by two row axpys with du_j, dz_j from the records
-//      (split from pass 1 so that neither pass holds both dx_t and the dot
-//      passes' rows, which lets each run twice the warps);
+//   1. u = x . Wu^T for every token on the tensor cores as well, and per
+//      stored slot the record {h, du, dz, token} from u_j, dh_j and the stored
+//      g (cheaper than a dot product over a gathered Wu row per slot);
+//   1b. per token (one warp per token, like the forward's fused kernel): dx_t
+//      by two row axpys with du_j, dz_j from the records;
 //   2. per hidden unit: the records are sorted by column (count, scan, scatter
 //      of whole 16-byte records) and one warp per (unit, 256-wide slice of d)
 //      reads its unit's records in order and sums h dy_t, du x_t, dz x_t into
@@ -46,71 +45,11 @@ struct BwdParams {
   int* dev_status;
 };
 
-// Warps per block of the two per-token passes. The dot pass holds x_t in
-// shared memory and two weight rows in registers; the dx pass holds dx_t and
-// two weight rows in registers.
-constexpr int bwd_dots_warps(int nch) {
-  // registers (two rows of d per lane and the reductions) cap it before shared memory does
-  return nch <= 6 ? 16 : (nch <= 8 ? 12 : 8);
-}
+// Warps per block of the per-token dx pass, which holds dx_t and two weight
+// rows in registers.
 constexpr int bwd_dx_warps(int nch) { return nch <= 4 ? 16 : (nch <= 7 ? 12 : 8); }
 
-constexpr size_t bwd_dots_smem_bytes(int nch) {
-  return static_cast<size_t>(bwd_dots_warps(nch)) * (nch * 32 * 16 + kListCap * 6);
-}
 constexpr size_t bwd_dx_smem_bytes(int nch) { return static_cast<size_t>(bwd_dx_warps(nch)) * kListCap * 6; }
-
-// 16-byte shared-memory load that the compiler keeps inside its loop (x_t is
-// reread per entry instead of being held in registers across it).
-__device__ __forceinline__ uint4 lds_v4(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(smem_u32(p)));
-  return v;
-}
-
-// For the entries s < ns of a batch (column my_j on lane s): lane s receives
-// <src, M[j_s, :]>, src being a row parked in shared memory. Two row buffers
-// alternate so the gather of entry s + 1 is in flight while entry s is reduced.
-template <int NCH>
-__device__ __forceinline__ float bwd_dot_pass(const uint4* src, const uint16_t* M, int my_j, int ns, int lane,
-                                              int d) {
-  float mine = 0.0f;
-  uint4 wa[NCH], wb[NCH];
-  load_row<NCH>(wa, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, 0)) * d, lane, d);
-#pragma unroll 1
-  for (int s = 0; s < ns; s += 2) {
-    if (s + 1 < ns) load_row<NCH>(wb, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 1)) * d, lane, d);
-    {
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int i = 0; i < NCH; i += 2) {
-        mixdot8(lds_v4(src + i * 32 + lane), wa[i], a0, a1);
-        if (i + 1 < NCH) mixdot8(lds_v4(src + (i + 1) * 32 + lane), wa[i + 1], a2, a3);
-      }
-      float acc = (a0 + a1) + (a2 + a3);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == s) mine = acc;
-    }
-    if (s + 1 < ns) {
-      if (s + 2 < ns)
-        load_row<NCH>(wa, M + static_cast<size_t>(__shfl_sync(0xffffffffu, my_j, s + 2)) * d, lane, d);
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-      for (int i = 0; i < NCH; i += 2) {
-        mixdot8(lds_v4(src + i * 32 + lane), wb[i], a0, a1);
-        if (i + 1 < NCH) mixdot8(lds_v4(src + (i + 1) * 32 + lane), wb[i + 1], a2, a3);
-      }
-      float acc = (a0 + a1) + (a2 + a3);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == s + 1) mine = acc;
-    }
-  }
-  return mine;
-}
 
 // acc += c_s * M[j_s, :] for the entries s < ns (c_s on lane s), with the same
 // two-buffer gather.
@@ -191,66 +130,7 @@ __device__ __forceinline__ int bwd_next_row(int* next_row, int lane) {
   return __shfl_sync(0xffffffffu, t, 0);
 }
 
-// Pass 1, one warp per token that fits: u_j = x_t . Wu[:, j] and
-// dh_j = dy_t . Wd[j, :] for every stored slot (x_t and dy_t parked in shared
-// memory), and the slot's record {h = g u, du = dh g, dz = dh u, t}.
-template <int NCH, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32, 1) bwd_dots_kernel(const BwdParams p) {
-  griddep_launch_dependents();
-  griddep_wait();
-  extern __shared__ uint4 bwd_smem[];
-  __shared__ int next_row;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int d = p.d;
-  uint4* xs = bwd_smem + warp * NCH * 32;
-  uint32_t* list = reinterpret_cast<uint32_t*>(bwd_smem + WARPS * NCH * 32) + warp * kListCap;
-  uint16_t* lpos = reinterpret_cast<uint16_t*>(reinterpret_cast<uint32_t*>(bwd_smem + WARPS * NCH * 32) +
-                                               WARPS * kListCap) +
-                   warp * kListCap;
-  const int group_tiles = max(1, kListCap / p.W);
-  bool bad_index = false;
-  const int r_end = static_cast<int>(static_cast<long long>(p.rows) * (blockIdx.x + 1) / gridDim.x);
-  if (threadIdx.x == 0) next_row = static_cast<int>(static_cast<long long>(p.rows) * blockIdx.x / gridDim.x);
-  __syncthreads();
-#pragma unroll 1
-  for (;;) {
-    const int t = bwd_next_row(&next_row, lane);
-    if (t >= r_end) break;
-    if (p.row_ovf[t]) continue;
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int k0 = (i * 32 + lane) * 8;
-      const bool in = k0 < d;
-      xs[i * 32 + lane] = in ? ldg_nc_v4(p.x + static_cast<size_t>(t) * d + k0) : make_uint4(0, 0, 0, 0);
-    }
-    const float* dh_row = p.dh + static_cast<size_t>(t) * p.f;
-    const size_t slot_row = static_cast<size_t>(t) * p.nT * p.W;
-#pragma unroll 1
-    for (int c0 = 0; c0 < p.nT; c0 += group_tiles) {
-      const int total = bwd_build_list(p, t, c0, min(p.nT, c0 + group_tiles), list, lpos, lane, bad_index);
-      __syncwarp();
-#pragma unroll 1
-      for (int s0 = 0; s0 < total; s0 += 32) {
-        const int ns = min(32, total - s0);
-        const uint32_t my_e = lane < ns ? list[s0 + lane] : 0u;
-        const int my_j = entry_j(my_e);
-        const uint16_t my_pos = lane < ns ? lpos[s0 + lane] : 0x8000u;
-        const float my_u = bwd_dot_pass<NCH>(xs, p.WuT, my_j, ns, lane, d);
-        // my_j is a checked column (0 for an entry that was out of range)
-        const float my_dh = lane < ns ? __ldg(dh_row + my_j) : 0.0f;
-        const float my_g = entry_g(my_e);
-        if ((my_pos & 0x8000u) == 0)
-          p.s_rec[slot_row + my_pos] = make_float4(my_g * my_u, my_dh * my_g, my_dh * my_u, __int_as_float(t));
-      }
-      __syncwarp();
-    }
-  }
-  if (__any_sync(0xffffffffu, bad_index) && lane == 0) raise_status(p.dev_status, kDevIndex);
-}
-
-// Pass 2, one warp per token that fits: dx_t = sum over its stored slots of
+// The dx pass, one warp per token that fits: dx_t = sum over its stored slots of
 // dz_j Wg[:, j] + du_j Wu[:, j], with du_j, dz_j from the slots' records and
 // dx_t in registers (two alternating weight-row buffers, as in the forward).
 template <int NCH, int WARPS>
@@ -318,43 +198,40 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dx_kernel(const BwdParams p
 
 // The stored slots of one pass, as the column sort sees them.
 // The records of the rows that fit from dense u = x . Wu^T and dh = dy . Wd^T
-// ([rows][f] fp32 each, from two tensor-core GEMMs) instead of a dot pass per
-// stored slot: one thread per (row, tile) reads its stored slots (j, g) and
-// writes {h = g u_j, du = dh_j g, dz = dh_j u_j, t}. A stored index outside
-// [0, f) raises TWELL_ERR_INDEX and leaves its record unwritten, as the dot
-// pass does.
+// ([rows][f] fp32 each, from two tensor-core GEMMs) instead of a dot product
+// over a gathered Wu row per stored slot: each stored slot (j, g) gets
+// {h = g u_j, du = dh_j g, dz = dh_j u_j, t}. Eight lanes per (row, tile), four
+// consecutive tiles per warp, the lanes of a tile taking its slots side by side
+// (a thread per tile walking its slots one after another took 0.12 ms at the
+// 0.5B layer). A stored index outside [0, f) raises TWELL_ERR_INDEX and leaves
+// its record unwritten; the dx pass skips such slots too.
 __global__ void __launch_bounds__(256) bwd_records_kernel(const BwdParams p, const float* __restrict__ u) {
   griddep_launch_dependents();
   griddep_wait();
   bool bad = false;
+  const int lane = threadIdx.x & 31;
   const long long pairs = static_cast<long long>(p.rows) * p.nT;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < pairs;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+  const long long groups = (pairs + 3) / 4;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long g = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); g < groups;
+       g += nw) {
+    const long long i = g * 4 + (lane >> 3);
+    if (i >= pairs) continue;
     const int t = static_cast<int>(i / p.nT);
     if (p.row_ovf[t]) continue;
     const int n = min(max(static_cast<int>(p.counts[i]), 0), p.W);
     const size_t base = static_cast<size_t>(i) * p.W;
     const float* urow = u + static_cast<size_t>(t) * p.f;
     const float* dhrow = p.dh + static_cast<size_t>(t) * p.f;
-    for (int k = 0; k < n; k += 8) {
-      // 8 slots per 16-byte load; k + 8 <= W since W is a multiple of 8
-      const uint4 iv = ldg_nc_v4(p.idx + base + k);
-      const uint4 vv = ldg_nc_v4(p.vals + base + k);
-      const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
-      const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (k + e < n) {
-          const int j = static_cast<int16_t>((e & 1) ? (iw[e >> 1] >> 16) : (iw[e >> 1] & 0xffffu));
-          const float g = __uint_as_float((e & 1) ? (vw[e >> 1] & 0xffff0000u) : (vw[e >> 1] << 16));
-          if (j < 0 || j >= p.f) {
-            bad = true;
-            continue;
-          }
-          const float uj = __ldg(urow + j), dh = __ldg(dhrow + j);
-          p.s_rec[base + k + e] = make_float4(g * uj, dh * g, dh * uj, __int_as_float(t));
-        }
+    for (int k = lane & 7; k < n; k += 8) {
+      const int j = p.idx[base + k];
+      const float gv = __uint_as_float(static_cast<uint32_t>(p.vals[base + k]) << 16);
+      if (j < 0 || j >= p.f) {
+        bad = true;
+        continue;
       }
+      const float uj = __ldg(urow + j), dh = __ldg(dhrow + j);
+      p.s_rec[base + k] = make_float4(gv * uj, dh * gv, dh * uj, __int_as_float(t));
     }
   }
   if (bad) raise_status(p.dev_status, kDevIndex);

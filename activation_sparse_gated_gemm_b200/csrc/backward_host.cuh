@@ -61,39 +61,36 @@ twell_status launch_bwd_pass(void (*kern)(BwdParams), size_t smem, const BwdPara
   return launch(kern, dim3(blocks), dim3(WARPS * 32), smem, s, p);
 }
 
-// The per-token passes of the rows that fit: the dot pass (records), then dx
-// (unless the tensor cores form dx).
+// The per-token dx pass of the rows that fit.
 template <int NCH>
-twell_status launch_bwd_token_n(const BwdParams& p, int sms, cudaStream_t s, bool with_dx) {
-  constexpr int kDots = bwd_dots_warps(NCH), kDx = bwd_dx_warps(NCH);
-  TW_TRY((launch_bwd_pass<NCH, kDots>(bwd_dots_kernel<NCH, kDots>, bwd_dots_smem_bytes(NCH), p, sms, s)));
-  if (!with_dx) return TWELL_OK;
+twell_status launch_bwd_dx_n(const BwdParams& p, int sms, cudaStream_t s) {
+  constexpr int kDx = bwd_dx_warps(NCH);
   return launch_bwd_pass<NCH, kDx>(bwd_dx_kernel<NCH, kDx>, bwd_dx_smem_bytes(NCH), p, sms, s);
 }
 
-twell_status launch_bwd_token(const BwdParams& p, int sms, cudaStream_t s, bool with_dx) {
+twell_status launch_bwd_dx(const BwdParams& p, int sms, cudaStream_t s) {
   switch ((p.d + 255) / 256) {
-    case 1: return launch_bwd_token_n<1>(p, sms, s, with_dx);
-    case 2: return launch_bwd_token_n<2>(p, sms, s, with_dx);
-    case 3: return launch_bwd_token_n<3>(p, sms, s, with_dx);
-    case 4: return launch_bwd_token_n<4>(p, sms, s, with_dx);
-    case 5: return launch_bwd_token_n<5>(p, sms, s, with_dx);
-    case 6: return launch_bwd_token_n<6>(p, sms, s, with_dx);
-    case 7: return launch_bwd_token_n<7>(p, sms, s, with_dx);
-    case 8: return launch_bwd_token_n<8>(p, sms, s, with_dx);
-    case 9: return launch_bwd_token_n<9>(p, sms, s, with_dx);
-    case 10: return launch_bwd_token_n<10>(p, sms, s, with_dx);
-    case 11: return launch_bwd_token_n<11>(p, sms, s, with_dx);
-    case 12: return launch_bwd_token_n<12>(p, sms, s, with_dx);
-    case 13: return launch_bwd_token_n<13>(p, sms, s, with_dx);
-    case 14: return launch_bwd_token_n<14>(p, sms, s, with_dx);
-    case 15: return launch_bwd_token_n<15>(p, sms, s, with_dx);
-    case 16: return launch_bwd_token_n<16>(p, sms, s, with_dx);
+    case 1: return launch_bwd_dx_n<1>(p, sms, s);
+    case 2: return launch_bwd_dx_n<2>(p, sms, s);
+    case 3: return launch_bwd_dx_n<3>(p, sms, s);
+    case 4: return launch_bwd_dx_n<4>(p, sms, s);
+    case 5: return launch_bwd_dx_n<5>(p, sms, s);
+    case 6: return launch_bwd_dx_n<6>(p, sms, s);
+    case 7: return launch_bwd_dx_n<7>(p, sms, s);
+    case 8: return launch_bwd_dx_n<8>(p, sms, s);
+    case 9: return launch_bwd_dx_n<9>(p, sms, s);
+    case 10: return launch_bwd_dx_n<10>(p, sms, s);
+    case 11: return launch_bwd_dx_n<11>(p, sms, s);
+    case 12: return launch_bwd_dx_n<12>(p, sms, s);
+    case 13: return launch_bwd_dx_n<13>(p, sms, s);
+    case 14: return launch_bwd_dx_n<14>(p, sms, s);
+    case 15: return launch_bwd_dx_n<15>(p, sms, s);
+    case 16: return launch_bwd_dx_n<16>(p, sms, s);
     default: return TWELL_ERR_SHAPE;
   }
 }
 
-// dx, and the per-slot scalars of both passes in the workspace. tc_dx: the
+// dx, and the per-slot records the weight gradients read, in the workspace. tc_dx: the
 // rows that fit get dx from one tensor-core GEMM over their scattered dz, du
 // instead of the per-token axpy pass.
 twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, const uint16_t* Wd,
@@ -127,20 +124,19 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   p0.dx = dx;
   p0.s_rec = w.rec;
   p0.dev_status = dev_status;
-  if (tc_dx) {
+  {
     // 1a. the records from dense u = x Wu^T (a second tensor-core GEMM, into the
     // idle half of the [z | u] region) and dh, in place of the per-slot dot
     // pass that gathers a Wu row for every stored slot
     float* ubuf = w.zu + static_cast<size_t>(T) * f;
     if (dh_tiles < sms) TW_TRY(zero_async(s, sms, ubuf, static_cast<size_t>(T) * f * sizeof(float)));
     TW_TRY(f32_gemm_impl(x, T, WuT, f, d, ubuf, f, dev_status, s, sms));
-    const long long pairs = static_cast<long long>(T) * nT;
-    const int rb = static_cast<int>(std::min<long long>((pairs + 255) / 256, 8LL * sms));
+    const long long pairs = static_cast<long long>(T) * nT;  // four per warp, eight warps per block
+    const int rb = static_cast<int>(std::min<long long>((pairs + 31) / 32, 8LL * sms));
     TW_TRY(launch(bwd_records_kernel, dim3(std::max(rb, 1)), dim3(256), 0, s, p0, static_cast<const float*>(ubuf)));
     TW_TRY(cuda_ok(cudaGetLastError()));
-  } else {
-    TW_TRY(launch_bwd_token(p0, sms, s, true));
   }
+  if (!tc_dx) TW_TRY(launch_bwd_dx(p0, sms, s));
   if (tc_dx) {
     // 1b. dx of every token = [dz | du | dz_lo | du_lo] [Wg; Wu; Wg; Wu]^T on
     // the tensor cores, the rows that fit scattered token-major into the

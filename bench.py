@@ -783,7 +783,7 @@ def run_gpu_backward(args, world, rank, local):
     nnz_ovf = int(counts[ovf_mask].sum())  # true counts: every active unit of an overflow row
     # CUDA-core work of the rows that fit (the overflow rows' dense branch runs
     # on the tensor cores: 12 n_ovf d f FLOPs, reported beside it)
-    flops_dx = 8.0 * d * nnz_fit  # u and dh per stored unit (dh from the dense GEMM), two axpys
+    flops_dx = 4.0 * d * nnz_fit  # two axpys per stored unit (u and dh come from dense GEMMs)
     flops_dw = 6.0 * d * nnz_fit  # three axpys per stored unit
     clocks = sampler.summary()
     peaks = load_peaks()
@@ -836,10 +836,11 @@ def run_gpu_backward(args, world, rank, local):
         "speedup_vs_own_dense": dense_ms / step_ms,
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
-        # per step: the dh GEMM, the dots pass and the dx pass (tensor-core form: zeroing, scatter and the dx
-        # GEMM), two gathers and three dense-branch GEMMs; five launches of either weight-gradient form and
-        # the overflow rows' three weight-gradient GEMMs
-        "gpu_launches": (18 if dx_form == "tensor_cores" else 16) * K,
+        # per step, dx: the dh and u GEMMs, the records, then the dx pass (tensor-core form: the dense rows
+        # and the dx GEMM), two gathers and three dense-branch GEMMs (9 or 10 launches); weight gradients:
+        # the column sort (four launches) and the per-unit sums, or the dense rows and three zeroed GEMMs
+        # (5 or 7), then the overflow rows' three GEMMs
+        "gpu_launches": ((10 if dx_form == "tensor_cores" else 9) + (10 if dw_form == "tensor_cores" else 8)) * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -363,8 +363,9 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
  *   dWgT [f][d] = dz^T x, dWuT [f][d] = du^T x, dWd [f][d] = h^T dy   (fp32,
  *   overwritten; the layouts of WgT, WuT and Wd)
  * tw, ovf_rows and n_ovf are the outputs of twell_ffn_hybrid_forward on the
- * same x (the gate form: tw's values are the bf16 gate). dh is formed for
- * every token by one tensor-core GEMM (dy Wd^T, fp32 sums). Rows that fit use
+ * same x (the gate form: tw's values are the bf16 gate). dh and u are formed
+ * for every token by two tensor-core GEMMs (dy Wd^T and x Wu^T, fp32 sums),
+ * and each stored slot's record {h, du, dz} from them. Rows that fit use
  * their stored slots with the stored bf16 gate g (h = g u), so the result is
  * the method's, within one bf16 rounding per term of the exact gradients;
  * their weight gradients are summed per hidden unit over a column sort of the
@@ -420,12 +421,11 @@ twell_status twell_ffn_hybrid_backward_dw_tc(const uint16_t* x, const uint16_t* 
 
 /*
  * Tensor-core form of twell_ffn_hybrid_backward_dx (same arguments, same
- * workspace; twell_ffn_hybrid_backward_dw or _dw_tc may follow it). Every
- * dense step runs on the tensor cores: u = x Wu^T for every token is a
- * tcgen05 GEMM beside dh = dy Wd^T (fp32, in the workspace), so the rows
- * that fit build their per-slot records {h, du, dz} by reading u_j and dh_j
- * instead of gathering a Wu row per stored slot; their dx then comes from one
- * tcgen05 GEMM: their dz and du are written by token into dense rows
+ * workspace; twell_ffn_hybrid_backward_dw or _dw_tc may follow it). The
+ * records are built as in twell_ffn_hybrid_backward_dx (u and dh for every
+ * token by tcgen05 GEMMs), and the rows that fit get their dx from one
+ * tcgen05 GEMM instead of the per-token pass: their dz and du are written by
+ * token into dense rows
  * [dz | du | dz_lo | du_lo] (bf16 value plus bf16 remainder, zeros elsewhere)
  * and multiplied by [Wg; Wu] read twice along K, the layout the overflow
  * rows' dense branch uses. Pays where the rows hold many stored units (the
