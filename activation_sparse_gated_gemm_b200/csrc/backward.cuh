@@ -42,6 +42,10 @@ struct BwdParams {
   int d, f, nT, W;
   float* dx;      // [rows][d] fp32
   float4* s_rec;  // per stored slot [rows][nT][W]: {h, du, dz, token (int bits)}
+  // dx pass: which of dz Wg^T (bit 0) and du Wu^T (bit 1) it sums, and
+  // whether it adds them to dx instead of storing them
+  int dx_mats;
+  int dx_accumulate;
   int* dev_status;
 };
 
@@ -177,8 +181,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dx_kernel(const BwdParams p
           my_du = rec.y;
           my_dz = rec.z;
         }
-        bwd_axpy_pass<NCH>(acc, p.WgT, my_j, my_dz, ns, lane, d);
-        bwd_axpy_pass<NCH>(acc, p.WuT, my_j, my_du, ns, lane, d);
+        if (p.dx_mats & 1) bwd_axpy_pass<NCH>(acc, p.WgT, my_j, my_dz, ns, lane, d);
+        if (p.dx_mats & 2) bwd_axpy_pass<NCH>(acc, p.WuT, my_j, my_du, ns, lane, d);
       }
     }
 #pragma unroll
@@ -186,6 +190,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dx_kernel(const BwdParams p
       const int k0 = (i * 32 + lane) * 8;
       if (k0 < d) {
         float4* dst = reinterpret_cast<float4*>(p.dx + static_cast<size_t>(t) * d + k0);
+        if (p.dx_accumulate) {
+          const float4 a = dst[0], b = dst[1];
+          acc[i][0] += a.x; acc[i][1] += a.y; acc[i][2] += a.z; acc[i][3] += a.w;
+          acc[i][4] += b.x; acc[i][5] += b.y; acc[i][6] += b.z; acc[i][7] += b.w;
+        }
         dst[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
         dst[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
       }

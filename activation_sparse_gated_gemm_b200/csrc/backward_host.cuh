@@ -61,6 +61,9 @@ twell_status launch_bwd_pass(void (*kern)(BwdParams), size_t smem, const BwdPara
   return launch(kern, dim3(blocks), dim3(WARPS * 32), smem, s, p);
 }
 
+// Wg and Wu bytes above which the per-token dx pass runs once per matrix.
+constexpr size_t kDxSplitBytes = 64u << 20;
+
 // The per-token dx pass of the rows that fit.
 template <int NCH>
 twell_status launch_bwd_dx_n(const BwdParams& p, int sms, cudaStream_t s) {
@@ -136,7 +139,19 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
     TW_TRY(launch(bwd_records_kernel, dim3(std::max(rb, 1)), dim3(256), 0, s, p0, static_cast<const float*>(ubuf)));
     TW_TRY(cuda_ok(cudaGetLastError()));
   }
-  if (!tc_dx) TW_TRY(launch_bwd_dx(p0, sms, s));
+  if (!tc_dx) {
+    // 1b. dx of the rows that fit, per token. When Wg and Wu together would not
+    // stay in L2 beside the streamed rows, one pass per matrix (the second
+    // adding into dx) keeps each pass's gathered rows resident.
+    p0.dx_mats = 3;
+    if (2ull * static_cast<size_t>(f) * d * 2 > kDxSplitBytes) {
+      p0.dx_mats = 1;
+      TW_TRY(launch_bwd_dx(p0, sms, s));
+      p0.dx_mats = 2;
+      p0.dx_accumulate = 1;
+    }
+    TW_TRY(launch_bwd_dx(p0, sms, s));
+  }
   if (tc_dx) {
     // 1b. dx of every token = [dz | du | dz_lo | du_lo] [Wg; Wu; Wg; Wu]^T on
     // the tensor cores, the rows that fit scattered token-major into the
