@@ -102,14 +102,6 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
                               int sms, bool tc_dx = false) {
   const int nT = f / 128;
   BwdWorkspace w = bwd_carve(ws, T, d, f, tw->W);
-  // 0. dh = dy . Wd^T for every token, fp32 [T][f], in the [z | u] region
-  // (free until the overflow rows' dense branch below). K is split over the
-  // grid, with partial sums added into zeroed rows, when the output tiles
-  // cannot fill it.
-  const long long dh_tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((f + kBN - 1) / kBN);
-  if (dh_tiles < sms) TW_TRY(zero_async(s, sms, w.zu, static_cast<size_t>(T) * f * sizeof(float)));
-  TW_TRY(f32_gemm_impl(dy, T, Wd, f, d, w.zu, f, dev_status, s, sms));
-  // 1. rows that fit: per-token pass over their stored slots
   BwdParams p0{};
   p0.x = x;
   p0.WgT = WgT;
@@ -127,12 +119,42 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
   p0.dx = dx;
   p0.s_rec = w.rec;
   p0.dev_status = dev_status;
-  {
-    // 1a. the records from dense u = x Wu^T (a second tensor-core GEMM, into the
-    // idle half of the [z | u] region) and dh, in place of the per-slot dot
-    // pass that gathers a Wu row for every stored slot
+  // 0. the records {h, du, dz, t} of the stored slots of the rows that fit,
+  // from dh = dy . Wd^T and u = x Wu^T on the tensor cores (cheaper than a
+  // dot product over a gathered weight row per slot).
+  const long long dh_tiles = static_cast<long long>((T + kBM - 1) / kBM) * ((f + kBN - 1) / kBN);
+  if (dh_tiles >= sms) {
+    // The output tiles fill the GPU without splitting K: two GEMMs whose
+    // epilogues take only the stored slots' entries, dh_j into the records
+    // first, then the records from u_j (dh and u are never written in full).
+    const uint16_t* a_op[2] = {dy, x};
+    const uint16_t* b_op[2] = {Wd, WuT};
+    for (int pass = 0; pass < 2; ++pass) {
+      CUtensorMap ma, mb;
+      if (!make_map(&ma, a_op[pass], d, T, kBK, kBM) || !make_map(&mb, b_op[pass], d, f, kBK, kBN))
+        return TWELL_ERR_CUDA;
+      GemmParams q{};
+      q.M = T;
+      q.N = f;
+      q.K = d;
+      q.counts = const_cast<int16_t*>(tw->counts);
+      q.idx = const_cast<int16_t*>(tw->idx);
+      q.vals = const_cast<uint16_t*>(tw->vals);
+      q.row_ovf = const_cast<uint8_t*>(tw->row_ovf);
+      q.nT = nT;
+      q.W = tw->W;
+      q.s_rec = w.rec;
+      q.slots_pass = pass;
+      q.dev_status = dev_status;
+      TW_TRY(launch_gemm<kModeSlots>(ma, mb, mb, q, gemm_grid(T, f, kBN, sms), s));
+    }
+  } else {
+    // Small batches: both products in full, fp32 [T][f] in the [z | u] region
+    // (free until the overflow rows' dense branch below), with K split over
+    // the grid (partial sums added into zeroed rows), then the records.
     float* ubuf = w.zu + static_cast<size_t>(T) * f;
-    if (dh_tiles < sms) TW_TRY(zero_async(s, sms, ubuf, static_cast<size_t>(T) * f * sizeof(float)));
+    TW_TRY(zero_async(s, sms, w.zu, static_cast<size_t>(T) * f * 2 * sizeof(float)));
+    TW_TRY(f32_gemm_impl(dy, T, Wd, f, d, w.zu, f, dev_status, s, sms));
     TW_TRY(f32_gemm_impl(x, T, WuT, f, d, ubuf, f, dev_status, s, sms));
     const long long pairs = static_cast<long long>(T) * nT;  // four per warp, eight warps per block
     const int rb = static_cast<int>(std::min<long long>((pairs + 31) / 32, 8LL * sms));

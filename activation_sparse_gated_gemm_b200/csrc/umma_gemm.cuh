@@ -35,10 +35,17 @@
 //   kModeBwdDh  -- dh = dy . Wd^T (B = Wd, K-major) with the backward's
 //                  elementwise step in the epilogue: from the stored z and u,
 //                  dz = dh u [z > 0], du = dh ReLU(z), h = ReLU(z) u, each kept
-//                  as bf16 plus bf16 remainder, written row-major as
-//                  [dz | du | dz_lo | du_lo] (the A operand of dx) and
-//                  transposed, unit-major over tokens (the A operands of the
-//                  weight gradients).
+//                  as bf16 plus bf16 remainder, written token-major as
+//                  [dz | du | dz_lo | du_lo | h | h_lo] (the A operand of dx
+//                  over its first 4N columns, and read MN-major with the
+//                  tokens as K, of the weight gradients).
+//   kModeSlots  -- C = A . B^T as in kModeF32, but only the entries at the
+//                  stored slots of a TwELL pack leave the accumulator: with
+//                  slots_pass 0 (A = dy, B = Wd) each slot's dh_j goes to its
+//                  record; with slots_pass 1 (A = x, B = Wu) the record becomes
+//                  {h = g u_j, du = dh_j g, dz = dh_j u_j, token} from u_j, the
+//                  stored g and the dh_j left there (the backward's records
+//                  without writing dh and u in full).
 //   kModeDown   -- y = h . Wd with Wd read N-major ([K][N] in memory); the
 //                  epilogue stores fp32 rows, optionally scattered through a
 //                  row map (the dense branch of the hybrid route). With the
@@ -75,7 +82,8 @@ enum GemmMode : int {
   kModeF32 = 6,
   kModeZU = 7,
   kModeBwdDh = 8,
-  kModeUnion = 9
+  kModeUnion = 9,
+  kModeSlots = 10
 };
 
 constexpr int kBM = 128;
@@ -177,6 +185,10 @@ struct GemmParams {
   int* slot_row;
   int* ovf_n;
   uint16_t* ovf_h;
+  // kModeSlots: the records ([M][nT][W] float4, beside the TwELL slots of
+  // counts / idx / vals / row_ovf above) and the pass (see the mode's note).
+  float4* s_rec;
+  int slots_pass;
   int* dev_status;
 };
 
@@ -483,7 +495,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(a_dst, &tmA, &full[s], kc * kBK, m_blk * kBM);
           }
           if (MODE == kModeTwell || MODE == kModeRelu || MODE == kModeActivity || MODE == kModeF32 ||
-              MODE == kModeBwdDh) {
+              MODE == kModeBwdDh || MODE == kModeSlots) {
             tma_load_2d(b_dst, &tmB0, &full[s], kc * kBK, n_blk * kBN);
           } else if (kStacked) {
             tma_load_2d(b_dst, &tmB0, &full[s], kc * kBK, n_blk * 128);
@@ -920,6 +932,82 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             store_h32(h, p.out + static_cast<size_t>(my_row) * p.ldo, col, p.N, p.h_split != 0);
           }
         }
+      } else if (MODE == kModeSlots) {
+        // Per row (the thread's TMEM lane) and each of the block's two TwELL
+        // tiles: the tile's stored slots, ascending, are walked beside its four
+        // 32-column chunks; a half-chunk that holds one of the row's slots is
+        // parked in the thread's row of the shared staging buffer and the
+        // slot's entry read back from there. A slot whose column is not in its
+        // own tile raises TWELL_ERR_INDEX and (second pass) gets a zero record,
+        // so that it adds nothing downstream.
+        uint32_t* vrow = ebuf + lane * kEpiPitch;
+        const bool row_ok = my_row < M && p.row_ovf[my_row] == 0;
+        bool bad = false;
+        int ptr = 0, n = 0, iq_at = -1;
+        size_t base = 0;
+        uint4 iq = make_uint4(0u, 0u, 0u, 0u);  // the slot indices iq_at .. iq_at + 7
+        auto cur_j = [&]() -> int {  // column of slot ptr (a large value past the last)
+          if (ptr >= n) return 0x7fffffff;
+          if ((ptr & ~7) != iq_at) {
+            iq_at = ptr & ~7;
+            iq = *reinterpret_cast<const uint4*>(p.idx + base + iq_at);  // W is a multiple of 8
+          }
+          const uint32_t w2 = (ptr & 4) ? ((ptr & 2) ? iq.w : iq.z) : ((ptr & 2) ? iq.y : iq.x);
+          return static_cast<int16_t>((ptr & 1) ? (w2 >> 16) : (w2 & 0xffffu));
+        };
+        auto drop = [&]() {  // slot ptr is not in its tile
+          bad = true;
+          if (p.slots_pass == 1) p.s_rec[base + ptr] = make_float4(0.f, 0.f, 0.f, __int_as_float(my_row));
+          ++ptr;
+        };
+#pragma unroll 1
+        for (int k = 0; k < kBN / 32; ++k) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(k * 32), r);
+          tmem_wait_ld(r);
+          if (k == kBN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+          }
+          const int c = n_blk * 2 + (k >> 2);
+          if (!row_ok || c >= p.nT) continue;
+          if ((k & 3) == 0) {
+            while (ptr < n) drop();  // the previous tile's slots past its last column
+            base = (static_cast<size_t>(my_row) * p.nT + c) * p.W;
+            n = min(max(static_cast<int>(p.counts[static_cast<size_t>(my_row) * p.nT + c]), 0), p.W);
+            ptr = 0;
+            iq_at = -1;
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int wlo = c * 128 + (k & 3) * 32 + 16 * h, whi = wlo + 16;
+            int j = cur_j();
+            if (j < whi) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) vrow[e] = r[16 * h + e];
+              while (j < whi) {
+                if (j >= wlo) {
+                  const float v = __uint_as_float(vrow[j - wlo]);
+                  float4* rec = p.s_rec + base + ptr;
+                  if (p.slots_pass == 0) {
+                    reinterpret_cast<float*>(rec)[0] = v;  // dh_j, until the second pass
+                  } else {
+                    const float dh = reinterpret_cast<const float*>(rec)[0];
+                    const float g = __uint_as_float(static_cast<uint32_t>(p.vals[base + ptr]) << 16);
+                    *rec = make_float4(g * v, dh * g, dh * v, __int_as_float(my_row));
+                  }
+                  ++ptr;
+                } else {
+                  drop();  // below this half-chunk: outside the tile, or out of order
+                }
+                j = cur_j();
+              }
+            }
+          }
+        }
+        while (ptr < n) drop();
+        if (bad) raise_status(p.dev_status, kDevIndex);
       } else {  // kModeDown, kModeF32: fp32 rows (through the row map when given)
         int orow = my_row;
         bool valid = my_row < M;
