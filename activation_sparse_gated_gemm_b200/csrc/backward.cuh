@@ -9,11 +9,11 @@
 //   dWd[j, :] = sum_t h_tj dy_t, dWu[:, j] = sum_t du_tj x_t, dWg[:, j] = sum_t dz_tj x_t
 //
 // Rows that fit the ELL width take three passes over their stored units:
-//   0. dh = dy . Wd^T for every token on the tensor cores (a plain dense
-//      contraction, [T][f] fp32): cheaper than gathering a row of Wd per slot;
-//   1. u = x . Wu^T for every token on the tensor cores as well, and per
-//      stored slot the record {h, du, dz, token} from u_j, dh_j and the stored
-//      g (cheaper than a dot product over a gathered Wu row per slot);
+//   0. dh = dy . Wd^T and u = x . Wu^T on the tensor cores (plain dense
+//      contractions: cheaper than gathering a Wd and a Wu row per slot), and
+//      per stored slot the record {h, du, dz, token} from u_j, dh_j and the
+//      stored g (in the GEMMs' epilogues, or by bwd_records_kernel from the
+//      full products for small batches);
 //   1b. per token (one warp per token, like the forward's fused kernel): dx_t
 //      by two row axpys with du_j, dz_j from the records;
 //   2. per hidden unit: the records are sorted by column (count, scan, scatter

@@ -364,8 +364,8 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
  *   overwritten; the layouts of WgT, WuT and Wd)
  * tw, ovf_rows and n_ovf are the outputs of twell_ffn_hybrid_forward on the
  * same x (the gate form: tw's values are the bf16 gate). dh and u are formed
- * for every token by two tensor-core GEMMs (dy Wd^T and x Wu^T, fp32 sums),
- * and each stored slot's record {h, du, dz} from them. Rows that fit use
+ * by two tensor-core GEMMs (dy Wd^T and x Wu^T, fp32 sums), whose epilogues
+ * keep only the stored slots' entries as each slot's record {h, du, dz}. Rows that fit use
  * their stored slots with the stored bf16 gate g (h = g u), so the result is
  * the method's, within one bf16 rounding per term of the exact gradients;
  * their weight gradients are summed per hidden unit over a column sort of the
