@@ -212,8 +212,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dx_kernel(const BwdParams p
 // {h = g u_j, du = dh_j g, dz = dh_j u_j, t}. Eight lanes per (row, tile), four
 // consecutive tiles per warp, the lanes of a tile taking its slots side by side
 // (a thread per tile walking its slots one after another took 0.12 ms at the
-// 0.5B layer). A stored index outside [0, f) raises TWELL_ERR_INDEX and leaves
-// its record unwritten; the dx pass skips such slots too.
+// 0.5B layer). A stored index outside its own column tile raises
+// TWELL_ERR_INDEX and gets a zero record, so that it adds nothing downstream.
 __global__ void __launch_bounds__(256) bwd_records_kernel(const BwdParams p, const float* __restrict__ u) {
   griddep_launch_dependents();
   griddep_wait();
@@ -232,11 +232,13 @@ __global__ void __launch_bounds__(256) bwd_records_kernel(const BwdParams p, con
     const size_t base = static_cast<size_t>(i) * p.W;
     const float* urow = u + static_cast<size_t>(t) * p.f;
     const float* dhrow = p.dh + static_cast<size_t>(t) * p.f;
+    const int c = static_cast<int>(i - static_cast<long long>(t) * p.nT);
     for (int k = lane & 7; k < n; k += 8) {
       const int j = p.idx[base + k];
       const float gv = __uint_as_float(static_cast<uint32_t>(p.vals[base + k]) << 16);
-      if (j < 0 || j >= p.f) {
+      if (j < c * 128 || j >= (c + 1) * 128 || j >= p.f) {
         bad = true;
+        p.s_rec[base + k] = make_float4(0.f, 0.f, 0.f, __int_as_float(t));
         continue;
       }
       const float uj = __ldg(urow + j), dh = __ldg(dhrow + j);

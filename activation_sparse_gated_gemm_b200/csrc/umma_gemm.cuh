@@ -979,30 +979,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptr = 0;
             iq_at = -1;
           }
+          const int tile_hi = (c + 1) * 128;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int wlo = c * 128 + (k & 3) * 32 + 16 * h, whi = wlo + 16;
-            int j = cur_j();
-            if (j < whi) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) vrow[e] = r[16 * h + e];
-              while (j < whi) {
-                if (j >= wlo) {
-                  const float v = __uint_as_float(vrow[j - wlo]);
-                  float4* rec = p.s_rec + base + ptr;
-                  if (p.slots_pass == 0) {
-                    reinterpret_cast<float*>(rec)[0] = v;  // dh_j, until the second pass
-                  } else {
-                    const float dh = reinterpret_cast<const float*>(rec)[0];
-                    const float g = __uint_as_float(static_cast<uint32_t>(p.vals[base + ptr]) << 16);
-                    *rec = make_float4(g * v, dh * g, dh * v, __int_as_float(my_row));
-                  }
-                  ++ptr;
-                } else {
-                  drop();  // below this half-chunk: outside the tile, or out of order
-                }
-                j = cur_j();
+            bool staged = false;
+            while (ptr < n) {
+              const int j = cur_j();
+              if (j < wlo || j >= tile_hi) {
+                drop();  // below this half-chunk (outside the tile, or out of order) or past the tile
+                continue;
               }
+              if (j >= whi) break;  // a later half-chunk's
+              if (!staged) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) vrow[e] = r[16 * h + e];
+                staged = true;
+              }
+              const float v = __uint_as_float(vrow[j - wlo]);
+              float4* rec = p.s_rec + base + ptr;
+              if (p.slots_pass == 0) {
+                reinterpret_cast<float*>(rec)[0] = v;  // dh_j, until the second pass
+              } else {
+                const float dh = reinterpret_cast<const float*>(rec)[0];
+                const float g = __uint_as_float(static_cast<uint32_t>(p.vals[base + ptr]) << 16);
+                *rec = make_float4(g * v, dh * g, dh * v, __int_as_float(my_row));
+              }
+              ++ptr;
             }
           }
         }

@@ -20,6 +20,18 @@ from tests.test_gpu_parity import IDS, SMALL
 pytestmark = pytest.mark.gpu
 
 GRADS = ("dx", "dWgT", "dWuT", "dWd")
+
+# Batches whose dh and u output tiles fill the GPU, so that the records come
+# from the GEMMs' slot epilogues (the small configurations build them from the
+# full products): a ragged last M tile, an odd number of column tiles (the
+# last 256-column block holds one tile), d of 3 x 64, heavy rows.
+LC = synth.LayerConfig
+MID = [
+    LC("slots_mid", T=2000, d=256, f=4608, tile=128, W=16, density=0.03, sigma=0.5, heavy_frac=0.05,
+       heavy_lo=0.2, heavy_hi=0.35),
+    LC("slots_odd_tiles", T=2500, d=192, f=3968, tile=128, W=8, density=0.02, sigma=0.5),
+]
+MID_IDS = [c.name for c in MID]
 TIGHT = 1e-3
 CONTRACT = 2e-2
 
@@ -89,7 +101,7 @@ def dense_branch_bounds(L, dy_bits, ovf, rows=None, cols=None, k=2.0**-15) -> di
     return out
 
 
-@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+@pytest.mark.parametrize("cfg", SMALL + MID, ids=IDS + MID_IDS)
 def test_hybrid_backward(cfg):
     L = synth.make_layer(cfg, seed=0)
     dy = make_dy(cfg.T, cfg.d, 0)
@@ -190,7 +202,7 @@ def test_dense_backward_baseline(cfg):
         assert np.all(err <= bound), (k, float((err / bound).max()))
 
 
-@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+@pytest.mark.parametrize("cfg", SMALL + MID, ids=IDS + MID_IDS)
 def test_tensor_core_weight_gradients(cfg):
     """The tensor-core form of the weight gradients (dz, du, h of the rows that
     fit as bf16 value plus remainder, GEMMs over the tokens) against the
@@ -238,7 +250,7 @@ def _forward_for_backward(L, cfg):
     return dev, tw, ovf_rows, n_ovf, st
 
 
-@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+@pytest.mark.parametrize("cfg", SMALL + MID, ids=IDS + MID_IDS)
 def test_tensor_core_dx(cfg):
     """The tensor-core form of dx (dz, du of the rows that fit as bf16 value
     plus remainder, one GEMM against [Wg; Wu]) against the oracle: within the
@@ -288,3 +300,42 @@ def test_full_size_tensor_core_dx():
     ref = O.hybrid_ffn_backward(L["x"][rows], L["WgT"], L["WuT"], L["Wd"], dy_bits[rows], cfg.tile, cfg.W)
     b = dense_branch_bounds(L, dy_bits, rows, rows=rows)
     assert_grad_close(got[rows], ref["dx"], "dx", b["dx"])
+
+
+@pytest.mark.parametrize("cfg", [SMALL[0], MID[0]], ids=["full_products", "slot_epilogues"])
+def test_a_stored_index_outside_its_tile_is_reported_and_adds_nothing(cfg):
+    """One stored slot of a row that fits is moved to a column of another tile
+    (still inside [0, f)): the backward raises TWELL_ERR_INDEX, every gradient
+    stays finite, and the rows and units that slot does not touch keep the
+    oracle's values."""
+    L = synth.make_layer(cfg, seed=0)
+    dy_bits = make_dy(cfg.T, cfg.d, 11)
+    dev, tw, ovf_rows, n_ovf, st = _forward_for_backward(L, cfg)
+    assert tl.status_get(st) == 0
+    T, d, f, W = cfg.T, cfg.d, cfg.f, cfg.W
+    counts = tw.counts.cpu().numpy()
+    row_ovf = tw.row_ovf.cpu().numpy()
+    cand = [(t, c) for t in range(T) if not row_ovf[t] for c in range(f // 128) if counts[t, c] > 0]
+    t, c = cand[len(cand) // 2]
+    idx = tw.idx.view(T, f // 128, W)
+    j_old = int(idx[t, c, 0].item())
+    idx[t, c, 0] = (j_old + 128) % f  # the same unit of the next tile
+    dy = tl.to_device_bf16(dy_bits)
+    dx = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    dW = [torch.full((f, d), float("nan"), dtype=torch.float32, device="cuda") for _ in range(3)]
+    wsb = torch.empty(tl.backward_workspace_bytes(T, d, f, W), dtype=torch.uint8, device="cuda")
+    tl.ffn_hybrid_backward(dev["x"], dev["WgT"], dev["WuT"], dev["Wd"], dy, tw, ovf_rows, n_ovf,
+                           dx, dW[0], dW[1], dW[2], wsb, st)
+    assert tl.status_get(st) == tl.TWELL_ERR_INDEX
+    got = {"dx": dx.double().cpu().numpy(), **{k: v.double().cpu().numpy() for k, v in zip(GRADS[1:], dW)}}
+    for k in GRADS:
+        assert np.isfinite(got[k]).all(), k
+    ref = O.hybrid_ffn_backward(L["x"], L["WgT"], L["WuT"], L["Wd"], dy_bits, cfg.tile, cfg.W)
+    keep_rows = np.setdiff1d(np.arange(T), [t])
+    keep_units = np.setdiff1d(np.arange(f), [j_old, (j_old + 128) % f])
+    ovf = ref["ovf_rows"]
+    b = dense_branch_bounds(L, dy_bits, ovf, rows=keep_rows) if ovf.size else {}
+    assert_grad_close(got["dx"][keep_rows], ref["dx"][keep_rows], "dx", b.get("dx"))
+    bw = dense_branch_bounds(L, dy_bits, ovf, cols=keep_units) if ovf.size else {}
+    for k in GRADS[1:]:
+        assert_grad_close(got[k][keep_units], ref[k][keep_units], k, bw.get(k))
