@@ -946,6 +946,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int ptr = 0, n = 0, iq_at = -1;
         size_t base = 0;
         uint4 iq = make_uint4(0u, 0u, 0u, 0u);  // the slot indices iq_at .. iq_at + 7
+        // second pass: dh_j and g of the tile's first eight slots, loaded as
+        // the tile starts so that the walk does not wait on them one by one
+        float dh8[8];
+        uint4 g8 = make_uint4(0u, 0u, 0u, 0u);
         auto cur_j = [&]() -> int {  // column of slot ptr (a large value past the last)
           if (ptr >= n) return 0x7fffffff;
           if ((ptr & ~7) != iq_at) {
@@ -978,6 +982,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             n = min(max(static_cast<int>(p.counts[static_cast<size_t>(my_row) * p.nT + c]), 0), p.W);
             ptr = 0;
             iq_at = -1;
+            if (p.slots_pass == 1 && n > 0) {
+              g8 = *reinterpret_cast<const uint4*>(p.vals + base);  // W is a multiple of 8
+#pragma unroll
+              for (int e = 0; e < 8; ++e) dh8[e] = e < n ? reinterpret_cast<const float*>(p.s_rec + base + e)[0] : 0.0f;
+            }
           }
           const int tile_hi = (c + 1) * 128;
 #pragma unroll
@@ -1001,8 +1010,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               if (p.slots_pass == 0) {
                 reinterpret_cast<float*>(rec)[0] = v;  // dh_j, until the second pass
               } else {
-                const float dh = reinterpret_cast<const float*>(rec)[0];
-                const float g = __uint_as_float(static_cast<uint32_t>(p.vals[base + ptr]) << 16);
+                float dh;
+                uint32_t gb;
+                if (ptr < 8) {
+                  dh = dh8[0];
+#pragma unroll
+                  for (int e = 1; e < 8; ++e) dh = ptr == e ? dh8[e] : dh;
+                  const uint32_t w2 = (ptr & 4) ? ((ptr & 2) ? g8.w : g8.z) : ((ptr & 2) ? g8.y : g8.x);
+                  gb = (ptr & 1) ? (w2 & 0xffff0000u) : (w2 << 16);
+                } else {
+                  dh = reinterpret_cast<const float*>(rec)[0];
+                  gb = static_cast<uint32_t>(p.vals[base + ptr]) << 16;
+                }
+                const float g = __uint_as_float(gb);
                 *rec = make_float4(g * v, dh * g, dh * v, __int_as_float(my_row));
               }
               ++ptr;
