@@ -265,7 +265,10 @@ __device__ __forceinline__ int source_rows(const SlotSource& s) {
 
 // SCATTER == false: colcnt[j] += number of slots with column j.
 // SCATTER == true: each slot's record is copied to list[colptr[j] +
-// cursor[j]++] (the order inside a column is that of the atomics).
+// cursor[j]++] (the order inside a column is that of the atomics). Eight
+// lanes per (row, tile), four consecutive tiles per warp, the lanes of a tile
+// taking its slots side by side (a warp per tile left most lanes idle at the
+// configured densities).
 template <bool SCATTER>
 __global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colptr, float4* list) {
   griddep_launch_dependents();
@@ -273,13 +276,16 @@ __global__ void bwd_columns_kernel(SlotSource src, int* colcnt, const int* colpt
   const int lane = threadIdx.x & 31;
   const int rows = source_rows(src);
   const long long pairs = static_cast<long long>(rows) * src.nT;
+  const long long groups = (pairs + 3) / 4;
   const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < pairs;
-       w += nw) {
+  for (long long g = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); g < groups;
+       g += nw) {
+    const long long w = g * 4 + (lane >> 3);
+    if (w >= pairs) continue;
     const int t = static_cast<int>(w / src.nT);
     if (src.skip_ovf && src.row_ovf[t]) continue;
     const int n = min(max(static_cast<int>(src.counts[w]), 0), src.W);
-    for (int k = lane; k < n; k += 32) {
+    for (int k = lane & 7; k < n; k += 8) {
       const size_t slot = static_cast<size_t>(w) * src.W + k;
       const int j = src.idx[slot];
       if (j < 0 || j >= src.f) continue;
@@ -350,7 +356,11 @@ struct WgradParams {
 
 // One warp per (hidden unit j, 256-wide slice of d): lane l owns 8 consecutive
 // elements of the slice; the unit's slots are read 32 at a time (lane e
-// fetches entry e's scalars and row), then broadcast one by one.
+// fetches entry e's scalars and row), then broadcast one by one. The warps run
+// slice by slice (every unit of slice 0 first), so the x and dy columns being
+// gathered at any time are one or two slices of them (T x 512 bytes each),
+// which stay in L2; unit by unit, every warp in flight touched all of x and
+// dy.
 __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
   griddep_launch_dependents();
   griddep_wait();
@@ -358,8 +368,9 @@ __global__ void __launch_bounds__(256) bwd_wgrad_kernel(const WgradParams p) {
   const int slices = (p.d + 255) / 256;
   const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (w >= static_cast<long long>(p.f) * slices) return;
-  const int j = static_cast<int>(w / slices);
-  const int k0 = static_cast<int>(w - static_cast<long long>(j) * slices) * 256 + lane * 8;
+  const int sl = static_cast<int>(w / p.f);
+  const int j = static_cast<int>(w - static_cast<long long>(sl) * p.f);
+  const int k0 = sl * 256 + lane * 8;
   const bool mine = k0 < p.d;
   float ag[8], au[8], ad[8];
 #pragma unroll
