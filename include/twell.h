@@ -376,7 +376,9 @@ twell_status twell_relu_dense_ffn_forward(const uint16_t* x, const uint16_t* W1T
  * their share of the weight gradients added by three GEMMs over their tokens.
  * workspace: twell_backward_workspace_bytes(T, d, f, tw->W) bytes (worst case:
  * every row overflows). T == 0 zeroes the weight gradients. Errors as for
- * twell_ffn_hybrid_forward; T * (f / 128) * W must stay below 2^31.
+ * twell_ffn_hybrid_forward; a stored index outside its own column tile raises
+ * TWELL_ERR_INDEX and that slot adds nothing to any gradient. T * (f / 128) *
+ * W must stay below 2^31.
  */
 size_t twell_backward_workspace_bytes(int T, int d, int f, int W);
 twell_status twell_ffn_hybrid_backward(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT,
