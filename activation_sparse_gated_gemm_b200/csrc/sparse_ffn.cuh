@@ -36,6 +36,11 @@ struct SparseParams {
   uint8_t* route_flags;
   int* route_rows;
   int* route_n;
+  // sparse_ffn_warp_kernel: when set (a zeroed int), every warp of the grid
+  // draws its next work unit from this one counter instead of from its
+  // block's share, so that blocks whose tokens hold more slots do not set the
+  // kernel's end.
+  int* work_next;
   int* dev_status;
 };
 
@@ -143,19 +148,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) sparse_ffn_warp_kernel(const Sp
   const uint64_t stream_pol = l2_evict_first_policy();
   // Block b owns the contiguous tokens [t_begin, t_end); its warps take them
   // one at a time from a shared counter, so a warp that drew light tokens
-  // keeps working while another finishes a heavy one.
+  // keeps working while another finishes a heavy one. With work_next every
+  // warp of the grid takes them from that one counter instead.
   __shared__ int next_unit;
   const int units_per_token = (p.nT + p.unit_tiles - 1) / p.unit_tiles;
   const bool partial = units_per_token > 1;
   const long long n_units = static_cast<long long>(p.T) * units_per_token;
   const int u_begin = static_cast<int>(n_units * blockIdx.x / gridDim.x);
-  const int u_end = static_cast<int>(n_units * (blockIdx.x + 1) / gridDim.x);
+  const int u_end = p.work_next != nullptr ? static_cast<int>(n_units)
+                                           : static_cast<int>(n_units * (blockIdx.x + 1) / gridDim.x);
   if (threadIdx.x == 0) next_unit = u_begin;
   __syncthreads();
 #pragma unroll 1
   for (;;) {
     int u = 0;
-    if (lane == 0) u = atomicAdd(&next_unit, 1);
+    if (lane == 0) u = p.work_next != nullptr ? atomicAdd(p.work_next, 1) : atomicAdd(&next_unit, 1);
     u = __shfl_sync(0xffffffffu, u, 0);
     if (u >= u_end) break;
     const int t = u / units_per_token;

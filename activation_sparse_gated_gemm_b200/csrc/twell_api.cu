@@ -209,13 +209,17 @@ int gemm_grid(int M, int N, int tile_n, int sms) {
 }
 
 // With slot_of_row set, the GEMM also writes the exact ReLU(z) of every
-// overflowing (row, tile) into ovf_h at the row's compact slot (see GemmParams).
+// overflowing (row, tile) into ovf_h at the row's compact slot (see GemmParams),
+// and the int after *ovf_n (the sparse step's work counter) is zeroed with it;
+// work_next alone: that counter is zeroed beside the overflow flags.
 twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d, int f, const twell_t* tw,
                             int32_t* dev_status, cudaStream_t s, int sms, const int* M_dev = nullptr,
                             int* slot_of_row = nullptr, int* slot_row = nullptr, int* ovf_n = nullptr,
-                            uint16_t* ovf_h = nullptr) {
-  if (slot_of_row != nullptr) {
-    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), slot_of_row, static_cast<size_t>(T) * 4, ovf_n, 4));
+                            uint16_t* ovf_h = nullptr, int* work_next = nullptr) {
+  if (work_next != nullptr && slot_of_row == nullptr) {
+    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), work_next, 4));
+  } else if (slot_of_row != nullptr) {
+    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), slot_of_row, static_cast<size_t>(T) * 4, ovf_n, 8));
   } else {
     TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
   }
@@ -242,13 +246,14 @@ twell_status gate_pack_impl(const uint16_t* x, const uint16_t* WgT, int T, int d
 
 // Gate and up GEMM in one pass; TwELL of the gate pattern holding h = z * u.
 // With slot_of_row set, the GEMM also writes the exact h of every overflowing
-// (row, tile) into ovf_h at the row's compact slot (see GemmParams).
+// (row, tile) into ovf_h at the row's compact slot (see GemmParams), and the
+// int after *ovf_n (the sparse step's work counter) is zeroed with it.
 twell_status gate_up_pack_impl(const uint16_t* x, const uint16_t* WgT, const uint16_t* WuT, int T, int d, int f,
                                const twell_t* tw, int32_t* dev_status, cudaStream_t s, int sms,
                                int* slot_of_row = nullptr, int* slot_row = nullptr, int* ovf_n = nullptr,
                                uint16_t* ovf_h = nullptr) {
   if (slot_of_row != nullptr) {
-    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), slot_of_row, static_cast<size_t>(T) * 4, ovf_n, 4));
+    TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T), slot_of_row, static_cast<size_t>(T) * 4, ovf_n, 8));
   } else {
     TW_TRY(zero_async(s, sms, tw->row_ovf, static_cast<size_t>(T)));
   }
@@ -334,8 +339,9 @@ twell_status sparse_launch(const SparseParams& p, int d, int sms, cudaStream_t s
 
 twell_status sparse_impl(const uint16_t* x, const uint16_t* WuT, const uint16_t* Wd, int T, int d, int f,
                          const twell_t* tw, int skip, float* y, int32_t* dev_status, cudaStream_t s, int sms,
-                         bool down_only = false, bool y_zeroed = false) {
+                         bool down_only = false, bool y_zeroed = false, int* work_next = nullptr) {
   SparseParams p{};
+  p.work_next = work_next;
   p.x = x;
   p.WuT = WuT;
   p.Wd = Wd;
@@ -411,8 +417,8 @@ twell_status sparse_small_impl(const uint16_t* x, const uint16_t* WuT, const uin
 
 // Down projection from a TwELL of hidden activations (per-token gathers of Wd rows).
 twell_status down_impl(const uint16_t* Wd, int T, int d, int f, const twell_t* tw, int skip, float* y,
-                       int32_t* dev_status, cudaStream_t s, int sms) {
-  return sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, skip, y, dev_status, s, sms, true);
+                       int32_t* dev_status, cudaStream_t s, int sms, int* work_next = nullptr) {
+  return sparse_impl(nullptr, nullptr, Wd, T, d, f, tw, skip, y, dev_status, s, sms, true, false, work_next);
 }
 
 twell_status dense_down_impl(const uint16_t* h_buf, int M, const int* M_dev, const uint16_t* Wd, int d, int f,
@@ -866,7 +872,7 @@ twell_status twell_ffn_hybrid_forward_tc_up(const uint16_t* x, const uint16_t* W
   TW_TRY(gate_up_pack_impl(x, WgT, WuT, T, d, f, tw, dev_status, s, sms, slot_of_row, slot_row, n_slots, ho));
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms));
+  TW_TRY(down_impl(Wd, T, d, f, tw, 1, y, dev_status, s, sms, n_slots + 1));
   return slot_branch_impl(tw, Wd, T, d, f, slot_row, n_slots, ho, y, dev_status, s, sms);
 }
 
@@ -913,10 +919,13 @@ twell_status twell_ffn_hybrid_forward(const uint16_t* x, const uint16_t* WgT, co
     TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms, false, zero_y));
     return dense_impl(xo, T, n_ovf, WgT, WuT, Wd, d, f, ho, true, ovf_rows, y, T, dev_status, s, sms);
   }
-  TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms));
+  // the sparse step's work counter in the h region of the dense branch (free until that branch runs)
+  int* work_next = reinterpret_cast<int*>(ho);
+  TW_TRY(gate_pack_impl(x, WgT, T, d, f, tw, dev_status, s, sms, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        work_next));
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms));
+  TW_TRY(sparse_impl(x, WuT, Wd, T, d, f, tw, 1, y, dev_status, s, sms, false, false, work_next));
   return dense_rows_impl(x, WgT, WuT, Wd, T, d, f, ovf_rows, n_ovf, y, xo, ho, dev_status, s, sms);
 }
 
@@ -1012,7 +1021,7 @@ twell_status twell_relu_ffn_hybrid_forward(const uint16_t* x, const uint16_t* W1
   TW_TRY(gate_pack_impl(x, W1T, T, d, f, tw, dev_status, s, sms, nullptr, slot_of_row, slot_row, n_slots, ho));
   TW_TRY(launch(route_kernel, dim3(1), dim3(1024), 0, s, tw->row_ovf, T, ovf_rows, n_ovf, static_cast<const uint16_t*>(nullptr), 0, static_cast<uint16_t*>(nullptr), static_cast<float*>(nullptr)));
   TW_TRY(cuda_ok(cudaGetLastError()));
-  TW_TRY(down_impl(W2, T, d, f, tw, 1, y, dev_status, s, sms));
+  TW_TRY(down_impl(W2, T, d, f, tw, 1, y, dev_status, s, sms, n_slots + 1));
   return slot_branch_impl(tw, W2, T, d, f, slot_row, n_slots, ho, y, dev_status, s, sms);
 }
 
