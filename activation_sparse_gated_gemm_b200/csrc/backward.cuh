@@ -46,6 +46,9 @@ struct BwdParams {
   // whether it adds them to dx instead of storing them
   int dx_mats;
   int dx_accumulate;
+  // dx pass: when set (a zeroed int), every warp of the grid takes its next
+  // token from this one counter instead of from its block's share
+  int* next_row_global;
   int* dev_status;
 };
 
@@ -127,7 +130,7 @@ __device__ __forceinline__ int bwd_build_list(const BwdParams& p, int t, int c0,
 }
 
 // Tokens are handed out one at a time from a per-block counter over the
-// block's contiguous share of the rows.
+// block's contiguous share of the rows, or from one counter for the grid.
 __device__ __forceinline__ int bwd_next_row(int* next_row, int lane) {
   int t = 0;
   if (lane == 0) t = atomicAdd(next_row, 1);
@@ -151,12 +154,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) bwd_dx_kernel(const BwdParams p
                    warp * kListCap;
   const int group_tiles = max(1, kListCap / p.W);
   bool bad_index = false;
-  const int r_end = static_cast<int>(static_cast<long long>(p.rows) * (blockIdx.x + 1) / gridDim.x);
+  const int r_end = p.next_row_global != nullptr
+                        ? p.rows
+                        : static_cast<int>(static_cast<long long>(p.rows) * (blockIdx.x + 1) / gridDim.x);
   if (threadIdx.x == 0) next_row = static_cast<int>(static_cast<long long>(p.rows) * blockIdx.x / gridDim.x);
   __syncthreads();
 #pragma unroll 1
   for (;;) {
-    const int t = bwd_next_row(&next_row, lane);
+    const int t = bwd_next_row(p.next_row_global != nullptr ? p.next_row_global : &next_row, lane);
     if (t >= r_end) break;
     if (p.row_ovf[t]) continue;
     float acc[NCH][8];

@@ -22,6 +22,7 @@ struct BwdWorkspace {
   uint16_t* a2;
   int *colcnt, *colptr;
   float4* list;
+  int* counters;    // work counters of the dx passes
   uint16_t* dense;  // tensor-core form: the rows that fit, [T][6f] bf16 (dz, du, their remainders, h, its remainder)
   int t_pad;
   size_t bytes;
@@ -47,6 +48,7 @@ BwdWorkspace bwd_carve(char* base, int T, int d, int f, int W) {
   w.colptr = reinterpret_cast<int*>(take((static_cast<size_t>(f) + 1) * 4));
   w.list = reinterpret_cast<float4*>(take(s0 * 16));
   w.dense = reinterpret_cast<uint16_t*>(take(3 * static_cast<size_t>(f) * 2 * tp * 2));
+  w.counters = reinterpret_cast<int*>(take(16));
   w.t_pad = static_cast<int>(tp);
   w.bytes = off;
   return w;
@@ -165,12 +167,17 @@ twell_status backward_dx_impl(const uint16_t* x, const uint16_t* WgT, const uint
     // 1b. dx of the rows that fit, per token. When Wg and Wu together would not
     // stay in L2 beside the streamed rows, one pass per matrix (the second
     // adding into dx) keeps each pass's gathered rows resident.
+    // Every warp of a pass takes its tokens from one counter (a zeroed int per
+    // pass), so blocks whose tokens hold more slots do not set its end.
+    TW_TRY(zero_async(s, sms, w.counters, 8));
     p0.dx_mats = 3;
+    p0.next_row_global = w.counters;
     if (2ull * static_cast<size_t>(f) * d * 2 > kDxSplitBytes) {
       p0.dx_mats = 1;
       TW_TRY(launch_bwd_dx(p0, sms, s));
       p0.dx_mats = 2;
       p0.dx_accumulate = 1;
+      p0.next_row_global = w.counters + 1;
     }
     TW_TRY(launch_bwd_dx(p0, sms, s));
   }
