@@ -87,22 +87,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   return r == CUDA_SUCCESS;
 }
 
-// Row-major bf16 matrix [outer][inner] with plain (unswizzled) boxes: a box
-// lands in shared memory as box_outer rows of box_inner elements.
-bool make_map_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                    uint32_t box_outer) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 // ------------------------------------------------------------------ checks
 
 twell_status check_shape(int T, int d, int f) {
