@@ -836,11 +836,12 @@ def run_gpu_backward(args, world, rank, local):
         "speedup_vs_own_dense": dense_ms / step_ms,
         "e2e": {"value": job_rate(T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 4 + 3 * f * d * 4},
-        # per step, dx: the dh and u GEMMs, the records, then the dx pass (tensor-core form: the dense rows
-        # and the dx GEMM), two gathers and three dense-branch GEMMs (9 or 10 launches); weight gradients:
-        # the column sort (four launches) and the per-unit sums, or the dense rows and three zeroed GEMMs
-        # (5 or 7), then the overflow rows' three GEMMs
-        "gpu_launches": ((10 if dx_form == "tensor_cores" else 9) + (10 if dw_form == "tensor_cores" else 8)) * K,
+        # per step, dx: the two slot-epilogue GEMMs (the records), then the tensor-core form's dense rows and
+        # dx GEMM, or the CUDA-core form's counter zeroing and dx pass (two passes when Wg and Wu exceed
+        # 64 MB), two gathers and three dense-branch GEMMs; weight gradients: the column sort (four launches)
+        # and the per-unit sums, or the dense rows and three zeroed GEMMs, then the overflow rows' three GEMMs
+        "gpu_launches": ((9 if dx_form == "tensor_cores" else 9 + (4 * f * d > (64 << 20)))
+                         + (10 if dw_form == "tensor_cores" else 8)) * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
