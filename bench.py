@@ -612,9 +612,10 @@ def run_gpu(args, world, rank, local):
                 "pipelined": "copy-in, compute and copy-out on three streams, two buffer sets",
                 "path": "the library's hybrid forward of the chosen form",
                 "l2": "not flushed: each step touches ~0.26 GB, above the 126 MB L2"},
-        # per step: zeroing, gate (or gate+up) GEMM, routing, sparse step, row gather, two dense-branch GEMMs
-        # (the down projection over tile unions is two launches: its preparation and its GEMM)
-        "gpu_launches": (6 if chosen == "tc_up" else 7) * K,
+        # per step: zeroing, the pack GEMM, routing, the sparse step, then the dense branch: the gate form's row
+        # gather and two GEMMs, or (tc_up and the non-gated layer, which take the routed rows' h from the pack
+        # GEMM) the fill of their other tiles and one down GEMM
+        "gpu_launches": (7 if chosen == "gate" else 6) * K,
         "down_projection": "fused up+down per token" if chosen == "gate" else "per token",
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
