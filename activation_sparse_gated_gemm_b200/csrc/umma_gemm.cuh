@@ -613,6 +613,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t* ebuf = reinterpret_cast<uint32_t*>(smem + kOffEpi) + (warp - 2) * 32 * kEpiPitch;
     uint32_t tph = 0;
     for (int tile = blockIdx.x + buf * gridDim.x; tile < num_tiles; tile += 2 * gridDim.x) {
+      // kModeSlots: the row's slot data for the block's two TwELL tiles (count,
+      // first eight indices, and for the second pass their g and dh), loaded
+      // while the accumulator is still being formed
+      bool pre_skip = true;
+      int pre_n[2] = {0, 0};
+      uint4 pre_iq[2], pre_g8[2];
+      float pre_dh[2][8];
+      if (MODE == kModeSlots) {
+        int mb0, nb0;
+        tile_mn(tile / k_splits, num_m, num_n, group_n, mb0, nb0);
+        const int r0 = mb0 * kBM + q * 32 + lane;
+        pre_skip = r0 >= M || p.row_ovf[r0] != 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = nb0 * 2 + h;
+          pre_iq[h] = pre_g8[h] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pre_dh[h][e] = 0.0f;
+          if (!pre_skip && c < p.nT) {
+            const size_t b = (static_cast<size_t>(r0) * p.nT + c) * p.W;  // W is a multiple of 8
+            pre_n[h] = p.counts[static_cast<size_t>(r0) * p.nT + c];
+            pre_iq[h] = *reinterpret_cast<const uint4*>(p.idx + b);
+            if (p.slots_pass == 1) {
+              pre_g8[h] = *reinterpret_cast<const uint4*>(p.vals + b);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) pre_dh[h][e] = reinterpret_cast<const float*>(p.s_rec + b + e)[0];
+            }
+          }
+        }
+      }
       const bool got = mbar_wait(&tfull[buf], tph, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         *abort_flag = 1;
@@ -941,7 +971,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // own tile raises TWELL_ERR_INDEX and (second pass) gets a zero record,
         // so that it adds nothing downstream.
         uint32_t* vrow = ebuf + lane * kEpiPitch;
-        const bool row_ok = my_row < M && p.row_ovf[my_row] == 0;
+        const bool row_ok = !pre_skip;
         bool bad = false;
         int ptr = 0, n = 0, iq_at = -1;
         size_t base = 0;
@@ -978,15 +1008,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!row_ok || c >= p.nT) continue;
           if ((k & 3) == 0) {
             while (ptr < n) drop();  // the previous tile's slots past its last column
+            const bool second = (k >> 2) != 0;
             base = (static_cast<size_t>(my_row) * p.nT + c) * p.W;
-            n = min(max(static_cast<int>(p.counts[static_cast<size_t>(my_row) * p.nT + c]), 0), p.W);
+            n = min(max(second ? pre_n[1] : pre_n[0], 0), p.W);
             ptr = 0;
-            iq_at = -1;
-            if (p.slots_pass == 1 && n > 0) {
-              g8 = *reinterpret_cast<const uint4*>(p.vals + base);  // W is a multiple of 8
+            iq = second ? pre_iq[1] : pre_iq[0];  // the indices of slots 0 .. 7
+            iq_at = 0;
+            g8 = second ? pre_g8[1] : pre_g8[0];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) dh8[e] = e < n ? reinterpret_cast<const float*>(p.s_rec + base + e)[0] : 0.0f;
-            }
+            for (int e = 0; e < 8; ++e) dh8[e] = second ? pre_dh[1][e] : pre_dh[0][e];
           }
           const int tile_hi = (c + 1) * 128;
 #pragma unroll
