@@ -357,6 +357,8 @@ twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, i
   const uint16_t* bT[3] = {x, x, dy};
   float* outs[3] = {dWgT, dWuT, dWd};
   const int col_hi[3] = {0, f, 4 * f}, col_lo[3] = {2 * f, 3 * f, 5 * f};
+  const size_t wbytes = static_cast<size_t>(f) * d * sizeof(float);
+  TW_TRY(zero_async(s, sms, dWgT, wbytes, dWuT, wbytes, dWd, wbytes));  // the split GEMMs add into them
   for (int i = 0; i < 3; ++i) {
     CUtensorMap mb;
     if (!make_map(&mb, bT[i], d, T, 64, kBK)) return TWELL_ERR_CUDA;
@@ -372,7 +374,6 @@ twell_status backward_dw_tc_impl(const uint16_t* x, const uint16_t* dy, int T, i
     q.ldo = d;
     q.k_splits_max = 32;
     q.split_waves = 1;
-    TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
     TW_TRY(launch_gemm<kModeDown>(ma, mb, mb, q, sms, s));
   }
   return backward_dw_overflow(d, f, n_ovf, dWgT, dWuT, dWd, w, s, sms);

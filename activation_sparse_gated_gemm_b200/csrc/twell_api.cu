@@ -1253,6 +1253,8 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
   if (!make_map(&maT, a2, 3 * static_cast<uint64_t>(f), tp, 64, kBK)) return TWELL_ERR_CUDA;
   const uint16_t* bT[3] = {x, x, dy};
   float* outs[3] = {dWgT, dWuT, dWd};
+  const size_t wbytes = static_cast<size_t>(f) * d * sizeof(float);
+  TW_TRY(zero_async(s, sms, dWgT, wbytes, dWuT, wbytes, dWd, wbytes));  // the split GEMMs add into them
   for (int i = 0; i < 3; ++i) {
     CUtensorMap mb;
     if (!make_map(&mb, bT[i], d, T, 64, kBK)) return TWELL_ERR_CUDA;
@@ -1267,7 +1269,6 @@ twell_status twell_dense_ffn_backward(const uint16_t* x, const uint16_t* WgT, co
     q.k_splits_max = 32;
     q.split_waves = 1;
     q.dev_status = dev_status;
-    TW_TRY(zero_async(s, sms, outs[i], static_cast<size_t>(f) * d * sizeof(float)));
     TW_TRY(launch_gemm<kModeDown>(maT, mb, mb, q, sms, s));
   }
   return TWELL_OK;

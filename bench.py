@@ -840,9 +840,9 @@ def run_gpu_backward(args, world, rank, local):
         # per step, dx: the two slot-epilogue GEMMs (the records), then the tensor-core form's dense rows and
         # dx GEMM, or the CUDA-core form's counter zeroing and dx pass (two passes when Wg and Wu exceed
         # 64 MB), two gathers and three dense-branch GEMMs; weight gradients: the column sort (four launches)
-        # and the per-unit sums, or the dense rows and three zeroed GEMMs, then the overflow rows' three GEMMs
-        "gpu_launches": ((9 if dx_form == "tensor_cores" else 9 + (4 * f * d > (64 << 20)))
-                         + (10 if dw_form == "tensor_cores" else 8)) * K,
+        # and the per-unit sums, or the dense rows, one zeroing and three GEMMs, then the overflow rows' three
+        # GEMMs (eight launches either way)
+        "gpu_launches": ((9 if dx_form == "tensor_cores" else 9 + (4 * f * d > (64 << 20))) + 8) * K,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons", "samples")},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
